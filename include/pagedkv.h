@@ -1,0 +1,202 @@
+/*
+ * pagedkv.h — C-ABI of libpagedkv.so: the paged KV-cache decode path on B200 (sm_100a).
+ *
+ * The KV cache of every layer is split into fixed-size physical blocks ("pages")
+ * reached through a per-sequence block table; decode attention reads the pages
+ * through the table, a cache write scatters each step's new K/V into slots, and a
+ * block copy duplicates shared pages before they are written (copy-on-write).
+ * Sources: "vLLM / PagedAttention — 分页 KV Cache 分析" §2.2 (pages + block table),
+ * §2.3 (block manager, block table, copy-on-write), §3.1 (the attention kernel reads
+ * non-contiguous KV; its simplified per-page loop), §3.2 (copy a shared page before
+ * changing it); "vLLM" entity page, 是什么 (blocks on demand, refcount sharing).
+ *
+ * Conventions (every entry point):
+ *  - returns int: PKV_OK (0) or a negative PKV_ERR_* code; nothing throws across the ABI.
+ *  - device pointers are raw CUDA device addresses owned by the caller; the library
+ *    keeps no reference to them after the call returns.
+ *  - device work is enqueued on `stream` (NULL = legacy default stream) and is
+ *    asynchronous: a PKV_OK return means "arguments valid and launched", not
+ *    "finished". Only pkv_get_device_status synchronises.
+ *  - arguments are checked on the host before any launch; a rejected call launches
+ *    nothing and changes nothing.
+ *  - device-side index errors (a block id or slot outside the pool, a context length
+ *    above the stated maximum) never fault: the kernel skips the access (or reads
+ *    zeros), sets a bit in a per-device status word and continues. Read it with
+ *    pkv_get_device_status.
+ *
+ * Layouts (row-major, element = 2 bytes, fp16 or bf16 as `dtype`):
+ *  - q, out        [num_seqs][num_heads][head_dim]
+ *  - k_cache, v_cache (one layer) [num_blocks][num_kv_heads][block_size][head_dim]
+ *    (one (block, kv head) tile is block_size*head_dim contiguous elements)
+ *  - k_new, v_new  [num_tokens][num_kv_heads][head_dim]
+ *  - block_tables  int32 [num_seqs][max_blocks_per_seq], unused entries ignored
+ *  - context_lens  int32 [num_seqs]  (tokens attended, including the one written this step)
+ *  - slot_mapping  int64 [num_tokens] (slot = block * block_size + row; < 0 = skip)
+ *  - block_pairs   int32 [num_pairs][2] = (src, dst)
+ */
+#ifndef PAGEDKV_H
+#define PAGEDKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL means the legacy default stream. */
+typedef struct CUstream_st *pkv_stream_t;
+
+enum pkv_status {
+    PKV_OK = 0,
+    PKV_ERR_INVALID_ARG = -1,   /* a size, pointer or dtype outside the documented range */
+    PKV_ERR_OUT_OF_BLOCKS = -2, /* allocator: too few free blocks; state unchanged        */
+    PKV_ERR_UNKNOWN_SEQ = -3,   /* allocator: no sequence with that id                    */
+    PKV_ERR_SEQ_EXISTS = -4,    /* allocator: fork target id already in use                */
+    PKV_ERR_TABLE_FULL = -5,    /* allocator: table would exceed max_blocks_per_seq        */
+    PKV_ERR_BAD_INDEX = -6,     /* device status: a kernel met an out-of-pool index       */
+    PKV_ERR_TIMEOUT = -7,       /* device status: a bounded wait in a kernel gave up      */
+    PKV_ERR_CUDA = -8,          /* a CUDA runtime call failed                             */
+    PKV_ERR_WORKSPACE = -9      /* workspace pointer NULL or smaller than required        */
+};
+
+enum pkv_dtype { PKV_F16 = 0, PKV_BF16 = 1 };
+
+/* Bits of the per-device status word (pkv_get_device_status). */
+enum pkv_device_status_bits {
+    PKV_STATUS_BAD_SLOT = 1u << 0,     /* reshape_and_cache: slot >= num_blocks*block_size      */
+    PKV_STATUS_BAD_PAIR = 1u << 1,     /* copy_blocks: src or dst outside [0, num_blocks)       */
+    PKV_STATUS_BAD_BLOCK = 1u << 2,    /* decode: block id outside [0, num_blocks) (read as 0)  */
+    PKV_STATUS_BAD_LEN = 1u << 3,      /* decode: context_len < 0 or above its bound (clamped)  */
+    PKV_STATUS_WAIT_TIMEOUT = 1u << 4  /* decode: a pipeline wait exceeded its iteration limit  */
+};
+
+/* Human-readable name of a status code (static string). */
+const char *pkv_status_string(int code);
+
+/* ------------------------------------------------------------------------------
+ * Paged single-query decode attention ("分页 KV Cache 分析" §3.1; its per-page loop
+ * read as one softmax per (sequence, query head) over all context tokens).
+ *
+ *   out[s][h][:] = sum_t softmax_t(scale * q[s][h] . K_s[t]) * V_s[t],  t < context_lens[s]
+ *   K_s[t] = k_cache[block_tables[s][t / block_size]][h / G][t % block_size][:]   (V alike)
+ *   G = num_heads / num_kv_heads (query heads h*G .. h*G+G-1 share KV head h).
+ *
+ * fp16/bf16 inputs, fp32 accumulation, output rounded to nearest even into `dtype`.
+ * A zero-length context gives out = 0. Slots past context_lens[s] in the last block
+ * are never used (any bits, NaN included, are ignored).
+ * Long contexts are split into partitions of `partition_size` tokens (a multiple of
+ * 64, at most 128 blocks; 0 = automatic) whose partial results are merged exactly
+ * (log-sum-exp) by a second kernel; that needs `workspace` of at least
+ * pkv_decode_workspace_size(...) bytes of device memory (256-byte aligned), which the
+ * caller owns and may reuse between calls that are ordered on one stream.
+ *
+ * Limits: head_dim in {64, 128}; block_size in {8, 16, 32}; 1 <= G <= 16;
+ * num_kv_heads >= 1; num_seqs >= 0; max_context_len <= max_blocks_per_seq*block_size;
+ * num_blocks*num_kv_heads*block_size < 2^31. context_lens[s] is clamped on the
+ * device to [0, max_context_len] (PKV_STATUS_BAD_LEN if it had to be).
+ * Errors: PKV_ERR_INVALID_ARG, PKV_ERR_WORKSPACE, PKV_ERR_CUDA (launch failure).
+ * ---------------------------------------------------------------------------- */
+int pkv_paged_attention_decode(void *out, const void *q, const void *k_cache,
+                               const void *v_cache, const int32_t *block_tables,
+                               const int32_t *context_lens, int num_seqs, int num_heads,
+                               int num_kv_heads, int head_dim, int block_size,
+                               int max_blocks_per_seq, int num_blocks, int max_context_len,
+                               float scale, int dtype, int partition_size, void *workspace,
+                               size_t workspace_bytes, pkv_stream_t stream);
+
+/* Workspace bytes pkv_paged_attention_decode needs for these sizes (0 when the
+ * given partition size makes every context a single partition). Same argument
+ * meaning as the decode call. */
+int pkv_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                              int block_size, int max_context_len, int partition_size,
+                              size_t *bytes_out);
+
+/* The partition size the decode call uses for these sizes (resolves 0 = automatic). */
+int pkv_decode_partition_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                              int block_size, int max_context_len, int partition_size,
+                              int *partition_out);
+
+/* ------------------------------------------------------------------------------
+ * Cache write ("分页 KV Cache 分析" §3.2: a new token is written into its page).
+ *   for t < num_tokens with slot = slot_mapping[t] >= 0:
+ *     k_cache[slot / block_size][h][slot % block_size][:] = k_new[t][h][:]   (V alike)
+ * Bit-exact copy. Slots must be distinct. A slot >= num_blocks*block_size is skipped
+ * and sets PKV_STATUS_BAD_SLOT. Limits as for decode (head_dim, block_size).
+ * ---------------------------------------------------------------------------- */
+int pkv_reshape_and_cache(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+                          const int64_t *slot_mapping, int num_tokens, int num_kv_heads,
+                          int head_dim, int block_size, int num_blocks, int dtype,
+                          pkv_stream_t stream);
+
+/* ------------------------------------------------------------------------------
+ * Copy-on-write block copy ("分页 KV Cache 分析" §3.2: copy first, then modify).
+ *   for each layer l < num_layers and pair (src, dst) in block_pairs:
+ *     k_caches[l][dst] = k_caches[l][src]; v_caches[l][dst] = v_caches[l][src]
+ * (all KV heads). k_caches / v_caches are DEVICE arrays of num_layers device pointers,
+ * each a cache in the layout above. block_pairs is a device array. Every dst must be
+ * distinct and no dst may also be a src in the same call (then pair order does not
+ * matter). A pair with src or dst outside [0, num_blocks) is skipped and sets
+ * PKV_STATUS_BAD_PAIR.
+ * ---------------------------------------------------------------------------- */
+int pkv_copy_blocks(void *const *k_caches, void *const *v_caches, int num_layers,
+                    const int32_t *block_pairs, int num_pairs, int num_kv_heads, int head_dim,
+                    int block_size, int num_blocks, int dtype, pkv_stream_t stream);
+
+/* Synchronise `stream`, then read (and with clear != 0 reset) the status word of the
+ * current device. *status_out gets the PKV_STATUS_* bits. Returns PKV_OK, or
+ * PKV_ERR_CUDA if synchronisation or the read failed. */
+int pkv_get_device_status(uint32_t *status_out, int clear, pkv_stream_t stream);
+
+/* ------------------------------------------------------------------------------
+ * Host block manager ("vLLM" entity page, 是什么; "分页 KV Cache 分析" §2.3, §3.2, §3.3).
+ * Pure host code; no CUDA call. Not thread-safe: one handle per thread at a time.
+ *
+ * Rules (the pages fix no order; these are the library's readings):
+ *  - free list: LIFO stack seeded so successive allocations return
+ *    initial_order[0], initial_order[1], ... (NULL = 0, 1, 2, ...).
+ *  - append of one token at length n: if n % block_size == 0 take a new block
+ *    (refcount 1); else if the last block's refcount > 1 take a new block b', emit the
+ *    copy-on-write pair (last, b'), drop one reference to `last`, put b' in the table.
+ *    The token's slot is table[n / bs] * bs + n % bs; then n += 1.
+ *  - append of k tokens is all-or-nothing (PKV_ERR_TABLE_FULL / PKV_ERR_OUT_OF_BLOCKS
+ *    leave every state unchanged).
+ *  - fork copies the parent's table and length, adding one reference per block.
+ *  - free walks the table from the last logical block to the first, drops one
+ *    reference each and returns blocks whose count reaches 0 to the free list.
+ * ---------------------------------------------------------------------------- */
+typedef struct pkv_alloc pkv_alloc;
+
+/* Creates a manager of num_blocks blocks. initial_order: NULL or a host array that is a
+ * permutation of 0..num_blocks-1 (copied). Errors: PKV_ERR_INVALID_ARG. */
+int pkv_alloc_create(pkv_alloc **out, int num_blocks, int block_size, int max_blocks_per_seq,
+                     const int32_t *initial_order);
+int pkv_alloc_destroy(pkv_alloc *a);
+
+/* Appends n_tokens tokens to seq_id (creating it on first use). slots_out: host int64
+ * [n_tokens] (may be NULL when n_tokens == 0). cow_pairs_out: host int32 [n_tokens][2],
+ * receives *n_cow_out (src, dst) pairs to copy before writing. */
+int pkv_seq_append(pkv_alloc *a, int64_t seq_id, int n_tokens, int64_t *slots_out,
+                   int32_t *cow_pairs_out, int *n_cow_out);
+/* Errors: PKV_ERR_UNKNOWN_SEQ (no parent), PKV_ERR_SEQ_EXISTS (child id in use). */
+int pkv_seq_fork(pkv_alloc *a, int64_t parent, int64_t child);
+/* Errors: PKV_ERR_UNKNOWN_SEQ. */
+int pkv_seq_free(pkv_alloc *a, int64_t seq_id);
+
+/* Writes the block tables of n sequences into host tables_out [n][max_blocks_per_seq]
+ * (unused entries -1) and their lengths into lens_out [n] (may be NULL).
+ * Errors: PKV_ERR_UNKNOWN_SEQ (nothing written past the first unknown id). */
+int pkv_block_tables(const pkv_alloc *a, const int64_t *seq_ids, int n, int32_t *tables_out,
+                     int32_t *lens_out);
+
+/* free + held = num_blocks; logical_tokens = sum of lengths; utilisation =
+ * logical_tokens / (held * block_size) ("分页 KV Cache 分析" §4.2), 0 when nothing is
+ * held. Any output pointer may be NULL. */
+int pkv_stats(const pkv_alloc *a, int *free_blocks, int *held_blocks, int64_t *logical_tokens,
+              double *utilisation);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H */

@@ -1,5 +1,19 @@
 """B200-native paged KV-cache decode path (sm_100a CUDA behind a C-ABI library).
 
-``synth`` builds seeded synthetic workloads. The device entry points are bound
-in ``_binding`` (loaded on first use; it raises if the CUDA library is missing).
+``synth`` builds seeded synthetic workloads. The device entry points and the host
+block manager are bound from ``libpagedkv.so`` (built in-tree by
+``python -m paged_kv_cache_320_b200.build``); calling any of them without the
+library raises — there is no CPU fallback.
 """
+from ._binding import (  # noqa: F401
+    BlockManager,
+    PagedKVError,
+    lib,
+    pkv_copy_blocks,
+    pkv_decode_partition_size,
+    pkv_decode_workspace_size,
+    pkv_get_device_status,
+    pkv_paged_attention_decode,
+    pkv_reshape_and_cache,
+)
+from ._binding import PKV_BF16, PKV_F16  # noqa: F401

@@ -1,0 +1,250 @@
+"""ctypes binding of libpagedkv.so: argument marshalling only.
+
+Every function here reads pointers, sizes and the current CUDA stream from torch
+tensors and calls the C entry point of the same name; all device work runs in the
+library's kernels. There is no fallback: if the library is missing, the first call
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libpagedkv.so")
+
+PKV_OK = 0
+PKV_ERR_INVALID_ARG = -1
+PKV_ERR_OUT_OF_BLOCKS = -2
+PKV_ERR_UNKNOWN_SEQ = -3
+PKV_ERR_SEQ_EXISTS = -4
+PKV_ERR_TABLE_FULL = -5
+PKV_ERR_BAD_INDEX = -6
+PKV_ERR_TIMEOUT = -7
+PKV_ERR_CUDA = -8
+PKV_ERR_WORKSPACE = -9
+
+PKV_F16 = 0
+PKV_BF16 = 1
+
+STATUS_BAD_SLOT = 1 << 0
+STATUS_BAD_PAIR = 1 << 1
+STATUS_BAD_BLOCK = 1 << 2
+STATUS_BAD_LEN = 1 << 3
+STATUS_WAIT_TIMEOUT = 1 << 4
+
+_lib = None
+
+
+class PagedKVError(RuntimeError):
+    def __init__(self, code, what=""):
+        self.code = code
+        msg = lib().pkv_status_string(code).decode() if _lib is not None else str(code)
+        super().__init__(f"{what}: {msg} ({code})")
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m paged_kv_cache_320_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+        L.pkv_status_string.argtypes = [I]
+        L.pkv_status_string.restype = ctypes.c_char_p
+        L.pkv_paged_attention_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I,
+                                                 ctypes.c_float, I, I, P, SZ, P]
+        L.pkv_decode_workspace_size.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(SZ)]
+        L.pkv_decode_partition_size.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(I)]
+        L.pkv_reshape_and_cache.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P]
+        L.pkv_copy_blocks.argtypes = [P, P, I, P, I, I, I, I, I, I, P]
+        L.pkv_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), I, P]
+        L.pkv_alloc_create.argtypes = [ctypes.POINTER(P), I, I, I, P]
+        L.pkv_alloc_destroy.argtypes = [P]
+        L.pkv_seq_append.argtypes = [P, I64, I, P, P, ctypes.POINTER(I)]
+        L.pkv_seq_fork.argtypes = [P, I64, I64]
+        L.pkv_seq_free.argtypes = [P, I64]
+        L.pkv_block_tables.argtypes = [P, P, I, P, P]
+        L.pkv_stats.argtypes = [P, ctypes.POINTER(I), ctypes.POINTER(I),
+                                ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_double)]
+        for name in ("pkv_paged_attention_decode", "pkv_decode_workspace_size",
+                     "pkv_decode_partition_size", "pkv_reshape_and_cache", "pkv_copy_blocks",
+                     "pkv_get_device_status", "pkv_alloc_create", "pkv_alloc_destroy",
+                     "pkv_seq_append", "pkv_seq_fork", "pkv_seq_free", "pkv_block_tables",
+                     "pkv_stats"):
+            getattr(L, name).restype = I
+        _lib = L
+    return _lib
+
+
+def _check(rc, what):
+    if rc != PKV_OK:
+        raise PagedKVError(rc, what)
+
+
+# ---------------------------------------------------------------------------
+# tensor marshalling helpers
+# ---------------------------------------------------------------------------
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.float16:
+        return PKV_F16
+    if t.dtype == torch.bfloat16:
+        return PKV_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libpagedkv must be contiguous")
+    return t.data_ptr()
+
+
+# ---------------------------------------------------------------------------
+# device entry points
+# ---------------------------------------------------------------------------
+def pkv_decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                              max_context_len, partition_size=0) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib().pkv_decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim,
+                                           block_size, max_context_len, partition_size,
+                                           ctypes.byref(out)), "pkv_decode_workspace_size")
+    return out.value
+
+
+def pkv_decode_partition_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                              max_context_len, partition_size=0) -> int:
+    out = ctypes.c_int(0)
+    _check(lib().pkv_decode_partition_size(num_seqs, num_heads, num_kv_heads, head_dim,
+                                           block_size, max_context_len, partition_size,
+                                           ctypes.byref(out)), "pkv_decode_partition_size")
+    return out.value
+
+
+def pkv_paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens,
+                               max_context_len, scale=None, partition_size=0, workspace=None,
+                               stream=None):
+    """out/q [B, Hq, D]; k_cache/v_cache [NB, Hkv, BS, D]; block_tables int32 [B, MB];
+    context_lens int32 [B]; workspace: uint8 tensor of pkv_decode_workspace_size bytes
+    (allocated here when None and needed)."""
+    B, Hq, D = q.shape
+    NB, Hkv, BS, D2 = k_cache.shape
+    if D2 != D or out.shape != q.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if workspace is None:
+        need = pkv_decode_workspace_size(B, Hq, Hkv, D, BS, max_context_len, partition_size)
+        if need:
+            import torch
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _ptr(workspace) if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().pkv_paged_attention_decode(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
+        B, Hq, Hkv, D, BS, block_tables.shape[1], NB, int(max_context_len), float(scale),
+        _dtype_code(q), int(partition_size), ws_ptr, ws_bytes, _stream(stream)),
+        "pkv_paged_attention_decode")
+    return out
+
+
+def pkv_reshape_and_cache(k_new, v_new, k_cache, v_cache, slot_mapping, stream=None):
+    """k_new/v_new [T, Hkv, D]; caches [NB, Hkv, BS, D]; slot_mapping int64 [T]."""
+    T, Hkv, D = k_new.shape
+    NB, _, BS, _ = k_cache.shape
+    _check(lib().pkv_reshape_and_cache(_ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
+                                       _ptr(slot_mapping), T, Hkv, D, BS, NB,
+                                       _dtype_code(k_cache), _stream(stream)),
+           "pkv_reshape_and_cache")
+
+
+def pkv_copy_blocks(k_cache_ptrs, v_cache_ptrs, block_pairs, num_kv_heads, head_dim, block_size,
+                    num_blocks, dtype, stream=None):
+    """k_cache_ptrs / v_cache_ptrs: int64 device tensors [L] of cache addresses;
+    block_pairs: int32 device tensor [n, 2]."""
+    n = block_pairs.shape[0] if block_pairs.numel() else 0
+    _check(lib().pkv_copy_blocks(_ptr(k_cache_ptrs), _ptr(v_cache_ptrs), k_cache_ptrs.numel(),
+                                 _ptr(block_pairs), n, num_kv_heads, head_dim, block_size,
+                                 num_blocks, dtype, _stream(stream)), "pkv_copy_blocks")
+
+
+def pkv_get_device_status(clear=True, stream=None) -> int:
+    v = ctypes.c_uint32(0)
+    _check(lib().pkv_get_device_status(ctypes.byref(v), int(bool(clear)), _stream(stream)),
+           "pkv_get_device_status")
+    return v.value
+
+
+# ---------------------------------------------------------------------------
+# host block manager
+# ---------------------------------------------------------------------------
+class BlockManager:
+    """Owner of a pkv_alloc handle (host-only; no CUDA call)."""
+
+    def __init__(self, num_blocks, block_size, max_blocks_per_seq, initial_order=None):
+        import numpy as np
+        self.num_blocks, self.block_size, self.max_blocks_per_seq = (
+            num_blocks, block_size, max_blocks_per_seq)
+        h = ctypes.c_void_p()
+        order = None
+        if initial_order is not None:
+            order = np.ascontiguousarray(initial_order, dtype=np.int32)
+        _check(lib().pkv_alloc_create(ctypes.byref(h), num_blocks, block_size, max_blocks_per_seq,
+                                      order.ctypes.data if order is not None else None),
+               "pkv_alloc_create")
+        self._h = h
+
+    def close(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            lib().pkv_alloc_destroy(self._h)
+            self._h = None
+
+    __del__ = close
+
+    def pkv_seq_append(self, seq_id, n_tokens):
+        """Returns (status, slots int64 array, cow pairs int32 [k, 2])."""
+        import numpy as np
+        slots = np.zeros(max(n_tokens, 1), dtype=np.int64)
+        cows = np.zeros((max(n_tokens, 1), 2), dtype=np.int32)
+        n_cow = ctypes.c_int(0)
+        rc = lib().pkv_seq_append(self._h, int(seq_id), int(n_tokens), slots.ctypes.data,
+                                  cows.ctypes.data, ctypes.byref(n_cow))
+        if rc != PKV_OK:
+            return rc, slots[:0], cows[:0]
+        return rc, slots[:n_tokens], cows[:n_cow.value]
+
+    def pkv_seq_fork(self, parent, child):
+        return lib().pkv_seq_fork(self._h, int(parent), int(child))
+
+    def pkv_seq_free(self, seq_id):
+        return lib().pkv_seq_free(self._h, int(seq_id))
+
+    def pkv_block_tables(self, seq_ids):
+        """Returns (status, tables int32 [n, MB], lens int32 [n])."""
+        import numpy as np
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        n = ids.shape[0]
+        tables = np.zeros((n, self.max_blocks_per_seq), dtype=np.int32)
+        lens = np.zeros(n, dtype=np.int32)
+        rc = lib().pkv_block_tables(self._h, ids.ctypes.data, n, tables.ctypes.data,
+                                    lens.ctypes.data)
+        return rc, tables, lens
+
+    def pkv_stats(self):
+        """Returns (free, held, logical_tokens, utilisation)."""
+        f, h = ctypes.c_int(), ctypes.c_int()
+        t, u = ctypes.c_int64(), ctypes.c_double()
+        _check(lib().pkv_stats(self._h, ctypes.byref(f), ctypes.byref(h), ctypes.byref(t),
+                               ctypes.byref(u)), "pkv_stats")
+        return f.value, h.value, t.value, u.value

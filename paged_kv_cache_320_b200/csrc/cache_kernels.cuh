@@ -1,0 +1,68 @@
+// Cache maintenance kernels: the cache write through a slot mapping and the
+// copy-on-write block copy ("vLLM / PagedAttention — 分页 KV Cache 分析" §3.2: a new
+// token goes into its page; a shared page is copied before it is changed).
+//
+// Both are pure data movement: 16-byte vector loads/stores, every 32-byte sector
+// fully used (a (token, KV head) row is head_dim*2 = 128 or 256 contiguous bytes).
+#pragma once
+
+#include <stdint.h>
+
+namespace pkv {
+
+// One thread per 16-byte vector of one (token, KV head) row; K and V together.
+//   k_cache[slot / BS][h][slot % BS][:] = k_new[t][h][:]   (V alike), slot >= 0
+template <int D>
+__global__ void __launch_bounds__(256)
+reshape_and_cache_kernel(const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new,
+                         uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache,
+                         const int64_t *__restrict__ slot_mapping, int num_tokens, int Hkv,
+                         int BS, int num_blocks, unsigned *status) {
+    constexpr int VPR = D * 2 / 16;   // vectors per row
+    const int64_t total = (int64_t)num_tokens * Hkv * VPR;
+    const int64_t limit = (int64_t)num_blocks * BS;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t row = i / VPR;          // t * Hkv + h
+        const int v = (int)(i - row * VPR);
+        const int64_t t = row / Hkv;
+        const int h = (int)(row - t * Hkv);
+        const int64_t slot = slot_mapping[t];
+        if (slot < 0) continue;
+        if (slot >= limit) {
+            if (h == 0 && v == 0) atomicOr(status, 1u /* bad slot */);
+            continue;
+        }
+        const int64_t blk = slot / BS;
+        const int64_t r = slot - blk * BS;
+        const int64_t dst = ((blk * Hkv + h) * BS + r) * VPR + v;
+        k_cache[dst] = k_new[i];
+        v_cache[dst] = v_new[i];
+    }
+}
+
+// One CTA per (pair, layer, K|V): copies the whole block (all KV heads).
+__global__ void __launch_bounds__(256)
+copy_blocks_kernel(void *const *__restrict__ k_caches, void *const *__restrict__ v_caches,
+                   const int32_t *__restrict__ block_pairs, int num_blocks, int block_vecs,
+                   unsigned *status) {
+    const int pair = blockIdx.x;
+    const int layer = blockIdx.y;
+    const int src = block_pairs[2 * pair];
+    const int dst = block_pairs[2 * pair + 1];
+    if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+        if (threadIdx.x == 0 && blockIdx.z == 0) atomicOr(status, 2u /* bad pair */);
+        return;
+    }
+    uint4 *base = reinterpret_cast<uint4 *>(blockIdx.z ? v_caches[layer] : k_caches[layer]);
+    const uint4 *s = base + (int64_t)src * block_vecs;
+    uint4 *d = base + (int64_t)dst * block_vecs;
+    int i = threadIdx.x;
+    for (; i + 3 * 256 < block_vecs; i += 4 * 256) {
+        const uint4 a = s[i], b = s[i + 256], c = s[i + 512], e = s[i + 768];
+        d[i] = a; d[i + 256] = b; d[i + 512] = c; d[i + 768] = e;
+    }
+    for (; i < block_vecs; i += 256) d[i] = s[i];
+}
+
+}  // namespace pkv

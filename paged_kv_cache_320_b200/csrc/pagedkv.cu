@@ -1,0 +1,386 @@
+// C-ABI entry points of libpagedkv.so (declared and documented in pagedkv.h):
+// host-side argument checks, TMA descriptor encoding, launch configuration and the
+// per-device status word. All device work is in decode_kernels.cuh and
+// cache_kernels.cuh.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "cache_kernels.cuh"
+#include "decode_kernels.cuh"
+#include "pagedkv.h"
+
+namespace {
+
+// One status word per device (each device that loads the library gets its own copy).
+__device__ unsigned int g_pkv_status;
+
+constexpr int kMaxDevices = 64;
+
+std::mutex g_mu;
+unsigned int *g_status_ptr[kMaxDevices];
+int g_sm_count[kMaxDevices];
+
+int current_device(int *dev) {
+    if (cudaGetDevice(dev) != cudaSuccess || *dev < 0 || *dev >= kMaxDevices) return PKV_ERR_CUDA;
+    return PKV_OK;
+}
+
+int device_status_ptr(unsigned int **out) {
+    int dev;
+    if (current_device(&dev) != PKV_OK) return PKV_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_status_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_pkv_status) != cudaSuccess) return PKV_ERR_CUDA;
+        g_status_ptr[dev] = static_cast<unsigned int *>(p);
+    }
+    *out = g_status_ptr[dev];
+    return PKV_OK;
+}
+
+int sm_count(int *out) {
+    int dev;
+    if (current_device(&dev) != PKV_OK) return PKV_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_sm_count[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            return PKV_ERR_CUDA;
+        g_sm_count[dev] = n;
+    }
+    *out = g_sm_count[dev];
+    return PKV_OK;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link-time
+// dependency on libcuda, so the library also loads on a machine without a GPU).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D view of one layer's cache: rows = num_blocks*Hkv*BS, columns = head_dim;
+// box = 64 columns (128 bytes, swizzled) x BS rows = one slab of one page.
+int encode_cache_map(CUtensorMap *map, const void *base, int dtype, int D, int BS, int NB,
+                     int Hkv) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return PKV_ERR_CUDA;
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)NB * Hkv * BS};
+    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)BS};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r =
+        fn(map, dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+           2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? PKV_OK : PKV_ERR_CUDA;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+// Automatic partition size: 512 tokens for GQA groups up to 4 and 1024 above (the
+// fp32 partials grow with the group), at most 128 blocks, halved while the batch
+// offers fewer than 1024 work items (about 7 per CTA on 148 SMs).
+int auto_partition(int B, int Hq, int Hkv, int BS, int max_len) {
+    const int G = Hq / Hkv;
+    int p = G <= 4 ? 512 : 1024;
+    if (p > pkv::kMaxItemBlocks * BS) p = pkv::kMaxItemBlocks * BS;
+    while (p > 64 && (long long)B * Hkv * cdiv(max_len, p) < 1024) p /= 2;
+    return p;
+}
+
+int check_decode_sizes(int B, int Hq, int Hkv, int D, int BS, int max_len, int partition,
+                       int *P_out) {
+    if (B < 0 || Hkv < 1 || Hq < 1 || Hq % Hkv != 0 || Hq / Hkv > pkv::kMaxGroup)
+        return PKV_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return PKV_ERR_INVALID_ARG;
+    if (BS != 8 && BS != 16 && BS != 32) return PKV_ERR_INVALID_ARG;
+    if (max_len < 0) return PKV_ERR_INVALID_ARG;
+    int P = partition;
+    if (P == 0) P = auto_partition(B, Hq, Hkv, BS, max_len);
+    if (P <= 0 || P % pkv::kStageTokens != 0 || P > pkv::kMaxItemBlocks * BS)
+        return PKV_ERR_INVALID_ARG;
+    const long long pmax = max_len <= P ? 1 : cdiv(max_len, P);
+    if ((long long)B * Hkv * pmax >= INT_MAX) return PKV_ERR_INVALID_ARG;
+    *P_out = P;
+    return PKV_OK;
+}
+
+struct WsLayout {
+    size_t ml, o, total;
+};
+
+WsLayout ws_layout(int B, int Hq, int D, int max_len, int P) {
+    WsLayout w{0, 0, 0};
+    const long long pmax = max_len <= P ? 1 : cdiv(max_len, P);
+    if (pmax <= 1 || B == 0) return w;
+    const size_t rows = (size_t)B * Hq * pmax;
+    w.ml = align_up((size_t)B * sizeof(int32_t), 256);
+    w.o = w.ml + align_up(rows * 2 * sizeof(float), 256);
+    w.total = w.o + rows * D * sizeof(float);
+    return w;
+}
+
+template <typename T, int D, int BS>
+int launch_decode(const CUtensorMap &mk, const CUtensorMap &mv, const pkv::DecodeParams &prm,
+                  long long items_upper, cudaStream_t st) {
+    using L = pkv::DecodeLayout<D>;
+    auto kern = pkv::paged_decode_partition_kernel<T, D, BS>;
+    const size_t smem = L::smem_bytes(prm.group);
+    int dev;
+    if (current_device(&dev) != PKV_OK) return PKV_ERR_CUDA;
+    static int occ[kMaxDevices][pkv::kMaxGroup + 1];
+    int nsm;
+    if (sm_count(&nsm) != PKV_OK) return PKV_ERR_CUDA;
+    int &o = occ[dev][prm.group];
+    if (o == 0) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+            return PKV_ERR_CUDA;
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, pkv::kDecodeThreads, smem) !=
+                cudaSuccess ||
+            n <= 0)
+            return PKV_ERR_CUDA;
+        o = n;
+    }
+    long long grid = (long long)nsm * o;
+    if (grid > items_upper) grid = items_upper;
+    if (grid < 1) grid = 1;
+    kern<<<(unsigned)grid, pkv::kDecodeThreads, smem, st>>>(mk, mv, prm);
+    if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
+    return PKV_OK;
+}
+
+template <typename T, int D>
+int launch_reduce(const pkv::DecodeParams &prm, int pmax, cudaStream_t st) {
+    dim3 grid(prm.num_heads, prm.num_seqs);
+    pkv::paged_decode_reduce_kernel<T, D><<<grid, D, (size_t)pmax * sizeof(float), st>>>(prm);
+    if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
+    return PKV_OK;
+}
+
+template <typename T, int D>
+int dispatch_bs(int BS, const CUtensorMap &mk, const CUtensorMap &mv,
+                const pkv::DecodeParams &prm, long long items, cudaStream_t st) {
+    switch (BS) {
+        case 8: return launch_decode<T, D, 8>(mk, mv, prm, items, st);
+        case 16: return launch_decode<T, D, 16>(mk, mv, prm, items, st);
+        case 32: return launch_decode<T, D, 32>(mk, mv, prm, items, st);
+    }
+    return PKV_ERR_INVALID_ARG;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *pkv_status_string(int code) {
+    switch (code) {
+        case PKV_OK: return "ok";
+        case PKV_ERR_INVALID_ARG: return "invalid argument";
+        case PKV_ERR_OUT_OF_BLOCKS: return "out of blocks";
+        case PKV_ERR_UNKNOWN_SEQ: return "unknown sequence";
+        case PKV_ERR_SEQ_EXISTS: return "sequence id already in use";
+        case PKV_ERR_TABLE_FULL: return "block table full";
+        case PKV_ERR_BAD_INDEX: return "out-of-pool index met on the device";
+        case PKV_ERR_TIMEOUT: return "bounded device wait gave up";
+        case PKV_ERR_CUDA: return "CUDA runtime error";
+        case PKV_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+int pkv_decode_partition_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                              int block_size, int max_context_len, int partition_size,
+                              int *partition_out) {
+    if (!partition_out) return PKV_ERR_INVALID_ARG;
+    return check_decode_sizes(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                              max_context_len, partition_size, partition_out);
+}
+
+int pkv_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                              int block_size, int max_context_len, int partition_size,
+                              size_t *bytes_out) {
+    if (!bytes_out) return PKV_ERR_INVALID_ARG;
+    int P;
+    const int rc = check_decode_sizes(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                      max_context_len, partition_size, &P);
+    if (rc != PKV_OK) return rc;
+    *bytes_out = ws_layout(num_seqs, num_heads, head_dim, max_context_len, P).total;
+    return PKV_OK;
+}
+
+int pkv_paged_attention_decode(void *out, const void *q, const void *k_cache,
+                               const void *v_cache, const int32_t *block_tables,
+                               const int32_t *context_lens, int num_seqs, int num_heads,
+                               int num_kv_heads, int head_dim, int block_size,
+                               int max_blocks_per_seq, int num_blocks, int max_context_len,
+                               float scale, int dtype, int partition_size, void *workspace,
+                               size_t workspace_bytes, pkv_stream_t stream) {
+    int P;
+    int rc = check_decode_sizes(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                max_context_len, partition_size, &P);
+    if (rc != PKV_OK) return rc;
+    if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return PKV_ERR_INVALID_ARG;
+    if (max_blocks_per_seq < 1 || num_blocks < 1) return PKV_ERR_INVALID_ARG;
+    if ((long long)max_context_len > (long long)max_blocks_per_seq * block_size)
+        return PKV_ERR_INVALID_ARG;
+    if ((long long)num_blocks * num_kv_heads * block_size >= INT_MAX) return PKV_ERR_INVALID_ARG;
+    if (num_seqs == 0) return PKV_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+        return PKV_ERR_INVALID_ARG;
+    if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(q, 4) || !aligned(out, 2) ||
+        !aligned(block_tables, 4) || !aligned(context_lens, 4))
+        return PKV_ERR_INVALID_ARG;
+    const WsLayout ws = ws_layout(num_seqs, num_heads, head_dim, max_context_len, P);
+    if (ws.total > 0 && (!workspace || workspace_bytes < ws.total || !aligned(workspace, 16)))
+        return PKV_ERR_WORKSPACE;
+
+    unsigned int *status;
+    if ((rc = device_status_ptr(&status)) != PKV_OK) return rc;
+    CUtensorMap mk, mv;
+    if ((rc = encode_cache_map(&mk, k_cache, dtype, head_dim, block_size, num_blocks,
+                               num_kv_heads)) != PKV_OK)
+        return rc;
+    if ((rc = encode_cache_map(&mv, v_cache, dtype, head_dim, block_size, num_blocks,
+                               num_kv_heads)) != PKV_OK)
+        return rc;
+
+    pkv::DecodeParams prm;
+    prm.out = out;
+    prm.q = q;
+    prm.block_tables = block_tables;
+    prm.context_lens = context_lens;
+    uint8_t *wsb = static_cast<uint8_t *>(workspace);
+    prm.ws_seq_base = ws.total ? reinterpret_cast<int32_t *>(wsb) : nullptr;
+    prm.ws_ml = ws.total ? reinterpret_cast<float *>(wsb + ws.ml) : nullptr;
+    prm.ws_o = ws.total ? reinterpret_cast<float *>(wsb + ws.o) : nullptr;
+    prm.status = status;
+    prm.num_seqs = num_seqs;
+    prm.num_heads = num_heads;
+    prm.num_kv_heads = num_kv_heads;
+    prm.group = num_heads / num_kv_heads;
+    prm.max_blocks_per_seq = max_blocks_per_seq;
+    prm.num_blocks = num_blocks;
+    prm.max_context_len = max_context_len;
+    prm.partition = P;
+    prm.scale_log2 = (float)((double)scale * 1.4426950408889634);
+
+    const int pmax = max_context_len <= P ? 1 : cdiv(max_context_len, P);
+    const long long items = (long long)num_seqs * num_kv_heads * pmax;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (dtype == PKV_BF16) {
+        rc = head_dim == 128 ? dispatch_bs<__nv_bfloat16, 128>(block_size, mk, mv, prm, items, st)
+                             : dispatch_bs<__nv_bfloat16, 64>(block_size, mk, mv, prm, items, st);
+        if (rc == PKV_OK && pmax > 1)
+            rc = head_dim == 128 ? launch_reduce<__nv_bfloat16, 128>(prm, pmax, st)
+                                 : launch_reduce<__nv_bfloat16, 64>(prm, pmax, st);
+    } else {
+        rc = head_dim == 128 ? dispatch_bs<__half, 128>(block_size, mk, mv, prm, items, st)
+                             : dispatch_bs<__half, 64>(block_size, mk, mv, prm, items, st);
+        if (rc == PKV_OK && pmax > 1)
+            rc = head_dim == 128 ? launch_reduce<__half, 128>(prm, pmax, st)
+                                 : launch_reduce<__half, 64>(prm, pmax, st);
+    }
+    return rc;
+}
+
+int pkv_reshape_and_cache(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+                          const int64_t *slot_mapping, int num_tokens, int num_kv_heads,
+                          int head_dim, int block_size, int num_blocks, int dtype,
+                          pkv_stream_t stream) {
+    if (num_tokens < 0 || num_kv_heads < 1 || num_blocks < 1) return PKV_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return PKV_ERR_INVALID_ARG;
+    if (block_size != 8 && block_size != 16 && block_size != 32) return PKV_ERR_INVALID_ARG;
+    if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_ERR_INVALID_ARG;
+    if (num_tokens == 0) return PKV_OK;
+    if (!k_new || !v_new || !k_cache || !v_cache || !slot_mapping) return PKV_ERR_INVALID_ARG;
+    if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_cache, 16) ||
+        !aligned(v_cache, 16) || !aligned(slot_mapping, 8))
+        return PKV_ERR_INVALID_ARG;
+    unsigned int *status;
+    int rc;
+    if ((rc = device_status_ptr(&status)) != PKV_OK) return rc;
+    int nsm;
+    if ((rc = sm_count(&nsm)) != PKV_OK) return rc;
+    const long long total = (long long)num_tokens * num_kv_heads * (head_dim * 2 / 16);
+    long long blocks = (total + 255) / 256;
+    if (blocks > (long long)nsm * 16) blocks = (long long)nsm * 16;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    auto *kn = static_cast<const uint4 *>(k_new);
+    auto *vn = static_cast<const uint4 *>(v_new);
+    auto *kc = static_cast<uint4 *>(k_cache);
+    auto *vc = static_cast<uint4 *>(v_cache);
+    if (head_dim == 128)
+        pkv::reshape_and_cache_kernel<128><<<(unsigned)blocks, 256, 0, st>>>(
+            kn, vn, kc, vc, slot_mapping, num_tokens, num_kv_heads, block_size, num_blocks, status);
+    else
+        pkv::reshape_and_cache_kernel<64><<<(unsigned)blocks, 256, 0, st>>>(
+            kn, vn, kc, vc, slot_mapping, num_tokens, num_kv_heads, block_size, num_blocks, status);
+    return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+int pkv_copy_blocks(void *const *k_caches, void *const *v_caches, int num_layers,
+                    const int32_t *block_pairs, int num_pairs, int num_kv_heads, int head_dim,
+                    int block_size, int num_blocks, int dtype, pkv_stream_t stream) {
+    if (num_pairs < 0 || num_layers < 1 || num_layers > 65535 || num_kv_heads < 1 ||
+        num_blocks < 1)
+        return PKV_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return PKV_ERR_INVALID_ARG;
+    if (block_size != 8 && block_size != 16 && block_size != 32) return PKV_ERR_INVALID_ARG;
+    if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_ERR_INVALID_ARG;
+    if (num_pairs == 0) return PKV_OK;
+    if (!k_caches || !v_caches || !block_pairs) return PKV_ERR_INVALID_ARG;
+    const long long vecs = (long long)num_kv_heads * block_size * head_dim * 2 / 16;
+    if (vecs >= INT_MAX) return PKV_ERR_INVALID_ARG;
+    unsigned int *status;
+    int rc;
+    if ((rc = device_status_ptr(&status)) != PKV_OK) return rc;
+    dim3 grid((unsigned)num_pairs, (unsigned)num_layers, 2);
+    pkv::copy_blocks_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        k_caches, v_caches, block_pairs, num_blocks, (int)vecs, status);
+    return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+int pkv_get_device_status(uint32_t *status_out, int clear, pkv_stream_t stream) {
+    if (!status_out) return PKV_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_pkv_status, sizeof(v)) != cudaSuccess) return PKV_ERR_CUDA;
+    if (clear) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(g_pkv_status, &zero, sizeof(zero)) != cudaSuccess)
+            return PKV_ERR_CUDA;
+    }
+    *status_out = v;
+    return PKV_OK;
+}
+
+}  // extern "C"

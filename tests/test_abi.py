@@ -1,0 +1,111 @@
+"""The C-ABI library loads and exports every entry point its header declares, and
+host-side argument checks reject bad sizes before any device work (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import paged_kv_cache_320_b200 as pkv
+from paged_kv_cache_320_b200 import _binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    names = set()
+    inc = os.path.join(ROOT, "include")
+    for f in os.listdir(inc):
+        if f.endswith(".h"):
+            text = open(os.path.join(inc, f)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(pkv_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
+
+
+def test_header_declares_the_entry_points():
+    names = declared_symbols()
+    for must in ("pkv_paged_attention_decode", "pkv_reshape_and_cache", "pkv_copy_blocks",
+                 "pkv_alloc_create", "pkv_seq_append", "pkv_seq_fork", "pkv_seq_free",
+                 "pkv_block_tables", "pkv_stats"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(B.LIB_PATH)
+    missing = [n for n in declared_symbols() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+@pytest.mark.parametrize("args", [
+    (4, 8, 8, 96, 16, 128, 0),       # head_dim
+    (4, 8, 8, 64, 12, 128, 0),       # block_size
+    (4, 8, 3, 64, 16, 128, 0),       # Hq % Hkv
+    (4, 64, 2, 64, 16, 128, 0),      # group > 16
+    (4, 8, 8, 64, 16, 128, 100),     # partition not a multiple of 64
+    (4, 8, 8, 64, 8, 128, 2048),     # partition > 128 blocks
+    (-1, 8, 8, 64, 16, 128, 0),      # negative batch
+])
+def test_decode_size_checks(args):
+    with pytest.raises(pkv.PagedKVError) as e:
+        pkv.pkv_decode_workspace_size(*args)
+    assert e.value.code == B.PKV_ERR_INVALID_ARG
+
+
+def test_workspace_size_formula():
+    # single partition -> no workspace
+    assert pkv.pkv_decode_workspace_size(4, 8, 8, 64, 16, 100, 128) == 0
+    # B=2, Hq=4, D=64, max_len=300, P=128 -> 3 partitions
+    rows = 2 * 4 * 3
+    expect = 256 + ((rows * 8 + 255) // 256) * 256 + rows * 64 * 4
+    assert pkv.pkv_decode_workspace_size(2, 4, 2, 64, 16, 300, 128) == expect
+
+
+def test_auto_partition_choices():
+    assert pkv.pkv_decode_partition_size(256, 32, 8, 128, 16, 8192) == 512     # G = 4
+    assert pkv.pkv_decode_partition_size(8, 64, 8, 128, 16, 131072) == 1024    # G = 8
+    assert pkv.pkv_decode_partition_size(8, 64, 8, 128, 8, 131072) == 1024     # 128 blocks of 8
+    assert pkv.pkv_decode_partition_size(4, 8, 8, 64, 16, 128) == 64          # tiny batch
+
+
+def test_decode_rejects_bad_args_without_a_device():
+    L = B.lib()
+    # head_dim 96 -> rejected before any CUDA call
+    rc = L.pkv_paged_attention_decode(None, None, None, None, None, None, 4, 8, 8, 96, 16, 8, 64,
+                                      100, 0.1, 0, 0, None, 0, None)
+    assert rc == B.PKV_ERR_INVALID_ARG
+    # max_context_len above max_blocks_per_seq * block_size
+    rc = L.pkv_paged_attention_decode(None, None, None, None, None, None, 4, 8, 8, 64, 16, 8, 64,
+                                      129, 0.1, 0, 0, None, 0, None)
+    assert rc == B.PKV_ERR_INVALID_ARG
+    # bad dtype / non-finite scale
+    rc = L.pkv_paged_attention_decode(None, None, None, None, None, None, 4, 8, 8, 64, 16, 8, 64,
+                                      100, 0.1, 7, 0, None, 0, None)
+    assert rc == B.PKV_ERR_INVALID_ARG
+    rc = L.pkv_paged_attention_decode(None, None, None, None, None, None, 4, 8, 8, 64, 16, 8, 64,
+                                      100, float("inf"), 0, 0, None, 0, None)
+    assert rc == B.PKV_ERR_INVALID_ARG
+    # zero sequences: nothing to do
+    rc = L.pkv_paged_attention_decode(None, None, None, None, None, None, 0, 8, 8, 64, 16, 8, 64,
+                                      100, 0.1, 0, 0, None, 0, None)
+    assert rc == B.PKV_OK
+    # null pointers with work to do
+    rc = L.pkv_paged_attention_decode(None, None, None, None, None, None, 4, 8, 8, 64, 16, 8, 64,
+                                      100, 0.1, 0, 0, None, 0, None)
+    assert rc == B.PKV_ERR_INVALID_ARG
+
+
+def test_cache_op_checks_without_a_device():
+    L = B.lib()
+    assert L.pkv_reshape_and_cache(None, None, None, None, None, 0, 8, 64, 16, 64, 0, None) == B.PKV_OK
+    assert L.pkv_reshape_and_cache(None, None, None, None, None, 4, 8, 64, 16, 64, 0, None) == B.PKV_ERR_INVALID_ARG
+    assert L.pkv_reshape_and_cache(None, None, None, None, None, 4, 8, 80, 16, 64, 0, None) == B.PKV_ERR_INVALID_ARG
+    assert L.pkv_copy_blocks(None, None, 1, None, 0, 8, 64, 16, 64, 0, None) == B.PKV_OK
+    assert L.pkv_copy_blocks(None, None, 1, None, 3, 8, 64, 16, 64, 0, None) == B.PKV_ERR_INVALID_ARG
+    assert L.pkv_copy_blocks(None, None, 0, None, 3, 8, 64, 16, 64, 0, None) == B.PKV_ERR_INVALID_ARG
+
+
+def test_status_strings():
+    L = B.lib()
+    for code in range(-9, 1):
+        assert L.pkv_status_string(code)

@@ -1,0 +1,96 @@
+"""The C++ block manager (through the C-ABI) against the hand-worked traces in
+tests/golden/alloc_traces.json and, op by op, against the oracle's independent
+Python model on seeded random op sequences: identical statuses, slots,
+copy-on-write pairs, block tables and statistics (CPU only)."""
+import json
+import os
+
+import numpy as np
+import pytest
+
+from oracle import block_manager as BM
+from paged_kv_cache_320_b200 import BlockManager, synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "alloc_traces.json")
+
+
+@pytest.mark.parametrize("trace", json.load(open(GOLDEN))["traces"], ids=lambda t: t["name"])
+def test_hand_worked_traces(trace):
+    mgr = BlockManager(trace["num_blocks"], trace["block_size"], trace["max_blocks_per_seq"],
+                       trace["initial_order"])
+    for op in trace["ops"]:
+        if op["op"] == "append":
+            st, slots, cows = mgr.pkv_seq_append(op["seq"], op["n"])
+            assert st == op["status"], op
+            if st == 0:
+                assert slots.tolist() == op["slots"], op
+                assert cows.tolist() == op["cow"], op
+        elif op["op"] == "fork":
+            assert mgr.pkv_seq_fork(op["parent"], op["child"]) == op["status"], op
+        else:
+            assert mgr.pkv_seq_free(op["seq"]) == op["status"], op
+    for seq, (row, n) in trace["final_tables"].items():
+        st, tables, lens = mgr.pkv_block_tables([int(seq)])
+        assert st == 0 and tables[0].tolist() == row and lens[0] == n
+    free, held, tokens, util = mgr.pkv_stats()
+    fs = trace["final_stats"]
+    assert (free, held, tokens) == (fs["free"], fs["held"], fs["tokens"])
+    assert util == pytest.approx(fs["util"], abs=1e-15)
+
+
+def compare_states(c, m, seqs):
+    fc, hc, tc, uc = c.pkv_stats()
+    fm, hm, tm, um = m.stats()
+    assert (fc, hc, tc) == (fm, hm, tm)
+    assert uc == pytest.approx(um, abs=1e-12)
+    if seqs:
+        st, tables, lens = c.pkv_block_tables(seqs)
+        assert st == 0
+        for i, s in enumerate(seqs):
+            row, n = m.block_table(s)
+            assert tables[i].tolist() == row and lens[i] == n
+
+
+@pytest.mark.parametrize("chunk", range(8))
+def test_random_op_sequences_match_the_model(chunk):
+    """2000 seeded op sequences (250 per chunk) of 40 ops each, with errors."""
+    for seed in range(chunk * 250, (chunk + 1) * 250):
+        rng = np.random.default_rng(seed)
+        nb = int(rng.integers(4, 24))
+        bs = int(rng.choice([1, 2, 4, 8]))
+        mb = int(rng.integers(1, 6))
+        order = rng.permutation(nb)
+        c = BlockManager(nb, bs, mb, order)
+        m = BM.BlockManagerModel(nb, bs, mb, order)
+        ids = list(range(6))
+        for _ in range(40):
+            r = rng.random()
+            a = int(rng.choice(ids))
+            if r < 0.6:
+                n = int(rng.integers(0, 2 * bs + 2))
+                sc, slc, cwc = c.pkv_seq_append(a, n)
+                sm, slm, cwm = m.append(a, n)
+                assert sc == sm, (seed, a, n)
+                assert slc.tolist() == slm
+                assert cwc.tolist() == [list(x) for x in cwm]
+            elif r < 0.8:
+                b = int(rng.choice(ids))
+                assert c.pkv_seq_fork(a, b) == m.fork(a, b)
+            else:
+                assert c.pkv_seq_free(a) == m.free(a)
+        compare_states(c, m, sorted(m.tables))
+        c.close()
+
+
+def test_workload_placement_reproduced_by_in_order_appends():
+    wl = synth.make_workload("long_context", values_on="none", block_size=8)
+    mgr = BlockManager(wl.num_blocks, 8, wl.max_blocks_per_seq, wl.perm)
+    last = []
+    for s, n in enumerate(wl.context_lens):
+        st, slots, cows = mgr.pkv_seq_append(s, int(n))
+        assert st == 0 and len(cows) == 0
+        last.append(slots[-1])
+    st, tables, lens = mgr.pkv_block_tables(np.arange(wl.num_seqs))
+    np.testing.assert_array_equal(tables, wl.block_tables)
+    np.testing.assert_array_equal(lens, wl.context_lens)
+    np.testing.assert_array_equal(last, wl.slot_mapping)
