@@ -309,3 +309,51 @@ def sample_sequences(wl: Workload, n: int, seed: int = 0) -> np.ndarray:
             break
         pick.add(int(s))
     return np.array(sorted(pick))
+
+
+# ----------------------------------------------------------------------------
+# copy-on-write step of the shared-prefix workload
+# ----------------------------------------------------------------------------
+@dataclasses.dataclass
+class CowStep:
+    """Inputs of one parallel-sampling step whose last prefix block is shared.
+
+    Each of ``prompts`` parents has ``parent_lens[p] = prefix + u_p`` tokens,
+    u_p uniform in [1, 255] and not a multiple of 16, so its last block is partly
+    filled; it is forked into ``samples`` sequences and every sample then appends
+    one token. Which blocks hold what is decided by the block manager under test
+    (seeded with ``initial_order``); the values here are the whole pool's contents."""
+    spec: Spec
+    parent_lens: np.ndarray
+    initial_order: np.ndarray
+    num_blocks: int
+    max_blocks_per_seq: int
+    num_layers: int
+    q: np.ndarray            # [B, Hq, d] bits
+    k_cache: np.ndarray      # [L, NB, Hkv, bs, d] bits (every row a value; the test masks)
+    v_cache: np.ndarray
+    k_new: np.ndarray        # [B, Hkv, d] bits
+    v_new: np.ndarray
+
+
+def make_cow_step(num_layers: int = 2, seed: Optional[int] = None) -> CowStep:
+    sp = SPECS["shared_prefix"]
+    rng = np.random.default_rng(sp.seed if seed is None else seed)
+    bs = sp.block_size
+    choices = np.array([u for u in range(1, 256) if u % bs != 0])
+    u = rng.choice(choices, size=sp.prompts)
+    parent_lens = (sp.prefix + u).astype(np.int32)
+    need = int(sum(cdiv(int(n), bs) for n in parent_lens)) + sp.prompts * (sp.samples - 1)
+    nb = int(math.ceil(sp.pool_factor * need))
+    order = rng.permutation(nb).astype(np.int32)
+    B = sp.prompts * sp.samples
+
+    def draw(shape):
+        return round_to_bits(rng.standard_normal(shape, dtype=np.float32), sp.dtype)
+
+    q = draw((B, sp.num_heads, sp.head_dim))
+    kc = draw((num_layers, nb, sp.num_kv_heads, bs, sp.head_dim))
+    vc = draw((num_layers, nb, sp.num_kv_heads, bs, sp.head_dim))
+    kn = draw((B, sp.num_kv_heads, sp.head_dim))
+    vn = draw((B, sp.num_kv_heads, sp.head_dim))
+    return CowStep(sp, parent_lens, order, nb, cdiv(sp.max_len, bs), num_layers, q, kc, vc, kn, vn)
