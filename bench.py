@@ -1,0 +1,574 @@
+"""Benchmark of the paged KV-cache decode path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--block-size BS]
+    python bench.py --impl reference ...      # the CPU oracle, timed on the host cores
+
+One step = one decode step of the workload through the whole hot path: for every
+layer, the cache write of this step's tokens (reshape_and_cache), paged decode
+attention (partition kernel, plus the log-sum-exp reduce when a context spans
+several partitions) and, for workloads with shared blocks, the copy-on-write block
+copy before the write. The host block manager runs in the end-to-end loop.
+
+Metric: paged decode attention KV-read GB/s = algorithmic K+V bytes the step reads
+(sum over layers and sequences of len * Hkv * head_dim * 2 * 2 bytes) / step time;
+also decode tokens/s = sequences / step time. Multi-GPU (torchrun): every rank runs
+its own replica of the workload (weak scaling, no collective on the data path);
+the step time is the maximum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from paged_kv_cache_320_b200 import synth  # noqa: E402
+
+WORKLOADS = {
+    "llama7b_mha": "Llama-7B-shaped MHA decode: B 64, 32/32 heads, d 128, fp16, bs 16, "
+                   "lognormal(median 512, sigma 1) clip 16-2048, 32 layers",
+    "llama3_8b_gqa": "Llama-3-8B-shaped GQA decode: B 256, 32q/8kv, d 128, bf16, bs 16, "
+                     "lognormal(median 1024, sigma 1) clip 8-8192, 1 layer, 256 new tokens",
+    "shared_prefix": "shared-prefix parallel sampling: 16 prompts x 8 samples, prefix 1024 "
+                     "(refcount 8), suffix U[0,256], 32q/8kv, d 128, bf16, bs 16, 1 layer",
+    "long_context": "long-context decode: B 8, U[32768,131072], 64q/8kv, d 128, bf16, 1 layer",
+}
+METRIC = "paged decode attention KV-read GB/s (% of B200 HBM peak); decode tokens/s"
+KERNEL_SOURCES = ["paged_kv_cache_320_b200/csrc/decode_kernels.cuh",
+                  "paged_kv_cache_320_b200/csrc/pkv_ptx.cuh"]
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, p), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def read_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def read_traffic(workload, block_size):
+    """dram bytes per launch of the decode partition kernel from the committed ncu
+    summary, only if it was taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", f"paged_decode_partition__{workload}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_hash = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", text)
+    m_bytes = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    m_bs = re.search(r"block_size:\s*(\d+)", text)
+    if not (m_hash and m_bytes) or m_hash.group(1) != kernel_source_hash():
+        return None
+    if m_bs and int(m_bs.group(1)) != block_size:
+        return None
+    return float(m_bytes.group(1))
+
+
+# ----------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ----------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.lines = []
+        target = None
+        try:
+            import torch
+            u = getattr(torch.cuda.get_device_properties(device_index), "uuid", None)
+            if u is not None:
+                target = "GPU-" + str(u)
+        except Exception:
+            target = None
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "50"]
+        if target:
+            cmd += ["-i", target]
+        self.cmd = cmd
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# the GPU arm
+# ----------------------------------------------------------------------------
+def algorithmic_bytes(wl):
+    """Per layer: K+V bytes (the metric) and the full roofline traffic of the decode
+    kernel: K+V + q/out + block-table entries + context lengths."""
+    sp = wl.spec
+    lens = wl.context_lens.astype(np.int64)
+    kv = int(lens.sum()) * sp.num_kv_heads * sp.head_dim * 2 * 2
+    qo = wl.num_seqs * sp.num_heads * sp.head_dim * 2 * 2
+    tables = int(((lens + sp.block_size - 1) // sp.block_size).sum()) * 4 + wl.num_seqs * 4
+    return kv, kv + qo + tables
+
+
+def gpu_arm(args, rank, world, local_rank):
+    import torch
+    import paged_kv_cache_320_b200 as pkv
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    overrides = {}
+    if args.block_size:
+        overrides["block_size"] = args.block_size
+    if args.layers:
+        overrides["num_layers"] = args.layers
+    sp0 = synth.spec(args.workload, **overrides)
+    # block tables wide enough, and pool blocks for, the tokens the end-to-end loop appends
+    grow = args.steps + args.warmup + 1
+    overrides["max_len"] = sp0.max_len + grow + 2 * sp0.block_size
+    nseqs = sp0.batch or len(sp0.lens) or sp0.prompts * sp0.samples
+    overrides["pool_extra"] = nseqs * (-(-grow // sp0.block_size) + 1)
+    # weak scaling: every rank holds its own replica of the same workload
+    wl = synth.make_workload(args.workload, values_on="cuda", device=str(dev), **overrides)
+    sp = wl.spec
+    L = sp.num_layers
+    B = wl.num_seqs
+    dtype_code = pkv.PKV_F16 if sp.dtype == synth.F16 else pkv.PKV_BF16
+    max_len = wl.max_blocks_per_seq * sp.block_size
+    P = pkv.pkv_decode_partition_size(B, sp.num_heads, sp.num_kv_heads, sp.head_dim,
+                                      sp.block_size, max_len, args.partition)
+    pmax = max(1, -(-max_len // P))
+    ws_bytes = pkv.pkv_decode_workspace_size(B, sp.num_heads, sp.num_kv_heads, sp.head_dim,
+                                             sp.block_size, max_len, P)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    bt = torch.from_numpy(wl.block_tables).to(dev)
+    lens = torch.from_numpy(wl.context_lens).to(dev)
+    slots = torch.from_numpy(wl.slot_mapping).to(dev)
+    outs = [torch.empty_like(wl.q[l]) for l in range(L)]
+    stream = torch.cuda.current_stream(dev)
+    kv_layer, roof_layer = algorithmic_bytes(wl)
+    kv_step = kv_layer * L
+
+    k1_events = []
+
+    def step(record=False):
+        for l in range(L):
+            pkv.pkv_reshape_and_cache(wl.k_new[l], wl.v_new[l], wl.k_cache[l], wl.v_cache[l],
+                                      slots, stream=stream)
+            if record:
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+            pkv.pkv_paged_attention_decode(outs[l], wl.q[l], wl.k_cache[l], wl.v_cache[l], bt,
+                                           lens, max_len, scale=wl.scale, partition_size=P,
+                                           workspace=ws, stream=stream)
+            if record:
+                e1.record(stream)
+                k1_events.append((e0, e1))
+
+    launches_per_step = L * (2 + (1 if pmax > 1 else 0))
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    # ---- device-timed region: inputs resident in HBM
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    with ClockSampler(local_rank) as clocks:
+        barrier()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(args.steps):
+            step(record=True)
+        t1.record(stream)
+        barrier()
+    ms_total = t0.elapsed_time(t1)
+    k1_ms = [a.elapsed_time(b) for a, b in k1_events]
+    if pkv.pkv_get_device_status(stream=stream) != 0:
+        raise RuntimeError("device status word set during the benchmark")
+
+    def max_over_ranks(x):
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    ms_total = max_over_ranks(ms_total)
+    ms_step = ms_total / args.steps
+    value = kv_step * world / (ms_step * 1e-3) / 1e9
+    tokens_per_s = B * world / (ms_step * 1e-3)
+    k1_avg_ms = statistics.mean(k1_ms)
+    k1_avg_ms = max_over_ranks(k1_avg_ms)
+    peak, peak_kind = read_peaks()
+    achieved = roof_layer / (k1_avg_ms * 1e-3) / 1e9
+    traffic = read_traffic(args.workload, sp.block_size)
+
+    # ---- end to end: host block manager + pinned host buffers through the public API
+    e2e = e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, world)
+
+    result = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": synth.DTYPE_NAMES[sp.dtype],
+        "data": "synthetic (seeded N(0,1) values, lognormal/uniform lengths, random block placement)",
+        "config": {
+            "workload": args.workload,
+            "description": WORKLOADS[args.workload],
+            "num_seqs": B, "num_heads": sp.num_heads, "num_kv_heads": sp.num_kv_heads,
+            "head_dim": sp.head_dim, "block_size": sp.block_size, "layers": L,
+            "sum_context_tokens": int(wl.context_lens.sum()),
+            "partition_size": P,
+            "kv_bytes_per_step": kv_step,
+            "l2": f"inputs larger than L2: {kv_layer / 1e6:.0f} MB of K/V per layer vs 126 MB L2",
+            "parallelism": f"replicas x{world}",
+        },
+        "tokens_per_s": round(tokens_per_s, 1),
+        "pct_of_hbm_peak": round(100 * value / world / peak, 2),
+        "clocks": clocks.summary(),
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "roofline": {
+            "kernel": "paged_decode_partition_kernel",
+            "bound": "hbm",
+            "achieved": round(achieved, 1),
+            "peak": peak,
+            "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+            else "fallback",
+            "unit": "GB/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": traffic,
+            "algorithmic_bytes_per_launch": roof_layer,
+            "avg_launch_us": round(k1_avg_ms * 1e3, 2),
+        },
+    }
+    return result
+
+
+def replay_block_manager(wl):
+    """Rebuild the workload's block tables with the library's block manager seeded
+    by the workload's placement permutation: sequences appended in order (shared
+    prefix: per prompt, the prefix on the first sample, forks, then each sample's
+    suffix). The result must equal the generated tables exactly."""
+    import paged_kv_cache_320_b200 as pkv
+    sp = wl.spec
+    mgr = pkv.BlockManager(wl.num_blocks, sp.block_size, wl.max_blocks_per_seq, wl.perm)
+
+    def append(s, n):
+        st, _, cows = mgr.pkv_seq_append(s, n)
+        if st != 0 or len(cows):
+            raise RuntimeError(f"block manager replay failed ({st})")
+
+    if sp.prompts:
+        for p in range(sp.prompts):
+            first = p * sp.samples
+            append(first, sp.prefix)
+            for k in range(1, sp.samples):
+                if mgr.pkv_seq_fork(first, first + k) != 0:
+                    raise RuntimeError("fork failed")
+            for i in range(first, first + sp.samples):
+                append(i, int(wl.context_lens[i]) - sp.prefix)
+    else:
+        for s, n in enumerate(wl.context_lens):
+            append(s, int(n))
+    st, tables, lens = mgr.pkv_block_tables(np.arange(wl.num_seqs))
+    if st != 0 or not np.array_equal(tables, wl.block_tables) or not np.array_equal(
+            lens, wl.context_lens):
+        raise RuntimeError("block manager replay does not reproduce the workload's tables")
+    return mgr
+
+
+def e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, world):
+    """Each step: the host block manager appends one token per sequence, the step's
+    inputs (q, k_new, v_new for every layer, slot mapping, block tables, lengths) go
+    host->device from pinned memory, the kernels run, and every layer's output comes
+    back device->host. Timed with CUDA events on the launching stream."""
+    import torch
+    import paged_kv_cache_320_b200 as pkv
+
+    sp = wl.spec
+    L, B = sp.num_layers, wl.num_seqs
+    mgr = replay_block_manager(wl)
+    pin = dict(pin_memory=True)
+    q_h = torch.empty((L,) + tuple(wl.q.shape[1:]), dtype=wl.q.dtype, **pin)
+    q_h.copy_(wl.q.cpu())
+    kn_h = torch.empty(tuple(wl.k_new.shape), dtype=wl.k_new.dtype, **pin)
+    kn_h.copy_(wl.k_new.cpu())
+    vn_h = torch.empty(tuple(wl.v_new.shape), dtype=wl.v_new.dtype, **pin)
+    vn_h.copy_(wl.v_new.cpu())
+    out_h = torch.empty(q_h.shape, dtype=q_h.dtype, **pin)
+    slots_h = torch.empty(B, dtype=torch.int64, **pin)
+    bt_h = torch.empty((B, wl.max_blocks_per_seq), dtype=torch.int32, **pin)
+    lens_h = torch.empty(B, dtype=torch.int32, **pin)
+    q_d, kn_d, vn_d = torch.empty_like(wl.q), torch.empty_like(wl.k_new), torch.empty_like(wl.v_new)
+    out_d = torch.empty_like(wl.q)
+    slots_d = torch.empty(B, dtype=torch.int64, device=dev)
+    bt_d = torch.empty((B, wl.max_blocks_per_seq), dtype=torch.int32, device=dev)
+    lens_d = torch.empty(B, dtype=torch.int32, device=dev)
+    ids = np.arange(B, dtype=np.int64)
+    h2d = (q_h.numel() * 2 + kn_h.numel() * 2 + vn_h.numel() * 2 + slots_h.numel() * 8 +
+           bt_h.numel() * 4 + lens_h.numel() * 4)
+    d2h = out_h.numel() * 2
+    kv_total = [0]
+
+    def one_step():
+        # host: allocate this step's slots (may hand out a new block or a CoW pair)
+        sl = np.empty(B, dtype=np.int64)
+        for s in range(B):
+            st, slot, cows = mgr.pkv_seq_append(s, 1)
+            if st != 0 or len(cows):
+                raise RuntimeError(f"append failed ({st}) or needed a copy in an unshared workload")
+            sl[s] = slot[0]
+        st, tables, lens = mgr.pkv_block_tables(ids)
+        slots_h.numpy()[:] = sl
+        bt_h.numpy()[:] = tables
+        lens_h.numpy()[:] = lens
+        kv_total[0] += int(lens.astype(np.int64).sum()) * sp.num_kv_heads * sp.head_dim * 4 * L
+        q_d.copy_(q_h, non_blocking=True)
+        kn_d.copy_(kn_h, non_blocking=True)
+        vn_d.copy_(vn_h, non_blocking=True)
+        slots_d.copy_(slots_h, non_blocking=True)
+        bt_d.copy_(bt_h, non_blocking=True)
+        lens_d.copy_(lens_h, non_blocking=True)
+        for l in range(L):
+            pkv.pkv_reshape_and_cache(kn_d[l], vn_d[l], wl.k_cache[l], wl.v_cache[l], slots_d,
+                                      stream=stream)
+            pkv.pkv_paged_attention_decode(out_d[l], q_d[l], wl.k_cache[l], wl.v_cache[l], bt_d,
+                                           lens_d, max_len, scale=wl.scale, partition_size=P,
+                                           workspace=ws, stream=stream)
+        out_h.copy_(out_d, non_blocking=True)
+
+    for _ in range(args.warmup):
+        one_step()
+    barrier()
+    kv_total[0] = 0
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        one_step()
+        stream.synchronize()          # the step's result is on the host
+    t1.record(stream)
+    barrier()
+    ms = max_over_ranks(t0.elapsed_time(t1)) / args.steps
+    mgr.close()
+    value = kv_total[0] / args.steps * world / (ms * 1e-3) / 1e9
+    return {"value": round(value, 1), "unit": "GB/s", "ms_per_step": round(ms, 4),
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "includes": "host block-manager appends, block-table export, pinned H2D of "
+                        "q/k_new/v_new/tables, all layers' kernels, D2H of every output"}
+
+
+# ----------------------------------------------------------------------------
+# the CPU oracle (baseline leg and reference arm)
+# ----------------------------------------------------------------------------
+def oracle_sample(workload, block_size, nseq, seed=0):
+    """Host copies of a sample of the workload for the C oracle: the lengths and
+    layout of the first ``nseq`` sequences of layer 0, values drawn with numpy."""
+    overrides = {"block_size": block_size} if block_size else {}
+    wl = synth.make_workload(workload, values_on="none", **overrides)
+    sp = wl.spec
+    bs = sp.block_size
+    lens = wl.context_lens[:nseq].copy()
+    nblk = [-(-int(n) // bs) for n in lens]
+    nb = sum(nblk)
+    rng = np.random.default_rng(sp.seed + 77 + seed)
+    kc = synth.round_to_bits(rng.standard_normal((nb, sp.num_kv_heads, bs, sp.head_dim),
+                                                 dtype=np.float32), sp.dtype)
+    vc = synth.round_to_bits(rng.standard_normal((nb, sp.num_kv_heads, bs, sp.head_dim),
+                                                 dtype=np.float32), sp.dtype)
+    q = synth.round_to_bits(rng.standard_normal((nseq, sp.num_heads, sp.head_dim),
+                                                dtype=np.float32), sp.dtype)
+    kn = synth.round_to_bits(rng.standard_normal((nseq, sp.num_kv_heads, sp.head_dim),
+                                                 dtype=np.float32), sp.dtype)
+    vn = synth.round_to_bits(rng.standard_normal((nseq, sp.num_kv_heads, sp.head_dim),
+                                                 dtype=np.float32), sp.dtype)
+    bt = np.full((nseq, max(nblk)), -1, np.int32)
+    order = rng.permutation(nb).astype(np.int32)
+    off = 0
+    for s in range(nseq):
+        bt[s, :nblk[s]] = order[off:off + nblk[s]]
+        off += nblk[s]
+    last = lens.astype(np.int64) - 1
+    slots = bt[np.arange(nseq), last // bs].astype(np.int64) * bs + last % bs
+    kv = int(lens.astype(np.int64).sum()) * sp.num_kv_heads * sp.head_dim * 4
+    return dict(spec=sp, q=q, kc=kc, vc=vc, kn=kn, vn=vn, bt=bt, lens=lens, slots=slots, kv=kv,
+                scale=1.0 / math.sqrt(sp.head_dim))
+
+
+def oracle_step(smp):
+    from oracle import c_oracle
+    kc, vc = c_oracle.reshape_and_cache(smp["kn"], smp["vn"], smp["kc"], smp["vc"], smp["slots"])
+    c_oracle.paged_decode_attention(smp["q"], kc, vc, smp["bt"], smp["lens"], smp["scale"],
+                                    smp["spec"].dtype)
+
+
+def pick_nseq(workload, block_size):
+    return {"llama7b_mha": 16, "llama3_8b_gqa": 32, "shared_prefix": 16,
+            "long_context": 1}[workload]
+
+
+def cpu_baseline(args):
+    from oracle import c_oracle
+    nseq = pick_nseq(args.workload, args.block_size)
+    smp = oracle_sample(args.workload, args.block_size, nseq)
+    oracle_step(smp)                       # warm-up
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        oracle_step(smp)
+        n += 1
+        if time.perf_counter() - t0 >= args.cpu_seconds:
+            break
+    dt = (time.perf_counter() - t0) / n
+    return {"value": round(smp["kv"] / dt / 1e9, 3), "unit": "GB/s",
+            "cores": c_oracle.num_threads(), "kind": "oracle",
+            "sample": f"layer 0, first {nseq} sequences ({int(smp['lens'].sum())} context tokens) "
+                      f"of the workload: cache write + attention in the plain-C fp64 oracle, "
+                      f"{n} repetitions over {args.cpu_seconds:.0f}+ s"}
+
+
+def reference_arm(args, rank):
+    if rank != 0:
+        return None
+    from oracle import c_oracle
+    c_oracle.build()
+    nseq = pick_nseq(args.workload, args.block_size)
+    smp = oracle_sample(args.workload, args.block_size, nseq)
+    for _ in range(args.warmup):
+        oracle_step(smp)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(smp)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = smp["kv"] / dt / 1e9
+    sp = smp["spec"]
+    sample = (f"each step: layer 0, first {nseq} sequences ({int(smp['lens'].sum())} context "
+              f"tokens) of the workload, cache write + attention, plain-C fp64 oracle")
+    return {
+        "impl": "reference",
+        "metric": METRIC, "value": round(value, 3), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "description": WORKLOADS[args.workload],
+                   "block_size": sp.block_size},
+        "tokens_per_s": round(nseq / dt, 2),
+        "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "kind": "oracle",
+                         "cores": c_oracle.num_threads(), "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="llama7b_mha", choices=sorted(WORKLOADS))
+    ap.add_argument("--block-size", type=int, default=0)
+    ap.add_argument("--layers", type=int, default=0, help="override the workload's layer count")
+    ap.add_argument("--partition", type=int, default=0, help="decode partition size (0 = auto)")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be at least 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        res = reference_arm(args, rank)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    import torch
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    res = gpu_arm(args, rank, world, local_rank)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(args)
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

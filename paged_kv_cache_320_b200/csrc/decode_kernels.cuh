@@ -8,21 +8,24 @@
 // Work decomposition. A work item is (sequence s, KV head hk, partition p): the
 // tokens [p*P, min((p+1)*P, len_s)) of one KV head, for all G query heads that read
 // it, so every K/V byte is read from HBM once. Items are numbered sequence-major
-// (then KV head, then partition); persistent CTAs take items blockIdx.x,
-// blockIdx.x + gridDim.x, ... A sequence with one partition writes `out` directly;
-// otherwise each item leaves (max, sum, normalised partial output) in fp32 scratch
-// and paged_decode_reduce merges them exactly (log-sum-exp).
+// (then KV head, then partition); persistent CTAs (two per SM where shared memory
+// allows) take items blockIdx.x, blockIdx.x + gridDim.x, ... A sequence with one
+// partition writes `out` directly; otherwise each item leaves (max, sum,
+// normalised partial output) in fp32 scratch and paged_decode_reduce merges them
+// exactly (log-sum-exp).
 //
-// Inside a CTA (160 threads): warp 4 is the producer. It walks the item list, reads
-// each item's block-table slice into registers (one coalesced load per lane), and
-// for every 64-token stage issues TMA tile loads of the K and V pages into a ring of
-// shared-memory stages (128-byte swizzle), completing on a per-stage mbarrier.
+// Inside a CTA (160 threads): warp 4 is the producer. It walks the item list one
+// item ahead, prefetching the next item's block-table slice into registers (one
+// coalesced load per lane) while the current one streams, and for every 64-token
+// stage issues one TMA box per page for K and one for V (the whole
+// block_size x head_dim tile, 128-byte swizzle) plus, with an item's first stage,
+// one box for the item's G query rows; all complete on the stage's mbarrier.
 // Warps 0-3 are consumers: each takes 16 of the stage's 64 tokens, computes the
-// scores for the whole GQA group with m16n8k16 tensor-core MMAs (query heads on M,
+// scores of the whole GQA group with m16n8k16 tensor-core MMAs (query heads on M,
 // padded to 16; tokens on N; head_dim on K), keeps an online max / sum in fp32,
-// and accumulates P.V with a second MMA (P kept in registers as the A operand).
-// At the end of an item the four warps merge their partial softmax states through
-// shared memory. Masking is by selection: scores of tokens at or past len_s become
+// and accumulates P.V with a second MMA (P stays in registers as the A operand).
+// At the end of an item the four warps merge their softmax states through
+// shared memory. Masking is by selection: scores of tokens at or past len_s are
 // -inf and their V rows are zeroed in registers, so stale bits (NaN) never reach
 // the result.
 #pragma once
@@ -55,7 +58,6 @@ constexpr int kFirst = 1, kLast = 2, kEnd = 4;
 
 struct DecodeParams {
     void *out;
-    const void *q;
     const int32_t *block_tables;
     const int32_t *context_lens;
     float *ws_o;         // [items * G][D]
@@ -67,19 +69,29 @@ struct DecodeParams {
     float scale_log2;    // scale * log2(e)
 };
 
+// Shared-memory plan. A stage holds 64 tokens of K then V as [token][head_dim]
+// rows (head_dim*2 bytes each); TMA's 128-byte swizzle permutes the 16-byte
+// chunks of every 128-byte line by (line index mod 8), so line L = token*halves +
+// half has chunk c at L*128 + ((c ^ (L & 7)) * 16).
 template <int D>
 struct DecodeLayout {
-    static constexpr int kHalves = D / 64;                     // 128-byte column slabs
-    static constexpr int kSlabBytes = kStageTokens * 128;      // one slab of 64 tokens
-    static constexpr int kKBytes = kHalves * kSlabBytes;
+    static constexpr int kHalves = D / 64;
+    static constexpr int kRowBytes = D * 2;
+    static constexpr int kKBytes = kStageTokens * kRowBytes;
     static constexpr int kStageBytes = 2 * kKBytes;            // K + V
-    static constexpr int kStages = D == 128 ? 4 : 8;
+    static constexpr int kStages = D == 128 ? 3 : 6;
     static constexpr int kRingBytes = kStages * kStageBytes;
     static constexpr int kObufStride = D + 8;                  // floats per merge row
     static constexpr int kMetaBytes = 1024;                    // infos + barriers + ml
+    __host__ __device__ static constexpr int q_slot_bytes(int group) {
+        return (group * kRowBytes + 1023) / 1024 * 1024;
+    }
+    __host__ __device__ static constexpr int obuf_bytes(int group) {
+        return (group * kObufStride * 4 + 127) / 128 * 128;
+    }
     static constexpr size_t smem_bytes(int group) {
-        return 1024 /*alignment slack*/ + kRingBytes + kMetaBytes +
-               (size_t)kConsumerWarps * group * kObufStride * sizeof(float);
+        return 1024 /*alignment slack*/ + kRingBytes + (size_t)kStages * q_slot_bytes(group) +
+               obuf_bytes(group) + kMetaBytes;
     }
 };
 
@@ -98,25 +110,97 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
     return __all_sync(0xffffffffu, mine);
 }
 
+// Byte offset of 16-byte chunk c of 128-byte line L in a 128B-swizzled region.
+__device__ __forceinline__ uint32_t swz(int line, int c) {
+    return (uint32_t)(line * 128 + ((c ^ (line & 7)) << 4));
+}
+
+// Position of one work item in the list (lane-uniform).
+struct ItemPos {
+    int item, s, hk, p, np, ntok, nst, nblk;
+    bool valid;
+};
+
+// Walks the item list in increasing order, 32 sequences at a time (one context
+// length per lane, warp prefix sum of items per sequence).
+struct ItemWalker {
+    int cs = 0, chunk_base = 0, chunk_total = 0, incl = 0, my_items = 0, my_np = 0, my_len = 0;
+    bool loaded = false;
+
+    __device__ ItemPos find(int item, const DecodeParams &prm, int lane) {
+        ItemPos r;
+        r.item = item;
+        r.valid = false;
+        const int B = prm.num_seqs, P = prm.partition, Hkv = prm.num_kv_heads;
+        for (;;) {
+            if (cs >= B) return r;
+            if (!loaded) {
+                const int s = cs + lane;
+                int len = 0;
+                if (s < B) {
+                    len = prm.context_lens[s];
+                    if (len < 0 || len > prm.max_context_len) {
+                        if (blockIdx.x == 0) atomicOr(prm.status, kStatusBadLen);
+                        len = len < 0 ? 0 : prm.max_context_len;
+                    }
+                }
+                my_len = len;
+                my_np = s < B ? max(1, (len + P - 1) / P) : 0;
+                my_items = my_np * Hkv;
+                incl = my_items;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += v;
+                }
+                chunk_total = __shfl_sync(0xffffffffu, incl, 31);
+                loaded = true;
+            }
+            if (item < chunk_base + chunk_total) break;
+            chunk_base += chunk_total;
+            cs += 32;
+            loaded = false;
+        }
+        const unsigned hit = __ballot_sync(0xffffffffu, item < chunk_base + incl);
+        const int ln = __ffs(hit) - 1;
+        const int excl = __shfl_sync(0xffffffffu, incl - my_items, ln);
+        const int len = __shfl_sync(0xffffffffu, my_len, ln);
+        r.s = cs + ln;
+        r.np = __shfl_sync(0xffffffffu, my_np, ln);
+        const int rem = item - chunk_base - excl;
+        r.hk = rem / r.np;
+        r.p = rem - r.hk * r.np;
+        r.ntok = max(0, min(P, len - r.p * P));
+        r.nst = max(1, (r.ntok + kStageTokens - 1) / kStageTokens);
+        r.valid = true;
+        return r;
+    }
+};
+
 template <typename T, int D, int BS>
-__global__ void __launch_bounds__(kDecodeThreads, 1)
+__global__ void __launch_bounds__(kDecodeThreads, 2)
 paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
-                              const __grid_constant__ CUtensorMap tmap_v, DecodeParams prm) {
+                              const __grid_constant__ CUtensorMap tmap_v,
+                              const __grid_constant__ CUtensorMap tmap_q, DecodeParams prm) {
     using L = DecodeLayout<D>;
     constexpr int kBPS = kStageTokens / BS;   // blocks per stage
+    constexpr int H = L::kHalves;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int G = prm.group;
+    const int qslot_bytes = L::q_slot_bytes(G);
     uint8_t *ring = smem;
-    StageInfo *info = reinterpret_cast<StageInfo *>(smem + L::kRingBytes);
+    uint8_t *qring = smem + L::kRingBytes;
+    float *obuf = reinterpret_cast<float *>(qring + L::kStages * qslot_bytes);
+    StageInfo *info = reinterpret_cast<StageInfo *>(reinterpret_cast<uint8_t *>(obuf) +
+                                                    L::obuf_bytes(G));
     uint64_t *full = reinterpret_cast<uint64_t *>(info + L::kStages);
     uint64_t *empty = full + L::kStages;
     float2 *ml = reinterpret_cast<float2 *>(empty + L::kStages);            // [4][16]
-    float *obuf = reinterpret_cast<float *>(smem + L::kRingBytes + L::kMetaBytes);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int G = prm.group;
     const int Hkv = prm.num_kv_heads;
     const int P = prm.partition;
 
@@ -134,70 +218,36 @@ paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
         if (lane == 0) {
             prefetch_tensormap(&tmap_k);
             prefetch_tensormap(&tmap_v);
+            prefetch_tensormap(&tmap_q);
         }
-        const uint64_t policy = l2_evict_first_policy();
-        const int B = prm.num_seqs;
+        const uint64_t kv_policy = l2_evict_first_policy();
+        ItemWalker walker;
         int it = 0;
         bool ok = true;
-        // cursor over chunks of 32 sequences
-        int cs = 0, chunk_base = 0, chunk_total = 0, incl = 0, my_items = 0, my_np = 0,
-            my_len = 0;
-        bool loaded = false;
-        for (int item = blockIdx.x; ok; item += gridDim.x) {
-            bool done = false;
-            for (;;) {
-                if (cs >= B) { done = true; break; }
-                if (!loaded) {
-                    const int s = cs + lane;
-                    int len = 0;
-                    if (s < B) {
-                        len = prm.context_lens[s];
-                        if (len < 0 || len > prm.max_context_len) {
-                            if (blockIdx.x == 0) atomicOr(prm.status, kStatusBadLen);
-                            len = len < 0 ? 0 : prm.max_context_len;
-                        }
-                    }
-                    my_len = len;
-                    my_np = s < B ? max(1, (len + P - 1) / P) : 0;
-                    my_items = my_np * Hkv;
-                    incl = my_items;
-#pragma unroll
-                    for (int o = 1; o < 32; o <<= 1) {
-                        const int v = __shfl_up_sync(0xffffffffu, incl, o);
-                        if (lane >= o) incl += v;
-                    }
-                    chunk_total = __shfl_sync(0xffffffffu, incl, 31);
-                    loaded = true;
-                }
-                if (item < chunk_base + chunk_total) break;
-                chunk_base += chunk_total;
-                cs += 32;
-                loaded = false;
-            }
-            if (done) break;
-            const unsigned hit = __ballot_sync(0xffffffffu, item < chunk_base + incl);
-            const int ln = __ffs(hit) - 1;
-            const int s = cs + ln;
-            const int excl = __shfl_sync(0xffffffffu, incl - my_items, ln);
-            const int np = __shfl_sync(0xffffffffu, my_np, ln);
-            const int len = __shfl_sync(0xffffffffu, my_len, ln);
-            const int r = item - chunk_base - excl;
-            const int hk = r / np;
-            const int p = r - hk * np;
-            const int tok0 = p * P;
-            const int ntok = max(0, min(P, len - tok0));
-            const int nst = max(1, (ntok + kStageTokens - 1) / kStageTokens);
-            const int nblk = (ntok + BS - 1) / BS;
-            if (hk == 0 && p == 0 && lane == 0 && prm.ws_seq_base) prm.ws_seq_base[s] = item;
-            // this item's slice of the block table: entry e lives in lane e%32, reg e/32
-            int ent[kMaxItemBlocks / 32];
-            const int32_t *bt = prm.block_tables + (size_t)s * prm.max_blocks_per_seq + tok0 / BS;
+
+        auto load_entries = [&](const ItemPos &ip, int (&ent)[kMaxItemBlocks / 32]) {
+            const int nblk = ip.valid ? (ip.ntok + BS - 1) / BS : 0;
+            const int32_t *bt = ip.valid ? prm.block_tables +
+                                               (size_t)ip.s * prm.max_blocks_per_seq +
+                                               ip.p * (P / BS)
+                                         : prm.block_tables;
 #pragma unroll
             for (int k = 0; k < kMaxItemBlocks / 32; ++k) {
                 const int e = k * 32 + lane;
                 ent[k] = e < nblk ? bt[e] : 0;
             }
-            for (int st = 0; st < nst; ++st, ++it) {
+        };
+
+        ItemPos cur = walker.find(blockIdx.x, prm, lane);
+        int cur_ent[kMaxItemBlocks / 32];
+        load_entries(cur, cur_ent);
+        while (cur.valid) {
+            if (cur.hk == 0 && cur.p == 0 && lane == 0 && prm.ws_seq_base)
+                prm.ws_seq_base[cur.s] = cur.item;
+            ItemPos nxt;
+            nxt.valid = false;
+            int nxt_ent[kMaxItemBlocks / 32];
+            for (int st = 0; st < cur.nst; ++st, ++it) {
                 const int slot = it % L::kStages;
                 const uint32_t ph = ((it / L::kStages) & 1) ^ 1;
                 if (!warp_wait(smem_u32(&empty[slot]), ph)) {
@@ -205,45 +255,66 @@ paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     ok = false;
                     break;
                 }
-                const int sntok = max(0, min(kStageTokens, ntok - st * kStageTokens));
+                const int sntok = max(0, min(kStageTokens, cur.ntok - st * kStageTokens));
                 const int nb_st = (sntok + BS - 1) / BS;
                 const int e0 = st * kBPS;
                 const int reg = e0 >> 5;
-                int v = ent[0];
+                int v = cur_ent[0];
 #pragma unroll
                 for (int k = 1; k < kMaxItemBlocks / 32; ++k)
-                    if (reg == k) v = ent[k];
+                    if (reg == k) v = cur_ent[k];
                 const int bid = __shfl_sync(0xffffffffu, v, (e0 + lane) & 31);
+                const uint32_t bar = smem_u32(&full[slot]);
                 if (lane == 0) {
                     StageInfo in;
-                    in.s = s; in.hk = hk; in.p = p; in.npart = np; in.item = item;
+                    in.s = cur.s; in.hk = cur.hk; in.p = cur.p; in.npart = cur.np;
+                    in.item = cur.item;
                     in.ntok = sntok;
-                    in.flags = (st == 0 ? kFirst : 0) | (st == nst - 1 ? kLast : 0);
+                    in.flags = (st == 0 ? kFirst : 0) | (st == cur.nst - 1 ? kLast : 0);
                     in.pad = 0;
                     info[slot] = in;
-                    mbar_arrive_expect_tx(smem_u32(&full[slot]),
-                                          (uint32_t)(nb_st * BS * D * 2 * 2));
+                    const uint32_t qbytes = st == 0 ? (uint32_t)(G * L::kRowBytes) : 0u;
+                    mbar_arrive_expect_tx(bar, (uint32_t)(nb_st * BS * L::kRowBytes * 2) + qbytes);
                 }
                 __syncwarp();
+                uint8_t *stage = ring + slot * L::kStageBytes;
                 if (lane < nb_st) {
                     int y;
                     if (bid >= 0 && bid < prm.num_blocks) {
-                        y = (bid * Hkv + hk) * BS;
+                        y = (bid * Hkv + cur.hk) * BS;
                     } else {
                         atomicOr(prm.status, kStatusBadBlock);
                         y = prm.num_blocks * Hkv * BS;   // fully out of range: reads zeros
                     }
-                    uint8_t *stage = ring + slot * L::kStageBytes;
-                    const uint32_t bar = smem_u32(&full[slot]);
-#pragma unroll
-                    for (int hf = 0; hf < L::kHalves; ++hf) {
-                        const uint32_t off = hf * L::kSlabBytes + lane * BS * 128;
-                        tma_load_2d(smem_u32(stage + off), &tmap_k, hf * 64, y, bar, policy);
-                        tma_load_2d(smem_u32(stage + L::kKBytes + off), &tmap_v, hf * 64, y, bar,
-                                    policy);
+                    const uint32_t off = lane * BS * L::kRowBytes;
+                    if (H == 2) {
+                        tma_load_3d(smem_u32(stage + off), &tmap_k, 0, 0, y, bar, kv_policy);
+                        tma_load_3d(smem_u32(stage + L::kKBytes + off), &tmap_v, 0, 0, y, bar,
+                                    kv_policy);
+                    } else {
+                        tma_load_2d(smem_u32(stage + off), &tmap_k, 0, y, bar, kv_policy);
+                        tma_load_2d(smem_u32(stage + L::kKBytes + off), &tmap_v, 0, y, bar,
+                                    kv_policy);
                     }
                 }
+                if (st == 0 && lane == 31) {
+                    const int qrow = cur.s * prm.num_heads + cur.hk * G;
+                    const uint32_t qdst = smem_u32(qring + slot * qslot_bytes);
+                    if (H == 2)
+                        tma_load_3d(qdst, &tmap_q, 0, 0, qrow, bar, kv_policy);
+                    else
+                        tma_load_2d(qdst, &tmap_q, 0, qrow, bar, kv_policy);
+                }
+                if (st == 0) {
+                    // look one item ahead: position and block-table slice
+                    nxt = walker.find(cur.item + gridDim.x, prm, lane);
+                    load_entries(nxt, nxt_ent);
+                }
             }
+            if (!ok) break;
+            cur = nxt;
+#pragma unroll
+            for (int k = 0; k < kMaxItemBlocks / 32; ++k) cur_ent[k] = nxt_ent[k];
         }
         if (ok) {
             const int slot = it % L::kStages;
@@ -278,7 +349,6 @@ paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
     uint32_t qa[KS][4];
     float o[NT][4];
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-    const T *qbase = reinterpret_cast<const T *>(prm.q);
 
     for (int it = 0;; ++it) {
         const int slot = it % L::kStages;
@@ -290,17 +360,17 @@ paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
         if (in.flags & kEnd) break;
 
         if (in.flags & kFirst) {
-            const T *qs = qbase + ((size_t)in.s * prm.num_heads + (size_t)in.hk * G) * D;
-            const bool r0 = gid < G, r1 = gid + 8 < G;
-            const uint32_t *q0 = reinterpret_cast<const uint32_t *>(qs + gid * D);
-            const uint32_t *q1 = reinterpret_cast<const uint32_t *>(qs + (gid + 8) * D);
+            // A fragments of the G query rows (rows >= G are zero)
+            const uint32_t qbase = smem_u32(qring + slot * qslot_bytes);
+            const int mi = lane >> 3;
+            const int row = min((mi & 1) * 8 + (lane & 7), G - 1);
 #pragma unroll
             for (int ks = 0; ks < KS; ++ks) {
-                const int c = ks * 8 + tig;   // 32-bit word index of dims 16ks + 2tig
-                qa[ks][0] = r0 ? __ldg(q0 + c) : 0u;
-                qa[ks][1] = r1 ? __ldg(q1 + c) : 0u;
-                qa[ks][2] = r0 ? __ldg(q0 + c + 4) : 0u;
-                qa[ks][3] = r1 ? __ldg(q1 + c + 4) : 0u;
+                const int hf = ks >> 2;
+                const int c = 2 * (ks & 3) + (mi >> 1);
+                ldsm_x4(qbase + swz(row * H + hf, c), qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3]);
+                if (gid >= G) qa[ks][0] = qa[ks][2] = 0u;
+                if (gid + 8 >= G) qa[ks][1] = qa[ks][3] = 0u;
             }
 #pragma unroll
             for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
@@ -321,14 +391,11 @@ paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 const int t = 16 * w + 8 * nt + (lane & 7);
                 const int mi = lane >> 3;
 #pragma unroll
-                for (int hf = 0; hf < L::kHalves; ++hf) {
+                for (int hf = 0; hf < H; ++hf) {
 #pragma unroll
                     for (int c2 = 0; c2 < 2; ++c2) {
-                        const int c = c2 * 4 + mi;
-                        const uint32_t addr =
-                            kbase + hf * L::kSlabBytes + t * 128 + ((c ^ (t & 7)) << 4);
                         uint32_t b0, b1, b2, b3;
-                        ldsm_x4(addr, b0, b1, b2, b3);
+                        ldsm_x4(kbase + swz(t * H + hf, c2 * 4 + mi), b0, b1, b2, b3);
                         const int ks = hf * 4 + c2 * 2;
                         Mma<T>::run(sc[nt], qa[ks], b0, b1);
                         Mma<T>::run(sc[nt], qa[ks + 1], b2, b3);
@@ -392,10 +459,8 @@ paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
             for (int dp = 0; dp < D / 16; ++dp) {
                 const int hf = dp >> 2;
                 const int c = 2 * (dp & 3) + (mi >> 1);
-                const uint32_t addr =
-                    vbase + hf * L::kSlabBytes + tv * 128 + ((c ^ (tv & 7)) << 4);
                 uint32_t b0, b1, b2, b3;
-                ldsm_x4_trans(addr, b0, b1, b2, b3);
+                ldsm_x4_trans(vbase + swz(tv * H + hf, c), b0, b1, b2, b3);
                 b0 &= keep_lo; b1 &= keep_hi; b2 &= keep_lo; b3 &= keep_hi;
                 Mma<T>::run(o[2 * dp], pa, b0, b1);
                 Mma<T>::run(o[2 * dp + 1], pa, b2, b3);
@@ -416,53 +481,65 @@ paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 ml[w * kMaxGroup + gid + 8] = make_float2(m1, lt1);
             }
             named_bar_sync(1, kConsumerWarps * 32);
+            // my rows' scale factors f = 2^(m_self - M) / L  (0 when the item is empty)
+            float fr[2];
 #pragma unroll
             for (int rr = 0; rr < 2; ++rr) {
-                const int row = gid + 8 * rr;
-                if (row < G) {
-                    float M = -INFINITY;
+                const int row = min(gid + 8 * rr, G - 1);
+                float M = -INFINITY;
 #pragma unroll
-                    for (int ww = 0; ww < kConsumerWarps; ++ww)
-                        M = fmaxf(M, ml[ww * kMaxGroup + row].x);
-                    float Lsum = 0.f;
-                    if (M != -INFINITY) {
+                for (int ww = 0; ww < kConsumerWarps; ++ww)
+                    M = fmaxf(M, ml[ww * kMaxGroup + row].x);
+                float Lsum = 0.f;
+                if (M != -INFINITY) {
 #pragma unroll
-                        for (int ww = 0; ww < kConsumerWarps; ++ww) {
-                            const float2 v = ml[ww * kMaxGroup + row];
-                            Lsum += v.y * ex2(v.x - M);
+                    for (int ww = 0; ww < kConsumerWarps; ++ww) {
+                        const float2 v = ml[ww * kMaxGroup + row];
+                        Lsum += v.y * ex2(v.x - M);
+                    }
+                }
+                const float mself = rr ? m1 : m0;
+                fr[rr] = (Lsum > 0.f) ? ex2(mself - M) / Lsum : 0.f;
+            }
+            // accumulate the four warps' scaled outputs in a fixed order (deterministic)
+#pragma unroll
+            for (int ww = 0; ww < kConsumerWarps; ++ww) {
+                if (w == ww) {
+#pragma unroll
+                    for (int rr = 0; rr < 2; ++rr) {
+                        const int row = gid + 8 * rr;
+                        if (row < G) {
+                            float2 *dst =
+                                reinterpret_cast<float2 *>(obuf + row * L::kObufStride + 2 * tig);
+#pragma unroll
+                            for (int n = 0; n < NT; ++n) {
+                                float2 v = make_float2(o[n][2 * rr] * fr[rr],
+                                                       o[n][2 * rr + 1] * fr[rr]);
+                                if (ww > 0) {
+                                    const float2 prev = dst[n * 4];
+                                    v.x += prev.x;
+                                    v.y += prev.y;
+                                }
+                                dst[n * 4] = v;
+                            }
                         }
                     }
-                    const float mself = rr ? m1 : m0;
-                    const float f = (Lsum > 0.f) ? ex2(mself - M) / Lsum : 0.f;
-                    float *dst = obuf + ((size_t)w * G + row) * L::kObufStride + 2 * tig;
-#pragma unroll
-                    for (int n = 0; n < NT; ++n)
-                        *reinterpret_cast<float2 *>(dst + n * 8) =
-                            make_float2(o[n][2 * rr] * f, o[n][2 * rr + 1] * f);
                 }
+                named_bar_sync(1, kConsumerWarps * 32);
             }
-            named_bar_sync(1, kConsumerWarps * 32);
             const int tid = threadIdx.x;   // 0..127
             if (in.npart == 1) {
                 T *out = reinterpret_cast<T *>(prm.out) +
                          ((size_t)in.s * prm.num_heads + (size_t)in.hk * G) * D;
                 for (int idx = tid; idx < G * D; idx += kConsumerWarps * 32) {
                     const int row = idx / D, dim = idx - row * D;
-                    float acc = 0.f;
-#pragma unroll
-                    for (int ww = 0; ww < kConsumerWarps; ++ww)
-                        acc += obuf[((size_t)ww * G + row) * L::kObufStride + dim];
-                    out[idx] = from_float<T>(acc);
+                    out[idx] = from_float<T>(obuf[row * L::kObufStride + dim]);
                 }
             } else {
                 float *dst = prm.ws_o + (size_t)in.item * G * D;
                 for (int idx = tid; idx < G * D; idx += kConsumerWarps * 32) {
                     const int row = idx / D, dim = idx - row * D;
-                    float acc = 0.f;
-#pragma unroll
-                    for (int ww = 0; ww < kConsumerWarps; ++ww)
-                        acc += obuf[((size_t)ww * G + row) * L::kObufStride + dim];
-                    dst[idx] = acc;
+                    dst[idx] = obuf[row * L::kObufStride + dim];
                 }
                 if (tid < G) {
                     float M = -INFINITY;

@@ -78,21 +78,33 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 2-D view of one layer's cache: rows = num_blocks*Hkv*BS, columns = head_dim;
-// box = 64 columns (128 bytes, swizzled) x BS rows = one slab of one page.
-int encode_cache_map(CUtensorMap *map, const void *base, int dtype, int D, int BS, int NB,
-                     int Hkv) {
+// View of one layer's cache for TMA: rows = num_blocks*Hkv*BS of head_dim elements.
+// head_dim 128: 3-D (64 elements, 2 halves, rows) with a box of one page tile
+// (64 x 2 x BS); head_dim 64: 2-D (64, rows) with a box of 64 x BS. 128-byte swizzle.
+int encode_rows_map(CUtensorMap *map, const void *base, int dtype, int D, long long rows,
+                    int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return PKV_ERR_CUDA;
-    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)NB * Hkv * BS};
-    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-    const cuuint32_t box[2] = {64, (cuuint32_t)BS};
-    const cuuint32_t estr[2] = {1, 1};
-    const CUresult r =
-        fn(map, dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-           2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    const CUtensorMapDataType dt =
+        dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    CUresult r;
+    if (D == 128) {
+        const cuuint64_t dims[3] = {64, 2, (cuuint64_t)rows};
+        const cuuint64_t strides[2] = {128, 256};
+        const cuuint32_t box[3] = {64, 2, (cuuint32_t)box_rows};
+        const cuuint32_t estr[3] = {1, 1, 1};
+        r = fn(map, dt, 3, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    } else {
+        const cuuint64_t dims[2] = {64, (cuuint64_t)rows};
+        const cuuint64_t strides[1] = {128};
+        const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+        const cuuint32_t estr[2] = {1, 1};
+        r = fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    }
     return r == CUDA_SUCCESS ? PKV_OK : PKV_ERR_CUDA;
 }
 
@@ -146,21 +158,27 @@ WsLayout ws_layout(int B, int Hq, int D, int max_len, int P) {
 }
 
 template <typename T, int D, int BS>
-int launch_decode(const CUtensorMap &mk, const CUtensorMap &mv, const pkv::DecodeParams &prm,
-                  long long items_upper, cudaStream_t st) {
+int launch_decode(const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mq,
+                  const pkv::DecodeParams &prm, long long items_upper, cudaStream_t st) {
     using L = pkv::DecodeLayout<D>;
     auto kern = pkv::paged_decode_partition_kernel<T, D, BS>;
     const size_t smem = L::smem_bytes(prm.group);
     int dev;
     if (current_device(&dev) != PKV_OK) return PKV_ERR_CUDA;
     static int occ[kMaxDevices][pkv::kMaxGroup + 1];
+    static bool attr_set[kMaxDevices];
     int nsm;
     if (sm_count(&nsm) != PKV_OK) return PKV_ERR_CUDA;
     int &o = occ[dev][prm.group];
     if (o == 0) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-            cudaSuccess)
-            return PKV_ERR_CUDA;
+        std::lock_guard<std::mutex> lk(g_mu);
+        // the largest layout any group size needs, so every later launch fits
+        if (!attr_set[dev]) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)L::smem_bytes(pkv::kMaxGroup)) != cudaSuccess)
+                return PKV_ERR_CUDA;
+            attr_set[dev] = true;
+        }
         int n = 0;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, pkv::kDecodeThreads, smem) !=
                 cudaSuccess ||
@@ -171,7 +189,7 @@ int launch_decode(const CUtensorMap &mk, const CUtensorMap &mv, const pkv::Decod
     long long grid = (long long)nsm * o;
     if (grid > items_upper) grid = items_upper;
     if (grid < 1) grid = 1;
-    kern<<<(unsigned)grid, pkv::kDecodeThreads, smem, st>>>(mk, mv, prm);
+    kern<<<(unsigned)grid, pkv::kDecodeThreads, smem, st>>>(mk, mv, mq, prm);
     if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
     return PKV_OK;
 }
@@ -185,12 +203,12 @@ int launch_reduce(const pkv::DecodeParams &prm, int pmax, cudaStream_t st) {
 }
 
 template <typename T, int D>
-int dispatch_bs(int BS, const CUtensorMap &mk, const CUtensorMap &mv,
+int dispatch_bs(int BS, const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mq,
                 const pkv::DecodeParams &prm, long long items, cudaStream_t st) {
     switch (BS) {
-        case 8: return launch_decode<T, D, 8>(mk, mv, prm, items, st);
-        case 16: return launch_decode<T, D, 16>(mk, mv, prm, items, st);
-        case 32: return launch_decode<T, D, 32>(mk, mv, prm, items, st);
+        case 8: return launch_decode<T, D, 8>(mk, mv, mq, prm, items, st);
+        case 16: return launch_decode<T, D, 16>(mk, mv, mq, prm, items, st);
+        case 32: return launch_decode<T, D, 32>(mk, mv, mq, prm, items, st);
     }
     return PKV_ERR_INVALID_ARG;
 }
@@ -255,7 +273,7 @@ int pkv_paged_attention_decode(void *out, const void *q, const void *k_cache,
     if (num_seqs == 0) return PKV_OK;
     if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
         return PKV_ERR_INVALID_ARG;
-    if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(q, 4) || !aligned(out, 2) ||
+    if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(q, 16) || !aligned(out, 2) ||
         !aligned(block_tables, 4) || !aligned(context_lens, 4))
         return PKV_ERR_INVALID_ARG;
     const WsLayout ws = ws_layout(num_seqs, num_heads, head_dim, max_context_len, P);
@@ -264,17 +282,19 @@ int pkv_paged_attention_decode(void *out, const void *q, const void *k_cache,
 
     unsigned int *status;
     if ((rc = device_status_ptr(&status)) != PKV_OK) return rc;
-    CUtensorMap mk, mv;
-    if ((rc = encode_cache_map(&mk, k_cache, dtype, head_dim, block_size, num_blocks,
-                               num_kv_heads)) != PKV_OK)
+    CUtensorMap mk, mv, mq;
+    const long long cache_rows = (long long)num_blocks * num_kv_heads * block_size;
+    const int group = num_heads / num_kv_heads;
+    if ((rc = encode_rows_map(&mk, k_cache, dtype, head_dim, cache_rows, block_size)) != PKV_OK)
         return rc;
-    if ((rc = encode_cache_map(&mv, v_cache, dtype, head_dim, block_size, num_blocks,
-                               num_kv_heads)) != PKV_OK)
+    if ((rc = encode_rows_map(&mv, v_cache, dtype, head_dim, cache_rows, block_size)) != PKV_OK)
+        return rc;
+    if ((rc = encode_rows_map(&mq, q, dtype, head_dim, (long long)num_seqs * num_heads, group)) !=
+        PKV_OK)
         return rc;
 
     pkv::DecodeParams prm;
     prm.out = out;
-    prm.q = q;
     prm.block_tables = block_tables;
     prm.context_lens = context_lens;
     uint8_t *wsb = static_cast<uint8_t *>(workspace);
@@ -296,14 +316,14 @@ int pkv_paged_attention_decode(void *out, const void *q, const void *k_cache,
     const long long items = (long long)num_seqs * num_kv_heads * pmax;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (dtype == PKV_BF16) {
-        rc = head_dim == 128 ? dispatch_bs<__nv_bfloat16, 128>(block_size, mk, mv, prm, items, st)
-                             : dispatch_bs<__nv_bfloat16, 64>(block_size, mk, mv, prm, items, st);
+        rc = head_dim == 128 ? dispatch_bs<__nv_bfloat16, 128>(block_size, mk, mv, mq, prm, items, st)
+                             : dispatch_bs<__nv_bfloat16, 64>(block_size, mk, mv, mq, prm, items, st);
         if (rc == PKV_OK && pmax > 1)
             rc = head_dim == 128 ? launch_reduce<__nv_bfloat16, 128>(prm, pmax, st)
                                  : launch_reduce<__nv_bfloat16, 64>(prm, pmax, st);
     } else {
-        rc = head_dim == 128 ? dispatch_bs<__half, 128>(block_size, mk, mv, prm, items, st)
-                             : dispatch_bs<__half, 64>(block_size, mk, mv, prm, items, st);
+        rc = head_dim == 128 ? dispatch_bs<__half, 128>(block_size, mk, mv, mq, prm, items, st)
+                             : dispatch_bs<__half, 64>(block_size, mk, mv, mq, prm, items, st);
         if (rc == PKV_OK && pmax > 1)
             rc = head_dim == 128 ? launch_reduce<__half, 128>(prm, pmax, st)
                                  : launch_reduce<__half, 64>(prm, pmax, st);

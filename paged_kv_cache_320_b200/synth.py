@@ -73,6 +73,7 @@ class Spec:
     batch: int = 0
     pool_blocks: int = 0          # explicit pool size (tiny), else pool_factor * need
     pool_factor: float = 1.2
+    pool_extra: int = 0           # blocks added to the pool (room for tokens appended later)
     max_len: int = 0              # length bound used for max_blocks_per_seq
     prompts: int = 0              # shared prefix: prompts x samples
     samples: int = 0
@@ -162,9 +163,9 @@ class Workload:
 def _placement(sp: Spec, lens: np.ndarray, rng: np.random.Generator):
     """Block tables built by handing out a seeded permutation of the pool in order.
 
-    Sequence s takes the next ceil(len_s / bs) entries of the permutation (shared
-    prefix: each prompt's 1024-token prefix blocks are handed out once and every
-    sample of that prompt points at them)."""
+    Sequence s takes the next ceil(len_s / bs) entries of the permutation. Shared
+    prefix: per prompt, the prefix's blocks are handed out once (every sample of the
+    prompt points at them), then each sample's private suffix blocks in sample order."""
     bs = sp.block_size
     mb = cdiv(sp.max_len, bs)
     if sp.prompts:
@@ -173,21 +174,20 @@ def _placement(sp: Spec, lens: np.ndarray, rng: np.random.Generator):
         need = sp.prompts * pre_blocks + sum(own)
     else:
         need = int(sum(cdiv(int(n), bs) for n in lens))
-    nb = sp.pool_blocks or int(math.ceil(sp.pool_factor * need))
+    nb = (sp.pool_blocks or int(math.ceil(sp.pool_factor * need))) + sp.pool_extra
     perm = rng.permutation(nb).astype(np.int32)
     bt = np.full((len(lens), mb), -1, dtype=np.int32)
     off = 0
     if sp.prompts:
-        prefix_ids = []
+        # per prompt: its prefix blocks, then each of its samples' private blocks
         for p in range(sp.prompts):
-            prefix_ids.append(perm[off:off + pre_blocks])
+            prefix_ids = perm[off:off + pre_blocks]
             off += pre_blocks
-        for i, n in enumerate(lens):
-            p = i // sp.samples
-            bt[i, :pre_blocks] = prefix_ids[p]
-            k = own[i]
-            bt[i, pre_blocks:pre_blocks + k] = perm[off:off + k]
-            off += k
+            for i in range(p * sp.samples, (p + 1) * sp.samples):
+                bt[i, :pre_blocks] = prefix_ids
+                k = own[i]
+                bt[i, pre_blocks:pre_blocks + k] = perm[off:off + k]
+                off += k
     else:
         for i, n in enumerate(lens):
             k = cdiv(int(n), bs)
