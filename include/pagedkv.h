@@ -105,6 +105,40 @@ int pkv_paged_attention_decode(void *out, const void *q, const void *k_cache,
                                float scale, int dtype, int partition_size, void *workspace,
                                size_t workspace_bytes, pkv_stream_t stream);
 
+/* ------------------------------------------------------------------------------
+ * pkv_paged_attention_decode for callers that cannot allocate device memory.
+ * The paper has no counterpart: this is a library convenience.
+ *
+ * Some callers may not call cudaMalloc at all: plugin code inside a host framework
+ * that owns every device allocation and hands the plugin only its input and output
+ * buffers, serving loops that reserve all HBM for the KV pool up front, and latency-
+ * critical code where an allocation may synchronise the device. This entry point
+ * takes the same arguments as pkv_paged_attention_decode minus the workspace; the
+ * partition scratch is a fixed array inside the library of PKV_NOALLOC_SCRATCH_BYTES
+ * per device (every GPU that loads the library holds it until the process exits).
+ * It calls no cudaMalloc, cudaFree or other allocating routine.
+ *
+ * - Sizes whose scratch (pkv_decode_workspace_size) exceeds PKV_NOALLOC_SCRATCH_BYTES
+ *   are rejected with PKV_ERR_WORKSPACE before any device work; a larger
+ *   partition_size needs less scratch.
+ * - The first call on a device looks up the scratch array's device address (once per
+ *   device, with that device current); make that first call before any stream capture.
+ * - Every call on a device shares the one array, which keeps the last call's
+ *   contents (nothing in it needs to start at zero). Calls that can overlap on the
+ *   GPU (unordered streams, several host threads) race on it and corrupt each
+ *   other's results: order them on one stream.
+ * Errors: as pkv_paged_attention_decode, plus PKV_ERR_CUDA if the address lookup fails.
+ * ---------------------------------------------------------------------------- */
+#define PKV_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+
+int pkv_paged_attention_decode_noalloc(void *out, const void *q, const void *k_cache,
+                                       const void *v_cache, const int32_t *block_tables,
+                                       const int32_t *context_lens, int num_seqs, int num_heads,
+                                       int num_kv_heads, int head_dim, int block_size,
+                                       int max_blocks_per_seq, int num_blocks,
+                                       int max_context_len, float scale, int dtype,
+                                       int partition_size, pkv_stream_t stream);
+
 /* Workspace bytes pkv_paged_attention_decode needs for these sizes (0 when the
  * given partition size makes every context a single partition). Same argument
  * meaning as the decode call. */

@@ -14,6 +14,7 @@ from ._binding import (  # noqa: F401
     pkv_decode_workspace_size,
     pkv_get_device_status,
     pkv_paged_attention_decode,
+    pkv_paged_attention_decode_noalloc,
     pkv_reshape_and_cache,
 )
 from ._binding import PKV_BF16, PKV_F16  # noqa: F401

@@ -56,6 +56,8 @@ def lib() -> ctypes.CDLL:
         L.pkv_status_string.restype = ctypes.c_char_p
         L.pkv_paged_attention_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I,
                                                  ctypes.c_float, I, I, P, SZ, P]
+        L.pkv_paged_attention_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I,
+                                                         I, I, ctypes.c_float, I, I, P]
         L.pkv_decode_workspace_size.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(SZ)]
         L.pkv_decode_partition_size.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(I)]
         L.pkv_reshape_and_cache.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P]
@@ -69,7 +71,8 @@ def lib() -> ctypes.CDLL:
         L.pkv_block_tables.argtypes = [P, P, I, P, P]
         L.pkv_stats.argtypes = [P, ctypes.POINTER(I), ctypes.POINTER(I),
                                 ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_double)]
-        for name in ("pkv_paged_attention_decode", "pkv_decode_workspace_size",
+        for name in ("pkv_paged_attention_decode", "pkv_paged_attention_decode_noalloc",
+                     "pkv_decode_workspace_size",
                      "pkv_decode_partition_size", "pkv_reshape_and_cache", "pkv_copy_blocks",
                      "pkv_get_device_status", "pkv_alloc_create", "pkv_alloc_destroy",
                      "pkv_seq_append", "pkv_seq_fork", "pkv_seq_free", "pkv_block_tables",
@@ -156,6 +159,26 @@ def pkv_paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_l
         B, Hq, Hkv, D, BS, block_tables.shape[1], NB, int(max_context_len), float(scale),
         _dtype_code(q), int(partition_size), ws_ptr, ws_bytes, _stream(stream)),
         "pkv_paged_attention_decode")
+    return out
+
+
+def pkv_paged_attention_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens,
+                                       max_context_len, scale=None, partition_size=0,
+                                       stream=None):
+    """pkv_paged_attention_decode without a workspace: the library's fixed scratch
+    array is used instead (see pagedkv.h); raises PagedKVError(PKV_ERR_WORKSPACE)
+    when the sizes need more scratch than it holds."""
+    B, Hq, D = q.shape
+    NB, Hkv, BS, D2 = k_cache.shape
+    if D2 != D or out.shape != q.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    _check(lib().pkv_paged_attention_decode_noalloc(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
+        B, Hq, Hkv, D, BS, block_tables.shape[1], NB, int(max_context_len), float(scale),
+        _dtype_code(q), int(partition_size), _stream(stream)),
+        "pkv_paged_attention_decode_noalloc")
     return out
 
 

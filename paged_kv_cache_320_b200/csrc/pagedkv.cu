@@ -43,6 +43,27 @@ int device_status_ptr(unsigned int **out) {
     return PKV_OK;
 }
 
+// Scratch of pkv_paged_attention_decode_noalloc: a fixed device array (one copy per
+// device that loads the library). Host code must not pass the symbol itself to a
+// kernel (on the host it only names the array); its device address is looked up
+// once per device with cudaGetSymbolAddress.
+constexpr size_t kNoAllocScratchBytes = PKV_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+void *g_noalloc_ptr[kMaxDevices];
+
+int noalloc_scratch_ptr(void **out) {
+    int dev;
+    if (current_device(&dev) != PKV_OK) return PKV_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return PKV_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return PKV_OK;
+}
+
 int sm_count(int *out) {
     int dev;
     if (current_device(&dev) != PKV_OK) return PKV_ERR_CUDA;
@@ -329,6 +350,31 @@ int pkv_paged_attention_decode(void *out, const void *q, const void *k_cache,
                                  : launch_reduce<__half, 64>(prm, pmax, st);
     }
     return rc;
+}
+
+int pkv_paged_attention_decode_noalloc(void *out, const void *q, const void *k_cache,
+                                       const void *v_cache, const int32_t *block_tables,
+                                       const int32_t *context_lens, int num_seqs, int num_heads,
+                                       int num_kv_heads, int head_dim, int block_size,
+                                       int max_blocks_per_seq, int num_blocks,
+                                       int max_context_len, float scale, int dtype,
+                                       int partition_size, pkv_stream_t stream) {
+    int P;
+    const int rc = check_decode_sizes(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                      max_context_len, partition_size, &P);
+    if (rc != PKV_OK) return rc;
+    const size_t need = ws_layout(num_seqs, num_heads, head_dim, max_context_len, P).total;
+    if (need > kNoAllocScratchBytes) return PKV_ERR_WORKSPACE;
+    void *scratch = nullptr;
+    if (need > 0) {
+        const int r = noalloc_scratch_ptr(&scratch);
+        if (r != PKV_OK) return r;
+    }
+    return pkv_paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens,
+                                      num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                      max_blocks_per_seq, num_blocks, max_context_len, scale,
+                                      dtype, P, scratch, need > 0 ? kNoAllocScratchBytes : 0,
+                                      stream);
 }
 
 int pkv_reshape_and_cache(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
