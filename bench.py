@@ -172,6 +172,8 @@ def gpu_arm(args, rank, world, local_rank):
         overrides["block_size"] = args.block_size
     if args.layers:
         overrides["num_layers"] = args.layers
+    if args.batch:
+        overrides["batch"] = args.batch
     sp0 = synth.spec(args.workload, **overrides)
     # block tables wide enough, and pool blocks for, the tokens the end-to-end loop appends
     grow = args.steps + args.warmup + 1
@@ -190,7 +192,7 @@ def gpu_arm(args, rank, world, local_rank):
     pmax = max(1, -(-max_len // P))
     ws_bytes = pkv.pkv_decode_workspace_size(B, sp.num_heads, sp.num_kv_heads, sp.head_dim,
                                              sp.block_size, max_len, P)
-    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    ws = torch.zeros(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
     bt = torch.from_numpy(wl.block_tables).to(dev)
     lens = torch.from_numpy(wl.context_lens).to(dev)
     slots = torch.from_numpy(wl.slot_mapping).to(dev)
@@ -259,6 +261,7 @@ def gpu_arm(args, rank, world, local_rank):
     k1_avg_ms = max_over_ranks(k1_avg_ms)
     peak, peak_kind = read_peaks()
     achieved = roof_layer / (k1_avg_ms * 1e-3) / 1e9
+    read_probe = hbm_read_probe(dev, stream)
     traffic = read_traffic(args.workload, sp.block_size)
 
     # ---- end to end: host block manager + pinned host buffers through the public API
@@ -304,6 +307,7 @@ def gpu_arm(args, rank, world, local_rank):
             "frac": round(achieved / peak, 4),
             "traffic": traffic,
             "algorithmic_bytes_per_launch": roof_layer,
+            "hbm_read_probe_gbs": round(read_probe, 1),
             "avg_launch_us": round(k1_avg_ms * 1e3, 2),
         },
     }
@@ -341,6 +345,24 @@ def replay_block_manager(wl):
             lens, wl.context_lens):
         raise RuntimeError("block manager replay does not reproduce the workload's tables")
     return mgr
+
+
+def hbm_read_probe(dev, stream):
+    """Streaming-read bandwidth on this GPU (context for the roofline, not its
+    denominator): a 4 GiB fp32 sum, best of 5, timed with CUDA events."""
+    import torch
+    x = torch.ones(1 << 30, dtype=torch.float32, device=dev)
+    best = float("inf")
+    for _ in range(6):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        torch.sum(x)
+        b.record(stream)
+        b.synchronize()
+        best = min(best, a.elapsed_time(b))
+    del x
+    return (1 << 32) / (best * 1e-3) / 1e9
 
 
 def e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, world):
@@ -535,6 +557,8 @@ def main():
     ap.add_argument("--block-size", type=int, default=0)
     ap.add_argument("--layers", type=int, default=0, help="override the workload's layer count")
     ap.add_argument("--partition", type=int, default=0, help="decode partition size (0 = auto)")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the sequence count of a length-distribution workload")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -12,7 +12,8 @@ import math
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libpagedkv.so")
+# PAGEDKV_LIB may name a library built elsewhere (e.g. with other compile options)
+LIB_PATH = os.environ.get("PAGEDKV_LIB") or os.path.join(HERE, "libpagedkv.so")
 
 PKV_OK = 0
 PKV_ERR_INVALID_ARG = -1

@@ -9,7 +9,8 @@
 // tokens [p*P, min((p+1)*P, len_s)) of one KV head, for all G query heads that read
 // it, so every K/V byte is read from HBM once. Items are numbered sequence-major
 // (then KV head, then partition); persistent CTAs (two per SM where shared memory
-// allows) take items blockIdx.x, blockIdx.x + gridDim.x, ... A sequence with one
+// allows) take the next free item from a counter in the workspace (or, without
+// one, items blockIdx.x, blockIdx.x + gridDim.x, ...). A sequence with one
 // partition writes `out` directly; otherwise each item leaves (max, sum,
 // normalised partial output) in fp32 scratch and paged_decode_reduce merges them
 // exactly (log-sum-exp).
@@ -34,6 +35,12 @@
 
 namespace pkv {
 
+// L2 policy of the K/V tile loads: evict-first (each byte is read once per call)
+// unless built with PKV_KV_EVICT_FIRST=0.
+#ifndef PKV_KV_EVICT_FIRST
+#define PKV_KV_EVICT_FIRST 1
+#endif
+
 constexpr int kStageTokens = 64;
 constexpr int kConsumerWarps = 4;
 constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
@@ -56,7 +63,19 @@ struct StageInfo {
 };
 constexpr int kFirst = 1, kLast = 2, kEnd = 4;
 
+// Dynamic work distribution: producers take item indices from `next`. The reduce
+// kernel, which follows every decode that has a workspace, re-arms it (next = 0,
+// armed = kSchedArmed) for the next call; a header that is not armed (a workspace
+// never used before) makes that call fall back to the static schedule.
+constexpr unsigned kSchedArmed = 0x9A6EDC0Du;
+struct SchedHeader {
+    unsigned armed;
+    int next;
+    int pad[62];
+};
+
 struct DecodeParams {
+    SchedHeader *sched;  // null: static schedule (items blockIdx.x + k * gridDim.x)
     void *out;
     const int32_t *block_tables;
     const int32_t *context_lens;
@@ -113,6 +132,15 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
 // Byte offset of 16-byte chunk c of 128-byte line L in a 128B-swizzled region.
 __device__ __forceinline__ uint32_t swz(int line, int c) {
     return (uint32_t)(line * 128 + ((c ^ (line & 7)) << 4));
+}
+
+// Line of (stage token t, column half h) in a stage: each page tile lands as
+// [half][row][64 elements], so eight consecutive tokens of one half occupy eight
+// consecutive lines (eight different swizzle phases: conflict-free ldmatrix).
+template <int H, int BS>
+__device__ __forceinline__ int kv_line(int t, int h) {
+    if (H == 1) return t;
+    return (t / BS) * (2 * BS) + h * BS + (t % BS);
 }
 
 // Position of one work item in the list (lane-uniform).
@@ -220,27 +248,45 @@ paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
             prefetch_tensormap(&tmap_v);
             prefetch_tensormap(&tmap_q);
         }
+#if PKV_KV_EVICT_FIRST
         const uint64_t kv_policy = l2_evict_first_policy();
+#else
+        const uint64_t kv_policy = l2_evict_normal_policy();
+#endif
         ItemWalker walker;
         int it = 0;
         bool ok = true;
 
-        auto load_entries = [&](const ItemPos &ip, int (&ent)[kMaxItemBlocks / 32]) {
-            const int nblk = ip.valid ? (ip.ntok + BS - 1) / BS : 0;
-            const int32_t *bt = ip.valid ? prm.block_tables +
-                                               (size_t)ip.s * prm.max_blocks_per_seq +
-                                               ip.p * (P / BS)
-                                         : prm.block_tables;
-#pragma unroll
-            for (int k = 0; k < kMaxItemBlocks / 32; ++k) {
-                const int e = k * 32 + lane;
-                ent[k] = e < nblk ? bt[e] : 0;
-            }
-        };
+        // this item's slice of the block table: entry e lives in lane e % 32, register e / 32
+#define PKV_LOAD_ENTRIES(ip, ent)                                                         \
+    {                                                                                   \
+        const int nblk_ = (ip).valid ? ((ip).ntok + BS - 1) / BS : 0;                   \
+        const int32_t *bt_ = prm.block_tables +                                         \
+                             ((ip).valid ? (size_t)(ip).s * prm.max_blocks_per_seq +    \
+                                               (size_t)(ip).p * (P / BS)                \
+                                         : 0);                                          \
+        _Pragma("unroll") for (int k_ = 0; k_ < kMaxItemBlocks / 32; ++k_) {            \
+            const int e_ = k_ * 32 + lane;                                              \
+            ent[k_] = e_ < nblk_ ? bt_[e_] : 0;                                         \
+        }                                                                               \
+    }
 
-        ItemPos cur = walker.find(blockIdx.x, prm, lane);
+        // dynamic schedule when the workspace header is armed (read before any CTA
+        // can change it: no CTA takes from `next` unless it saw the header armed)
+        const bool dynamic = prm.sched != nullptr &&
+                             __shfl_sync(0xffffffffu, lane == 0 ? *(volatile unsigned *)&prm.sched->armed : 0u, 0) == kSchedArmed;
+        // A ticket is requested one item before it is resolved, so the atomic's
+        // latency overlaps a whole item; the value lives in lane 0 until used.
+        auto request = [&](int static_item) {
+            int v = static_item;
+            if (dynamic && lane == 0) v = atomicAdd(&prm.sched->next, 1);
+            return v;
+        };
+        auto redeem = [&](int ticket) { return __shfl_sync(0xffffffffu, ticket, 0); };
+        ItemPos cur = walker.find(redeem(request(blockIdx.x)), prm, lane);
+        int pending = request(cur.item + gridDim.x);
         int cur_ent[kMaxItemBlocks / 32];
-        load_entries(cur, cur_ent);
+        PKV_LOAD_ENTRIES(cur, cur_ent);
         while (cur.valid) {
             if (cur.hk == 0 && cur.p == 0 && lane == 0 && prm.ws_seq_base)
                 prm.ws_seq_base[cur.s] = cur.item;
@@ -288,8 +334,8 @@ paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     }
                     const uint32_t off = lane * BS * L::kRowBytes;
                     if (H == 2) {
-                        tma_load_3d(smem_u32(stage + off), &tmap_k, 0, 0, y, bar, kv_policy);
-                        tma_load_3d(smem_u32(stage + L::kKBytes + off), &tmap_v, 0, 0, y, bar,
+                        tma_load_3d(smem_u32(stage + off), &tmap_k, 0, y, 0, bar, kv_policy);
+                        tma_load_3d(smem_u32(stage + L::kKBytes + off), &tmap_v, 0, y, 0, bar,
                                     kv_policy);
                     } else {
                         tma_load_2d(smem_u32(stage + off), &tmap_k, 0, y, bar, kv_policy);
@@ -301,14 +347,15 @@ paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     const int qrow = cur.s * prm.num_heads + cur.hk * G;
                     const uint32_t qdst = smem_u32(qring + slot * qslot_bytes);
                     if (H == 2)
-                        tma_load_3d(qdst, &tmap_q, 0, 0, qrow, bar, kv_policy);
+                        tma_load_3d(qdst, &tmap_q, 0, qrow, 0, bar, kv_policy);
                     else
                         tma_load_2d(qdst, &tmap_q, 0, qrow, bar, kv_policy);
                 }
                 if (st == 0) {
                     // look one item ahead: position and block-table slice
-                    nxt = walker.find(cur.item + gridDim.x, prm, lane);
-                    load_entries(nxt, nxt_ent);
+                    nxt = walker.find(redeem(pending), prm, lane);
+                    PKV_LOAD_ENTRIES(nxt, nxt_ent);
+                    if (nxt.valid) pending = request(nxt.item + gridDim.x);
                 }
             }
             if (!ok) break;
@@ -316,6 +363,7 @@ paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
 #pragma unroll
             for (int k = 0; k < kMaxItemBlocks / 32; ++k) cur_ent[k] = nxt_ent[k];
         }
+#undef PKV_LOAD_ENTRIES
         if (ok) {
             const int slot = it % L::kStages;
             const uint32_t ph = ((it / L::kStages) & 1) ^ 1;
@@ -368,7 +416,7 @@ paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
             for (int ks = 0; ks < KS; ++ks) {
                 const int hf = ks >> 2;
                 const int c = 2 * (ks & 3) + (mi >> 1);
-                ldsm_x4(qbase + swz(row * H + hf, c), qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3]);
+                ldsm_x4(qbase + swz(hf * G + row, c), qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3]);
                 if (gid >= G) qa[ks][0] = qa[ks][2] = 0u;
                 if (gid + 8 >= G) qa[ks][1] = qa[ks][3] = 0u;
             }
@@ -395,7 +443,7 @@ paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
 #pragma unroll
                     for (int c2 = 0; c2 < 2; ++c2) {
                         uint32_t b0, b1, b2, b3;
-                        ldsm_x4(kbase + swz(t * H + hf, c2 * 4 + mi), b0, b1, b2, b3);
+                        ldsm_x4(kbase + swz(kv_line<H, BS>(t, hf), c2 * 4 + mi), b0, b1, b2, b3);
                         const int ks = hf * 4 + c2 * 2;
                         Mma<T>::run(sc[nt], qa[ks], b0, b1);
                         Mma<T>::run(sc[nt], qa[ks + 1], b2, b3);
@@ -460,7 +508,7 @@ paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 const int hf = dp >> 2;
                 const int c = 2 * (dp & 3) + (mi >> 1);
                 uint32_t b0, b1, b2, b3;
-                ldsm_x4_trans(vbase + swz(tv * H + hf, c), b0, b1, b2, b3);
+                ldsm_x4_trans(vbase + swz(kv_line<H, BS>(tv, hf), c), b0, b1, b2, b3);
                 b0 &= keep_lo; b1 &= keep_hi; b2 &= keep_lo; b3 &= keep_hi;
                 Mma<T>::run(o[2 * dp], pa, b0, b1);
                 Mma<T>::run(o[2 * dp + 1], pa, b2, b3);
@@ -567,6 +615,12 @@ __global__ void __launch_bounds__(D)
 paged_decode_reduce_kernel(DecodeParams prm) {
     const int h = blockIdx.x;
     const int s = blockIdx.y;
+    if (h == 0 && s == 0 && threadIdx.x == 0 && prm.sched) {
+        // every decode CTA has finished (stream order): re-arm the scheduler
+        prm.sched->next = 0;
+        __threadfence();
+        prm.sched->armed = kSchedArmed;
+    }
     int len = prm.context_lens[s];
     len = len < 0 ? 0 : (len > prm.max_context_len ? prm.max_context_len : len);
     const int P = prm.partition;

@@ -100,8 +100,9 @@ EncodeTiledFn encode_fn() {
 }
 
 // View of one layer's cache for TMA: rows = num_blocks*Hkv*BS of head_dim elements.
-// head_dim 128: 3-D (64 elements, 2 halves, rows) with a box of one page tile
-// (64 x 2 x BS); head_dim 64: 2-D (64, rows) with a box of 64 x BS. 128-byte swizzle.
+// head_dim 128: 3-D (64 elements, rows, 2 halves of a row) with a box of one page tile
+// (64 x BS x 2), landing half-major in shared memory; head_dim 64: 2-D (64, rows) with a
+// box of 64 x BS. 128-byte swizzle.
 int encode_rows_map(CUtensorMap *map, const void *base, int dtype, int D, long long rows,
                     int box_rows) {
     EncodeTiledFn fn = encode_fn();
@@ -110,9 +111,9 @@ int encode_rows_map(CUtensorMap *map, const void *base, int dtype, int D, long l
         dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     CUresult r;
     if (D == 128) {
-        const cuuint64_t dims[3] = {64, 2, (cuuint64_t)rows};
-        const cuuint64_t strides[2] = {128, 256};
-        const cuuint32_t box[3] = {64, 2, (cuuint32_t)box_rows};
+        const cuuint64_t dims[3] = {64, (cuuint64_t)rows, 2};
+        const cuuint64_t strides[2] = {256, 128};
+        const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 2};
         const cuuint32_t estr[3] = {1, 1, 1};
         r = fn(map, dt, 3, const_cast<void *>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -163,16 +164,19 @@ int check_decode_sizes(int B, int Hq, int Hkv, int D, int BS, int max_len, int p
     return PKV_OK;
 }
 
+// Workspace: [scheduler header 256 B][first item of each sequence][partials (max,
+// sum)][partial outputs]. Only needed when some context spans several partitions.
 struct WsLayout {
-    size_t ml, o, total;
+    size_t seq_base, ml, o, total;
 };
 
 WsLayout ws_layout(int B, int Hq, int D, int max_len, int P) {
-    WsLayout w{0, 0, 0};
+    WsLayout w{0, 0, 0, 0};
     const long long pmax = max_len <= P ? 1 : cdiv(max_len, P);
     if (pmax <= 1 || B == 0) return w;
     const size_t rows = (size_t)B * Hq * pmax;
-    w.ml = align_up((size_t)B * sizeof(int32_t), 256);
+    w.seq_base = sizeof(pkv::SchedHeader);
+    w.ml = w.seq_base + align_up((size_t)B * sizeof(int32_t), 256);
     w.o = w.ml + align_up(rows * 2 * sizeof(float), 256);
     w.total = w.o + rows * D * sizeof(float);
     return w;
@@ -319,7 +323,8 @@ int pkv_paged_attention_decode(void *out, const void *q, const void *k_cache,
     prm.block_tables = block_tables;
     prm.context_lens = context_lens;
     uint8_t *wsb = static_cast<uint8_t *>(workspace);
-    prm.ws_seq_base = ws.total ? reinterpret_cast<int32_t *>(wsb) : nullptr;
+    prm.sched = ws.total ? reinterpret_cast<pkv::SchedHeader *>(wsb) : nullptr;
+    prm.ws_seq_base = ws.total ? reinterpret_cast<int32_t *>(wsb + ws.seq_base) : nullptr;
     prm.ws_ml = ws.total ? reinterpret_cast<float *>(wsb + ws.ml) : nullptr;
     prm.ws_o = ws.total ? reinterpret_cast<float *>(wsb + ws.o) : nullptr;
     prm.status = status;

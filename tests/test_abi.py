@@ -55,9 +55,10 @@ def test_decode_size_checks(args):
 def test_workspace_size_formula():
     # single partition -> no workspace
     assert pkv.pkv_decode_workspace_size(4, 8, 8, 64, 16, 100, 128) == 0
-    # B=2, Hq=4, D=64, max_len=300, P=128 -> 3 partitions
+    # B=2, Hq=4, D=64, max_len=300, P=128 -> 3 partitions;
+    # scheduler header + first item per sequence + (max, sum) rows + output rows
     rows = 2 * 4 * 3
-    expect = 256 + ((rows * 8 + 255) // 256) * 256 + rows * 64 * 4
+    expect = 256 + 256 + ((rows * 8 + 255) // 256) * 256 + rows * 64 * 4
     assert pkv.pkv_decode_workspace_size(2, 4, 2, 64, 16, 300, 128) == expect
 
 
