@@ -65,20 +65,18 @@ def read_peaks():
 
 
 def read_traffic(workload, block_size):
-    """dram bytes per launch of the decode partition kernel from the committed ncu
-    summary, only if it was taken on the current kernel source."""
+    """DRAM bytes (read + write) per launch of the decode partition kernel from the
+    committed ncu summary for this workload and block size, only if it was taken on
+    the current kernel source; else None."""
     path = os.path.join(ROOT, "profiles", f"paged_decode_partition__{workload}.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
     m_hash = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", text)
-    m_bytes = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    m_bs = re.search(r"block_size:\s*(\d+)", text)
-    if not (m_hash and m_bytes) or m_hash.group(1) != kernel_source_hash():
+    if not m_hash or m_hash.group(1) != kernel_source_hash():
         return None
-    if m_bs and int(m_bs.group(1)) != block_size:
-        return None
-    return float(m_bytes.group(1))
+    m = re.search(r"traffic_bytes_per_launch\[block_size=%d\]:\s*([0-9]+)" % block_size, text)
+    return float(m.group(1)) if m else None
 
 
 # ----------------------------------------------------------------------------
@@ -159,6 +157,23 @@ def algorithmic_bytes(wl):
     qo = wl.num_seqs * sp.num_heads * sp.head_dim * 2 * 2
     tables = int(((lens + sp.block_size - 1) // sp.block_size).sum()) * 4 + wl.num_seqs * 4
     return kv, kv + qo + tables
+
+
+def reduce_max(x, dist, device):
+    """Maximum of a per-rank scalar over all ranks (the identity on one process)."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_rates(kv_bytes_per_rank_step, seqs_per_rank, world, ms_step):
+    """Whole-job rates when every rank runs its own replica for the same step time
+    (the slowest rank's): K/V GB/s and decode tokens/s summed over ranks."""
+    sec = ms_step * 1e-3
+    return kv_bytes_per_rank_step * world / sec / 1e9, seqs_per_rank * world / sec
 
 
 def gpu_arm(args, rank, world, local_rank):
@@ -247,16 +262,11 @@ def gpu_arm(args, rank, world, local_rank):
         raise RuntimeError("device status word set during the benchmark")
 
     def max_over_ranks(x):
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(x, dist, dev)
 
     ms_total = max_over_ranks(ms_total)
     ms_step = ms_total / args.steps
-    value = kv_step * world / (ms_step * 1e-3) / 1e9
-    tokens_per_s = B * world / (ms_step * 1e-3)
+    value, tokens_per_s = weak_scaling_rates(kv_step, B, world, ms_step)
     k1_avg_ms = statistics.mean(k1_ms)
     k1_avg_ms = max_over_ranks(k1_avg_ms)
     peak, peak_kind = read_peaks()

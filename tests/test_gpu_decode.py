@@ -230,3 +230,34 @@ def test_shared_prefix_decode_sampled(cuda_device):
 def test_long_context_sampled(cuda_device, bs):
     wl = synth.make_workload("long_context", values_on="cuda", block_size=bs)
     full_step_and_sample(wl, 0, 2)
+
+
+def test_one_workspace_reused_across_calls_and_batch_sizes(cuda_device):
+    """One workspace serves calls of different batch sizes in turn: the work counter
+    in its header is re-armed after every call and the partial rows of each call are
+    written before they are read. Three rounds over three batch sizes."""
+    rng = np.random.default_rng(55)
+    dtype = synth.BF16
+    cases = [random_case(rng, rng.integers(1, 700, n), 16, 4, 128, 16, dtype) for n in (5, 40, 17)]
+    need = max(pkv.pkv_decode_workspace_size(len(c[4]), 16, 4, 128, 16, c[5], 64) for c in cases)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    refs = [A.paged_decode_attention(c[0], c[1], c[2], c[3], c[4], 0.09, dtype) for c in cases]
+    dev = [tuple(to_dev(x, dtype) for x in c[:3]) + (torch.from_numpy(c[3]).cuda(),
+                                                      torch.from_numpy(c[4]).cuda())
+           for c in cases]
+    for rnd in range(3):
+        for i, (c, r, d) in enumerate(zip(cases, refs, dev)):
+            out = torch.empty_like(d[0])
+            pkv.pkv_paged_attention_decode(out, d[0], d[1], d[2], d[3], d[4], c[5], scale=0.09,
+                                           partition_size=64, workspace=ws)
+            torch.cuda.synchronize()
+            assert_close(to_bits(out), r, dtype, f"round {rnd} case {i}")
+    assert pkv.pkv_get_device_status() == 0
+
+
+def test_many_partitions_merge(cuda_device):
+    """Contexts of up to 5000 tokens at 64-token partitions: up to 79 partials merged."""
+    rng = np.random.default_rng(56)
+    dtype = synth.F16
+    q, kc, vc, bt, lens, max_len = random_case(rng, [5000, 4097, 64, 65, 1], 8, 1, 128, 32, dtype)
+    check_case(q, kc, vc, bt, lens, max_len, dtype, 0.088, 64, "P=64 long")
