@@ -212,6 +212,15 @@ int pkv_alloc_destroy(pkv_alloc *a);
  * receives *n_cow_out (src, dst) pairs to copy before writing. */
 int pkv_seq_append(pkv_alloc *a, int64_t seq_id, int n_tokens, int64_t *slots_out,
                    int32_t *cow_pairs_out, int *n_cow_out);
+/* One decode step for a batch: pkv_seq_append(a, seq_ids[i], n_tokens, ...) for i = 0..n-1 in
+ * order. Sequence i's slots go to slots_out[i*n_tokens .. i*n_tokens+n_tokens); all copy-on-write
+ * pairs go to cow_pairs_out (host int32 [n*n_tokens][2]) in call order, *n_cow_out of them.
+ * Stops at the first sequence whose append fails and returns its error; *n_done_out (may be
+ * NULL) = sequences appended before it, whose results stand (the failing one changed nothing). */
+int pkv_seq_append_batch(pkv_alloc *a, const int64_t *seq_ids, int n, int n_tokens,
+                         int64_t *slots_out, int32_t *cow_pairs_out, int *n_cow_out,
+                         int *n_done_out);
+
 /* Errors: PKV_ERR_UNKNOWN_SEQ (no parent), PKV_ERR_SEQ_EXISTS (child id in use). */
 int pkv_seq_fork(pkv_alloc *a, int64_t parent, int64_t child);
 /* Errors: PKV_ERR_UNKNOWN_SEQ. */

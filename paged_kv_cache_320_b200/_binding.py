@@ -67,6 +67,8 @@ def lib() -> ctypes.CDLL:
         L.pkv_alloc_create.argtypes = [ctypes.POINTER(P), I, I, I, P]
         L.pkv_alloc_destroy.argtypes = [P]
         L.pkv_seq_append.argtypes = [P, I64, I, P, P, ctypes.POINTER(I)]
+        L.pkv_seq_append_batch.argtypes = [P, P, I, I, P, P, ctypes.POINTER(I),
+                                           ctypes.POINTER(I)]
         L.pkv_seq_fork.argtypes = [P, I64, I64]
         L.pkv_seq_free.argtypes = [P, I64]
         L.pkv_block_tables.argtypes = [P, P, I, P, P]
@@ -76,7 +78,8 @@ def lib() -> ctypes.CDLL:
                      "pkv_decode_workspace_size",
                      "pkv_decode_partition_size", "pkv_reshape_and_cache", "pkv_copy_blocks",
                      "pkv_get_device_status", "pkv_alloc_create", "pkv_alloc_destroy",
-                     "pkv_seq_append", "pkv_seq_fork", "pkv_seq_free", "pkv_block_tables",
+                     "pkv_seq_append", "pkv_seq_append_batch", "pkv_seq_fork", "pkv_seq_free",
+                     "pkv_block_tables",
                      "pkv_stats"):
             getattr(L, name).restype = I
         _lib = L
@@ -247,6 +250,19 @@ class BlockManager:
         if rc != PKV_OK:
             return rc, slots[:0], cows[:0]
         return rc, slots[:n_tokens], cows[:n_cow.value]
+
+    def pkv_seq_append_batch(self, seq_ids, n_tokens):
+        """Returns (status, n_done, slots int64 [n, n_tokens], cow pairs int32 [k, 2])."""
+        import numpy as np
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        n = ids.shape[0]
+        slots = np.zeros((max(n, 1), max(n_tokens, 1)), dtype=np.int64)
+        cows = np.zeros((max(n * n_tokens, 1), 2), dtype=np.int32)
+        n_cow, n_done = ctypes.c_int(0), ctypes.c_int(0)
+        rc = lib().pkv_seq_append_batch(self._h, ids.ctypes.data, n, int(n_tokens),
+                                        slots.ctypes.data, cows.ctypes.data,
+                                        ctypes.byref(n_cow), ctypes.byref(n_done))
+        return rc, n_done.value, slots[:n, :n_tokens], cows[:n_cow.value]
 
     def pkv_seq_fork(self, parent, child):
         return lib().pkv_seq_fork(self._h, int(parent), int(child))

@@ -129,6 +129,32 @@ int pkv_seq_append(pkv_alloc *a, int64_t seq_id, int n_tokens, int64_t *slots_ou
     return PKV_OK;
 }
 
+int pkv_seq_append_batch(pkv_alloc *a, const int64_t *seq_ids, int n, int n_tokens,
+                         int64_t *slots_out, int32_t *cow_pairs_out, int *n_cow_out,
+                         int *n_done_out) {
+    if (n_done_out) *n_done_out = 0;
+    if (n_cow_out) *n_cow_out = 0;
+    if (!a || n < 0 || n_tokens < 0 || (n > 0 && !seq_ids)) return PKV_ERR_INVALID_ARG;
+    if (n > 0 && n_tokens > 0 && (!slots_out || !cow_pairs_out)) return PKV_ERR_INVALID_ARG;
+    int total_cow = 0;
+    for (int i = 0; i < n; ++i) {
+        int k = 0;
+        const int rc = pkv_seq_append(a, seq_ids[i], n_tokens,
+                                      slots_out ? slots_out + (size_t)i * n_tokens : nullptr,
+                                      cow_pairs_out ? cow_pairs_out + 2 * (size_t)total_cow
+                                                    : nullptr,
+                                      &k);
+        if (rc != PKV_OK) {
+            if (n_cow_out) *n_cow_out = total_cow;
+            return rc;
+        }
+        total_cow += k;
+        if (n_done_out) *n_done_out = i + 1;
+    }
+    if (n_cow_out) *n_cow_out = total_cow;
+    return PKV_OK;
+}
+
 int pkv_seq_fork(pkv_alloc *a, int64_t parent, int64_t child) {
     if (!a) return PKV_ERR_INVALID_ARG;
     auto it = a->seqs.find(parent);

@@ -8,6 +8,8 @@
 
 #include <stdint.h>
 
+#include "pkv_ptx.cuh"
+
 namespace pkv {
 
 // One thread per 16-byte vector of one (token, KV head) row; K and V together.
@@ -18,6 +20,7 @@ reshape_and_cache_kernel(const uint4 *__restrict__ k_new, const uint4 *__restric
                          uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache,
                          const int64_t *__restrict__ slot_mapping, int num_tokens, int Hkv,
                          int BS, int num_blocks, unsigned *status) {
+    pdl_wait_and_release();
     constexpr int VPR = D * 2 / 16;   // vectors per row
     const int64_t total = (int64_t)num_tokens * Hkv * VPR;
     const int64_t limit = (int64_t)num_blocks * BS;
@@ -46,6 +49,7 @@ __global__ void __launch_bounds__(256)
 copy_blocks_kernel(void *const *__restrict__ k_caches, void *const *__restrict__ v_caches,
                    const int32_t *__restrict__ block_pairs, int num_blocks, int block_vecs,
                    unsigned *status) {
+    pdl_wait_and_release();
     const int pair = blockIdx.x;
     const int layer = blockIdx.y;
     const int src = block_pairs[2 * pair];

@@ -239,6 +239,7 @@ paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
         }
         fence_mbar_init();
     }
+    pdl_wait_and_release();
     __syncthreads();
 
     if (warp == kConsumerWarps) {
@@ -609,78 +610,84 @@ paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
 
 // Merge of a sequence's partitions for one query head (log-sum-exp):
 //   M = max_p m_p;  w_p = l_p 2^(m_p - M);  out = sum_p w_p o_p / sum_p w_p
-// (m_p in log2 units, o_p normalised). One CTA per (query head, sequence), D threads.
+// (m_p in log2 units, o_p normalised). CTAs of D threads loop over the (query head,
+// sequence) pairs; pairs of single-partition sequences are skipped.
 template <typename T, int D>
 __global__ void __launch_bounds__(D)
 paged_decode_reduce_kernel(DecodeParams prm) {
-    const int h = blockIdx.x;
-    const int s = blockIdx.y;
-    if (h == 0 && s == 0 && threadIdx.x == 0 && prm.sched) {
+    pdl_wait_and_release();
+    if (blockIdx.x == 0 && threadIdx.x == 0 && prm.sched) {
         // every decode CTA has finished (stream order): re-arm the scheduler
         prm.sched->next = 0;
         __threadfence();
         prm.sched->armed = kSchedArmed;
     }
-    int len = prm.context_lens[s];
-    len = len < 0 ? 0 : (len > prm.max_context_len ? prm.max_context_len : len);
-    const int P = prm.partition;
-    const int np = max(1, (len + P - 1) / P);
-    if (np == 1) return;
-    const int G = prm.group;
-    const int hk = h / G, g = h - hk * G;
-    const int base = prm.ws_seq_base[s] + hk * np;
     extern __shared__ float wsm[];   // [np] weights
     __shared__ float red[D / 32];
     __shared__ float bcast;
     const float2 *mlp = reinterpret_cast<const float2 *>(prm.ws_ml);
     const int tid = threadIdx.x;
+    const int G = prm.group;
+    const int P = prm.partition;
+    const int pairs = prm.num_seqs * prm.num_heads;
+    for (int pr = blockIdx.x; pr < pairs; pr += gridDim.x) {
+        const int s = pr / prm.num_heads;
+        const int h = pr - s * prm.num_heads;
+        int len = prm.context_lens[s];
+        len = len < 0 ? 0 : (len > prm.max_context_len ? prm.max_context_len : len);
+        const int np = max(1, (len + P - 1) / P);
+        if (np == 1) continue;
+        const int hk = h / G, g = h - hk * G;
+        const int base = prm.ws_seq_base[s] + hk * np;
 
-    float M = -INFINITY;
-    for (int p = tid; p < np; p += D) M = fmaxf(M, mlp[(size_t)(base + p) * G + g].x);
+        float M = -INFINITY;
+        for (int p = tid; p < np; p += D) M = fmaxf(M, mlp[(size_t)(base + p) * G + g].x);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    if ((tid & 31) == 0) red[tid >> 5] = M;
-    __syncthreads();
-    if (tid == 0) {
-        float v = red[0];
-        for (int i = 1; i < D / 32; ++i) v = fmaxf(v, red[i]);
-        bcast = v;
-    }
-    __syncthreads();
-    M = bcast;
-    float Ls = 0.f;
-    for (int p = tid; p < np; p += D) {
-        const float2 v = mlp[(size_t)(base + p) * G + g];
-        const float wv = (M == -INFINITY) ? 0.f : v.y * ex2(v.x - M);
-        wsm[p] = wv;
-        Ls += wv;
-    }
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        if ((tid & 31) == 0) red[tid >> 5] = M;
+        __syncthreads();
+        if (tid == 0) {
+            float v = red[0];
+            for (int i = 1; i < D / 32; ++i) v = fmaxf(v, red[i]);
+            bcast = v;
+        }
+        __syncthreads();
+        M = bcast;
+        float Ls = 0.f;
+        for (int p = tid; p < np; p += D) {
+            const float2 v = mlp[(size_t)(base + p) * G + g];
+            const float wv = (M == -INFINITY) ? 0.f : v.y * ex2(v.x - M);
+            wsm[p] = wv;
+            Ls += wv;
+        }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
-    __syncthreads();
-    if ((tid & 31) == 0) red[tid >> 5] = Ls;
-    __syncthreads();
-    if (tid == 0) {
-        float v = 0.f;
-        for (int i = 0; i < D / 32; ++i) v += red[i];
-        bcast = v;
+        for (int o = 16; o > 0; o >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
+        __syncthreads();
+        if ((tid & 31) == 0) red[tid >> 5] = Ls;
+        __syncthreads();
+        if (tid == 0) {
+            float v = 0.f;
+            for (int i = 0; i < D / 32; ++i) v += red[i];
+            bcast = v;
+        }
+        __syncthreads();
+        Ls = bcast;
+        const float *op = prm.ws_o + ((size_t)base * G + g) * D + tid;
+        const size_t stride = (size_t)G * D;
+        float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+        int p = 0;
+        for (; p + 4 <= np; p += 4) {
+            acc0 += wsm[p] * op[(size_t)p * stride];
+            acc1 += wsm[p + 1] * op[(size_t)(p + 1) * stride];
+            acc2 += wsm[p + 2] * op[(size_t)(p + 2) * stride];
+            acc3 += wsm[p + 3] * op[(size_t)(p + 3) * stride];
+        }
+        for (; p < np; ++p) acc0 += wsm[p] * op[(size_t)p * stride];
+        const float acc = (acc0 + acc1) + (acc2 + acc3);
+        T *out = reinterpret_cast<T *>(prm.out) + ((size_t)s * prm.num_heads + h) * D;
+        out[tid] = from_float<T>(Ls > 0.f ? acc / Ls : 0.f);
+        __syncthreads();   // wsm / red / bcast are reused by the next pair
     }
-    __syncthreads();
-    Ls = bcast;
-    const float *op = prm.ws_o + ((size_t)base * G + g) * D + tid;
-    const size_t stride = (size_t)G * D;
-    float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
-    int p = 0;
-    for (; p + 4 <= np; p += 4) {
-        acc0 += wsm[p] * op[(size_t)p * stride];
-        acc1 += wsm[p + 1] * op[(size_t)(p + 1) * stride];
-        acc2 += wsm[p + 2] * op[(size_t)(p + 2) * stride];
-        acc3 += wsm[p + 3] * op[(size_t)(p + 3) * stride];
-    }
-    for (; p < np; ++p) acc0 += wsm[p] * op[(size_t)p * stride];
-    const float acc = (acc0 + acc1) + (acc2 + acc3);
-    T *out = reinterpret_cast<T *>(prm.out) + ((size_t)s * prm.num_heads + h) * D;
-    out[tid] = from_float<T>(Ls > 0.f ? acc / Ls : 0.f);
 }
 
 }  // namespace pkv

@@ -9,6 +9,7 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "cache_kernels.cuh"
 #include "decode_kernels.cuh"
@@ -130,6 +131,31 @@ int encode_rows_map(CUtensorMap *map, const void *base, int dtype, int D, long l
     return r == CUDA_SUCCESS ? PKV_OK : PKV_ERR_CUDA;
 }
 
+// Launch with programmatic stream serialization: the kernel may begin while the
+// previous kernel of the stream finishes; every kernel of this library waits
+// (griddepcontrol.wait) before touching global memory, so stream order is kept.
+// Built with PKV_USE_PDL=0 the launches are ordinary.
+#ifndef PKV_USE_PDL
+#define PKV_USE_PDL 1
+#endif
+template <typename... KArgs, typename... Args>
+int launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+           Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = PKV_USE_PDL;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -214,17 +240,17 @@ int launch_decode(const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMa
     long long grid = (long long)nsm * o;
     if (grid > items_upper) grid = items_upper;
     if (grid < 1) grid = 1;
-    kern<<<(unsigned)grid, pkv::kDecodeThreads, smem, st>>>(mk, mv, mq, prm);
-    if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
-    return PKV_OK;
+    return launch(kern, dim3((unsigned)grid), dim3(pkv::kDecodeThreads), smem, st, mk, mv, mq, prm);
 }
 
 template <typename T, int D>
 int launch_reduce(const pkv::DecodeParams &prm, int pmax, cudaStream_t st) {
-    dim3 grid(prm.num_heads, prm.num_seqs);
-    pkv::paged_decode_reduce_kernel<T, D><<<grid, D, (size_t)pmax * sizeof(float), st>>>(prm);
-    if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
-    return PKV_OK;
+    int nsm;
+    if (sm_count(&nsm) != PKV_OK) return PKV_ERR_CUDA;
+    long long grid = (long long)prm.num_seqs * prm.num_heads;
+    if (grid > 8LL * nsm) grid = 8LL * nsm;
+    return launch(pkv::paged_decode_reduce_kernel<T, D>, dim3((unsigned)grid), dim3(D),
+                  (size_t)pmax * sizeof(float), st, prm);
 }
 
 template <typename T, int D>
@@ -409,12 +435,12 @@ int pkv_reshape_and_cache(const void *k_new, const void *v_new, void *k_cache, v
     auto *kc = static_cast<uint4 *>(k_cache);
     auto *vc = static_cast<uint4 *>(v_cache);
     if (head_dim == 128)
-        pkv::reshape_and_cache_kernel<128><<<(unsigned)blocks, 256, 0, st>>>(
-            kn, vn, kc, vc, slot_mapping, num_tokens, num_kv_heads, block_size, num_blocks, status);
-    else
-        pkv::reshape_and_cache_kernel<64><<<(unsigned)blocks, 256, 0, st>>>(
-            kn, vn, kc, vc, slot_mapping, num_tokens, num_kv_heads, block_size, num_blocks, status);
-    return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+        return launch(pkv::reshape_and_cache_kernel<128>, dim3((unsigned)blocks), dim3(256), 0, st,
+                      kn, vn, kc, vc, slot_mapping, num_tokens, num_kv_heads, block_size,
+                      num_blocks, status);
+    return launch(pkv::reshape_and_cache_kernel<64>, dim3((unsigned)blocks), dim3(256), 0, st, kn,
+                  vn, kc, vc, slot_mapping, num_tokens, num_kv_heads, block_size, num_blocks,
+                  status);
 }
 
 int pkv_copy_blocks(void *const *k_caches, void *const *v_caches, int num_layers,
@@ -434,9 +460,9 @@ int pkv_copy_blocks(void *const *k_caches, void *const *v_caches, int num_layers
     int rc;
     if ((rc = device_status_ptr(&status)) != PKV_OK) return rc;
     dim3 grid((unsigned)num_pairs, (unsigned)num_layers, 2);
-    pkv::copy_blocks_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        k_caches, v_caches, block_pairs, num_blocks, (int)vecs, status);
-    return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+    return launch(pkv::copy_blocks_kernel, grid, dim3(256), 0,
+                  reinterpret_cast<cudaStream_t>(stream), k_caches, v_caches, block_pairs,
+                  num_blocks, (int)vecs, status);
 }
 
 int pkv_get_device_status(uint32_t *status_out, int clear, pkv_stream_t stream) {

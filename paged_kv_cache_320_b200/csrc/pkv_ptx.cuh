@@ -60,6 +60,16 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     return false;
 }
 
+// ---- programmatic dependent launch ----------------------------------------
+// Kernels of this library are launched so that they may start while the previous
+// kernel of the stream finishes. Each one waits here before its first global-memory
+// access (the previous grid has then completed and its writes are visible) and lets
+// the next kernel start launching right away.
+__device__ __forceinline__ void pdl_wait_and_release() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---- TMA -----------------------------------------------------------------
 // 2-D tiled load global -> shared, completion counted on mbarrier `bar`.
 // Coordinates: x = innermost (elements), y = row. Out-of-range boxes read zeros.

@@ -94,3 +94,38 @@ def test_workload_placement_reproduced_by_in_order_appends():
     np.testing.assert_array_equal(tables, wl.block_tables)
     np.testing.assert_array_equal(lens, wl.context_lens)
     np.testing.assert_array_equal(last, wl.slot_mapping)
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_batched_append_equals_appends_in_order(seed):
+    """pkv_seq_append_batch == pkv_seq_append per sequence, in order, against the model;
+    on failure the sequences before the failing one keep their appends."""
+    rng = np.random.default_rng(500 + seed)
+    nb, bs, mb = int(rng.integers(6, 30)), int(rng.choice([2, 4, 8])), int(rng.integers(2, 6))
+    order = rng.permutation(nb)
+    c = BlockManager(nb, bs, mb, order)
+    m = BM.BlockManagerModel(nb, bs, mb, order)
+    for s in range(4):
+        n0 = int(rng.integers(1, bs * 2))
+        assert c.pkv_seq_append(s, n0)[0] == m.append(s, n0)[0]
+    if rng.random() < 0.5:
+        assert c.pkv_seq_fork(0, 7) == m.fork(0, 7)
+    for _ in range(6):
+        ids = [int(x) for x in rng.choice([0, 1, 2, 3, 7, 9], size=int(rng.integers(1, 6)))]
+        k = int(rng.integers(0, 3))
+        st, done, slots, cows = c.pkv_seq_append_batch(ids, k)
+        exp_slots, exp_cows, exp_done, exp_st = [], [], 0, 0
+        for sid in ids:
+            s2, sl, cw = m.append(sid, k)
+            if s2 != 0:
+                exp_st = s2
+                break
+            exp_slots.append(sl)
+            exp_cows += [list(x) for x in cw]
+            exp_done += 1
+        assert st == exp_st and done == exp_done
+        for i in range(done):
+            assert slots[i].tolist() == exp_slots[i]
+        assert cows.tolist() == exp_cows
+        compare_states(c, m, sorted(m.tables))
+    c.close()
