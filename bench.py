@@ -43,6 +43,10 @@ WORKLOADS = {
     "shared_prefix": "shared-prefix parallel sampling: 16 prompts x 8 samples, prefix 1024 "
                      "(refcount 8), suffix U[0,256], 32q/8kv, d 128, bf16, bs 16, 1 layer",
     "long_context": "long-context decode: B 8, U[32768,131072], 64q/8kv, d 128, bf16, 1 layer",
+    "shared_prefix_cow": "shared-prefix copy-on-write step: 16 parent prompts of 1024 + u tokens "
+                         "(u in [1,255], not a multiple of 16) each forked into 8 samples that "
+                         "append one token (128 block copies), then cache write and decode; "
+                         "32q/8kv, d 128, bf16, bs 16, 1 layer",
 }
 METRIC = "paged decode attention KV-read GB/s (% of B200 HBM peak); decode tokens/s"
 KERNEL_SOURCES = ["paged_kv_cache_320_b200/csrc/decode_kernels.cuh",
@@ -159,6 +163,168 @@ def algorithmic_bytes(wl):
     return kv, kv + qo + tables
 
 
+def cow_arm(args, rank, world, local_rank):
+    """The copy-on-write decode step. Each step the block manager forks every parent
+    prompt into its samples and appends one token to each sample: the shared, partly
+    filled last block is copied for every sample (128 pairs), then copy_blocks ->
+    reshape_and_cache -> paged decode. The device-timed step repeats one such step
+    (idempotent); the end-to-end step frees the samples, forks and appends again through
+    the host block manager every step."""
+    import torch
+    import paged_kv_cache_320_b200 as pkv
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream(dev)
+    cs = synth.make_cow_step(num_layers=1)
+    sp = cs.spec
+    prompts, samples = len(cs.parent_lens), sp.samples
+    B = prompts * samples
+    mgr = pkv.BlockManager(cs.num_blocks, sp.block_size, cs.max_blocks_per_seq, cs.initial_order)
+    parents = [10_000 + p for p in range(prompts)]
+    kids = np.array([p * samples + k for p in range(prompts) for k in range(samples)], np.int64)
+    for p, n in zip(parents, cs.parent_lens):
+        if mgr.pkv_seq_append(p, int(n))[0] != 0:
+            raise RuntimeError("pool too small for the parents")
+
+    def host_step():
+        for p in range(prompts):
+            for k in range(samples):
+                mgr.pkv_seq_free(p * samples + k)       # (no-op error the first time)
+        for p in range(prompts):
+            for k in range(samples):
+                if mgr.pkv_seq_fork(parents[p], p * samples + k) != 0:
+                    raise RuntimeError("fork failed")
+        st, done, slots, cows = mgr.pkv_seq_append_batch(kids, 1)
+        if st != 0:
+            raise RuntimeError(f"append failed ({st})")
+        st, tables, lens = mgr.pkv_block_tables(kids)
+        return slots[:, 0].copy(), cows.copy(), tables, lens
+
+    dt = synth.torch_dtype(sp.dtype)
+
+    def to_dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(dt)
+
+    kc, vc = to_dev(cs.k_cache[0]), to_dev(cs.v_cache[0])
+    q, kn, vn = to_dev(cs.q), to_dev(cs.k_new), to_dev(cs.v_new)
+    out = torch.empty_like(q)
+    kp = torch.tensor([kc.data_ptr()], dtype=torch.int64, device=dev)
+    vp = torch.tensor([vc.data_ptr()], dtype=torch.int64, device=dev)
+    slots, cows, tables, lens = host_step()
+    n_pairs = cows.shape[0]
+    max_len = cs.max_blocks_per_seq * sp.block_size
+    P = pkv.pkv_decode_partition_size(B, sp.num_heads, sp.num_kv_heads, sp.head_dim,
+                                      sp.block_size, max_len, args.partition)
+    ws = torch.zeros(max(16, pkv.pkv_decode_workspace_size(
+        B, sp.num_heads, sp.num_kv_heads, sp.head_dim, sp.block_size, max_len, P)),
+        dtype=torch.uint8, device=dev)
+    slots_d = torch.from_numpy(slots).to(dev)
+    pairs_d = torch.from_numpy(cows).to(dev)
+    bt_d = torch.from_numpy(tables).to(dev)
+    lens_d = torch.from_numpy(lens).to(dev)
+    dtype_code = pkv.PKV_BF16 if sp.dtype == synth.BF16 else pkv.PKV_F16
+    kv_step = int(lens.astype(np.int64).sum()) * sp.num_kv_heads * sp.head_dim * 4
+    ev = {"copy": [], "decode": []}
+
+    def step(record=False):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)] if record else None
+        if record:
+            e[0].record(stream)
+        pkv.pkv_copy_blocks(kp, vp, pairs_d, sp.num_kv_heads, sp.head_dim, sp.block_size,
+                            cs.num_blocks, dtype_code, stream=stream)
+        pkv.pkv_reshape_and_cache(kn, vn, kc, vc, slots_d, stream=stream)
+        if record:
+            e[1].record(stream)
+        pkv.pkv_paged_attention_decode(out, q, kc, vc, bt_d, lens_d, max_len, scale=1 / math.sqrt(
+            sp.head_dim), partition_size=P, workspace=ws, stream=stream)
+        if record:
+            e[2].record(stream)
+            ev["copy"].append((e[0], e[1]))
+            ev["decode"].append((e[1], e[2]))
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local_rank) as clocks:
+        torch.cuda.synchronize(dev)
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(args.steps):
+            step(record=True)
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+    ms_step = t0.elapsed_time(t1) / args.steps
+    if pkv.pkv_get_device_status(stream=stream) != 0:
+        raise RuntimeError("device status word set during the benchmark")
+    copy_us = 1e3 * statistics.mean(a.elapsed_time(b) for a, b in ev["copy"])
+    dec_us = 1e3 * statistics.mean(a.elapsed_time(b) for a, b in ev["decode"])
+    value, tokens_per_s = weak_scaling_rates(kv_step, B, 1, ms_step)
+    copy_bytes = n_pairs * 2 * sp.num_kv_heads * sp.block_size * sp.head_dim * 2 * 2
+
+    # end to end: the host block manager re-forks and appends every step
+    pin = dict(pin_memory=True)
+    q_h = torch.empty(tuple(q.shape), dtype=dt, **pin); q_h.copy_(q.cpu())
+    kn_h = torch.empty(tuple(kn.shape), dtype=dt, **pin); kn_h.copy_(kn.cpu())
+    vn_h = torch.empty(tuple(vn.shape), dtype=dt, **pin); vn_h.copy_(vn.cpu())
+    out_h = torch.empty(tuple(q.shape), dtype=dt, **pin)
+    sl_h = torch.empty(B, dtype=torch.int64, **pin)
+    pr_h = torch.empty((n_pairs, 2), dtype=torch.int32, **pin)
+    bt_h = torch.empty(tuple(tables.shape), dtype=torch.int32, **pin)
+    ln_h = torch.empty(B, dtype=torch.int32, **pin)
+
+    def e2e_step():
+        sl, cw, tb, ln = host_step()
+        if cw.shape[0] != n_pairs:
+            raise RuntimeError("copy-on-write pair count changed")
+        sl_h.numpy()[:] = sl
+        pr_h.numpy()[:] = cw
+        bt_h.numpy()[:] = tb
+        ln_h.numpy()[:] = ln
+        for d_, h_ in ((q, q_h), (kn, kn_h), (vn, vn_h), (slots_d, sl_h), (pairs_d, pr_h),
+                       (bt_d, bt_h), (lens_d, ln_h)):
+            d_.copy_(h_, non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+        stream.synchronize()
+
+    for _ in range(args.warmup):
+        e2e_step()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = a.elapsed_time(b) / args.steps
+    mgr.close()
+    peak, peak_kind = read_peaks()
+    h2d = (q_h.numel() + kn_h.numel() + vn_h.numel()) * 2 + B * 8 + n_pairs * 8 + bt_h.numel() * 4 + B * 4
+    return {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": synth.DTYPE_NAMES[sp.dtype], "data": "synthetic",
+        "config": {"workload": "shared_prefix_cow", "description": WORKLOADS["shared_prefix_cow"],
+                   "num_seqs": B, "copy_pairs_per_step": n_pairs, "partition_size": P,
+                   "sum_context_tokens": int(lens.sum()), "kv_bytes_per_step": kv_step},
+        "tokens_per_s": round(tokens_per_s, 1),
+        "pct_of_hbm_peak": round(100 * value / peak, 2),
+        "copy_and_write_us": round(copy_us, 2),
+        "copy_blocks_bytes": copy_bytes,
+        "decode_us": round(dec_us, 2),
+        "clocks": clocks.summary(),
+        "e2e": {"value": round(kv_step / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(out_h.numel() * 2),
+                "includes": "host frees, forks and batched appends (copy-on-write pairs), table "
+                            "export, pinned H2D, copy_blocks + cache write + decode, D2H"},
+        "gpu_launches": args.steps * 3,
+    }
+
+
 def reduce_max(x, dist, device):
     """Maximum of a per-rank scalar over all ranks (the identity on one process)."""
     if dist is None:
@@ -215,6 +381,29 @@ def gpu_arm(args, rank, world, local_rank):
     stream = torch.cuda.current_stream(dev)
     kv_layer, roof_layer = algorithmic_bytes(wl)
     kv_step = kv_layer * L
+    shared = args.decode == "shared"
+    if shared:
+        if not sp.prompts:
+            raise SystemExit("--decode shared needs a workload with shared prefixes")
+        starts = torch.arange(0, B + 1, sp.samples, dtype=torch.int32, device=dev)
+        prefix = torch.full((sp.prompts,), sp.prefix, dtype=torch.int32, device=dev)
+        ws = torch.empty(max(16, pkv.pkv_decode_shared_prefix_workspace_size(
+            B, sp.num_heads, sp.num_kv_heads, sp.head_dim, sp.block_size, max_len, P)),
+            dtype=torch.uint8, device=dev)
+        # unique K/V: each prompt's prefix once per KV head, every private suffix
+        uniq = (sp.prompts * sp.prefix + int((wl.context_lens - sp.prefix).sum())) * \
+            sp.num_kv_heads * sp.head_dim * 4
+        roof_layer = roof_layer - kv_layer + uniq
+
+    def decode(l, out_t, q_t, bt_t, lens_t):
+        if shared:
+            pkv.pkv_paged_attention_decode_shared_prefix(
+                out_t, q_t, wl.k_cache[l], wl.v_cache[l], bt_t, lens_t, starts, prefix, max_len,
+                scale=wl.scale, partition_size=P, workspace=ws, stream=stream)
+        else:
+            pkv.pkv_paged_attention_decode(out_t, q_t, wl.k_cache[l], wl.v_cache[l], bt_t,
+                                           lens_t, max_len, scale=wl.scale, partition_size=P,
+                                           workspace=ws, stream=stream)
 
     k1_events = []
 
@@ -226,14 +415,12 @@ def gpu_arm(args, rank, world, local_rank):
                 e0 = torch.cuda.Event(enable_timing=True)
                 e1 = torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
-            pkv.pkv_paged_attention_decode(outs[l], wl.q[l], wl.k_cache[l], wl.v_cache[l], bt,
-                                           lens, max_len, scale=wl.scale, partition_size=P,
-                                           workspace=ws, stream=stream)
+            decode(l, outs[l], wl.q[l], bt, lens)
             if record:
                 e1.record(stream)
                 k1_events.append((e0, e1))
 
-    launches_per_step = L * (2 + (1 if pmax > 1 else 0))
+    launches_per_step = L * (4 if shared else 2 + (1 if pmax > 1 else 0))
     dist = None
     if world > 1:
         import torch.distributed as dist
@@ -272,10 +459,10 @@ def gpu_arm(args, rank, world, local_rank):
     peak, peak_kind = read_peaks()
     achieved = roof_layer / (k1_avg_ms * 1e-3) / 1e9
     read_probe = hbm_read_probe(dev, stream)
-    traffic = read_traffic(args.workload, sp.block_size)
+    traffic = None if shared else read_traffic(args.workload, sp.block_size)
 
     # ---- end to end: host block manager + pinned host buffers through the public API
-    e2e = e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, world)
+    e2e = e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, world, decode)
 
     result = {
         "metric": METRIC,
@@ -297,6 +484,7 @@ def gpu_arm(args, rank, world, local_rank):
             "head_dim": sp.head_dim, "block_size": sp.block_size, "layers": L,
             "sum_context_tokens": int(wl.context_lens.sum()),
             "partition_size": P,
+            "decode": args.decode,
             "kv_bytes_per_step": kv_step,
             "l2": f"inputs larger than L2: {kv_layer / 1e6:.0f} MB of K/V per layer vs 126 MB L2",
             "parallelism": f"replicas x{world}",
@@ -307,7 +495,8 @@ def gpu_arm(args, rank, world, local_rank):
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
         "roofline": {
-            "kernel": "paged_decode_partition_kernel",
+            "kernel": "paged_decode_shared_kernel (+ plan, reduce)" if shared
+            else "paged_decode_partition_kernel",
             "bound": "hbm",
             "achieved": round(achieved, 1),
             "peak": peak,
@@ -375,7 +564,7 @@ def hbm_read_probe(dev, stream):
     return (1 << 32) / (best * 1e-3) / 1e9
 
 
-def e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, world):
+def e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, world, decode):
     """Each step: the host block manager appends one token to every sequence (one batched
     call) and exports the tables; the step's inputs (slots, tables, lengths, and q, k_new,
     v_new of every layer) go host->device from pinned memory on a copy stream, layer by
@@ -436,9 +625,7 @@ def e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, worl
             stream.wait_event(ev_in[l])
             pkv.pkv_reshape_and_cache(kn_d[l], vn_d[l], wl.k_cache[l], wl.v_cache[l], slots_d,
                                       stream=stream)
-            pkv.pkv_paged_attention_decode(out_d[l], q_d[l], wl.k_cache[l], wl.v_cache[l], bt_d,
-                                           lens_d, max_len, scale=wl.scale, partition_size=P,
-                                           workspace=ws, stream=stream)
+            decode(l, out_d[l], q_d[l], bt_d, lens_d)
             ev_out[l].record(stream)
         with torch.cuda.stream(copy_out):
             for l in range(L):
@@ -475,6 +662,8 @@ def e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, worl
 def oracle_sample(workload, block_size, nseq, seed=0):
     """Host copies of a sample of the workload for the C oracle: the lengths and
     layout of the first ``nseq`` sequences of layer 0, values drawn with numpy."""
+    if workload == "shared_prefix_cow":
+        workload = "shared_prefix"          # same shapes and lengths
     overrides = {"block_size": block_size} if block_size else {}
     wl = synth.make_workload(workload, values_on="none", **overrides)
     sp = wl.spec
@@ -515,7 +704,7 @@ def oracle_step(smp):
 
 def pick_nseq(workload, block_size):
     return {"llama7b_mha": 16, "llama3_8b_gqa": 32, "shared_prefix": 16,
-            "long_context": 1}[workload]
+            "shared_prefix_cow": 16, "long_context": 1}[workload]
 
 
 def cpu_baseline(args):
@@ -580,6 +769,8 @@ def main():
     ap.add_argument("--block-size", type=int, default=0)
     ap.add_argument("--layers", type=int, default=0, help="override the workload's layer count")
     ap.add_argument("--partition", type=int, default=0, help="decode partition size (0 = auto)")
+    ap.add_argument("--decode", default="plain", choices=["plain", "shared"],
+                    help="shared: the shared-prefix-aware decode (shared-prefix workload)")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the sequence count of a length-distribution workload")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -606,13 +797,14 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
-    res = gpu_arm(args, rank, world, local_rank)
+    res = (cow_arm if args.workload == "shared_prefix_cow" else gpu_arm)(args, rank, world,
+                                                                          local_rank)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and args.workload != "shared_prefix_cow":
             res["cpu_baseline"] = cpu_baseline(args)
         print(json.dumps(res), flush=True)
 

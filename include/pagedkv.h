@@ -139,6 +139,38 @@ int pkv_paged_attention_decode_noalloc(void *out, const void *q, const void *k_c
                                        int max_context_len, float scale, int dtype,
                                        int partition_size, pkv_stream_t stream);
 
+/* ------------------------------------------------------------------------------
+ * Shared-prefix-aware decode: the same result as pkv_paged_attention_decode, for
+ * batches where groups of sequences share their first pages (parallel sampling, common
+ * prompts: "vLLM" entity page, 是什么; "分页 KV Cache 分析" §3.2). Each shared prefix page
+ * of a KV head is read once for up to 16 query rows (the G heads of several member
+ * sequences) instead of once per sequence; private suffixes are read per sequence; the
+ * pieces are merged exactly (log-sum-exp).
+ *
+ * group_start  device int32 [num_groups + 1]: sequences group_start[g] ..
+ *              group_start[g+1]-1 form group g (0 = group_start[0] < ... <
+ *              group_start[num_groups] = num_seqs). Unshared sequences are groups of one.
+ * prefix_lens  device int32 [num_groups]: tokens the group's members share. Taken as a
+ *              hint: it is cut to a multiple of block_size, to the shortest member, and at
+ *              the first logical block where a member's table differs from the group's
+ *              first member — a wrong value costs sharing, never correctness.
+ * A malformed group_start is treated as one group per sequence and sets
+ * PKV_STATUS_BAD_LEN. Workspace: pkv_decode_shared_prefix_workspace_size bytes, no
+ * initial contents required. Other arguments, limits and errors as
+ * pkv_paged_attention_decode (num_groups >= 1, <= num_seqs). Three kernel launches.
+ * ---------------------------------------------------------------------------- */
+int pkv_paged_attention_decode_shared_prefix(
+    void *out, const void *q, const void *k_cache, const void *v_cache,
+    const int32_t *block_tables, const int32_t *context_lens, const int32_t *group_start,
+    const int32_t *prefix_lens, int num_groups, int num_seqs, int num_heads, int num_kv_heads,
+    int head_dim, int block_size, int max_blocks_per_seq, int num_blocks, int max_context_len,
+    float scale, int dtype, int partition_size, void *workspace, size_t workspace_bytes,
+    pkv_stream_t stream);
+
+int pkv_decode_shared_prefix_workspace_size(int num_seqs, int num_heads, int num_kv_heads,
+                                            int head_dim, int block_size, int max_context_len,
+                                            int partition_size, size_t *bytes_out);
+
 /* Workspace bytes pkv_paged_attention_decode needs for these sizes (0 when the
  * given partition size makes every context a single partition). Same argument
  * meaning as the decode call. */

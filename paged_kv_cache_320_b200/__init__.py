@@ -15,6 +15,8 @@ from ._binding import (  # noqa: F401
     pkv_get_device_status,
     pkv_paged_attention_decode,
     pkv_paged_attention_decode_noalloc,
+    pkv_paged_attention_decode_shared_prefix,
+    pkv_decode_shared_prefix_workspace_size,
     pkv_reshape_and_cache,
 )
 from ._binding import PKV_BF16, PKV_F16  # noqa: F401

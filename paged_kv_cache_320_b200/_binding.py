@@ -60,6 +60,10 @@ def lib() -> ctypes.CDLL:
         L.pkv_paged_attention_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I,
                                                          I, I, ctypes.c_float, I, I, P]
         L.pkv_decode_workspace_size.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(SZ)]
+        L.pkv_paged_attention_decode_shared_prefix.argtypes = [
+            P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, ctypes.c_float, I, I, P, SZ, P]
+        L.pkv_decode_shared_prefix_workspace_size.argtypes = [I, I, I, I, I, I, I,
+                                                              ctypes.POINTER(SZ)]
         L.pkv_decode_partition_size.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(I)]
         L.pkv_reshape_and_cache.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P]
         L.pkv_copy_blocks.argtypes = [P, P, I, P, I, I, I, I, I, I, P]
@@ -75,7 +79,8 @@ def lib() -> ctypes.CDLL:
         L.pkv_stats.argtypes = [P, ctypes.POINTER(I), ctypes.POINTER(I),
                                 ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_double)]
         for name in ("pkv_paged_attention_decode", "pkv_paged_attention_decode_noalloc",
-                     "pkv_decode_workspace_size",
+                     "pkv_paged_attention_decode_shared_prefix",
+                     "pkv_decode_shared_prefix_workspace_size", "pkv_decode_workspace_size",
                      "pkv_decode_partition_size", "pkv_reshape_and_cache", "pkv_copy_blocks",
                      "pkv_get_device_status", "pkv_alloc_create", "pkv_alloc_destroy",
                      "pkv_seq_append", "pkv_seq_append_batch", "pkv_seq_fork", "pkv_seq_free",
@@ -183,6 +188,41 @@ def pkv_paged_attention_decode_noalloc(out, q, k_cache, v_cache, block_tables, c
         B, Hq, Hkv, D, BS, block_tables.shape[1], NB, int(max_context_len), float(scale),
         _dtype_code(q), int(partition_size), _stream(stream)),
         "pkv_paged_attention_decode_noalloc")
+    return out
+
+
+def pkv_decode_shared_prefix_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim,
+                                            block_size, max_context_len, partition_size=0):
+    out = ctypes.c_size_t(0)
+    _check(lib().pkv_decode_shared_prefix_workspace_size(
+        num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len, partition_size,
+        ctypes.byref(out)), "pkv_decode_shared_prefix_workspace_size")
+    return out.value
+
+
+def pkv_paged_attention_decode_shared_prefix(out, q, k_cache, v_cache, block_tables,
+                                             context_lens, group_start, prefix_lens,
+                                             max_context_len, scale=None, partition_size=0,
+                                             workspace=None, stream=None):
+    """As pkv_paged_attention_decode, with group_start int32 [num_groups + 1] and
+    prefix_lens int32 [num_groups] device tensors describing shared prefixes."""
+    B, Hq, D = q.shape
+    NB, Hkv, BS, D2 = k_cache.shape
+    if D2 != D or out.shape != q.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if workspace is None:
+        import torch
+        need = pkv_decode_shared_prefix_workspace_size(B, Hq, Hkv, D, BS, max_context_len,
+                                                       partition_size)
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check(lib().pkv_paged_attention_decode_shared_prefix(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
+        _ptr(group_start), _ptr(prefix_lens), prefix_lens.numel(), B, Hq, Hkv, D, BS,
+        block_tables.shape[1], NB, int(max_context_len), float(scale), _dtype_code(q),
+        int(partition_size), _ptr(workspace), workspace.numel(), _stream(stream)),
+        "pkv_paged_attention_decode_shared_prefix")
     return out
 
 

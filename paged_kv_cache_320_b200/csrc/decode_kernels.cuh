@@ -205,6 +205,193 @@ struct ItemWalker {
     }
 };
 
+// Online-softmax state of one consumer warp for a 16-row query tile: lane (gid, tig)
+// holds rows gid and gid + 8 (max m, partial sum l, output accumulators o).
+template <int D>
+struct WarpState {
+    uint32_t qa[D / 16][4];   // A fragments of Q (rows >= the tile's row count are zero)
+    float o[D / 8][4];
+    float m0, m1, l0, l1;
+};
+
+template <int D>
+__device__ __forceinline__ void reset_state(WarpState<D> &st) {
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) st.o[n][0] = st.o[n][1] = st.o[n][2] = st.o[n][3] = 0.f;
+    st.m0 = st.m1 = -INFINITY;
+    st.l0 = st.l1 = 0.f;
+}
+
+// One warp's share of a stage: tokens 16w .. 16w+15 of the stage's K and V tiles,
+// of which the first `valid` belong to the sequence.
+//   S = Q K^T (two n-tiles of 8 tokens), scale, mask, online softmax, O += P V.
+template <typename T, int D, int BS>
+__device__ __forceinline__ void consume_stage(WarpState<D> &st, uint32_t kbase, uint32_t vbase,
+                                              int w, int lane, int valid, float scale_log2) {
+    constexpr int H = D / 64;
+    constexpr int NT = D / 8;
+    const int tig = lane & 3;
+    float sc[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+        const int t = 16 * w + 8 * nt + (lane & 7);
+        const int mi = lane >> 3;
+#pragma unroll
+        for (int hf = 0; hf < H; ++hf) {
+#pragma unroll
+            for (int c2 = 0; c2 < 2; ++c2) {
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4(kbase + swz(kv_line<H, BS>(t, hf), c2 * 4 + mi), b0, b1, b2, b3);
+                const int ks = hf * 4 + c2 * 2;
+                Mma<T>::run(sc[nt], st.qa[ks], b0, b1);
+                Mma<T>::run(sc[nt], st.qa[ks + 1], b2, b3);
+            }
+        }
+    }
+    // scale, mask, online softmax (rows gid and gid+8)
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const bool in_seq = 8 * nt + 2 * tig + e < valid;
+            sc[nt][e] = in_seq ? sc[nt][e] * scale_log2 : -INFINITY;
+            sc[nt][2 + e] = in_seq ? sc[nt][2 + e] * scale_log2 : -INFINITY;
+            mx0 = fmaxf(mx0, sc[nt][e]);
+            mx1 = fmaxf(mx1, sc[nt][2 + e]);
+        }
+    }
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+    const float mn0 = fmaxf(st.m0, mx0), mn1 = fmaxf(st.m1, mx1);
+    const float a0 = ex2(st.m0 - mn0), a1 = ex2(st.m1 - mn1);
+    st.m0 = mn0;
+    st.m1 = mn1;
+    float ps0 = 0.f, ps1 = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            sc[nt][e] = ex2(sc[nt][e] - mn0);
+            sc[nt][2 + e] = ex2(sc[nt][2 + e] - mn1);
+            ps0 += sc[nt][e];
+            ps1 += sc[nt][2 + e];
+        }
+    }
+    st.l0 = st.l0 * a0 + ps0;
+    st.l1 = st.l1 * a1 + ps1;
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+        st.o[n][0] *= a0; st.o[n][1] *= a0;
+        st.o[n][2] *= a1; st.o[n][3] *= a1;
+    }
+    uint32_t pa[4];
+    pa[0] = Mma<T>::pack(sc[0][0], sc[0][1]);
+    pa[1] = Mma<T>::pack(sc[0][2], sc[0][3]);
+    pa[2] = Mma<T>::pack(sc[1][0], sc[1][1]);
+    pa[3] = Mma<T>::pack(sc[1][2], sc[1][3]);
+    // O += P V  (V rows of tokens past the sequence are zeroed)
+    uint32_t keep_lo = 0xffffffffu, keep_hi = 0xffffffffu;
+    if (valid < 16) {
+        const int t0 = 2 * tig, t1 = 2 * tig + 8;
+        keep_lo = (t0 < valid ? 0x0000ffffu : 0u) | (t0 + 1 < valid ? 0xffff0000u : 0u);
+        keep_hi = (t1 < valid ? 0x0000ffffu : 0u) | (t1 + 1 < valid ? 0xffff0000u : 0u);
+    }
+    const int mi = lane >> 3;
+    const int tv = 16 * w + (mi & 1) * 8 + (lane & 7);
+#pragma unroll
+    for (int dp = 0; dp < D / 16; ++dp) {
+        const int hf = dp >> 2;
+        const int c = 2 * (dp & 3) + (mi >> 1);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_trans(vbase + swz(kv_line<H, BS>(tv, hf), c), b0, b1, b2, b3);
+        b0 &= keep_lo; b1 &= keep_hi; b2 &= keep_lo; b3 &= keep_hi;
+        Mma<T>::run(st.o[2 * dp], pa, b0, b1);
+        Mma<T>::run(st.o[2 * dp + 1], pa, b2, b3);
+    }
+}
+
+// End of an item: combine the four consumer warps' states. Leaves the normalised
+// output of rows < nrows in obuf (row stride obuf_stride floats) and every warp's
+// (m, l) per row in ml[warp * 16 + row]. All 128 consumer threads call it; the first
+// barrier also protects obuf and ml from the previous item's readers.
+template <int D>
+__device__ __forceinline__ void merge_warps(WarpState<D> &st, int nrows, float *obuf,
+                                            int obuf_stride, float2 *ml, int w, int lane) {
+    constexpr int NT = D / 8;
+    const int gid = lane >> 2;
+    const int tig = lane & 3;
+    float lt0 = st.l0 + __shfl_xor_sync(0xffffffffu, st.l0, 1);
+    lt0 += __shfl_xor_sync(0xffffffffu, lt0, 2);
+    float lt1 = st.l1 + __shfl_xor_sync(0xffffffffu, st.l1, 1);
+    lt1 += __shfl_xor_sync(0xffffffffu, lt1, 2);
+    named_bar_sync(1, kConsumerWarps * 32);
+    if (tig == 0) {
+        ml[w * kMaxGroup + gid] = make_float2(st.m0, lt0);
+        ml[w * kMaxGroup + gid + 8] = make_float2(st.m1, lt1);
+    }
+    named_bar_sync(1, kConsumerWarps * 32);
+    // my rows' scale factors f = 2^(m_self - M) / L  (0 when the item is empty)
+    float fr[2];
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+        const int row = min(gid + 8 * rr, nrows - 1);
+        float M = -INFINITY;
+#pragma unroll
+        for (int ww = 0; ww < kConsumerWarps; ++ww) M = fmaxf(M, ml[ww * kMaxGroup + row].x);
+        float Lsum = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int ww = 0; ww < kConsumerWarps; ++ww) {
+                const float2 v = ml[ww * kMaxGroup + row];
+                Lsum += v.y * ex2(v.x - M);
+            }
+        }
+        const float mself = rr ? st.m1 : st.m0;
+        fr[rr] = (Lsum > 0.f) ? ex2(mself - M) / Lsum : 0.f;
+    }
+    // accumulate the four warps' scaled outputs in a fixed order (deterministic)
+#pragma unroll
+    for (int ww = 0; ww < kConsumerWarps; ++ww) {
+        if (w == ww) {
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+                const int row = gid + 8 * rr;
+                if (row < nrows) {
+                    float2 *dst = reinterpret_cast<float2 *>(obuf + row * obuf_stride + 2 * tig);
+#pragma unroll
+                    for (int n = 0; n < NT; ++n) {
+                        float2 v = make_float2(st.o[n][2 * rr] * fr[rr], st.o[n][2 * rr + 1] * fr[rr]);
+                        if (ww > 0) {
+                            const float2 prev = dst[n * 4];
+                            v.x += prev.x;
+                            v.y += prev.y;
+                        }
+                        dst[n * 4] = v;
+                    }
+                }
+            }
+        }
+        named_bar_sync(1, kConsumerWarps * 32);
+    }
+}
+
+// (M, L) of one row over the four warps' (m, l) pairs.
+__device__ __forceinline__ float2 row_stats(const float2 *ml, int row) {
+    float M = -INFINITY;
+    for (int ww = 0; ww < kConsumerWarps; ++ww) M = fmaxf(M, ml[ww * kMaxGroup + row].x);
+    float Lsum = 0.f;
+    if (M != -INFINITY)
+        for (int ww = 0; ww < kConsumerWarps; ++ww) {
+            const float2 v = ml[ww * kMaxGroup + row];
+            Lsum += v.y * ex2(v.x - M);
+        }
+    return make_float2(M, Lsum);
+}
+
 template <typename T, int D, int BS>
 __global__ void __launch_bounds__(kDecodeThreads, 2)
 paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
@@ -392,12 +579,9 @@ paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
     // ---------------------------------------------------------------- consumers
     const int w = warp;
     const int gid = lane >> 2;
-    const int tig = lane & 3;
     constexpr int KS = D / 16;   // k-steps of QK
-    constexpr int NT = D / 8;    // n-tiles of PV
-    uint32_t qa[KS][4];
-    float o[NT][4];
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    WarpState<D> st;
+    reset_state(st);
 
     for (int it = 0;; ++it) {
         const int slot = it % L::kStages;
@@ -417,165 +601,25 @@ paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
             for (int ks = 0; ks < KS; ++ks) {
                 const int hf = ks >> 2;
                 const int c = 2 * (ks & 3) + (mi >> 1);
-                ldsm_x4(qbase + swz(hf * G + row, c), qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3]);
-                if (gid >= G) qa[ks][0] = qa[ks][2] = 0u;
-                if (gid + 8 >= G) qa[ks][1] = qa[ks][3] = 0u;
+                ldsm_x4(qbase + swz(hf * G + row, c), st.qa[ks][0], st.qa[ks][1], st.qa[ks][2],
+                        st.qa[ks][3]);
+                if (gid >= G) st.qa[ks][0] = st.qa[ks][2] = 0u;
+                if (gid + 8 >= G) st.qa[ks][1] = st.qa[ks][3] = 0u;
             }
-#pragma unroll
-            for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-            m0 = m1 = -INFINITY;
-            l0 = l1 = 0.f;
+            reset_state(st);
         }
 
         const int valid = in.ntok - 16 * w;   // tokens of my 16-token slice in the sequence
         if (valid > 0) {
             const uint8_t *stage = ring + slot * L::kStageBytes;
-            const uint32_t kbase = smem_u32(stage);
-            const uint32_t vbase = smem_u32(stage + L::kKBytes);
-            // ---- S = Q K^T for tokens 16w .. 16w+15 (two n-tiles of 8)
-            float sc[2][4];
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
-                const int t = 16 * w + 8 * nt + (lane & 7);
-                const int mi = lane >> 3;
-#pragma unroll
-                for (int hf = 0; hf < H; ++hf) {
-#pragma unroll
-                    for (int c2 = 0; c2 < 2; ++c2) {
-                        uint32_t b0, b1, b2, b3;
-                        ldsm_x4(kbase + swz(kv_line<H, BS>(t, hf), c2 * 4 + mi), b0, b1, b2, b3);
-                        const int ks = hf * 4 + c2 * 2;
-                        Mma<T>::run(sc[nt], qa[ks], b0, b1);
-                        Mma<T>::run(sc[nt], qa[ks + 1], b2, b3);
-                    }
-                }
-            }
-            // ---- scale, mask, online softmax (rows gid and gid+8)
-            float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const bool in_seq = 8 * nt + 2 * tig + e < valid;
-                    sc[nt][e] = in_seq ? sc[nt][e] * prm.scale_log2 : -INFINITY;
-                    sc[nt][2 + e] = in_seq ? sc[nt][2 + e] * prm.scale_log2 : -INFINITY;
-                    mx0 = fmaxf(mx0, sc[nt][e]);
-                    mx1 = fmaxf(mx1, sc[nt][2 + e]);
-                }
-            }
-            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-            const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-            const float a0 = ex2(m0 - mn0), a1 = ex2(m1 - mn1);
-            m0 = mn0;
-            m1 = mn1;
-            float ps0 = 0.f, ps1 = 0.f;
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    sc[nt][e] = ex2(sc[nt][e] - mn0);
-                    sc[nt][2 + e] = ex2(sc[nt][2 + e] - mn1);
-                    ps0 += sc[nt][e];
-                    ps1 += sc[nt][2 + e];
-                }
-            }
-            l0 = l0 * a0 + ps0;
-            l1 = l1 * a1 + ps1;
-#pragma unroll
-            for (int n = 0; n < NT; ++n) {
-                o[n][0] *= a0; o[n][1] *= a0;
-                o[n][2] *= a1; o[n][3] *= a1;
-            }
-            uint32_t pa[4];
-            pa[0] = Mma<T>::pack(sc[0][0], sc[0][1]);
-            pa[1] = Mma<T>::pack(sc[0][2], sc[0][3]);
-            pa[2] = Mma<T>::pack(sc[1][0], sc[1][1]);
-            pa[3] = Mma<T>::pack(sc[1][2], sc[1][3]);
-            // ---- O += P V  (V rows of tokens past the sequence are zeroed)
-            uint32_t keep_lo = 0xffffffffu, keep_hi = 0xffffffffu;
-            if (valid < 16) {
-                const int t0 = 2 * tig, t1 = 2 * tig + 8;
-                keep_lo = (t0 < valid ? 0x0000ffffu : 0u) | (t0 + 1 < valid ? 0xffff0000u : 0u);
-                keep_hi = (t1 < valid ? 0x0000ffffu : 0u) | (t1 + 1 < valid ? 0xffff0000u : 0u);
-            }
-            const int mi = lane >> 3;
-            const int tv = 16 * w + (mi & 1) * 8 + (lane & 7);
-#pragma unroll
-            for (int dp = 0; dp < D / 16; ++dp) {
-                const int hf = dp >> 2;
-                const int c = 2 * (dp & 3) + (mi >> 1);
-                uint32_t b0, b1, b2, b3;
-                ldsm_x4_trans(vbase + swz(kv_line<H, BS>(tv, hf), c), b0, b1, b2, b3);
-                b0 &= keep_lo; b1 &= keep_hi; b2 &= keep_lo; b3 &= keep_hi;
-                Mma<T>::run(o[2 * dp], pa, b0, b1);
-                Mma<T>::run(o[2 * dp + 1], pa, b2, b3);
-            }
+            consume_stage<T, D, BS>(st, smem_u32(stage), smem_u32(stage + L::kKBytes), w, lane,
+                                    valid, prm.scale_log2);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&empty[slot]));
 
         if (in.flags & kLast) {
-            // ---- merge the four warps' softmax states, then write
-            float lt0 = l0 + __shfl_xor_sync(0xffffffffu, l0, 1);
-            lt0 += __shfl_xor_sync(0xffffffffu, lt0, 2);
-            float lt1 = l1 + __shfl_xor_sync(0xffffffffu, l1, 1);
-            lt1 += __shfl_xor_sync(0xffffffffu, lt1, 2);
-            named_bar_sync(1, kConsumerWarps * 32);
-            if (tig == 0) {
-                ml[w * kMaxGroup + gid] = make_float2(m0, lt0);
-                ml[w * kMaxGroup + gid + 8] = make_float2(m1, lt1);
-            }
-            named_bar_sync(1, kConsumerWarps * 32);
-            // my rows' scale factors f = 2^(m_self - M) / L  (0 when the item is empty)
-            float fr[2];
-#pragma unroll
-            for (int rr = 0; rr < 2; ++rr) {
-                const int row = min(gid + 8 * rr, G - 1);
-                float M = -INFINITY;
-#pragma unroll
-                for (int ww = 0; ww < kConsumerWarps; ++ww)
-                    M = fmaxf(M, ml[ww * kMaxGroup + row].x);
-                float Lsum = 0.f;
-                if (M != -INFINITY) {
-#pragma unroll
-                    for (int ww = 0; ww < kConsumerWarps; ++ww) {
-                        const float2 v = ml[ww * kMaxGroup + row];
-                        Lsum += v.y * ex2(v.x - M);
-                    }
-                }
-                const float mself = rr ? m1 : m0;
-                fr[rr] = (Lsum > 0.f) ? ex2(mself - M) / Lsum : 0.f;
-            }
-            // accumulate the four warps' scaled outputs in a fixed order (deterministic)
-#pragma unroll
-            for (int ww = 0; ww < kConsumerWarps; ++ww) {
-                if (w == ww) {
-#pragma unroll
-                    for (int rr = 0; rr < 2; ++rr) {
-                        const int row = gid + 8 * rr;
-                        if (row < G) {
-                            float2 *dst =
-                                reinterpret_cast<float2 *>(obuf + row * L::kObufStride + 2 * tig);
-#pragma unroll
-                            for (int n = 0; n < NT; ++n) {
-                                float2 v = make_float2(o[n][2 * rr] * fr[rr],
-                                                       o[n][2 * rr + 1] * fr[rr]);
-                                if (ww > 0) {
-                                    const float2 prev = dst[n * 4];
-                                    v.x += prev.x;
-                                    v.y += prev.y;
-                                }
-                                dst[n * 4] = v;
-                            }
-                        }
-                    }
-                }
-                named_bar_sync(1, kConsumerWarps * 32);
-            }
+            merge_warps<D>(st, G, obuf, L::kObufStride, ml, w, lane);
             const int tid = threadIdx.x;   // 0..127
             if (in.npart == 1) {
                 T *out = reinterpret_cast<T *>(prm.out) +
@@ -590,19 +634,9 @@ paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     const int row = idx / D, dim = idx - row * D;
                     dst[idx] = obuf[row * L::kObufStride + dim];
                 }
-                if (tid < G) {
-                    float M = -INFINITY;
-                    for (int ww = 0; ww < kConsumerWarps; ++ww)
-                        M = fmaxf(M, ml[ww * kMaxGroup + tid].x);
-                    float Lsum = 0.f;
-                    if (M != -INFINITY)
-                        for (int ww = 0; ww < kConsumerWarps; ++ww) {
-                            const float2 v = ml[ww * kMaxGroup + tid];
-                            Lsum += v.y * ex2(v.x - M);
-                        }
+                if (tid < G)
                     reinterpret_cast<float2 *>(prm.ws_ml)[(size_t)in.item * G + tid] =
-                        make_float2(M, Lsum);
-                }
+                        row_stats(ml, tid);
             }
         }
     }

@@ -5,6 +5,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <climits>
 #include <cmath>
 #include <cstring>
@@ -13,6 +14,7 @@
 
 #include "cache_kernels.cuh"
 #include "decode_kernels.cuh"
+#include "shared_prefix_kernels.cuh"
 #include "pagedkv.h"
 
 namespace {
@@ -264,6 +266,77 @@ int dispatch_bs(int BS, const CUtensorMap &mk, const CUtensorMap &mv, const CUte
     return PKV_ERR_INVALID_ARG;
 }
 
+// ---- shared-prefix decode ------------------------------------------------
+// Workspace: [counters 256 B][np, row_base, seq_group, gpre, gmin, gmis: B ints each]
+// [items][partials (max, sum)][partial outputs].
+struct SharedWs {
+    size_t ints, items, ml, o, total;
+    int max_items;
+    long long rows;
+};
+
+SharedWs shared_ws_layout(int B, int Hq, int Hkv, int D, int max_len, int P) {
+    SharedWs w{};
+    const long long pmax = max_len <= P ? 1 : cdiv(max_len, P);
+    w.max_items = (int)std::min<long long>(2LL * Hkv * B * pmax, INT_MAX / 2);
+    w.rows = (long long)B * Hq * (pmax + 1);
+    w.ints = sizeof(pkv::SharedCounters);
+    w.items = w.ints + 6 * align_up((size_t)B * sizeof(int), 256);
+    w.ml = w.items + align_up((size_t)w.max_items * sizeof(pkv::SharedItem), 256);
+    w.o = w.ml + align_up((size_t)w.rows * 2 * sizeof(float), 256);
+    w.total = w.o + (size_t)w.rows * D * sizeof(float);
+    return w;
+}
+
+template <typename T, int D, int BS>
+int launch_shared_decode(const CUtensorMap &mk, const CUtensorMap &mv,
+                         const pkv::SharedParams &prm, cudaStream_t st) {
+    using L = pkv::DecodeLayout<D>;
+    auto kern = pkv::paged_decode_shared_kernel<T, D, BS>;
+    const size_t smem = 1024 + L::kRingBytes + L::obuf_bytes(pkv::kMaxGroup) + L::kMetaBytes;
+    int dev;
+    if (current_device(&dev) != PKV_OK) return PKV_ERR_CUDA;
+    static int occ[kMaxDevices];
+    int nsm;
+    if (sm_count(&nsm) != PKV_OK) return PKV_ERR_CUDA;
+    if (occ[dev] == 0) {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+            return PKV_ERR_CUDA;
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, pkv::kDecodeThreads, smem) !=
+                cudaSuccess ||
+            n <= 0)
+            return PKV_ERR_CUDA;
+        occ[dev] = n;
+    }
+    long long grid = (long long)nsm * occ[dev];
+    if (grid > prm.max_items) grid = prm.max_items;
+    if (grid < 1) grid = 1;
+    return launch(kern, dim3((unsigned)grid), dim3(pkv::kDecodeThreads), smem, st, mk, mv, prm);
+}
+
+template <typename T, int D>
+int launch_shared_path(int BS, const CUtensorMap &mk, const CUtensorMap &mv,
+                       const pkv::SharedParams &prm, cudaStream_t st) {
+    int rc = launch(pkv::shared_prefix_plan_kernel, dim3(1), dim3(pkv::kPlanThreads), 0, st, prm);
+    if (rc != PKV_OK) return rc;
+    switch (BS) {
+        case 8: rc = launch_shared_decode<T, D, 8>(mk, mv, prm, st); break;
+        case 16: rc = launch_shared_decode<T, D, 16>(mk, mv, prm, st); break;
+        case 32: rc = launch_shared_decode<T, D, 32>(mk, mv, prm, st); break;
+        default: return PKV_ERR_INVALID_ARG;
+    }
+    if (rc != PKV_OK) return rc;
+    int nsm;
+    if (sm_count(&nsm) != PKV_OK) return PKV_ERR_CUDA;
+    long long grid = (long long)prm.num_seqs * prm.num_heads;
+    if (grid > 8LL * nsm) grid = 8LL * nsm;
+    return launch(pkv::paged_decode_shared_reduce_kernel<T, D>, dim3((unsigned)grid), dim3(D), 0,
+                  st, prm);
+}
+
 }  // namespace
 
 extern "C" {
@@ -406,6 +479,98 @@ int pkv_paged_attention_decode_noalloc(void *out, const void *q, const void *k_c
                                       max_blocks_per_seq, num_blocks, max_context_len, scale,
                                       dtype, P, scratch, need > 0 ? kNoAllocScratchBytes : 0,
                                       stream);
+}
+
+int pkv_decode_shared_prefix_workspace_size(int num_seqs, int num_heads, int num_kv_heads,
+                                            int head_dim, int block_size, int max_context_len,
+                                            int partition_size, size_t *bytes_out) {
+    if (!bytes_out) return PKV_ERR_INVALID_ARG;
+    int P;
+    const int rc = check_decode_sizes(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                      max_context_len, partition_size, &P);
+    if (rc != PKV_OK) return rc;
+    *bytes_out = num_seqs ? shared_ws_layout(num_seqs, num_heads, num_kv_heads, head_dim,
+                                             max_context_len, P).total
+                          : 0;
+    return PKV_OK;
+}
+
+int pkv_paged_attention_decode_shared_prefix(
+    void *out, const void *q, const void *k_cache, const void *v_cache,
+    const int32_t *block_tables, const int32_t *context_lens, const int32_t *group_start,
+    const int32_t *prefix_lens, int num_groups, int num_seqs, int num_heads, int num_kv_heads,
+    int head_dim, int block_size, int max_blocks_per_seq, int num_blocks, int max_context_len,
+    float scale, int dtype, int partition_size, void *workspace, size_t workspace_bytes,
+    pkv_stream_t stream) {
+    int P;
+    int rc = check_decode_sizes(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                max_context_len, partition_size, &P);
+    if (rc != PKV_OK) return rc;
+    if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return PKV_ERR_INVALID_ARG;
+    if (max_blocks_per_seq < 1 || num_blocks < 1 || num_groups < 1) return PKV_ERR_INVALID_ARG;
+    if ((long long)max_context_len > (long long)max_blocks_per_seq * block_size)
+        return PKV_ERR_INVALID_ARG;
+    if ((long long)num_blocks * num_kv_heads * block_size >= INT_MAX) return PKV_ERR_INVALID_ARG;
+    if (num_seqs == 0) return PKV_OK;
+    if (num_groups > num_seqs) return PKV_ERR_INVALID_ARG;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !group_start ||
+        !prefix_lens)
+        return PKV_ERR_INVALID_ARG;
+    if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(q, 4) || !aligned(out, 2) ||
+        !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(group_start, 4) ||
+        !aligned(prefix_lens, 4))
+        return PKV_ERR_INVALID_ARG;
+    const SharedWs ws =
+        shared_ws_layout(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len, P);
+    if (!workspace || workspace_bytes < ws.total || !aligned(workspace, 16))
+        return PKV_ERR_WORKSPACE;
+    unsigned int *status;
+    if ((rc = device_status_ptr(&status)) != PKV_OK) return rc;
+    CUtensorMap mk, mv;
+    const long long cache_rows = (long long)num_blocks * num_kv_heads * block_size;
+    if ((rc = encode_rows_map(&mk, k_cache, dtype, head_dim, cache_rows, block_size)) != PKV_OK)
+        return rc;
+    if ((rc = encode_rows_map(&mv, v_cache, dtype, head_dim, cache_rows, block_size)) != PKV_OK)
+        return rc;
+    uint8_t *wsb = static_cast<uint8_t *>(workspace);
+    const size_t ib = align_up((size_t)num_seqs * sizeof(int), 256);
+    pkv::SharedParams prm;
+    prm.counters = reinterpret_cast<pkv::SharedCounters *>(wsb);
+    prm.np = reinterpret_cast<int *>(wsb + ws.ints);
+    prm.row_base = reinterpret_cast<int *>(wsb + ws.ints + ib);
+    prm.seq_group = reinterpret_cast<int *>(wsb + ws.ints + 2 * ib);
+    prm.gpre = reinterpret_cast<int *>(wsb + ws.ints + 3 * ib);
+    prm.gmin = reinterpret_cast<int *>(wsb + ws.ints + 4 * ib);
+    prm.gmis = reinterpret_cast<int *>(wsb + ws.ints + 5 * ib);
+    prm.items = reinterpret_cast<pkv::SharedItem *>(wsb + ws.items);
+    prm.ws_ml = reinterpret_cast<float *>(wsb + ws.ml);
+    prm.ws_o = reinterpret_cast<float *>(wsb + ws.o);
+    prm.out = out;
+    prm.q = q;
+    prm.block_tables = block_tables;
+    prm.context_lens = context_lens;
+    prm.group_start = group_start;
+    prm.prefix_lens = prefix_lens;
+    prm.status = status;
+    prm.num_groups = num_groups;
+    prm.num_seqs = num_seqs;
+    prm.num_heads = num_heads;
+    prm.num_kv_heads = num_kv_heads;
+    prm.group = num_heads / num_kv_heads;
+    prm.max_blocks_per_seq = max_blocks_per_seq;
+    prm.num_blocks = num_blocks;
+    prm.max_context_len = max_context_len;
+    prm.partition = P;
+    prm.block_size = block_size;
+    prm.max_items = ws.max_items;
+    prm.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (dtype == PKV_BF16)
+        return head_dim == 128 ? launch_shared_path<__nv_bfloat16, 128>(block_size, mk, mv, prm, st)
+                               : launch_shared_path<__nv_bfloat16, 64>(block_size, mk, mv, prm, st);
+    return head_dim == 128 ? launch_shared_path<__half, 128>(block_size, mk, mv, prm, st)
+                           : launch_shared_path<__half, 64>(block_size, mk, mv, prm, st);
 }
 
 int pkv_reshape_and_cache(const void *k_new, const void *v_new, void *k_cache, void *v_cache,

@@ -1,0 +1,489 @@
+// Shared-prefix-aware paged decode attention for sm_100a.
+//
+// Parallel sampling and common prompts make several sequences point at the same
+// physical prefix pages ("vLLM" entity page, 是什么; "vLLM / PagedAttention — 分页 KV
+// Cache 分析" §3.2). Plain decode streams such a page once per sequence. Here the
+// sequences of a group share the prefix: every prefix page of a KV head is streamed
+// ONCE for up to 16 query rows (the G heads of several member sequences on the MMA's
+// M dimension), each sequence's private suffix is streamed for its own G rows, and
+// the partial softmax states of the pieces are merged exactly (log-sum-exp). The
+// result is the same attention as plain decode:
+//   out[s][h] = sum_t softmax_t(scale * q[s][h] . K_s[t]) V_s[t],  t < len_s.
+//
+// Three launches: a one-CTA plan builds the item list in the workspace (and checks
+// the declared prefix against the block tables: the shared length of a group is cut
+// at the first logical block where a member's table differs from the group's first
+// member, so a wrong declaration costs sharing, never correctness); the decode kernel
+// runs the items with the same TMA / mbarrier / tensor-core pipeline as plain decode;
+// the reduce merges each (sequence, head)'s partials.
+#pragma once
+
+#include "decode_kernels.cuh"
+
+namespace pkv {
+
+struct SharedItem {
+    int table_seq;   // sequence whose block-table row holds the item's pages
+    int tok0;        // first token (a multiple of the block size)
+    int ntok;        // tokens
+    int hk;          // KV head
+    int first_seq;   // query rows: sequences first_seq .. first_seq + nseq - 1, G heads each
+    int nseq;
+    int part;        // index of this piece in each row's list of partials
+    int pad;
+};
+
+struct SharedCounters {
+    unsigned next;    // next work item
+    int count;        // items in the list
+    int pad[62];
+};
+
+struct SharedParams {
+    SharedCounters *counters;
+    SharedItem *items;
+    int *np;           // [B] partials per (sequence, head)
+    int *row_base;     // [B] scratch row of (s, h, j) = row_base[s] + h * np[s] + j
+    int *seq_group;    // [B] group of each sequence (plan scratch)
+    int *gpre;         // [B] shared tokens per group (plan scratch)
+    int *gmin;         // [B] shortest member per group (plan scratch)
+    int *gmis;         // [B] first logical block where a member's table differs (plan scratch)
+    float *ws_o;       // [rows][D]
+    float *ws_ml;      // [rows][2]
+    void *out;
+    const void *q;
+    const int32_t *block_tables;
+    const int32_t *context_lens;
+    const int32_t *group_start;   // [num_groups + 1]
+    const int32_t *prefix_lens;   // [num_groups] declared shared tokens
+    unsigned *status;
+    int num_groups, num_seqs, num_heads, num_kv_heads, group;
+    int max_blocks_per_seq, num_blocks, max_context_len, partition, block_size, max_items;
+    float scale_log2;
+};
+
+constexpr int kPlanThreads = 1024;
+
+__device__ __forceinline__ int clamp_len(int len, int max_len) {
+    return len < 0 ? 0 : (len > max_len ? max_len : len);
+}
+
+// Exclusive block-wide prefix sum of one value per thread (kPlanThreads threads);
+// returns the exclusive sum and writes the block total to *total.
+__device__ __forceinline__ int block_exclusive_scan(int v, int *sm, int *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) sm[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < kPlanThreads / 32 ? sm[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += y;
+        }
+        sm[lane] = w;   // inclusive sums of warps
+    }
+    __syncthreads();
+    const int before = warp ? sm[warp - 1] : 0;
+    *total = sm[kPlanThreads / 32 - 1];
+    __syncthreads();
+    return before + x - v;
+}
+
+// One CTA builds the item list. Groups are contiguous runs of sequences; a malformed
+// group_start makes every sequence its own group (no sharing) and sets the length
+// status bit. A group's shared length is its declared prefix cut to a multiple of the
+// block size, to its shortest member and at the first logical block where a member's
+// table differs from the first member's; a group of one shares nothing.
+__global__ void __launch_bounds__(kPlanThreads)
+shared_prefix_plan_kernel(SharedParams p) {
+    pdl_wait_and_release();
+    __shared__ int sm[kPlanThreads / 32];
+    __shared__ int bad, max_pre_blocks;
+    const int B = p.num_seqs, Hkv = p.num_kv_heads, G = p.group, P = p.partition;
+    const int BS = p.block_size;
+    const int R = kMaxGroup / G;   // member sequences per 16-row tile
+    const int tid = threadIdx.x;
+    if (tid == 0) {
+        bad = 0;
+        max_pre_blocks = 0;
+        p.counters->next = 0u;
+        const int ng = p.num_groups;
+        if (ng < 1 || ng > B || p.group_start[0] != 0 || p.group_start[ng] != B) bad = 1;
+    }
+    __syncthreads();
+    if (!bad)
+        for (int g = tid; g < p.num_groups; g += kPlanThreads)
+            if (p.group_start[g + 1] <= p.group_start[g]) atomicOr(&bad, 1);
+    __syncthreads();
+    if (tid == 0 && bad) atomicOr(p.status, kStatusBadLen);
+    const int ng = bad ? B : p.num_groups;
+    // pass 0 (per group): membership, declared prefix, identities for the minima
+    for (int g = tid; g < ng; g += kPlanThreads) {
+        const int first = bad ? g : p.group_start[g];
+        const int last = bad ? g + 1 : p.group_start[g + 1];
+        int pre = (bad || last - first < 2) ? 0 : p.prefix_lens[g];
+        pre = pre < 0 ? 0 : pre - pre % BS;
+        p.gpre[g] = pre;
+        p.gmin[g] = 0x7fffffff;
+        p.gmis[g] = 0x7fffffff;
+        for (int s = first; s < last; ++s) p.seq_group[s] = g;
+        atomicMax(&max_pre_blocks, pre / BS);
+    }
+    __syncthreads();
+    // pass 1 (per sequence): shortest member
+    for (int s = tid; s < B; s += kPlanThreads) {
+        const int g = __ldcg(&p.seq_group[s]);
+        atomicMin(&p.gmin[g], clamp_len(p.context_lens[s], p.max_context_len));
+    }
+    // pass 2 (per (sequence, prefix block)): first block where a member's table differs
+    const int mpb = max_pre_blocks;
+    for (long long i = tid; i < (long long)B * mpb; i += kPlanThreads) {
+        const int s = (int)(i / mpb), b = (int)(i - (long long)s * mpb);
+        const int g = __ldcg(&p.seq_group[s]);
+        const int first = bad ? g : p.group_start[g];
+        if (s == first || b >= __ldcg(&p.gpre[g]) / BS) continue;
+        const int mine = p.block_tables[(size_t)s * p.max_blocks_per_seq + b];
+        const int ref = p.block_tables[(size_t)first * p.max_blocks_per_seq + b];
+        if (mine != ref) atomicMin(&p.gmis[g], b);
+    }
+    __syncthreads();
+    // pass 3 (per group): shared length, prefix items
+    int base_items = 0;
+    for (int g0 = 0; g0 < ng; g0 += kPlanThreads) {
+        const int g = g0 + tid;
+        int first = 0, last = 0, pre = 0, cnt = 0;
+        if (g < ng) {
+            first = bad ? g : p.group_start[g];
+            last = bad ? g + 1 : p.group_start[g + 1];
+            const int shortest = __ldcg(&p.gmin[g]);
+            pre = min(__ldcg(&p.gpre[g]), shortest - shortest % BS);
+            pre = min(pre, min(__ldcg(&p.gmis[g]), pre / BS) * BS);
+            p.gpre[g] = pre;
+            if (pre > 0) cnt = Hkv * ((last - first + R - 1) / R) * ((pre + P - 1) / P);
+        }
+        int total;
+        int at = base_items + block_exclusive_scan(cnt, sm, &total);
+        if (cnt > 0) {
+            const int npp = (pre + P - 1) / P;
+            const int chunks = (last - first + R - 1) / R;
+            for (int hk = 0; hk < Hkv; ++hk)
+                for (int c = 0; c < chunks; ++c)
+                    for (int j = 0; j < npp; ++j, ++at) {
+                        if (at >= p.max_items) continue;
+                        SharedItem it;
+                        it.table_seq = first;
+                        it.tok0 = j * P;
+                        it.ntok = min(P, pre - j * P);
+                        it.hk = hk;
+                        it.first_seq = first + c * R;
+                        it.nseq = min(R, last - (first + c * R));
+                        it.part = j;
+                        it.pad = 0;
+                        p.items[at] = it;
+                    }
+        }
+        base_items += total;
+    }
+    __syncthreads();
+    // pass 4 (per sequence): suffix items, partial counts and scratch rows
+    int base_rows = 0;
+    for (int s0 = 0; s0 < B; s0 += kPlanThreads) {
+        const int s = s0 + tid;
+        int pre = 0, len = 0, npp = 0, nps = 0;
+        if (s < B) {
+            pre = __ldcg(&p.gpre[__ldcg(&p.seq_group[s])]);
+            len = clamp_len(p.context_lens[s], p.max_context_len);
+            npp = (pre + P - 1) / P;
+            nps = max(1, (len - pre + P - 1) / P);
+        }
+        int total_items, total_rows;
+        int at = base_items + block_exclusive_scan(s < B ? Hkv * nps : 0, sm, &total_items);
+        const int row =
+            base_rows + block_exclusive_scan(s < B ? (npp + nps) : 0, sm, &total_rows);
+        if (s < B) {
+            p.np[s] = npp + nps;
+            p.row_base[s] = row * p.num_heads;
+            for (int hk = 0; hk < Hkv; ++hk)
+                for (int j = 0; j < nps; ++j, ++at) {
+                    if (at >= p.max_items) continue;
+                    SharedItem it;
+                    it.table_seq = s;
+                    it.tok0 = pre + j * P;
+                    it.ntok = max(0, min(P, len - pre - j * P));
+                    it.hk = hk;
+                    it.first_seq = s;
+                    it.nseq = 1;
+                    it.part = npp + j;
+                    it.pad = 0;
+                    p.items[at] = it;
+                }
+        }
+        base_items += total_items;
+        base_rows += total_rows;
+    }
+    if (tid == 0) {
+        if (base_items > p.max_items) atomicOr(p.status, kStatusBadLen);
+        p.counters->count = min(base_items, p.max_items);
+    }
+}
+
+template <typename T, int D, int BS>
+__global__ void __launch_bounds__(kDecodeThreads, 2)
+paged_decode_shared_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                           const __grid_constant__ CUtensorMap tmap_v, SharedParams prm) {
+    using L = DecodeLayout<D>;
+    constexpr int kBPS = kStageTokens / BS;
+    constexpr int H = L::kHalves;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *ring = smem;
+    float *obuf = reinterpret_cast<float *>(smem + L::kRingBytes);
+    StageInfo *info = reinterpret_cast<StageInfo *>(reinterpret_cast<uint8_t *>(obuf) +
+                                                    L::obuf_bytes(kMaxGroup));
+    uint64_t *full = reinterpret_cast<uint64_t *>(info + L::kStages);
+    uint64_t *empty = full + L::kStages;
+    float2 *ml = reinterpret_cast<float2 *>(empty + L::kStages);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int G = prm.group;
+    const int Hkv = prm.num_kv_heads;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < L::kStages; ++i) {
+            mbar_init(smem_u32(&full[i]), 1);
+            mbar_init(smem_u32(&empty[i]), kConsumerWarps);
+        }
+        fence_mbar_init();
+    }
+    pdl_wait_and_release();
+    __syncthreads();
+
+    if (warp == kConsumerWarps) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            prefetch_tensormap(&tmap_k);
+            prefetch_tensormap(&tmap_v);
+        }
+        const uint64_t kv_policy = l2_evict_first_policy();
+        const int count = prm.counters->count;
+        int it = 0;
+        bool ok = true;
+        // item descriptor: lane k < 8 holds field k
+        auto fetch = [&](int idx) {
+            int v = 0;
+            if (idx < count && lane < 8) v = reinterpret_cast<const int *>(prm.items + idx)[lane];
+            return v;
+        };
+        auto take = [&]() {
+            unsigned v = 0;
+            if (lane == 0) v = atomicAdd(&prm.counters->next, 1u);
+            v = __shfl_sync(0xffffffffu, v, 0);
+            return v > 0x7fffffffu ? 0x7fffffff : (int)v;
+        };
+        int cur_idx = take();
+        int cur_f = fetch(cur_idx);
+        while (cur_idx < count && ok) {
+            const int table_seq = __shfl_sync(0xffffffffu, cur_f, 0);
+            const int tok0 = __shfl_sync(0xffffffffu, cur_f, 1);
+            const int ntok = __shfl_sync(0xffffffffu, cur_f, 2);
+            const int hk = __shfl_sync(0xffffffffu, cur_f, 3);
+            const int first_seq = __shfl_sync(0xffffffffu, cur_f, 4);
+            const int nseq = __shfl_sync(0xffffffffu, cur_f, 5);
+            const int part = __shfl_sync(0xffffffffu, cur_f, 6);
+            const int nst = max(1, (ntok + kStageTokens - 1) / kStageTokens);
+            const int nblk = (ntok + BS - 1) / BS;
+            int ent[kMaxItemBlocks / 32];
+            const int32_t *bt =
+                prm.block_tables + (size_t)table_seq * prm.max_blocks_per_seq + tok0 / BS;
+#pragma unroll
+            for (int k = 0; k < kMaxItemBlocks / 32; ++k) {
+                const int e = k * 32 + lane;
+                ent[k] = e < nblk ? bt[e] : 0;
+            }
+            int nxt_idx = 0, nxt_f = 0;
+            for (int st = 0; st < nst; ++st, ++it) {
+                const int slot = it % L::kStages;
+                const uint32_t ph = ((it / L::kStages) & 1) ^ 1;
+                if (!warp_wait(smem_u32(&empty[slot]), ph)) {
+                    if (lane == 0) atomicOr(prm.status, kStatusTimeout);
+                    ok = false;
+                    break;
+                }
+                const int sntok = max(0, min(kStageTokens, ntok - st * kStageTokens));
+                const int nb_st = (sntok + BS - 1) / BS;
+                const int e0 = st * kBPS;
+                const int reg = e0 >> 5;
+                int v = ent[0];
+#pragma unroll
+                for (int k = 1; k < kMaxItemBlocks / 32; ++k)
+                    if (reg == k) v = ent[k];
+                const int bid = __shfl_sync(0xffffffffu, v, (e0 + lane) & 31);
+                const uint32_t bar = smem_u32(&full[slot]);
+                if (lane == 0) {
+                    StageInfo in;
+                    in.s = first_seq; in.hk = hk; in.p = part; in.npart = nseq;
+                    in.item = cur_idx;
+                    in.ntok = sntok;
+                    in.flags = (st == 0 ? kFirst : 0) | (st == nst - 1 ? kLast : 0);
+                    in.pad = 0;
+                    info[slot] = in;
+                    mbar_arrive_expect_tx(bar, (uint32_t)(nb_st * BS * L::kRowBytes * 2));
+                }
+                __syncwarp();
+                if (lane < nb_st) {
+                    int y;
+                    if (bid >= 0 && bid < prm.num_blocks) {
+                        y = (bid * Hkv + hk) * BS;
+                    } else {
+                        atomicOr(prm.status, kStatusBadBlock);
+                        y = prm.num_blocks * Hkv * BS;
+                    }
+                    uint8_t *stage = ring + slot * L::kStageBytes;
+                    const uint32_t off = lane * BS * L::kRowBytes;
+                    if (H == 2) {
+                        tma_load_3d(smem_u32(stage + off), &tmap_k, 0, y, 0, bar, kv_policy);
+                        tma_load_3d(smem_u32(stage + L::kKBytes + off), &tmap_v, 0, y, 0, bar,
+                                    kv_policy);
+                    } else {
+                        tma_load_2d(smem_u32(stage + off), &tmap_k, 0, y, bar, kv_policy);
+                        tma_load_2d(smem_u32(stage + L::kKBytes + off), &tmap_v, 0, y, bar,
+                                    kv_policy);
+                    }
+                }
+                if (st == 0) {
+                    nxt_idx = take();
+                    nxt_f = fetch(nxt_idx);
+                }
+            }
+            cur_idx = nxt_idx;
+            cur_f = nxt_f;
+        }
+        if (ok) {
+            const int slot = it % L::kStages;
+            const uint32_t ph = ((it / L::kStages) & 1) ^ 1;
+            if (warp_wait(smem_u32(&empty[slot]), ph)) {
+                if (lane == 0) {
+                    StageInfo in = {};
+                    in.s = -1;
+                    in.flags = kEnd;
+                    info[slot] = in;
+                    mbar_arrive(smem_u32(&full[slot]));
+                }
+            } else {
+                if (lane == 0) atomicOr(prm.status, kStatusTimeout);
+                ok = false;
+            }
+        }
+        if (!ok) {
+            for (int j = max(0, it - L::kStages); j < it; ++j)
+                warp_wait(smem_u32(&full[j % L::kStages]), (j / L::kStages) & 1);
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------------- consumers
+    const int w = warp;
+    const int gid = lane >> 2;
+    const int tig = lane & 3;
+    constexpr int KS = D / 16;
+    WarpState<D> st;
+    reset_state(st);
+    const T *qg = reinterpret_cast<const T *>(prm.q);
+
+    for (int it = 0;; ++it) {
+        const int slot = it % L::kStages;
+        if (!warp_wait(smem_u32(&full[slot]), (it / L::kStages) & 1)) {
+            if (lane == 0) atomicOr(prm.status, kStatusTimeout);
+            break;
+        }
+        const StageInfo in = info[slot];
+        if (in.flags & kEnd) break;
+        const int nrows = in.npart * G;
+
+        if (in.flags & kFirst) {
+            // A fragments of the item's rows r = member * G + head (rows >= nrows are zero)
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int r = gid + 8 * half;
+                const uint32_t *qr = nullptr;
+                if (r < nrows) {
+                    const int s = in.s + r / G, h = in.hk * G + r % G;
+                    qr = reinterpret_cast<const uint32_t *>(
+                        qg + ((size_t)s * prm.num_heads + h) * D);
+                }
+#pragma unroll
+                for (int ks = 0; ks < KS; ++ks) {
+                    st.qa[ks][half] = qr ? __ldg(qr + ks * 8 + tig) : 0u;
+                    st.qa[ks][2 + half] = qr ? __ldg(qr + ks * 8 + tig + 4) : 0u;
+                }
+            }
+            reset_state(st);
+        }
+
+        const int valid = in.ntok - 16 * w;
+        if (valid > 0) {
+            const uint8_t *stage = ring + slot * L::kStageBytes;
+            consume_stage<T, D, BS>(st, smem_u32(stage), smem_u32(stage + L::kKBytes), w, lane,
+                                    valid, prm.scale_log2);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&empty[slot]));
+
+        if (in.flags & kLast) {
+            merge_warps<D>(st, nrows, obuf, L::kObufStride, ml, w, lane);
+            const int tid = threadIdx.x;
+            for (int idx = tid; idx < nrows * D; idx += kConsumerWarps * 32) {
+                const int r = idx / D, dim = idx - r * D;
+                const int s = in.s + r / G, h = in.hk * G + r % G;
+                const size_t row = (size_t)prm.row_base[s] + (size_t)h * prm.np[s] + in.p;
+                prm.ws_o[row * D + dim] = obuf[r * L::kObufStride + dim];
+            }
+            if (tid < nrows) {
+                const int s = in.s + tid / G, h = in.hk * G + tid % G;
+                const size_t row = (size_t)prm.row_base[s] + (size_t)h * prm.np[s] + in.p;
+                reinterpret_cast<float2 *>(prm.ws_ml)[row] = row_stats(ml, tid);
+            }
+        }
+    }
+}
+
+// Merge of every (sequence, head)'s partials: rows row_base[s] + h*np[s] + j, j < np[s].
+//   M = max m_j;  w_j = l_j 2^(m_j - M);  out = sum w_j o_j / sum w_j
+template <typename T, int D>
+__global__ void __launch_bounds__(D)
+paged_decode_shared_reduce_kernel(SharedParams prm) {
+    pdl_wait_and_release();
+    const float2 *mlp = reinterpret_cast<const float2 *>(prm.ws_ml);
+    const int tid = threadIdx.x;
+    const int pairs = prm.num_seqs * prm.num_heads;
+    for (int pr = blockIdx.x; pr < pairs; pr += gridDim.x) {
+        const int s = pr / prm.num_heads;
+        const int h = pr - s * prm.num_heads;
+        const int np = prm.np[s];
+        const size_t row0 = (size_t)prm.row_base[s] + (size_t)h * np;
+        float M = -INFINITY;
+        for (int j = 0; j < np; ++j) M = fmaxf(M, mlp[row0 + j].x);
+        float Lsum = 0.f, acc = 0.f;
+        if (M != -INFINITY) {
+            for (int j = 0; j < np; ++j) {
+                const float2 v = mlp[row0 + j];
+                const float wv = v.y * ex2(v.x - M);
+                Lsum += wv;
+                acc += wv * prm.ws_o[(row0 + j) * D + tid];
+            }
+        }
+        T *out = reinterpret_cast<T *>(prm.out) + ((size_t)s * prm.num_heads + h) * D;
+        out[tid] = from_float<T>(Lsum > 0.f ? acc / Lsum : 0.f);
+    }
+}
+
+}  // namespace pkv
