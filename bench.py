@@ -459,6 +459,7 @@ def gpu_arm(args, rank, world, local_rank):
     peak, peak_kind = read_peaks()
     achieved = roof_layer / (k1_avg_ms * 1e-3) / 1e9
     read_probe = hbm_read_probe(dev, stream)
+    swap = swap_measurement(wl, dev, stream) if args.swap else None
     traffic = None if shared else read_traffic(args.workload, sp.block_size)
 
     # ---- end to end: host block manager + pinned host buffers through the public API
@@ -491,6 +492,7 @@ def gpu_arm(args, rank, world, local_rank):
         },
         "tokens_per_s": round(tokens_per_s, 1),
         "pct_of_hbm_peak": round(100 * value / world / peak, 2),
+        **({"swap_blocks": swap} if swap else {}),
         "clocks": clocks.summary(),
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
@@ -544,6 +546,57 @@ def replay_block_manager(wl):
             lens, wl.context_lens):
         raise RuntimeError("block manager replay does not reproduce the workload's tables")
     return mgr
+
+
+def swap_measurement(wl, dev, stream, budget=512 << 20, reps=5):
+    """Preemption swap: every block (all layers, K and V) of whole sequences, longest
+    first until ~budget bytes, out to pinned host memory and back in with one kernel each
+    way; beside it a contiguous pinned copy of the same bytes (what the link gives)."""
+    import torch
+    import paged_kv_cache_320_b200 as pkv
+    sp = wl.spec
+    L = sp.num_layers
+    tile = sp.num_kv_heads * sp.block_size * sp.head_dim * 2
+    per_block = L * 2 * tile
+    ids, seqs = [], []
+    for s in np.argsort(-wl.context_lens.astype(np.int64), kind="stable"):
+        nb = -(-int(wl.context_lens[s]) // sp.block_size)
+        if ids and (len(ids) + nb) * per_block > budget:
+            break
+        ids += [int(b) for b in wl.block_tables[s, :nb]]
+        seqs.append(int(s))
+    nbytes = len(ids) * per_block
+    kp = torch.tensor([t.data_ptr() for t in wl.k_cache], dtype=torch.int64, device=dev)
+    vp = torch.tensor([t.data_ptr() for t in wl.v_cache], dtype=torch.int64, device=dev)
+    ids_d = torch.tensor(ids, dtype=torch.int32, device=dev)
+    host = torch.empty(nbytes // 2, dtype=torch.int16).pin_memory()
+    code = pkv.PKV_F16 if sp.dtype == synth.F16 else pkv.PKV_BF16
+
+    def timed(fn):
+        fn()
+        best = float("inf")
+        for _ in range(reps):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            b.synchronize()
+            best = min(best, a.elapsed_time(b))
+        return nbytes / (best * 1e-3) / 1e9
+
+    swap = lambda to_host: pkv.pkv_swap_blocks(kp, vp, ids_d, host, to_host, sp.num_kv_heads,
+                                               sp.head_dim, sp.block_size, wl.num_blocks, code,
+                                               stream=stream)
+    out_gbs = timed(lambda: swap(1))
+    in_gbs = timed(lambda: swap(0))
+    dbuf = torch.empty(nbytes // 2, dtype=torch.int16, device=dev)
+    with torch.cuda.stream(stream):
+        d2h = timed(lambda: host.copy_(dbuf, non_blocking=True))
+        h2d = timed(lambda: dbuf.copy_(host, non_blocking=True))
+    return {"sequences": len(seqs), "blocks": len(ids), "bytes": nbytes,
+            "out_gbs": round(out_gbs, 1), "in_gbs": round(in_gbs, 1),
+            "contiguous_d2h_gbs": round(d2h, 1), "contiguous_h2d_gbs": round(h2d, 1)}
 
 
 def hbm_read_probe(dev, stream):
@@ -769,6 +822,8 @@ def main():
     ap.add_argument("--block-size", type=int, default=0)
     ap.add_argument("--layers", type=int, default=0, help="override the workload's layer count")
     ap.add_argument("--partition", type=int, default=0, help="decode partition size (0 = auto)")
+    ap.add_argument("--swap", action="store_true",
+                    help="also time pkv_swap_blocks (preemption) against a contiguous copy")
     ap.add_argument("--decode", default="plain", choices=["plain", "shared"],
                     help="shared: the shared-prefix-aware decode (shared-prefix workload)")
     ap.add_argument("--batch", type=int, default=0,

@@ -65,7 +65,7 @@ enum pkv_dtype { PKV_F16 = 0, PKV_BF16 = 1 };
 /* Bits of the per-device status word (pkv_get_device_status). */
 enum pkv_device_status_bits {
     PKV_STATUS_BAD_SLOT = 1u << 0,     /* reshape_and_cache: slot >= num_blocks*block_size      */
-    PKV_STATUS_BAD_PAIR = 1u << 1,     /* copy_blocks: src or dst outside [0, num_blocks)       */
+    PKV_STATUS_BAD_PAIR = 1u << 1,     /* copy_blocks / swap_blocks: block id outside the pool  */
     PKV_STATUS_BAD_BLOCK = 1u << 2,    /* decode: block id outside [0, num_blocks) (read as 0)  */
     PKV_STATUS_BAD_LEN = 1u << 3,      /* decode: context_len < 0 or above its bound (clamped)  */
     PKV_STATUS_WAIT_TIMEOUT = 1u << 4  /* decode: a pipeline wait exceeded its iteration limit  */
@@ -143,7 +143,7 @@ int pkv_paged_attention_decode_noalloc(void *out, const void *q, const void *k_c
  * Shared-prefix-aware decode: the same result as pkv_paged_attention_decode, for
  * batches where groups of sequences share their first pages (parallel sampling, common
  * prompts: "vLLM" entity page, 是什么; "分页 KV Cache 分析" §3.2). Each shared prefix page
- * of a KV head is read once for up to 16 query rows (the G heads of several member
+ * of a KV head is read once for up to 16 query rows (the G heads of up to 16/G member
  * sequences) instead of once per sequence; private suffixes are read per sequence; the
  * pieces are merged exactly (log-sum-exp).
  *
@@ -207,6 +207,28 @@ int pkv_reshape_and_cache(const void *k_new, const void *v_new, void *k_cache, v
  * ---------------------------------------------------------------------------- */
 int pkv_copy_blocks(void *const *k_caches, void *const *v_caches, int num_layers,
                     const int32_t *block_pairs, int num_pairs, int num_kv_heads, int head_dim,
+                    int block_size, int num_blocks, int dtype, pkv_stream_t stream);
+
+/* ------------------------------------------------------------------------------
+ * Swap of whole blocks between the device caches and pinned host memory, for
+ * preemption ("vLLM/PagedAttention — L3 Cross-Paper Synthesis" §3: eviction swaps every
+ * block of a request out; "vLLM" entity page, observation 2: host transfers made of many
+ * small copies leave the link mostly idle). One kernel moves every listed block of every
+ * layer, K and V, through mapped host memory:
+ *   to_host = 1: host_buffer[l][kv][i][:] = (kv ? v_caches : k_caches)[l][block_ids[i]]
+ *   to_host = 0: the reverse (blocks are written back to the listed ids)
+ * host_buffer: HOST pointer to pinned memory (cudaHostAlloc / a pinned torch tensor) that
+ * the current device can address; layout [num_layers][2][num_ids][Hkv*BS*D] elements,
+ * at least num_layers*2*num_ids*Hkv*BS*D*2 bytes, 16-byte aligned. Anything else
+ * (pageable or device memory, too small) is rejected with PKV_ERR_INVALID_ARG before
+ * launch. k_caches / v_caches / block_ids are device arrays as for pkv_copy_blocks; ids
+ * outside [0, num_blocks) are skipped and set PKV_STATUS_BAD_PAIR. For to_host = 0 the
+ * ids must be distinct. The copy is asynchronous on `stream`: the host buffer is
+ * complete (or may be refilled) once the stream reaches this point.
+ * ---------------------------------------------------------------------------- */
+int pkv_swap_blocks(void *const *k_caches, void *const *v_caches, int num_layers,
+                    const int32_t *block_ids, int num_ids, void *host_buffer,
+                    size_t host_buffer_bytes, int to_host, int num_kv_heads, int head_dim,
                     int block_size, int num_blocks, int dtype, pkv_stream_t stream);
 
 /* Synchronise `stream`, then read (and with clear != 0 reset) the status word of the

@@ -43,3 +43,29 @@ def copy_blocks(k_caches, v_caches, block_pairs):
             out_k[layer][int(dst)] = k_caches[layer][int(src)]
             out_v[layer][int(dst)] = v_caches[layer][int(src)]
     return out_k, out_v
+
+
+def swap_out(k_caches, v_caches, block_ids):
+    """Host buffer [L][2][n][Hkv, bs, d] holding every layer's K and V page of each listed
+    block, in list order ("vLLM/PagedAttention — L3 Cross-Paper Synthesis" §3: a
+    preempted request's pages are swapped out whole)."""
+    ids = [int(b) for b in np.asarray(block_ids).reshape(-1)]
+    L = len(k_caches)
+    tile = k_caches[0].shape[1:]
+    buf = np.empty((L, 2, len(ids)) + tuple(tile), dtype=k_caches[0].dtype)
+    for layer in range(L):
+        for i, b in enumerate(ids):
+            buf[layer, 0, i] = k_caches[layer][b]
+            buf[layer, 1, i] = v_caches[layer][b]
+    return buf
+
+
+def swap_in(k_caches, v_caches, block_ids, buf):
+    """Copies of the caches with page block_ids[i] of every layer set from the buffer."""
+    out_k = [np.array(c, copy=True) for c in k_caches]
+    out_v = [np.array(c, copy=True) for c in v_caches]
+    for layer in range(len(out_k)):
+        for i, b in enumerate(np.asarray(block_ids).reshape(-1)):
+            out_k[layer][int(b)] = buf[layer, 0, i]
+            out_v[layer][int(b)] = buf[layer, 1, i]
+    return out_k, out_v

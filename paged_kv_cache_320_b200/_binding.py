@@ -68,6 +68,7 @@ def lib() -> ctypes.CDLL:
         L.pkv_reshape_and_cache.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P]
         L.pkv_copy_blocks.argtypes = [P, P, I, P, I, I, I, I, I, I, P]
         L.pkv_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), I, P]
+        L.pkv_swap_blocks.argtypes = [P, P, I, P, I, P, SZ, I, I, I, I, I, I, P]
         L.pkv_alloc_create.argtypes = [ctypes.POINTER(P), I, I, I, P]
         L.pkv_alloc_destroy.argtypes = [P]
         L.pkv_seq_append.argtypes = [P, I64, I, P, P, ctypes.POINTER(I)]
@@ -82,6 +83,7 @@ def lib() -> ctypes.CDLL:
                      "pkv_paged_attention_decode_shared_prefix",
                      "pkv_decode_shared_prefix_workspace_size", "pkv_decode_workspace_size",
                      "pkv_decode_partition_size", "pkv_reshape_and_cache", "pkv_copy_blocks",
+                     "pkv_swap_blocks",
                      "pkv_get_device_status", "pkv_alloc_create", "pkv_alloc_destroy",
                      "pkv_seq_append", "pkv_seq_append_batch", "pkv_seq_fork", "pkv_seq_free",
                      "pkv_block_tables",
@@ -244,6 +246,19 @@ def pkv_copy_blocks(k_cache_ptrs, v_cache_ptrs, block_pairs, num_kv_heads, head_
     _check(lib().pkv_copy_blocks(_ptr(k_cache_ptrs), _ptr(v_cache_ptrs), k_cache_ptrs.numel(),
                                  _ptr(block_pairs), n, num_kv_heads, head_dim, block_size,
                                  num_blocks, dtype, _stream(stream)), "pkv_copy_blocks")
+
+
+def pkv_swap_blocks(k_cache_ptrs, v_cache_ptrs, block_ids, host_buffer, to_host, num_kv_heads,
+                    head_dim, block_size, num_blocks, dtype, stream=None):
+    """Moves whole blocks between the caches and a pinned host tensor (see pagedkv.h).
+    k_cache_ptrs / v_cache_ptrs: int64 device tensors of cache addresses; block_ids:
+    int32 device tensor; host_buffer: pinned CPU tensor."""
+    n = block_ids.numel()
+    _check(lib().pkv_swap_blocks(_ptr(k_cache_ptrs), _ptr(v_cache_ptrs), k_cache_ptrs.numel(),
+                                 _ptr(block_ids), n, _ptr(host_buffer),
+                                 host_buffer.numel() * host_buffer.element_size(), int(to_host),
+                                 num_kv_heads, head_dim, block_size, num_blocks, dtype,
+                                 _stream(stream)), "pkv_swap_blocks")
 
 
 def pkv_get_device_status(clear=True, stream=None) -> int:

@@ -69,4 +69,39 @@ copy_blocks_kernel(void *const *__restrict__ k_caches, void *const *__restrict__
     for (; i < block_vecs; i += 256) d[i] = s[i];
 }
 
+// Swap of whole blocks between the device caches and a pinned host buffer, for
+// preemption ("vLLM/PagedAttention — L3 Cross-Paper Synthesis" §3: all-or-nothing
+// eviction swaps every block of a request; "vLLM" entity page, observation 2: copies
+// of small fragments one cudaMemcpyAsync at a time leave the host link mostly idle).
+// One kernel moves every listed block of every layer through mapped host memory.
+// Host buffer layout: [layer][K, V][i][Hkv * BS * D elements] for block_ids[i].
+//   to_host = 1: host[l][kv][i] = cache_l,kv[block_ids[i]]
+//   to_host = 0: cache_l,kv[block_ids[i]] = host[l][kv][i]
+// One CTA per (block, layer, K|V); 16-byte vectors, four in flight per thread.
+__global__ void __launch_bounds__(256)
+swap_blocks_kernel(void *const *__restrict__ k_caches, void *const *__restrict__ v_caches,
+                   const int32_t *__restrict__ block_ids, int n_blocks, uint4 *host,
+                   int num_blocks, int block_vecs, int to_host, unsigned *status) {
+    pdl_wait_and_release();
+    const int i = blockIdx.x;
+    const int layer = blockIdx.y;
+    const int kv = blockIdx.z;
+    const int b = block_ids[i];
+    if (b < 0 || b >= num_blocks) {
+        if (threadIdx.x == 0 && kv == 0 && layer == 0) atomicOr(status, 2u /* bad pair */);
+        return;
+    }
+    uint4 *cache = reinterpret_cast<uint4 *>(kv ? v_caches[layer] : k_caches[layer]) +
+                   (int64_t)b * block_vecs;
+    uint4 *h = host + (((int64_t)layer * 2 + kv) * n_blocks + i) * block_vecs;
+    const uint4 *src = to_host ? cache : h;
+    uint4 *dst = to_host ? h : cache;
+    int t = threadIdx.x;
+    for (; t + 3 * 256 < block_vecs; t += 4 * 256) {
+        const uint4 a = src[t], c = src[t + 256], d = src[t + 512], e = src[t + 768];
+        dst[t] = a; dst[t + 256] = c; dst[t + 512] = d; dst[t + 768] = e;
+    }
+    for (; t < block_vecs; t += 256) dst[t] = src[t];
+}
+
 }  // namespace pkv

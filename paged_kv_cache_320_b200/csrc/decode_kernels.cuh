@@ -222,12 +222,12 @@ __device__ __forceinline__ void reset_state(WarpState<D> &st) {
     st.l0 = st.l1 = 0.f;
 }
 
-// One warp's share of a stage: tokens 16w .. 16w+15 of the stage's K and V tiles,
-// of which the first `valid` belong to the sequence.
+// One warp's share of a stage: tokens tok0 .. tok0+15 of the stage's K and V tiles
+// (tok0 a multiple of 16), of which the first `valid` belong to the sequence.
 //   S = Q K^T (two n-tiles of 8 tokens), scale, mask, online softmax, O += P V.
 template <typename T, int D, int BS>
 __device__ __forceinline__ void consume_stage(WarpState<D> &st, uint32_t kbase, uint32_t vbase,
-                                              int w, int lane, int valid, float scale_log2) {
+                                              int tok0, int lane, int valid, float scale_log2) {
     constexpr int H = D / 64;
     constexpr int NT = D / 8;
     const int tig = lane & 3;
@@ -235,7 +235,7 @@ __device__ __forceinline__ void consume_stage(WarpState<D> &st, uint32_t kbase, 
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
         sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
-        const int t = 16 * w + 8 * nt + (lane & 7);
+        const int t = tok0 + 8 * nt + (lane & 7);
         const int mi = lane >> 3;
 #pragma unroll
         for (int hf = 0; hf < H; ++hf) {
@@ -301,7 +301,7 @@ __device__ __forceinline__ void consume_stage(WarpState<D> &st, uint32_t kbase, 
         keep_hi = (t1 < valid ? 0x0000ffffu : 0u) | (t1 + 1 < valid ? 0xffff0000u : 0u);
     }
     const int mi = lane >> 3;
-    const int tv = 16 * w + (mi & 1) * 8 + (lane & 7);
+    const int tv = tok0 + (mi & 1) * 8 + (lane & 7);
 #pragma unroll
     for (int dp = 0; dp < D / 16; ++dp) {
         const int hf = dp >> 2;
@@ -612,8 +612,8 @@ paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const int valid = in.ntok - 16 * w;   // tokens of my 16-token slice in the sequence
         if (valid > 0) {
             const uint8_t *stage = ring + slot * L::kStageBytes;
-            consume_stage<T, D, BS>(st, smem_u32(stage), smem_u32(stage + L::kKBytes), w, lane,
-                                    valid, prm.scale_log2);
+            consume_stage<T, D, BS>(st, smem_u32(stage), smem_u32(stage + L::kKBytes), 16 * w,
+                                    lane, valid, prm.scale_log2);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&empty[slot]));
@@ -642,12 +642,63 @@ paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
     }
 }
 
-// Merge of a sequence's partitions for one query head (log-sum-exp):
-//   M = max_p m_p;  w_p = l_p 2^(m_p - M);  out = sum_p w_p o_p / sum_p w_p
-// (m_p in log2 units, o_p normalised). CTAs of D threads loop over the (query head,
-// sequence) pairs; pairs of single-partition sequences are skipped.
+// Log-sum-exp merge of n partials (m_j in log2 units, l_j, normalised o_j) of one
+// (sequence, query head), by one warp: lane k owns output dims k*D/32 .. (k+1)*D/32-1.
+//   M = max m_j;  w_j = l_j 2^(m_j - M);  out = sum_j w_j o_j / sum_j w_j
+// Partial j's (m, l) is at ml[j * ml_stride], its output row at o + j * o_stride.
 template <typename T, int D>
-__global__ void __launch_bounds__(D)
+__device__ __forceinline__ void warp_merge(const float2 *ml, size_t ml_stride, const float *o,
+                                           size_t o_stride, int n, T *out, int lane) {
+    constexpr int V = D / 32;   // dims per lane (4 or 2)
+    float M = -INFINITY;
+    for (int j = lane; j < n; j += 32) M = fmaxf(M, ml[(size_t)j * ml_stride].x);
+#pragma unroll
+    for (int x = 16; x > 0; x >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, x));
+    float L = 0.f;
+    if (M != -INFINITY)
+        for (int j = lane; j < n; j += 32) {
+            const float2 v = ml[(size_t)j * ml_stride];
+            L += v.y * ex2(v.x - M);
+        }
+#pragma unroll
+    for (int x = 16; x > 0; x >>= 1) L += __shfl_xor_sync(0xffffffffu, L, x);
+    float acc[V];
+#pragma unroll
+    for (int i = 0; i < V; ++i) acc[i] = 0.f;
+    if (L > 0.f) {
+        const float inv = 1.f / L;
+        for (int j0 = 0; j0 < n; j0 += 32) {
+            float wmine = 0.f;
+            if (j0 + lane < n) {
+                const float2 v = ml[(size_t)(j0 + lane) * ml_stride];
+                wmine = v.y * ex2(v.x - M) * inv;
+            }
+            const int cnt = min(32, n - j0);
+#pragma unroll 4
+            for (int k = 0; k < cnt; ++k) {
+                const float wj = __shfl_sync(0xffffffffu, wmine, k);
+                const float *row = o + (size_t)(j0 + k) * o_stride + lane * V;
+                if (V == 4) {
+                    const float4 x = *reinterpret_cast<const float4 *>(row);
+                    acc[0] += wj * x.x; acc[1] += wj * x.y; acc[2] += wj * x.z; acc[3] += wj * x.w;
+                } else {
+                    const float2 x = *reinterpret_cast<const float2 *>(row);
+                    acc[0] += wj * x.x; acc[1] += wj * x.y;
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < V; ++i) out[lane * V + i] = from_float<T>(acc[i]);
+}
+
+constexpr int kReduceWarps = 8;
+
+// Merge of a sequence's partitions for one query head; one warp per (sequence,
+// query head) pair, pairs of single-partition sequences skipped. Block 0 re-arms the
+// work counter of the workspace for the next decode.
+template <typename T, int D>
+__global__ void __launch_bounds__(kReduceWarps * 32)
 paged_decode_reduce_kernel(DecodeParams prm) {
     pdl_wait_and_release();
     if (blockIdx.x == 0 && threadIdx.x == 0 && prm.sched) {
@@ -656,72 +707,22 @@ paged_decode_reduce_kernel(DecodeParams prm) {
         __threadfence();
         prm.sched->armed = kSchedArmed;
     }
-    extern __shared__ float wsm[];   // [np] weights
-    __shared__ float red[D / 32];
-    __shared__ float bcast;
-    const float2 *mlp = reinterpret_cast<const float2 *>(prm.ws_ml);
-    const int tid = threadIdx.x;
-    const int G = prm.group;
+    const int lane = threadIdx.x & 31;
+    const int pair = blockIdx.x * kReduceWarps + (threadIdx.x >> 5);
+    if (pair >= prm.num_seqs * prm.num_heads) return;
+    const int s = pair / prm.num_heads;
+    const int h = pair - s * prm.num_heads;
+    int len = prm.context_lens[s];
+    len = len < 0 ? 0 : (len > prm.max_context_len ? prm.max_context_len : len);
     const int P = prm.partition;
-    const int pairs = prm.num_seqs * prm.num_heads;
-    for (int pr = blockIdx.x; pr < pairs; pr += gridDim.x) {
-        const int s = pr / prm.num_heads;
-        const int h = pr - s * prm.num_heads;
-        int len = prm.context_lens[s];
-        len = len < 0 ? 0 : (len > prm.max_context_len ? prm.max_context_len : len);
-        const int np = max(1, (len + P - 1) / P);
-        if (np == 1) continue;
-        const int hk = h / G, g = h - hk * G;
-        const int base = prm.ws_seq_base[s] + hk * np;
-
-        float M = -INFINITY;
-        for (int p = tid; p < np; p += D) M = fmaxf(M, mlp[(size_t)(base + p) * G + g].x);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-        if ((tid & 31) == 0) red[tid >> 5] = M;
-        __syncthreads();
-        if (tid == 0) {
-            float v = red[0];
-            for (int i = 1; i < D / 32; ++i) v = fmaxf(v, red[i]);
-            bcast = v;
-        }
-        __syncthreads();
-        M = bcast;
-        float Ls = 0.f;
-        for (int p = tid; p < np; p += D) {
-            const float2 v = mlp[(size_t)(base + p) * G + g];
-            const float wv = (M == -INFINITY) ? 0.f : v.y * ex2(v.x - M);
-            wsm[p] = wv;
-            Ls += wv;
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
-        __syncthreads();
-        if ((tid & 31) == 0) red[tid >> 5] = Ls;
-        __syncthreads();
-        if (tid == 0) {
-            float v = 0.f;
-            for (int i = 0; i < D / 32; ++i) v += red[i];
-            bcast = v;
-        }
-        __syncthreads();
-        Ls = bcast;
-        const float *op = prm.ws_o + ((size_t)base * G + g) * D + tid;
-        const size_t stride = (size_t)G * D;
-        float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
-        int p = 0;
-        for (; p + 4 <= np; p += 4) {
-            acc0 += wsm[p] * op[(size_t)p * stride];
-            acc1 += wsm[p + 1] * op[(size_t)(p + 1) * stride];
-            acc2 += wsm[p + 2] * op[(size_t)(p + 2) * stride];
-            acc3 += wsm[p + 3] * op[(size_t)(p + 3) * stride];
-        }
-        for (; p < np; ++p) acc0 += wsm[p] * op[(size_t)p * stride];
-        const float acc = (acc0 + acc1) + (acc2 + acc3);
-        T *out = reinterpret_cast<T *>(prm.out) + ((size_t)s * prm.num_heads + h) * D;
-        out[tid] = from_float<T>(Ls > 0.f ? acc / Ls : 0.f);
-        __syncthreads();   // wsm / red / bcast are reused by the next pair
-    }
+    const int np = max(1, (len + P - 1) / P);
+    if (np == 1) return;
+    const int G = prm.group;
+    const int hk = h / G, g = h - hk * G;
+    const size_t row0 = (size_t)(prm.ws_seq_base[s] + hk * np) * G + g;   // partition 0
+    warp_merge<T, D>(reinterpret_cast<const float2 *>(prm.ws_ml) + row0, G,
+                     prm.ws_o + row0 * D, (size_t)G * D, np,
+                     reinterpret_cast<T *>(prm.out) + ((size_t)s * prm.num_heads + h) * D, lane);
 }
 
 }  // namespace pkv

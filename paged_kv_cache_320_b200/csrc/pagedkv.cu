@@ -247,12 +247,11 @@ int launch_decode(const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMa
 
 template <typename T, int D>
 int launch_reduce(const pkv::DecodeParams &prm, int pmax, cudaStream_t st) {
-    int nsm;
-    if (sm_count(&nsm) != PKV_OK) return PKV_ERR_CUDA;
-    long long grid = (long long)prm.num_seqs * prm.num_heads;
-    if (grid > 8LL * nsm) grid = 8LL * nsm;
-    return launch(pkv::paged_decode_reduce_kernel<T, D>, dim3((unsigned)grid), dim3(D),
-                  (size_t)pmax * sizeof(float), st, prm);
+    (void)pmax;
+    const long long pairs = (long long)prm.num_seqs * prm.num_heads;
+    const long long grid = (pairs + pkv::kReduceWarps - 1) / pkv::kReduceWarps;
+    return launch(pkv::paged_decode_reduce_kernel<T, D>, dim3((unsigned)grid),
+                  dim3(pkv::kReduceWarps * 32), 0, st, prm);
 }
 
 template <typename T, int D>
@@ -320,7 +319,23 @@ int launch_shared_decode(const CUtensorMap &mk, const CUtensorMap &mv,
 template <typename T, int D>
 int launch_shared_path(int BS, const CUtensorMap &mk, const CUtensorMap &mv,
                        const pkv::SharedParams &prm, cudaStream_t st) {
-    int rc = launch(pkv::shared_prefix_plan_kernel, dim3(1), dim3(pkv::kPlanThreads), 0, st, prm);
+    const size_t plan_smem =
+        prm.num_seqs <= pkv::kPlanSmemSeqs ? (size_t)6 * prm.num_seqs * sizeof(int) : 0;
+    {
+        int dev;
+        if (current_device(&dev) != PKV_OK) return PKV_ERR_CUDA;
+        static bool attr[kMaxDevices];
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!attr[dev]) {
+            if (cudaFuncSetAttribute(pkv::shared_prefix_plan_kernel,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     6 * pkv::kPlanSmemSeqs * (int)sizeof(int)) != cudaSuccess)
+                return PKV_ERR_CUDA;
+            attr[dev] = true;
+        }
+    }
+    int rc = launch(pkv::shared_prefix_plan_kernel, dim3(1), dim3(pkv::kPlanThreads), plan_smem,
+                    st, prm);
     if (rc != PKV_OK) return rc;
     switch (BS) {
         case 8: rc = launch_shared_decode<T, D, 8>(mk, mv, prm, st); break;
@@ -329,12 +344,10 @@ int launch_shared_path(int BS, const CUtensorMap &mk, const CUtensorMap &mv,
         default: return PKV_ERR_INVALID_ARG;
     }
     if (rc != PKV_OK) return rc;
-    int nsm;
-    if (sm_count(&nsm) != PKV_OK) return PKV_ERR_CUDA;
-    long long grid = (long long)prm.num_seqs * prm.num_heads;
-    if (grid > 8LL * nsm) grid = 8LL * nsm;
-    return launch(pkv::paged_decode_shared_reduce_kernel<T, D>, dim3((unsigned)grid), dim3(D), 0,
-                  st, prm);
+    const long long pairs = (long long)prm.num_seqs * prm.num_heads;
+    const long long grid = (pairs + pkv::kReduceWarps - 1) / pkv::kReduceWarps;
+    return launch(pkv::paged_decode_shared_reduce_kernel<T, D>, dim3((unsigned)grid),
+                  dim3(pkv::kReduceWarps * 32), 0, st, prm);
 }
 
 }  // namespace
@@ -628,6 +641,42 @@ int pkv_copy_blocks(void *const *k_caches, void *const *v_caches, int num_layers
     return launch(pkv::copy_blocks_kernel, grid, dim3(256), 0,
                   reinterpret_cast<cudaStream_t>(stream), k_caches, v_caches, block_pairs,
                   num_blocks, (int)vecs, status);
+}
+
+int pkv_swap_blocks(void *const *k_caches, void *const *v_caches, int num_layers,
+                    const int32_t *block_ids, int num_ids, void *host_buffer,
+                    size_t host_buffer_bytes, int to_host, int num_kv_heads, int head_dim,
+                    int block_size, int num_blocks, int dtype, pkv_stream_t stream) {
+    if (num_ids < 0 || num_layers < 1 || num_layers > 65535 || num_kv_heads < 1 ||
+        num_blocks < 1 || (to_host != 0 && to_host != 1))
+        return PKV_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return PKV_ERR_INVALID_ARG;
+    if (block_size != 8 && block_size != 16 && block_size != 32) return PKV_ERR_INVALID_ARG;
+    if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_ERR_INVALID_ARG;
+    if (num_ids == 0) return PKV_OK;
+    if (!k_caches || !v_caches || !block_ids || !host_buffer || !aligned(host_buffer, 16))
+        return PKV_ERR_INVALID_ARG;
+    const long long vecs = (long long)num_kv_heads * block_size * head_dim * 2 / 16;
+    if (vecs >= INT_MAX) return PKV_ERR_INVALID_ARG;
+    const unsigned long long need = (unsigned long long)num_layers * 2 * num_ids * vecs * 16;
+    if (host_buffer_bytes < need) return PKV_ERR_INVALID_ARG;
+    // the kernel reads / writes the buffer through unified addressing: it must be
+    // pinned host memory that this device can reach
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, host_buffer) != cudaSuccess) {
+        cudaGetLastError();
+        return PKV_ERR_INVALID_ARG;
+    }
+    if (attr.type != cudaMemoryTypeHost || attr.devicePointer != host_buffer)
+        return PKV_ERR_INVALID_ARG;
+    unsigned int *status;
+    int rc;
+    if ((rc = device_status_ptr(&status)) != PKV_OK) return rc;
+    dim3 grid((unsigned)num_ids, (unsigned)num_layers, 2);
+    return launch(pkv::swap_blocks_kernel, grid, dim3(256), 0,
+                  reinterpret_cast<cudaStream_t>(stream), k_caches, v_caches, block_ids,
+                  num_ids, static_cast<uint4 *>(host_buffer), num_blocks, (int)vecs, to_host,
+                  status);
 }
 
 int pkv_get_device_status(uint32_t *status_out, int clear, pkv_stream_t stream) {

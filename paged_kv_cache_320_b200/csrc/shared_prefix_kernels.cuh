@@ -4,7 +4,7 @@
 // physical prefix pages ("vLLM" entity page, 是什么; "vLLM / PagedAttention — 分页 KV
 // Cache 分析" §3.2). Plain decode streams such a page once per sequence. Here the
 // sequences of a group share the prefix: every prefix page of a KV head is streamed
-// ONCE for up to 16 query rows (the G heads of several member sequences on the MMA's
+// once for up to 16 query rows (the G heads of several member sequences on the MMA's
 // M dimension), each sequence's private suffix is streamed for its own G rows, and
 // the partial softmax states of the pieces are merged exactly (log-sum-exp). The
 // result is the same attention as plain decode:
@@ -96,6 +96,10 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *sm, int *total) 
     return before + x - v;
 }
 
+// Per-sequence scratch arrays of the plan kept in shared memory up to this batch size
+// (6 ints per sequence); larger batches use the workspace copies.
+constexpr int kPlanSmemSeqs = 8192;
+
 // One CTA builds the item list. Groups are contiguous runs of sequences; a malformed
 // group_start makes every sequence its own group (no sharing) and sets the length
 // status bit. A group's shared length is its declared prefix cut to a multiple of the
@@ -104,12 +108,21 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *sm, int *total) 
 __global__ void __launch_bounds__(kPlanThreads)
 shared_prefix_plan_kernel(SharedParams p) {
     pdl_wait_and_release();
+    extern __shared__ int plan_smem[];
     __shared__ int sm[kPlanThreads / 32];
     __shared__ int bad, max_pre_blocks;
     const int B = p.num_seqs, Hkv = p.num_kv_heads, G = p.group, P = p.partition;
     const int BS = p.block_size;
-    const int R = kMaxGroup / G;   // member sequences per 16-row tile
+    const int R = kMaxGroup / G;   // member sequences per 16-row prefix item
     const int tid = threadIdx.x;
+    // scratch: in shared memory when it fits (generic pointers address either space)
+    const bool in_smem = B <= kPlanSmemSeqs;
+    int *seq_group = in_smem ? plan_smem : p.seq_group;
+    int *gpre = in_smem ? plan_smem + B : p.gpre;
+    int *gmin = in_smem ? plan_smem + 2 * B : p.gmin;
+    int *gmis = in_smem ? plan_smem + 3 * B : p.gmis;
+    int *slen = in_smem ? plan_smem + 4 * B : p.np;          // clamped lengths
+    int *gfirst = in_smem ? plan_smem + 5 * B : p.row_base;  // first member of each group
     if (tid == 0) {
         bad = 0;
         max_pre_blocks = 0;
@@ -124,34 +137,48 @@ shared_prefix_plan_kernel(SharedParams p) {
     __syncthreads();
     if (tid == 0 && bad) atomicOr(p.status, kStatusBadLen);
     const int ng = bad ? B : p.num_groups;
-    // pass 0 (per group): membership, declared prefix, identities for the minima
+    // pass 0 (per group): membership, declared prefix, identities for the minima;
+    // (per sequence): clamped length
     for (int g = tid; g < ng; g += kPlanThreads) {
         const int first = bad ? g : p.group_start[g];
         const int last = bad ? g + 1 : p.group_start[g + 1];
         int pre = (bad || last - first < 2) ? 0 : p.prefix_lens[g];
         pre = pre < 0 ? 0 : pre - pre % BS;
-        p.gpre[g] = pre;
-        p.gmin[g] = 0x7fffffff;
-        p.gmis[g] = 0x7fffffff;
-        for (int s = first; s < last; ++s) p.seq_group[s] = g;
+        gpre[g] = pre;
+        gmin[g] = 0x7fffffff;
+        gmis[g] = 0x7fffffff;
+        gfirst[g] = first;
+        for (int s = first; s < last; ++s) seq_group[s] = g;
         atomicMax(&max_pre_blocks, pre / BS);
     }
+    for (int s = tid; s < B; s += kPlanThreads)
+        slen[s] = clamp_len(p.context_lens[s], p.max_context_len);
     __syncthreads();
     // pass 1 (per sequence): shortest member
-    for (int s = tid; s < B; s += kPlanThreads) {
-        const int g = __ldcg(&p.seq_group[s]);
-        atomicMin(&p.gmin[g], clamp_len(p.context_lens[s], p.max_context_len));
-    }
-    // pass 2 (per (sequence, prefix block)): first block where a member's table differs
-    const int mpb = max_pre_blocks;
-    for (long long i = tid; i < (long long)B * mpb; i += kPlanThreads) {
-        const int s = (int)(i / mpb), b = (int)(i - (long long)s * mpb);
-        const int g = __ldcg(&p.seq_group[s]);
-        const int first = bad ? g : p.group_start[g];
-        if (s == first || b >= __ldcg(&p.gpre[g]) / BS) continue;
-        const int mine = p.block_tables[(size_t)s * p.max_blocks_per_seq + b];
-        const int ref = p.block_tables[(size_t)first * p.max_blocks_per_seq + b];
-        if (mine != ref) atomicMin(&p.gmis[g], b);
+    for (int s = tid; s < B; s += kPlanThreads) atomicMin(&gmin[seq_group[s]], slen[s]);
+    // pass 2 (per (sequence, 8 prefix blocks)): first block where a member's table
+    // differs from the group's first member (independent loads, one atomic per chunk)
+    const int nch = (max_pre_blocks + 7) / 8;
+    for (long long i = tid; i < (long long)B * nch; i += kPlanThreads) {
+        const int s = (int)(i / nch), c = (int)(i - (long long)s * nch);
+        const int g = seq_group[s];
+        const int first = gfirst[g];
+        const int nb = gpre[g] / BS;
+        if (s == first || c * 8 >= nb) continue;
+        const int32_t *mine = p.block_tables + (size_t)s * p.max_blocks_per_seq;
+        const int32_t *ref = p.block_tables + (size_t)first * p.max_blocks_per_seq;
+        int a[8], r[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int b = c * 8 + k;
+            a[k] = b < nb ? mine[b] : 0;
+            r[k] = b < nb ? ref[b] : 0;
+        }
+        int mis = 0x7fffffff;
+#pragma unroll
+        for (int k = 7; k >= 0; --k)
+            if (a[k] != r[k]) mis = c * 8 + k;
+        if (mis != 0x7fffffff) atomicMin(&gmis[g], mis);
     }
     __syncthreads();
     // pass 3 (per group): shared length, prefix items
@@ -160,16 +187,16 @@ shared_prefix_plan_kernel(SharedParams p) {
         const int g = g0 + tid;
         int first = 0, last = 0, pre = 0, cnt = 0;
         if (g < ng) {
-            first = bad ? g : p.group_start[g];
+            first = gfirst[g];
             last = bad ? g + 1 : p.group_start[g + 1];
-            const int shortest = __ldcg(&p.gmin[g]);
-            pre = min(__ldcg(&p.gpre[g]), shortest - shortest % BS);
-            pre = min(pre, min(__ldcg(&p.gmis[g]), pre / BS) * BS);
-            p.gpre[g] = pre;
-            if (pre > 0) cnt = Hkv * ((last - first + R - 1) / R) * ((pre + P - 1) / P);
+            const int shortest = gmin[g];
+            pre = min(gpre[g], shortest - shortest % BS);
+            pre = min(pre, min(gmis[g], pre / BS) * BS);
         }
+        if (g < ng && pre > 0) cnt = Hkv * ((last - first + R - 1) / R) * ((pre + P - 1) / P);
         int total;
         int at = base_items + block_exclusive_scan(cnt, sm, &total);
+        if (g < ng) gpre[g] = pre;   // every reader of gpre[g] in this pass is done (scan barriers)
         if (cnt > 0) {
             const int npp = (pre + P - 1) / P;
             const int chunks = (last - first + R - 1) / R;
@@ -198,8 +225,8 @@ shared_prefix_plan_kernel(SharedParams p) {
         const int s = s0 + tid;
         int pre = 0, len = 0, npp = 0, nps = 0;
         if (s < B) {
-            pre = __ldcg(&p.gpre[__ldcg(&p.seq_group[s])]);
-            len = clamp_len(p.context_lens[s], p.max_context_len);
+            pre = gpre[seq_group[s]];
+            len = slen[s];
             npp = (pre + P - 1) / P;
             nps = max(1, (len - pre + P - 1) / P);
         }
@@ -432,8 +459,8 @@ paged_decode_shared_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const int valid = in.ntok - 16 * w;
         if (valid > 0) {
             const uint8_t *stage = ring + slot * L::kStageBytes;
-            consume_stage<T, D, BS>(st, smem_u32(stage), smem_u32(stage + L::kKBytes), w, lane,
-                                    valid, prm.scale_log2);
+            consume_stage<T, D, BS>(st, smem_u32(stage), smem_u32(stage + L::kKBytes), 16 * w,
+                                    lane, valid, prm.scale_log2);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&empty[slot]));
@@ -456,34 +483,22 @@ paged_decode_shared_kernel(const __grid_constant__ CUtensorMap tmap_k,
     }
 }
 
-// Merge of every (sequence, head)'s partials: rows row_base[s] + h*np[s] + j, j < np[s].
-//   M = max m_j;  w_j = l_j 2^(m_j - M);  out = sum w_j o_j / sum w_j
+// Merge of every (sequence, head)'s partials: rows row_base[s] + h*np[s] + j, j < np[s];
+// one warp per pair.
 template <typename T, int D>
-__global__ void __launch_bounds__(D)
+__global__ void __launch_bounds__(kReduceWarps * 32)
 paged_decode_shared_reduce_kernel(SharedParams prm) {
     pdl_wait_and_release();
-    const float2 *mlp = reinterpret_cast<const float2 *>(prm.ws_ml);
-    const int tid = threadIdx.x;
-    const int pairs = prm.num_seqs * prm.num_heads;
-    for (int pr = blockIdx.x; pr < pairs; pr += gridDim.x) {
-        const int s = pr / prm.num_heads;
-        const int h = pr - s * prm.num_heads;
-        const int np = prm.np[s];
-        const size_t row0 = (size_t)prm.row_base[s] + (size_t)h * np;
-        float M = -INFINITY;
-        for (int j = 0; j < np; ++j) M = fmaxf(M, mlp[row0 + j].x);
-        float Lsum = 0.f, acc = 0.f;
-        if (M != -INFINITY) {
-            for (int j = 0; j < np; ++j) {
-                const float2 v = mlp[row0 + j];
-                const float wv = v.y * ex2(v.x - M);
-                Lsum += wv;
-                acc += wv * prm.ws_o[(row0 + j) * D + tid];
-            }
-        }
-        T *out = reinterpret_cast<T *>(prm.out) + ((size_t)s * prm.num_heads + h) * D;
-        out[tid] = from_float<T>(Lsum > 0.f ? acc / Lsum : 0.f);
-    }
+    const int lane = threadIdx.x & 31;
+    const int pair = blockIdx.x * kReduceWarps + (threadIdx.x >> 5);
+    if (pair >= prm.num_seqs * prm.num_heads) return;
+    const int s = pair / prm.num_heads;
+    const int h = pair - s * prm.num_heads;
+    const int np = prm.np[s];
+    const size_t row0 = (size_t)prm.row_base[s] + (size_t)h * np;
+    warp_merge<T, D>(reinterpret_cast<const float2 *>(prm.ws_ml) + row0, 1,
+                     prm.ws_o + row0 * D, D, np,
+                     reinterpret_cast<T *>(prm.out) + ((size_t)s * prm.num_heads + h) * D, lane);
 }
 
 }  // namespace pkv

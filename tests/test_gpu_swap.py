@@ -1,0 +1,75 @@
+"""GPU parity of pkv_swap_blocks (whole blocks of every layer between the caches and
+pinned host memory) against the oracle: bit-exact, untouched blocks unchanged, bad
+ids reported, buffers that are not pinned host memory rejected before any launch."""
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_cache_320_b200 as pkv
+from oracle import cache_ops as C
+from paged_kv_cache_320_b200 import synth
+from tests.gpu_util import to_bits, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def setup(rng, L, NB, Hkv, BS, D, dtype):
+    kcs = [rng.integers(0, 1 << 16, (NB, Hkv, BS, D), dtype=np.uint16) for _ in range(L)]
+    vcs = [rng.integers(0, 1 << 16, (NB, Hkv, BS, D), dtype=np.uint16) for _ in range(L)]
+    kd = [to_dev(c, dtype) for c in kcs]
+    vd = [to_dev(c, dtype) for c in vcs]
+    kp = torch.tensor([t.data_ptr() for t in kd], dtype=torch.int64, device="cuda")
+    vp = torch.tensor([t.data_ptr() for t in vd], dtype=torch.int64, device="cuda")
+    return kcs, vcs, kd, vd, kp, vp
+
+
+@pytest.mark.parametrize("L,D,BS", [(1, 128, 16), (3, 128, 8), (2, 64, 32)])
+def test_swap_out_and_in_bit_exact(cuda_device, L, D, BS):
+    rng = np.random.default_rng(80 + L + D + BS)
+    NB, Hkv, dtype = 40, 8, synth.BF16
+    kcs, vcs, kd, vd, kp, vp = setup(rng, L, NB, Hkv, BS, D, dtype)
+    out_ids = np.array(rng.choice(NB, size=13, replace=False), np.int32)
+    buf = torch.empty((L, 2, 13, Hkv, BS, D), dtype=torch.int16).pin_memory()
+    pkv.pkv_swap_blocks(kp, vp, torch.from_numpy(out_ids).cuda(), buf, 1, Hkv, D, BS, NB,
+                        pkv.PKV_BF16)
+    torch.cuda.synchronize()
+    expect = C.swap_out(kcs, vcs, out_ids)
+    np.testing.assert_array_equal(buf.numpy().view(np.uint16), expect)
+    # swap back into other blocks of the same pool
+    in_ids = np.array([b for b in range(NB) if b not in out_ids][:13], np.int32)
+    pkv.pkv_swap_blocks(kp, vp, torch.from_numpy(in_ids).cuda(), buf, 0, Hkv, D, BS, NB,
+                        pkv.PKV_BF16)
+    torch.cuda.synchronize()
+    ek, ev = C.swap_in(kcs, vcs, in_ids, expect)
+    for layer in range(L):
+        np.testing.assert_array_equal(to_bits(kd[layer]), ek[layer])
+        np.testing.assert_array_equal(to_bits(vd[layer]), ev[layer])
+    assert pkv.pkv_get_device_status() == 0
+
+
+def test_swap_rejects_buffers_that_are_not_pinned_host_memory(cuda_device):
+    rng = np.random.default_rng(81)
+    NB, Hkv, BS, D = 8, 2, 16, 64
+    kcs, vcs, kd, vd, kp, vp = setup(rng, 1, NB, Hkv, BS, D, synth.F16)
+    ids = torch.tensor([1, 2], dtype=torch.int32, device="cuda")
+    for buf in (torch.empty((1, 2, 2, Hkv, BS, D), dtype=torch.int16),            # pageable
+                torch.empty((1, 2, 2, Hkv, BS, D), dtype=torch.int16, device="cuda"),  # device
+                torch.empty((1, 2, 1, Hkv, BS, D), dtype=torch.int16).pin_memory()):   # small
+        with pytest.raises(pkv.PagedKVError) as e:
+            pkv.pkv_swap_blocks(kp, vp, ids, buf, 1, Hkv, D, BS, NB, pkv.PKV_F16)
+        assert e.value.code == pkv._binding.PKV_ERR_INVALID_ARG
+
+
+def test_swap_bad_id_skipped_and_reported(cuda_device):
+    rng = np.random.default_rng(82)
+    NB, Hkv, BS, D = 8, 2, 16, 64
+    kcs, vcs, kd, vd, kp, vp = setup(rng, 1, NB, Hkv, BS, D, synth.F16)
+    buf = torch.zeros((1, 2, 3, Hkv, BS, D), dtype=torch.int16).pin_memory()
+    pkv.pkv_get_device_status(clear=True)
+    pkv.pkv_swap_blocks(kp, vp, torch.tensor([2, NB + 5, 4], dtype=torch.int32, device="cuda"),
+                        buf, 1, Hkv, D, BS, NB, pkv.PKV_F16)
+    assert pkv.pkv_get_device_status(clear=True) & pkv._binding.STATUS_BAD_PAIR
+    b = buf.numpy().view(np.uint16)
+    np.testing.assert_array_equal(b[0, 0, 0], kcs[0][2])
+    np.testing.assert_array_equal(b[0, 0, 2], kcs[0][4])
+    assert (b[0, :, 1] == 0).all()

@@ -50,3 +50,25 @@ def test_copy_blocks_every_layer_and_nothing_else():
         others = [b for b in range(NB) if b not in pairs[:, 1]]
         np.testing.assert_array_equal(k2[layer][others], kcs[layer][others])
         np.testing.assert_array_equal(v2[layer][others], vcs[layer][others])
+
+
+def test_swap_round_trip_is_a_block_copy():
+    """swap_out then swap_in to other ids equals copy_blocks of the same pairs; the
+    buffer holds each layer's pages in list order; other blocks are untouched."""
+    rng = np.random.default_rng(32)
+    L, NB, Hkv, bs, d = 2, 12, 2, 8, 16
+    kcs = [rng.integers(0, 1 << 16, (NB, Hkv, bs, d), dtype=np.uint16) for _ in range(L)]
+    vcs = [rng.integers(0, 1 << 16, (NB, Hkv, bs, d), dtype=np.uint16) for _ in range(L)]
+    src = np.array([3, 7, 0], np.int32)
+    dst = np.array([9, 1, 11], np.int32)
+    buf = cache_ops.swap_out(kcs, vcs, src)
+    assert buf.shape == (L, 2, 3, Hkv, bs, d)
+    for layer in range(L):
+        for i, b in enumerate(src):
+            assert buf[layer, 0, i].tobytes() == kcs[layer][b].tobytes()
+            assert buf[layer, 1, i].tobytes() == vcs[layer][b].tobytes()
+    k2, v2 = cache_ops.swap_in(kcs, vcs, dst, buf)
+    k3, v3 = cache_ops.copy_blocks(kcs, vcs, np.stack([src, dst], 1))
+    for layer in range(L):
+        np.testing.assert_array_equal(k2[layer], k3[layer])
+        np.testing.assert_array_equal(v2[layer], v3[layer])
