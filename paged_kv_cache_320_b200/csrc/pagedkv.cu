@@ -266,7 +266,7 @@ int dispatch_bs(int BS, const CUtensorMap &mk, const CUtensorMap &mv, const CUte
 }
 
 // ---- shared-prefix decode ------------------------------------------------
-// Workspace: [counters 256 B][np, row_base, seq_group, gpre, gmin, gmis: B ints each]
+// Workspace: [counters 256 B][np, row_base, seq_group, gpre, gmin, gmis, ioff: B ints each]
 // [items][partials (max, sum)][partial outputs].
 struct SharedWs {
     size_t ints, items, ml, o, total;
@@ -280,7 +280,7 @@ SharedWs shared_ws_layout(int B, int Hq, int Hkv, int D, int max_len, int P) {
     w.max_items = (int)std::min<long long>(2LL * Hkv * B * pmax, INT_MAX / 2);
     w.rows = (long long)B * Hq * (pmax + 1);
     w.ints = sizeof(pkv::SharedCounters);
-    w.items = w.ints + 6 * align_up((size_t)B * sizeof(int), 256);
+    w.items = w.ints + 7 * align_up((size_t)B * sizeof(int), 256);
     w.ml = w.items + align_up((size_t)w.max_items * sizeof(pkv::SharedItem), 256);
     w.o = w.ml + align_up((size_t)w.rows * 2 * sizeof(float), 256);
     w.total = w.o + (size_t)w.rows * D * sizeof(float);
@@ -320,7 +320,7 @@ template <typename T, int D>
 int launch_shared_path(int BS, const CUtensorMap &mk, const CUtensorMap &mv,
                        const pkv::SharedParams &prm, cudaStream_t st) {
     const size_t plan_smem =
-        prm.num_seqs <= pkv::kPlanSmemSeqs ? (size_t)6 * prm.num_seqs * sizeof(int) : 0;
+        prm.num_seqs <= pkv::kPlanSmemSeqs ? (size_t)7 * prm.num_seqs * sizeof(int) : 0;
     {
         int dev;
         if (current_device(&dev) != PKV_OK) return PKV_ERR_CUDA;
@@ -329,7 +329,7 @@ int launch_shared_path(int BS, const CUtensorMap &mk, const CUtensorMap &mv,
         if (!attr[dev]) {
             if (cudaFuncSetAttribute(pkv::shared_prefix_plan_kernel,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     6 * pkv::kPlanSmemSeqs * (int)sizeof(int)) != cudaSuccess)
+                                     7 * pkv::kPlanSmemSeqs * (int)sizeof(int)) != cudaSuccess)
                 return PKV_ERR_CUDA;
             attr[dev] = true;
         }
@@ -556,6 +556,7 @@ int pkv_paged_attention_decode_shared_prefix(
     prm.gpre = reinterpret_cast<int *>(wsb + ws.ints + 3 * ib);
     prm.gmin = reinterpret_cast<int *>(wsb + ws.ints + 4 * ib);
     prm.gmis = reinterpret_cast<int *>(wsb + ws.ints + 5 * ib);
+    prm.ioff = reinterpret_cast<int *>(wsb + ws.ints + 6 * ib);
     prm.items = reinterpret_cast<pkv::SharedItem *>(wsb + ws.items);
     prm.ws_ml = reinterpret_cast<float *>(wsb + ws.ml);
     prm.ws_o = reinterpret_cast<float *>(wsb + ws.o);

@@ -48,6 +48,7 @@ struct SharedParams {
     int *gpre;         // [B] shared tokens per group (plan scratch)
     int *gmin;         // [B] shortest member per group (plan scratch)
     int *gmis;         // [B] first logical block where a member's table differs (plan scratch)
+    int *ioff;         // [B] first suffix item of each sequence (plan scratch)
     float *ws_o;       // [rows][D]
     float *ws_ml;      // [rows][2]
     void *out;
@@ -97,8 +98,18 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *sm, int *total) 
 }
 
 // Per-sequence scratch arrays of the plan kept in shared memory up to this batch size
-// (6 ints per sequence); larger batches use the workspace copies.
-constexpr int kPlanSmemSeqs = 8192;
+// (7 ints per sequence); larger batches use the workspace copies.
+constexpr int kPlanSmemSeqs = 6144;
+
+// Largest i in [0, n) with off[i] <= x (off ascending, off[0] = 0).
+__device__ __forceinline__ int owner_of(const int *off, int n, int x) {
+    int lo = 0, hi = n - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (off[mid] <= x) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
 
 // One CTA builds the item list. Groups are contiguous runs of sequences; a malformed
 // group_start makes every sequence its own group (no sharing) and sets the length
@@ -123,6 +134,7 @@ shared_prefix_plan_kernel(SharedParams p) {
     int *gmis = in_smem ? plan_smem + 3 * B : p.gmis;
     int *slen = in_smem ? plan_smem + 4 * B : p.np;          // clamped lengths
     int *gfirst = in_smem ? plan_smem + 5 * B : p.row_base;  // first member of each group
+    int *ioff = in_smem ? plan_smem + 6 * B : p.ioff;        // suffix-item offsets
     if (tid == 0) {
         bad = 0;
         max_pre_blocks = 0;
@@ -181,79 +193,103 @@ shared_prefix_plan_kernel(SharedParams p) {
         if (mis != 0x7fffffff) atomicMin(&gmis[g], mis);
     }
     __syncthreads();
-    // pass 3 (per group): shared length, prefix items
+    // pass 3 (per group): shared length and prefix-item offsets
     int base_items = 0;
     for (int g0 = 0; g0 < ng; g0 += kPlanThreads) {
         const int g = g0 + tid;
-        int first = 0, last = 0, pre = 0, cnt = 0;
+        int pre = 0, cnt = 0;
         if (g < ng) {
-            first = gfirst[g];
-            last = bad ? g + 1 : p.group_start[g + 1];
+            const int first = gfirst[g];
+            const int last = bad ? g + 1 : p.group_start[g + 1];
             const int shortest = gmin[g];
             pre = min(gpre[g], shortest - shortest % BS);
             pre = min(pre, min(gmis[g], pre / BS) * BS);
+            if (pre > 0) cnt = Hkv * ((last - first + R - 1) / R) * ((pre + P - 1) / P);
         }
-        if (g < ng && pre > 0) cnt = Hkv * ((last - first + R - 1) / R) * ((pre + P - 1) / P);
         int total;
-        int at = base_items + block_exclusive_scan(cnt, sm, &total);
-        if (g < ng) gpre[g] = pre;   // every reader of gpre[g] in this pass is done (scan barriers)
-        if (cnt > 0) {
-            const int npp = (pre + P - 1) / P;
-            const int chunks = (last - first + R - 1) / R;
-            for (int hk = 0; hk < Hkv; ++hk)
-                for (int c = 0; c < chunks; ++c)
-                    for (int j = 0; j < npp; ++j, ++at) {
-                        if (at >= p.max_items) continue;
-                        SharedItem it;
-                        it.table_seq = first;
-                        it.tok0 = j * P;
-                        it.ntok = min(P, pre - j * P);
-                        it.hk = hk;
-                        it.first_seq = first + c * R;
-                        it.nseq = min(R, last - (first + c * R));
-                        it.part = j;
-                        it.pad = 0;
-                        p.items[at] = it;
-                    }
+        const int at = base_items + block_exclusive_scan(cnt, sm, &total);
+        if (g < ng) {
+            gpre[g] = pre;   // only thread g reads gpre[g] in this pass
+            gmin[g] = at;    // first prefix item of group g
         }
         base_items += total;
     }
+    const int n_prefix = base_items;
     __syncthreads();
-    // pass 4 (per sequence): suffix items, partial counts and scratch rows
+    // pass 3b (per prefix item): item i belongs to the group g with gmin[g] <= i
+    for (int i = tid; i < n_prefix && i < p.max_items; i += kPlanThreads) {
+        const int g = owner_of(gmin, ng, i);
+        const int first = gfirst[g];
+        const int last = bad ? g + 1 : p.group_start[g + 1];
+        const int pre = gpre[g];
+        const int npp = (pre + P - 1) / P;
+        const int chunks = (last - first + R - 1) / R;
+        int local = i - gmin[g];
+        const int j = local % npp;
+        local /= npp;
+        const int c = local % chunks;
+        const int hk = local / chunks;
+        SharedItem it;
+        it.table_seq = first;
+        it.tok0 = j * P;
+        it.ntok = min(P, pre - j * P);
+        it.hk = hk;
+        it.first_seq = first + c * R;
+        it.nseq = min(R, last - (first + c * R));
+        it.part = j;
+        it.pad = 0;
+        p.items[i] = it;
+    }
+    __syncthreads();
+    // pass 4 (per sequence): partial counts, scratch rows, suffix-item offsets
     int base_rows = 0;
     for (int s0 = 0; s0 < B; s0 += kPlanThreads) {
         const int s = s0 + tid;
-        int pre = 0, len = 0, npp = 0, nps = 0;
+        int pre = 0, npp = 0, nps = 0;
         if (s < B) {
             pre = gpre[seq_group[s]];
-            len = slen[s];
             npp = (pre + P - 1) / P;
-            nps = max(1, (len - pre + P - 1) / P);
+            nps = max(1, (slen[s] - pre + P - 1) / P);
         }
         int total_items, total_rows;
-        int at = base_items + block_exclusive_scan(s < B ? Hkv * nps : 0, sm, &total_items);
+        const int at = base_items + block_exclusive_scan(s < B ? Hkv * nps : 0, sm, &total_items);
         const int row =
             base_rows + block_exclusive_scan(s < B ? (npp + nps) : 0, sm, &total_rows);
         if (s < B) {
-            p.np[s] = npp + nps;
+            ioff[s] = at - n_prefix;   // first suffix item of s (relative)
             p.row_base[s] = row * p.num_heads;
-            for (int hk = 0; hk < Hkv; ++hk)
-                for (int j = 0; j < nps; ++j, ++at) {
-                    if (at >= p.max_items) continue;
-                    SharedItem it;
-                    it.table_seq = s;
-                    it.tok0 = pre + j * P;
-                    it.ntok = max(0, min(P, len - pre - j * P));
-                    it.hk = hk;
-                    it.first_seq = s;
-                    it.nseq = 1;
-                    it.part = npp + j;
-                    it.pad = 0;
-                    p.items[at] = it;
-                }
         }
         base_items += total_items;
         base_rows += total_rows;
+    }
+    __syncthreads();
+    // pass 4b (per suffix item)
+    for (int i = tid; i < base_items - n_prefix && n_prefix + i < p.max_items;
+         i += kPlanThreads) {
+        const int s = owner_of(ioff, B, i);
+        const int pre = gpre[seq_group[s]];
+        const int npp = (pre + P - 1) / P;
+        const int len = slen[s];
+        const int nps = max(1, (len - pre + P - 1) / P);
+        const int local = i - ioff[s];
+        const int hk = local / nps, j = local - hk * nps;
+        SharedItem it;
+        it.table_seq = s;
+        it.tok0 = pre + j * P;
+        it.ntok = max(0, min(P, len - pre - j * P));
+        it.hk = hk;
+        it.first_seq = s;
+        it.nseq = 1;
+        it.part = npp + j;
+        it.pad = 0;
+        p.items[n_prefix + i] = it;
+    }
+    // partial counts last: np aliases the length scratch when it lives in the workspace
+    __syncthreads();
+    for (int s = tid; s < B; s += kPlanThreads) {
+        const int pre = gpre[seq_group[s]];
+        const int npp = (pre + P - 1) / P;
+        p.np[s] = npp + max(1, (slen[s] - pre + P - 1) / P);
     }
     if (tid == 0) {
         if (base_items > p.max_items) atomicOr(p.status, kStatusBadLen);

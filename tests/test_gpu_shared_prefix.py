@@ -141,3 +141,19 @@ def test_shared_prefix_workload_full_size(cuda_device):
     # both GPU paths approximate the same fp64 result: compare them on every sequence
     a, b = A.bits_to_f64(got_s, dt), A.bits_to_f64(got_p, dt)
     assert np.all(np.abs(a - b) <= 2 * (4e-3 + 1e-2 * np.abs(b)))
+
+
+def test_large_batch_plans_in_workspace_scratch(cuda_device):
+    """6400 short sequences in groups of 4: the plan's per-sequence scratch no longer
+    fits in shared memory and lives in the workspace."""
+    rng = np.random.default_rng(62)
+    dtype = synth.BF16
+    ngroups = 1600
+    q, kc, vc, bt, lens, starts, pre, max_len = grouped_case(
+        rng, [4] * ngroups, list(rng.integers(0, 3, ngroups)), 20, 8, 2, 64, 16, dtype)
+    assert len(lens) > 6144
+    ref = A.paged_decode_attention(q, kc, vc, bt, lens, 0.125, dtype)
+    pkv.pkv_get_device_status(clear=True)
+    got = run_shared(q, kc, vc, bt, lens, starts, pre, max_len, dtype, 0.125)
+    assert pkv.pkv_get_device_status() == 0
+    assert_close(got, ref, dtype, "6400 sequences")
