@@ -277,6 +277,43 @@ int pkv_seq_append_batch(pkv_alloc *a, const int64_t *seq_ids, int n, int n_toke
 
 /* Errors: PKV_ERR_UNKNOWN_SEQ (no parent), PKV_ERR_SEQ_EXISTS (child id in use). */
 int pkv_seq_fork(pkv_alloc *a, int64_t parent, int64_t child);
+
+/* ------------------------------------------------------------------------------
+ * Prefix caching ("分页 KV Cache 分析" §2.3 and §3.2: common prefixes such as a system
+ * prompt or few-shot examples are found automatically and their pages reused across
+ * requests; 五: only exactly identical token sequences share). Off by default; with it
+ * off every call below behaves as if no block were ever cached.
+ *
+ * Readings (the pages fix no mechanism):
+ *  - only full blocks are cached. A full block is identified by a 64-bit hash chained over
+ *    all tokens up to its end (splitmix64 applied token by token, starting from the hash
+ *    of the blocks before it, 0 for the first block); a match also compares the block's
+ *    own tokens and its parent hash exactly.
+ *  - a block becomes cached when a sequence whose every token came with its id (created
+ *    by pkv_seq_append_tokens or pkv_seq_share_prefix) fills it, unless an identical block
+ *    is already cached. Appending without ids stops that sequence from caching.
+ *  - a cached block nobody holds is kept (evictable) instead of freed; allocation takes a
+ *    free block first and otherwise reclaims the least recently released cached block.
+ *    Evictable blocks count as free in pkv_stats.
+ * ---------------------------------------------------------------------------- */
+int pkv_alloc_set_prefix_cache(pkv_alloc *a, int enable);
+
+/* pkv_seq_append with the appended tokens' ids (host int32 [n_tokens]). */
+int pkv_seq_append_tokens(pkv_alloc *a, int64_t seq_id, const int32_t *tokens, int n_tokens,
+                          int64_t *slots_out, int32_t *cow_pairs_out, int *n_cow_out);
+
+/* Creates sequence seq_id holding the longest cached run of full blocks that matches
+ * tokens[0..n_tokens) (one more reference each); *n_cached_out = tokens covered (a
+ * multiple of block_size, 0 when the cache is off or nothing matches). The caller then
+ * appends the remaining tokens with pkv_seq_append_tokens (to keep one token uncached,
+ * pass n_tokens - 1). Errors: PKV_ERR_SEQ_EXISTS. */
+int pkv_seq_share_prefix(pkv_alloc *a, int64_t seq_id, const int32_t *tokens, int n_tokens,
+                         int *n_cached_out);
+
+/* Blocks in the cache, of which evictable; tokens queried by pkv_seq_share_prefix and
+ * tokens it found cached. Any output pointer may be NULL. */
+int pkv_prefix_cache_stats(const pkv_alloc *a, int *cached_blocks, int *evictable_blocks,
+                           int64_t *query_tokens, int64_t *hit_tokens);
 /* Errors: PKV_ERR_UNKNOWN_SEQ. */
 int pkv_seq_free(pkv_alloc *a, int64_t seq_id);
 

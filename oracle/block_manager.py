@@ -27,8 +27,53 @@ The pages fix no order, so these are readings (identical in the C++ allocator):
   drops one reference each, and pushes a block whose count reaches 0.
 * When n sequences share a partial block, the first n-1 writers copy and the
   last writes in place (its count is 1 by then); the order is the call order.
+
+Prefix caching ("vLLM / PagedAttention — 分页 KV Cache 分析" §2.3 and §3.2: common
+prefixes such as system prompts are detected automatically and their pages reused
+across requests; §五: only an exactly identical token sequence may share). The pages
+give no mechanism; readings (the same in the C++ allocator):
+* Only full blocks are cached. Block j of a token list is identified by the 64-bit
+  hash of the whole prefix ``tokens[: (j+1)*bs]``: start at 0 and fold every token
+  in with ``h = splitmix64(h ^ token)``; a hit also requires the cached block's
+  prefix to equal the query's exactly.
+* A sequence takes part while every token it holds came with its id (created by
+  ``append_tokens`` or ``share_prefix`` with the cache on); an ``append`` without
+  ids stops it. When such a sequence fills a block whose prefix is not cached yet,
+  that block becomes cached.
+* A cached block whose count falls to 0 is kept (evictable), most recently released
+  last. A new block comes from the free stack first, else the least recently
+  released evictable block leaves the cache and is reused. Evictable blocks count
+  as free.
+* ``share_prefix(seq, tokens)`` creates ``seq`` on the longest run of cached full
+  blocks matching ``tokens`` from the start (at most ``max_blocks_per_seq``), one
+  reference more each, and reports the tokens covered.
+* Turning the cache off forgets every entry; evictable blocks go to the free stack
+  (in release order) and no sequence takes part any more.
 """
 from __future__ import annotations
+
+from collections import OrderedDict
+
+_MASK64 = (1 << 64) - 1
+
+
+def splitmix64(x):
+    """One step of splitmix64 (Steele, Lea and Flood, "Fast splittable pseudorandom
+    number generators", OOPSLA 2014): add the golden-ratio increment, then the
+    variant-13 finaliser. Seeded with 0, the generator's outputs are
+    splitmix64(0), splitmix64(gamma), ..."""
+    z = (x + 0x9E3779B97F4A7C15) & _MASK64
+    z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & _MASK64
+    z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & _MASK64
+    return z ^ (z >> 31)
+
+
+def prefix_hash(tokens):
+    """Hash of a whole token prefix (token ids as unsigned 32-bit values)."""
+    h = 0
+    for t in tokens:
+        h = splitmix64(h ^ (int(t) & 0xFFFFFFFF))
+    return h
 
 # status codes of the block-manager interface (same numeric values as the library)
 OK = 0
@@ -53,12 +98,53 @@ class BlockManagerModel:
         self.refcount = [0] * num_blocks
         self.tables = {}                            # seq id -> list of block ids
         self.lens = {}                              # seq id -> tokens
+        # prefix cache
+        self.prefix_cache = False
+        self.cache = {}                             # hash -> (prefix tuple, block)
+        self.block_hash = {}                        # cached block -> its hash
+        self.evictable = OrderedDict()              # block -> None, oldest release first
+        self.ids = {}                               # taking-part seq -> its token ids
+        self.query_tokens = 0
+        self.hit_tokens = 0
 
     # -- helpers -----------------------------------------------------------
     def _pop(self):
-        b = self.free_stack.pop()
+        if self.free_stack:
+            b = self.free_stack.pop()
+        else:
+            b, _ = self.evictable.popitem(last=False)
+            del self.cache[self.block_hash.pop(b)]
         self.refcount[b] = 1
         return b
+
+    def _unref(self, b):
+        self.refcount[b] -= 1
+        if self.refcount[b] == 0:
+            if b in self.block_hash:
+                self.evictable[b] = None
+            else:
+                self.free_stack.append(b)
+
+    def available(self):
+        return len(self.free_stack) + len(self.evictable)
+
+    def _placed(self, seq, token):
+        """Token `token` (None: no id) was just placed at position lens[seq]-1."""
+        if seq not in self.ids:
+            return
+        if token is None:
+            del self.ids[seq]
+            return
+        ids = self.ids[seq]
+        ids.append(int(token))
+        n = len(ids)
+        if n % self.bs:
+            return
+        h = prefix_hash(ids)
+        if h not in self.cache:
+            b = self.tables[seq][n // self.bs - 1]
+            self.cache[h] = (tuple(ids), b)
+            self.block_hash[b] = h
 
     def blocks_needed(self, seq, n_tokens):
         n = self.lens.get(seq, 0)
@@ -70,19 +156,21 @@ class BlockManagerModel:
         return need + new, -(-(n + n_tokens) // self.bs)
 
     # -- interface -----------------------------------------------------------
-    def append(self, seq, n_tokens):
-        """Returns (status, slots, cow_pairs)."""
+    def append(self, seq, n_tokens, token_ids=None):
+        """Returns (status, slots, cow_pairs). ``token_ids``: the appended tokens' ids."""
         if n_tokens < 0:
             return ERR_INVALID_ARG, [], []
         need, table_len = self.blocks_needed(seq, n_tokens)
         if table_len > self.mb:
             return ERR_TABLE_FULL, [], []
-        if need > len(self.free_stack):
+        if need > self.available():
             return ERR_OUT_OF_BLOCKS, [], []
+        if seq not in self.tables and self.prefix_cache and token_ids is not None:
+            self.ids[seq] = []
         table = self.tables.setdefault(seq, [])
         self.lens.setdefault(seq, 0)
         slots, cows = [], []
-        for _ in range(n_tokens):
+        for i in range(n_tokens):
             n = self.lens[seq]
             if n % self.bs == 0:
                 table.append(self._pop())
@@ -94,7 +182,51 @@ class BlockManagerModel:
                 table[-1] = new
             slots.append(table[n // self.bs] * self.bs + n % self.bs)
             self.lens[seq] = n + 1
+            self._placed(seq, None if token_ids is None else token_ids[i])
         return OK, slots, cows
+
+    def append_tokens(self, seq, token_ids):
+        return self.append(seq, len(token_ids), list(token_ids))
+
+    def set_prefix_cache(self, enable):
+        if self.prefix_cache and not enable:
+            for b in self.evictable:
+                self.free_stack.append(b)
+            self.evictable.clear()
+            self.cache.clear()
+            self.block_hash.clear()
+            self.ids.clear()
+        self.prefix_cache = bool(enable)
+        return OK
+
+    def share_prefix(self, seq, token_ids):
+        """Returns (status, tokens covered)."""
+        if seq in self.tables:
+            return ERR_SEQ_EXISTS, 0
+        toks = [int(t) for t in token_ids]
+        table = []
+        if self.prefix_cache:
+            j = 0
+            while (j + 1) * self.bs <= len(toks) and j < self.mb:
+                pre = tuple(toks[: (j + 1) * self.bs])
+                hit = self.cache.get(prefix_hash(pre))
+                if hit is None or hit[0] != pre:
+                    break
+                b = hit[1]
+                if self.refcount[b] == 0:
+                    del self.evictable[b]
+                self.refcount[b] += 1
+                table.append(b)
+                j += 1
+            self.query_tokens += len(toks)
+            self.hit_tokens += len(table) * self.bs
+            self.ids[seq] = toks[: len(table) * self.bs]
+        self.tables[seq] = table
+        self.lens[seq] = len(table) * self.bs
+        return OK, self.lens[seq]
+
+    def prefix_cache_stats(self):
+        return len(self.cache), len(self.evictable), self.query_tokens, self.hit_tokens
 
     def fork(self, parent, child):
         if parent not in self.tables:
@@ -103,6 +235,8 @@ class BlockManagerModel:
             return ERR_SEQ_EXISTS
         self.tables[child] = list(self.tables[parent])
         self.lens[child] = self.lens[parent]
+        if parent in self.ids:
+            self.ids[child] = list(self.ids[parent])
         for b in self.tables[child]:
             self.refcount[b] += 1
         return OK
@@ -111,11 +245,10 @@ class BlockManagerModel:
         if seq not in self.tables:
             return ERR_UNKNOWN_SEQ
         for b in reversed(self.tables[seq]):
-            self.refcount[b] -= 1
-            if self.refcount[b] == 0:
-                self.free_stack.append(b)
+            self._unref(b)
         del self.tables[seq]
         del self.lens[seq]
+        self.ids.pop(seq, None)
         return OK
 
     def block_table(self, seq):
@@ -123,7 +256,7 @@ class BlockManagerModel:
         return row, self.lens[seq]
 
     def stats(self):
-        free = len(self.free_stack)
+        free = self.available()
         held = self.nb - free
         tokens = sum(self.lens.values())
         util = tokens / (held * self.bs) if held else 0.0

@@ -79,6 +79,12 @@ def lib() -> ctypes.CDLL:
         L.pkv_block_tables.argtypes = [P, P, I, P, P]
         L.pkv_stats.argtypes = [P, ctypes.POINTER(I), ctypes.POINTER(I),
                                 ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_double)]
+        L.pkv_alloc_set_prefix_cache.argtypes = [P, I]
+        L.pkv_seq_append_tokens.argtypes = [P, I64, P, I, P, P, ctypes.POINTER(I)]
+        L.pkv_seq_share_prefix.argtypes = [P, I64, P, I, ctypes.POINTER(I)]
+        L.pkv_prefix_cache_stats.argtypes = [P, ctypes.POINTER(I), ctypes.POINTER(I),
+                                             ctypes.POINTER(ctypes.c_int64),
+                                             ctypes.POINTER(ctypes.c_int64)]
         for name in ("pkv_paged_attention_decode", "pkv_paged_attention_decode_noalloc",
                      "pkv_paged_attention_decode_shared_prefix",
                      "pkv_decode_shared_prefix_workspace_size", "pkv_decode_workspace_size",
@@ -86,8 +92,8 @@ def lib() -> ctypes.CDLL:
                      "pkv_swap_blocks",
                      "pkv_get_device_status", "pkv_alloc_create", "pkv_alloc_destroy",
                      "pkv_seq_append", "pkv_seq_append_batch", "pkv_seq_fork", "pkv_seq_free",
-                     "pkv_block_tables",
-                     "pkv_stats"):
+                     "pkv_block_tables", "pkv_stats", "pkv_alloc_set_prefix_cache",
+                     "pkv_seq_append_tokens", "pkv_seq_share_prefix", "pkv_prefix_cache_stats"):
             getattr(L, name).restype = I
         _lib = L
     return _lib
@@ -318,6 +324,44 @@ class BlockManager:
                                         slots.ctypes.data, cows.ctypes.data,
                                         ctypes.byref(n_cow), ctypes.byref(n_done))
         return rc, n_done.value, slots[:n, :n_tokens], cows[:n_cow.value]
+
+    def pkv_alloc_set_prefix_cache(self, enable):
+        return lib().pkv_alloc_set_prefix_cache(self._h, int(bool(enable)))
+
+    def pkv_seq_append_tokens(self, seq_id, tokens):
+        """Append with token ids (int32); returns (status, slots, cow pairs [k, 2])."""
+        import numpy as np
+        tok = np.ascontiguousarray(tokens, dtype=np.int32).reshape(-1)
+        n = tok.shape[0]
+        slots = np.zeros(max(n, 1), dtype=np.int64)
+        cows = np.zeros((max(n, 1), 2), dtype=np.int32)
+        n_cow = ctypes.c_int(0)
+        rc = lib().pkv_seq_append_tokens(self._h, int(seq_id), tok.ctypes.data if n else None,
+                                         n, slots.ctypes.data, cows.ctypes.data,
+                                         ctypes.byref(n_cow))
+        if rc != PKV_OK:
+            return rc, slots[:0], cows[:0]
+        return rc, slots[:n], cows[:n_cow.value]
+
+    def pkv_seq_share_prefix(self, seq_id, tokens):
+        """Create seq_id on the longest cached prefix of tokens; returns (status,
+        tokens covered)."""
+        import numpy as np
+        tok = np.ascontiguousarray(tokens, dtype=np.int32).reshape(-1)
+        got = ctypes.c_int(0)
+        rc = lib().pkv_seq_share_prefix(self._h, int(seq_id),
+                                        tok.ctypes.data if tok.shape[0] else None,
+                                        tok.shape[0], ctypes.byref(got))
+        return rc, got.value
+
+    def pkv_prefix_cache_stats(self):
+        """Returns (cached blocks, evictable blocks, queried tokens, hit tokens)."""
+        c, e = ctypes.c_int(), ctypes.c_int()
+        q, h = ctypes.c_int64(), ctypes.c_int64()
+        _check(lib().pkv_prefix_cache_stats(self._h, ctypes.byref(c), ctypes.byref(e),
+                                            ctypes.byref(q), ctypes.byref(h)),
+               "pkv_prefix_cache_stats")
+        return c.value, e.value, q.value, h.value
 
     def pkv_seq_fork(self, parent, child):
         return lib().pkv_seq_fork(self._h, int(parent), int(child))

@@ -12,6 +12,7 @@
 // appends). Pure host code: no CUDA call.
 #include <algorithm>
 #include <cstring>
+#include <list>
 #include <new>
 #include <unordered_map>
 #include <vector>
@@ -20,9 +21,36 @@
 
 namespace {
 
+// splitmix64 (Steele, Lea, Flood: "Fast splittable pseudorandom number generators",
+// OOPSLA 2014), used as a mixing function for the prefix hash chain.
+uint64_t splitmix64(uint64_t x) {
+    uint64_t z = x + 0x9E3779B97F4A7C15ull;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+}
+
+// Hash of a full block given the hash of everything before it (0 for the first).
+uint64_t chain_hash(uint64_t parent, const int32_t *tokens, int n) {
+    uint64_t h = parent;
+    for (int i = 0; i < n; ++i) h = splitmix64(h ^ (uint64_t)(uint32_t)tokens[i]);
+    return h;
+}
+
 struct Seq {
     std::vector<int32_t> table;  // logical block -> physical block
     int64_t len = 0;             // tokens written
+    // prefix caching: token ids of the partly filled last block and the chain hash of
+    // the full blocks before it; `tracked` = every token so far came with its id
+    bool tracked = false;
+    uint64_t hash = 0;
+    std::vector<int32_t> partial;
+};
+
+struct CachedBlock {
+    uint64_t parent;              // chain hash of the blocks before it
+    std::vector<int32_t> tokens;  // its block_size token ids
+    int32_t block;
 };
 
 }  // namespace
@@ -35,12 +63,70 @@ struct pkv_alloc {
     std::vector<int32_t> refcount;
     std::unordered_map<int64_t, Seq> seqs;
     int64_t logical_tokens = 0;
+    // prefix cache: chain hash -> cached block; blocks whose count fell to 0 while cached
+    // wait, least recently released first, in `evictable` until a free block is needed
+    bool prefix_cache = false;
+    std::unordered_map<uint64_t, CachedBlock> cache;
+    std::vector<uint64_t> block_key;   // per block: its cache key (valid if cached[b])
+    std::vector<char> cached;
+    std::list<int32_t> evictable;
+    std::vector<std::list<int32_t>::iterator> evict_pos;
+    int64_t query_tokens = 0, hit_tokens = 0;
+
+    int available() const { return (int)(free_stack.size() + evictable.size()); }
 
     int32_t take() {
-        int32_t b = free_stack.back();
-        free_stack.pop_back();
+        int32_t b;
+        if (!free_stack.empty()) {
+            b = free_stack.back();
+            free_stack.pop_back();
+        } else {
+            // reclaim the least recently released cached block: its contents go
+            b = evictable.front();
+            evictable.pop_front();
+            cache.erase(block_key[b]);
+            cached[b] = 0;
+        }
         refcount[b] = 1;
         return b;
+    }
+
+    // one reference fewer; a block nobody holds is freed, or kept for reuse if cached
+    void release(int32_t b) {
+        if (--refcount[b] != 0) return;
+        if (cached[b]) {
+            evictable.push_back(b);
+            evict_pos[b] = std::prev(evictable.end());
+        } else {
+            free_stack.push_back(b);
+        }
+    }
+
+    // a new holder of cached block b (from the prefix cache)
+    void acquire_cached(int32_t b) {
+        if (refcount[b] == 0) evictable.erase(evict_pos[b]);
+        refcount[b] += 1;
+    }
+
+    // the token at position n of s (already placed) completes or extends its block
+    void record_token(Seq &s, int64_t n, const int32_t *token) {
+        if (!prefix_cache || !s.tracked) return;
+        if (!token) {
+            s.tracked = false;   // an id is missing: this sequence stops sharing
+            s.partial.clear();
+            return;
+        }
+        s.partial.push_back(*token);
+        if ((int)s.partial.size() < block_size) return;
+        const uint64_t key = chain_hash(s.hash, s.partial.data(), block_size);
+        const int32_t b = s.table[n / block_size];
+        if (!cache.count(key) && !cached[b]) {
+            cache.emplace(key, CachedBlock{s.hash, s.partial, b});
+            block_key[b] = key;
+            cached[b] = 1;
+        }
+        s.hash = key;
+        s.partial.clear();
     }
 
     // Blocks an append of n tokens to `s` (nullptr = new sequence) would take.
@@ -80,6 +166,9 @@ int pkv_alloc_create(pkv_alloc **out, int num_blocks, int block_size, int max_bl
     a->block_size = block_size;
     a->max_blocks = max_blocks_per_seq;
     a->refcount.assign(num_blocks, 0);
+    a->block_key.assign(num_blocks, 0);
+    a->cached.assign(num_blocks, 0);
+    a->evict_pos.resize(num_blocks);
     a->free_stack.resize(num_blocks);
     for (int i = 0; i < num_blocks; ++i)
         a->free_stack[num_blocks - 1 - i] = initial_order ? initial_order[i] : i;
@@ -92,8 +181,11 @@ int pkv_alloc_destroy(pkv_alloc *a) {
     return PKV_OK;
 }
 
-int pkv_seq_append(pkv_alloc *a, int64_t seq_id, int n_tokens, int64_t *slots_out,
-                   int32_t *cow_pairs_out, int *n_cow_out) {
+namespace {
+
+// tokens == nullptr: an append without ids (with_ids false)
+int append_impl(pkv_alloc *a, int64_t seq_id, int n_tokens, bool with_ids, const int32_t *tokens,
+                int64_t *slots_out, int32_t *cow_pairs_out, int *n_cow_out) {
     if (!a || n_tokens < 0) return PKV_ERR_INVALID_ARG;
     if (n_tokens > 0 && !slots_out) return PKV_ERR_INVALID_ARG;
     auto it = a->seqs.find(seq_id);
@@ -101,11 +193,13 @@ int pkv_seq_append(pkv_alloc *a, int64_t seq_id, int n_tokens, int64_t *slots_ou
     int64_t need, table_len;
     a->needs(existing, n_tokens, &need, &table_len);
     if (table_len > a->max_blocks) return PKV_ERR_TABLE_FULL;
-    if (need > (int64_t)a->free_stack.size()) return PKV_ERR_OUT_OF_BLOCKS;
+    if (need > (int64_t)a->available()) return PKV_ERR_OUT_OF_BLOCKS;
     if (need > 0 && !cow_pairs_out && existing && existing->len % a->block_size != 0 &&
         a->refcount[existing->table.back()] > 1)
         return PKV_ERR_INVALID_ARG;  // a copy-on-write pair would be lost
+    const bool created = !existing;
     Seq &s = a->seqs[seq_id];
+    if (created) s.tracked = a->prefix_cache && with_ids;
     const int bs = a->block_size;
     int n_cow = 0;
     for (int i = 0; i < n_tokens; ++i) {
@@ -123,9 +217,81 @@ int pkv_seq_append(pkv_alloc *a, int64_t seq_id, int n_tokens, int64_t *slots_ou
         }
         slots_out[i] = (int64_t)s.table[n / bs] * bs + n % bs;
         s.len = n + 1;
+        a->record_token(s, n, with_ids ? tokens + i : nullptr);
     }
     a->logical_tokens += n_tokens;
     if (n_cow_out) *n_cow_out = n_cow;
+    return PKV_OK;
+}
+
+}  // namespace
+
+int pkv_seq_append(pkv_alloc *a, int64_t seq_id, int n_tokens, int64_t *slots_out,
+                   int32_t *cow_pairs_out, int *n_cow_out) {
+    return append_impl(a, seq_id, n_tokens, false, nullptr, slots_out, cow_pairs_out, n_cow_out);
+}
+
+int pkv_seq_append_tokens(pkv_alloc *a, int64_t seq_id, const int32_t *tokens, int n_tokens,
+                          int64_t *slots_out, int32_t *cow_pairs_out, int *n_cow_out) {
+    if (n_tokens > 0 && !tokens) return PKV_ERR_INVALID_ARG;
+    return append_impl(a, seq_id, n_tokens, true, tokens, slots_out, cow_pairs_out, n_cow_out);
+}
+
+int pkv_alloc_set_prefix_cache(pkv_alloc *a, int enable) {
+    if (!a || (enable != 0 && enable != 1)) return PKV_ERR_INVALID_ARG;
+    if (a->prefix_cache && !enable) {
+        // forget every cached block; the ones nobody holds become free
+        for (int32_t b : a->evictable) a->free_stack.push_back(b);
+        a->evictable.clear();
+        a->cache.clear();
+        std::fill(a->cached.begin(), a->cached.end(), 0);
+        for (auto &kv : a->seqs) {
+            kv.second.tracked = false;
+            kv.second.partial.clear();
+        }
+    }
+    a->prefix_cache = enable != 0;
+    return PKV_OK;
+}
+
+int pkv_seq_share_prefix(pkv_alloc *a, int64_t seq_id, const int32_t *tokens, int n_tokens,
+                         int *n_cached_out) {
+    if (!a || n_tokens < 0 || (n_tokens > 0 && !tokens)) return PKV_ERR_INVALID_ARG;
+    if (a->seqs.count(seq_id)) return PKV_ERR_SEQ_EXISTS;
+    Seq s;
+    s.tracked = a->prefix_cache;
+    const int bs = a->block_size;
+    int matched = 0;
+    if (a->prefix_cache) {
+        for (int j = 0; (j + 1) * bs <= n_tokens && j < a->max_blocks; ++j) {
+            const int32_t *blk = tokens + (size_t)j * bs;
+            const uint64_t key = chain_hash(s.hash, blk, bs);
+            auto hit = a->cache.find(key);
+            if (hit == a->cache.end() || hit->second.parent != s.hash ||
+                std::memcmp(hit->second.tokens.data(), blk, sizeof(int32_t) * bs) != 0)
+                break;
+            a->acquire_cached(hit->second.block);
+            s.table.push_back(hit->second.block);
+            s.hash = key;
+            matched += bs;
+        }
+        a->query_tokens += n_tokens;
+        a->hit_tokens += matched;
+    }
+    s.len = matched;
+    a->logical_tokens += matched;
+    a->seqs.emplace(seq_id, std::move(s));
+    if (n_cached_out) *n_cached_out = matched;
+    return PKV_OK;
+}
+
+int pkv_prefix_cache_stats(const pkv_alloc *a, int *cached_blocks, int *evictable_blocks,
+                           int64_t *query_tokens, int64_t *hit_tokens) {
+    if (!a) return PKV_ERR_INVALID_ARG;
+    if (cached_blocks) *cached_blocks = (int)a->cache.size();
+    if (evictable_blocks) *evictable_blocks = (int)a->evictable.size();
+    if (query_tokens) *query_tokens = a->query_tokens;
+    if (hit_tokens) *hit_tokens = a->hit_tokens;
     return PKV_OK;
 }
 
@@ -173,7 +339,7 @@ int pkv_seq_free(pkv_alloc *a, int64_t seq_id) {
     if (it == a->seqs.end()) return PKV_ERR_UNKNOWN_SEQ;
     const Seq &s = it->second;
     for (auto b = s.table.rbegin(); b != s.table.rend(); ++b) {
-        if (--a->refcount[*b] == 0) a->free_stack.push_back(*b);
+        a->release(*b);
     }
     a->logical_tokens -= s.len;
     a->seqs.erase(it);
@@ -200,7 +366,7 @@ int pkv_block_tables(const pkv_alloc *a, const int64_t *seq_ids, int n, int32_t 
 int pkv_stats(const pkv_alloc *a, int *free_blocks, int *held_blocks, int64_t *logical_tokens,
               double *utilisation) {
     if (!a) return PKV_ERR_INVALID_ARG;
-    const int fr = (int)a->free_stack.size();
+    const int fr = a->available();
     const int held = a->num_blocks - fr;
     if (free_blocks) *free_blocks = fr;
     if (held_blocks) *held_blocks = held;
