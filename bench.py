@@ -460,6 +460,7 @@ def gpu_arm(args, rank, world, local_rank):
     achieved = roof_layer / (k1_avg_ms * 1e-3) / 1e9
     read_probe = hbm_read_probe(dev, stream)
     swap = swap_measurement(wl, dev, stream) if args.swap else None
+    prefix_cache = prefix_cache_measurement(sp) if args.prefix_cache else None
     traffic = None if shared else read_traffic(args.workload, sp.block_size)
 
     # ---- end to end: host block manager + pinned host buffers through the public API
@@ -493,6 +494,7 @@ def gpu_arm(args, rank, world, local_rank):
         "tokens_per_s": round(tokens_per_s, 1),
         "pct_of_hbm_peak": round(100 * value / world / peak, 2),
         **({"swap_blocks": swap} if swap else {}),
+        **({"prefix_cache": prefix_cache} if prefix_cache else {}),
         "clocks": clocks.summary(),
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
@@ -546,6 +548,65 @@ def replay_block_manager(wl):
             lens, wl.context_lens):
         raise RuntimeError("block manager replay does not reproduce the workload's tables")
     return mgr
+
+
+def prefix_cache_measurement(sp, requests=1024, concurrency=128, decode_len=64, seed=11):
+    """Host-side prefix caching ("vLLM / PagedAttention — 分页 KV Cache 分析" §2.3, §3.2):
+    a stream of requests, each one of the workload's system prompts (its shared-prefix
+    length) plus a private question of 32..511 tokens, decoded for decode_len tokens with
+    `concurrency` requests live at a time, run once with the cache off and once on.
+    Reports the prefill tokens found cached, the blocks held at the peak and the host
+    time of admissions (share_prefix + append of the uncached tokens)."""
+    import time
+    import paged_kv_cache_320_b200 as pkv
+    rng = np.random.default_rng(seed)
+    prompts = max(sp.prompts, 1)
+    prefix = sp.prefix if sp.prompts else 1024
+    bs = sp.block_size
+    system = [rng.integers(0, 32000, prefix, dtype=np.int32) for _ in range(prompts)]
+    reqs = [(int(rng.integers(0, prompts)), rng.integers(0, 32000, int(rng.integers(32, 512)),
+                                                          dtype=np.int32))
+            for _ in range(requests)]
+    max_tokens = prefix + 512 + decode_len
+    mb = -(-max_tokens // bs)
+    nb = concurrency * mb + prompts * (-(-prefix // bs))
+    out = {"requests": requests, "concurrency": concurrency, "decode_tokens": decode_len,
+           "prompts": prompts, "prefix_tokens": prefix, "block_size": bs, "num_blocks": nb}
+    for on in (0, 1):
+        mgr = pkv.BlockManager(nb, bs, mb)
+        mgr.pkv_alloc_set_prefix_cache(on)
+        live = {}
+        nxt = 0
+        admit_s = 0.0
+        prefill = cached = peak = 0
+        while nxt < len(reqs) or live:
+            while nxt < len(reqs) and len(live) < concurrency:
+                p, q = reqs[nxt]
+                toks = np.concatenate([system[p], q])
+                t0 = time.perf_counter()
+                st, got = mgr.pkv_seq_share_prefix(nxt, toks[:-1])
+                st2, _, _ = mgr.pkv_seq_append_tokens(nxt, toks[got:])
+                admit_s += time.perf_counter() - t0
+                if st or st2:
+                    raise RuntimeError(f"prefix-cache admission failed ({st}, {st2})")
+                prefill += len(toks)
+                cached += got
+                live[nxt] = decode_len
+                nxt += 1
+            peak = max(peak, mgr.pkv_stats()[1])
+            for r in list(live):
+                if mgr.pkv_seq_append_tokens(r, rng.integers(0, 32000, 1, dtype=np.int32))[0]:
+                    raise RuntimeError("prefix-cache decode append failed")
+                live[r] -= 1
+                if live[r] == 0:
+                    mgr.pkv_seq_free(r)
+                    del live[r]
+        key = "cache_on" if on else "cache_off"
+        out[key] = {"prefill_tokens": prefill, "prefill_tokens_cached": cached,
+                    "hit_rate": round(cached / prefill, 4), "peak_blocks_held": peak,
+                    "admit_us_per_request": round(1e6 * admit_s / len(reqs), 2)}
+        mgr.close()
+    return out
 
 
 def swap_measurement(wl, dev, stream, budget=512 << 20, reps=5):
@@ -824,6 +885,8 @@ def main():
     ap.add_argument("--partition", type=int, default=0, help="decode partition size (0 = auto)")
     ap.add_argument("--swap", action="store_true",
                     help="also time pkv_swap_blocks (preemption) against a contiguous copy")
+    ap.add_argument("--prefix-cache", action="store_true",
+                    help="also replay a request stream through the block manager's prefix cache")
     ap.add_argument("--decode", default="plain", choices=["plain", "shared"],
                     help="shared: the shared-prefix-aware decode (shared-prefix workload)")
     ap.add_argument("--batch", type=int, default=0,

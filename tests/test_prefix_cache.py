@@ -298,3 +298,18 @@ def test_invalid_arguments():
     assert L.pkv_seq_share_prefix(mgr._h, 0, None, 0, None) == 0
     assert L.pkv_seq_share_prefix(mgr._h, 0, None, 0, None) == B.PKV_ERR_SEQ_EXISTS
     assert L.pkv_prefix_cache_stats(None, None, None, None, None) == B.PKV_ERR_INVALID_ARG
+
+
+def test_bench_request_stream_hits_every_repeated_prompt():
+    """The benchmark's request stream (small): with the cache on, every request after the
+    first of its prompt finds the whole prompt cached (whole blocks of it); off, none."""
+    import bench
+    from paged_kv_cache_320_b200 import synth
+    sp = synth.SPECS["shared_prefix"]
+    r = bench.prefix_cache_measurement(sp, requests=64, concurrency=8, decode_len=4)
+    assert r["cache_off"]["prefill_tokens_cached"] == 0
+    full = (sp.prefix // sp.block_size) * sp.block_size
+    first_uses = r["prompts"]
+    on = r["cache_on"]["prefill_tokens_cached"]
+    assert on >= (64 - first_uses) * full
+    assert r["cache_on"]["peak_blocks_held"] < r["cache_off"]["peak_blocks_held"]
