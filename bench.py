@@ -395,6 +395,22 @@ def gpu_arm(args, rank, world, local_rank):
             sp.num_kv_heads * sp.head_dim * 4
         roof_layer = roof_layer - kv_layer + uniq
 
+    fused = args.step == "fused"
+    if fused and shared:
+        raise SystemExit("--step fused runs the plain decode")
+    if fused:
+        ws = torch.zeros(pkv.pkv_decode_step_workspace_size(
+            B, sp.num_heads, sp.num_kv_heads, sp.head_dim, sp.block_size, max_len, P),
+            dtype=torch.uint8, device=dev)
+    # this step's K/V rows as [B, Hkv, D] (one new token per sequence)
+    kn3 = [wl.k_new[l].view(B, sp.num_kv_heads, sp.head_dim) for l in range(L)]
+    vn3 = [wl.v_new[l].view(B, sp.num_kv_heads, sp.head_dim) for l in range(L)]
+
+    def fused_layer(l, out_t, q_t, kn_t, vn_t, bt_t, lens_t):
+        pkv.pkv_paged_decode_step(out_t, q_t, kn_t, vn_t, wl.k_cache[l], wl.v_cache[l], bt_t,
+                                  lens_t, max_len, ws, scale=wl.scale, partition_size=P,
+                                  stream=stream)
+
     def decode(l, out_t, q_t, bt_t, lens_t):
         if shared:
             pkv.pkv_paged_attention_decode_shared_prefix(
@@ -409,18 +425,23 @@ def gpu_arm(args, rank, world, local_rank):
 
     def step(record=False):
         for l in range(L):
-            pkv.pkv_reshape_and_cache(wl.k_new[l], wl.v_new[l], wl.k_cache[l], wl.v_cache[l],
-                                      slots, stream=stream)
+            if not fused:
+                pkv.pkv_reshape_and_cache(wl.k_new[l], wl.v_new[l], wl.k_cache[l],
+                                          wl.v_cache[l], slots, stream=stream)
             if record:
                 e0 = torch.cuda.Event(enable_timing=True)
                 e1 = torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
-            decode(l, outs[l], wl.q[l], bt, lens)
+            if fused:
+                # the workload's slot of each sequence is its newest position (len - 1)
+                fused_layer(l, outs[l], wl.q[l], kn3[l], vn3[l], bt, lens)
+            else:
+                decode(l, outs[l], wl.q[l], bt, lens)
             if record:
                 e1.record(stream)
                 k1_events.append((e0, e1))
 
-    launches_per_step = L * (4 if shared else 2 + (1 if pmax > 1 else 0))
+    launches_per_step = L * (1 if fused else 4 if shared else 2 + (1 if pmax > 1 else 0))
     dist = None
     if world > 1:
         import torch.distributed as dist
@@ -461,10 +482,11 @@ def gpu_arm(args, rank, world, local_rank):
     read_probe = hbm_read_probe(dev, stream)
     swap = swap_measurement(wl, dev, stream) if args.swap else None
     prefix_cache = prefix_cache_measurement(sp) if args.prefix_cache else None
-    traffic = None if shared else read_traffic(args.workload, sp.block_size)
+    traffic = None if shared or fused else read_traffic(args.workload, sp.block_size)
 
     # ---- end to end: host block manager + pinned host buffers through the public API
-    e2e = e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, world, decode)
+    e2e = e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, world, decode,
+                  fused_layer if fused else None)
 
     result = {
         "metric": METRIC,
@@ -487,6 +509,7 @@ def gpu_arm(args, rank, world, local_rank):
             "sum_context_tokens": int(wl.context_lens.sum()),
             "partition_size": P,
             "decode": args.decode,
+            "step": args.step,
             "kv_bytes_per_step": kv_step,
             "l2": f"inputs larger than L2: {kv_layer / 1e6:.0f} MB of K/V per layer vs 126 MB L2",
             "parallelism": f"replicas x{world}",
@@ -500,7 +523,8 @@ def gpu_arm(args, rank, world, local_rank):
         "gpu_launches": launches_per_step * args.steps,
         "roofline": {
             "kernel": "paged_decode_shared_kernel (+ plan, reduce)" if shared
-            else "paged_decode_partition_kernel",
+            else "paged_decode_step_kernel (cache write + decode + merge)" if fused
+            else "paged_decode_partition_kernel (+ reduce)",
             "bound": "hbm",
             "achieved": round(achieved, 1),
             "peak": peak,
@@ -678,7 +702,8 @@ def hbm_read_probe(dev, stream):
     return (1 << 32) / (best * 1e-3) / 1e9
 
 
-def e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, world, decode):
+def e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, world, decode,
+            fused_layer=None):
     """Each step: the host block manager appends one token to every sequence (one batched
     call) and exports the tables; the step's inputs (slots, tables, lengths, and q, k_new,
     v_new of every layer) go host->device from pinned memory on a copy stream, layer by
@@ -710,6 +735,17 @@ def e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, worl
     ids = np.arange(B, dtype=np.int64)
     h2d = (q_h.numel() * 2 + kn_h.numel() * 2 + vn_h.numel() * 2 + slots_h.numel() * 8 +
            bt_h.numel() * 4 + lens_h.numel() * 4)
+    if fused_layer is not None:
+        # tables, lengths and the free list live on the device: uploaded once here, then
+        # updated by pkv_device_append every step (the host allocator mirrors it)
+        st, tables, lens = mgr.pkv_block_tables(ids)
+        bt_d.copy_(torch.from_numpy(tables))
+        lens_d.copy_(torch.from_numpy(lens))
+        free_d = torch.from_numpy(mgr.pkv_alloc_free_list()).to(dev)
+        used_d = torch.zeros(1, dtype=torch.int32, device=dev)
+        kn3_d = kn_d.view(L, B, sp.num_kv_heads, sp.head_dim)
+        vn3_d = vn_d.view(L, B, sp.num_kv_heads, sp.head_dim)
+        h2d = q_h.numel() * 2 + kn_h.numel() * 2 + vn_h.numel() * 2
     d2h = out_h.numel() * 2
     copy_in = torch.cuda.Stream(dev)
     copy_out = torch.cuda.Stream(dev)
@@ -717,7 +753,36 @@ def e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, worl
     ev_out = [torch.cuda.Event() for _ in range(L)]
     kv_total = [0]
 
+    def one_step_fused():
+        with torch.cuda.stream(copy_in):
+            for l in range(L):
+                kn_d[l].copy_(kn_h[l], non_blocking=True)
+                vn_d[l].copy_(vn_h[l], non_blocking=True)
+                q_d[l].copy_(q_h[l], non_blocking=True)
+                ev_in[l].record(copy_in)
+        pkv.pkv_device_append(bt_d, lens_d, free_d, used_d, wl.num_blocks, max_len,
+                              sp.block_size, stream=stream)
+        for l in range(L):
+            stream.wait_event(ev_in[l])
+            fused_layer(l, out_d[l], q_d[l], kn3_d[l], vn3_d[l], bt_d, lens_d)
+            ev_out[l].record(stream)
+        with torch.cuda.stream(copy_out):
+            for l in range(L):
+                copy_out.wait_event(ev_out[l])
+                out_h[l].copy_(out_d[l], non_blocking=True)
+        # the host allocator mirrors the device append while the GPU works
+        st, done, sl, cows = mgr.pkv_seq_append_batch(ids, 1)
+        if st != 0 or len(cows):
+            raise RuntimeError(f"host mirror append failed ({st})")
+        kv_total[0] += int(mirror_lens[0].sum() + B) * sp.num_kv_heads * sp.head_dim * 4 * L
+        mirror_lens[0] += 1
+        copy_out.synchronize()          # the step's result is on the host
+
+    mirror_lens = [mgr.pkv_block_tables(ids)[2].astype(np.int64)]
+
     def one_step():
+        if fused_layer is not None:
+            return one_step_fused()
         st, done, sl, cows = mgr.pkv_seq_append_batch(ids, 1)
         if st != 0 or len(cows):
             raise RuntimeError(f"append failed ({st}) or needed a copy in an unshared workload")
@@ -760,14 +825,26 @@ def e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, worl
     t1.record(stream)
     barrier()
     ms = max_over_ranks(t0.elapsed_time(t1)) / args.steps
+    if fused_layer is not None:
+        # the device's tables and lengths must equal the host allocator's after all steps
+        st, tables, lens = mgr.pkv_block_tables(ids)
+        if (pkv.pkv_get_device_status(stream=stream) != 0 or
+                not np.array_equal(bt_d.cpu().numpy(), tables) or
+                not np.array_equal(lens_d.cpu().numpy(), lens)):
+            raise RuntimeError("device append diverged from the host block manager")
     mgr.close()
     value = kv_total[0] / args.steps * world / (ms * 1e-3) / 1e9
     return {"value": round(value, 1), "unit": "GB/s", "ms_per_step": round(ms, 4),
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "includes": "host block-manager append (one batched call) and table export, pinned "
-                        "H2D of slots/tables/lengths and every layer's q/k_new/v_new, all "
-                        "layers' kernels, D2H of every layer's output (copies overlap kernels "
-                        "of other layers)"}
+            "includes": ("device append of one token per sequence (tables, lengths and free "
+                         "list resident on the GPU; the host allocator mirrors it with one "
+                         "batched call), pinned H2D of every layer's q/k_new/v_new, one fused "
+                         "kernel per layer, D2H of every layer's output"
+                         if fused_layer is not None else
+                         "host block-manager append (one batched call) and table export, pinned "
+                         "H2D of slots/tables/lengths and every layer's q/k_new/v_new, all "
+                         "layers' kernels, D2H of every layer's output (copies overlap kernels "
+                         "of other layers)")}
 
 
 # ----------------------------------------------------------------------------
@@ -887,6 +964,9 @@ def main():
                     help="also time pkv_swap_blocks (preemption) against a contiguous copy")
     ap.add_argument("--prefix-cache", action="store_true",
                     help="also replay a request stream through the block manager's prefix cache")
+    ap.add_argument("--step", default="separate", choices=["separate", "fused"],
+                    help="fused: one launch per layer (cache write + decode + merge) and the "
+                         "block-table update on the device")
     ap.add_argument("--decode", default="plain", choices=["plain", "shared"],
                     help="shared: the shared-prefix-aware decode (shared-prefix workload)")
     ap.add_argument("--batch", type=int, default=0,

@@ -68,7 +68,9 @@ enum pkv_device_status_bits {
     PKV_STATUS_BAD_PAIR = 1u << 1,     /* copy_blocks / swap_blocks: block id outside the pool  */
     PKV_STATUS_BAD_BLOCK = 1u << 2,    /* decode: block id outside [0, num_blocks) (read as 0)  */
     PKV_STATUS_BAD_LEN = 1u << 3,      /* decode: context_len < 0 or above its bound (clamped)  */
-    PKV_STATUS_WAIT_TIMEOUT = 1u << 4  /* decode: a pipeline wait exceeded its iteration limit  */
+    PKV_STATUS_WAIT_TIMEOUT = 1u << 4, /* decode: a pipeline wait exceeded its iteration limit  */
+    PKV_STATUS_NO_BLOCKS = 1u << 5,    /* device append: step refused, nothing changed          */
+    PKV_STATUS_WORKSPACE = 1u << 6     /* decode step: workspace header not zero nor its own    */
 };
 
 /* Human-readable name of a status code (static string). */
@@ -231,6 +233,65 @@ int pkv_swap_blocks(void *const *k_caches, void *const *v_caches, int num_layers
                     size_t host_buffer_bytes, int to_host, int num_kv_heads, int head_dim,
                     int block_size, int num_blocks, int dtype, pkv_stream_t stream);
 
+/* ------------------------------------------------------------------------------
+ * Decode step on the device ("分页 KV Cache 分析" §3.1: each decode step writes the new
+ * token's K/V into its page, then attention reads the pages; §2.3: the block manager
+ * hands a sequence a new page when its last one is full; "vLLM" entity page, 关键观察:
+ * a kernel launch costs a few microseconds, a visible share of a decode step). Two calls
+ * replace, per step, the host table update + upload and, per layer, the cache write,
+ * decode and merge launches:
+ *
+ * pkv_device_append (once per step, before the layers): appends one token to each of
+ * num_seqs sequences, in place on device arrays.
+ *   n = context_lens[s]; if n % block_size == 0 the sequence takes the next entry of
+ *   free_blocks (entries free_blocks[*free_used], [*free_used + 1], ... go to the
+ *   sequences that need one, in increasing s) into block_tables[s][n / block_size];
+ *   slots_out[s] = block_tables[s][n / block_size] * block_size + n % block_size (or -1,
+ *   with PKV_STATUS_BAD_BLOCK, if that entry is outside [0, num_blocks));
+ *   context_lens[s] = n + 1; finally *free_used += blocks taken.
+ * With free_blocks holding the host block manager's free blocks in the order it would
+ * pop them, the result equals pkv_seq_append(.., 1, ..) on s = 0, 1, ... (no sequence may
+ * share its partly filled last block: copy-on-write stays on the host).
+ * All or nothing: if fewer than the needed entries remain (free_count - *free_used), an
+ * entry is outside [0, num_blocks), some n < 0, n + 1 > max_context_len or
+ * n / block_size >= max_blocks_per_seq, nothing is written and PKV_STATUS_NO_BLOCKS is
+ * set. block_tables int32 [num_seqs][max_blocks_per_seq], context_lens int32 [num_seqs],
+ * free_blocks int32 [free_count], free_used int32 [1] (all device), slots_out int64
+ * [num_seqs] device or NULL. One CTA; asynchronous on `stream`.
+ * Errors: PKV_ERR_INVALID_ARG, PKV_ERR_CUDA.
+ * ---------------------------------------------------------------------------- */
+int pkv_device_append(int32_t *block_tables, int32_t *context_lens, const int32_t *free_blocks,
+                      int free_count, int32_t *free_used, int64_t *slots_out, int num_seqs,
+                      int max_blocks_per_seq, int block_size, int num_blocks,
+                      int max_context_len, pkv_stream_t stream);
+
+/* pkv_paged_decode_step (once per layer): one launch that writes every sequence's newest
+ * token and computes the decode attention over it:
+ *   for each s with len = context_lens[s] >= 1, slot = block_tables[s][(len-1)/bs]*bs +
+ *   (len-1)%bs: k_cache[slot / bs][h][slot % bs][:] = k_new[s][h][:] (V alike), then
+ *   out = pkv_paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens).
+ * Same arguments, layouts, limits and results as pkv_reshape_and_cache with that slot
+ * mapping followed by pkv_paged_attention_decode (same partition size: identical bits),
+ * plus k_new / v_new [num_seqs][num_kv_heads][head_dim] device, 16-byte aligned.
+ * Workspace: pkv_decode_step_workspace_size bytes (at least 256), 256-byte aligned, owned
+ * by the caller, ZERO-FILLED before its first use and then reused only by this call on one
+ * stream (each launch leaves it ready for the next). A workspace whose header is neither
+ * zero nor left by this call is refused on the device (PKV_STATUS_WORKSPACE, no output).
+ * When some context spans several partitions the launch is cooperative (all CTAs resident)
+ * and merges the partitions after a bounded grid barrier (PKV_STATUS_WAIT_TIMEOUT if it
+ * gives up). Errors: as pkv_paged_attention_decode. */
+int pkv_paged_decode_step(void *out, const void *q, const void *k_new, const void *v_new,
+                          void *k_cache, void *v_cache, const int32_t *block_tables,
+                          const int32_t *context_lens, int num_seqs, int num_heads,
+                          int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                          int num_blocks, int max_context_len, float scale, int dtype,
+                          int partition_size, void *workspace, size_t workspace_bytes,
+                          pkv_stream_t stream);
+
+int pkv_decode_step_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                   int block_size, int max_context_len, int partition_size,
+                                   size_t *bytes_out);
+
 /* Synchronise `stream`, then read (and with clear != 0 reset) the status word of the
  * current device. *status_out gets the PKV_STATUS_* bits. Returns PKV_OK, or
  * PKV_ERR_CUDA if synchronisation or the read failed. */
@@ -277,6 +338,12 @@ int pkv_seq_append_batch(pkv_alloc *a, const int64_t *seq_ids, int n, int n_toke
 
 /* Errors: PKV_ERR_UNKNOWN_SEQ (no parent), PKV_ERR_SEQ_EXISTS (child id in use). */
 int pkv_seq_fork(pkv_alloc *a, int64_t parent, int64_t child);
+
+/* The blocks the next allocations would take, in that order (free blocks, then cached
+ * blocks nobody holds, least recently released first): at most max_out of them into
+ * blocks_out, their count into *n_out. Uploaded to the device, this is the free list
+ * pkv_device_append takes from. */
+int pkv_alloc_free_list(const pkv_alloc *a, int32_t *blocks_out, int max_out, int *n_out);
 
 /* ------------------------------------------------------------------------------
  * Prefix caching ("分页 KV Cache 分析" §2.3 and §3.2: common prefixes such as a system

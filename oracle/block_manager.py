@@ -225,6 +225,10 @@ class BlockManagerModel:
         self.lens[seq] = len(table) * self.bs
         return OK, self.lens[seq]
 
+    def free_list(self):
+        """The blocks the next allocations take, in order."""
+        return list(reversed(self.free_stack)) + list(self.evictable)
+
     def prefix_cache_stats(self):
         return len(self.cache), len(self.evictable), self.query_tokens, self.hit_tokens
 

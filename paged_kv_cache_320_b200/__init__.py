@@ -11,6 +11,9 @@ from ._binding import (  # noqa: F401
     lib,
     pkv_copy_blocks,
     pkv_decode_partition_size,
+    pkv_decode_step_workspace_size,
+    pkv_device_append,
+    pkv_paged_decode_step,
     pkv_decode_workspace_size,
     pkv_get_device_status,
     pkv_paged_attention_decode,

@@ -34,6 +34,8 @@ STATUS_BAD_PAIR = 1 << 1
 STATUS_BAD_BLOCK = 1 << 2
 STATUS_BAD_LEN = 1 << 3
 STATUS_WAIT_TIMEOUT = 1 << 4
+STATUS_NO_BLOCKS = 1 << 5
+STATUS_WORKSPACE = 1 << 6
 
 _lib = None
 
@@ -79,6 +81,11 @@ def lib() -> ctypes.CDLL:
         L.pkv_block_tables.argtypes = [P, P, I, P, P]
         L.pkv_stats.argtypes = [P, ctypes.POINTER(I), ctypes.POINTER(I),
                                 ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_double)]
+        L.pkv_paged_decode_step.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I,
+                                            ctypes.c_float, I, I, P, SZ, P]
+        L.pkv_decode_step_workspace_size.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(SZ)]
+        L.pkv_device_append.argtypes = [P, P, P, I, P, P, I, I, I, I, I, P]
+        L.pkv_alloc_free_list.argtypes = [P, P, I, ctypes.POINTER(I)]
         L.pkv_alloc_set_prefix_cache.argtypes = [P, I]
         L.pkv_seq_append_tokens.argtypes = [P, I64, P, I, P, P, ctypes.POINTER(I)]
         L.pkv_seq_share_prefix.argtypes = [P, I64, P, I, ctypes.POINTER(I)]
@@ -93,6 +100,8 @@ def lib() -> ctypes.CDLL:
                      "pkv_get_device_status", "pkv_alloc_create", "pkv_alloc_destroy",
                      "pkv_seq_append", "pkv_seq_append_batch", "pkv_seq_fork", "pkv_seq_free",
                      "pkv_block_tables", "pkv_stats", "pkv_alloc_set_prefix_cache",
+                     "pkv_paged_decode_step", "pkv_decode_step_workspace_size", "pkv_device_append",
+                     "pkv_alloc_free_list",
                      "pkv_seq_append_tokens", "pkv_seq_share_prefix", "pkv_prefix_cache_stats"):
             getattr(L, name).restype = I
         _lib = L
@@ -234,6 +243,48 @@ def pkv_paged_attention_decode_shared_prefix(out, q, k_cache, v_cache, block_tab
     return out
 
 
+def pkv_decode_step_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                   max_context_len, partition_size=0) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib().pkv_decode_step_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim,
+                                                block_size, max_context_len, partition_size,
+                                                ctypes.byref(out)),
+           "pkv_decode_step_workspace_size")
+    return out.value
+
+
+def pkv_paged_decode_step(out, q, k_new, v_new, k_cache, v_cache, block_tables, context_lens,
+                          max_context_len, workspace, scale=None, partition_size=0, stream=None):
+    """Cache write of each sequence's newest token + decode attention in one launch.
+    k_new/v_new [B, Hkv, D]; workspace: uint8 device tensor of
+    pkv_decode_step_workspace_size bytes, zero-filled before its first use (torch.zeros)."""
+    B, Hq, D = q.shape
+    NB, Hkv, BS, D2 = k_cache.shape
+    if (D2 != D or out.shape != q.shape or v_cache.shape != k_cache.shape
+            or tuple(k_new.shape) != (B, Hkv, D) or v_new.shape != k_new.shape):
+        raise ValueError("shape mismatch")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    _check(lib().pkv_paged_decode_step(
+        _ptr(out), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
+        _ptr(block_tables), _ptr(context_lens), B, Hq, Hkv, D, BS, block_tables.shape[1], NB,
+        int(max_context_len), float(scale), _dtype_code(q), int(partition_size), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)), "pkv_paged_decode_step")
+    return out
+
+
+def pkv_device_append(block_tables, context_lens, free_blocks, free_used, num_blocks,
+                      max_context_len, block_size, slots_out=None, stream=None):
+    """One token appended to every sequence on the device (see pagedkv.h): block_tables
+    int32 [B, MB] and context_lens int32 [B] updated in place; free_blocks int32 [F] in pop
+    order; free_used int32 [1] advanced by the blocks taken; slots_out int64 [B] or None."""
+    B = context_lens.numel()
+    _check(lib().pkv_device_append(
+        _ptr(block_tables), _ptr(context_lens), _ptr(free_blocks), free_blocks.numel(),
+        _ptr(free_used), _ptr(slots_out), B, block_tables.shape[1], int(block_size),
+        int(num_blocks), int(max_context_len), _stream(stream)), "pkv_device_append")
+
+
 def pkv_reshape_and_cache(k_new, v_new, k_cache, v_cache, slot_mapping, stream=None):
     """k_new/v_new [T, Hkv, D]; caches [NB, Hkv, BS, D]; slot_mapping int64 [T]."""
     T, Hkv, D = k_new.shape
@@ -324,6 +375,16 @@ class BlockManager:
                                         slots.ctypes.data, cows.ctypes.data,
                                         ctypes.byref(n_cow), ctypes.byref(n_done))
         return rc, n_done.value, slots[:n, :n_tokens], cows[:n_cow.value]
+
+    def pkv_alloc_free_list(self, max_out=None):
+        """Blocks the next allocations would take, in order (int32 array)."""
+        import numpy as np
+        m = self.num_blocks if max_out is None else int(max_out)
+        buf = np.zeros(max(m, 1), dtype=np.int32)
+        n = ctypes.c_int(0)
+        _check(lib().pkv_alloc_free_list(self._h, buf.ctypes.data, m, ctypes.byref(n)),
+               "pkv_alloc_free_list")
+        return buf[:n.value].copy()
 
     def pkv_alloc_set_prefix_cache(self, enable):
         return lib().pkv_alloc_set_prefix_cache(self._h, int(bool(enable)))

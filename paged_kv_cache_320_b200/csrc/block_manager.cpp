@@ -363,6 +363,17 @@ int pkv_block_tables(const pkv_alloc *a, const int64_t *seq_ids, int n, int32_t 
     return PKV_OK;
 }
 
+int pkv_alloc_free_list(const pkv_alloc *a, int32_t *blocks_out, int max_out, int *n_out) {
+    if (!a || !n_out || max_out < 0 || (max_out > 0 && !blocks_out)) return PKV_ERR_INVALID_ARG;
+    int n = 0;
+    for (auto it = a->free_stack.rbegin(); it != a->free_stack.rend() && n < max_out; ++it)
+        blocks_out[n++] = *it;
+    for (auto it = a->evictable.begin(); it != a->evictable.end() && n < max_out; ++it)
+        blocks_out[n++] = *it;
+    *n_out = n;
+    return PKV_OK;
+}
+
 int pkv_stats(const pkv_alloc *a, int *free_blocks, int *held_blocks, int64_t *logical_tokens,
               double *utilisation) {
     if (!a) return PKV_ERR_INVALID_ARG;

@@ -86,6 +86,9 @@ struct DecodeParams {
     int num_seqs, num_heads, num_kv_heads, group;
     int max_blocks_per_seq, num_blocks, max_context_len, partition;
     float scale_log2;    // scale * log2(e)
+    // fused decode step only: this step's K/V rows [B][Hkv][D] and the caches they go to
+    const void *k_new, *v_new;
+    void *k_cache, *v_cache;
 };
 
 // Shared-memory plan. A stage holds 64 tokens of K then V as [token][head_dim]
@@ -392,49 +395,83 @@ __device__ __forceinline__ float2 row_stats(const float2 *ml, int row) {
     return make_float2(M, Lsum);
 }
 
-template <typename T, int D, int BS>
-__global__ void __launch_bounds__(kDecodeThreads, 2)
-paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
-                              const __grid_constant__ CUtensorMap tmap_v,
-                              const __grid_constant__ CUtensorMap tmap_q, DecodeParams prm) {
+// Carve-up of the decode kernels' dynamic shared memory (base aligned to 1024 B).
+template <int D>
+struct DecodeSmem {
+    uint8_t *ring, *qring;
+    float *obuf;
+    StageInfo *info;
+    uint64_t *full, *empty;
+    float2 *ml;   // [4][16]
+    int qslot_bytes;
+    __device__ DecodeSmem(uint8_t *smem, int G) {
+        using L = DecodeLayout<D>;
+        qslot_bytes = L::q_slot_bytes(G);
+        ring = smem;
+        qring = smem + L::kRingBytes;
+        obuf = reinterpret_cast<float *>(qring + L::kStages * qslot_bytes);
+        info = reinterpret_cast<StageInfo *>(reinterpret_cast<uint8_t *>(obuf) + L::obuf_bytes(G));
+        full = reinterpret_cast<uint64_t *>(info + L::kStages);
+        empty = full + L::kStages;
+        ml = reinterpret_cast<float2 *>(empty + L::kStages);
+    }
+    __device__ void init_barriers() {
+        if (threadIdx.x == 0) {
+            for (int i = 0; i < DecodeLayout<D>::kStages; ++i) {
+                mbar_init(smem_u32(&full[i]), 1);
+                mbar_init(smem_u32(&empty[i]), kConsumerWarps);
+            }
+            fence_mbar_init();
+        }
+    }
+};
+
+__device__ __forceinline__ uint8_t *aligned_dynamic_smem() {
+    extern __shared__ uint8_t smem_raw[];
+    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                       ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// The work-item loop shared by the decode kernels: warp 4 produces, warps 0-3
+// consume, until the item list is exhausted (barriers already initialised).
+// sched_mode 0: take items from prm.sched only if its header is armed (kSchedArmed);
+// sched_mode 1: the caller validated prm.sched (dynamic whenever it is non-null).
+// kStep: before loading the page that holds a sequence's last token (position
+// len_s - 1), the producer writes that token's K and V rows (prm.k_new / prm.v_new,
+// [B][Hkv][D]) for its KV head into the cache, so the cache write of the decode step
+// needs no launch of its own.
+template <typename T, int D, int BS, bool kStep>
+__device__ __forceinline__ void decode_items(const CUtensorMap *tmap_k, const CUtensorMap *tmap_v,
+                                             const CUtensorMap *tmap_q, const DecodeParams &prm,
+                                             DecodeSmem<D> &sm, int sched_mode) {
     using L = DecodeLayout<D>;
     constexpr int kBPS = kStageTokens / BS;   // blocks per stage
     constexpr int H = L::kHalves;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int G = prm.group;
-    const int qslot_bytes = L::q_slot_bytes(G);
-    uint8_t *ring = smem;
-    uint8_t *qring = smem + L::kRingBytes;
-    float *obuf = reinterpret_cast<float *>(qring + L::kStages * qslot_bytes);
-    StageInfo *info = reinterpret_cast<StageInfo *>(reinterpret_cast<uint8_t *>(obuf) +
-                                                    L::obuf_bytes(G));
-    uint64_t *full = reinterpret_cast<uint64_t *>(info + L::kStages);
-    uint64_t *empty = full + L::kStages;
-    float2 *ml = reinterpret_cast<float2 *>(empty + L::kStages);            // [4][16]
+    const int qslot_bytes = sm.qslot_bytes;
+    uint8_t *ring = sm.ring;
+    uint8_t *qring = sm.qring;
+    float *obuf = sm.obuf;
+    StageInfo *info = sm.info;
+    uint64_t *full = sm.full;
+    uint64_t *empty = sm.empty;
+    float2 *ml = sm.ml;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int Hkv = prm.num_kv_heads;
     const int P = prm.partition;
 
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < L::kStages; ++i) {
-            mbar_init(smem_u32(&full[i]), 1);
-            mbar_init(smem_u32(&empty[i]), kConsumerWarps);
-        }
-        fence_mbar_init();
-    }
-    pdl_wait_and_release();
-    __syncthreads();
-
     if (warp == kConsumerWarps) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            prefetch_tensormap(&tmap_k);
-            prefetch_tensormap(&tmap_v);
-            prefetch_tensormap(&tmap_q);
+            prefetch_tensormap(tmap_k);
+            prefetch_tensormap(tmap_v);
+            prefetch_tensormap(tmap_q);
         }
 #if PKV_KV_EVICT_FIRST
         const uint64_t kv_policy = l2_evict_first_policy();
@@ -461,8 +498,11 @@ paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
 
         // dynamic schedule when the workspace header is armed (read before any CTA
         // can change it: no CTA takes from `next` unless it saw the header armed)
-        const bool dynamic = prm.sched != nullptr &&
-                             __shfl_sync(0xffffffffu, lane == 0 ? *(volatile unsigned *)&prm.sched->armed : 0u, 0) == kSchedArmed;
+        const bool dynamic =
+            prm.sched != nullptr &&
+            (sched_mode == 1 ||
+             __shfl_sync(0xffffffffu, lane == 0 ? *(volatile unsigned *)&prm.sched->armed : 0u,
+                         0) == kSchedArmed);
         // A ticket is requested one item before it is resolved, so the atomic's
         // latency overlaps a whole item; the value lives in lane 0 until used.
         auto request = [&](int static_item) {
@@ -510,6 +550,26 @@ paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     const uint32_t qbytes = st == 0 ? (uint32_t)(G * L::kRowBytes) : 0u;
                     mbar_arrive_expect_tx(bar, (uint32_t)(nb_st * BS * L::kRowBytes * 2) + qbytes);
                 }
+                if constexpr (kStep) {
+                    if (cur.p == cur.np - 1 && st == cur.nst - 1 && cur.ntok > 0) {
+                        // this stage holds the sequence's last token: write its K/V row first
+                        const int tl = cur.ntok - 1 - st * kStageTokens;
+                        const int wb = __shfl_sync(0xffffffffu, bid, tl / BS);
+                        constexpr int VPR = D * 2 / 16;   // 16-byte vectors per row
+                        if (wb >= 0 && wb < prm.num_blocks && lane < 2 * VPR) {
+                            const bool isv = lane >= VPR;
+                            const int vi = lane - (isv ? VPR : 0);
+                            const uint4 *src = reinterpret_cast<const uint4 *>(isv ? prm.v_new : prm.k_new) +
+                                               ((size_t)cur.s * Hkv + cur.hk) * VPR + vi;
+                            uint4 *dst = reinterpret_cast<uint4 *>(isv ? prm.v_cache : prm.k_cache) +
+                                         (((size_t)wb * Hkv + cur.hk) * BS + tl % BS) * VPR + vi;
+                            *dst = *src;
+                            fence_proxy_async_global();   // before the tensor-map read of it
+                        }
+                        __syncwarp();
+                        fence_proxy_async_global();
+                    }
+                }
                 __syncwarp();
                 uint8_t *stage = ring + slot * L::kStageBytes;
                 if (lane < nb_st) {
@@ -522,12 +582,12 @@ paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     }
                     const uint32_t off = lane * BS * L::kRowBytes;
                     if (H == 2) {
-                        tma_load_3d(smem_u32(stage + off), &tmap_k, 0, y, 0, bar, kv_policy);
-                        tma_load_3d(smem_u32(stage + L::kKBytes + off), &tmap_v, 0, y, 0, bar,
+                        tma_load_3d(smem_u32(stage + off), tmap_k, 0, y, 0, bar, kv_policy);
+                        tma_load_3d(smem_u32(stage + L::kKBytes + off), tmap_v, 0, y, 0, bar,
                                     kv_policy);
                     } else {
-                        tma_load_2d(smem_u32(stage + off), &tmap_k, 0, y, bar, kv_policy);
-                        tma_load_2d(smem_u32(stage + L::kKBytes + off), &tmap_v, 0, y, bar,
+                        tma_load_2d(smem_u32(stage + off), tmap_k, 0, y, bar, kv_policy);
+                        tma_load_2d(smem_u32(stage + L::kKBytes + off), tmap_v, 0, y, bar,
                                     kv_policy);
                     }
                 }
@@ -535,9 +595,9 @@ paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     const int qrow = cur.s * prm.num_heads + cur.hk * G;
                     const uint32_t qdst = smem_u32(qring + slot * qslot_bytes);
                     if (H == 2)
-                        tma_load_3d(qdst, &tmap_q, 0, qrow, 0, bar, kv_policy);
+                        tma_load_3d(qdst, tmap_q, 0, qrow, 0, bar, kv_policy);
                     else
-                        tma_load_2d(qdst, &tmap_q, 0, qrow, bar, kv_policy);
+                        tma_load_2d(qdst, tmap_q, 0, qrow, bar, kv_policy);
                 }
                 if (st == 0) {
                     // look one item ahead: position and block-table slice
@@ -640,6 +700,18 @@ paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
             }
         }
     }
+}
+
+template <typename T, int D, int BS>
+__global__ void __launch_bounds__(kDecodeThreads, 2)
+paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                              const __grid_constant__ CUtensorMap tmap_v,
+                              const __grid_constant__ CUtensorMap tmap_q, DecodeParams prm) {
+    DecodeSmem<D> sm(aligned_dynamic_smem(), prm.group);
+    sm.init_barriers();
+    pdl_wait_and_release();
+    __syncthreads();
+    decode_items<T, D, BS, false>(&tmap_k, &tmap_v, &tmap_q, prm, sm, 0);
 }
 
 // Log-sum-exp merge of n partials (m_j in log2 units, l_j, normalised o_j) of one

@@ -15,6 +15,7 @@
 #include "cache_kernels.cuh"
 #include "decode_kernels.cuh"
 #include "shared_prefix_kernels.cuh"
+#include "step_kernels.cuh"
 #include "pagedkv.h"
 
 namespace {
@@ -350,6 +351,71 @@ int launch_shared_path(int BS, const CUtensorMap &mk, const CUtensorMap &mv,
                   dim3(pkv::kReduceWarps * 32), 0, st, prm);
 }
 
+// ---- fused decode step -----------------------------------------------------
+// Workspace: the decode workspace when some context spans several partitions,
+// else the 256-byte header alone (dynamic schedule).
+size_t step_ws_bytes(int B, int Hq, int D, int max_len, int P) {
+    const size_t t = ws_layout(B, Hq, D, max_len, P).total;
+    return t ? t : sizeof(pkv::StepHeader);
+}
+
+template <typename T, int D, int BS>
+int launch_step(const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mq,
+                const pkv::DecodeParams &prm, long long items, int merge, cudaStream_t st) {
+    using L = pkv::DecodeLayout<D>;
+    auto kern = pkv::paged_decode_step_kernel<T, D, BS>;
+    const size_t smem = L::smem_bytes(prm.group);
+    int dev;
+    if (current_device(&dev) != PKV_OK) return PKV_ERR_CUDA;
+    static int occ[kMaxDevices][pkv::kMaxGroup + 1];
+    static bool attr_set[kMaxDevices];
+    int nsm;
+    if (sm_count(&nsm) != PKV_OK) return PKV_ERR_CUDA;
+    int &o = occ[dev][prm.group];
+    if (o == 0) {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!attr_set[dev]) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)L::smem_bytes(pkv::kMaxGroup)) != cudaSuccess)
+                return PKV_ERR_CUDA;
+            attr_set[dev] = true;
+        }
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, pkv::kDecodeThreads, smem) !=
+                cudaSuccess ||
+            n <= 0)
+            return PKV_ERR_CUDA;
+        o = n;
+    }
+    long long grid = (long long)nsm * o;
+    if (grid > items) grid = items;
+    if (grid < 1) grid = 1;
+    // the merge phase waits at a grid barrier: all CTAs must be resident at once
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(pkv::kDecodeThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = merge ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, mk, mv, mq, prm, merge) != cudaSuccess) return PKV_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+template <typename T, int D>
+int dispatch_step(int BS, const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mq,
+                  const pkv::DecodeParams &prm, long long items, int merge, cudaStream_t st) {
+    switch (BS) {
+        case 8: return launch_step<T, D, 8>(mk, mv, mq, prm, items, merge, st);
+        case 16: return launch_step<T, D, 16>(mk, mv, mq, prm, items, merge, st);
+        case 32: return launch_step<T, D, 32>(mk, mv, mq, prm, items, merge, st);
+    }
+    return PKV_ERR_INVALID_ARG;
+}
+
 }  // namespace
 
 extern "C" {
@@ -430,7 +496,7 @@ int pkv_paged_attention_decode(void *out, const void *q, const void *k_cache,
         PKV_OK)
         return rc;
 
-    pkv::DecodeParams prm;
+    pkv::DecodeParams prm{};
     prm.out = out;
     prm.block_tables = block_tables;
     prm.context_lens = context_lens;
@@ -492,6 +558,118 @@ int pkv_paged_attention_decode_noalloc(void *out, const void *q, const void *k_c
                                       max_blocks_per_seq, num_blocks, max_context_len, scale,
                                       dtype, P, scratch, need > 0 ? kNoAllocScratchBytes : 0,
                                       stream);
+}
+
+int pkv_decode_step_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                   int block_size, int max_context_len, int partition_size,
+                                   size_t *bytes_out) {
+    if (!bytes_out) return PKV_ERR_INVALID_ARG;
+    int P;
+    const int rc = check_decode_sizes(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                      max_context_len, partition_size, &P);
+    if (rc != PKV_OK) return rc;
+    *bytes_out = step_ws_bytes(num_seqs, num_heads, head_dim, max_context_len, P);
+    return PKV_OK;
+}
+
+int pkv_paged_decode_step(void *out, const void *q, const void *k_new, const void *v_new,
+                          void *k_cache, void *v_cache, const int32_t *block_tables,
+                          const int32_t *context_lens, int num_seqs, int num_heads,
+                          int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                          int num_blocks, int max_context_len, float scale, int dtype,
+                          int partition_size, void *workspace, size_t workspace_bytes,
+                          pkv_stream_t stream) {
+    int P;
+    int rc = check_decode_sizes(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                max_context_len, partition_size, &P);
+    if (rc != PKV_OK) return rc;
+    if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return PKV_ERR_INVALID_ARG;
+    if (max_blocks_per_seq < 1 || num_blocks < 1) return PKV_ERR_INVALID_ARG;
+    if ((long long)max_context_len > (long long)max_blocks_per_seq * block_size)
+        return PKV_ERR_INVALID_ARG;
+    if ((long long)num_blocks * num_kv_heads * block_size >= INT_MAX) return PKV_ERR_INVALID_ARG;
+    if (num_seqs == 0) return PKV_OK;
+    if (!out || !q || !k_new || !v_new || !k_cache || !v_cache || !block_tables || !context_lens)
+        return PKV_ERR_INVALID_ARG;
+    if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(q, 16) || !aligned(k_new, 16) ||
+        !aligned(v_new, 16) || !aligned(out, 2) || !aligned(block_tables, 4) ||
+        !aligned(context_lens, 4))
+        return PKV_ERR_INVALID_ARG;
+    const size_t need = step_ws_bytes(num_seqs, num_heads, head_dim, max_context_len, P);
+    if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return PKV_ERR_WORKSPACE;
+    const WsLayout ws = ws_layout(num_seqs, num_heads, head_dim, max_context_len, P);
+
+    unsigned int *status;
+    if ((rc = device_status_ptr(&status)) != PKV_OK) return rc;
+    CUtensorMap mk, mv, mq;
+    const long long cache_rows = (long long)num_blocks * num_kv_heads * block_size;
+    const int group = num_heads / num_kv_heads;
+    if ((rc = encode_rows_map(&mk, k_cache, dtype, head_dim, cache_rows, block_size)) != PKV_OK)
+        return rc;
+    if ((rc = encode_rows_map(&mv, v_cache, dtype, head_dim, cache_rows, block_size)) != PKV_OK)
+        return rc;
+    if ((rc = encode_rows_map(&mq, q, dtype, head_dim, (long long)num_seqs * num_heads, group)) !=
+        PKV_OK)
+        return rc;
+
+    pkv::DecodeParams prm{};
+    prm.out = out;
+    prm.block_tables = block_tables;
+    prm.context_lens = context_lens;
+    uint8_t *wsb = static_cast<uint8_t *>(workspace);
+    prm.sched = reinterpret_cast<pkv::SchedHeader *>(wsb);
+    prm.ws_seq_base = ws.total ? reinterpret_cast<int32_t *>(wsb + ws.seq_base) : nullptr;
+    prm.ws_ml = ws.total ? reinterpret_cast<float *>(wsb + ws.ml) : nullptr;
+    prm.ws_o = ws.total ? reinterpret_cast<float *>(wsb + ws.o) : nullptr;
+    prm.status = status;
+    prm.num_seqs = num_seqs;
+    prm.num_heads = num_heads;
+    prm.num_kv_heads = num_kv_heads;
+    prm.group = group;
+    prm.max_blocks_per_seq = max_blocks_per_seq;
+    prm.num_blocks = num_blocks;
+    prm.max_context_len = max_context_len;
+    prm.partition = P;
+    prm.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    prm.k_new = k_new;
+    prm.v_new = v_new;
+    prm.k_cache = k_cache;
+    prm.v_cache = v_cache;
+
+    const int pmax = max_context_len <= P ? 1 : cdiv(max_context_len, P);
+    const long long items = (long long)num_seqs * num_kv_heads * pmax;
+    const int merge = pmax > 1;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (dtype == PKV_BF16)
+        return head_dim == 128
+                   ? dispatch_step<__nv_bfloat16, 128>(block_size, mk, mv, mq, prm, items, merge, st)
+                   : dispatch_step<__nv_bfloat16, 64>(block_size, mk, mv, mq, prm, items, merge, st);
+    return head_dim == 128 ? dispatch_step<__half, 128>(block_size, mk, mv, mq, prm, items, merge, st)
+                           : dispatch_step<__half, 64>(block_size, mk, mv, mq, prm, items, merge, st);
+}
+
+int pkv_device_append(int32_t *block_tables, int32_t *context_lens, const int32_t *free_blocks,
+                      int free_count, int32_t *free_used, int64_t *slots_out, int num_seqs,
+                      int max_blocks_per_seq, int block_size, int num_blocks,
+                      int max_context_len, pkv_stream_t stream) {
+    if (num_seqs < 0 || free_count < 0 || max_blocks_per_seq < 1 || block_size < 1 ||
+        num_blocks < 1 || max_context_len < 0)
+        return PKV_ERR_INVALID_ARG;
+    if ((long long)num_blocks * block_size >= (1LL << 62)) return PKV_ERR_INVALID_ARG;
+    if (!free_used) return PKV_ERR_INVALID_ARG;
+    if (num_seqs > 0 && (!block_tables || !context_lens)) return PKV_ERR_INVALID_ARG;
+    if (free_count > 0 && !free_blocks) return PKV_ERR_INVALID_ARG;
+    if (!aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(free_blocks, 4) ||
+        !aligned(free_used, 4) || !aligned(slots_out, 8))
+        return PKV_ERR_INVALID_ARG;
+    unsigned int *status;
+    int rc;
+    if ((rc = device_status_ptr(&status)) != PKV_OK) return rc;
+    return launch(pkv::device_append_kernel, dim3(1), dim3(pkv::kPlanThreads), 0,
+                  reinterpret_cast<cudaStream_t>(stream), block_tables, context_lens, free_blocks,
+                  free_count, reinterpret_cast<int *>(free_used), slots_out, num_seqs,
+                  max_blocks_per_seq, block_size, num_blocks, max_context_len, status);
 }
 
 int pkv_decode_shared_prefix_workspace_size(int num_seqs, int num_heads, int num_kv_heads,

@@ -1,0 +1,299 @@
+"""GPU parity of the decode step on the device: pkv_device_append against the oracle's
+block-manager model (bit-exact tables, lengths, slots and free-list use, the same
+rules as an in-order host append), and pkv_paged_decode_step against the cache write
+followed by the decode (identical bits) and against the fp64 oracle (4e-3 + 1e-2|ref|),
+with refusals (short free list, full table, length bound, a foreign workspace) leaving
+everything unchanged."""
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_cache_320_b200 as pkv
+from oracle import attention as A
+from oracle import block_manager as BM
+from oracle import cache_ops as C
+from paged_kv_cache_320_b200 import synth
+from tests.gpu_util import assert_close, sampled_oracle, to_bits, to_dev
+from tests.test_gpu_decode import random_case
+
+pytestmark = pytest.mark.gpu
+
+NO_BLOCKS = pkv._binding.STATUS_NO_BLOCKS
+WORKSPACE = pkv._binding.STATUS_WORKSPACE
+
+
+def model_state(rng, nb, bs, mb, nseq, max_len0):
+    """A model allocator with nseq sequences (ids 0..nseq-1), some of them forks of a
+    block-aligned parent, and a free stack shuffled by frees."""
+    order = rng.permutation(nb)
+    m = BM.BlockManagerModel(nb, bs, mb, order)
+    junk = 10_000
+    for j in range(6):                      # sequences that are freed again: shuffle the stack
+        m.append(junk + j, int(rng.integers(1, 3 * bs)))
+    s = 0
+    while s < nseq:
+        if s and rng.random() < 0.2:
+            parent = int(rng.integers(0, s))
+            if m.lens[parent] % bs == 0:
+                assert m.fork(parent, s) == 0
+                s += 1
+                continue
+        n = int(rng.integers(0, max_len0))
+        if rng.random() < 0.25:
+            n = (n // bs) * bs                 # block-aligned: the append takes a new block
+        assert m.append(s, n)[0] == 0
+        s += 1
+    for j in range(6):
+        m.free(junk + j)
+    return m
+
+
+def upload_model(m, nseq):
+    rows = [m.block_table(s) for s in range(nseq)]
+    bt = np.array([r for r, _ in rows], np.int32)
+    lens = np.array([n for _, n in rows], np.int32)
+    return bt, lens
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_device_append_matches_model(cuda_device, seed):
+    rng = np.random.default_rng(900 + seed)
+    bs = int(rng.choice([8, 16, 32]))
+    nseq = int(rng.choice([1, 7, 300, 1500]))
+    mb = 12
+    nb = nseq * mb + 64
+    m = model_state(rng, nb, bs, mb, nseq, (mb - 1) * bs)
+    bt, lens = upload_model(m, nseq)
+    fl = np.array(m.free_list(), np.int32)
+    skip = int(rng.integers(0, 5))            # entries already used by earlier steps
+    fl_dev = np.concatenate([np.full(skip, -1, np.int32), fl])
+    bt_d, lens_d = torch.from_numpy(bt).cuda(), torch.from_numpy(lens).cuda()
+    used = torch.tensor([skip], dtype=torch.int32, device="cuda")
+    slots = torch.full((nseq,), -7, dtype=torch.int64, device="cuda")
+    pkv.pkv_get_device_status(clear=True)
+    pkv.pkv_device_append(bt_d, lens_d, torch.from_numpy(fl_dev).cuda(), used, nb, mb * bs, bs,
+                          slots_out=slots)
+    assert pkv.pkv_get_device_status() == 0
+    exp_slots = []
+    before = len(m.free_stack)
+    for s in range(nseq):
+        st, sl, cw = m.append(s, 1)
+        assert st == 0 and not cw
+        exp_slots.append(sl[0])
+    taken = before - len(m.free_stack)
+    ebt, elens = upload_model(m, nseq)
+    np.testing.assert_array_equal(bt_d.cpu().numpy(), ebt)
+    np.testing.assert_array_equal(lens_d.cpu().numpy(), elens)
+    np.testing.assert_array_equal(slots.cpu().numpy(), np.array(exp_slots, np.int64))
+    assert int(used.item()) == skip + taken
+
+
+@pytest.mark.parametrize("why", ["short list", "table full", "length bound", "bad entry"])
+def test_device_append_refuses_and_changes_nothing(cuda_device, why):
+    rng = np.random.default_rng(77)
+    bs, mb, nseq = 16, 6, 40
+    lens = rng.integers(1, (mb - 1) * bs, nseq).astype(np.int32)
+    lens[::5] = (lens[::5] // bs) * bs + bs     # these take a block
+    bt = rng.integers(0, 500, (nseq, mb)).astype(np.int32)
+    fl = np.arange(600, 700, dtype=np.int32)
+    max_len = mb * bs
+    need = int((lens % bs == 0).sum())
+    if why == "short list":
+        fl = fl[:need - 1]
+    elif why == "table full":
+        lens[3] = mb * bs
+        max_len = mb * bs + 1
+    elif why == "length bound":
+        max_len = int(lens.max())
+    else:
+        fl[need // 2] = 10_000                  # outside the pool of 1000 blocks
+    bt_d, lens_d = torch.from_numpy(bt).cuda(), torch.from_numpy(lens).cuda()
+    used = torch.zeros(1, dtype=torch.int32, device="cuda")
+    slots = torch.full((nseq,), -7, dtype=torch.int64, device="cuda")
+    pkv.pkv_get_device_status(clear=True)
+    pkv.pkv_device_append(bt_d, lens_d, torch.from_numpy(fl).cuda(), used, 1000, max_len, bs,
+                          slots_out=slots)
+    assert pkv.pkv_get_device_status() & NO_BLOCKS
+    np.testing.assert_array_equal(bt_d.cpu().numpy(), bt)
+    np.testing.assert_array_equal(lens_d.cpu().numpy(), lens)
+    assert int(used.item()) == 0
+    assert (slots.cpu().numpy() == -7).all()
+
+
+def step_case(rng, lens, Hq, Hkv, D, BS, dtype):
+    """random_case with post-step lengths; the newest token's row holds the NaN canary
+    (only the step's own write may fill it)."""
+    q, kc, vc, bt, lens, max_len = random_case(rng, lens, Hq, Hkv, D, BS, dtype)
+    slots = np.full(len(lens), -1, np.int64)
+    for s, n in enumerate(lens):
+        if n > 0:
+            slots[s] = int(bt[s, (n - 1) // BS]) * BS + (n - 1) % BS
+            kc[slots[s] // BS, :, slots[s] % BS, :] = synth.CANARY[dtype]
+            vc[slots[s] // BS, :, slots[s] % BS, :] = synth.CANARY[dtype]
+    kn = synth.round_to_bits(rng.standard_normal((len(lens), Hkv, D), dtype=np.float32), dtype)
+    vn = synth.round_to_bits(rng.standard_normal((len(lens), Hkv, D), dtype=np.float32), dtype)
+    return q, kc, vc, bt, lens, max_len, slots, kn, vn
+
+
+def step_ws(q, kc, max_len, P):
+    B, Hq, D = q.shape
+    _, Hkv, BS, _ = kc.shape
+    n = pkv.pkv_decode_step_workspace_size(B, Hq, Hkv, D, BS, max_len, P)
+    return torch.zeros(n, dtype=torch.uint8, device="cuda")
+
+
+@pytest.mark.parametrize("dtype", [synth.F16, synth.BF16])
+@pytest.mark.parametrize("Hq,Hkv,D,BS,P", [(32, 8, 128, 16, 0), (32, 8, 128, 16, 64),
+                                           (64, 8, 128, 32, 128), (8, 8, 64, 8, 64),
+                                           (16, 1, 128, 16, 0), (6, 2, 64, 16, 192),
+                                           (12, 4, 128, 8, 64)])
+def test_step_equals_cache_write_then_decode(cuda_device, dtype, Hq, Hkv, D, BS, P):
+    rng = np.random.default_rng(Hq + 3 * Hkv + D + BS + P + dtype)
+    lens = list(rng.integers(1, 700, 29)) + [0, 1, BS, BS + 1, 64, 65, 512, 513]
+    q, kc, vc, bt, lens, max_len, slots, kn, vn = step_case(rng, lens, Hq, Hkv, D, BS, dtype)
+    qd, knd, vnd = to_dev(q, dtype), to_dev(kn, dtype), to_dev(vn, dtype)
+    btd, lensd = torch.from_numpy(bt).cuda(), torch.from_numpy(lens).cuda()
+    # unfused: cache write, then decode
+    kc1, vc1 = to_dev(kc, dtype), to_dev(vc, dtype)
+    pkv.pkv_reshape_and_cache(knd, vnd, kc1, vc1, torch.from_numpy(slots).cuda())
+    out1 = torch.empty_like(qd)
+    pkv.pkv_paged_attention_decode(out1, qd, kc1, vc1, btd, lensd, max_len, scale=0.11,
+                                   partition_size=P)
+    # fused
+    kc2, vc2 = to_dev(kc, dtype), to_dev(vc, dtype)
+    out2 = torch.empty_like(qd)
+    pkv.pkv_get_device_status(clear=True)
+    pkv.pkv_paged_decode_step(out2, qd, knd, vnd, kc2, vc2, btd, lensd, max_len,
+                              step_ws(q, kc, max_len, P), scale=0.11, partition_size=P)
+    torch.cuda.synchronize()
+    assert pkv.pkv_get_device_status() == 0
+    assert torch.equal(kc1.view(torch.int16), kc2.view(torch.int16))
+    assert torch.equal(vc1.view(torch.int16), vc2.view(torch.int16))
+    assert np.array_equal(to_bits(out1), to_bits(out2))
+    # and against the oracle
+    ek, ev = C.reshape_and_cache(kn, vn, kc, vc, slots)
+    ref = A.paged_decode_attention(q, ek, ev, bt, lens, 0.11, dtype)
+    assert_close(to_bits(out2), ref, dtype, f"P={P}")
+
+
+def test_full_step_append_then_layers_matches_oracle(cuda_device):
+    """Device append, then three layers of decode steps (own caches, shared tables),
+    against the oracle model's append and the fp64 oracle per layer."""
+    rng = np.random.default_rng(31)
+    dtype, Hq, Hkv, D, BS, L = synth.BF16, 16, 4, 128, 16, 3
+    nseq, mb = 24, 40
+    nb = nseq * mb + 16
+    m = model_state(rng, nb, BS, mb, nseq, 30 * BS)
+    bt, lens = upload_model(m, nseq)
+    fl = np.array(m.free_list(), np.int32)
+    for s in range(nseq):
+        m.append(s, 1)
+    ebt, elens = upload_model(m, nseq)
+    eslots = np.array([int(ebt[s, (n - 1) // BS]) * BS + (n - 1) % BS for s, n in enumerate(elens)])
+    max_len = mb * BS
+    btd, lensd = torch.from_numpy(bt).cuda(), torch.from_numpy(lens).cuda()
+    used = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pkv.pkv_get_device_status(clear=True)
+    pkv.pkv_device_append(btd, lensd, torch.from_numpy(fl).cuda(), used, nb, max_len, BS)
+    ws = None
+    for layer in range(L):
+        kc = synth.round_to_bits(rng.standard_normal((nb, Hkv, BS, D), dtype=np.float32), dtype)
+        vc = synth.round_to_bits(rng.standard_normal((nb, Hkv, BS, D), dtype=np.float32), dtype)
+        q = synth.round_to_bits(rng.standard_normal((nseq, Hq, D), dtype=np.float32), dtype)
+        kn = synth.round_to_bits(rng.standard_normal((nseq, Hkv, D), dtype=np.float32), dtype)
+        vn = synth.round_to_bits(rng.standard_normal((nseq, Hkv, D), dtype=np.float32), dtype)
+        kcd, vcd, qd = to_dev(kc, dtype), to_dev(vc, dtype), to_dev(q, dtype)
+        if ws is None:
+            ws = step_ws(q, kc, max_len, 64)
+        out = torch.empty_like(qd)
+        pkv.pkv_paged_decode_step(out, qd, to_dev(kn, dtype), to_dev(vn, dtype), kcd, vcd, btd,
+                                  lensd, max_len, ws, partition_size=64)
+        torch.cuda.synchronize()
+        ek, ev = C.reshape_and_cache(kn, vn, kc, vc, eslots)
+        assert np.array_equal(to_bits(kcd), ek) and np.array_equal(to_bits(vcd), ev)
+        ref = A.paged_decode_attention(q, ek, ev, ebt, elens, 1 / np.sqrt(D), dtype)
+        assert_close(to_bits(out), ref, dtype, f"layer {layer}")
+    assert pkv.pkv_get_device_status() == 0
+    np.testing.assert_array_equal(btd.cpu().numpy(), ebt)
+    np.testing.assert_array_equal(lensd.cpu().numpy(), elens)
+
+
+def test_workspace_reused_across_shapes(cuda_device):
+    """One zero-filled workspace through 12 launches of different batch sizes, grids and
+    partition counts: each launch leaves the header ready for the next."""
+    rng = np.random.default_rng(44)
+    dtype = synth.F16
+    ws = torch.zeros(64 << 20, dtype=torch.uint8, device="cuda")
+    pkv.pkv_get_device_status(clear=True)
+    for i in range(12):
+        nseq = int(rng.choice([1, 5, 64, 300]))
+        P = int(rng.choice([64, 128, 0]))
+        lens = rng.integers(1, 1200, nseq)
+        q, kc, vc, bt, lens, max_len, slots, kn, vn = step_case(rng, lens, 8, 2, 64, 16, dtype)
+        qd = to_dev(q, dtype)
+        out = torch.empty_like(qd)
+        kcd, vcd = to_dev(kc, dtype), to_dev(vc, dtype)
+        pkv.pkv_paged_decode_step(out, qd, to_dev(kn, dtype), to_dev(vn, dtype), kcd, vcd,
+                                  torch.from_numpy(bt).cuda(), torch.from_numpy(lens).cuda(),
+                                  max_len, ws, scale=0.2, partition_size=P)
+        torch.cuda.synchronize()
+        assert pkv.pkv_get_device_status() == 0, i
+        ek, ev = C.reshape_and_cache(kn, vn, kc, vc, slots)
+        ref = A.paged_decode_attention(q, ek, ev, bt, lens, 0.2, dtype)
+        assert_close(to_bits(out), ref, dtype, f"launch {i}")
+
+
+def test_foreign_workspace_is_refused(cuda_device):
+    rng = np.random.default_rng(45)
+    dtype = synth.BF16
+    q, kc, vc, bt, lens, max_len, slots, kn, vn = step_case(rng, [900, 40, 2000], 16, 4, 128, 16,
+                                                            dtype)
+    qd = to_dev(q, dtype)
+    ws = step_ws(q, kc, max_len, 64)
+    ws.fill_(0x5A)                              # never zeroed: not a step workspace
+    out = torch.full_like(qd, 7.0)
+    kcd = to_dev(kc, dtype)
+    pkv.pkv_get_device_status(clear=True)
+    pkv.pkv_paged_decode_step(out, qd, to_dev(kn, dtype), to_dev(vn, dtype), kcd,
+                              to_dev(vc, dtype), torch.from_numpy(bt).cuda(),
+                              torch.from_numpy(lens).cuda(), max_len, ws, partition_size=64)
+    assert pkv.pkv_get_device_status() & WORKSPACE
+    assert (out == 7.0).all()
+    assert np.array_equal(to_bits(kcd), kc)     # no write either
+
+
+@pytest.mark.slow
+def test_gqa_workload_step_full_size(cuda_device):
+    """The GQA workload (256 sequences, 1 layer) as the benchmark's fused step runs it:
+    sampled sequences against the oracle, all of them against the unfused path."""
+    wl = synth.make_workload("llama3_8b_gqa", values_on="cuda")
+    sp = wl.spec
+    dt = sp.dtype
+    seqs = synth.sample_sequences(wl, 8, seed=5)
+    kc, vc = wl.k_cache[0], wl.v_cache[0]
+    ref = sampled_oracle(to_bits(wl.q[0]), kc, vc, wl.block_tables, wl.context_lens, seqs,
+                         wl.scale, dt, to_bits(wl.k_new[0]), to_bits(wl.v_new[0]),
+                         wl.slot_mapping)
+    bt = torch.from_numpy(wl.block_tables).cuda()
+    lens = torch.from_numpy(wl.context_lens).cuda()
+    kc2, vc2 = kc.clone(), vc.clone()
+    out_f = torch.empty_like(wl.q[0])
+    ws = torch.zeros(pkv.pkv_decode_step_workspace_size(wl.num_seqs, sp.num_heads,
+                                                        sp.num_kv_heads, sp.head_dim,
+                                                        sp.block_size, sp.max_len),
+                     dtype=torch.uint8, device="cuda")
+    kn = wl.k_new[0].view(wl.num_seqs, sp.num_kv_heads, sp.head_dim)
+    vn = wl.v_new[0].view(wl.num_seqs, sp.num_kv_heads, sp.head_dim)
+    pkv.pkv_get_device_status(clear=True)
+    pkv.pkv_paged_decode_step(out_f, wl.q[0], kn, vn, kc2, vc2, bt, lens, sp.max_len, ws,
+                              scale=wl.scale)
+    pkv.pkv_reshape_and_cache(wl.k_new[0], wl.v_new[0], kc, vc,
+                              torch.from_numpy(wl.slot_mapping).cuda())
+    out_u = torch.empty_like(wl.q[0])
+    pkv.pkv_paged_attention_decode(out_u, wl.q[0], kc, vc, bt, lens, sp.max_len, scale=wl.scale)
+    torch.cuda.synchronize()
+    assert pkv.pkv_get_device_status() == 0
+    assert torch.equal(kc.view(torch.int16), kc2.view(torch.int16))
+    assert torch.equal(vc.view(torch.int16), vc2.view(torch.int16))
+    assert np.array_equal(to_bits(out_f), to_bits(out_u))
+    assert_close(to_bits(out_f)[seqs], ref, dt, "fused step, sampled")

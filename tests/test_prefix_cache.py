@@ -69,6 +69,9 @@ class ModelAdapter:
     def prefix_stats(self):
         return self.m.prefix_cache_stats()
 
+    def free_list(self):
+        return self.m.free_list()
+
     def table(self, s):
         return self.m.block_table(s)
 
@@ -100,6 +103,9 @@ class LibAdapter:
 
     def prefix_stats(self):
         return self.c.pkv_prefix_cache_stats()
+
+    def free_list(self):
+        return self.c.pkv_alloc_free_list().tolist()
 
     def table(self, s):
         st, tables, lens = self.c.pkv_block_tables([s])
@@ -241,6 +247,14 @@ def random_stream(seed, impl_factory, check_contents=True):
                 assert contents.read(row, n) == SlotContents.expected(want), (seed, s)
     for s in sorted(ids):
         log.append(("table", s, x.table(s)))
+    # the free list is the order the next allocations take
+    fl = list(x.free_list())
+    log.append(("free_list", tuple(fl)))
+    k = min(len(fl), mb)
+    if k:
+        st, slots, _ = x.append(10_000, k * bs)
+        assert st == 0
+        assert [sl // bs for sl in slots[::bs]] == fl[:k]
     return log
 
 
