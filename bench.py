@@ -51,11 +51,12 @@ WORKLOADS = {
 METRIC = "paged decode attention KV-read GB/s (% of B200 HBM peak); decode tokens/s"
 KERNEL_SOURCES = ["paged_kv_cache_320_b200/csrc/decode_kernels.cuh",
                   "paged_kv_cache_320_b200/csrc/pkv_ptx.cuh"]
+STEP_SOURCES = KERNEL_SOURCES + ["paged_kv_cache_320_b200/csrc/step_kernels.cuh"]
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(sources=None) -> str:
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES:
+    for p in sources or KERNEL_SOURCES:
         h.update(open(os.path.join(ROOT, p), "rb").read())
     return h.hexdigest()[:16]
 
@@ -68,16 +69,17 @@ def read_peaks():
     return 6650.0, "fallback"
 
 
-def read_traffic(workload, block_size):
-    """DRAM bytes (read + write) per launch of the decode partition kernel from the
-    committed ncu summary for this workload and block size, only if it was taken on
-    the current kernel source; else None."""
-    path = os.path.join(ROOT, "profiles", f"paged_decode_partition__{workload}.md")
+def read_traffic(workload, block_size, kernel="paged_decode_partition"):
+    """DRAM bytes (read + write) per launch of the decode kernel (the partition kernel,
+    or the fused step kernel) from the committed ncu summary for this workload and block
+    size, only if it was taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}__{workload}.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
     m_hash = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", text)
-    if not m_hash or m_hash.group(1) != kernel_source_hash():
+    sources = STEP_SOURCES if kernel == "paged_decode_step" else KERNEL_SOURCES
+    if not m_hash or m_hash.group(1) != kernel_source_hash(sources):
         return None
     m = re.search(r"traffic_bytes_per_launch\[block_size=%d\]:\s*([0-9]+)" % block_size, text)
     return float(m.group(1)) if m else None
@@ -482,7 +484,8 @@ def gpu_arm(args, rank, world, local_rank):
     read_probe = hbm_read_probe(dev, stream)
     swap = swap_measurement(wl, dev, stream) if args.swap else None
     prefix_cache = prefix_cache_measurement(sp) if args.prefix_cache else None
-    traffic = None if shared or fused else read_traffic(args.workload, sp.block_size)
+    traffic = None if shared else read_traffic(
+        args.workload, sp.block_size, "paged_decode_step" if fused else "paged_decode_partition")
 
     # ---- end to end: host block manager + pinned host buffers through the public API
     e2e = e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, world, decode,
