@@ -397,9 +397,7 @@ def gpu_arm(args, rank, world, local_rank):
             sp.num_kv_heads * sp.head_dim * 4
         roof_layer = roof_layer - kv_layer + uniq
 
-    fused = args.step == "fused"
-    if fused and shared:
-        raise SystemExit("--step fused runs the plain decode")
+    fused = args.step == "fused" and not shared   # the shared-prefix decode has its own launches
     if fused:
         ws = torch.zeros(pkv.pkv_decode_step_workspace_size(
             B, sp.num_heads, sp.num_kv_heads, sp.head_dim, sp.block_size, max_len, P),
@@ -443,7 +441,11 @@ def gpu_arm(args, rank, world, local_rank):
                 e1.record(stream)
                 k1_events.append((e0, e1))
 
-    launches_per_step = L * (1 if fused else 4 if shared else 2 + (1 if pmax > 1 else 0))
+    if fused:
+        launches_per_step = L * pkv.pkv_decode_step_launches(
+            B, sp.num_heads, sp.num_kv_heads, sp.head_dim, sp.block_size, max_len, P)
+    else:
+        launches_per_step = L * (4 if shared else 2 + (1 if pmax > 1 else 0))
     dist = None
     if world > 1:
         import torch.distributed as dist
@@ -484,8 +486,14 @@ def gpu_arm(args, rank, world, local_rank):
     read_probe = hbm_read_probe(dev, stream)
     swap = swap_measurement(wl, dev, stream) if args.swap else None
     prefix_cache = prefix_cache_measurement(sp) if args.prefix_cache else None
-    traffic = None if shared else read_traffic(
-        args.workload, sp.block_size, "paged_decode_step" if fused else "paged_decode_partition")
+    # the dominant kernel: the partition kernel, or for the fused step the write-and-decode
+    # kernel (merge by the reduce kernel) or the step kernel (merge in the same launch)
+    if fused:
+        kernel_key = ("paged_decode_partition_write" if launches_per_step > L
+                      else "paged_decode_step")
+    else:
+        kernel_key = "paged_decode_partition"
+    traffic = None if shared else read_traffic(args.workload, sp.block_size, kernel_key)
 
     # ---- end to end: host block manager + pinned host buffers through the public API
     e2e = e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, world, decode,
@@ -512,7 +520,7 @@ def gpu_arm(args, rank, world, local_rank):
             "sum_context_tokens": int(wl.context_lens.sum()),
             "partition_size": P,
             "decode": args.decode,
-            "step": args.step,
+            "step": "fused" if fused else "separate",
             "kv_bytes_per_step": kv_step,
             "l2": f"inputs larger than L2: {kv_layer / 1e6:.0f} MB of K/V per layer vs 126 MB L2",
             "parallelism": f"replicas x{world}",
@@ -526,7 +534,8 @@ def gpu_arm(args, rank, world, local_rank):
         "gpu_launches": launches_per_step * args.steps,
         "roofline": {
             "kernel": "paged_decode_shared_kernel (+ plan, reduce)" if shared
-            else "paged_decode_step_kernel (cache write + decode + merge)" if fused
+            else f"{kernel_key}_kernel (cache write + decode"
+                 + (" + reduce)" if launches_per_step > L else " + merge)") if fused
             else "paged_decode_partition_kernel (+ reduce)",
             "bound": "hbm",
             "achieved": round(achieved, 1),
@@ -707,18 +716,25 @@ def hbm_read_probe(dev, stream):
 
 def e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, world, decode,
             fused_layer=None):
-    """Each step: the host block manager appends one token to every sequence (one batched
-    call) and exports the tables; the step's inputs (slots, tables, lengths, and q, k_new,
-    v_new of every layer) go host->device from pinned memory on a copy stream, layer by
-    layer, while the kernels of earlier layers run; every layer's output goes back
-    device->host on a second copy stream; the step ends when the last output is on the
-    host. Timed with CUDA events."""
+    """End to end through the public API, software-pipelined two steps deep. Each step the
+    host block manager appends one token to every sequence (one batched call) and its tables
+    are exported and sent up (separate kernels), or the device appends and the host
+    allocator mirrors it (fused step: tables, lengths and free list stay on the GPU). The
+    step's q / k_new / v_new go host->device from pinned memory on a copy stream layer by
+    layer, each layer's kernels start once its inputs have landed, and each layer's output
+    goes device->host on a second copy stream. Inputs and outputs are double-buffered, so
+    step k+1's host work and copies overlap step k's kernels; a buffer set is refilled only
+    after the step that used it two steps earlier is done with it. Timed with CUDA events
+    from before the first step's host work to the last step's output on the host."""
     import torch
     import paged_kv_cache_320_b200 as pkv
 
     sp = wl.spec
-    L, B = sp.num_layers, wl.num_seqs
+    L, B, MB = sp.num_layers, wl.num_seqs, wl.max_blocks_per_seq
+    fused = fused_layer is not None
     mgr = replay_block_manager(wl)
+    ids = np.arange(B, dtype=np.int64)
+    NBUF = 2
     pin = dict(pin_memory=True)
     q_h = torch.empty(tuple(wl.q.shape), dtype=wl.q.dtype, **pin)
     q_h.copy_(wl.q.cpu())
@@ -726,114 +742,115 @@ def e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, worl
     kn_h.copy_(wl.k_new.cpu())
     vn_h = torch.empty(tuple(wl.v_new.shape), dtype=wl.v_new.dtype, **pin)
     vn_h.copy_(wl.v_new.cpu())
-    out_h = torch.empty(tuple(q_h.shape), dtype=q_h.dtype, **pin)
-    slots_h = torch.empty(B, dtype=torch.int64, **pin)
-    bt_h = torch.empty((B, wl.max_blocks_per_seq), dtype=torch.int32, **pin)
-    lens_h = torch.empty(B, dtype=torch.int32, **pin)
-    q_d, kn_d, vn_d = torch.empty_like(wl.q), torch.empty_like(wl.k_new), torch.empty_like(wl.v_new)
-    out_d = torch.empty_like(wl.q)
-    slots_d = torch.empty(B, dtype=torch.int64, device=dev)
-    bt_d = torch.empty((B, wl.max_blocks_per_seq), dtype=torch.int32, device=dev)
-    lens_d = torch.empty(B, dtype=torch.int32, device=dev)
-    ids = np.arange(B, dtype=np.int64)
-    h2d = (q_h.numel() * 2 + kn_h.numel() * 2 + vn_h.numel() * 2 + slots_h.numel() * 8 +
-           bt_h.numel() * 4 + lens_h.numel() * 4)
-    if fused_layer is not None:
-        # tables, lengths and the free list live on the device: uploaded once here, then
-        # updated by pkv_device_append every step (the host allocator mirrors it)
+    out_h = [torch.empty(tuple(q_h.shape), dtype=q_h.dtype, **pin) for _ in range(NBUF)]
+    slots_h = [torch.empty(B, dtype=torch.int64, **pin) for _ in range(NBUF)]
+    bt_h = [torch.empty((B, MB), dtype=torch.int32, **pin) for _ in range(NBUF)]
+    lens_h = [torch.empty(B, dtype=torch.int32, **pin) for _ in range(NBUF)]
+    q_d = [torch.empty_like(wl.q) for _ in range(NBUF)]
+    kn_d = [torch.empty_like(wl.k_new) for _ in range(NBUF)]
+    vn_d = [torch.empty_like(wl.v_new) for _ in range(NBUF)]
+    out_d = [torch.empty_like(wl.q) for _ in range(NBUF)]
+    slots_d = [torch.empty(B, dtype=torch.int64, device=dev) for _ in range(NBUF)]
+    bt_d = [torch.empty((B, MB), dtype=torch.int32, device=dev) for _ in range(NBUF)]
+    lens_d = [torch.empty(B, dtype=torch.int32, device=dev) for _ in range(NBUF)]
+    h2d = q_h.numel() * 2 + kn_h.numel() * 2 + vn_h.numel() * 2
+    if not fused:
+        h2d += B * 8 + B * MB * 4 + B * 4
+    d2h = q_h.numel() * 2
+    if fused:
+        # resident on the GPU: uploaded once, then advanced by pkv_device_append every step
         st, tables, lens = mgr.pkv_block_tables(ids)
-        bt_d.copy_(torch.from_numpy(tables))
-        lens_d.copy_(torch.from_numpy(lens))
+        bt_dev = torch.from_numpy(tables).to(dev)
+        lens_dev = torch.from_numpy(lens).to(dev)
         free_d = torch.from_numpy(mgr.pkv_alloc_free_list()).to(dev)
         used_d = torch.zeros(1, dtype=torch.int32, device=dev)
-        kn3_d = kn_d.view(L, B, sp.num_kv_heads, sp.head_dim)
-        vn3_d = vn_d.view(L, B, sp.num_kv_heads, sp.head_dim)
-        h2d = q_h.numel() * 2 + kn_h.numel() * 2 + vn_h.numel() * 2
-    d2h = out_h.numel() * 2
     copy_in = torch.cuda.Stream(dev)
     copy_out = torch.cuda.Stream(dev)
-    ev_in = [torch.cuda.Event() for _ in range(L)]
-    ev_out = [torch.cuda.Event() for _ in range(L)]
+    def ev():
+        return [torch.cuda.Event() for _ in range(NBUF)]
+
+    ev_in = [[torch.cuda.Event() for _ in range(L)] for _ in range(NBUF)]
+    ev_out = [[torch.cuda.Event() for _ in range(L)] for _ in range(NBUF)]
+    ev_tables, ev_step_done, ev_d2h_done = ev(), ev(), ev()
+    mirror_lens = mgr.pkv_block_tables(ids)[2].astype(np.int64)
     kv_total = [0]
-
-    def one_step_fused():
-        with torch.cuda.stream(copy_in):
-            for l in range(L):
-                kn_d[l].copy_(kn_h[l], non_blocking=True)
-                vn_d[l].copy_(vn_h[l], non_blocking=True)
-                q_d[l].copy_(q_h[l], non_blocking=True)
-                ev_in[l].record(copy_in)
-        pkv.pkv_device_append(bt_d, lens_d, free_d, used_d, wl.num_blocks, max_len,
-                              sp.block_size, stream=stream)
-        for l in range(L):
-            stream.wait_event(ev_in[l])
-            fused_layer(l, out_d[l], q_d[l], kn3_d[l], vn3_d[l], bt_d, lens_d)
-            ev_out[l].record(stream)
-        with torch.cuda.stream(copy_out):
-            for l in range(L):
-                copy_out.wait_event(ev_out[l])
-                out_h[l].copy_(out_d[l], non_blocking=True)
-        # the host allocator mirrors the device append while the GPU works
-        st, done, sl, cows = mgr.pkv_seq_append_batch(ids, 1)
-        if st != 0 or len(cows):
-            raise RuntimeError(f"host mirror append failed ({st})")
-        kv_total[0] += int(mirror_lens[0].sum() + B) * sp.num_kv_heads * sp.head_dim * 4 * L
-        mirror_lens[0] += 1
-        copy_out.synchronize()          # the step's result is on the host
-
-    mirror_lens = [mgr.pkv_block_tables(ids)[2].astype(np.int64)]
+    k = [0]
 
     def one_step():
-        if fused_layer is not None:
-            return one_step_fused()
-        st, done, sl, cows = mgr.pkv_seq_append_batch(ids, 1)
-        if st != 0 or len(cows):
-            raise RuntimeError(f"append failed ({st}) or needed a copy in an unshared workload")
-        st, tables, lens = mgr.pkv_block_tables(ids)
-        slots_h.numpy()[:] = sl[:, 0]
-        bt_h.numpy()[:] = tables
-        lens_h.numpy()[:] = lens
-        kv_total[0] += int(lens.astype(np.int64).sum()) * sp.num_kv_heads * sp.head_dim * 4 * L
-        with torch.cuda.stream(copy_in):
-            slots_d.copy_(slots_h, non_blocking=True)
-            bt_d.copy_(bt_h, non_blocking=True)
-            lens_d.copy_(lens_h, non_blocking=True)
-            for l in range(L):
-                kn_d[l].copy_(kn_h[l], non_blocking=True)
-                vn_d[l].copy_(vn_h[l], non_blocking=True)
-                q_d[l].copy_(q_h[l], non_blocking=True)
-                ev_in[l].record(copy_in)
+        b = k[0] % NBUF
+        k[0] += 1
+        if fused:
+            st, done, sl, cows = mgr.pkv_seq_append_batch(ids, 1)   # host mirror
+            if st != 0 or len(cows):
+                raise RuntimeError(f"host mirror append failed ({st})")
+        else:
+            st, done, sl, cows = mgr.pkv_seq_append_batch(ids, 1)
+            if st != 0 or len(cows):
+                raise RuntimeError(f"append failed ({st}) or needed a copy in an unshared workload")
+            st, tables, lens = mgr.pkv_block_tables(ids)
+            ev_tables[b].synchronize()      # the H2D that last read these host buffers is done
+            slots_h[b].numpy()[:] = sl[:, 0]
+            bt_h[b].numpy()[:] = tables
+            lens_h[b].numpy()[:] = lens
+        mirror_lens[:] += 1
+        kv_total[0] += int(mirror_lens.sum()) * sp.num_kv_heads * sp.head_dim * 4 * L
+        # buffer set b was last used two steps ago: its kernels must be done before refilling
+        copy_in.wait_event(ev_step_done[b])
+        if not fused:
+            with torch.cuda.stream(copy_in):
+                slots_d[b].copy_(slots_h[b], non_blocking=True)
+                bt_d[b].copy_(bt_h[b], non_blocking=True)
+                lens_d[b].copy_(lens_h[b], non_blocking=True)
+            ev_tables[b].record(copy_in)
+        else:
+            pkv.pkv_device_append(bt_dev, lens_dev, free_d, used_d, wl.num_blocks, max_len,
+                                  sp.block_size, stream=stream)
+        stream.wait_event(ev_d2h_done[b])   # out_d[b] has been read back
         for l in range(L):
-            stream.wait_event(ev_in[l])
-            pkv.pkv_reshape_and_cache(kn_d[l], vn_d[l], wl.k_cache[l], wl.v_cache[l], slots_d,
-                                      stream=stream)
-            decode(l, out_d[l], q_d[l], bt_d, lens_d)
-            ev_out[l].record(stream)
-        with torch.cuda.stream(copy_out):
-            for l in range(L):
-                copy_out.wait_event(ev_out[l])
-                out_h[l].copy_(out_d[l], non_blocking=True)
-        copy_out.synchronize()          # the step's result is on the host
+            with torch.cuda.stream(copy_in):
+                kn_d[b][l].copy_(kn_h[l], non_blocking=True)
+                vn_d[b][l].copy_(vn_h[l], non_blocking=True)
+                q_d[b][l].copy_(q_h[l], non_blocking=True)
+            ev_in[b][l].record(copy_in)
+            stream.wait_event(ev_in[b][l])
+            if fused:
+                fused_layer(l, out_d[b][l], q_d[b][l],
+                            kn_d[b][l].view(B, sp.num_kv_heads, sp.head_dim),
+                            vn_d[b][l].view(B, sp.num_kv_heads, sp.head_dim), bt_dev, lens_dev)
+            else:
+                pkv.pkv_reshape_and_cache(kn_d[b][l], vn_d[b][l], wl.k_cache[l], wl.v_cache[l],
+                                          slots_d[b], stream=stream)
+                decode(l, out_d[b][l], q_d[b][l], bt_d[b], lens_d[b])
+            ev_out[b][l].record(stream)
+            copy_out.wait_event(ev_out[b][l])
+            with torch.cuda.stream(copy_out):
+                out_h[b][l].copy_(out_d[b][l], non_blocking=True)
+        ev_step_done[b].record(stream)
+        ev_d2h_done[b].record(copy_out)
 
     for _ in range(args.warmup):
         one_step()
+    torch.cuda.synchronize(dev)
     barrier()
     kv_total[0] = 0
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
+    copy_in.wait_event(t0)
     for _ in range(args.steps):
         one_step()
     stream.wait_stream(copy_out)
+    stream.wait_stream(copy_in)
     t1.record(stream)
+    torch.cuda.synchronize(dev)
     barrier()
     ms = max_over_ranks(t0.elapsed_time(t1)) / args.steps
-    if fused_layer is not None:
+    if fused:
         # the device's tables and lengths must equal the host allocator's after all steps
         st, tables, lens = mgr.pkv_block_tables(ids)
         if (pkv.pkv_get_device_status(stream=stream) != 0 or
-                not np.array_equal(bt_d.cpu().numpy(), tables) or
-                not np.array_equal(lens_d.cpu().numpy(), lens)):
+                not np.array_equal(bt_dev.cpu().numpy(), tables) or
+                not np.array_equal(lens_dev.cpu().numpy(), lens)):
             raise RuntimeError("device append diverged from the host block manager")
     mgr.close()
     value = kv_total[0] / args.steps * world / (ms * 1e-3) / 1e9
@@ -842,12 +859,12 @@ def e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, worl
             "includes": ("device append of one token per sequence (tables, lengths and free "
                          "list resident on the GPU; the host allocator mirrors it with one "
                          "batched call), pinned H2D of every layer's q/k_new/v_new, one fused "
-                         "kernel per layer, D2H of every layer's output"
-                         if fused_layer is not None else
+                         "kernel per layer, D2H of every layer's output; two steps in flight"
+                         if fused else
                          "host block-manager append (one batched call) and table export, pinned "
                          "H2D of slots/tables/lengths and every layer's q/k_new/v_new, all "
-                         "layers' kernels, D2H of every layer's output (copies overlap kernels "
-                         "of other layers)")}
+                         "layers' kernels, D2H of every layer's output; two steps in flight "
+                         "(double-buffered inputs and outputs)")}
 
 
 # ----------------------------------------------------------------------------
@@ -967,9 +984,11 @@ def main():
                     help="also time pkv_swap_blocks (preemption) against a contiguous copy")
     ap.add_argument("--prefix-cache", action="store_true",
                     help="also replay a request stream through the block manager's prefix cache")
-    ap.add_argument("--step", default="separate", choices=["separate", "fused"],
-                    help="fused: one launch per layer (cache write + decode + merge) and the "
-                         "block-table update on the device")
+    ap.add_argument("--step", default="fused", choices=["separate", "fused"],
+                    help="fused (default): the block-table update on the device and the cache "
+                         "write folded into the decode launch (partitions merged in the same "
+                         "launch or by the reduce kernel); separate: cache-write, decode and "
+                         "reduce launches with host-built tables")
     ap.add_argument("--decode", default="plain", choices=["plain", "shared"],
                     help="shared: the shared-prefix-aware decode (shared-prefix workload)")
     ap.add_argument("--batch", type=int, default=0,

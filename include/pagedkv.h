@@ -275,11 +275,15 @@ int pkv_device_append(int32_t *block_tables, int32_t *context_lens, const int32_
  * plus k_new / v_new [num_seqs][num_kv_heads][head_dim] device, 16-byte aligned.
  * Workspace: pkv_decode_step_workspace_size bytes (at least 256), 256-byte aligned, owned
  * by the caller, ZERO-FILLED before its first use and then reused only by this call on one
- * stream (each launch leaves it ready for the next). A workspace whose header is neither
- * zero nor left by this call is refused on the device (PKV_STATUS_WORKSPACE, no output).
- * When some context spans several partitions the launch is cooperative (all CTAs resident)
- * and merges the partitions after a bounded grid barrier (PKV_STATUS_WAIT_TIMEOUT if it
- * gives up). Errors: as pkv_paged_attention_decode. */
+ * stream (each launch leaves it ready for the next). A launch that merges in the step
+ * kernel refuses, on the device, a workspace whose header is neither zero nor left by
+ * these kernels (PKV_STATUS_WORKSPACE, no output).
+ * When some context spans several partitions they are merged either in the same launch
+ * (cooperative, all CTAs resident: after a bounded grid barrier every warp merges
+ * (sequence, head) pairs; PKV_STATUS_WAIT_TIMEOUT if the barrier gives up), chosen when
+ * num_seqs * num_heads is at most the grid's warp count (2 CTAs of 5 warps per SM, at most
+ * one CTA per work item), or else by the partition-merge kernel launched right after
+ * (pkv_decode_step_launches tells which). Errors: as pkv_paged_attention_decode. */
 int pkv_paged_decode_step(void *out, const void *q, const void *k_new, const void *v_new,
                           void *k_cache, void *v_cache, const int32_t *block_tables,
                           const int32_t *context_lens, int num_seqs, int num_heads,
@@ -291,6 +295,12 @@ int pkv_paged_decode_step(void *out, const void *q, const void *k_new, const voi
 int pkv_decode_step_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
                                    int block_size, int max_context_len, int partition_size,
                                    size_t *bytes_out);
+
+/* Kernel launches one pkv_paged_decode_step call with these sizes makes (0, 1 or 2), into
+ * *launches_out. Needs the current device (its SM count). */
+int pkv_decode_step_launches(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                             int block_size, int max_context_len, int partition_size,
+                             int *launches_out);
 
 /* Synchronise `stream`, then read (and with clear != 0 reset) the status word of the
  * current device. *status_out gets the PKV_STATUS_* bits. Returns PKV_OK, or

@@ -85,6 +85,7 @@ def lib() -> ctypes.CDLL:
                                             ctypes.c_float, I, I, P, SZ, P]
         L.pkv_decode_step_workspace_size.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(SZ)]
         L.pkv_device_append.argtypes = [P, P, P, I, P, P, I, I, I, I, I, P]
+        L.pkv_decode_step_launches.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(I)]
         L.pkv_alloc_free_list.argtypes = [P, P, I, ctypes.POINTER(I)]
         L.pkv_alloc_set_prefix_cache.argtypes = [P, I]
         L.pkv_seq_append_tokens.argtypes = [P, I64, P, I, P, P, ctypes.POINTER(I)]
@@ -101,7 +102,7 @@ def lib() -> ctypes.CDLL:
                      "pkv_seq_append", "pkv_seq_append_batch", "pkv_seq_fork", "pkv_seq_free",
                      "pkv_block_tables", "pkv_stats", "pkv_alloc_set_prefix_cache",
                      "pkv_paged_decode_step", "pkv_decode_step_workspace_size", "pkv_device_append",
-                     "pkv_alloc_free_list",
+                     "pkv_alloc_free_list", "pkv_decode_step_launches",
                      "pkv_seq_append_tokens", "pkv_seq_share_prefix", "pkv_prefix_cache_stats"):
             getattr(L, name).restype = I
         _lib = L
@@ -250,6 +251,15 @@ def pkv_decode_step_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, 
                                                 block_size, max_context_len, partition_size,
                                                 ctypes.byref(out)),
            "pkv_decode_step_workspace_size")
+    return out.value
+
+
+def pkv_decode_step_launches(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                             max_context_len, partition_size=0) -> int:
+    out = ctypes.c_int(0)
+    _check(lib().pkv_decode_step_launches(num_seqs, num_heads, num_kv_heads, head_dim,
+                                          block_size, max_context_len, partition_size,
+                                          ctypes.byref(out)), "pkv_decode_step_launches")
     return out.value
 
 

@@ -714,6 +714,21 @@ paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
     decode_items<T, D, BS, false>(&tmap_k, &tmap_v, &tmap_q, prm, sm, 0);
 }
 
+// The same with the decode step's cache write (each sequence's newest token written by
+// the producer before its page is loaded); partitions are merged by
+// paged_decode_reduce_kernel.
+template <typename T, int D, int BS>
+__global__ void __launch_bounds__(kDecodeThreads, 2)
+paged_decode_partition_write_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                                    const __grid_constant__ CUtensorMap tmap_v,
+                                    const __grid_constant__ CUtensorMap tmap_q, DecodeParams prm) {
+    DecodeSmem<D> sm(aligned_dynamic_smem(), prm.group);
+    sm.init_barriers();
+    pdl_wait_and_release();
+    __syncthreads();
+    decode_items<T, D, BS, true>(&tmap_k, &tmap_v, &tmap_q, prm, sm, 0);
+}
+
 // Log-sum-exp merge of n partials (m_j in log2 units, l_j, normalised o_j) of one
 // (sequence, query head), by one warp: lane k owns output dims k*D/32 .. (k+1)*D/32-1.
 //   M = max m_j;  w_j = l_j 2^(m_j - M);  out = sum_j w_j o_j / sum_j w_j

@@ -211,11 +211,12 @@ WsLayout ws_layout(int B, int Hq, int D, int max_len, int P) {
     return w;
 }
 
-template <typename T, int D, int BS>
+template <typename T, int D, int BS, bool kWrite = false>
 int launch_decode(const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mq,
                   const pkv::DecodeParams &prm, long long items_upper, cudaStream_t st) {
     using L = pkv::DecodeLayout<D>;
-    auto kern = pkv::paged_decode_partition_kernel<T, D, BS>;
+    auto kern = kWrite ? pkv::paged_decode_partition_write_kernel<T, D, BS>
+                       : pkv::paged_decode_partition_kernel<T, D, BS>;
     const size_t smem = L::smem_bytes(prm.group);
     int dev;
     if (current_device(&dev) != PKV_OK) return PKV_ERR_CUDA;
@@ -405,15 +406,47 @@ int launch_step(const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap 
     return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
+// Where a decode step with several partitions merges them: in the step launch (one
+// cooperative launch; after a grid barrier every warp of the persistent grid merges
+// pairs) when every (sequence, query head) pair gets a warp of its own, so the merge is
+// one pass; otherwise in paged_decode_reduce_kernel after the write-and-decode kernel
+// (two launches, both with programmatic dependent launch), which runs all pairs at once
+// across the GPU. The grid is two CTAs of kDecodeThreads per SM (the launch bounds and
+// shared-memory plan of the decode kernels), at most one per work item.
+// Built with PKV_STEP_INKERNEL_MERGE=0 the reduce kernel is always used.
+#ifndef PKV_STEP_INKERNEL_MERGE
+#define PKV_STEP_INKERNEL_MERGE 1
+#endif
+
+int step_merges_in_kernel(int B, int Hq, long long items, int pmax, int nsm) {
+    if (!PKV_STEP_INKERNEL_MERGE || pmax <= 1) return 0;
+    const long long grid = std::min<long long>(2LL * nsm, items);
+    return (long long)B * Hq <= grid * (pkv::kDecodeThreads / 32);
+}
+
 template <typename T, int D>
 int dispatch_step(int BS, const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mq,
-                  const pkv::DecodeParams &prm, long long items, int merge, cudaStream_t st) {
-    switch (BS) {
-        case 8: return launch_step<T, D, 8>(mk, mv, mq, prm, items, merge, st);
-        case 16: return launch_step<T, D, 16>(mk, mv, mq, prm, items, merge, st);
-        case 32: return launch_step<T, D, 32>(mk, mv, mq, prm, items, merge, st);
+                  const pkv::DecodeParams &prm, long long items, int merge, int in_kernel,
+                  cudaStream_t st) {
+    if (in_kernel) {
+        switch (BS) {
+            case 8: return launch_step<T, D, 8>(mk, mv, mq, prm, items, merge, st);
+            case 16: return launch_step<T, D, 16>(mk, mv, mq, prm, items, merge, st);
+            case 32: return launch_step<T, D, 32>(mk, mv, mq, prm, items, merge, st);
+        }
+        return PKV_ERR_INVALID_ARG;
     }
-    return PKV_ERR_INVALID_ARG;
+    // the work counter is only used when the reduce kernel follows to re-arm it
+    pkv::DecodeParams p = prm;
+    if (!merge) p.sched = nullptr;
+    int rc = PKV_ERR_INVALID_ARG;
+    switch (BS) {
+        case 8: rc = launch_decode<T, D, 8, true>(mk, mv, mq, p, items, st); break;
+        case 16: rc = launch_decode<T, D, 16, true>(mk, mv, mq, p, items, st); break;
+        case 32: rc = launch_decode<T, D, 32, true>(mk, mv, mq, p, items, st); break;
+    }
+    if (rc == PKV_OK && merge) rc = launch_reduce<T, D>(p, 0, st);
+    return rc;
 }
 
 }  // namespace
@@ -640,13 +673,39 @@ int pkv_paged_decode_step(void *out, const void *q, const void *k_new, const voi
     const int pmax = max_context_len <= P ? 1 : cdiv(max_context_len, P);
     const long long items = (long long)num_seqs * num_kv_heads * pmax;
     const int merge = pmax > 1;
+    int nsm;
+    if ((rc = sm_count(&nsm)) != PKV_OK) return rc;
+    const int ink = step_merges_in_kernel(num_seqs, num_heads, items, pmax, nsm);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (dtype == PKV_BF16)
-        return head_dim == 128
-                   ? dispatch_step<__nv_bfloat16, 128>(block_size, mk, mv, mq, prm, items, merge, st)
-                   : dispatch_step<__nv_bfloat16, 64>(block_size, mk, mv, mq, prm, items, merge, st);
-    return head_dim == 128 ? dispatch_step<__half, 128>(block_size, mk, mv, mq, prm, items, merge, st)
-                           : dispatch_step<__half, 64>(block_size, mk, mv, mq, prm, items, merge, st);
+        return head_dim == 128 ? dispatch_step<__nv_bfloat16, 128>(block_size, mk, mv, mq, prm,
+                                                                   items, merge, ink, st)
+                               : dispatch_step<__nv_bfloat16, 64>(block_size, mk, mv, mq, prm,
+                                                                  items, merge, ink, st);
+    return head_dim == 128
+               ? dispatch_step<__half, 128>(block_size, mk, mv, mq, prm, items, merge, ink, st)
+               : dispatch_step<__half, 64>(block_size, mk, mv, mq, prm, items, merge, ink, st);
+}
+
+int pkv_decode_step_launches(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                             int block_size, int max_context_len, int partition_size,
+                             int *launches_out) {
+    if (!launches_out) return PKV_ERR_INVALID_ARG;
+    int P;
+    int rc = check_decode_sizes(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                max_context_len, partition_size, &P);
+    if (rc != PKV_OK) return rc;
+    if (num_seqs == 0) {
+        *launches_out = 0;
+        return PKV_OK;
+    }
+    const int pmax = max_context_len <= P ? 1 : cdiv(max_context_len, P);
+    const long long items = (long long)num_seqs * num_kv_heads * pmax;
+    int nsm;
+    if ((rc = sm_count(&nsm)) != PKV_OK) return rc;
+    *launches_out =
+        pmax > 1 && !step_merges_in_kernel(num_seqs, num_heads, items, pmax, nsm) ? 2 : 1;
+    return PKV_OK;
 }
 
 int pkv_device_append(int32_t *block_tables, int32_t *context_lens, const int32_t *free_blocks,

@@ -96,7 +96,9 @@ paged_decode_step_kernel(const __grid_constant__ CUtensorMap tmap_k,
         int ok = 1;
         if (hdr) {
             const unsigned a = *(volatile unsigned *)&hdr->armed;
-            ok = a == 0u || a == kStepArmed;
+            // zero-filled, left by this kernel, or re-armed by paged_decode_reduce_kernel
+            // (which leaves the barrier words as this kernel left them)
+            ok = a == 0u || a == kStepArmed || a == kSchedArmed;
             s_gen = *(volatile unsigned *)&hdr->gen;
             if (!ok && blockIdx.x == 0) atomicOr(prm.status, kStatusWorkspace);
         }

@@ -144,10 +144,13 @@ def step_ws(q, kc, max_len, P):
 
 @pytest.mark.parametrize("dtype", [synth.F16, synth.BF16])
 @pytest.mark.parametrize("Hq,Hkv,D,BS,P", [(32, 8, 128, 16, 0), (32, 8, 128, 16, 64),
+                                           (32, 8, 128, 16, 1024), (8, 2, 64, 32, 2048),
                                            (64, 8, 128, 32, 128), (8, 8, 64, 8, 64),
                                            (16, 1, 128, 16, 0), (6, 2, 64, 16, 192),
                                            (12, 4, 128, 8, 64)])
 def test_step_equals_cache_write_then_decode(cuda_device, dtype, Hq, Hkv, D, BS, P):
+    """Several partitions (merged in the step launch) and, with P >= the longest context,
+    one partition (the write-and-decode kernel alone)."""
     rng = np.random.default_rng(Hq + 3 * Hkv + D + BS + P + dtype)
     lens = list(rng.integers(1, 700, 29)) + [0, 1, BS, BS + 1, 64, 65, 512, 513]
     q, kc, vc, bt, lens, max_len, slots, kn, vn = step_case(rng, lens, Hq, Hkv, D, BS, dtype)
