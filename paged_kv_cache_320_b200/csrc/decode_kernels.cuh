@@ -503,15 +503,17 @@ __device__ __forceinline__ void decode_items(const CUtensorMap *tmap_k, const CU
             (sched_mode == 1 ||
              __shfl_sync(0xffffffffu, lane == 0 ? *(volatile unsigned *)&prm.sched->armed : 0u,
                          0) == kSchedArmed);
-        // A ticket is requested one item before it is resolved, so the atomic's
-        // latency overlaps a whole item; the value lives in lane 0 until used.
+        // Every CTA's first item is its index (the grid never exceeds the item count);
+        // later tickets come from the counter, offset by the grid. A ticket is requested
+        // one item before it is resolved, so the atomic's latency overlaps a whole item;
+        // the value lives in lane 0 until used.
         auto request = [&](int static_item) {
             int v = static_item;
-            if (dynamic && lane == 0) v = atomicAdd(&prm.sched->next, 1);
+            if (dynamic && lane == 0) v = (int)gridDim.x + atomicAdd(&prm.sched->next, 1);
             return v;
         };
         auto redeem = [&](int ticket) { return __shfl_sync(0xffffffffu, ticket, 0); };
-        ItemPos cur = walker.find(redeem(request(blockIdx.x)), prm, lane);
+        ItemPos cur = walker.find((int)blockIdx.x, prm, lane);
         int pending = request(cur.item + gridDim.x);
         int cur_ent[kMaxItemBlocks / 32];
         PKV_LOAD_ENTRIES(cur, cur_ent);

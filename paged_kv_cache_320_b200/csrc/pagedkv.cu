@@ -165,12 +165,13 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 int cdiv(int a, int b) { return (a + b - 1) / b; }
 
-// Automatic partition size: 512 tokens for GQA groups up to 4 and 1024 above (the
-// fp32 partials grow with the group), at most 128 blocks, halved while the batch
-// offers fewer than 1024 work items (about 7 per CTA on 148 SMs).
+// Automatic partition size: 512 tokens for GQA groups up to 4 and 2048 above (the
+// fp32 partials grow with the group; measured best at the GQA-4 and GQA-8 workloads),
+// at most 128 blocks, halved while the batch offers fewer than 1024 work items (about
+// 7 per CTA on 148 SMs).
 int auto_partition(int B, int Hq, int Hkv, int BS, int max_len) {
     const int G = Hq / Hkv;
-    int p = G <= 4 ? 512 : 1024;
+    int p = G <= 4 ? 512 : 2048;
     if (p > pkv::kMaxItemBlocks * BS) p = pkv::kMaxItemBlocks * BS;
     while (p > 64 && (long long)B * Hkv * cdiv(max_len, p) < 1024) p /= 2;
     return p;

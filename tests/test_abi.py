@@ -64,7 +64,7 @@ def test_workspace_size_formula():
 
 def test_auto_partition_choices():
     assert pkv.pkv_decode_partition_size(256, 32, 8, 128, 16, 8192) == 512     # G = 4
-    assert pkv.pkv_decode_partition_size(8, 64, 8, 128, 16, 131072) == 1024    # G = 8
+    assert pkv.pkv_decode_partition_size(8, 64, 8, 128, 16, 131072) == 2048    # G = 8
     assert pkv.pkv_decode_partition_size(8, 64, 8, 128, 8, 131072) == 1024     # 128 blocks of 8
     assert pkv.pkv_decode_partition_size(4, 8, 8, 64, 16, 128) == 64          # tiny batch
 
