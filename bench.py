@@ -858,8 +858,9 @@ def e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, worl
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "includes": ("device append of one token per sequence (tables, lengths and free "
                          "list resident on the GPU; the host allocator mirrors it with one "
-                         "batched call), pinned H2D of every layer's q/k_new/v_new, one fused "
-                         "kernel per layer, D2H of every layer's output; two steps in flight"
+                         "batched call), pinned H2D of every layer's q/k_new/v_new, the fused "
+                         "step's launches per layer, D2H of every layer's output; two steps in "
+                         "flight"
                          if fused else
                          "host block-manager append (one batched call) and table export, pinned "
                          "H2D of slots/tables/lengths and every layer's q/k_new/v_new, all "

@@ -104,7 +104,7 @@ struct DecodeLayout {
     static constexpr int kStages = D == 128 ? 3 : 6;
     static constexpr int kRingBytes = kStages * kStageBytes;
     static constexpr int kObufStride = D + 8;                  // floats per merge row
-    static constexpr int kMetaBytes = 1024;                    // infos + barriers + ml
+    static constexpr int kMetaBytes = 1536;    // infos + barriers + ml + item-order table
     __host__ __device__ static constexpr int q_slot_bytes(int group) {
         return (group * kRowBytes + 1023) / 1024 * 1024;
     }
@@ -149,6 +149,7 @@ __device__ __forceinline__ int kv_line(int t, int h) {
 // Position of one work item in the list (lane-uniform).
 struct ItemPos {
     int item, s, hk, p, np, ntok, nst, nblk;
+    int ticket;   // position in the hand-out order (== item in sequence-major order)
     bool valid;
 };
 
@@ -161,6 +162,7 @@ struct ItemWalker {
     __device__ ItemPos find(int item, const DecodeParams &prm, int lane) {
         ItemPos r;
         r.item = item;
+        r.ticket = item;
         r.valid = false;
         const int B = prm.num_seqs, P = prm.partition, Hkv = prm.num_kv_heads;
         for (;;) {
@@ -201,6 +203,141 @@ struct ItemWalker {
         const int rem = item - chunk_base - excl;
         r.hk = rem / r.np;
         r.p = rem - r.hk * r.np;
+        r.ntok = max(0, min(P, len - r.p * P));
+        r.nst = max(1, (r.ntok + kStageTokens - 1) / kStageTokens);
+        r.valid = true;
+        return r;
+    }
+};
+
+// Longest-first order, for small batches of long contexts. Items are handed out by
+// their number of 64-token stages, largest first (within a count: sequence, then KV
+// head, then partition), so the last items any CTA takes are the shortest and the
+// launch drains evenly (long context: 99.3 % instead of 97.9 % of the copy peak). With
+// many sequences the sequence-major order is kept: it measured faster there (GQA, 256
+// sequences: 2.3 % ahead), as concurrently running CTAs then read neighbouring pages of
+// the same sequences and the walker never rescans the batch. An item's stage
+// count is P/64 for every partition but a sequence's last, which holds the remainder.
+// Tickets of stage count c are [first[c], first[c - 1]); first[S] = 0 and first[0] is
+// the item total (S = P/64). The table is built in shared memory by order_table() at
+// the start of the kernel; the walker keeps, per count, a cursor over the sequences
+// (32 at a time), so tickets must reach it in increasing order. Results carry the
+// canonical item number (sequence-major, as ItemWalker numbers them), which indexes
+// the partials.
+constexpr int kMaxStageCount = kMaxItemBlocks * 32 / kStageTokens;   // P <= 128 blocks of 32
+constexpr int kOrderMaxSeqs = 32;   // longest-first order up to this batch size
+
+__device__ __forceinline__ int clamp_ctx(int len, const DecodeParams &prm, bool flag) {
+    if (len < 0 || len > prm.max_context_len) {
+        if (flag) atomicOr(prm.status, kStatusBadLen);
+        len = len < 0 ? 0 : prm.max_context_len;
+    }
+    return len;
+}
+
+// Last partition's stage count of a context of len tokens (1 for an empty context).
+__device__ __forceinline__ int last_stages(int len, int np, int P) {
+    const int ntok = len - (np - 1) * P;
+    return ntok <= 0 ? 1 : (ntok + kStageTokens - 1) / kStageTokens;
+}
+
+// All threads of the CTA: first[0..S] (int[kMaxStageCount + 1]) from the context lengths;
+// cnt is scratch of the same size. Ends with a barrier.
+__device__ __forceinline__ void order_table(const DecodeParams &prm, int *first, int *cnt) {
+    const int P = prm.partition, S = P / kStageTokens, Hkv = prm.num_kv_heads;
+    for (int c = threadIdx.x; c <= S; c += blockDim.x) cnt[c] = 0;
+    __syncthreads();
+    for (int s = threadIdx.x; s < prm.num_seqs; s += blockDim.x) {
+        const int len = clamp_ctx(prm.context_lens[s], prm, blockIdx.x == 0);
+        const int np = max(1, (len + P - 1) / P);
+        if (np > 1) atomicAdd(&cnt[S], (np - 1) * Hkv);
+        atomicAdd(&cnt[last_stages(len, np, P)], Hkv);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int acc = 0;
+        for (int c = S; c >= 1; --c) {
+            first[c] = acc;
+            acc += cnt[c];
+        }
+        first[0] = acc;
+    }
+    __syncthreads();
+}
+
+struct OrderWalker {
+    const int *first;
+    int c = 0;   // stage count whose sequences are being walked (0: none yet)
+    int cs = 0, base = 0, cbase = 0, total = 0, ctotal = 0;
+    int my_len = 0, my_np = 0, my_k = 0, incl = 0, cincl = 0;
+    bool loaded = false;
+
+    __device__ ItemPos find(int ticket, const DecodeParams &prm, int lane) {
+        ItemPos r;
+        r.item = ticket;
+        r.ticket = ticket;
+        r.valid = false;
+        const int B = prm.num_seqs, P = prm.partition, Hkv = prm.num_kv_heads;
+        const int S = P / kStageTokens;
+        if (ticket < 0 || ticket >= first[0]) return r;
+        int cc = c ? c : S;
+        while (cc > 1 && ticket >= first[cc - 1]) --cc;
+        if (cc != c) {   // a new stage count: walk the sequences from the start
+            c = cc;
+            cs = 0;
+            base = 0;
+            cbase = 0;
+            loaded = false;
+        }
+        const int rank = ticket - first[c];
+        for (;;) {
+            if (cs >= B) return r;   // cannot happen while first[] matches the lengths
+            if (!loaded) {
+                const int s = cs + lane;
+                int len = 0, np = 0, k = 0;
+                if (s < B) {
+                    len = clamp_ctx(prm.context_lens[s], prm, false);
+                    np = max(1, (len + P - 1) / P);
+                    const int cl = last_stages(len, np, P);
+                    k = (c == S ? np - 1 : 0) + (cl == c ? 1 : 0);
+                }
+                my_len = len;
+                my_np = np;
+                my_k = k;
+                incl = k * Hkv;
+                cincl = np * Hkv;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                    const int w = __shfl_up_sync(0xffffffffu, cincl, o);
+                    if (lane >= o) {
+                        incl += v;
+                        cincl += w;
+                    }
+                }
+                total = __shfl_sync(0xffffffffu, incl, 31);
+                ctotal = __shfl_sync(0xffffffffu, cincl, 31);
+                loaded = true;
+            }
+            if (rank < base + total) break;
+            base += total;
+            cbase += ctotal;
+            cs += 32;
+            loaded = false;
+        }
+        const unsigned hit = __ballot_sync(0xffffffffu, rank < base + incl);
+        const int ln = __ffs(hit) - 1;
+        const int k = __shfl_sync(0xffffffffu, my_k, ln);
+        const int excl = __shfl_sync(0xffffffffu, incl - my_k * Hkv, ln);
+        const int cexcl = __shfl_sync(0xffffffffu, cincl - my_np * Hkv, ln);
+        const int len = __shfl_sync(0xffffffffu, my_len, ln);
+        r.s = cs + ln;
+        r.np = __shfl_sync(0xffffffffu, my_np, ln);
+        const int rem = rank - base - excl;
+        r.hk = rem / k;
+        const int j = rem - r.hk * k;
+        r.p = (c == S) ? j : r.np - 1;
+        r.item = cbase + cexcl + r.hk * r.np + r.p;
         r.ntok = max(0, min(P, len - r.p * P));
         r.nst = max(1, (r.ntok + kStageTokens - 1) / kStageTokens);
         r.valid = true;
@@ -403,6 +540,7 @@ struct DecodeSmem {
     StageInfo *info;
     uint64_t *full, *empty;
     float2 *ml;   // [4][16]
+    int *order_first, *order_cnt;   // [kMaxStageCount + 1] each
     int qslot_bytes;
     __device__ DecodeSmem(uint8_t *smem, int G) {
         using L = DecodeLayout<D>;
@@ -414,6 +552,8 @@ struct DecodeSmem {
         full = reinterpret_cast<uint64_t *>(info + L::kStages);
         empty = full + L::kStages;
         ml = reinterpret_cast<float2 *>(empty + L::kStages);
+        order_first = reinterpret_cast<int *>(ml + kConsumerWarps * kMaxGroup);
+        order_cnt = order_first + kMaxStageCount + 1;
     }
     __device__ void init_barriers() {
         if (threadIdx.x == 0) {
@@ -466,6 +606,8 @@ __device__ __forceinline__ void decode_items(const CUtensorMap *tmap_k, const CU
     const int Hkv = prm.num_kv_heads;
     const int P = prm.partition;
 
+    if (prm.num_seqs <= kOrderMaxSeqs) order_table(prm, sm.order_first, sm.order_cnt);
+
     if (warp == kConsumerWarps) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
@@ -479,6 +621,9 @@ __device__ __forceinline__ void decode_items(const CUtensorMap *tmap_k, const CU
         const uint64_t kv_policy = l2_evict_normal_policy();
 #endif
         ItemWalker walker;
+        OrderWalker owalk;
+        owalk.first = sm.order_first;
+        const bool ordered = prm.num_seqs <= kOrderMaxSeqs;
         int it = 0;
         bool ok = true;
 
@@ -513,8 +658,9 @@ __device__ __forceinline__ void decode_items(const CUtensorMap *tmap_k, const CU
             return v;
         };
         auto redeem = [&](int ticket) { return __shfl_sync(0xffffffffu, ticket, 0); };
-        ItemPos cur = walker.find((int)blockIdx.x, prm, lane);
-        int pending = request(cur.item + gridDim.x);
+        ItemPos cur = ordered ? owalk.find((int)blockIdx.x, prm, lane)
+                              : walker.find((int)blockIdx.x, prm, lane);
+        int pending = request(cur.ticket + gridDim.x);
         int cur_ent[kMaxItemBlocks / 32];
         PKV_LOAD_ENTRIES(cur, cur_ent);
         while (cur.valid) {
@@ -603,9 +749,10 @@ __device__ __forceinline__ void decode_items(const CUtensorMap *tmap_k, const CU
                 }
                 if (st == 0) {
                     // look one item ahead: position and block-table slice
-                    nxt = walker.find(redeem(pending), prm, lane);
+                    nxt = ordered ? owalk.find(redeem(pending), prm, lane)
+                                  : walker.find(redeem(pending), prm, lane);
                     PKV_LOAD_ENTRIES(nxt, nxt_ent);
-                    if (nxt.valid) pending = request(nxt.item + gridDim.x);
+                    if (nxt.valid) pending = request(nxt.ticket + gridDim.x);
                 }
             }
             if (!ok) break;

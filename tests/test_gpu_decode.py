@@ -261,3 +261,17 @@ def test_many_partitions_merge(cuda_device):
     dtype = synth.F16
     q, kc, vc, bt, lens, max_len = random_case(rng, [5000, 4097, 64, 65, 1], 8, 1, 128, 32, dtype)
     check_case(q, kc, vc, bt, lens, max_len, dtype, 0.088, 64, "P=64 long")
+
+
+@pytest.mark.parametrize("nseq", [31, 32, 33, 1100])
+def test_both_item_orders(cuda_device, nseq):
+    """Up to 32 sequences the work items go out longest first; above, in sequence order.
+    Both orders cover every item once: short, empty and multi-partition contexts mixed."""
+    rng = np.random.default_rng(57 + nseq)
+    dtype = synth.BF16
+    lens = rng.integers(0, 300, nseq)
+    lens[::7] = rng.integers(300, 3000, len(lens[::7]))
+    lens[1] = 0
+    q, kc, vc, bt, lens, max_len = random_case(rng, lens, 8, 2, 64, 16, dtype)
+    for P in (64, 0):
+        check_case(q, kc, vc, bt, lens, max_len, dtype, 0.125, P, f"B={nseq} P={P}")
