@@ -249,8 +249,7 @@ int launch_decode(const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMa
 }
 
 template <typename T, int D>
-int launch_reduce(const pkv::DecodeParams &prm, int pmax, cudaStream_t st) {
-    (void)pmax;
+int launch_reduce(const pkv::DecodeParams &prm, cudaStream_t st) {
     const long long pairs = (long long)prm.num_seqs * prm.num_heads;
     const long long grid = (pairs + pkv::kReduceWarps - 1) / pkv::kReduceWarps;
     return launch(pkv::paged_decode_reduce_kernel<T, D>, dim3((unsigned)grid),
@@ -446,7 +445,7 @@ int dispatch_step(int BS, const CUtensorMap &mk, const CUtensorMap &mv, const CU
         case 16: rc = launch_decode<T, D, 16, true>(mk, mv, mq, p, items, st); break;
         case 32: rc = launch_decode<T, D, 32, true>(mk, mv, mq, p, items, st); break;
     }
-    if (rc == PKV_OK && merge) rc = launch_reduce<T, D>(p, 0, st);
+    if (rc == PKV_OK && merge) rc = launch_reduce<T, D>(p, st);
     return rc;
 }
 
@@ -557,14 +556,14 @@ int pkv_paged_attention_decode(void *out, const void *q, const void *k_cache,
         rc = head_dim == 128 ? dispatch_bs<__nv_bfloat16, 128>(block_size, mk, mv, mq, prm, items, st)
                              : dispatch_bs<__nv_bfloat16, 64>(block_size, mk, mv, mq, prm, items, st);
         if (rc == PKV_OK && pmax > 1)
-            rc = head_dim == 128 ? launch_reduce<__nv_bfloat16, 128>(prm, pmax, st)
-                                 : launch_reduce<__nv_bfloat16, 64>(prm, pmax, st);
+            rc = head_dim == 128 ? launch_reduce<__nv_bfloat16, 128>(prm, st)
+                                 : launch_reduce<__nv_bfloat16, 64>(prm, st);
     } else {
         rc = head_dim == 128 ? dispatch_bs<__half, 128>(block_size, mk, mv, mq, prm, items, st)
                              : dispatch_bs<__half, 64>(block_size, mk, mv, mq, prm, items, st);
         if (rc == PKV_OK && pmax > 1)
-            rc = head_dim == 128 ? launch_reduce<__half, 128>(prm, pmax, st)
-                                 : launch_reduce<__half, 64>(prm, pmax, st);
+            rc = head_dim == 128 ? launch_reduce<__half, 128>(prm, st)
+                                 : launch_reduce<__half, 64>(prm, st);
     }
     return rc;
 }
