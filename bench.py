@@ -189,14 +189,18 @@ def cow_arm(args, rank, world, local_rank):
         if mgr.pkv_seq_append(p, int(n))[0] != 0:
             raise RuntimeError("pool too small for the parents")
 
+    kid_parents = np.repeat(np.array(parents, np.int64), samples)
+    live = [False]
+
     def host_step():
-        for p in range(prompts):
-            for k in range(samples):
-                mgr.pkv_seq_free(p * samples + k)       # (no-op error the first time)
-        for p in range(prompts):
-            for k in range(samples):
-                if mgr.pkv_seq_fork(parents[p], p * samples + k) != 0:
-                    raise RuntimeError("fork failed")
+        if live[0]:
+            st, done = mgr.pkv_seq_free_batch(kids)
+            if st != 0:
+                raise RuntimeError(f"free failed ({st})")
+        st, done = mgr.pkv_seq_fork_batch(kid_parents, kids)
+        if st != 0:
+            raise RuntimeError(f"fork failed ({st})")
+        live[0] = True
         st, done, slots, cows = mgr.pkv_seq_append_batch(kids, 1)
         if st != 0:
             raise RuntimeError(f"append failed ({st})")
@@ -265,45 +269,85 @@ def cow_arm(args, rank, world, local_rank):
     value, tokens_per_s = weak_scaling_rates(kv_step, B, 1, ms_step)
     copy_bytes = n_pairs * 2 * sp.num_kv_heads * sp.block_size * sp.head_dim * 2 * 2
 
-    # end to end: the host block manager re-forks and appends every step
+    # end to end: the host block manager frees, re-forks and appends every step (batched
+    # calls); two steps in flight with double-buffered inputs and outputs, as in e2e_arm
+    NBUF = 2
     pin = dict(pin_memory=True)
     q_h = torch.empty(tuple(q.shape), dtype=dt, **pin); q_h.copy_(q.cpu())
     kn_h = torch.empty(tuple(kn.shape), dtype=dt, **pin); kn_h.copy_(kn.cpu())
     vn_h = torch.empty(tuple(vn.shape), dtype=dt, **pin); vn_h.copy_(vn.cpu())
-    out_h = torch.empty(tuple(q.shape), dtype=dt, **pin)
-    sl_h = torch.empty(B, dtype=torch.int64, **pin)
-    pr_h = torch.empty((n_pairs, 2), dtype=torch.int32, **pin)
-    bt_h = torch.empty(tuple(tables.shape), dtype=torch.int32, **pin)
-    ln_h = torch.empty(B, dtype=torch.int32, **pin)
+    out_h = [torch.empty(tuple(q.shape), dtype=dt, **pin) for _ in range(NBUF)]
+    sl_h = [torch.empty(B, dtype=torch.int64, **pin) for _ in range(NBUF)]
+    pr_h = [torch.empty((n_pairs, 2), dtype=torch.int32, **pin) for _ in range(NBUF)]
+    bt_h = [torch.empty(tuple(tables.shape), dtype=torch.int32, **pin) for _ in range(NBUF)]
+    ln_h = [torch.empty(B, dtype=torch.int32, **pin) for _ in range(NBUF)]
+    q_e = [torch.empty_like(q) for _ in range(NBUF)]
+    kn_e = [torch.empty_like(kn) for _ in range(NBUF)]
+    vn_e = [torch.empty_like(vn) for _ in range(NBUF)]
+    out_e = [torch.empty_like(out) for _ in range(NBUF)]
+    sl_e = [torch.empty_like(slots_d) for _ in range(NBUF)]
+    pr_e = [torch.empty_like(pairs_d) for _ in range(NBUF)]
+    bt_e = [torch.empty_like(bt_d) for _ in range(NBUF)]
+    ln_e = [torch.empty_like(lens_d) for _ in range(NBUF)]
+    copy_in = torch.cuda.Stream(dev)
+    copy_out = torch.cuda.Stream(dev)
+
+    def evs():
+        return [torch.cuda.Event() for _ in range(NBUF)]
+
+    ev_h2d, ev_in, ev_done, ev_d2h = evs(), evs(), evs(), evs()
+    kstep = [0]
 
     def e2e_step():
+        b = kstep[0] % NBUF
+        kstep[0] += 1
         sl, cw, tb, ln = host_step()
         if cw.shape[0] != n_pairs:
             raise RuntimeError("copy-on-write pair count changed")
-        sl_h.numpy()[:] = sl
-        pr_h.numpy()[:] = cw
-        bt_h.numpy()[:] = tb
-        ln_h.numpy()[:] = ln
-        for d_, h_ in ((q, q_h), (kn, kn_h), (vn, vn_h), (slots_d, sl_h), (pairs_d, pr_h),
-                       (bt_d, bt_h), (lens_d, ln_h)):
-            d_.copy_(h_, non_blocking=True)
-        step()
-        out_h.copy_(out, non_blocking=True)
-        stream.synchronize()
+        ev_h2d[b].synchronize()            # the H2D that last read these host buffers is done
+        sl_h[b].numpy()[:] = sl
+        pr_h[b].numpy()[:] = cw
+        bt_h[b].numpy()[:] = tb
+        ln_h[b].numpy()[:] = ln
+        copy_in.wait_event(ev_done[b])     # buffer set b's kernels (two steps ago) are done
+        with torch.cuda.stream(copy_in):
+            for d_, h_ in ((q_e[b], q_h), (kn_e[b], kn_h), (vn_e[b], vn_h), (sl_e[b], sl_h[b]),
+                           (pr_e[b], pr_h[b]), (bt_e[b], bt_h[b]), (ln_e[b], ln_h[b])):
+                d_.copy_(h_, non_blocking=True)
+        ev_h2d[b].record(copy_in)
+        stream.wait_event(ev_h2d[b])
+        stream.wait_event(ev_d2h[b])       # out_e[b] has been read back
+        pkv.pkv_copy_blocks(kp, vp, pr_e[b], sp.num_kv_heads, sp.head_dim, sp.block_size,
+                            cs.num_blocks, dtype_code, stream=stream)
+        pkv.pkv_reshape_and_cache(kn_e[b], vn_e[b], kc, vc, sl_e[b], stream=stream)
+        pkv.pkv_paged_attention_decode(out_e[b], q_e[b], kc, vc, bt_e[b], ln_e[b], max_len,
+                                       scale=1 / math.sqrt(sp.head_dim), partition_size=P,
+                                       workspace=ws, stream=stream)
+        ev_done[b].record(stream)
+        copy_out.wait_event(ev_done[b])
+        with torch.cuda.stream(copy_out):
+            out_h[b].copy_(out_e[b], non_blocking=True)
+        ev_d2h[b].record(copy_out)
 
     for _ in range(args.warmup):
         e2e_step()
+    torch.cuda.synchronize(dev)
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
     a.record(stream)
+    copy_in.wait_event(a)
     for _ in range(args.steps):
         e2e_step()
+    stream.wait_stream(copy_out)
+    stream.wait_stream(copy_in)
     b.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = a.elapsed_time(b) / args.steps
     mgr.close()
     peak, peak_kind = read_peaks()
-    h2d = (q_h.numel() + kn_h.numel() + vn_h.numel()) * 2 + B * 8 + n_pairs * 8 + bt_h.numel() * 4 + B * 4
+    h2d = ((q_h.numel() + kn_h.numel() + vn_h.numel()) * 2 + B * 8 + n_pairs * 8 +
+           bt_h[0].numel() * 4 + B * 4)
+    pmax = max(1, -(-max_len // P))
     return {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
@@ -320,10 +364,11 @@ def cow_arm(args, rank, world, local_rank):
         "clocks": clocks.summary(),
         "e2e": {"value": round(kv_step / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": int(h2d),
-                "d2h_bytes_per_step": int(out_h.numel() * 2),
-                "includes": "host frees, forks and batched appends (copy-on-write pairs), table "
-                            "export, pinned H2D, copy_blocks + cache write + decode, D2H"},
-        "gpu_launches": args.steps * 3,
+                "d2h_bytes_per_step": int(out_h[0].numel() * 2),
+                "includes": "host batched frees, forks and appends (copy-on-write pairs), table "
+                            "export, pinned H2D, copy_blocks + cache write + decode, D2H; two "
+                            "steps in flight (double-buffered inputs and outputs)"},
+        "gpu_launches": args.steps * (3 + (1 if pmax > 1 else 0)),
     }
 
 
@@ -480,6 +525,7 @@ def gpu_arm(args, rank, world, local_rank):
     ms_step = ms_total / args.steps
     value, tokens_per_s = weak_scaling_rates(kv_step, B, world, ms_step)
     k1_avg_ms = statistics.mean(k1_ms)
+    k1_q = np.percentile(np.array(k1_ms), [10, 50, 90]) * 1e3     # this rank's spread, us
     k1_avg_ms = max_over_ranks(k1_avg_ms)
     peak, peak_kind = read_peaks()
     achieved = roof_layer / (k1_avg_ms * 1e-3) / 1e9
@@ -548,6 +594,7 @@ def gpu_arm(args, rank, world, local_rank):
             "algorithmic_bytes_per_launch": roof_layer,
             "hbm_read_probe_gbs": round(read_probe, 1),
             "avg_launch_us": round(k1_avg_ms * 1e3, 2),
+            "launch_us_p10_p50_p90": [round(float(x), 2) for x in k1_q],
         },
     }
     return result

@@ -349,6 +349,14 @@ int pkv_seq_append_batch(pkv_alloc *a, const int64_t *seq_ids, int n, int n_toke
 /* Errors: PKV_ERR_UNKNOWN_SEQ (no parent), PKV_ERR_SEQ_EXISTS (child id in use). */
 int pkv_seq_fork(pkv_alloc *a, int64_t parent, int64_t child);
 
+/* pkv_seq_fork(parents[i], children[i]) and pkv_seq_free(seq_ids[i]) for i = 0, 1, ... in
+ * one call each (host arrays of n ids), for parallel sampling and beam search, which fork
+ * and retire many sequences per step. They stop at the first failing call and return its
+ * status; *n_done_out (may be NULL) = calls that succeeded, whose effects stay. */
+int pkv_seq_fork_batch(pkv_alloc *a, const int64_t *parents, const int64_t *children, int n,
+                       int *n_done_out);
+int pkv_seq_free_batch(pkv_alloc *a, const int64_t *seq_ids, int n, int *n_done_out);
+
 /* The blocks the next allocations would take, in that order (free blocks, then cached
  * blocks nobody holds, least recently released first): at most max_out of them into
  * blocks_out, their count into *n_out. Uploaded to the device, this is the free list

@@ -87,6 +87,8 @@ def lib() -> ctypes.CDLL:
         L.pkv_device_append.argtypes = [P, P, P, I, P, P, I, I, I, I, I, P]
         L.pkv_decode_step_launches.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(I)]
         L.pkv_alloc_free_list.argtypes = [P, P, I, ctypes.POINTER(I)]
+        L.pkv_seq_fork_batch.argtypes = [P, P, P, I, ctypes.POINTER(I)]
+        L.pkv_seq_free_batch.argtypes = [P, P, I, ctypes.POINTER(I)]
         L.pkv_alloc_set_prefix_cache.argtypes = [P, I]
         L.pkv_seq_append_tokens.argtypes = [P, I64, P, I, P, P, ctypes.POINTER(I)]
         L.pkv_seq_share_prefix.argtypes = [P, I64, P, I, ctypes.POINTER(I)]
@@ -102,7 +104,8 @@ def lib() -> ctypes.CDLL:
                      "pkv_seq_append", "pkv_seq_append_batch", "pkv_seq_fork", "pkv_seq_free",
                      "pkv_block_tables", "pkv_stats", "pkv_alloc_set_prefix_cache",
                      "pkv_paged_decode_step", "pkv_decode_step_workspace_size", "pkv_device_append",
-                     "pkv_alloc_free_list", "pkv_decode_step_launches",
+                     "pkv_alloc_free_list", "pkv_decode_step_launches", "pkv_seq_fork_batch",
+                     "pkv_seq_free_batch",
                      "pkv_seq_append_tokens", "pkv_seq_share_prefix", "pkv_prefix_cache_stats"):
             getattr(L, name).restype = I
         _lib = L
@@ -439,6 +442,26 @@ class BlockManager:
 
     def pkv_seq_free(self, seq_id):
         return lib().pkv_seq_free(self._h, int(seq_id))
+
+    def pkv_seq_fork_batch(self, parents, children):
+        """Returns (status, forks done)."""
+        import numpy as np
+        pa = np.ascontiguousarray(parents, dtype=np.int64)
+        ch = np.ascontiguousarray(children, dtype=np.int64)
+        if pa.shape != ch.shape:
+            raise ValueError("parents and children differ in length")
+        done = ctypes.c_int(0)
+        rc = lib().pkv_seq_fork_batch(self._h, pa.ctypes.data, ch.ctypes.data, pa.shape[0],
+                                      ctypes.byref(done))
+        return rc, done.value
+
+    def pkv_seq_free_batch(self, seq_ids):
+        """Returns (status, frees done)."""
+        import numpy as np
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        done = ctypes.c_int(0)
+        rc = lib().pkv_seq_free_batch(self._h, ids.ctypes.data, ids.shape[0], ctypes.byref(done))
+        return rc, done.value
 
     def pkv_block_tables(self, seq_ids):
         """Returns (status, tables int32 [n, MB], lens int32 [n])."""

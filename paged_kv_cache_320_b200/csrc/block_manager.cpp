@@ -333,6 +333,29 @@ int pkv_seq_fork(pkv_alloc *a, int64_t parent, int64_t child) {
     return PKV_OK;
 }
 
+int pkv_seq_fork_batch(pkv_alloc *a, const int64_t *parents, const int64_t *children, int n,
+                       int *n_done_out) {
+    if (n_done_out) *n_done_out = 0;
+    if (!a || n < 0 || (n > 0 && (!parents || !children))) return PKV_ERR_INVALID_ARG;
+    for (int i = 0; i < n; ++i) {
+        const int rc = pkv_seq_fork(a, parents[i], children[i]);
+        if (rc != PKV_OK) return rc;
+        if (n_done_out) *n_done_out = i + 1;
+    }
+    return PKV_OK;
+}
+
+int pkv_seq_free_batch(pkv_alloc *a, const int64_t *seq_ids, int n, int *n_done_out) {
+    if (n_done_out) *n_done_out = 0;
+    if (!a || n < 0 || (n > 0 && !seq_ids)) return PKV_ERR_INVALID_ARG;
+    for (int i = 0; i < n; ++i) {
+        const int rc = pkv_seq_free(a, seq_ids[i]);
+        if (rc != PKV_OK) return rc;
+        if (n_done_out) *n_done_out = i + 1;
+    }
+    return PKV_OK;
+}
+
 int pkv_seq_free(pkv_alloc *a, int64_t seq_id) {
     if (!a) return PKV_ERR_INVALID_ARG;
     auto it = a->seqs.find(seq_id);

@@ -129,3 +129,43 @@ def test_batched_append_equals_appends_in_order(seed):
         assert cows.tolist() == exp_cows
         compare_states(c, m, sorted(m.tables))
     c.close()
+
+
+@pytest.mark.parametrize("seed", range(30))
+def test_batched_fork_and_free_equal_calls_in_order(seed):
+    """pkv_seq_fork_batch / pkv_seq_free_batch == the single calls in order, against the
+    model; on the first failure the calls before it keep their effects."""
+    rng = np.random.default_rng(700 + seed)
+    nb, bs, mb = int(rng.integers(10, 40)), int(rng.choice([2, 4, 8])), int(rng.integers(2, 6))
+    order = rng.permutation(nb)
+    c = BlockManager(nb, bs, mb, order)
+    m = BM.BlockManagerModel(nb, bs, mb, order)
+    for s in range(4):
+        n0 = int(rng.integers(0, bs * 2))
+        assert c.pkv_seq_append(s, n0)[0] == m.append(s, n0)[0]
+    for _ in range(8):
+        k = int(rng.integers(0, 6))
+        if rng.random() < 0.5:
+            parents = [int(x) for x in rng.choice([0, 1, 2, 3, 11, 12], size=k)]
+            children = [int(x) for x in rng.choice([10, 11, 12, 13, 14, 0], size=k)]
+            st, done = c.pkv_seq_fork_batch(parents, children)
+            exp_st, exp_done = 0, 0
+            for pa, ch in zip(parents, children):
+                r = m.fork(pa, ch)
+                if r != 0:
+                    exp_st = r
+                    break
+                exp_done += 1
+        else:
+            ids = [int(x) for x in rng.choice([0, 1, 2, 3, 10, 11, 12, 13, 14], size=k)]
+            st, done = c.pkv_seq_free_batch(ids)
+            exp_st, exp_done = 0, 0
+            for sid in ids:
+                r = m.free(sid)
+                if r != 0:
+                    exp_st = r
+                    break
+                exp_done += 1
+        assert (st, done) == (exp_st, exp_done)
+        compare_states(c, m, sorted(m.tables))
+    c.close()
