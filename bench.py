@@ -954,11 +954,11 @@ def oracle_sample(workload, block_size, nseq, seed=0):
                 scale=1.0 / math.sqrt(sp.head_dim))
 
 
-def oracle_step(smp):
+def oracle_step(smp, nthreads=0):
     from oracle import c_oracle
     kc, vc = c_oracle.reshape_and_cache(smp["kn"], smp["vn"], smp["kc"], smp["vc"], smp["slots"])
     c_oracle.paged_decode_attention(smp["q"], kc, vc, smp["bt"], smp["lens"], smp["scale"],
-                                    smp["spec"].dtype)
+                                    smp["spec"].dtype, nthreads=nthreads)
 
 
 def pick_nseq(workload, block_size):
@@ -979,8 +979,18 @@ def cpu_baseline(args):
         if time.perf_counter() - t0 >= args.cpu_seconds:
             break
     dt = (time.perf_counter() - t0) / n
+    # the same sample on one core, for a fraction of the time
+    t1 = time.perf_counter()
+    n1 = 0
+    while True:
+        oracle_step(smp, nthreads=1)
+        n1 += 1
+        if time.perf_counter() - t1 >= max(1.0, args.cpu_seconds / 4):
+            break
+    dt1 = (time.perf_counter() - t1) / n1
     return {"value": round(smp["kv"] / dt / 1e9, 3), "unit": "GB/s",
             "cores": c_oracle.num_threads(), "kind": "oracle",
+            "value_one_core": round(smp["kv"] / dt1 / 1e9, 4),
             "sample": f"layer 0, first {nseq} sequences ({int(smp['lens'].sum())} context tokens) "
                       f"of the workload: cache write + attention in the plain-C fp64 oracle, "
                       f"{n} repetitions over {args.cpu_seconds:.0f}+ s"}
