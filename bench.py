@@ -458,9 +458,14 @@ def gpu_arm(args, rank, world, local_rank):
 
     def decode(l, out_t, q_t, bt_t, lens_t):
         if shared:
-            pkv.pkv_paged_attention_decode_shared_prefix(
-                out_t, q_t, wl.k_cache[l], wl.v_cache[l], bt_t, lens_t, starts, prefix, max_len,
-                scale=wl.scale, partition_size=P, workspace=ws, stream=stream)
+            # one plan per step serves every layer (the layers share tables and lengths)
+            if l == 0:
+                pkv.pkv_shared_prefix_plan(bt_t, lens_t, starts, prefix, sp.num_heads,
+                                           sp.num_kv_heads, sp.head_dim, sp.block_size, max_len,
+                                           ws, partition_size=P, stream=stream)
+            pkv.pkv_paged_attention_decode_shared_prefix_planned(
+                out_t, q_t, wl.k_cache[l], wl.v_cache[l], bt_t, lens_t, max_len, ws,
+                scale=wl.scale, partition_size=P, stream=stream)
         else:
             pkv.pkv_paged_attention_decode(out_t, q_t, wl.k_cache[l], wl.v_cache[l], bt_t,
                                            lens_t, max_len, scale=wl.scale, partition_size=P,
@@ -490,7 +495,7 @@ def gpu_arm(args, rank, world, local_rank):
         launches_per_step = L * pkv.pkv_decode_step_launches(
             B, sp.num_heads, sp.num_kv_heads, sp.head_dim, sp.block_size, max_len, P)
     else:
-        launches_per_step = L * (4 if shared else 2 + (1 if pmax > 1 else 0))
+        launches_per_step = (3 * L + 1) if shared else L * (2 + (1 if pmax > 1 else 0))
     dist = None
     if world > 1:
         import torch.distributed as dist

@@ -70,7 +70,7 @@ enum pkv_device_status_bits {
     PKV_STATUS_BAD_LEN = 1u << 3,      /* decode: context_len < 0 or above its bound (clamped)  */
     PKV_STATUS_WAIT_TIMEOUT = 1u << 4, /* decode: a pipeline wait exceeded its iteration limit  */
     PKV_STATUS_NO_BLOCKS = 1u << 5,    /* device append: step refused, nothing changed          */
-    PKV_STATUS_WORKSPACE = 1u << 6     /* decode step: workspace header not zero nor its own    */
+    PKV_STATUS_WORKSPACE = 1u << 6     /* workspace not prepared for the call (step, planned)   */
 };
 
 /* Human-readable name of a status code (static string). */
@@ -168,6 +168,29 @@ int pkv_paged_attention_decode_shared_prefix(
     int head_dim, int block_size, int max_blocks_per_seq, int num_blocks, int max_context_len,
     float scale, int dtype, int partition_size, void *workspace, size_t workspace_bytes,
     pkv_stream_t stream);
+
+/* The same call in two parts, so that one plan serves every layer of a step (the plan
+ * depends only on the tables, lengths and groups, which the layers share):
+ * pkv_shared_prefix_plan builds the item list in the workspace (one launch);
+ * pkv_paged_attention_decode_shared_prefix_planned runs the decode and the merge over it
+ * (two launches) and may be called any number of times on the same workspace, ordered on
+ * one stream, while the tables and lengths stay as planned. A planned call whose sizes
+ * (num_seqs, num_heads, num_kv_heads, partition size) differ from the plan's writes nothing
+ * and sets PKV_STATUS_WORKSPACE. Arguments as pkv_paged_attention_decode_shared_prefix;
+ * pkv_paged_attention_decode_shared_prefix is the plan followed by one planned call. */
+int pkv_shared_prefix_plan(const int32_t *block_tables, const int32_t *context_lens,
+                           const int32_t *group_start, const int32_t *prefix_lens, int num_groups,
+                           int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                           int block_size, int max_blocks_per_seq, int max_context_len,
+                           int partition_size, void *workspace, size_t workspace_bytes,
+                           pkv_stream_t stream);
+
+int pkv_paged_attention_decode_shared_prefix_planned(
+    void *out, const void *q, const void *k_cache, const void *v_cache,
+    const int32_t *block_tables, const int32_t *context_lens, int num_seqs, int num_heads,
+    int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int num_blocks,
+    int max_context_len, float scale, int dtype, int partition_size, void *workspace,
+    size_t workspace_bytes, pkv_stream_t stream);
 
 int pkv_decode_shared_prefix_workspace_size(int num_seqs, int num_heads, int num_kv_heads,
                                             int head_dim, int block_size, int max_context_len,

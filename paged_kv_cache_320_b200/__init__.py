@@ -20,6 +20,8 @@ from ._binding import (  # noqa: F401
     pkv_paged_attention_decode,
     pkv_paged_attention_decode_noalloc,
     pkv_paged_attention_decode_shared_prefix,
+    pkv_paged_attention_decode_shared_prefix_planned,
+    pkv_shared_prefix_plan,
     pkv_decode_shared_prefix_workspace_size,
     pkv_reshape_and_cache,
     pkv_swap_blocks,

@@ -87,6 +87,9 @@ def lib() -> ctypes.CDLL:
         L.pkv_device_append.argtypes = [P, P, P, I, P, P, I, I, I, I, I, P]
         L.pkv_decode_step_launches.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(I)]
         L.pkv_alloc_free_list.argtypes = [P, P, I, ctypes.POINTER(I)]
+        L.pkv_shared_prefix_plan.argtypes = [P, P, P, P, I, I, I, I, I, I, I, I, I, P, SZ, P]
+        L.pkv_paged_attention_decode_shared_prefix_planned.argtypes = [
+            P, P, P, P, P, P, I, I, I, I, I, I, I, I, ctypes.c_float, I, I, P, SZ, P]
         L.pkv_seq_fork_batch.argtypes = [P, P, P, I, ctypes.POINTER(I)]
         L.pkv_seq_free_batch.argtypes = [P, P, I, ctypes.POINTER(I)]
         L.pkv_alloc_set_prefix_cache.argtypes = [P, I]
@@ -105,7 +108,8 @@ def lib() -> ctypes.CDLL:
                      "pkv_block_tables", "pkv_stats", "pkv_alloc_set_prefix_cache",
                      "pkv_paged_decode_step", "pkv_decode_step_workspace_size", "pkv_device_append",
                      "pkv_alloc_free_list", "pkv_decode_step_launches", "pkv_seq_fork_batch",
-                     "pkv_seq_free_batch",
+                     "pkv_seq_free_batch", "pkv_shared_prefix_plan",
+                     "pkv_paged_attention_decode_shared_prefix_planned",
                      "pkv_seq_append_tokens", "pkv_seq_share_prefix", "pkv_prefix_cache_stats"):
             getattr(L, name).restype = I
         _lib = L
@@ -296,6 +300,38 @@ def pkv_device_append(block_tables, context_lens, free_blocks, free_used, num_bl
         _ptr(block_tables), _ptr(context_lens), _ptr(free_blocks), free_blocks.numel(),
         _ptr(free_used), _ptr(slots_out), B, block_tables.shape[1], int(block_size),
         int(num_blocks), int(max_context_len), _stream(stream)), "pkv_device_append")
+
+
+def pkv_shared_prefix_plan(block_tables, context_lens, group_start, prefix_lens, num_heads,
+                           num_kv_heads, head_dim, block_size, max_context_len, workspace,
+                           partition_size=0, stream=None):
+    """Build the shared-prefix item list in workspace (uint8 device tensor of
+    pkv_decode_shared_prefix_workspace_size bytes) for every layer of a step."""
+    B = context_lens.numel()
+    _check(lib().pkv_shared_prefix_plan(
+        _ptr(block_tables), _ptr(context_lens), _ptr(group_start), _ptr(prefix_lens),
+        prefix_lens.numel(), B, int(num_heads), int(num_kv_heads), int(head_dim),
+        int(block_size), block_tables.shape[1], int(max_context_len), int(partition_size),
+        _ptr(workspace), workspace.numel(), _stream(stream)), "pkv_shared_prefix_plan")
+
+
+def pkv_paged_attention_decode_shared_prefix_planned(out, q, k_cache, v_cache, block_tables,
+                                                     context_lens, max_context_len, workspace,
+                                                     scale=None, partition_size=0,
+                                                     stream=None):
+    """Decode over the plan pkv_shared_prefix_plan left in workspace."""
+    B, Hq, D = q.shape
+    NB, Hkv, BS, D2 = k_cache.shape
+    if D2 != D or out.shape != q.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    _check(lib().pkv_paged_attention_decode_shared_prefix_planned(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
+        B, Hq, Hkv, D, BS, block_tables.shape[1], NB, int(max_context_len), float(scale),
+        _dtype_code(q), int(partition_size), _ptr(workspace), workspace.numel(), _stream(stream)),
+        "pkv_paged_attention_decode_shared_prefix_planned")
+    return out
 
 
 def pkv_reshape_and_cache(k_new, v_new, k_cache, v_cache, slot_mapping, stream=None):

@@ -318,9 +318,7 @@ int launch_shared_decode(const CUtensorMap &mk, const CUtensorMap &mv,
     return launch(kern, dim3((unsigned)grid), dim3(pkv::kDecodeThreads), smem, st, mk, mv, prm);
 }
 
-template <typename T, int D>
-int launch_shared_path(int BS, const CUtensorMap &mk, const CUtensorMap &mv,
-                       const pkv::SharedParams &prm, cudaStream_t st) {
+int launch_shared_plan(const pkv::SharedParams &prm, cudaStream_t st) {
     const size_t plan_smem =
         prm.num_seqs <= pkv::kPlanSmemSeqs ? (size_t)7 * prm.num_seqs * sizeof(int) : 0;
     {
@@ -336,9 +334,14 @@ int launch_shared_path(int BS, const CUtensorMap &mk, const CUtensorMap &mv,
             attr[dev] = true;
         }
     }
-    int rc = launch(pkv::shared_prefix_plan_kernel, dim3(1), dim3(pkv::kPlanThreads), plan_smem,
-                    st, prm);
-    if (rc != PKV_OK) return rc;
+    return launch(pkv::shared_prefix_plan_kernel, dim3(1), dim3(pkv::kPlanThreads), plan_smem,
+                  st, prm);
+}
+
+template <typename T, int D>
+int launch_shared_decode_reduce(int BS, const CUtensorMap &mk, const CUtensorMap &mv,
+                                const pkv::SharedParams &prm, cudaStream_t st) {
+    int rc;
     switch (BS) {
         case 8: rc = launch_shared_decode<T, D, 8>(mk, mv, prm, st); break;
         case 16: rc = launch_shared_decode<T, D, 16>(mk, mv, prm, st); break;
@@ -350,6 +353,42 @@ int launch_shared_path(int BS, const CUtensorMap &mk, const CUtensorMap &mv,
     const long long grid = (pairs + pkv::kReduceWarps - 1) / pkv::kReduceWarps;
     return launch(pkv::paged_decode_shared_reduce_kernel<T, D>, dim3((unsigned)grid),
                   dim3(pkv::kReduceWarps * 32), 0, st, prm);
+}
+
+// Workspace pointers and sizes of the shared-prefix path (no output, query or scale).
+pkv::SharedParams shared_params(const SharedWs &ws, void *workspace, int num_seqs, int num_heads,
+                                int num_kv_heads, int block_size, int max_blocks_per_seq,
+                                int num_blocks, int max_context_len, int P,
+                                const int32_t *block_tables, const int32_t *context_lens,
+                                unsigned *status) {
+    uint8_t *wsb = static_cast<uint8_t *>(workspace);
+    const size_t ib = align_up((size_t)num_seqs * sizeof(int), 256);
+    pkv::SharedParams prm{};
+    prm.counters = reinterpret_cast<pkv::SharedCounters *>(wsb);
+    prm.np = reinterpret_cast<int *>(wsb + ws.ints);
+    prm.row_base = reinterpret_cast<int *>(wsb + ws.ints + ib);
+    prm.seq_group = reinterpret_cast<int *>(wsb + ws.ints + 2 * ib);
+    prm.gpre = reinterpret_cast<int *>(wsb + ws.ints + 3 * ib);
+    prm.gmin = reinterpret_cast<int *>(wsb + ws.ints + 4 * ib);
+    prm.gmis = reinterpret_cast<int *>(wsb + ws.ints + 5 * ib);
+    prm.ioff = reinterpret_cast<int *>(wsb + ws.ints + 6 * ib);
+    prm.items = reinterpret_cast<pkv::SharedItem *>(wsb + ws.items);
+    prm.ws_ml = reinterpret_cast<float *>(wsb + ws.ml);
+    prm.ws_o = reinterpret_cast<float *>(wsb + ws.o);
+    prm.block_tables = block_tables;
+    prm.context_lens = context_lens;
+    prm.status = status;
+    prm.num_seqs = num_seqs;
+    prm.num_heads = num_heads;
+    prm.num_kv_heads = num_kv_heads;
+    prm.group = num_heads / num_kv_heads;
+    prm.max_blocks_per_seq = max_blocks_per_seq;
+    prm.num_blocks = num_blocks;
+    prm.max_context_len = max_context_len;
+    prm.partition = P;
+    prm.block_size = block_size;
+    prm.max_items = ws.max_items;
+    return prm;
 }
 
 // ---- fused decode step -----------------------------------------------------
@@ -745,31 +784,68 @@ int pkv_decode_shared_prefix_workspace_size(int num_seqs, int num_heads, int num
     return PKV_OK;
 }
 
-int pkv_paged_attention_decode_shared_prefix(
-    void *out, const void *q, const void *k_cache, const void *v_cache,
-    const int32_t *block_tables, const int32_t *context_lens, const int32_t *group_start,
-    const int32_t *prefix_lens, int num_groups, int num_seqs, int num_heads, int num_kv_heads,
-    int head_dim, int block_size, int max_blocks_per_seq, int num_blocks, int max_context_len,
-    float scale, int dtype, int partition_size, void *workspace, size_t workspace_bytes,
-    pkv_stream_t stream) {
-    int P;
+// Host checks shared by the shared-prefix entry points; resolves the partition size.
+static int check_shared(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+                 int max_blocks_per_seq, int num_blocks, int max_context_len, int partition_size,
+                 int *P) {
     int rc = check_decode_sizes(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
-                                max_context_len, partition_size, &P);
+                                max_context_len, partition_size, P);
     if (rc != PKV_OK) return rc;
-    if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_ERR_INVALID_ARG;
-    if (!std::isfinite(scale)) return PKV_ERR_INVALID_ARG;
-    if (max_blocks_per_seq < 1 || num_blocks < 1 || num_groups < 1) return PKV_ERR_INVALID_ARG;
+    if (max_blocks_per_seq < 1 || num_blocks < 1) return PKV_ERR_INVALID_ARG;
     if ((long long)max_context_len > (long long)max_blocks_per_seq * block_size)
         return PKV_ERR_INVALID_ARG;
     if ((long long)num_blocks * num_kv_heads * block_size >= INT_MAX) return PKV_ERR_INVALID_ARG;
+    return PKV_OK;
+}
+
+int pkv_shared_prefix_plan(const int32_t *block_tables, const int32_t *context_lens,
+                           const int32_t *group_start, const int32_t *prefix_lens, int num_groups,
+                           int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                           int block_size, int max_blocks_per_seq, int max_context_len,
+                           int partition_size, void *workspace, size_t workspace_bytes,
+                           pkv_stream_t stream) {
+    int P;
+    int rc = check_shared(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                          max_blocks_per_seq, 1, max_context_len, partition_size, &P);
+    if (rc != PKV_OK) return rc;
     if (num_seqs == 0) return PKV_OK;
-    if (num_groups > num_seqs) return PKV_ERR_INVALID_ARG;
-    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !group_start ||
-        !prefix_lens)
+    if (num_groups < 1 || num_groups > num_seqs) return PKV_ERR_INVALID_ARG;
+    if (!block_tables || !context_lens || !group_start || !prefix_lens) return PKV_ERR_INVALID_ARG;
+    if (!aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(group_start, 4) ||
+        !aligned(prefix_lens, 4))
+        return PKV_ERR_INVALID_ARG;
+    const SharedWs ws =
+        shared_ws_layout(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len, P);
+    if (!workspace || workspace_bytes < ws.total || !aligned(workspace, 16))
+        return PKV_ERR_WORKSPACE;
+    unsigned int *status;
+    if ((rc = device_status_ptr(&status)) != PKV_OK) return rc;
+    pkv::SharedParams prm = shared_params(ws, workspace, num_seqs, num_heads, num_kv_heads,
+                                          block_size, max_blocks_per_seq, 1, max_context_len, P,
+                                          block_tables, context_lens, status);
+    prm.group_start = group_start;
+    prm.prefix_lens = prefix_lens;
+    prm.num_groups = num_groups;
+    return launch_shared_plan(prm, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int pkv_paged_attention_decode_shared_prefix_planned(
+    void *out, const void *q, const void *k_cache, const void *v_cache,
+    const int32_t *block_tables, const int32_t *context_lens, int num_seqs, int num_heads,
+    int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int num_blocks,
+    int max_context_len, float scale, int dtype, int partition_size, void *workspace,
+    size_t workspace_bytes, pkv_stream_t stream) {
+    int P;
+    int rc = check_shared(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                          max_blocks_per_seq, num_blocks, max_context_len, partition_size, &P);
+    if (rc != PKV_OK) return rc;
+    if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return PKV_ERR_INVALID_ARG;
+    if (num_seqs == 0) return PKV_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
         return PKV_ERR_INVALID_ARG;
     if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(q, 4) || !aligned(out, 2) ||
-        !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(group_start, 4) ||
-        !aligned(prefix_lens, 4))
+        !aligned(block_tables, 4) || !aligned(context_lens, 4))
         return PKV_ERR_INVALID_ARG;
     const SharedWs ws =
         shared_ws_layout(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len, P);
@@ -783,45 +859,46 @@ int pkv_paged_attention_decode_shared_prefix(
         return rc;
     if ((rc = encode_rows_map(&mv, v_cache, dtype, head_dim, cache_rows, block_size)) != PKV_OK)
         return rc;
-    uint8_t *wsb = static_cast<uint8_t *>(workspace);
-    const size_t ib = align_up((size_t)num_seqs * sizeof(int), 256);
-    pkv::SharedParams prm;
-    prm.counters = reinterpret_cast<pkv::SharedCounters *>(wsb);
-    prm.np = reinterpret_cast<int *>(wsb + ws.ints);
-    prm.row_base = reinterpret_cast<int *>(wsb + ws.ints + ib);
-    prm.seq_group = reinterpret_cast<int *>(wsb + ws.ints + 2 * ib);
-    prm.gpre = reinterpret_cast<int *>(wsb + ws.ints + 3 * ib);
-    prm.gmin = reinterpret_cast<int *>(wsb + ws.ints + 4 * ib);
-    prm.gmis = reinterpret_cast<int *>(wsb + ws.ints + 5 * ib);
-    prm.ioff = reinterpret_cast<int *>(wsb + ws.ints + 6 * ib);
-    prm.items = reinterpret_cast<pkv::SharedItem *>(wsb + ws.items);
-    prm.ws_ml = reinterpret_cast<float *>(wsb + ws.ml);
-    prm.ws_o = reinterpret_cast<float *>(wsb + ws.o);
+    pkv::SharedParams prm = shared_params(ws, workspace, num_seqs, num_heads, num_kv_heads,
+                                          block_size, max_blocks_per_seq, num_blocks,
+                                          max_context_len, P, block_tables, context_lens, status);
     prm.out = out;
     prm.q = q;
-    prm.block_tables = block_tables;
-    prm.context_lens = context_lens;
-    prm.group_start = group_start;
-    prm.prefix_lens = prefix_lens;
-    prm.status = status;
-    prm.num_groups = num_groups;
-    prm.num_seqs = num_seqs;
-    prm.num_heads = num_heads;
-    prm.num_kv_heads = num_kv_heads;
-    prm.group = num_heads / num_kv_heads;
-    prm.max_blocks_per_seq = max_blocks_per_seq;
-    prm.num_blocks = num_blocks;
-    prm.max_context_len = max_context_len;
-    prm.partition = P;
-    prm.block_size = block_size;
-    prm.max_items = ws.max_items;
     prm.scale_log2 = (float)((double)scale * 1.4426950408889634);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (dtype == PKV_BF16)
-        return head_dim == 128 ? launch_shared_path<__nv_bfloat16, 128>(block_size, mk, mv, prm, st)
-                               : launch_shared_path<__nv_bfloat16, 64>(block_size, mk, mv, prm, st);
-    return head_dim == 128 ? launch_shared_path<__half, 128>(block_size, mk, mv, prm, st)
-                           : launch_shared_path<__half, 64>(block_size, mk, mv, prm, st);
+        return head_dim == 128
+                   ? launch_shared_decode_reduce<__nv_bfloat16, 128>(block_size, mk, mv, prm, st)
+                   : launch_shared_decode_reduce<__nv_bfloat16, 64>(block_size, mk, mv, prm, st);
+    return head_dim == 128 ? launch_shared_decode_reduce<__half, 128>(block_size, mk, mv, prm, st)
+                           : launch_shared_decode_reduce<__half, 64>(block_size, mk, mv, prm, st);
+}
+
+int pkv_paged_attention_decode_shared_prefix(
+    void *out, const void *q, const void *k_cache, const void *v_cache,
+    const int32_t *block_tables, const int32_t *context_lens, const int32_t *group_start,
+    const int32_t *prefix_lens, int num_groups, int num_seqs, int num_heads, int num_kv_heads,
+    int head_dim, int block_size, int max_blocks_per_seq, int num_blocks, int max_context_len,
+    float scale, int dtype, int partition_size, void *workspace, size_t workspace_bytes,
+    pkv_stream_t stream) {
+    int P;
+    int rc = check_shared(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                          max_blocks_per_seq, num_blocks, max_context_len, partition_size, &P);
+    if (rc != PKV_OK) return rc;
+    if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return PKV_ERR_INVALID_ARG;
+    if (num_seqs == 0) return PKV_OK;
+    if (num_groups < 1 || num_groups > num_seqs) return PKV_ERR_INVALID_ARG;
+    if (!out || !q || !k_cache || !v_cache) return PKV_ERR_INVALID_ARG;
+    rc = pkv_shared_prefix_plan(block_tables, context_lens, group_start, prefix_lens, num_groups,
+                                num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                max_blocks_per_seq, max_context_len, P, workspace,
+                                workspace_bytes, stream);
+    if (rc != PKV_OK) return rc;
+    return pkv_paged_attention_decode_shared_prefix_planned(
+        out, q, k_cache, v_cache, block_tables, context_lens, num_seqs, num_heads, num_kv_heads,
+        head_dim, block_size, max_blocks_per_seq, num_blocks, max_context_len, scale, dtype, P,
+        workspace, workspace_bytes, stream);
 }
 
 int pkv_reshape_and_cache(const void *k_new, const void *v_new, void *k_cache, void *v_cache,

@@ -34,10 +34,23 @@ struct SharedItem {
 };
 
 struct SharedCounters {
-    unsigned next;    // next work item
+    unsigned next;    // next work item (0 after the plan and after every reduce)
     int count;        // items in the list
-    int pad[62];
+    int sig[4];       // sizes the plan was built for (kPlanMagic, B, Hq | Hkv << 16, P)
+    int pad[58];
 };
+
+// The plan stays valid for every layer of a step (it depends on the tables, lengths and
+// groups only): decode and reduce launches check that the workspace holds a plan for
+// their sizes and otherwise write nothing and set the workspace status bit.
+constexpr int kPlanMagic = 0x51A9ED01;
+constexpr unsigned kStatusPlanMismatch = 1u << 6;   // the status word's workspace bit
+
+__device__ __forceinline__ bool plan_matches(const SharedCounters *c, int B, int Hq, int Hkv,
+                                             int P) {
+    return c->sig[0] == kPlanMagic && c->sig[1] == B && c->sig[2] == (Hq | (Hkv << 16)) &&
+           c->sig[3] == P;
+}
 
 struct SharedParams {
     SharedCounters *counters;
@@ -294,6 +307,10 @@ shared_prefix_plan_kernel(SharedParams p) {
     if (tid == 0) {
         if (base_items > p.max_items) atomicOr(p.status, kStatusBadLen);
         p.counters->count = min(base_items, p.max_items);
+        p.counters->sig[0] = kPlanMagic;
+        p.counters->sig[1] = B;
+        p.counters->sig[2] = p.num_heads | (Hkv << 16);
+        p.counters->sig[3] = P;
     }
 }
 
@@ -329,6 +346,11 @@ paged_decode_shared_kernel(const __grid_constant__ CUtensorMap tmap_k,
     }
     pdl_wait_and_release();
     __syncthreads();
+    // every CTA reads the same signature (nothing writes it during this launch)
+    if (!plan_matches(prm.counters, prm.num_seqs, prm.num_heads, Hkv, prm.partition)) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(prm.status, kStatusPlanMismatch);
+        return;
+    }
 
     if (warp == kConsumerWarps) {
         // ------------------------------------------------------------ producer
@@ -525,6 +547,11 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kReduceWarps * 32)
 paged_decode_shared_reduce_kernel(SharedParams prm) {
     pdl_wait_and_release();
+    if (!plan_matches(prm.counters, prm.num_seqs, prm.num_heads, prm.num_kv_heads, prm.partition))
+        return;
+    // the decode launch has finished (stream order): re-arm the work counter for the next
+    // decode over the same plan
+    if (blockIdx.x == 0 && threadIdx.x == 0) prm.counters->next = 0u;
     const int lane = threadIdx.x & 31;
     const int pair = blockIdx.x * kReduceWarps + (threadIdx.x >> 5);
     if (pair >= prm.num_seqs * prm.num_heads) return;

@@ -157,3 +157,67 @@ def test_large_batch_plans_in_workspace_scratch(cuda_device):
     got = run_shared(q, kc, vc, bt, lens, starts, pre, max_len, dtype, 0.125)
     assert pkv.pkv_get_device_status() == 0
     assert_close(got, ref, dtype, "6400 sequences")
+
+
+def test_one_plan_serves_several_layers(cuda_device):
+    """pkv_shared_prefix_plan once, then the planned decode for three layers (own caches
+    and queries, shared tables): each equals the one-call path bit for bit and the oracle."""
+    rng = np.random.default_rng(63)
+    dtype = synth.BF16
+    Hq, Hkv, D, BS = 32, 8, 128, 16
+    q0, kc0, vc0, bt, lens, starts, pre, max_len = grouped_case(rng, [8, 3, 5], [10, 2, 6], 120,
+                                                                Hq, Hkv, D, BS, dtype)
+    canary = kc0 == synth.CANARY[dtype]
+    layers = []
+    for _ in range(3):
+        kc = synth.round_to_bits(rng.standard_normal(kc0.shape, dtype=np.float32), dtype)
+        vc = synth.round_to_bits(rng.standard_normal(vc0.shape, dtype=np.float32), dtype)
+        kc[canary] = synth.CANARY[dtype]
+        vc[canary] = synth.CANARY[dtype]
+        q = synth.round_to_bits(rng.standard_normal(q0.shape, dtype=np.float32), dtype)
+        layers.append((q, kc, vc))
+    btd, lensd = torch.from_numpy(bt).cuda(), torch.from_numpy(lens).cuda()
+    startsd = torch.from_numpy(np.asarray(starts, np.int32)).cuda()
+    pred = torch.from_numpy(np.asarray(pre, np.int32)).cuda()
+    ws = torch.empty(pkv.pkv_decode_shared_prefix_workspace_size(len(lens), Hq, Hkv, D, BS,
+                                                                 max_len, 64),
+                     dtype=torch.uint8, device="cuda")
+    pkv.pkv_get_device_status(clear=True)
+    pkv.pkv_shared_prefix_plan(btd, lensd, startsd, pred, Hq, Hkv, D, BS, max_len, ws,
+                               partition_size=64)
+    for i, (q, kc, vc) in enumerate(layers):
+        qd, kcd, vcd = to_dev(q, dtype), to_dev(kc, dtype), to_dev(vc, dtype)
+        out = torch.empty_like(qd)
+        pkv.pkv_paged_attention_decode_shared_prefix_planned(out, qd, kcd, vcd, btd, lensd,
+                                                             max_len, ws, scale=0.1,
+                                                             partition_size=64)
+        torch.cuda.synchronize()
+        got = to_bits(out)
+        one_call = run_shared(q, kc, vc, bt, lens, starts, pre, max_len, dtype, 0.1, 64)
+        assert np.array_equal(got, one_call), f"layer {i}"
+        ref = A.paged_decode_attention(q, kc, vc, bt, lens, 0.1, dtype)
+        assert_close(got, ref, dtype, f"layer {i}")
+    assert pkv.pkv_get_device_status() == 0
+
+
+def test_planned_call_with_other_sizes_writes_nothing(cuda_device):
+    rng = np.random.default_rng(64)
+    dtype = synth.F16
+    q, kc, vc, bt, lens, starts, pre, max_len = grouped_case(rng, [4, 4], [3, 5], 60, 16, 4, 64,
+                                                             16, dtype)
+    btd, lensd = torch.from_numpy(bt).cuda(), torch.from_numpy(lens).cuda()
+    ws = torch.empty(max(pkv.pkv_decode_shared_prefix_workspace_size(len(lens), 16, 4, 64, 16,
+                                                                     max_len, p)
+                         for p in (64, 128)), dtype=torch.uint8, device="cuda")
+    pkv.pkv_shared_prefix_plan(btd, lensd, torch.from_numpy(np.asarray(starts, np.int32)).cuda(),
+                               torch.from_numpy(np.asarray(pre, np.int32)).cuda(), 16, 4, 64, 16,
+                               max_len, ws, partition_size=128)
+    qd = to_dev(q, dtype)
+    out = torch.full_like(qd, 3.0)
+    pkv.pkv_get_device_status(clear=True)
+    # planned for 128-token partitions, called with 64
+    pkv.pkv_paged_attention_decode_shared_prefix_planned(out, qd, to_dev(kc, dtype),
+                                                         to_dev(vc, dtype), btd, lensd, max_len,
+                                                         ws, partition_size=64)
+    assert pkv.pkv_get_device_status() & pkv._binding.STATUS_WORKSPACE
+    assert (out == 3.0).all()
