@@ -54,8 +54,8 @@ enum pkv_status {
     PKV_ERR_UNKNOWN_SEQ = -3,   /* allocator: no sequence with that id                    */
     PKV_ERR_SEQ_EXISTS = -4,    /* allocator: fork target id already in use                */
     PKV_ERR_TABLE_FULL = -5,    /* allocator: table would exceed max_blocks_per_seq        */
-    PKV_ERR_BAD_INDEX = -6,     /* device status: a kernel met an out-of-pool index       */
-    PKV_ERR_TIMEOUT = -7,       /* device status: a bounded wait in a kernel gave up      */
+    PKV_ERR_BAD_INDEX = -6,     /* for callers that turn status-word bits into codes: an   */
+    PKV_ERR_TIMEOUT = -7,       /* out-of-pool index / a wait that gave up (not returned)  */
     PKV_ERR_CUDA = -8,          /* a CUDA runtime call failed                             */
     PKV_ERR_WORKSPACE = -9      /* workspace pointer NULL or smaller than required        */
 };
@@ -90,7 +90,7 @@ const char *pkv_status_string(int code);
  * Long contexts are split into partitions of `partition_size` tokens (a multiple of
  * 64, at most 128 blocks; 0 = automatic) whose partial results are merged exactly
  * (log-sum-exp) by a second kernel; that needs `workspace` of at least
- * pkv_decode_workspace_size(...) bytes of device memory (256-byte aligned), which the
+ * pkv_decode_workspace_size(...) bytes of device memory (16-byte aligned), which the
  * caller owns and may reuse between calls that are ordered on one stream.
  *
  * Limits: head_dim in {64, 128}; block_size in {8, 16, 32}; 1 <= G <= 16;
