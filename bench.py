@@ -536,6 +536,9 @@ def gpu_arm(args, rank, world, local_rank):
     achieved = roof_layer / (k1_avg_ms * 1e-3) / 1e9
     read_probe = hbm_read_probe(dev, stream)
     swap = swap_measurement(wl, dev, stream) if args.swap else None
+    mem_mgr = replay_block_manager(wl)
+    memory = memory_utilisation(wl, mem_mgr)
+    mem_mgr.close()
     prefix_cache = prefix_cache_measurement(sp) if args.prefix_cache else None
     # the dominant kernel: the partition kernel, or for the fused step the write-and-decode
     # kernel (merge by the reduce kernel) or the step kernel (merge in the same launch)
@@ -578,6 +581,7 @@ def gpu_arm(args, rank, world, local_rank):
         },
         "tokens_per_s": round(tokens_per_s, 1),
         "pct_of_hbm_peak": round(100 * value / world / peak, 2),
+        "memory_utilisation": memory,
         **({"swap_blocks": swap} if swap else {}),
         **({"prefix_cache": prefix_cache} if prefix_cache else {}),
         "clocks": clocks.summary(),
@@ -695,6 +699,28 @@ def prefix_cache_measurement(sp, requests=1024, concurrency=128, decode_len=64, 
                     "admit_us_per_request": round(1e6 * admit_s / len(reqs), 2)}
         mgr.close()
     return out
+
+
+def memory_utilisation(wl, mgr):
+    """KV-pool utilisation of the workload's state (\"vLLM / PagedAttention — 分页 KV Cache
+    分析\" §4.2: tokens stored / (blocks x page size)): logical tokens over held blocks from
+    the block manager (above 1 when blocks are shared), the same with each shared slot
+    counted once, and a contiguous pre-allocation of max_len per sequence for contrast."""
+    sp = wl.spec
+    bs = sp.block_size
+    free, held, tokens, util = mgr.pkv_stats()
+    lens = wl.context_lens.astype(np.int64)
+    slots = []
+    for s, n in enumerate(lens):
+        nblk = -(-int(n) // bs)
+        blocks = wl.block_tables[s, :nblk].astype(np.int64)
+        slots.append((blocks[:, None] * bs + np.arange(bs)).reshape(-1)[:int(n)])
+    distinct = int(np.unique(np.concatenate(slots)).size) if slots else 0
+    max_len = int(sp.max_len)
+    return {"logical": round(util, 4),
+            "physical": round(distinct / (held * bs), 4) if held else 0.0,
+            "contiguous_prealloc": round(float(lens.sum()) / (len(lens) * max_len), 4),
+            "held_blocks": held, "block_size": bs}
 
 
 def swap_measurement(wl, dev, stream, budget=512 << 20, reps=5):

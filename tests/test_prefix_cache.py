@@ -327,3 +327,29 @@ def test_bench_request_stream_hits_every_repeated_prompt():
     on = r["cache_on"]["prefill_tokens_cached"]
     assert on >= (64 - first_uses) * full
     assert r["cache_on"]["peak_blocks_held"] < r["cache_off"]["peak_blocks_held"]
+
+
+def test_bench_memory_utilisation_matches_the_oracle():
+    """The benchmark's pool utilisation equals the oracle's closed forms: paged
+    Σ len / (Σ⌈len/bs⌉·bs) and contiguous Σ len / (B·max_len) on an unshared workload;
+    with shared prefixes each shared slot counts once in the physical form."""
+    import bench
+    from oracle import utilisation as U
+    from paged_kv_cache_320_b200 import synth
+    wl = synth.make_workload("llama7b_mha", values_on="none")
+    mgr = bench.replay_block_manager(wl)
+    m = bench.memory_utilisation(wl, mgr)
+    mgr.close()
+    lens = wl.context_lens
+    assert m["logical"] == pytest.approx(U.paged_utilisation(lens, 16), abs=1e-4)
+    assert m["physical"] == m["logical"]
+    assert m["contiguous_prealloc"] == pytest.approx(
+        U.contiguous_utilisation(lens, wl.spec.max_len), abs=1e-4)
+    wl = synth.make_workload("shared_prefix", values_on="none")
+    mgr = bench.replay_block_manager(wl)
+    m = bench.memory_utilisation(wl, mgr)
+    mgr.close()
+    sp = wl.spec
+    unique = sp.prompts * sp.prefix + int((wl.context_lens - sp.prefix).sum())
+    assert m["physical"] == pytest.approx(unique / (m["held_blocks"] * 16), abs=1e-4)
+    assert m["logical"] > 1.0
