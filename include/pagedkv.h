@@ -88,7 +88,7 @@ const char *pkv_status_string(int code);
  * A zero-length context gives out = 0. Slots past context_lens[s] in the last block
  * are never used (any bits, NaN included, are ignored).
  * Long contexts are split into partitions of `partition_size` tokens (a multiple of
- * 64, at most 128 blocks; 0 = automatic) whose partial results are merged exactly
+ * 64, at most 256 blocks; 0 = automatic) whose partial results are merged exactly
  * (log-sum-exp) by a second kernel; that needs `workspace` of at least
  * pkv_decode_workspace_size(...) bytes of device memory (16-byte aligned), which the
  * caller owns and may reuse between calls that are ordered on one stream.

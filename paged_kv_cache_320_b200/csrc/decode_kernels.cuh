@@ -45,7 +45,7 @@ constexpr int kStageTokens = 64;
 constexpr int kConsumerWarps = 4;
 constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
 constexpr int kMaxGroup = 16;               // query heads per KV head (MMA M)
-constexpr int kMaxItemBlocks = 128;         // block-table entries held per item (4 per lane)
+constexpr int kMaxItemBlocks = 256;         // block-table entries held per item (8 per lane)
 constexpr uint32_t kWaitLimit = 1u << 22;   // polls before a pipeline wait gives up
 
 constexpr unsigned kStatusBadSlot = 1u << 0;
@@ -104,7 +104,7 @@ struct DecodeLayout {
     static constexpr int kStages = D == 128 ? 3 : 6;
     static constexpr int kRingBytes = kStages * kStageBytes;
     static constexpr int kObufStride = D + 8;                  // floats per merge row
-    static constexpr int kMetaBytes = 1536;    // infos + barriers + ml + item-order table
+    static constexpr int kMetaBytes = 2048;    // infos + barriers + ml + item-order table
     __host__ __device__ static constexpr int q_slot_bytes(int group) {
         return (group * kRowBytes + 1023) / 1024 * 1024;
     }
@@ -224,7 +224,7 @@ struct ItemWalker {
 // (32 at a time), so tickets must reach it in increasing order. Results carry the
 // canonical item number (sequence-major, as ItemWalker numbers them), which indexes
 // the partials.
-constexpr int kMaxStageCount = kMaxItemBlocks * 32 / kStageTokens;   // P <= 128 blocks of 32
+constexpr int kMaxStageCount = kMaxItemBlocks * 32 / kStageTokens;   // P <= 256 blocks of 32
 constexpr int kOrderMaxSeqs = 32;   // longest-first order up to this batch size
 
 __device__ __forceinline__ int clamp_ctx(int len, const DecodeParams &prm, bool flag) {

@@ -167,7 +167,7 @@ int cdiv(int a, int b) { return (a + b - 1) / b; }
 
 // Automatic partition size: 512 tokens for GQA groups up to 4 and 2048 above (the
 // fp32 partials grow with the group; measured best at the GQA-4 and GQA-8 workloads),
-// at most 128 blocks, halved while the batch offers fewer than 1024 work items (about
+// at most 256 blocks, halved while the batch offers fewer than 1024 work items (about
 // 7 per CTA on 148 SMs).
 int auto_partition(int B, int Hq, int Hkv, int BS, int max_len) {
     const int G = Hq / Hkv;

@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol():
     (4, 8, 3, 64, 16, 128, 0),       # Hq % Hkv
     (4, 64, 2, 64, 16, 128, 0),      # group > 16
     (4, 8, 8, 64, 16, 128, 100),     # partition not a multiple of 64
-    (4, 8, 8, 64, 8, 128, 2048),     # partition > 128 blocks
+    (4, 8, 8, 64, 8, 128, 4096),     # partition > 256 blocks
     (-1, 8, 8, 64, 16, 128, 0),      # negative batch
 ])
 def test_decode_size_checks(args):
@@ -65,7 +65,10 @@ def test_workspace_size_formula():
 def test_auto_partition_choices():
     assert pkv.pkv_decode_partition_size(256, 32, 8, 128, 16, 8192) == 512     # G = 4
     assert pkv.pkv_decode_partition_size(8, 64, 8, 128, 16, 131072) == 2048    # G = 8
-    assert pkv.pkv_decode_partition_size(8, 64, 8, 128, 8, 131072) == 1024     # 128 blocks of 8
+    assert pkv.pkv_decode_partition_size(8, 64, 8, 128, 8, 131072) == 2048     # 256 blocks of 8
+    assert pkv.pkv_decode_partition_size(8, 64, 8, 128, 16, 131072, 4096) == 4096  # 256 of 16
+    with pytest.raises(pkv.PagedKVError):
+        pkv.pkv_decode_partition_size(8, 64, 8, 128, 8, 131072, 4096)            # 512 of 8
     assert pkv.pkv_decode_partition_size(4, 8, 8, 64, 16, 128) == 64          # tiny batch
 
 

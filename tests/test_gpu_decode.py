@@ -275,3 +275,14 @@ def test_both_item_orders(cuda_device, nseq):
     q, kc, vc, bt, lens, max_len = random_case(rng, lens, 8, 2, 64, 16, dtype)
     for P in (64, 0):
         check_case(q, kc, vc, bt, lens, max_len, dtype, 0.125, P, f"B={nseq} P={P}")
+
+
+@pytest.mark.parametrize("BS,P", [(8, 2048), (16, 4096)])
+def test_items_of_256_blocks(cuda_device, BS, P):
+    """Partitions of the largest size an item takes (256 blocks): eight table entries per
+    producer lane."""
+    rng = np.random.default_rng(58 + BS)
+    dtype = synth.BF16
+    q, kc, vc, bt, lens, max_len = random_case(rng, [9000, P, P + 1, 300, 2 * P - 5], 16, 2, 128,
+                                               BS, dtype)
+    check_case(q, kc, vc, bt, lens, max_len, dtype, 0.09, P, f"BS={BS} P={P}")
