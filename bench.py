@@ -472,15 +472,22 @@ def gpu_arm(args, rank, world, local_rank):
                                            workspace=ws, stream=stream)
 
     k1_events = []
+    k3_events = []
 
     def step(record=False):
         for l in range(L):
-            if not fused:
-                pkv.pkv_reshape_and_cache(wl.k_new[l], wl.v_new[l], wl.k_cache[l],
-                                          wl.v_cache[l], slots, stream=stream)
             if record:
                 e0 = torch.cuda.Event(enable_timing=True)
                 e1 = torch.cuda.Event(enable_timing=True)
+            if not fused:
+                if record:
+                    ec = torch.cuda.Event(enable_timing=True)
+                    ec.record(stream)
+                pkv.pkv_reshape_and_cache(wl.k_new[l], wl.v_new[l], wl.k_cache[l],
+                                          wl.v_cache[l], slots, stream=stream)
+                if record:
+                    k3_events.append((ec, e0))
+            if record:
                 e0.record(stream)
             if fused:
                 # the workload's slot of each sequence is its newest position (len - 1)
@@ -530,6 +537,13 @@ def gpu_arm(args, rank, world, local_rank):
     ms_step = ms_total / args.steps
     value, tokens_per_s = weak_scaling_rates(kv_step, B, world, ms_step)
     k1_avg_ms = statistics.mean(k1_ms)
+    cache_write = None
+    if k3_events:
+        k3_us = 1e3 * statistics.mean(a.elapsed_time(b) for a, b in k3_events)
+        k3_bytes = len(wl.slot_mapping) * sp.num_kv_heads * sp.head_dim * 2 * 2 * 2
+        cache_write = {"us_per_launch": round(k3_us, 2), "bytes_per_launch": k3_bytes,
+                       "gbs": round(k3_bytes / (k3_us * 1e-6) / 1e9, 1),
+                       "note": "launch-latency bound: reads and writes each new token's K/V rows"}
     k1_q = np.percentile(np.array(k1_ms), [10, 50, 90]) * 1e3     # this rank's spread, us
     k1_avg_ms = max_over_ranks(k1_avg_ms)
     peak, peak_kind = read_peaks()
@@ -582,6 +596,7 @@ def gpu_arm(args, rank, world, local_rank):
         "tokens_per_s": round(tokens_per_s, 1),
         "pct_of_hbm_peak": round(100 * value / world / peak, 2),
         "memory_utilisation": memory,
+        **({"cache_write": cache_write} if cache_write else {}),
         **({"swap_blocks": swap} if swap else {}),
         **({"prefix_cache": prefix_cache} if prefix_cache else {}),
         "clocks": clocks.summary(),
@@ -853,10 +868,12 @@ def e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, worl
     mirror_lens = mgr.pkv_block_tables(ids)[2].astype(np.int64)
     kv_total = [0]
     k = [0]
+    host_s = [0.0]
 
     def one_step():
         b = k[0] % NBUF
         k[0] += 1
+        th = time.perf_counter()
         if fused:
             st, done, sl, cows = mgr.pkv_seq_append_batch(ids, 1)   # host mirror
             if st != 0 or len(cows):
@@ -866,10 +883,14 @@ def e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, worl
             if st != 0 or len(cows):
                 raise RuntimeError(f"append failed ({st}) or needed a copy in an unshared workload")
             st, tables, lens = mgr.pkv_block_tables(ids)
+            host_s[0] += time.perf_counter() - th
+            th = None
             ev_tables[b].synchronize()      # the H2D that last read these host buffers is done
             slots_h[b].numpy()[:] = sl[:, 0]
             bt_h[b].numpy()[:] = tables
             lens_h[b].numpy()[:] = lens
+        if th is not None:
+            host_s[0] += time.perf_counter() - th
         mirror_lens[:] += 1
         kv_total[0] += int(mirror_lens.sum()) * sp.num_kv_heads * sp.head_dim * 4 * L
         # buffer set b was last used two steps ago: its kernels must be done before refilling
@@ -911,6 +932,7 @@ def e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, worl
     torch.cuda.synchronize(dev)
     barrier()
     kv_total[0] = 0
+    host_s[0] = 0.0
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
@@ -934,6 +956,7 @@ def e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, worl
     value = kv_total[0] / args.steps * world / (ms * 1e-3) / 1e9
     return {"value": round(value, 1), "unit": "GB/s", "ms_per_step": round(ms, 4),
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "host_block_manager_us_per_step": round(1e6 * host_s[0] / args.steps, 1),
             "includes": ("device append of one token per sequence (tables, lengths and free "
                          "list resident on the GPU; the host allocator mirrors it with one "
                          "batched call), pinned H2D of every layer's q/k_new/v_new, the fused "
