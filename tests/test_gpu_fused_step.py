@@ -300,3 +300,59 @@ def test_gqa_workload_step_full_size(cuda_device):
     assert torch.equal(vc.view(torch.int16), vc2.view(torch.int16))
     assert np.array_equal(to_bits(out_f), to_bits(out_u))
     assert_close(to_bits(out_f)[seqs], ref, dt, "fused step, sampled")
+
+
+def fused_full_size(wl, layer, nsample, seed):
+    """The benchmark's fused step on a full-size workload layer: sampled sequences against
+    the oracle, every sequence bit for bit against cache write + decode."""
+    sp = wl.spec
+    dt = sp.dtype
+    B = wl.num_seqs
+    seqs = synth.sample_sequences(wl, nsample, seed=seed)
+    kc, vc = wl.k_cache[layer], wl.v_cache[layer]
+    ref = sampled_oracle(to_bits(wl.q[layer]), kc, vc, wl.block_tables, wl.context_lens, seqs,
+                         wl.scale, dt, to_bits(wl.k_new[layer]), to_bits(wl.v_new[layer]),
+                         wl.slot_mapping)
+    bt = torch.from_numpy(wl.block_tables).cuda()
+    lens = torch.from_numpy(wl.context_lens).cuda()
+    kc2, vc2 = kc.clone(), vc.clone()
+    ws = torch.zeros(pkv.pkv_decode_step_workspace_size(B, sp.num_heads, sp.num_kv_heads,
+                                                        sp.head_dim, sp.block_size, sp.max_len),
+                     dtype=torch.uint8, device="cuda")
+    out_f = torch.empty_like(wl.q[layer])
+    pkv.pkv_get_device_status(clear=True)
+    pkv.pkv_paged_decode_step(out_f, wl.q[layer],
+                              wl.k_new[layer].view(B, sp.num_kv_heads, sp.head_dim),
+                              wl.v_new[layer].view(B, sp.num_kv_heads, sp.head_dim), kc2, vc2,
+                              bt, lens, sp.max_len, ws, scale=wl.scale)
+    pkv.pkv_reshape_and_cache(wl.k_new[layer], wl.v_new[layer], kc, vc,
+                              torch.from_numpy(wl.slot_mapping).cuda())
+    out_u = torch.empty_like(wl.q[layer])
+    pkv.pkv_paged_attention_decode(out_u, wl.q[layer], kc, vc, bt, lens, sp.max_len,
+                                   scale=wl.scale)
+    torch.cuda.synchronize()
+    assert pkv.pkv_get_device_status() == 0
+    assert torch.equal(kc.view(torch.int16), kc2.view(torch.int16))
+    assert torch.equal(vc.view(torch.int16), vc2.view(torch.int16))
+    assert np.array_equal(to_bits(out_f), to_bits(out_u))
+    assert_close(to_bits(out_f)[seqs], ref, dt, f"{sp.name} layer {layer}, fused step")
+
+
+@pytest.mark.slow
+def test_llama7b_mha_fused_step_full_size(cuda_device):
+    """The default workload's layers: write-and-decode kernel + reduce (2048 pairs)."""
+    wl = synth.make_workload("llama7b_mha", values_on="cuda", num_layers=2)
+    for layer in range(2):
+        fused_full_size(wl, layer, 6, seed=11 + layer)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("bs", [8, 32])
+def test_long_context_fused_step_full_size(cuda_device, bs):
+    """Long contexts: the step kernel merges in its own launch (512 pairs, longest-first
+    item order)."""
+    wl = synth.make_workload("long_context", values_on="cuda", block_size=bs)
+    B, sp = wl.num_seqs, wl.spec
+    assert pkv.pkv_decode_step_launches(B, sp.num_heads, sp.num_kv_heads, sp.head_dim, bs,
+                                        sp.max_len) == 1
+    fused_full_size(wl, 0, 2, seed=13)
