@@ -551,7 +551,7 @@ def gpu_arm(args, rank, world, local_rank):
     read_probe = hbm_read_probe(dev, stream)
     swap = swap_measurement(wl, dev, stream) if args.swap else None
     mem_mgr = replay_block_manager(wl)
-    memory = memory_utilisation(wl, mem_mgr)
+    memory = memory_utilisation(wl, mem_mgr, sp0.max_len)   # the workload's own length cap
     mem_mgr.close()
     prefix_cache = prefix_cache_measurement(sp) if args.prefix_cache else None
     # the dominant kernel: the partition kernel, or for the fused step the write-and-decode
@@ -716,7 +716,7 @@ def prefix_cache_measurement(sp, requests=1024, concurrency=128, decode_len=64, 
     return out
 
 
-def memory_utilisation(wl, mgr):
+def memory_utilisation(wl, mgr, max_len=None):
     """KV-pool utilisation of the workload's state (\"vLLM / PagedAttention — 分页 KV Cache
     分析\" §4.2: tokens stored / (blocks x page size)): logical tokens over held blocks from
     the block manager (above 1 when blocks are shared), the same with each shared slot
@@ -731,7 +731,7 @@ def memory_utilisation(wl, mgr):
         blocks = wl.block_tables[s, :nblk].astype(np.int64)
         slots.append((blocks[:, None] * bs + np.arange(bs)).reshape(-1)[:int(n)])
     distinct = int(np.unique(np.concatenate(slots)).size) if slots else 0
-    max_len = int(sp.max_len)
+    max_len = int(max_len or sp.max_len)
     return {"logical": round(util, 4),
             "physical": round(distinct / (held * bs), 4) if held else 0.0,
             "contiguous_prealloc": round(float(lens.sum()) / (len(lens) * max_len), 4),
