@@ -356,3 +356,70 @@ def test_long_context_fused_step_full_size(cuda_device, bs):
     assert pkv.pkv_decode_step_launches(B, sp.num_heads, sp.num_kv_heads, sp.head_dim, bs,
                                         sp.max_len) == 1
     fused_full_size(wl, 0, 2, seed=13)
+
+
+@pytest.mark.parametrize("nseq,Hq,P", [(12, 8, 64), (64, 32, 64)])
+def test_fused_step_replays_in_a_cuda_graph(cuda_device, nseq, Hq, P):
+    """Device append + two fused layers captured once in a CUDA graph and replayed three
+    times equal the same three steps run eagerly, bit for bit (tables, lengths, free-list
+    cursor, caches, outputs). Small batches merge in the step launch (cooperative), larger
+    ones launch the reduce kernel."""
+    rng = np.random.default_rng(70 + nseq)
+    dtype, Hkv, D, BS, L = synth.F16, 4, 64, 16, 2
+    mb = 24
+    nb = nseq * mb + 32
+    m = model_state(rng, nb, BS, mb, nseq, 12 * BS)
+    bt0, lens0 = upload_model(m, nseq)
+    fl = np.array(m.free_list(), np.int32)
+    max_len = mb * BS
+    kc0 = [synth.round_to_bits(rng.standard_normal((nb, Hkv, BS, D), dtype=np.float32), dtype)
+           for _ in range(L)]
+    vc0 = [synth.round_to_bits(rng.standard_normal((nb, Hkv, BS, D), dtype=np.float32), dtype)
+           for _ in range(L)]
+    q = [to_dev(synth.round_to_bits(rng.standard_normal((nseq, Hq, D), dtype=np.float32), dtype),
+                dtype) for _ in range(L)]
+    kn = [to_dev(synth.round_to_bits(rng.standard_normal((nseq, Hkv, D), dtype=np.float32),
+                                     dtype), dtype) for _ in range(L)]
+    vn = [to_dev(synth.round_to_bits(rng.standard_normal((nseq, Hkv, D), dtype=np.float32),
+                                     dtype), dtype) for _ in range(L)]
+
+    def fresh():
+        st = dict(bt=torch.from_numpy(bt0).cuda(), lens=torch.from_numpy(lens0).cuda(),
+                  free=torch.from_numpy(fl).cuda(), used=torch.zeros(1, dtype=torch.int32,
+                                                                     device="cuda"),
+                  kc=[to_dev(x, dtype) for x in kc0], vc=[to_dev(x, dtype) for x in vc0],
+                  out=[torch.empty_like(x) for x in q],
+                  ws=torch.zeros(pkv.pkv_decode_step_workspace_size(nseq, Hq, Hkv, D, BS,
+                                                                    max_len, P),
+                                 dtype=torch.uint8, device="cuda"))
+        return st
+
+    def step(st):
+        pkv.pkv_device_append(st["bt"], st["lens"], st["free"], st["used"], nb, max_len, BS)
+        for l in range(L):
+            pkv.pkv_paged_decode_step(st["out"][l], q[l], kn[l], vn[l], st["kc"][l], st["vc"][l],
+                                      st["bt"], st["lens"], max_len, st["ws"], scale=0.125,
+                                      partition_size=P)
+
+    pkv.pkv_get_device_status(clear=True)
+    eager = fresh()
+    for _ in range(3):
+        step(eager)
+    torch.cuda.synchronize()
+    graphed = fresh()
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(g, stream=side):
+        step(graphed)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    assert pkv.pkv_get_device_status() == 0
+    for key in ("bt", "lens", "used"):
+        assert torch.equal(eager[key], graphed[key]), key
+    for l in range(L):
+        assert torch.equal(eager["kc"][l].view(torch.int16), graphed["kc"][l].view(torch.int16))
+        assert torch.equal(eager["vc"][l].view(torch.int16), graphed["vc"][l].view(torch.int16))
+        assert torch.equal(eager["out"][l].view(torch.int16), graphed["out"][l].view(torch.int16))
+    del g
