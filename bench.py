@@ -451,10 +451,13 @@ def gpu_arm(args, rank, world, local_rank):
     kn3 = [wl.k_new[l].view(B, sp.num_kv_heads, sp.head_dim) for l in range(L)]
     vn3 = [wl.v_new[l].view(B, sp.num_kv_heads, sp.head_dim) for l in range(L)]
 
+    # the stream the step's kernels go to (a capture stream while a CUDA graph is recorded)
+    launch_stream = [stream]
+
     def fused_layer(l, out_t, q_t, kn_t, vn_t, bt_t, lens_t):
         pkv.pkv_paged_decode_step(out_t, q_t, kn_t, vn_t, wl.k_cache[l], wl.v_cache[l], bt_t,
                                   lens_t, max_len, ws, scale=wl.scale, partition_size=P,
-                                  stream=stream)
+                                  stream=launch_stream[0])
 
     def decode(l, out_t, q_t, bt_t, lens_t):
         if shared:
@@ -462,14 +465,14 @@ def gpu_arm(args, rank, world, local_rank):
             if l == 0:
                 pkv.pkv_shared_prefix_plan(bt_t, lens_t, starts, prefix, sp.num_heads,
                                            sp.num_kv_heads, sp.head_dim, sp.block_size, max_len,
-                                           ws, partition_size=P, stream=stream)
+                                           ws, partition_size=P, stream=launch_stream[0])
             pkv.pkv_paged_attention_decode_shared_prefix_planned(
                 out_t, q_t, wl.k_cache[l], wl.v_cache[l], bt_t, lens_t, max_len, ws,
-                scale=wl.scale, partition_size=P, stream=stream)
+                scale=wl.scale, partition_size=P, stream=launch_stream[0])
         else:
             pkv.pkv_paged_attention_decode(out_t, q_t, wl.k_cache[l], wl.v_cache[l], bt_t,
                                            lens_t, max_len, scale=wl.scale, partition_size=P,
-                                           workspace=ws, stream=stream)
+                                           workspace=ws, stream=launch_stream[0])
 
     k1_events = []
     k3_events = []
@@ -482,20 +485,20 @@ def gpu_arm(args, rank, world, local_rank):
             if not fused:
                 if record:
                     ec = torch.cuda.Event(enable_timing=True)
-                    ec.record(stream)
+                    ec.record(launch_stream[0])
                 pkv.pkv_reshape_and_cache(wl.k_new[l], wl.v_new[l], wl.k_cache[l],
-                                          wl.v_cache[l], slots, stream=stream)
+                                          wl.v_cache[l], slots, stream=launch_stream[0])
                 if record:
                     k3_events.append((ec, e0))
             if record:
-                e0.record(stream)
+                e0.record(launch_stream[0])
             if fused:
                 # the workload's slot of each sequence is its newest position (len - 1)
                 fused_layer(l, outs[l], wl.q[l], kn3[l], vn3[l], bt, lens)
             else:
                 decode(l, outs[l], wl.q[l], bt, lens)
             if record:
-                e1.record(stream)
+                e1.record(launch_stream[0])
                 k1_events.append((e0, e1))
 
     if fused:
@@ -516,8 +519,24 @@ def gpu_arm(args, rank, world, local_rank):
     for _ in range(args.warmup):
         step()
     barrier()
+    g = None
+    if not args.no_graph:
+        # the step recorded once as a CUDA graph (every layer's launches) and replayed: the
+        # headline timing, as a serving loop runs a decode step
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        launch_stream[0] = side
+        with torch.cuda.graph(g, stream=side):
+            step()
+        launch_stream[0] = stream
+        stream.wait_stream(side)
+        for _ in range(args.warmup):
+            g.replay()
+        barrier()
     with ClockSampler(local_rank) as clocks:
         barrier()
+        # eager launches with CUDA events around every decode call (per-launch times)
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
@@ -525,7 +544,18 @@ def gpu_arm(args, rank, world, local_rank):
             step(record=True)
         t1.record(stream)
         barrier()
-    ms_total = t0.elapsed_time(t1)
+        if g is not None:
+            g0 = torch.cuda.Event(enable_timing=True)
+            g1 = torch.cuda.Event(enable_timing=True)
+            g0.record(stream)
+            for _ in range(args.steps):
+                g.replay()
+            g1.record(stream)
+            barrier()
+    ms_eager = t0.elapsed_time(t1)
+    ms_total = g0.elapsed_time(g1) if g is not None else ms_eager
+    if g is not None:
+        del g
     k1_ms = [a.elapsed_time(b) for a, b in k1_events]
     if pkv.pkv_get_device_status(stream=stream) != 0:
         raise RuntimeError("device status word set during the benchmark")
@@ -536,6 +566,8 @@ def gpu_arm(args, rank, world, local_rank):
     ms_total = max_over_ranks(ms_total)
     ms_step = ms_total / args.steps
     value, tokens_per_s = weak_scaling_rates(kv_step, B, world, ms_step)
+    ms_eager_step = max_over_ranks(ms_eager) / args.steps
+    eager_value, _ = weak_scaling_rates(kv_step, B, world, ms_eager_step)
     k1_avg_ms = statistics.mean(k1_ms)
     cache_write = None
     if k3_events:
@@ -589,6 +621,7 @@ def gpu_arm(args, rank, world, local_rank):
             "partition_size": P,
             "decode": args.decode,
             "step": "fused" if fused else "separate",
+            "timed": "eager launches" if args.no_graph else "CUDA graph replays of the step",
             "kv_bytes_per_step": kv_step,
             "l2": f"inputs larger than L2: {kv_layer / 1e6:.0f} MB of K/V per layer vs 126 MB L2",
             "parallelism": f"replicas x{world}",
@@ -597,6 +630,9 @@ def gpu_arm(args, rank, world, local_rank):
         "pct_of_hbm_peak": round(100 * value / world / peak, 2),
         "memory_utilisation": memory,
         **({"cache_write": cache_write} if cache_write else {}),
+        "eager": {"value": round(eager_value, 1), "unit": "GB/s",
+                  "ms_per_step": round(ms_eager_step, 4),
+                  "note": "the same steps launched one kernel at a time (no graph)"},
         **({"swap_blocks": swap} if swap else {}),
         **({"prefix_cache": prefix_cache} if prefix_cache else {}),
         "clocks": clocks.summary(),
@@ -1094,6 +1130,9 @@ def main():
     ap.add_argument("--partition", type=int, default=0, help="decode partition size (0 = auto)")
     ap.add_argument("--swap", action="store_true",
                     help="also time pkv_swap_blocks (preemption) against a contiguous copy")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time eager launches only (by default the device step is recorded once "
+                         "as a CUDA graph and the replays are timed)")
     ap.add_argument("--prefix-cache", action="store_true",
                     help="also replay a request stream through the block manager's prefix cache")
     ap.add_argument("--step", default="fused", choices=["separate", "fused"],
