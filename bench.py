@@ -628,6 +628,7 @@ def gpu_arm(args, rank, world, local_rank):
         },
         "tokens_per_s": round(tokens_per_s, 1),
         "pct_of_hbm_peak": round(100 * value / world / peak, 2),
+        "pct_of_nominal_8tbs": round(100 * value / world / 8000.0, 2),
         "memory_utilisation": memory,
         **({"cache_write": cache_write} if cache_write else {}),
         "eager": {"value": round(eager_value, 1), "unit": "GB/s",
