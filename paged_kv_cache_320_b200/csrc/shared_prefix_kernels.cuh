@@ -374,19 +374,12 @@ paged_decode_shared_kernel(const __grid_constant__ CUtensorMap tmap_k,
             v = __shfl_sync(0xffffffffu, v, 0);
             return v > 0x7fffffffu ? 0x7fffffff : (int)v;
         };
-        int cur_idx = take();
-        int cur_f = fetch(cur_idx);
-        while (cur_idx < count && ok) {
-            const int table_seq = __shfl_sync(0xffffffffu, cur_f, 0);
-            const int tok0 = __shfl_sync(0xffffffffu, cur_f, 1);
-            const int ntok = __shfl_sync(0xffffffffu, cur_f, 2);
-            const int hk = __shfl_sync(0xffffffffu, cur_f, 3);
-            const int first_seq = __shfl_sync(0xffffffffu, cur_f, 4);
-            const int nseq = __shfl_sync(0xffffffffu, cur_f, 5);
-            const int part = __shfl_sync(0xffffffffu, cur_f, 6);
-            const int nst = max(1, (ntok + kStageTokens - 1) / kStageTokens);
+        // an item's slice of its block-table row: entry e in lane e % 32, register e / 32
+        auto load_entries = [&](int f, int (&ent)[kMaxItemBlocks / 32]) {
+            const int table_seq = __shfl_sync(0xffffffffu, f, 0);
+            const int tok0 = __shfl_sync(0xffffffffu, f, 1);
+            const int ntok = __shfl_sync(0xffffffffu, f, 2);
             const int nblk = (ntok + BS - 1) / BS;
-            int ent[kMaxItemBlocks / 32];
             const int32_t *bt =
                 prm.block_tables + (size_t)table_seq * prm.max_blocks_per_seq + tok0 / BS;
 #pragma unroll
@@ -394,7 +387,20 @@ paged_decode_shared_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 const int e = k * 32 + lane;
                 ent[k] = e < nblk ? bt[e] : 0;
             }
+        };
+        int cur_idx = take();
+        int cur_f = fetch(cur_idx);
+        int ent[kMaxItemBlocks / 32];
+        if (cur_idx < count) load_entries(cur_f, ent);
+        while (cur_idx < count && ok) {
+            const int ntok = __shfl_sync(0xffffffffu, cur_f, 2);
+            const int hk = __shfl_sync(0xffffffffu, cur_f, 3);
+            const int first_seq = __shfl_sync(0xffffffffu, cur_f, 4);
+            const int nseq = __shfl_sync(0xffffffffu, cur_f, 5);
+            const int part = __shfl_sync(0xffffffffu, cur_f, 6);
+            const int nst = max(1, (ntok + kStageTokens - 1) / kStageTokens);
             int nxt_idx = 0, nxt_f = 0;
+            int nxt_ent[kMaxItemBlocks / 32];
             for (int st = 0; st < nst; ++st, ++it) {
                 const int slot = it % L::kStages;
                 const uint32_t ph = ((it / L::kStages) & 1) ^ 1;
@@ -445,12 +451,16 @@ paged_decode_shared_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     }
                 }
                 if (st == 0) {
+                    // the next item and its table slice, while this item's stages stream
                     nxt_idx = take();
                     nxt_f = fetch(nxt_idx);
+                    if (nxt_idx < count) load_entries(nxt_f, nxt_ent);
                 }
             }
             cur_idx = nxt_idx;
             cur_f = nxt_f;
+#pragma unroll
+            for (int k = 0; k < kMaxItemBlocks / 32; ++k) ent[k] = nxt_ent[k];
         }
         if (ok) {
             const int slot = it % L::kStages;
