@@ -113,3 +113,39 @@ def test_status_strings():
     L = B.lib()
     for code in range(-9, 1):
         assert L.pkv_status_string(code)
+
+
+def test_step_and_shared_prefix_checks_without_a_device():
+    """The device-step and shared-prefix entry points reject bad arguments on the host,
+    before any CUDA call (no GPU here)."""
+    L = B.lib()
+    # decode step: bad head_dim, missing workspace, zero sequences
+    args = [None] * 8
+    assert L.pkv_paged_decode_step(*args, 4, 8, 8, 96, 16, 8, 64, 100, 0.1, 0, 0, None, 0,
+                                   None) == B.PKV_ERR_INVALID_ARG
+    assert L.pkv_paged_decode_step(*args, 0, 8, 8, 64, 16, 8, 64, 100, 0.1, 0, 0, None, 0,
+                                   None) == B.PKV_OK
+    assert L.pkv_paged_decode_step(*args, 4, 8, 8, 64, 16, 8, 64, 100, 0.1, 0, 0, None, 0,
+                                   None) == B.PKV_ERR_INVALID_ARG        # null tensors
+    # workspace size query: at least the 256-byte header, more with several partitions
+    one, many = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    assert L.pkv_decode_step_workspace_size(4, 8, 2, 64, 16, 64, 64, ctypes.byref(one)) == 0
+    assert L.pkv_decode_step_workspace_size(4, 8, 2, 64, 16, 1024, 64, ctypes.byref(many)) == 0
+    assert one.value == 256 and many.value > one.value
+    # device append: negative sizes, missing cursor
+    assert L.pkv_device_append(None, None, None, 0, None, None, 4, 8, 16, 64, 128,
+                               None) == B.PKV_ERR_INVALID_ARG
+    assert L.pkv_device_append(None, None, None, -1, None, None, 4, 8, 16, 64, 128,
+                               None) == B.PKV_ERR_INVALID_ARG
+    # shared-prefix plan / planned decode: too many groups, zero sequences
+    assert L.pkv_shared_prefix_plan(None, None, None, None, 5, 4, 8, 2, 64, 16, 8, 100, 0, None,
+                                    0, None) == B.PKV_ERR_INVALID_ARG
+    assert L.pkv_shared_prefix_plan(None, None, None, None, 1, 0, 8, 2, 64, 16, 8, 100, 0, None,
+                                    0, None) == B.PKV_OK
+    assert L.pkv_paged_attention_decode_shared_prefix_planned(
+        None, None, None, None, None, None, 4, 8, 2, 64, 16, 8, 64, 100, 0.1, 3, 0, None, 0,
+        None) == B.PKV_ERR_INVALID_ARG                                    # dtype 3
+    # launch-count query needs the device (SM count) only when there is work
+    n = ctypes.c_int(-1)
+    assert L.pkv_decode_step_launches(0, 8, 2, 64, 16, 100, 0, ctypes.byref(n)) == 0
+    assert n.value == 0
