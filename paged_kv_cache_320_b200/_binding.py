@@ -3,7 +3,10 @@
 Every function here reads pointers, sizes and the current CUDA stream from torch
 tensors and calls the C entry point of the same name; all device work runs in the
 library's kernels. There is no fallback: if the library is missing, the first call
-raises.
+raises. Before a call, every tensor whose address the library will dereference is checked
+to be a contiguous CUDA tensor on the query's device, of the element type and with at
+least the rows the C declaration reads (ValueError / TypeError otherwise), so that a host
+tensor or a short index array never reaches a kernel.
 """
 from __future__ import annotations
 
@@ -148,6 +151,70 @@ def _ptr(t):
     return t.data_ptr()
 
 
+def _nbytes(t):
+    return t.numel() * t.element_size()
+
+
+def _need(t, name, device=None, dtype=None, min_numel=0):
+    """Raise unless ``t`` is a contiguous CUDA tensor (on ``device`` when given, of
+    ``dtype`` when given) holding at least ``min_numel`` elements."""
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the call runs on {device}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, not {t.dtype}")
+    if t.numel() < min_numel:
+        raise ValueError(f"{name} holds {t.numel()} elements, the call reads {min_numel}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _tables(block_tables, context_lens, B, device):
+    """block_tables int32 [>= B, MB] and context_lens int32 [>= B] on ``device``."""
+    import torch
+    if block_tables.dim() != 2 or block_tables.shape[0] < B:
+        raise ValueError(f"block_tables must be [num_seqs >= {B}, max_blocks_per_seq], "
+                         f"not {tuple(block_tables.shape)}")
+    _need(block_tables, "block_tables", device, torch.int32)
+    _need(context_lens, "context_lens", device, torch.int32, B)
+
+
+def _decode_shapes(out, q, k_cache, v_cache, block_tables, context_lens, k_new=None,
+                   v_new=None):
+    """Checks the decode family's tensors; returns (B, Hq, D, NB, Hkv, BS)."""
+    if q.dim() != 3 or k_cache.dim() != 4:
+        raise ValueError("q must be [B, Hq, D] and k_cache [NB, Hkv, BS, D]")
+    B, Hq, D = q.shape
+    NB, Hkv, BS, D2 = k_cache.shape
+    if D2 != D or out.shape != q.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch")
+    _dtype_code(q)
+    dev = q.device
+    for name, t in (("out", out), ("q", q), ("k_cache", k_cache), ("v_cache", v_cache),
+                    ("k_new", k_new), ("v_new", v_new)):
+        if t is not None:
+            _need(t, name, dev, q.dtype)
+    _tables(block_tables, context_lens, B, dev)
+    return B, Hq, D, NB, Hkv, BS
+
+
+def _groups(group_start, prefix_lens, device):
+    """group_start int32 [num_groups + 1] and prefix_lens int32 [num_groups]."""
+    import torch
+    _need(prefix_lens, "prefix_lens", device, torch.int32)
+    _need(group_start, "group_start", device, torch.int32, prefix_lens.numel() + 1)
+
+
+def _cache_ptrs(k_cache_ptrs, v_cache_ptrs):
+    """Per-layer cache address arrays: int64 device tensors of one length."""
+    import torch
+    _need(k_cache_ptrs, "k_cache_ptrs", None, torch.int64)
+    _need(v_cache_ptrs, "v_cache_ptrs", k_cache_ptrs.device, torch.int64,
+          k_cache_ptrs.numel())
+
+
 # ---------------------------------------------------------------------------
 # device entry points
 # ---------------------------------------------------------------------------
@@ -175,10 +242,8 @@ def pkv_paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_l
     """out/q [B, Hq, D]; k_cache/v_cache [NB, Hkv, BS, D]; block_tables int32 [B, MB];
     context_lens int32 [B]; workspace: uint8 tensor of pkv_decode_workspace_size bytes
     (allocated here when None and needed)."""
-    B, Hq, D = q.shape
-    NB, Hkv, BS, D2 = k_cache.shape
-    if D2 != D or out.shape != q.shape or v_cache.shape != k_cache.shape:
-        raise ValueError("shape mismatch")
+    B, Hq, D, NB, Hkv, BS = _decode_shapes(out, q, k_cache, v_cache, block_tables,
+                                           context_lens)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     if workspace is None:
@@ -186,8 +251,10 @@ def pkv_paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_l
         if need:
             import torch
             workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if workspace is not None:
+        _need(workspace, "workspace", q.device)
     ws_ptr = _ptr(workspace) if workspace is not None else None
-    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    ws_bytes = _nbytes(workspace) if workspace is not None else 0
     _check(lib().pkv_paged_attention_decode(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
         B, Hq, Hkv, D, BS, block_tables.shape[1], NB, int(max_context_len), float(scale),
@@ -202,10 +269,8 @@ def pkv_paged_attention_decode_noalloc(out, q, k_cache, v_cache, block_tables, c
     """pkv_paged_attention_decode without a workspace: the library's fixed scratch
     array is used instead (see pagedkv.h); raises PagedKVError(PKV_ERR_WORKSPACE)
     when the sizes need more scratch than it holds."""
-    B, Hq, D = q.shape
-    NB, Hkv, BS, D2 = k_cache.shape
-    if D2 != D or out.shape != q.shape or v_cache.shape != k_cache.shape:
-        raise ValueError("shape mismatch")
+    B, Hq, D, NB, Hkv, BS = _decode_shapes(out, q, k_cache, v_cache, block_tables,
+                                           context_lens)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     _check(lib().pkv_paged_attention_decode_noalloc(
@@ -231,10 +296,9 @@ def pkv_paged_attention_decode_shared_prefix(out, q, k_cache, v_cache, block_tab
                                              workspace=None, stream=None):
     """As pkv_paged_attention_decode, with group_start int32 [num_groups + 1] and
     prefix_lens int32 [num_groups] device tensors describing shared prefixes."""
-    B, Hq, D = q.shape
-    NB, Hkv, BS, D2 = k_cache.shape
-    if D2 != D or out.shape != q.shape or v_cache.shape != k_cache.shape:
-        raise ValueError("shape mismatch")
+    B, Hq, D, NB, Hkv, BS = _decode_shapes(out, q, k_cache, v_cache, block_tables,
+                                           context_lens)
+    _groups(group_start, prefix_lens, q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     if workspace is None:
@@ -242,11 +306,12 @@ def pkv_paged_attention_decode_shared_prefix(out, q, k_cache, v_cache, block_tab
         need = pkv_decode_shared_prefix_workspace_size(B, Hq, Hkv, D, BS, max_context_len,
                                                        partition_size)
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _need(workspace, "workspace", q.device)
     _check(lib().pkv_paged_attention_decode_shared_prefix(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
         _ptr(group_start), _ptr(prefix_lens), prefix_lens.numel(), B, Hq, Hkv, D, BS,
         block_tables.shape[1], NB, int(max_context_len), float(scale), _dtype_code(q),
-        int(partition_size), _ptr(workspace), workspace.numel(), _stream(stream)),
+        int(partition_size), _ptr(workspace), _nbytes(workspace), _stream(stream)),
         "pkv_paged_attention_decode_shared_prefix")
     return out
 
@@ -275,18 +340,18 @@ def pkv_paged_decode_step(out, q, k_new, v_new, k_cache, v_cache, block_tables, 
     """Cache write of each sequence's newest token + decode attention in one launch.
     k_new/v_new [B, Hkv, D]; workspace: uint8 device tensor of
     pkv_decode_step_workspace_size bytes, zero-filled before its first use (torch.zeros)."""
-    B, Hq, D = q.shape
-    NB, Hkv, BS, D2 = k_cache.shape
-    if (D2 != D or out.shape != q.shape or v_cache.shape != k_cache.shape
-            or tuple(k_new.shape) != (B, Hkv, D) or v_new.shape != k_new.shape):
-        raise ValueError("shape mismatch")
+    B, Hq, D, NB, Hkv, BS = _decode_shapes(out, q, k_cache, v_cache, block_tables,
+                                           context_lens, k_new, v_new)
+    if tuple(k_new.shape) != (B, Hkv, D) or v_new.shape != k_new.shape:
+        raise ValueError("k_new / v_new must be [B, Hkv, D]")
+    _need(workspace, "workspace", q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     _check(lib().pkv_paged_decode_step(
         _ptr(out), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
         _ptr(block_tables), _ptr(context_lens), B, Hq, Hkv, D, BS, block_tables.shape[1], NB,
         int(max_context_len), float(scale), _dtype_code(q), int(partition_size), _ptr(workspace),
-        workspace.numel() * workspace.element_size(), _stream(stream)), "pkv_paged_decode_step")
+        _nbytes(workspace), _stream(stream)), "pkv_paged_decode_step")
     return out
 
 
@@ -295,7 +360,15 @@ def pkv_device_append(block_tables, context_lens, free_blocks, free_used, num_bl
     """One token appended to every sequence on the device (see pagedkv.h): block_tables
     int32 [B, MB] and context_lens int32 [B] updated in place; free_blocks int32 [F] in pop
     order; free_used int32 [1] advanced by the blocks taken; slots_out int64 [B] or None."""
+    import torch
+    _need(context_lens, "context_lens", None, torch.int32)
     B = context_lens.numel()
+    dev = context_lens.device
+    _tables(block_tables, context_lens, B, dev)
+    _need(free_blocks, "free_blocks", dev, torch.int32)
+    _need(free_used, "free_used", dev, torch.int32, 1)
+    if slots_out is not None:
+        _need(slots_out, "slots_out", dev, torch.int64, B)
     _check(lib().pkv_device_append(
         _ptr(block_tables), _ptr(context_lens), _ptr(free_blocks), free_blocks.numel(),
         _ptr(free_used), _ptr(slots_out), B, block_tables.shape[1], int(block_size),
@@ -307,12 +380,18 @@ def pkv_shared_prefix_plan(block_tables, context_lens, group_start, prefix_lens,
                            partition_size=0, stream=None):
     """Build the shared-prefix item list in workspace (uint8 device tensor of
     pkv_decode_shared_prefix_workspace_size bytes) for every layer of a step."""
+    import torch
+    _need(context_lens, "context_lens", None, torch.int32)
     B = context_lens.numel()
+    dev = context_lens.device
+    _tables(block_tables, context_lens, B, dev)
+    _groups(group_start, prefix_lens, dev)
+    _need(workspace, "workspace", dev)
     _check(lib().pkv_shared_prefix_plan(
         _ptr(block_tables), _ptr(context_lens), _ptr(group_start), _ptr(prefix_lens),
         prefix_lens.numel(), B, int(num_heads), int(num_kv_heads), int(head_dim),
         int(block_size), block_tables.shape[1], int(max_context_len), int(partition_size),
-        _ptr(workspace), workspace.numel(), _stream(stream)), "pkv_shared_prefix_plan")
+        _ptr(workspace), _nbytes(workspace), _stream(stream)), "pkv_shared_prefix_plan")
 
 
 def pkv_paged_attention_decode_shared_prefix_planned(out, q, k_cache, v_cache, block_tables,
@@ -320,24 +399,33 @@ def pkv_paged_attention_decode_shared_prefix_planned(out, q, k_cache, v_cache, b
                                                      scale=None, partition_size=0,
                                                      stream=None):
     """Decode over the plan pkv_shared_prefix_plan left in workspace."""
-    B, Hq, D = q.shape
-    NB, Hkv, BS, D2 = k_cache.shape
-    if D2 != D or out.shape != q.shape or v_cache.shape != k_cache.shape:
-        raise ValueError("shape mismatch")
+    B, Hq, D, NB, Hkv, BS = _decode_shapes(out, q, k_cache, v_cache, block_tables,
+                                           context_lens)
+    _need(workspace, "workspace", q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     _check(lib().pkv_paged_attention_decode_shared_prefix_planned(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
         B, Hq, Hkv, D, BS, block_tables.shape[1], NB, int(max_context_len), float(scale),
-        _dtype_code(q), int(partition_size), _ptr(workspace), workspace.numel(), _stream(stream)),
-        "pkv_paged_attention_decode_shared_prefix_planned")
+        _dtype_code(q), int(partition_size), _ptr(workspace), _nbytes(workspace),
+        _stream(stream)), "pkv_paged_attention_decode_shared_prefix_planned")
     return out
 
 
 def pkv_reshape_and_cache(k_new, v_new, k_cache, v_cache, slot_mapping, stream=None):
     """k_new/v_new [T, Hkv, D]; caches [NB, Hkv, BS, D]; slot_mapping int64 [T]."""
+    import torch
+    if k_new.dim() != 3 or k_cache.dim() != 4:
+        raise ValueError("k_new must be [T, Hkv, D] and k_cache [NB, Hkv, BS, D]")
     T, Hkv, D = k_new.shape
-    NB, _, BS, _ = k_cache.shape
+    NB, Hkv2, BS, D2 = k_cache.shape
+    if (Hkv2, D2) != (Hkv, D) or v_new.shape != k_new.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch")
+    dev = k_cache.device
+    for name, t in (("k_new", k_new), ("v_new", v_new), ("k_cache", k_cache),
+                    ("v_cache", v_cache)):
+        _need(t, name, dev, k_cache.dtype)
+    _need(slot_mapping, "slot_mapping", dev, torch.int64, T)
     _check(lib().pkv_reshape_and_cache(_ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
                                        _ptr(slot_mapping), T, Hkv, D, BS, NB,
                                        _dtype_code(k_cache), _stream(stream)),
@@ -348,7 +436,12 @@ def pkv_copy_blocks(k_cache_ptrs, v_cache_ptrs, block_pairs, num_kv_heads, head_
                     num_blocks, dtype, stream=None):
     """k_cache_ptrs / v_cache_ptrs: int64 device tensors [L] of cache addresses;
     block_pairs: int32 device tensor [n, 2]."""
+    import torch
     n = block_pairs.shape[0] if block_pairs.numel() else 0
+    if n and (block_pairs.dim() != 2 or block_pairs.shape[1] != 2):
+        raise ValueError("block_pairs must be [n, 2]")
+    _cache_ptrs(k_cache_ptrs, v_cache_ptrs)
+    _need(block_pairs, "block_pairs", k_cache_ptrs.device, torch.int32)
     _check(lib().pkv_copy_blocks(_ptr(k_cache_ptrs), _ptr(v_cache_ptrs), k_cache_ptrs.numel(),
                                  _ptr(block_pairs), n, num_kv_heads, head_dim, block_size,
                                  num_blocks, dtype, _stream(stream)), "pkv_copy_blocks")
@@ -358,11 +451,14 @@ def pkv_swap_blocks(k_cache_ptrs, v_cache_ptrs, block_ids, host_buffer, to_host,
                     head_dim, block_size, num_blocks, dtype, stream=None):
     """Moves whole blocks between the caches and a pinned host tensor (see pagedkv.h).
     k_cache_ptrs / v_cache_ptrs: int64 device tensors of cache addresses; block_ids:
-    int32 device tensor; host_buffer: pinned CPU tensor."""
+    int32 device tensor; host_buffer: pinned CPU tensor (checked by the library)."""
+    import torch
     n = block_ids.numel()
+    _cache_ptrs(k_cache_ptrs, v_cache_ptrs)
+    _need(block_ids, "block_ids", k_cache_ptrs.device, torch.int32)
     _check(lib().pkv_swap_blocks(_ptr(k_cache_ptrs), _ptr(v_cache_ptrs), k_cache_ptrs.numel(),
                                  _ptr(block_ids), n, _ptr(host_buffer),
-                                 host_buffer.numel() * host_buffer.element_size(), int(to_host),
+                                 _nbytes(host_buffer), int(to_host),
                                  num_kv_heads, head_dim, block_size, num_blocks, dtype,
                                  _stream(stream)), "pkv_swap_blocks")
 
