@@ -434,6 +434,10 @@ def gpu_arm(args, rank, world, local_rank):
             raise SystemExit("--decode shared needs a workload with shared prefixes")
         starts = torch.arange(0, B + 1, sp.samples, dtype=torch.int32, device=dev)
         prefix = torch.full((sp.prompts,), sp.prefix, dtype=torch.int32, device=dev)
+        # the shared-prefix path has its own automatic partition size
+        P = pkv.pkv_decode_shared_prefix_partition_size(B, sp.num_heads, sp.num_kv_heads,
+                                                        sp.head_dim, sp.block_size, max_len,
+                                                        args.partition)
         ws = torch.empty(max(16, pkv.pkv_decode_shared_prefix_workspace_size(
             B, sp.num_heads, sp.num_kv_heads, sp.head_dim, sp.block_size, max_len, P)),
             dtype=torch.uint8, device=dev)

@@ -158,7 +158,9 @@ int pkv_paged_attention_decode_noalloc(void *out, const void *q, const void *k_c
  *              first member — a wrong value costs sharing, never correctness.
  * A malformed group_start is treated as one group per sequence and sets
  * PKV_STATUS_BAD_LEN. Workspace: pkv_decode_shared_prefix_workspace_size bytes, no
- * initial contents required. Other arguments, limits and errors as
+ * initial contents required. partition_size 0 selects this path's own automatic size
+ * (pkv_decode_shared_prefix_partition_size: 1024 tokens for groups up to 4, 2048 above,
+ * at most 256 blocks, smaller for small batches). Other arguments, limits and errors as
  * pkv_paged_attention_decode (num_groups >= 1, <= num_seqs). Three kernel launches.
  * ---------------------------------------------------------------------------- */
 int pkv_paged_attention_decode_shared_prefix(
@@ -195,6 +197,12 @@ int pkv_paged_attention_decode_shared_prefix_planned(
 int pkv_decode_shared_prefix_workspace_size(int num_seqs, int num_heads, int num_kv_heads,
                                             int head_dim, int block_size, int max_context_len,
                                             int partition_size, size_t *bytes_out);
+
+/* The partition size the shared-prefix calls use for these sizes (resolves 0 to the
+ * shared path's automatic size). */
+int pkv_decode_shared_prefix_partition_size(int num_seqs, int num_heads, int num_kv_heads,
+                                            int head_dim, int block_size, int max_context_len,
+                                            int partition_size, int *partition_out);
 
 /* Workspace bytes pkv_paged_attention_decode needs for these sizes (0 when the
  * given partition size makes every context a single partition). Same argument

@@ -11,6 +11,7 @@ from ._binding import (  # noqa: F401
     lib,
     pkv_copy_blocks,
     pkv_decode_partition_size,
+    pkv_decode_shared_prefix_partition_size,
     pkv_decode_step_launches,
     pkv_decode_step_workspace_size,
     pkv_device_append,

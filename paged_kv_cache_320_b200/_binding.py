@@ -70,6 +70,8 @@ def lib() -> ctypes.CDLL:
         L.pkv_decode_shared_prefix_workspace_size.argtypes = [I, I, I, I, I, I, I,
                                                               ctypes.POINTER(SZ)]
         L.pkv_decode_partition_size.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(I)]
+        L.pkv_decode_shared_prefix_partition_size.argtypes = [I, I, I, I, I, I, I,
+                                                               ctypes.POINTER(I)]
         L.pkv_reshape_and_cache.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P]
         L.pkv_copy_blocks.argtypes = [P, P, I, P, I, I, I, I, I, I, P]
         L.pkv_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), I, P]
@@ -104,7 +106,8 @@ def lib() -> ctypes.CDLL:
         for name in ("pkv_paged_attention_decode", "pkv_paged_attention_decode_noalloc",
                      "pkv_paged_attention_decode_shared_prefix",
                      "pkv_decode_shared_prefix_workspace_size", "pkv_decode_workspace_size",
-                     "pkv_decode_partition_size", "pkv_reshape_and_cache", "pkv_copy_blocks",
+                     "pkv_decode_partition_size", "pkv_decode_shared_prefix_partition_size",
+                     "pkv_reshape_and_cache", "pkv_copy_blocks",
                      "pkv_swap_blocks",
                      "pkv_get_device_status", "pkv_alloc_create", "pkv_alloc_destroy",
                      "pkv_seq_append", "pkv_seq_append_batch", "pkv_seq_fork", "pkv_seq_free",
@@ -233,6 +236,15 @@ def pkv_decode_partition_size(num_seqs, num_heads, num_kv_heads, head_dim, block
     _check(lib().pkv_decode_partition_size(num_seqs, num_heads, num_kv_heads, head_dim,
                                            block_size, max_context_len, partition_size,
                                            ctypes.byref(out)), "pkv_decode_partition_size")
+    return out.value
+
+
+def pkv_decode_shared_prefix_partition_size(num_seqs, num_heads, num_kv_heads, head_dim,
+                                            block_size, max_context_len, partition_size=0) -> int:
+    out = ctypes.c_int(0)
+    _check(lib().pkv_decode_shared_prefix_partition_size(
+        num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len,
+        partition_size, ctypes.byref(out)), "pkv_decode_shared_prefix_partition_size")
     return out.value
 
 

@@ -83,6 +83,21 @@ def test_random_groups_match_oracle(cuda_device, dtype, Hq, Hkv, D, BS):
     assert pkv.pkv_get_device_status() == 0
 
 
+@pytest.mark.parametrize("Hq,Hkv,BS,P", [(32, 8, 16, 1024), (64, 8, 8, 2048), (32, 8, 32, 2048)])
+def test_long_prefix_items(cuda_device, Hq, Hkv, BS, P):
+    """Prefix items of 1024 and 2048 tokens (the shared path's automatic sizes at full
+    batch; 256 blocks of 8 at most), over prefixes that span several such items."""
+    rng = np.random.default_rng(Hq + BS + P)
+    dtype = synth.BF16
+    q, kc, vc, bt, lens, starts, pre, max_len = grouped_case(
+        rng, [5, 4], [2304 // BS, 1536 // BS], 300, Hq, Hkv, 128, BS, dtype)
+    ref = A.paged_decode_attention(q, kc, vc, bt, lens, 0.08, dtype)
+    pkv.pkv_get_device_status(clear=True)
+    got = run_shared(q, kc, vc, bt, lens, starts, pre, max_len, dtype, 0.08, P)
+    assert_close(got, ref, dtype, f"P={P}")
+    assert pkv.pkv_get_device_status() == 0
+
+
 def test_prefix_declared_longer_than_shared_is_cut(cuda_device):
     """Members share 6 pages but the caller declares 12 (and longer than one member):
     the plan cuts the prefix at the first differing page; results stay exact."""
