@@ -54,6 +54,15 @@ KERNEL_SOURCES = ["paged_kv_cache_320_b200/csrc/decode_kernels.cuh",
 STEP_SOURCES = KERNEL_SOURCES + ["paged_kv_cache_320_b200/csrc/step_kernels.cuh"]
 
 
+def describe(args) -> str:
+    """The named workload's description, with any size overridden on the command line."""
+    over = [f"{k} {v}" for k, v in (("block_size", getattr(args, "block_size", 0)),
+                                    ("layers", getattr(args, "layers", 0)),
+                                    ("batch", getattr(args, "batch", 0))) if v]
+    text = WORKLOADS[args.workload]
+    return text + (f" (run with {', '.join(over)})" if over else "")
+
+
 def kernel_source_hash(sources=None) -> str:
     h = hashlib.sha256()
     for p in sources or KERNEL_SOURCES:
@@ -618,7 +627,7 @@ def gpu_arm(args, rank, world, local_rank):
         "data": "synthetic (seeded N(0,1) values, lognormal/uniform lengths, random block placement)",
         "config": {
             "workload": args.workload,
-            "description": WORKLOADS[args.workload],
+            "description": describe(args),
             "num_seqs": B, "num_heads": sp.num_heads, "num_kv_heads": sp.num_kv_heads,
             "head_dim": sp.head_dim, "block_size": sp.block_size, "layers": L,
             "sum_context_tokens": int(wl.context_lens.sum()),
@@ -1114,7 +1123,7 @@ def reference_arm(args, rank):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": args.workload, "description": WORKLOADS[args.workload],
+        "config": {"workload": args.workload, "description": describe(args),
                    "block_size": sp.block_size},
         "tokens_per_s": round(nseq / dt, 2),
         "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "kind": "oracle",

@@ -54,4 +54,5 @@ def test_reference_arm_line():
     assert res["unit"] == "GB/s" and res["value"] > 0
     assert res["e2e"]["h2d_bytes_per_step"] == 0 and res["e2e"]["value"] == res["value"]
     assert res["cpu_baseline"]["kind"] == "oracle"
+    assert res["config"]["description"].endswith("(run with block_size 16)")
     assert bench.reference_arm(args, 1) is None                  # other ranks do nothing
