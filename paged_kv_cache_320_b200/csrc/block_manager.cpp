@@ -61,7 +61,11 @@ struct pkv_alloc {
     int max_blocks = 0;
     std::vector<int32_t> free_stack;  // back() is the next block handed out
     std::vector<int32_t> refcount;
-    std::unordered_map<int64_t, Seq> seqs;
+    // sequence records: a freed record's slot is reused with its vectors' capacity, so a
+    // steady fork / free cycle allocates no table memory
+    std::vector<Seq> pool;
+    std::vector<int32_t> free_slots;
+    std::unordered_map<int64_t, int32_t> index;   // sequence id -> slot in pool
     int64_t logical_tokens = 0;
     // prefix cache: chain hash -> cached block; blocks whose count fell to 0 while cached
     // wait, least recently released first, in `evictable` until a free block is needed
@@ -74,6 +78,36 @@ struct pkv_alloc {
     int64_t query_tokens = 0, hit_tokens = 0;
 
     int available() const { return (int)(free_stack.size() + evictable.size()); }
+
+    Seq *find(int64_t id) {
+        auto it = index.find(id);
+        return it == index.end() ? nullptr : &pool[it->second];
+    }
+    const Seq *find(int64_t id) const {
+        auto it = index.find(id);
+        return it == index.end() ? nullptr : &pool[it->second];
+    }
+
+    // An empty record for an id not in use; returns its slot. Growing the pool may move
+    // records: hold slots, not references, across this call.
+    int32_t add(int64_t id) {
+        int32_t slot;
+        if (!free_slots.empty()) {
+            slot = free_slots.back();
+            free_slots.pop_back();
+        } else {
+            slot = (int32_t)pool.size();
+            pool.emplace_back();
+        }
+        Seq &s = pool[slot];
+        s.table.clear();
+        s.len = 0;
+        s.tracked = false;
+        s.hash = 0;
+        s.partial.clear();
+        index.emplace(id, slot);
+        return slot;
+    }
 
     int32_t take() {
         int32_t b;
@@ -188,8 +222,7 @@ int append_impl(pkv_alloc *a, int64_t seq_id, int n_tokens, bool with_ids, const
                 int64_t *slots_out, int32_t *cow_pairs_out, int *n_cow_out) {
     if (!a || n_tokens < 0) return PKV_ERR_INVALID_ARG;
     if (n_tokens > 0 && !slots_out) return PKV_ERR_INVALID_ARG;
-    auto it = a->seqs.find(seq_id);
-    const Seq *existing = it == a->seqs.end() ? nullptr : &it->second;
+    const Seq *existing = a->find(seq_id);
     int64_t need, table_len;
     a->needs(existing, n_tokens, &need, &table_len);
     if (table_len > a->max_blocks) return PKV_ERR_TABLE_FULL;
@@ -198,7 +231,7 @@ int append_impl(pkv_alloc *a, int64_t seq_id, int n_tokens, bool with_ids, const
         a->refcount[existing->table.back()] > 1)
         return PKV_ERR_INVALID_ARG;  // a copy-on-write pair would be lost
     const bool created = !existing;
-    Seq &s = a->seqs[seq_id];
+    Seq &s = created ? a->pool[a->add(seq_id)] : *a->find(seq_id);
     if (created) s.tracked = a->prefix_cache && with_ids;
     const int bs = a->block_size;
     int n_cow = 0;
@@ -245,9 +278,9 @@ int pkv_alloc_set_prefix_cache(pkv_alloc *a, int enable) {
         a->evictable.clear();
         a->cache.clear();
         std::fill(a->cached.begin(), a->cached.end(), 0);
-        for (auto &kv : a->seqs) {
-            kv.second.tracked = false;
-            kv.second.partial.clear();
+        for (auto &kv : a->index) {
+            a->pool[kv.second].tracked = false;
+            a->pool[kv.second].partial.clear();
         }
     }
     a->prefix_cache = enable != 0;
@@ -257,7 +290,7 @@ int pkv_alloc_set_prefix_cache(pkv_alloc *a, int enable) {
 int pkv_seq_share_prefix(pkv_alloc *a, int64_t seq_id, const int32_t *tokens, int n_tokens,
                          int *n_cached_out) {
     if (!a || n_tokens < 0 || (n_tokens > 0 && !tokens)) return PKV_ERR_INVALID_ARG;
-    if (a->seqs.count(seq_id)) return PKV_ERR_SEQ_EXISTS;
+    if (a->index.count(seq_id)) return PKV_ERR_SEQ_EXISTS;
     Seq s;
     s.tracked = a->prefix_cache;
     const int bs = a->block_size;
@@ -280,7 +313,7 @@ int pkv_seq_share_prefix(pkv_alloc *a, int64_t seq_id, const int32_t *tokens, in
     }
     s.len = matched;
     a->logical_tokens += matched;
-    a->seqs.emplace(seq_id, std::move(s));
+    a->pool[a->add(seq_id)] = std::move(s);
     if (n_cached_out) *n_cached_out = matched;
     return PKV_OK;
 }
@@ -323,13 +356,20 @@ int pkv_seq_append_batch(pkv_alloc *a, const int64_t *seq_ids, int n, int n_toke
 
 int pkv_seq_fork(pkv_alloc *a, int64_t parent, int64_t child) {
     if (!a) return PKV_ERR_INVALID_ARG;
-    auto it = a->seqs.find(parent);
-    if (it == a->seqs.end()) return PKV_ERR_UNKNOWN_SEQ;
-    if (a->seqs.count(child)) return PKV_ERR_SEQ_EXISTS;
-    Seq copy = it->second;
-    for (int32_t b : copy.table) a->refcount[b] += 1;
-    a->logical_tokens += copy.len;
-    a->seqs.emplace(child, std::move(copy));
+    auto it = a->index.find(parent);
+    if (it == a->index.end()) return PKV_ERR_UNKNOWN_SEQ;
+    if (a->index.count(child)) return PKV_ERR_SEQ_EXISTS;
+    const int32_t from = it->second;
+    const int32_t to = a->add(child);
+    const Seq &p = a->pool[from];
+    Seq &c = a->pool[to];
+    c.table.assign(p.table.begin(), p.table.end());
+    c.len = p.len;
+    c.tracked = p.tracked;
+    c.hash = p.hash;
+    c.partial.assign(p.partial.begin(), p.partial.end());
+    for (int32_t b : c.table) a->refcount[b] += 1;
+    a->logical_tokens += c.len;
     return PKV_OK;
 }
 
@@ -358,14 +398,18 @@ int pkv_seq_free_batch(pkv_alloc *a, const int64_t *seq_ids, int n, int *n_done_
 
 int pkv_seq_free(pkv_alloc *a, int64_t seq_id) {
     if (!a) return PKV_ERR_INVALID_ARG;
-    auto it = a->seqs.find(seq_id);
-    if (it == a->seqs.end()) return PKV_ERR_UNKNOWN_SEQ;
-    const Seq &s = it->second;
+    auto it = a->index.find(seq_id);
+    if (it == a->index.end()) return PKV_ERR_UNKNOWN_SEQ;
+    const int32_t slot = it->second;
+    Seq &s = a->pool[slot];
     for (auto b = s.table.rbegin(); b != s.table.rend(); ++b) {
         a->release(*b);
     }
     a->logical_tokens -= s.len;
-    a->seqs.erase(it);
+    s.table.clear();
+    s.partial.clear();
+    a->index.erase(it);
+    a->free_slots.push_back(slot);
     return PKV_OK;
 }
 
@@ -374,9 +418,9 @@ int pkv_block_tables(const pkv_alloc *a, const int64_t *seq_ids, int n, int32_t 
     if (!a || n < 0 || (n > 0 && (!seq_ids || !tables_out))) return PKV_ERR_INVALID_ARG;
     const int mb = a->max_blocks;
     for (int i = 0; i < n; ++i) {
-        auto it = a->seqs.find(seq_ids[i]);
-        if (it == a->seqs.end()) return PKV_ERR_UNKNOWN_SEQ;
-        const Seq &s = it->second;
+        const Seq *sp = a->find(seq_ids[i]);
+        if (!sp) return PKV_ERR_UNKNOWN_SEQ;
+        const Seq &s = *sp;
         int32_t *row = tables_out + (size_t)i * mb;
         const int k = (int)s.table.size();
         std::memcpy(row, s.table.data(), sizeof(int32_t) * k);
