@@ -205,6 +205,7 @@ int check_decode_sizes(int B, int Hq, int Hkv, int D, int BS, int max_len, int p
         return PKV_ERR_INVALID_ARG;
     const long long pmax = max_len <= P ? 1 : cdiv(max_len, P);
     if ((long long)B * Hkv * pmax >= INT_MAX) return PKV_ERR_INVALID_ARG;
+    if ((long long)B * Hq >= INT_MAX) return PKV_ERR_INVALID_ARG;   // (sequence, head) pairs
     *P_out = P;
     return PKV_OK;
 }

@@ -72,6 +72,13 @@ def test_auto_partition_choices():
     assert pkv.pkv_decode_partition_size(4, 8, 8, 64, 16, 128) == 64          # tiny batch
 
 
+def test_pair_count_must_fit_an_int():
+    # 2^27 sequences x 16 query heads = 2^31 (sequence, head) pairs: refused on the host
+    with pytest.raises(pkv.PagedKVError):
+        pkv.pkv_decode_partition_size(1 << 27, 16, 1, 64, 16, 16)
+    assert pkv.pkv_decode_partition_size((1 << 27) - 1, 16, 1, 64, 16, 16) == 2048
+
+
 def test_shared_prefix_auto_partition_choices():
     f = pkv.pkv_decode_shared_prefix_partition_size
     assert f(128, 32, 8, 128, 16, 1300) == 1024        # G = 4: twice the plain path's 512
