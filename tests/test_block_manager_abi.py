@@ -169,3 +169,49 @@ def test_batched_fork_and_free_equal_calls_in_order(seed):
         assert (st, done) == (exp_st, exp_done)
         compare_states(c, m, sorted(m.tables))
     c.close()
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_many_sequences_forks_and_frees_match_the_model(seed):
+    """Hundreds of live sequences, fork chains and frees in a large pool: sequence records
+    are created, released and reused many times over (and their storage grows while
+    forks copy from it); every status, slot, copy-on-write pair and final table matches
+    the model."""
+    rng = np.random.default_rng(1000 + seed)
+    nb, bs, mb = 3000, int(rng.choice([4, 16])), 24
+    order = rng.permutation(nb)
+    c = BlockManager(nb, bs, mb, order)
+    m = BM.BlockManagerModel(nb, bs, mb, order)
+    live, next_id = [], 0
+    for step in range(1500):
+        r = rng.random()
+        if r < 0.35 or not live:
+            sid = next_id
+            next_id += 1
+            n = int(rng.integers(1, 3 * bs))
+            sc, slc, cwc = c.pkv_seq_append(sid, n)
+            sm, slm, cwm = m.append(sid, n)
+            assert sc == sm and slc.tolist() == slm, (seed, step)
+            if sc == 0:
+                live.append(sid)
+        elif r < 0.6:
+            parent = int(rng.choice(live))
+            child = next_id
+            next_id += 1
+            st = c.pkv_seq_fork(parent, child)
+            assert st == m.fork(parent, child), (seed, step)
+            if st == 0:
+                live.append(child)
+        elif r < 0.85:
+            sid = int(rng.choice(live))
+            n = int(rng.integers(0, bs + 2))
+            sc, slc, cwc = c.pkv_seq_append(sid, n)
+            sm, slm, cwm = m.append(sid, n)
+            assert sc == sm and slc.tolist() == slm, (seed, step)
+            assert cwc.tolist() == [list(x) for x in cwm]
+        else:
+            sid = live.pop(int(rng.integers(0, len(live))))
+            assert c.pkv_seq_free(sid) == m.free(sid)
+    assert len(live) > 100
+    compare_states(c, m, sorted(m.tables))
+    c.close()
