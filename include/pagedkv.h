@@ -57,7 +57,9 @@ enum pkv_status {
     PKV_ERR_BAD_INDEX = -6,     /* for callers that turn status-word bits into codes: an   */
     PKV_ERR_TIMEOUT = -7,       /* out-of-pool index / a wait that gave up (not returned)  */
     PKV_ERR_CUDA = -8,          /* a CUDA runtime call failed                             */
-    PKV_ERR_WORKSPACE = -9      /* workspace pointer NULL or smaller than required        */
+    PKV_ERR_WORKSPACE = -9,     /* workspace pointer NULL or smaller than required        */
+    PKV_ERR_HOST_MEMORY = -10   /* allocator: a host allocation failed; the call may have  */
+                                /* been partly applied: destroy the manager               */
 };
 
 enum pkv_dtype { PKV_F16 = 0, PKV_BF16 = 1 };

@@ -28,6 +28,7 @@ PKV_ERR_BAD_INDEX = -6
 PKV_ERR_TIMEOUT = -7
 PKV_ERR_CUDA = -8
 PKV_ERR_WORKSPACE = -9
+PKV_ERR_HOST_MEMORY = -10
 
 PKV_F16 = 0
 PKV_BF16 = 1

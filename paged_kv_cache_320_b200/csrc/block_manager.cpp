@@ -13,6 +13,7 @@
 #include <algorithm>
 #include <cstring>
 #include <list>
+#include <memory>
 #include <new>
 #include <unordered_map>
 #include <vector>
@@ -52,6 +53,18 @@ struct CachedBlock {
     std::vector<int32_t> tokens;  // its block_size token ids
     int32_t block;
 };
+
+// Runs f, turning any exception (a failed host allocation: std::bad_alloc, or a
+// container grown past its maximum size) into PKV_ERR_HOST_MEMORY, so that nothing
+// throws across the C ABI.
+template <class F>
+int guarded(F &&f) noexcept {
+    try {
+        return f();
+    } catch (...) {
+        return PKV_ERR_HOST_MEMORY;
+    }
+}
 
 }  // namespace
 
@@ -183,31 +196,33 @@ extern "C" {
 
 int pkv_alloc_create(pkv_alloc **out, int num_blocks, int block_size, int max_blocks_per_seq,
                      const int32_t *initial_order) {
-    if (!out || num_blocks <= 0 || block_size <= 0 || max_blocks_per_seq <= 0)
-        return PKV_ERR_INVALID_ARG;
-    *out = nullptr;
-    std::vector<char> seen(num_blocks, 0);
-    if (initial_order) {
-        for (int i = 0; i < num_blocks; ++i) {
-            const int32_t b = initial_order[i];
-            if (b < 0 || b >= num_blocks || seen[b]) return PKV_ERR_INVALID_ARG;
-            seen[b] = 1;
+    return guarded([&]() -> int {
+        if (!out || num_blocks <= 0 || block_size <= 0 || max_blocks_per_seq <= 0)
+            return PKV_ERR_INVALID_ARG;
+        *out = nullptr;
+        std::vector<char> seen(num_blocks, 0);
+        if (initial_order) {
+            for (int i = 0; i < num_blocks; ++i) {
+                const int32_t b = initial_order[i];
+                if (b < 0 || b >= num_blocks || seen[b]) return PKV_ERR_INVALID_ARG;
+                seen[b] = 1;
+            }
         }
-    }
-    pkv_alloc *a = new (std::nothrow) pkv_alloc();
-    if (!a) return PKV_ERR_INVALID_ARG;
-    a->num_blocks = num_blocks;
-    a->block_size = block_size;
-    a->max_blocks = max_blocks_per_seq;
-    a->refcount.assign(num_blocks, 0);
-    a->block_key.assign(num_blocks, 0);
-    a->cached.assign(num_blocks, 0);
-    a->evict_pos.resize(num_blocks);
-    a->free_stack.resize(num_blocks);
-    for (int i = 0; i < num_blocks; ++i)
-        a->free_stack[num_blocks - 1 - i] = initial_order ? initial_order[i] : i;
-    *out = a;
-    return PKV_OK;
+        std::unique_ptr<pkv_alloc> a(new (std::nothrow) pkv_alloc());
+        if (!a) return PKV_ERR_HOST_MEMORY;
+        a->num_blocks = num_blocks;
+        a->block_size = block_size;
+        a->max_blocks = max_blocks_per_seq;
+        a->refcount.assign(num_blocks, 0);
+        a->block_key.assign(num_blocks, 0);
+        a->cached.assign(num_blocks, 0);
+        a->evict_pos.resize(num_blocks);
+        a->free_stack.resize(num_blocks);
+        for (int i = 0; i < num_blocks; ++i)
+            a->free_stack[num_blocks - 1 - i] = initial_order ? initial_order[i] : i;
+        *out = a.release();
+        return PKV_OK;
+    });
 }
 
 int pkv_alloc_destroy(pkv_alloc *a) {
@@ -261,61 +276,69 @@ int append_impl(pkv_alloc *a, int64_t seq_id, int n_tokens, bool with_ids, const
 
 int pkv_seq_append(pkv_alloc *a, int64_t seq_id, int n_tokens, int64_t *slots_out,
                    int32_t *cow_pairs_out, int *n_cow_out) {
-    return append_impl(a, seq_id, n_tokens, false, nullptr, slots_out, cow_pairs_out, n_cow_out);
+    return guarded([&]() -> int {
+        return append_impl(a, seq_id, n_tokens, false, nullptr, slots_out, cow_pairs_out, n_cow_out);
+    });
 }
 
 int pkv_seq_append_tokens(pkv_alloc *a, int64_t seq_id, const int32_t *tokens, int n_tokens,
                           int64_t *slots_out, int32_t *cow_pairs_out, int *n_cow_out) {
-    if (n_tokens > 0 && !tokens) return PKV_ERR_INVALID_ARG;
-    return append_impl(a, seq_id, n_tokens, true, tokens, slots_out, cow_pairs_out, n_cow_out);
+    return guarded([&]() -> int {
+        if (n_tokens > 0 && !tokens) return PKV_ERR_INVALID_ARG;
+        return append_impl(a, seq_id, n_tokens, true, tokens, slots_out, cow_pairs_out, n_cow_out);
+    });
 }
 
 int pkv_alloc_set_prefix_cache(pkv_alloc *a, int enable) {
-    if (!a || (enable != 0 && enable != 1)) return PKV_ERR_INVALID_ARG;
-    if (a->prefix_cache && !enable) {
-        // forget every cached block; the ones nobody holds become free
-        for (int32_t b : a->evictable) a->free_stack.push_back(b);
-        a->evictable.clear();
-        a->cache.clear();
-        std::fill(a->cached.begin(), a->cached.end(), 0);
-        for (auto &kv : a->index) {
-            a->pool[kv.second].tracked = false;
-            a->pool[kv.second].partial.clear();
+    return guarded([&]() -> int {
+        if (!a || (enable != 0 && enable != 1)) return PKV_ERR_INVALID_ARG;
+        if (a->prefix_cache && !enable) {
+            // forget every cached block; the ones nobody holds become free
+            for (int32_t b : a->evictable) a->free_stack.push_back(b);
+            a->evictable.clear();
+            a->cache.clear();
+            std::fill(a->cached.begin(), a->cached.end(), 0);
+            for (auto &kv : a->index) {
+                a->pool[kv.second].tracked = false;
+                a->pool[kv.second].partial.clear();
+            }
         }
-    }
-    a->prefix_cache = enable != 0;
-    return PKV_OK;
+        a->prefix_cache = enable != 0;
+        return PKV_OK;
+    });
 }
 
 int pkv_seq_share_prefix(pkv_alloc *a, int64_t seq_id, const int32_t *tokens, int n_tokens,
                          int *n_cached_out) {
-    if (!a || n_tokens < 0 || (n_tokens > 0 && !tokens)) return PKV_ERR_INVALID_ARG;
-    if (a->index.count(seq_id)) return PKV_ERR_SEQ_EXISTS;
-    Seq s;
-    s.tracked = a->prefix_cache;
-    const int bs = a->block_size;
-    int matched = 0;
-    if (a->prefix_cache) {
-        for (int j = 0; (j + 1) * bs <= n_tokens && j < a->max_blocks; ++j) {
-            const int32_t *blk = tokens + (size_t)j * bs;
-            const uint64_t key = chain_hash(s.hash, blk, bs);
-            auto hit = a->cache.find(key);
-            if (hit == a->cache.end() || hit->second.parent != s.hash ||
-                std::memcmp(hit->second.tokens.data(), blk, sizeof(int32_t) * bs) != 0)
-                break;
-            a->acquire_cached(hit->second.block);
-            s.table.push_back(hit->second.block);
-            s.hash = key;
-            matched += bs;
+    return guarded([&]() -> int {
+        if (!a || n_tokens < 0 || (n_tokens > 0 && !tokens)) return PKV_ERR_INVALID_ARG;
+        if (a->index.count(seq_id)) return PKV_ERR_SEQ_EXISTS;
+        Seq s;
+        s.tracked = a->prefix_cache;
+        const int bs = a->block_size;
+        int matched = 0;
+        if (a->prefix_cache) {
+            for (int j = 0; (j + 1) * bs <= n_tokens && j < a->max_blocks; ++j) {
+                const int32_t *blk = tokens + (size_t)j * bs;
+                const uint64_t key = chain_hash(s.hash, blk, bs);
+                auto hit = a->cache.find(key);
+                if (hit == a->cache.end() || hit->second.parent != s.hash ||
+                    std::memcmp(hit->second.tokens.data(), blk, sizeof(int32_t) * bs) != 0)
+                    break;
+                a->acquire_cached(hit->second.block);
+                s.table.push_back(hit->second.block);
+                s.hash = key;
+                matched += bs;
+            }
+            a->query_tokens += n_tokens;
+            a->hit_tokens += matched;
         }
-        a->query_tokens += n_tokens;
-        a->hit_tokens += matched;
-    }
-    s.len = matched;
-    a->logical_tokens += matched;
-    a->pool[a->add(seq_id)] = std::move(s);
-    if (n_cached_out) *n_cached_out = matched;
-    return PKV_OK;
+        s.len = matched;
+        a->logical_tokens += matched;
+        a->pool[a->add(seq_id)] = std::move(s);
+        if (n_cached_out) *n_cached_out = matched;
+        return PKV_OK;
+    });
 }
 
 int pkv_prefix_cache_stats(const pkv_alloc *a, int *cached_blocks, int *evictable_blocks,
@@ -355,22 +378,24 @@ int pkv_seq_append_batch(pkv_alloc *a, const int64_t *seq_ids, int n, int n_toke
 }
 
 int pkv_seq_fork(pkv_alloc *a, int64_t parent, int64_t child) {
-    if (!a) return PKV_ERR_INVALID_ARG;
-    auto it = a->index.find(parent);
-    if (it == a->index.end()) return PKV_ERR_UNKNOWN_SEQ;
-    if (a->index.count(child)) return PKV_ERR_SEQ_EXISTS;
-    const int32_t from = it->second;
-    const int32_t to = a->add(child);
-    const Seq &p = a->pool[from];
-    Seq &c = a->pool[to];
-    c.table.assign(p.table.begin(), p.table.end());
-    c.len = p.len;
-    c.tracked = p.tracked;
-    c.hash = p.hash;
-    c.partial.assign(p.partial.begin(), p.partial.end());
-    for (int32_t b : c.table) a->refcount[b] += 1;
-    a->logical_tokens += c.len;
-    return PKV_OK;
+    return guarded([&]() -> int {
+        if (!a) return PKV_ERR_INVALID_ARG;
+        auto it = a->index.find(parent);
+        if (it == a->index.end()) return PKV_ERR_UNKNOWN_SEQ;
+        if (a->index.count(child)) return PKV_ERR_SEQ_EXISTS;
+        const int32_t from = it->second;
+        const int32_t to = a->add(child);
+        const Seq &p = a->pool[from];
+        Seq &c = a->pool[to];
+        c.table.assign(p.table.begin(), p.table.end());
+        c.len = p.len;
+        c.tracked = p.tracked;
+        c.hash = p.hash;
+        c.partial.assign(p.partial.begin(), p.partial.end());
+        for (int32_t b : c.table) a->refcount[b] += 1;
+        a->logical_tokens += c.len;
+        return PKV_OK;
+    });
 }
 
 int pkv_seq_fork_batch(pkv_alloc *a, const int64_t *parents, const int64_t *children, int n,
@@ -397,20 +422,22 @@ int pkv_seq_free_batch(pkv_alloc *a, const int64_t *seq_ids, int n, int *n_done_
 }
 
 int pkv_seq_free(pkv_alloc *a, int64_t seq_id) {
-    if (!a) return PKV_ERR_INVALID_ARG;
-    auto it = a->index.find(seq_id);
-    if (it == a->index.end()) return PKV_ERR_UNKNOWN_SEQ;
-    const int32_t slot = it->second;
-    Seq &s = a->pool[slot];
-    for (auto b = s.table.rbegin(); b != s.table.rend(); ++b) {
-        a->release(*b);
-    }
-    a->logical_tokens -= s.len;
-    s.table.clear();
-    s.partial.clear();
-    a->index.erase(it);
-    a->free_slots.push_back(slot);
-    return PKV_OK;
+    return guarded([&]() -> int {
+        if (!a) return PKV_ERR_INVALID_ARG;
+        auto it = a->index.find(seq_id);
+        if (it == a->index.end()) return PKV_ERR_UNKNOWN_SEQ;
+        const int32_t slot = it->second;
+        Seq &s = a->pool[slot];
+        for (auto b = s.table.rbegin(); b != s.table.rend(); ++b) {
+            a->release(*b);
+        }
+        a->logical_tokens -= s.len;
+        s.table.clear();
+        s.partial.clear();
+        a->index.erase(it);
+        a->free_slots.push_back(slot);
+        return PKV_OK;
+    });
 }
 
 int pkv_block_tables(const pkv_alloc *a, const int64_t *seq_ids, int n, int32_t *tables_out,

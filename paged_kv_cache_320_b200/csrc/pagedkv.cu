@@ -520,6 +520,7 @@ const char *pkv_status_string(int code) {
         case PKV_ERR_TIMEOUT: return "bounded device wait gave up";
         case PKV_ERR_CUDA: return "CUDA runtime error";
         case PKV_ERR_WORKSPACE: return "workspace missing or too small";
+        case PKV_ERR_HOST_MEMORY: return "host allocation failed in the block manager";
     }
     return "unknown status";
 }

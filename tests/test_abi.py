@@ -131,8 +131,8 @@ def test_cache_op_checks_without_a_device():
 
 def test_status_strings():
     L = B.lib()
-    for code in range(-9, 1):
-        assert L.pkv_status_string(code)
+    for code in range(-10, 1):
+        assert L.pkv_status_string(code) != b"unknown status", code
 
 
 def test_step_and_shared_prefix_checks_without_a_device():

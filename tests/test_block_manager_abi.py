@@ -215,3 +215,34 @@ def test_many_sequences_forks_and_frees_match_the_model(seed):
     assert len(live) > 100
     compare_states(c, m, sorted(m.tables))
     c.close()
+
+
+GUARD_PROBE = r"""
+import ctypes, resource, sys
+sys.path.insert(0, sys.argv[1])
+from paged_kv_cache_320_b200 import _binding as B
+L = B.lib()
+size = next(int(l.split()[1]) * 1024 for l in open("/proc/self/status") if l.startswith("VmSize:"))
+cap = size + (256 << 20)
+resource.setrlimit(resource.RLIMIT_AS, (cap, cap))
+h = ctypes.c_void_p()
+print(L.pkv_alloc_create(ctypes.byref(h), 100_000_000, 16, 8, None), h.value is None)
+print(L.pkv_alloc_create(ctypes.byref(h), 1000, 16, 8, None), h.value is not None)
+"""
+
+
+@pytest.mark.skipif(not os.path.exists("/proc/self/status"), reason="needs Linux /proc")
+def test_host_allocation_failure_is_a_status_not_an_exception():
+    """A manager too large for the process's address-space limit: std::bad_alloc inside
+    the library comes back as PKV_ERR_HOST_MEMORY (no exception crosses the C ABI, no
+    handle is returned), and the next, small manager is created normally."""
+    import subprocess
+    import sys
+    from paged_kv_cache_320_b200 import _binding as B
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", GUARD_PROBE, root], capture_output=True,
+                       text=True, timeout=120)
+    assert r.returncode == 0, r.stderr
+    lines = r.stdout.split("\n")
+    assert lines[0] == f"{B.PKV_ERR_HOST_MEMORY} True"
+    assert lines[1] == f"{B.PKV_OK} True"
