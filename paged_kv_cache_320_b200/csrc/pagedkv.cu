@@ -9,6 +9,7 @@
 #include <climits>
 #include <cmath>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <utility>
 
@@ -237,12 +238,14 @@ int launch_decode(const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMa
     const size_t smem = L::smem_bytes(prm.group);
     int dev;
     if (current_device(&dev) != PKV_OK) return PKV_ERR_CUDA;
-    static int occ[kMaxDevices][pkv::kMaxGroup + 1];
+    // blocks per SM, cached per device and group size (read without the lock)
+    static std::atomic<int> occ[kMaxDevices][pkv::kMaxGroup + 1];
     static bool attr_set[kMaxDevices];
     int nsm;
     if (sm_count(&nsm) != PKV_OK) return PKV_ERR_CUDA;
-    int &o = occ[dev][prm.group];
-    if (o == 0) {
+    std::atomic<int> &o = occ[dev][prm.group];
+    int per_sm = o.load(std::memory_order_acquire);
+    if (per_sm == 0) {
         std::lock_guard<std::mutex> lk(g_mu);
         // the largest layout any group size needs, so every later launch fits
         if (!attr_set[dev]) {
@@ -256,9 +259,10 @@ int launch_decode(const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMa
                 cudaSuccess ||
             n <= 0)
             return PKV_ERR_CUDA;
-        o = n;
+        o.store(n, std::memory_order_release);
+        per_sm = n;
     }
-    long long grid = (long long)nsm * o;
+    long long grid = (long long)nsm * per_sm;
     if (grid > items_upper) grid = items_upper;
     if (grid < 1) grid = 1;
     return launch(kern, dim3((unsigned)grid), dim3(pkv::kDecodeThreads), smem, st, mk, mv, mq, prm);
@@ -313,10 +317,11 @@ int launch_shared_decode(const CUtensorMap &mk, const CUtensorMap &mv,
     const size_t smem = 1024 + L::kRingBytes + L::obuf_bytes(pkv::kMaxGroup) + L::kMetaBytes;
     int dev;
     if (current_device(&dev) != PKV_OK) return PKV_ERR_CUDA;
-    static int occ[kMaxDevices];
+    static std::atomic<int> occ[kMaxDevices];   // blocks per SM (read without the lock)
     int nsm;
     if (sm_count(&nsm) != PKV_OK) return PKV_ERR_CUDA;
-    if (occ[dev] == 0) {
+    int per_sm = occ[dev].load(std::memory_order_acquire);
+    if (per_sm == 0) {
         std::lock_guard<std::mutex> lk(g_mu);
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
             cudaSuccess)
@@ -326,9 +331,10 @@ int launch_shared_decode(const CUtensorMap &mk, const CUtensorMap &mv,
                 cudaSuccess ||
             n <= 0)
             return PKV_ERR_CUDA;
-        occ[dev] = n;
+        occ[dev].store(n, std::memory_order_release);
+        per_sm = n;
     }
-    long long grid = (long long)nsm * occ[dev];
+    long long grid = (long long)nsm * per_sm;
     if (grid > prm.max_items) grid = prm.max_items;
     if (grid < 1) grid = 1;
     return launch(kern, dim3((unsigned)grid), dim3(pkv::kDecodeThreads), smem, st, mk, mv, prm);
@@ -423,12 +429,14 @@ int launch_step(const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap 
     const size_t smem = L::smem_bytes(prm.group);
     int dev;
     if (current_device(&dev) != PKV_OK) return PKV_ERR_CUDA;
-    static int occ[kMaxDevices][pkv::kMaxGroup + 1];
+    // blocks per SM, cached per device and group size (read without the lock)
+    static std::atomic<int> occ[kMaxDevices][pkv::kMaxGroup + 1];
     static bool attr_set[kMaxDevices];
     int nsm;
     if (sm_count(&nsm) != PKV_OK) return PKV_ERR_CUDA;
-    int &o = occ[dev][prm.group];
-    if (o == 0) {
+    std::atomic<int> &o = occ[dev][prm.group];
+    int per_sm = o.load(std::memory_order_acquire);
+    if (per_sm == 0) {
         std::lock_guard<std::mutex> lk(g_mu);
         if (!attr_set[dev]) {
             if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -441,9 +449,10 @@ int launch_step(const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap 
                 cudaSuccess ||
             n <= 0)
             return PKV_ERR_CUDA;
-        o = n;
+        o.store(n, std::memory_order_release);
+        per_sm = n;
     }
-    long long grid = (long long)nsm * o;
+    long long grid = (long long)nsm * per_sm;
     if (grid > items) grid = items;
     if (grid < 1) grid = 1;
     // the merge phase waits at a grid barrier: all CTAs must be resident at once
