@@ -1,6 +1,6 @@
 """Host-side pieces of bench.py (CPU only): algorithmic bytes against their formula, the
-profile-traffic lookup gated by the kernel-source hash, and the reference arm (the CPU
-oracle) producing its JSON line."""
+profile-traffic lookup gated by the kernel-source hash, the reference arm (the CPU
+oracle) producing its JSON line, and the parsing of sampled GPU clocks."""
 import argparse
 import os
 
@@ -56,3 +56,24 @@ def test_reference_arm_line():
     assert res["cpu_baseline"]["kind"] == "oracle"
     assert res["config"]["description"].endswith("(run with block_size 16)")
     assert bench.reference_arm(args, 1) is None                  # other ranks do nothing
+
+
+def test_clock_summary_parses_nvidia_smi_samples():
+    """Median SM clock, max clock and the throttle reasons that were active in any sample
+    ("Not Active" must not count); malformed lines are skipped."""
+    s = bench.ClockSampler.__new__(bench.ClockSampler)
+    s.lines = [
+        "0, 1965, 1965, 700.1, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "0, 1740, 1965, 998.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1800, 1965, 990.5, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, [N/A], 1965, 1.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "garbage",
+    ]
+    r = s.summary()
+    assert r == {"sm_mhz": 1800.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"],
+                 "samples": 3}
+    s.lines = ["0, 1200, 1965, 500, 0x8, Active, Not Active, Active, Not Active"]
+    assert s.summary()["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
+    s.lines = []
+    assert s.summary() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"],
+                           "samples": 0}
