@@ -159,8 +159,9 @@ int pkv_paged_attention_decode_noalloc(void *out, const void *q, const void *k_c
  *              the first logical block where a member's table differs from the group's
  *              first member — a wrong value costs sharing, never correctness.
  * A malformed group_start is treated as one group per sequence and sets
- * PKV_STATUS_BAD_LEN. Workspace: pkv_decode_shared_prefix_workspace_size bytes, no
- * initial contents required. partition_size 0 selects this path's own automatic size
+ * PKV_STATUS_BAD_LEN. Workspace: pkv_decode_shared_prefix_workspace_size bytes of device
+ * memory, 16-byte aligned, owned by the caller, no initial contents required (else
+ * PKV_ERR_WORKSPACE). partition_size 0 selects this path's own automatic size
  * (pkv_decode_shared_prefix_partition_size: 1024 tokens for groups up to 4, 2048 above,
  * at most 256 blocks, smaller for small batches). Other arguments, limits and errors as
  * pkv_paged_attention_decode (num_groups >= 1, <= num_seqs). Three kernel launches.
