@@ -906,6 +906,7 @@ def e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, worl
         bt_dev = torch.from_numpy(tables).to(dev)
         lens_dev = torch.from_numpy(lens).to(dev)
         free_d = torch.from_numpy(mgr.pkv_alloc_free_list()).to(dev)
+        refc_d = torch.from_numpy(mgr.pkv_alloc_refcounts()).to(dev)
         used_d = torch.zeros(1, dtype=torch.int32, device=dev)
     copy_in = torch.cuda.Stream(dev)
     copy_out = torch.cuda.Stream(dev)
@@ -953,7 +954,7 @@ def e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, worl
             ev_tables[b].record(copy_in)
         else:
             pkv.pkv_device_append(bt_dev, lens_dev, free_d, used_d, wl.num_blocks, max_len,
-                                  sp.block_size, stream=stream)
+                                  sp.block_size, block_refcounts=refc_d, stream=stream)
         stream.wait_event(ev_d2h_done[b])   # out_d[b] has been read back
         for l in range(L):
             with torch.cuda.stream(copy_in):

@@ -72,7 +72,9 @@ enum pkv_device_status_bits {
     PKV_STATUS_BAD_LEN = 1u << 3,      /* decode: context_len < 0 or above its bound (clamped)  */
     PKV_STATUS_WAIT_TIMEOUT = 1u << 4, /* decode: a pipeline wait exceeded its iteration limit  */
     PKV_STATUS_NO_BLOCKS = 1u << 5,    /* device append: step refused, nothing changed          */
-    PKV_STATUS_WORKSPACE = 1u << 6     /* workspace not prepared for the call (step, planned)   */
+    PKV_STATUS_WORKSPACE = 1u << 6,    /* workspace not prepared for the call (step, planned)   */
+    PKV_STATUS_SHARED_BLOCK = 1u << 7  /* device append refused: a sequence would write into a  */
+                                       /* shared, partly filled block (copy-on-write needed)    */
 };
 
 /* Human-readable name of a status code (static string). */
@@ -284,20 +286,27 @@ int pkv_swap_blocks(void *const *k_caches, void *const *v_caches, int num_layers
  *   with PKV_STATUS_BAD_BLOCK, if that entry is outside [0, num_blocks));
  *   context_lens[s] = n + 1; finally *free_used += blocks taken.
  * With free_blocks holding the host block manager's free blocks in the order it would
- * pop them, the result equals pkv_seq_append(.., 1, ..) on s = 0, 1, ... (no sequence may
- * share its partly filled last block: copy-on-write stays on the host).
+ * pop them, the result equals pkv_seq_append(.., 1, ..) on s = 0, 1, ... as long as no
+ * sequence writes into a block it shares: copy-on-write ("分页 KV Cache 分析" §3.2, copy a
+ * shared page before changing it) stays on the host. block_refcounts (device int32
+ * [num_blocks], the host manager's counts from pkv_alloc_refcounts, uploaded after its
+ * last fork or free; NULL = the caller guarantees that nothing is shared) lets the kernel
+ * check this: a sequence with n % block_size != 0 whose block block_tables[s][n /
+ * block_size] has a count above 1 refuses the step (PKV_STATUS_SHARED_BLOCK). Blocks the
+ * device append itself took from free_blocks count 0 there: they are private.
  * All or nothing: if fewer than the needed entries remain (free_count - *free_used), an
  * entry is outside [0, num_blocks), some n < 0, n + 1 > max_context_len or
  * n / block_size >= max_blocks_per_seq, nothing is written and PKV_STATUS_NO_BLOCKS is
- * set. block_tables int32 [num_seqs][max_blocks_per_seq], context_lens int32 [num_seqs],
- * free_blocks int32 [free_count], free_used int32 [1] (all device), slots_out int64
- * [num_seqs] device or NULL. One CTA; asynchronous on `stream`.
- * Errors: PKV_ERR_INVALID_ARG, PKV_ERR_CUDA.
+ * set; a shared block as above also writes nothing and sets PKV_STATUS_NO_BLOCKS |
+ * PKV_STATUS_SHARED_BLOCK. block_tables int32 [num_seqs][max_blocks_per_seq],
+ * context_lens int32 [num_seqs], free_blocks int32 [free_count], free_used int32 [1]
+ * (all device), slots_out int64 [num_seqs] device or NULL. One CTA; asynchronous on
+ * `stream`. Errors: PKV_ERR_INVALID_ARG, PKV_ERR_CUDA.
  * ---------------------------------------------------------------------------- */
 int pkv_device_append(int32_t *block_tables, int32_t *context_lens, const int32_t *free_blocks,
-                      int free_count, int32_t *free_used, int64_t *slots_out, int num_seqs,
-                      int max_blocks_per_seq, int block_size, int num_blocks,
-                      int max_context_len, pkv_stream_t stream);
+                      int free_count, int32_t *free_used, const int32_t *block_refcounts,
+                      int64_t *slots_out, int num_seqs, int max_blocks_per_seq, int block_size,
+                      int num_blocks, int max_context_len, pkv_stream_t stream);
 
 /* pkv_paged_decode_step (once per layer): one launch that writes every sequence's newest
  * token and computes the decode attention over it:
@@ -309,9 +318,14 @@ int pkv_device_append(int32_t *block_tables, int32_t *context_lens, const int32_
  * plus k_new / v_new [num_seqs][num_kv_heads][head_dim] device, 16-byte aligned.
  * Workspace: pkv_decode_step_workspace_size bytes (at least 256), 256-byte aligned, owned
  * by the caller, ZERO-FILLED before its first use and then reused only by this call on one
- * stream (each launch leaves it ready for the next). A launch that merges in the step
- * kernel refuses, on the device, a workspace whose header is neither zero nor left by
- * these kernels (PKV_STATUS_WORKSPACE, no output).
+ * stream (each launch leaves it ready for the next). A workspace that
+ * pkv_paged_attention_decode has used with several partitions (same layout; its merge
+ * kernel re-arms the header) also serves. A launch that merges in the step kernel
+ * refuses, on the device and before any write, a header that is none of these: zero
+ * (with a zero barrier generation), or left by these kernels with a zero exit count
+ * (PKV_STATUS_WORKSPACE, no output). A stale arrival count, which cannot be checked at
+ * the start, is caught at the grid barrier (PKV_STATUS_WORKSPACE; do not use that
+ * launch's output); the launch still leaves the header ready for the next one.
  * When some context spans several partitions they are merged either in the same launch
  * (cooperative, all CTAs resident: after a bounded grid barrier every warp merges
  * (sequence, head) pairs; PKV_STATUS_WAIT_TIMEOUT if the barrier gives up), chosen when
@@ -396,6 +410,12 @@ int pkv_seq_free_batch(pkv_alloc *a, const int64_t *seq_ids, int n, int *n_done_
  * blocks_out, their count into *n_out. Uploaded to the device, this is the free list
  * pkv_device_append takes from. */
 int pkv_alloc_free_list(const pkv_alloc *a, int32_t *blocks_out, int max_out, int *n_out);
+
+/* The reference count of every block (sequences whose table holds it; 0 = free or cached
+ * and unheld) into the host array refcounts_out [n], n >= num_blocks (entries past
+ * num_blocks untouched). Uploaded to the device, it is the block_refcounts argument of
+ * pkv_device_append. Errors: PKV_ERR_INVALID_ARG. */
+int pkv_alloc_refcounts(const pkv_alloc *a, int32_t *refcounts_out, int n);
 
 /* ------------------------------------------------------------------------------
  * Prefix caching ("分页 KV Cache 分析" §2.3 and §3.2: common prefixes such as a system

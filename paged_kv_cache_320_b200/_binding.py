@@ -40,6 +40,7 @@ STATUS_BAD_LEN = 1 << 3
 STATUS_WAIT_TIMEOUT = 1 << 4
 STATUS_NO_BLOCKS = 1 << 5
 STATUS_WORKSPACE = 1 << 6
+STATUS_SHARED_BLOCK = 1 << 7
 
 _lib = None
 
@@ -90,7 +91,8 @@ def lib() -> ctypes.CDLL:
         L.pkv_paged_decode_step.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I,
                                             ctypes.c_float, I, I, P, SZ, P]
         L.pkv_decode_step_workspace_size.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(SZ)]
-        L.pkv_device_append.argtypes = [P, P, P, I, P, P, I, I, I, I, I, P]
+        L.pkv_device_append.argtypes = [P, P, P, I, P, P, P, I, I, I, I, I, P]
+        L.pkv_alloc_refcounts.argtypes = [P, P, I]
         L.pkv_decode_step_launches.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(I)]
         L.pkv_alloc_free_list.argtypes = [P, P, I, ctypes.POINTER(I)]
         L.pkv_shared_prefix_plan.argtypes = [P, P, P, P, I, I, I, I, I, I, I, I, I, P, SZ, P]
@@ -114,7 +116,8 @@ def lib() -> ctypes.CDLL:
                      "pkv_seq_append", "pkv_seq_append_batch", "pkv_seq_fork", "pkv_seq_free",
                      "pkv_block_tables", "pkv_stats", "pkv_alloc_set_prefix_cache",
                      "pkv_paged_decode_step", "pkv_decode_step_workspace_size", "pkv_device_append",
-                     "pkv_alloc_free_list", "pkv_decode_step_launches", "pkv_seq_fork_batch",
+                     "pkv_alloc_free_list", "pkv_alloc_refcounts", "pkv_decode_step_launches",
+                     "pkv_seq_fork_batch",
                      "pkv_seq_free_batch", "pkv_shared_prefix_plan",
                      "pkv_paged_attention_decode_shared_prefix_planned",
                      "pkv_seq_append_tokens", "pkv_seq_share_prefix", "pkv_prefix_cache_stats"):
@@ -369,10 +372,13 @@ def pkv_paged_decode_step(out, q, k_new, v_new, k_cache, v_cache, block_tables, 
 
 
 def pkv_device_append(block_tables, context_lens, free_blocks, free_used, num_blocks,
-                      max_context_len, block_size, slots_out=None, stream=None):
+                      max_context_len, block_size, slots_out=None, block_refcounts=None,
+                      stream=None):
     """One token appended to every sequence on the device (see pagedkv.h): block_tables
     int32 [B, MB] and context_lens int32 [B] updated in place; free_blocks int32 [F] in pop
-    order; free_used int32 [1] advanced by the blocks taken; slots_out int64 [B] or None."""
+    order; free_used int32 [1] advanced by the blocks taken; slots_out int64 [B] or None;
+    block_refcounts int32 [num_blocks] (the host manager's pkv_alloc_refcounts) or None:
+    with it, a write into a shared partly filled block refuses the step."""
     import torch
     _need(context_lens, "context_lens", None, torch.int32)
     B = context_lens.numel()
@@ -382,10 +388,13 @@ def pkv_device_append(block_tables, context_lens, free_blocks, free_used, num_bl
     _need(free_used, "free_used", dev, torch.int32, 1)
     if slots_out is not None:
         _need(slots_out, "slots_out", dev, torch.int64, B)
+    if block_refcounts is not None:
+        _need(block_refcounts, "block_refcounts", dev, torch.int32, int(num_blocks))
     _check(lib().pkv_device_append(
         _ptr(block_tables), _ptr(context_lens), _ptr(free_blocks), free_blocks.numel(),
-        _ptr(free_used), _ptr(slots_out), B, block_tables.shape[1], int(block_size),
-        int(num_blocks), int(max_context_len), _stream(stream)), "pkv_device_append")
+        _ptr(free_used), _ptr(block_refcounts), _ptr(slots_out), B, block_tables.shape[1],
+        int(block_size), int(num_blocks), int(max_context_len), _stream(stream)),
+        "pkv_device_append")
 
 
 def pkv_shared_prefix_plan(block_tables, context_lens, group_start, prefix_lens, num_heads,
@@ -543,6 +552,14 @@ class BlockManager:
         _check(lib().pkv_alloc_free_list(self._h, buf.ctypes.data, m, ctypes.byref(n)),
                "pkv_alloc_free_list")
         return buf[:n.value].copy()
+
+    def pkv_alloc_refcounts(self):
+        """Reference count of every block (int32 array of num_blocks)."""
+        import numpy as np
+        buf = np.zeros(self.num_blocks, dtype=np.int32)
+        _check(lib().pkv_alloc_refcounts(self._h, buf.ctypes.data, self.num_blocks),
+               "pkv_alloc_refcounts")
+        return buf
 
     def pkv_alloc_set_prefix_cache(self, enable):
         return lib().pkv_alloc_set_prefix_cache(self._h, int(bool(enable)))

@@ -468,6 +468,12 @@ int pkv_alloc_free_list(const pkv_alloc *a, int32_t *blocks_out, int max_out, in
     return PKV_OK;
 }
 
+int pkv_alloc_refcounts(const pkv_alloc *a, int32_t *refcounts_out, int n) {
+    if (!a || !refcounts_out || n < a->num_blocks) return PKV_ERR_INVALID_ARG;
+    std::copy(a->refcount.begin(), a->refcount.end(), refcounts_out);
+    return PKV_OK;
+}
+
 int pkv_stats(const pkv_alloc *a, int *free_blocks, int *held_blocks, int64_t *logical_tokens,
               double *utilisation) {
     if (!a) return PKV_ERR_INVALID_ARG;

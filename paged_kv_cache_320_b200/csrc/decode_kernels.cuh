@@ -64,15 +64,21 @@ struct StageInfo {
 constexpr int kFirst = 1, kLast = 2, kEnd = 4;
 
 // Dynamic work distribution: producers take item indices from `next`. The reduce
-// kernel, which follows every decode that has a workspace, re-arms it (next = 0,
-// armed = kSchedArmed) for the next call; a header that is not armed (a workspace
-// never used before) makes that call fall back to the static schedule.
+// kernel, which follows every decode that has a workspace, re-arms it (next = 0, the
+// step kernel's barrier counters 0, armed = kSchedArmed) for the next call; a header
+// that is not armed (a workspace never used before) makes that call fall back to the
+// static schedule. The same header serves paged_decode_step_kernel, whose grid
+// barrier and exit count live in `arrive`, `gen` and `exit` (unused by the others).
 constexpr unsigned kSchedArmed = 0x9A6EDC0Du;
 struct SchedHeader {
     unsigned armed;
-    int next;
-    int pad[62];
+    int next;         // dynamic work counter
+    unsigned arrive;  // step kernel: CTAs arrived at the grid barrier
+    unsigned gen;     // step kernel: barrier generation
+    unsigned exit;    // step kernel: CTAs finished
+    int pad[59];
 };
+static_assert(sizeof(SchedHeader) == 256, "workspace header size");
 
 struct DecodeParams {
     SchedHeader *sched;  // null: static schedule (items blockIdx.x + k * gridDim.x)
@@ -938,8 +944,12 @@ __global__ void __launch_bounds__(kReduceWarps * 32)
 paged_decode_reduce_kernel(DecodeParams prm) {
     pdl_wait_and_release();
     if (blockIdx.x == 0 && threadIdx.x == 0 && prm.sched) {
-        // every decode CTA has finished (stream order): re-arm the scheduler
+        // every decode CTA has finished (stream order): re-arm the scheduler, and clear
+        // the step kernel's counters so that a workspace a plain decode used is also a
+        // valid step workspace
         prm.sched->next = 0;
+        prm.sched->arrive = 0;
+        prm.sched->exit = 0;
         __threadfence();
         prm.sched->armed = kSchedArmed;
     }

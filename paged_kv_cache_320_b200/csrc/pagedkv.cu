@@ -782,9 +782,9 @@ int pkv_decode_step_launches(int num_seqs, int num_heads, int num_kv_heads, int 
 }
 
 int pkv_device_append(int32_t *block_tables, int32_t *context_lens, const int32_t *free_blocks,
-                      int free_count, int32_t *free_used, int64_t *slots_out, int num_seqs,
-                      int max_blocks_per_seq, int block_size, int num_blocks,
-                      int max_context_len, pkv_stream_t stream) {
+                      int free_count, int32_t *free_used, const int32_t *block_refcounts,
+                      int64_t *slots_out, int num_seqs, int max_blocks_per_seq, int block_size,
+                      int num_blocks, int max_context_len, pkv_stream_t stream) {
     if (num_seqs < 0 || free_count < 0 || max_blocks_per_seq < 1 || block_size < 1 ||
         num_blocks < 1 || max_context_len < 0)
         return PKV_ERR_INVALID_ARG;
@@ -793,14 +793,15 @@ int pkv_device_append(int32_t *block_tables, int32_t *context_lens, const int32_
     if (num_seqs > 0 && (!block_tables || !context_lens)) return PKV_ERR_INVALID_ARG;
     if (free_count > 0 && !free_blocks) return PKV_ERR_INVALID_ARG;
     if (!aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(free_blocks, 4) ||
-        !aligned(free_used, 4) || !aligned(slots_out, 8))
+        !aligned(free_used, 4) || !aligned(block_refcounts, 4) || !aligned(slots_out, 8))
         return PKV_ERR_INVALID_ARG;
     unsigned int *status;
     int rc;
     if ((rc = device_status_ptr(&status)) != PKV_OK) return rc;
     return launch(pkv::device_append_kernel, dim3(1), dim3(pkv::kPlanThreads), 0,
                   reinterpret_cast<cudaStream_t>(stream), block_tables, context_lens, free_blocks,
-                  free_count, reinterpret_cast<int *>(free_used), slots_out, num_seqs,
+                  free_count, reinterpret_cast<int *>(free_used), block_refcounts, slots_out,
+                  num_seqs,
                   max_blocks_per_seq, block_size, num_blocks, max_context_len, status);
 }
 

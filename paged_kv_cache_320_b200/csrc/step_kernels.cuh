@@ -28,20 +28,17 @@ namespace pkv {
 
 constexpr unsigned kStatusNoBlocks = 1u << 5;
 constexpr unsigned kStatusWorkspace = 1u << 6;
+constexpr unsigned kStatusSharedBlock = 1u << 7;
 
-// Workspace header of the step kernel. It overlays SchedHeader (`armed`, `next` at the
-// same offsets) and holds the grid barrier. Zero-filled, or left by a previous step
-// launch (armed == kStepArmed), it is valid; anything else is rejected.
+// Workspace header of the step kernel: SchedHeader, whose `arrive`, `gen` and `exit`
+// hold the grid barrier and the exit count. Valid at launch: zero-filled (armed, gen
+// and exit 0), left by a previous step launch (armed == kStepArmed: the last CTA out
+// cleared the counters) or re-armed by paged_decode_reduce_kernel (armed ==
+// kSchedArmed: it cleared them too), always with exit == 0. Anything else is refused
+// before any write. `arrive` cannot be checked at the start (a CTA may reach the
+// barrier before another has started); a stale value is caught at the barrier instead.
 constexpr unsigned kStepArmed = 0x57E9A11Du;
-struct StepHeader {
-    unsigned armed;
-    int next;         // dynamic work counter
-    unsigned arrive;  // CTAs arrived at the barrier
-    unsigned gen;     // barrier generation
-    unsigned exit;    // CTAs finished
-    int pad[59];
-};
-static_assert(sizeof(StepHeader) == sizeof(SchedHeader), "header size");
+using StepHeader = SchedHeader;
 
 constexpr uint32_t kBarrierPolls = 1u << 22;
 
@@ -53,13 +50,17 @@ __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p) {
 
 // Grid-wide barrier for a co-resident grid; bounded (returns false when it gave up).
 // gen0 is the header's generation read at kernel start (it cannot change before every
-// CTA has arrived, so every CTA read the same value).
-__device__ __forceinline__ bool grid_barrier(StepHeader *h, unsigned gen0, int *flag) {
+// CTA has arrived, so every CTA read the same value). An arrival count at or past the
+// grid size means the header came in with a stale count: flagged as a workspace error
+// (the release may then have come early, so the launch's output is not to be used).
+__device__ __forceinline__ bool grid_barrier(StepHeader *h, unsigned gen0, int *flag,
+                                             unsigned *status) {
     __syncthreads();
     if (threadIdx.x == 0) {
         int ok = 1;
         __threadfence();
         const unsigned t = atomicAdd(&h->arrive, 1u);
+        if (t >= gridDim.x) atomicOr(status, kStatusWorkspace);
         if (t == gridDim.x - 1) {
             h->arrive = 0;
             __threadfence();
@@ -95,11 +96,15 @@ paged_decode_step_kernel(const __grid_constant__ CUtensorMap tmap_k,
     if (threadIdx.x == 0) {
         int ok = 1;
         if (hdr) {
+            // Read before this launch can change them: `armed` is written only by the last
+            // CTA out, `gen` only at the barrier's release and, with the merge (the only
+            // way this kernel is launched with a header), `exit` only after the barrier,
+            // which every CTA reaches after this check. So every CTA decides alike.
             const unsigned a = *(volatile unsigned *)&hdr->armed;
-            // zero-filled, left by this kernel, or re-armed by paged_decode_reduce_kernel
-            // (which leaves the barrier words as this kernel left them)
-            ok = a == 0u || a == kStepArmed || a == kSchedArmed;
-            s_gen = *(volatile unsigned *)&hdr->gen;
+            const unsigned g = *(volatile unsigned *)&hdr->gen;
+            const unsigned ex = merge ? *(volatile unsigned *)&hdr->exit : 0u;
+            ok = (a == kStepArmed || a == kSchedArmed || (a == 0u && g == 0u)) && ex == 0u;
+            s_gen = g;
             if (!ok && blockIdx.x == 0) atomicOr(prm.status, kStatusWorkspace);
         }
         s_flag = ok;
@@ -111,7 +116,7 @@ paged_decode_step_kernel(const __grid_constant__ CUtensorMap tmap_k,
     if (!hdr) return;
 
     if (merge) {
-        if (grid_barrier(hdr, s_gen, &s_flag)) {
+        if (grid_barrier(hdr, s_gen, &s_flag, prm.status)) {
             const int lane = threadIdx.x & 31;
             const int nwarps = gridDim.x * (kDecodeThreads / 32);
             const int G = prm.group, P = prm.partition;
@@ -153,30 +158,41 @@ paged_decode_step_kernel(const __grid_constant__ CUtensorMap tmap_k,
 //   n = context_lens[s];  if n % BS == 0: block_tables[s][n / BS] = free_blocks[used + r_s]
 //   (r_s = number of sequences before s that take a block);  slot_s =
 //   block_tables[s][n / BS] * BS + n % BS;  context_lens[s] = n + 1;  *free_used += taken.
+// With refcounts (the host manager's per-block counts), a sequence that would write into
+// a partly filled block held by more than one sequence refuses the step: that write
+// needs the copy-on-write of the host manager first.
 __global__ void __launch_bounds__(kPlanThreads)
 device_append_kernel(int32_t *block_tables, int32_t *context_lens, const int32_t *free_blocks,
-                     int free_count, int *free_used, int64_t *slots_out, int B, int MB, int BS,
-                     int num_blocks, int max_len, unsigned *status) {
+                     int free_count, int *free_used, const int32_t *refcounts, int64_t *slots_out,
+                     int B, int MB, int BS, int num_blocks, int max_len, unsigned *status) {
     pdl_wait_and_release();
     __shared__ int sm[kPlanThreads / 32];
-    __shared__ int s_used, s_bad;
+    __shared__ int s_used, s_bad, s_shared;
     const int tid = threadIdx.x;
     if (tid == 0) {
         s_used = *free_used;
         s_bad = 0;
+        s_shared = 0;
     }
     __syncthreads();
     const int used = s_used;
     // pass 1: blocks needed, and every reason to refuse the whole step
-    int need = 0, bad = 0;
+    int need = 0, bad = 0, shared = 0;
     for (int s = tid; s < B; s += kPlanThreads) {
         const int n = context_lens[s];
-        if (n < 0 || n + 1 > max_len || n / BS >= MB) bad = 1;
-        else need += (n % BS == 0);
+        if (n < 0 || n + 1 > max_len || n / BS >= MB) {
+            bad = 1;
+        } else if (n % BS == 0) {
+            need += 1;
+        } else if (refcounts) {
+            const int b = block_tables[(size_t)s * MB + n / BS];
+            if (b >= 0 && b < num_blocks && refcounts[b] > 1) shared = 1;
+        }
     }
     int total;
     block_exclusive_scan(need, sm, &total);
-    if (bad) atomicOr(&s_bad, 1);
+    if (bad || shared) atomicOr(&s_bad, 1);
+    if (shared) atomicOr(&s_shared, 1);
     __syncthreads();
     if (!s_bad && (used < 0 || used > free_count || total > free_count - used)) bad = 1;
     if (!s_bad && !bad)
@@ -187,7 +203,7 @@ device_append_kernel(int32_t *block_tables, int32_t *context_lens, const int32_t
     if (bad) atomicOr(&s_bad, 1);
     __syncthreads();
     if (s_bad) {
-        if (tid == 0) atomicOr(status, kStatusNoBlocks);
+        if (tid == 0) atomicOr(status, kStatusNoBlocks | (s_shared ? kStatusSharedBlock : 0u));
         return;
     }
     // pass 2: ranks in sequence order, table / length / slot updates

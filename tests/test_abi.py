@@ -153,9 +153,9 @@ def test_step_and_shared_prefix_checks_without_a_device():
     assert L.pkv_decode_step_workspace_size(4, 8, 2, 64, 16, 1024, 64, ctypes.byref(many)) == 0
     assert one.value == 256 and many.value > one.value
     # device append: negative sizes, missing cursor
-    assert L.pkv_device_append(None, None, None, 0, None, None, 4, 8, 16, 64, 128,
+    assert L.pkv_device_append(None, None, None, 0, None, None, None, 4, 8, 16, 64, 128,
                                None) == B.PKV_ERR_INVALID_ARG
-    assert L.pkv_device_append(None, None, None, -1, None, None, 4, 8, 16, 64, 128,
+    assert L.pkv_device_append(None, None, None, -1, None, None, None, 4, 8, 16, 64, 128,
                                None) == B.PKV_ERR_INVALID_ARG
     # shared-prefix plan / planned decode: too many groups, zero sequences
     assert L.pkv_shared_prefix_plan(None, None, None, None, 5, 4, 8, 2, 64, 16, 8, 100, 0, None,

@@ -43,6 +43,7 @@ def compare_states(c, m, seqs):
     fm, hm, tm, um = m.stats()
     assert (fc, hc, tc) == (fm, hm, tm)
     assert uc == pytest.approx(um, abs=1e-12)
+    assert c.pkv_alloc_refcounts().tolist() == m.refcount
     if seqs:
         st, tables, lens = c.pkv_block_tables(seqs)
         assert st == 0

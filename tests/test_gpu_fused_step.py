@@ -20,6 +20,8 @@ pytestmark = pytest.mark.gpu
 
 NO_BLOCKS = pkv._binding.STATUS_NO_BLOCKS
 WORKSPACE = pkv._binding.STATUS_WORKSPACE
+SHARED = pkv._binding.STATUS_SHARED_BLOCK
+TIMEOUT = pkv._binding.STATUS_WAIT_TIMEOUT
 
 
 def model_state(rng, nb, bs, mb, nseq, max_len0):
@@ -423,3 +425,156 @@ def test_fused_step_replays_in_a_cuda_graph(cuda_device, nseq, Hq, P):
         assert torch.equal(eager["vc"][l].view(torch.int16), graphed["vc"][l].view(torch.int16))
         assert torch.equal(eager["out"][l].view(torch.int16), graphed["out"][l].view(torch.int16))
     del g
+
+
+def test_device_append_refuses_a_shared_partial_block(cuda_device):
+    """A shared page is copied before it is changed ("分页 KV Cache 分析" §3.2). After a fork,
+    parent and child share a partly filled last block; given the host manager's reference
+    counts, the device append refuses the step (nothing written: tables, lengths, cursor
+    and slots as they were) instead of writing into the page the sibling still reads.
+    Sequences forked at a block boundary write into new blocks: that step is accepted and
+    equals the host manager's own append."""
+    bs, mb, nb = 16, 8, 64
+    mgr = pkv.BlockManager(nb, bs, mb, np.arange(nb, dtype=np.int32)[::-1].copy())
+    assert mgr.pkv_seq_append(0, 20)[0] == 0          # 16 + 4: partly filled last block
+    assert mgr.pkv_seq_append(1, 32)[0] == 0          # two full blocks
+    assert mgr.pkv_seq_fork(0, 2) == 0
+    assert mgr.pkv_seq_fork(1, 3) == 0
+    refc = torch.from_numpy(mgr.pkv_alloc_refcounts()).cuda()
+    free = torch.from_numpy(mgr.pkv_alloc_free_list()).cuda()
+
+    def upload(ids):
+        st, tables, lens = mgr.pkv_block_tables(np.array(ids, np.int64))
+        assert st == 0
+        return torch.from_numpy(tables).cuda(), torch.from_numpy(lens).cuda()
+
+    bt, lens = upload([0, 1, 2, 3])
+    bt0, lens0 = bt.clone(), lens.clone()
+    used = torch.zeros(1, dtype=torch.int32, device="cuda")
+    slots = torch.full((4,), -7, dtype=torch.int64, device="cuda")
+    pkv.pkv_get_device_status(clear=True)
+    pkv.pkv_device_append(bt, lens, free, used, nb, mb * bs, bs, slots_out=slots,
+                          block_refcounts=refc)
+    st = pkv.pkv_get_device_status(clear=True)
+    assert st & NO_BLOCKS and st & SHARED, st
+    assert torch.equal(bt, bt0) and torch.equal(lens, lens0)
+    assert used.item() == 0 and bool((slots == -7).all())
+
+    # block-aligned forks: both sequences take a fresh block, as the host manager does
+    bt, lens = upload([1, 3])
+    pkv.pkv_device_append(bt, lens, free, used, nb, mb * bs, bs, slots_out=slots[:2],
+                          block_refcounts=refc)
+    assert pkv.pkv_get_device_status(clear=True) == 0
+    st, done, sl, cows = mgr.pkv_seq_append_batch(np.array([1, 3], np.int64), 1)
+    assert st == 0 and len(cows) == 0
+    _, tables, lens_h = mgr.pkv_block_tables(np.array([1, 3], np.int64))
+    assert np.array_equal(bt.cpu().numpy(), tables) and np.array_equal(lens.cpu().numpy(), lens_h)
+    assert slots[:2].cpu().numpy().tolist() == sl[:, 0].tolist()
+    assert used.item() == 2
+    mgr.close()
+
+
+K_SCHED_ARMED = int(np.array([0x9A6EDC0D], np.uint32).view(np.int32)[0])
+K_STEP_ARMED = int(np.array([0x57E9A11D], np.uint32).view(np.int32)[0])
+
+
+def header(ws):
+    """The step workspace header's words: armed, next, arrive, gen, exit."""
+    return ws[:20].view(torch.int32)
+
+
+def in_launch_merge_case(seed):
+    """Three sequences of several 64-token partitions, merged inside the step launch."""
+    rng = np.random.default_rng(seed)
+    dtype = synth.BF16
+    case = step_case(rng, [900, 40, 2000], 16, 4, 128, 16, dtype)
+    q, kc = case[0], case[1]
+    assert pkv.pkv_decode_step_launches(len(case[4]), 16, 4, 128, 16, case[5], 64) == 1
+    return dtype, case
+
+
+def run_step(dtype, case, ws, out):
+    q, kc, vc, bt, lens, max_len, slots, kn, vn = case
+    kcd, vcd = to_dev(kc, dtype), to_dev(vc, dtype)
+    pkv.pkv_paged_decode_step(out, to_dev(q, dtype), to_dev(kn, dtype), to_dev(vn, dtype), kcd,
+                              vcd, torch.from_numpy(bt).cuda(), torch.from_numpy(lens).cuda(),
+                              max_len, ws, partition_size=64)
+    return kcd, vcd
+
+
+def oracle_step(dtype, case):
+    q, kc, vc, bt, lens, max_len, slots, kn, vn = case
+    ek, ev = C.reshape_and_cache(kn, vn, kc, vc, slots)
+    return ek, ev, A.paged_decode_attention(q, ek, ev, bt, lens, 1 / np.sqrt(128), dtype)
+
+
+def test_header_with_a_stale_exit_count_is_refused(cuda_device):
+    """A header armed by the reduce kernel must come with cleared counters: one whose
+    exit count is not 0 (no CTA would ever see itself last, the work counter would never
+    be reset and later launches would skip items) is refused before any write."""
+    dtype, case = in_launch_merge_case(46)
+    q, kc = case[0], case[1]
+    ws = step_ws(q, kc, case[5], 64)
+    h = header(ws)
+    h[0] = K_SCHED_ARMED
+    h[4] = 5
+    before = ws[:256].clone()
+    out = torch.full((len(case[4]), 16, 128), 7.0, dtype=torch.bfloat16, device="cuda")
+    pkv.pkv_get_device_status(clear=True)
+    kcd, vcd = run_step(dtype, case, ws, out)
+    assert pkv.pkv_get_device_status(clear=True) & WORKSPACE
+    assert (out == 7.0).all()
+    assert np.array_equal(to_bits(kcd), kc)            # no cache write either
+    assert torch.equal(ws[:256], before)
+
+
+def test_workspace_of_a_plain_decode_serves_the_step(cuda_device):
+    """A workspace never zero-filled, used first by the plain decode (whose reduce kernel
+    re-arms it and clears the step counters), is a valid step workspace afterwards."""
+    dtype, case = in_launch_merge_case(47)
+    q, kc, vc, bt, lens, max_len, slots, kn, vn = case
+    ws = step_ws(q, kc, max_len, 64)
+    ws.fill_(0x5A)
+    qd = to_dev(q, dtype)
+    out = torch.empty_like(qd)
+    pkv.pkv_get_device_status(clear=True)
+    pkv.pkv_paged_attention_decode(out, qd, to_dev(kc, dtype), to_dev(vc, dtype),
+                                   torch.from_numpy(bt).cuda(), torch.from_numpy(lens).cuda(),
+                                   max_len, partition_size=64, workspace=ws)
+    torch.cuda.synchronize()
+    h = header(ws).cpu().numpy()
+    assert h[0] == K_SCHED_ARMED and h[1] == 0 and h[2] == 0 and h[4] == 0
+    kcd, vcd = run_step(dtype, case, ws, out)
+    torch.cuda.synchronize()
+    assert pkv.pkv_get_device_status(clear=True) == 0
+    ek, ev, ref = oracle_step(dtype, case)
+    assert np.array_equal(to_bits(kcd), ek) and np.array_equal(to_bits(vcd), ev)
+    assert_close(to_bits(out), ref, dtype, "step after a plain decode")
+    assert header(ws)[0].item() == K_STEP_ARMED
+
+
+def test_grid_barrier_gives_up_and_the_workspace_recovers(cuda_device):
+    """The bounded grid barrier of the in-launch merge runs out: an arrival count left in
+    the header (as if by an interrupted launch) means no CTA is ever the last to arrive,
+    so every CTA gives up after its poll limit. The launch returns with
+    PKV_STATUS_WAIT_TIMEOUT (and PKV_STATUS_WORKSPACE for the stale count) set, skips the
+    merge, and the last CTA out leaves the header re-armed with its counters cleared; the
+    next step on the same workspace is correct."""
+    dtype, case = in_launch_merge_case(48)
+    q, kc = case[0], case[1]
+    ws = step_ws(q, kc, case[5], 64)
+    header(ws)[2] = -(1 << 31)                         # arrive = 0x80000000
+    out = torch.empty((len(case[4]), 16, 128), dtype=torch.bfloat16, device="cuda")
+    pkv.pkv_get_device_status(clear=True)
+    run_step(dtype, case, ws, out)
+    st = pkv.pkv_get_device_status(clear=True)
+    assert st & TIMEOUT and st & WORKSPACE, st
+    h = header(ws).cpu().numpy()
+    assert h[0] == K_STEP_ARMED and h[1] == 0 and h[2] == 0 and h[4] == 0
+    out2 = torch.empty_like(out)
+    kcd, vcd = run_step(dtype, case, ws, out2)
+    torch.cuda.synchronize()
+    assert pkv.pkv_get_device_status(clear=True) == 0
+    ek, ev, ref = oracle_step(dtype, case)
+    assert np.array_equal(to_bits(kcd), ek) and np.array_equal(to_bits(vcd), ev)
+    assert_close(to_bits(out2), ref, dtype, "step after a barrier timeout")

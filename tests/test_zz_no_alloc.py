@@ -3,10 +3,11 @@
 HBM to the KV pool, latency-critical code where an allocation may synchronise the
 device). It keeps its partition scratch in a fixed array inside the library.
 
-Called through the C-ABI (ctypes, raw pointers) and compared with the workspace
-entry point on the same inputs, twice in a row, within the attention tolerance
-used by the other GPU tests (4e-3 + 1e-2*|ref|). Self-contained so that it passes
-alone in a fresh process as well as after every other test."""
+Called through the C-ABI (ctypes, raw pointers) and compared, twice in a row, with
+the workspace entry point on the same inputs and element by element with the fp64
+oracle (one softmax per sequence and query head over the gathered pages), within the
+attention tolerance used by the other GPU tests (4e-3 + 1e-2*|ref|). Self-contained
+so that it passes alone in a fresh process as well as after every other test."""
 import ctypes
 import math
 
@@ -14,6 +15,7 @@ import numpy as np
 import pytest
 import torch
 
+from oracle import attention as A
 from paged_kv_cache_320_b200 import _binding as B
 
 pytestmark = pytest.mark.gpu
@@ -71,6 +73,13 @@ def test_noalloc_decode_matches_workspace_decode_twice(cuda_device):
     assert rc == B.PKV_OK
     torch.cuda.synchronize()
     r = ref.float().cpu().numpy()
+
+    def bits(t):
+        return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+    oracle = A.paged_decode_attention(bits(x["q"]), bits(x["kc"]), bits(x["vc"]),
+                                      x["bt"].cpu().numpy(), x["lens"].cpu().numpy(), x["scale"],
+                                      A.BF16)
     for call in range(2):
         out = torch.full_like(x["q"], float("nan"))
         assert call_noalloc(L, x, out, partition) == B.PKV_OK
@@ -78,6 +87,9 @@ def test_noalloc_decode_matches_workspace_decode_twice(cuda_device):
         o = out.float().cpu().numpy()
         err = np.abs(o - r)
         assert np.all(err <= 4e-3 + 1e-2 * np.abs(r)), (call, float(err.max()))
+        got = A.bits_to_f64(bits(out), A.BF16)
+        err_o = np.abs(got - oracle)
+        assert np.all(err_o <= 4e-3 + 1e-2 * np.abs(oracle)), (call, float(err_o.max()))
     st = ctypes.c_uint32(1)
     assert L.pkv_get_device_status(ctypes.byref(st), 1, None) == B.PKV_OK
     assert st.value == 0
