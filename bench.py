@@ -258,24 +258,33 @@ def cow_arm(args, rank, world, local_rank):
             ev["copy"].append((e[0], e[1]))
             ev["decode"].append((e[1], e[2]))
 
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
     for _ in range(args.warmup):
         step()
-    torch.cuda.synchronize(dev)
+    barrier()
     with ClockSampler(local_rank) as clocks:
-        torch.cuda.synchronize(dev)
+        barrier()
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
         for _ in range(args.steps):
             step(record=True)
         t1.record(stream)
-        torch.cuda.synchronize(dev)
-    ms_step = t0.elapsed_time(t1) / args.steps
+        barrier()
+    ms_step = reduce_max(t0.elapsed_time(t1) / args.steps, dist, dev)
     if pkv.pkv_get_device_status(stream=stream) != 0:
         raise RuntimeError("device status word set during the benchmark")
     copy_us = 1e3 * statistics.mean(a.elapsed_time(b) for a, b in ev["copy"])
     dec_us = 1e3 * statistics.mean(a.elapsed_time(b) for a, b in ev["decode"])
-    value, tokens_per_s = weak_scaling_rates(kv_step, B, 1, ms_step)
+    value, tokens_per_s = weak_scaling_rates(kv_step, B, world, ms_step)
     copy_bytes = n_pairs * 2 * sp.num_kv_heads * sp.block_size * sp.head_dim * 2 * 2
 
     # end to end: the host block manager frees, re-forks and appends every step (batched
@@ -340,7 +349,7 @@ def cow_arm(args, rank, world, local_rank):
 
     for _ in range(args.warmup):
         e2e_step()
-    torch.cuda.synchronize(dev)
+    barrier()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
     a.record(stream)
@@ -350,28 +359,29 @@ def cow_arm(args, rank, world, local_rank):
     stream.wait_stream(copy_out)
     stream.wait_stream(copy_in)
     b.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = a.elapsed_time(b) / args.steps
+    barrier()
+    e2e_ms = reduce_max(a.elapsed_time(b) / args.steps, dist, dev)
     mgr.close()
     peak, peak_kind = read_peaks()
     h2d = ((q_h.numel() + kn_h.numel() + vn_h.numel()) * 2 + B * 8 + n_pairs * 8 +
            bt_h[0].numel() * 4 + B * 4)
     pmax = max(1, -(-max_len // P))
     return {
-        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": 1,
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": synth.DTYPE_NAMES[sp.dtype], "data": "synthetic",
         "config": {"workload": "shared_prefix_cow", "description": WORKLOADS["shared_prefix_cow"],
                    "num_seqs": B, "copy_pairs_per_step": n_pairs, "partition_size": P,
-                   "sum_context_tokens": int(lens.sum()), "kv_bytes_per_step": kv_step},
+                   "sum_context_tokens": int(lens.sum()), "kv_bytes_per_step": kv_step,
+                   "parallelism": f"replicas x{world}"},
         "tokens_per_s": round(tokens_per_s, 1),
-        "pct_of_hbm_peak": round(100 * value / peak, 2),
+        "pct_of_hbm_peak": round(100 * value / world / peak, 2),
         "copy_and_write_us": round(copy_us, 2),
         "copy_blocks_bytes": copy_bytes,
         "decode_us": round(dec_us, 2),
         "clocks": clocks.summary(),
-        "e2e": {"value": round(kv_step / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+        "e2e": {"value": round(kv_step * world / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(out_h[0].numel() * 2),
                 "includes": "host batched frees, forks and appends (copy-on-write pairs), table "
@@ -398,7 +408,38 @@ def weak_scaling_rates(kv_bytes_per_rank_step, seqs_per_rank, world, ms_step):
     return kv_bytes_per_rank_step * world / sec / 1e9, seqs_per_rank * world / sec
 
 
-def gpu_arm(args, rank, world, local_rank):
+def record_graph(fn, dev, stream):
+    """fn(launch_stream)'s launches recorded once as a CUDA graph (captured on a side
+    stream that first waits for `stream`)."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.graph(g, stream=side):
+        fn(side)
+    stream.wait_stream(side)
+    return g
+
+
+def time_replays(g, replays, stream):
+    """ms per replay of graph g: `replays` replays between two CUDA events on `stream`
+    (the caller synchronises on both sides)."""
+    import torch
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        a.record(stream)
+        for _ in range(replays):
+            g.replay()
+        b.record(stream)
+    b.synchronize()
+    return a.elapsed_time(b) / replays
+
+
+def gpu_arm(args, rank, world, local_rank, light=False):
+    """The device-timed decode step of one workload (every rank its own replica). With
+    light, only the step, its dominant kernel and its clocks are timed (no end-to-end leg,
+    read probe, memory-utilisation replay or optional legs)."""
     import torch
     import paged_kv_cache_320_b200 as pkv
 
@@ -422,7 +463,6 @@ def gpu_arm(args, rank, world, local_rank):
     sp = wl.spec
     L = sp.num_layers
     B = wl.num_seqs
-    dtype_code = pkv.PKV_F16 if sp.dtype == synth.F16 else pkv.PKV_BF16
     max_len = wl.max_blocks_per_seq * sp.block_size
     P = pkv.pkv_decode_partition_size(B, sp.num_heads, sp.num_kv_heads, sp.head_dim,
                                       sp.block_size, max_len, args.partition)
@@ -464,61 +504,69 @@ def gpu_arm(args, rank, world, local_rank):
     kn3 = [wl.k_new[l].view(B, sp.num_kv_heads, sp.head_dim) for l in range(L)]
     vn3 = [wl.v_new[l].view(B, sp.num_kv_heads, sp.head_dim) for l in range(L)]
 
-    # the stream the step's kernels go to (a capture stream while a CUDA graph is recorded)
-    launch_stream = [stream]
-
-    def fused_layer(l, out_t, q_t, kn_t, vn_t, bt_t, lens_t):
+    def fused_layer(l, out_t, q_t, kn_t, vn_t, bt_t, lens_t, st):
         pkv.pkv_paged_decode_step(out_t, q_t, kn_t, vn_t, wl.k_cache[l], wl.v_cache[l], bt_t,
                                   lens_t, max_len, ws, scale=wl.scale, partition_size=P,
-                                  stream=launch_stream[0])
+                                  stream=st)
 
-    def decode(l, out_t, q_t, bt_t, lens_t):
+    def decode(l, out_t, q_t, bt_t, lens_t, st):
         if shared:
             # one plan per step serves every layer (the layers share tables and lengths)
             if l == 0:
                 pkv.pkv_shared_prefix_plan(bt_t, lens_t, starts, prefix, sp.num_heads,
                                            sp.num_kv_heads, sp.head_dim, sp.block_size, max_len,
-                                           ws, partition_size=P, stream=launch_stream[0])
+                                           ws, partition_size=P, stream=st)
             pkv.pkv_paged_attention_decode_shared_prefix_planned(
                 out_t, q_t, wl.k_cache[l], wl.v_cache[l], bt_t, lens_t, max_len, ws,
-                scale=wl.scale, partition_size=P, stream=launch_stream[0])
+                scale=wl.scale, partition_size=P, stream=st)
         else:
             pkv.pkv_paged_attention_decode(out_t, q_t, wl.k_cache[l], wl.v_cache[l], bt_t,
                                            lens_t, max_len, scale=wl.scale, partition_size=P,
-                                           workspace=ws, stream=launch_stream[0])
+                                           workspace=ws, stream=st)
 
-    k1_events = []
-    k3_events = []
-
-    def step(record=False):
+    def step(st):
         for l in range(L):
-            if record:
-                e0 = torch.cuda.Event(enable_timing=True)
-                e1 = torch.cuda.Event(enable_timing=True)
-            if not fused:
-                if record:
-                    ec = torch.cuda.Event(enable_timing=True)
-                    ec.record(launch_stream[0])
-                pkv.pkv_reshape_and_cache(wl.k_new[l], wl.v_new[l], wl.k_cache[l],
-                                          wl.v_cache[l], slots, stream=launch_stream[0])
-                if record:
-                    k3_events.append((ec, e0))
-            if record:
-                e0.record(launch_stream[0])
             if fused:
                 # the workload's slot of each sequence is its newest position (len - 1)
-                fused_layer(l, outs[l], wl.q[l], kn3[l], vn3[l], bt, lens)
+                fused_layer(l, outs[l], wl.q[l], kn3[l], vn3[l], bt, lens, st)
             else:
-                decode(l, outs[l], wl.q[l], bt, lens)
-            if record:
-                e1.record(launch_stream[0])
-                k1_events.append((e0, e1))
+                pkv.pkv_reshape_and_cache(wl.k_new[l], wl.v_new[l], wl.k_cache[l],
+                                          wl.v_cache[l], slots, stream=st)
+                decode(l, outs[l], wl.q[l], bt, lens, st)
 
+    # The dominant kernel's launches alone (the split entry points): the write-and-decode
+    # kernel of the fused step, or the partition kernel; and the merge kernel alone. The
+    # step kernel that merges in its own launch is its own call.
     if fused:
-        launches_per_step = L * pkv.pkv_decode_step_launches(
+        launches_per_layer = pkv.pkv_decode_step_launches(
             B, sp.num_heads, sp.num_kv_heads, sp.head_dim, sp.block_size, max_len, P)
+        launches_per_step = L * launches_per_layer
+        kernel_key = ("paged_decode_partition_write" if launches_per_layer > 1
+                      else "paged_decode_step")
     else:
-        launches_per_step = (3 * L + 1) if shared else L * (2 + (1 if pmax > 1 else 0))
+        launches_per_layer = 3 if shared else 2 + (1 if pmax > 1 else 0)
+        launches_per_step = (3 * L + 1) if shared else L * launches_per_layer
+        kernel_key = "paged_decode_shared" if shared else "paged_decode_partition"
+    split = not shared and (not fused or launches_per_layer > 1)
+
+    def kernel_only(st):
+        for l in range(L):
+            if fused:
+                pkv.pkv_paged_decode_step_partitions(outs[l], wl.q[l], kn3[l], vn3[l],
+                                                     wl.k_cache[l], wl.v_cache[l], bt, lens,
+                                                     max_len, ws, scale=wl.scale,
+                                                     partition_size=P, stream=st)
+            else:
+                pkv.pkv_paged_attention_decode_partitions(outs[l], wl.q[l], wl.k_cache[l],
+                                                          wl.v_cache[l], bt, lens, max_len, ws,
+                                                          scale=wl.scale, partition_size=P,
+                                                          stream=st)
+
+    def merge_only(st):
+        for l in range(L):
+            pkv.pkv_paged_attention_merge(outs[l], lens, sp.num_kv_heads, sp.block_size,
+                                          max_len, ws, partition_size=P, stream=st)
+
     dist = None
     if world > 1:
         import torch.distributed as dist
@@ -530,83 +578,101 @@ def gpu_arm(args, rank, world, local_rank):
 
     # ---- device-timed region: inputs resident in HBM
     for _ in range(args.warmup):
-        step()
+        step(stream)
     barrier()
-    g = None
+    graphs = {}
     if not args.no_graph:
         # the step recorded once as a CUDA graph (every layer's launches) and replayed: the
-        # headline timing, as a serving loop runs a decode step
-        g = torch.cuda.CUDAGraph()
-        side = torch.cuda.Stream(dev)
-        side.wait_stream(stream)
-        launch_stream[0] = side
-        with torch.cuda.graph(g, stream=side):
-            step()
-        launch_stream[0] = stream
-        stream.wait_stream(side)
-        for _ in range(args.warmup):
-            g.replay()
+        # headline timing, as a serving loop runs a decode step; the dominant kernel's and
+        # the merge kernel's launches alone in graphs of their own
+        graphs["step"] = record_graph(step, dev, stream)
+        if split:
+            graphs["kernel"] = record_graph(kernel_only, dev, stream)
+            if pmax > 1:
+                graphs["merge"] = record_graph(merge_only, dev, stream)
+        for g in graphs.values():
+            for _ in range(args.warmup):
+                g.replay()
         barrier()
+    ms = {}
     with ClockSampler(local_rank) as clocks:
         barrier()
-        # eager launches with CUDA events around every decode call (per-launch times)
+        # eager launches (the same steps, one kernel at a time)
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
         for _ in range(args.steps):
-            step(record=True)
+            step(stream)
         t1.record(stream)
         barrier()
-        if g is not None:
-            g0 = torch.cuda.Event(enable_timing=True)
-            g1 = torch.cuda.Event(enable_timing=True)
-            g0.record(stream)
-            for _ in range(args.steps):
-                g.replay()
-            g1.record(stream)
+        ms["eager"] = t0.elapsed_time(t1) / args.steps
+        for name, g in graphs.items():
+            ms[name] = time_replays(g, args.steps, stream)
             barrier()
-    ms_eager = t0.elapsed_time(t1)
-    ms_total = g0.elapsed_time(g1) if g is not None else ms_eager
-    if g is not None:
-        del g
-    k1_ms = [a.elapsed_time(b) for a, b in k1_events]
+    graphs.clear()
     if pkv.pkv_get_device_status(stream=stream) != 0:
         raise RuntimeError("device status word set during the benchmark")
 
     def max_over_ranks(x):
         return reduce_max(x, dist, dev)
 
-    ms_total = max_over_ranks(ms_total)
-    ms_step = ms_total / args.steps
+    ms = {k: max_over_ranks(v) for k, v in ms.items()}
+    ms_step = ms.get("step", ms["eager"])
     value, tokens_per_s = weak_scaling_rates(kv_step, B, world, ms_step)
-    ms_eager_step = max_over_ranks(ms_eager) / args.steps
-    eager_value, _ = weak_scaling_rates(kv_step, B, world, ms_eager_step)
-    k1_avg_ms = statistics.mean(k1_ms)
-    cache_write = None
-    if k3_events:
-        k3_us = 1e3 * statistics.mean(a.elapsed_time(b) for a, b in k3_events)
-        k3_bytes = len(wl.slot_mapping) * sp.num_kv_heads * sp.head_dim * 2 * 2 * 2
-        cache_write = {"us_per_launch": round(k3_us, 2), "bytes_per_launch": k3_bytes,
-                       "gbs": round(k3_bytes / (k3_us * 1e-6) / 1e9, 1),
-                       "note": "launch-latency bound: reads and writes each new token's K/V rows"}
-    k1_q = np.percentile(np.array(k1_ms), [10, 50, 90]) * 1e3     # this rank's spread, us
-    k1_avg_ms = max_over_ranks(k1_avg_ms)
+    eager_value, _ = weak_scaling_rates(kv_step, B, world, ms["eager"])
     peak, peak_kind = read_peaks()
-    achieved = roof_layer / (k1_avg_ms * 1e-3) / 1e9
-    read_probe = hbm_read_probe(dev, stream)
+    call_us = 1e3 * ms_step / L
+    kernel_us = 1e3 * ms["kernel"] / L if "kernel" in ms else call_us
+    merge_us = 1e3 * ms["merge"] / L if "merge" in ms else None
+    achieved = roof_layer / (kernel_us * 1e-6) / 1e9
+    call_achieved = roof_layer / (call_us * 1e-6) / 1e9
+    traffic = None if shared else read_traffic(args.workload, sp.block_size, kernel_key)
+    if fused:
+        call_desc = ("write-and-decode kernel + merge kernel" if launches_per_layer > 1 else
+                     "step kernel (cache write, decode and merge in one launch)")
+    else:
+        call_desc = ("plan (one per step) + shared-prefix decode + merge" if shared else
+                     "cache write + partition kernel" + (" + merge kernel" if pmax > 1 else ""))
+    roofline = {
+        "kernel": f"{kernel_key}_kernel",
+        "bound": "hbm",
+        "achieved": round(achieved, 1),
+        "peak": peak,
+        "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+        else "fallback",
+        "unit": "GB/s",
+        "frac": round(achieved / peak, 4),
+        "traffic": traffic,
+        "algorithmic_bytes_per_launch": roof_layer,
+        "avg_launch_us": round(kernel_us, 2),
+        "timed": ("CUDA graph of the kernel's launches alone (all layers), replayed `steps` "
+                  "times between CUDA events" if "kernel" in ms else
+                  "the step's CUDA graph replays (one launch per layer)"),
+        "call_level": {"includes": call_desc, "us_per_layer": round(call_us, 2),
+                       "achieved": round(call_achieved, 1),
+                       "frac": round(call_achieved / peak, 4)},
+    }
+    if merge_us is not None:
+        roofline["merge_kernel_us"] = round(merge_us, 2)
+    if light:
+        return {
+            "workload": args.workload, "block_size": sp.block_size, "layers": L,
+            "num_seqs": B, "num_heads": sp.num_heads, "num_kv_heads": sp.num_kv_heads,
+            "dtype": synth.DTYPE_NAMES[sp.dtype], "partition_size": P,
+            "sum_context_tokens": int(wl.context_lens.sum()), "kv_bytes_per_step": kv_step,
+            "value": round(value, 1), "unit": "GB/s", "ms_per_step": round(ms_step, 4),
+            "pct_of_hbm_peak": round(100 * value / world / peak, 2),
+            "tokens_per_s": round(tokens_per_s, 1),
+            "launches_per_layer": launches_per_layer,
+            "eager": {"value": round(eager_value, 1), "ms_per_step": round(ms["eager"], 4)},
+            "roofline": roofline, "clocks": clocks.summary()}
+
+    roofline["hbm_read_probe_gbs"] = round(hbm_read_probe(dev, stream), 1)
     swap = swap_measurement(wl, dev, stream) if args.swap else None
     mem_mgr = replay_block_manager(wl)
     memory = memory_utilisation(wl, mem_mgr, sp0.max_len)   # the workload's own length cap
     mem_mgr.close()
     prefix_cache = prefix_cache_measurement(sp) if args.prefix_cache else None
-    # the dominant kernel: the partition kernel, or for the fused step the write-and-decode
-    # kernel (merge by the reduce kernel) or the step kernel (merge in the same launch)
-    if fused:
-        kernel_key = ("paged_decode_partition_write" if launches_per_step > L
-                      else "paged_decode_step")
-    else:
-        kernel_key = "paged_decode_partition"
-    traffic = None if shared else read_traffic(args.workload, sp.block_size, kernel_key)
 
     # ---- end to end: host block manager + pinned host buffers through the public API
     e2e = e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, world, decode,
@@ -643,33 +709,15 @@ def gpu_arm(args, rank, world, local_rank):
         "pct_of_hbm_peak": round(100 * value / world / peak, 2),
         "pct_of_nominal_8tbs": round(100 * value / world / 8000.0, 2),
         "memory_utilisation": memory,
-        **({"cache_write": cache_write} if cache_write else {}),
         "eager": {"value": round(eager_value, 1), "unit": "GB/s",
-                  "ms_per_step": round(ms_eager_step, 4),
+                  "ms_per_step": round(ms["eager"], 4),
                   "note": "the same steps launched one kernel at a time (no graph)"},
         **({"swap_blocks": swap} if swap else {}),
         **({"prefix_cache": prefix_cache} if prefix_cache else {}),
         "clocks": clocks.summary(),
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
-        "roofline": {
-            "kernel": "paged_decode_shared_kernel (+ plan, reduce)" if shared
-            else f"{kernel_key}_kernel (cache write + decode"
-                 + (" + reduce)" if launches_per_step > L else " + merge)") if fused
-            else "paged_decode_partition_kernel (+ reduce)",
-            "bound": "hbm",
-            "achieved": round(achieved, 1),
-            "peak": peak,
-            "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
-            else "fallback",
-            "unit": "GB/s",
-            "frac": round(achieved / peak, 4),
-            "traffic": traffic,
-            "algorithmic_bytes_per_launch": roof_layer,
-            "hbm_read_probe_gbs": round(read_probe, 1),
-            "avg_launch_us": round(k1_avg_ms * 1e3, 2),
-            "launch_us_p10_p50_p90": [round(float(x), 2) for x in k1_q],
-        },
+        "roofline": roofline,
     }
     return result
 
@@ -966,11 +1014,12 @@ def e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, worl
             if fused:
                 fused_layer(l, out_d[b][l], q_d[b][l],
                             kn_d[b][l].view(B, sp.num_kv_heads, sp.head_dim),
-                            vn_d[b][l].view(B, sp.num_kv_heads, sp.head_dim), bt_dev, lens_dev)
+                            vn_d[b][l].view(B, sp.num_kv_heads, sp.head_dim), bt_dev, lens_dev,
+                            stream)
             else:
                 pkv.pkv_reshape_and_cache(kn_d[b][l], vn_d[b][l], wl.k_cache[l], wl.v_cache[l],
                                           slots_d[b], stream=stream)
-                decode(l, out_d[b][l], q_d[b][l], bt_d[b], lens_d[b])
+                decode(l, out_d[b][l], q_d[b][l], bt_d[b], lens_d[b], stream)
             ev_out[b][l].record(stream)
             copy_out.wait_event(ev_out[b][l])
             with torch.cuda.stream(copy_out):
@@ -1134,9 +1183,31 @@ def reference_arm(args, rank):
     }
 
 
-def main():
+CONFIG_WORKLOADS = [("llama3_8b_gqa", 16), ("long_context", 8), ("long_context", 16),
+                    ("long_context", 32)]
+
+
+def run_configs(args, local_rank):
+    """The other decode workloads at their own sizes (Llama-3-8B-shaped GQA; long context at
+    block sizes 8, 16 and 32), each timed like the headline workload: the fused step as CUDA
+    graph replays, `steps` timed after `warmup`, its dominant kernel alone, clocks sampled
+    during its timed region."""
+    import torch
+    out = {}
+    for workload, bs in CONFIG_WORKLOADS:
+        sub = argparse.Namespace(**vars(args))
+        sub.workload, sub.block_size, sub.layers, sub.batch = workload, bs, 0, 0
+        sub.decode, sub.swap, sub.prefix_cache, sub.partition = "plain", False, False, 0
+        out[f"{workload}_bs{bs}"] = gpu_arm(sub, 0, 1, local_rank, light=True)
+        torch.cuda.empty_cache()
+    return out
+
+
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--gpus", type=int, default=1,
+                    help="GPUs of this node, one process each (started here under "
+                         "torch.distributed.run unless already launched by it)")
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="llama7b_mha", choices=sorted(WORKLOADS))
@@ -1162,38 +1233,90 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    args = ap.parse_args()
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-workload `configs` lines of the default run")
+    args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")
+    if args.gpus < 1:
+        raise SystemExit("--gpus must be at least 1")
+    return args
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+def free_port():
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def launch_command(argv, nproc, port, script=None):
+    """torch.distributed.run over `nproc` local processes (one per GPU), rendezvous on
+    127.0.0.1, each running `script` (this file) with the same arguments."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={nproc}", "--master-addr", "127.0.0.1", "--master-port", str(port),
+            script or os.path.abspath(__file__), *argv]
+
+
+def rank_env():
+    """(rank, world size, local rank) from the launcher's environment (1 process if unset)."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def run_ranks(args, arm, backend="nccl"):
+    """This process's part of the run: with several ranks, a process group over the
+    launcher's rendezvous (short timeout), then arm(args, rank, world, local_rank) (every
+    rank its own replica; the arm takes the max over ranks of its times), then a closing
+    barrier. Returns the arm's result on rank 0, None elsewhere."""
+    rank, world, local_rank = rank_env()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but {world} process(es) were launched")
+    dist = None
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local_rank)
+            kw["device_id"] = torch.device("cuda", local_rank)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
+    res = arm(args, rank, world, local_rank)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return res if rank == 0 else None
+
+
+def main(argv=None):
+    argv = sys.argv[1:] if argv is None else list(argv)
+    args = parse_args(argv)
+    rank, world, local_rank = rank_env()
 
     if args.impl == "reference":
         res = reference_arm(args, rank)
         if res is not None:
             print(json.dumps(res), flush=True)
-        return
+        return 0
 
-    import torch
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local_rank)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local_rank))
-    res = (cow_arm if args.workload == "shared_prefix_cow" else gpu_arm)(args, rank, world,
-                                                                          local_rank)
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-        dist.destroy_process_group()
-    if rank == 0:
-        if world == 1 and not args.no_cpu_baseline and args.workload != "shared_prefix_cow":
-            res["cpu_baseline"] = cpu_baseline(args)
-        print(json.dumps(res), flush=True)
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        # one process per GPU: start them under torch.distributed.run with these arguments
+        return subprocess.call(launch_command(argv, args.gpus, free_port()))
+
+    arm = cow_arm if args.workload == "shared_prefix_cow" else gpu_arm
+    res = run_ranks(args, arm)
+    if res is None:
+        return 0
+    if (world == 1 and not args.no_configs and args.workload == "llama7b_mha"
+            and args.decode == "plain" and not args.block_size and not args.layers
+            and not args.batch and not args.partition):
+        res["configs"] = run_configs(args, local_rank)
+    if world == 1 and not args.no_cpu_baseline and args.workload != "shared_prefix_cow":
+        res["cpu_baseline"] = cpu_baseline(args)
+    print(json.dumps(res), flush=True)
+    return 0
 
 
 if __name__ == "__main__":
-    main()
+    sys.exit(main())

@@ -111,6 +111,34 @@ int pkv_paged_attention_decode(void *out, const void *q, const void *k_cache,
                                float scale, int dtype, int partition_size, void *workspace,
                                size_t workspace_bytes, pkv_stream_t stream);
 
+/* The two launches of pkv_paged_attention_decode as separate calls (the decode of each
+ * partition, "分页 KV Cache 分析" §3.1's per-page loop in streaming form, and the exact
+ * log-sum-exp merge of the partitions), for callers that put other work between them or
+ * time each:
+ *  - pkv_paged_attention_decode_partitions: arguments, checks and errors as
+ *    pkv_paged_attention_decode; launches the decode kernel only. Sequences whose context
+ *    is one partition get their output; the others leave fp32 partials in `workspace`.
+ *  - pkv_paged_attention_merge: merges those partials into `out` (outputs of one-partition
+ *    sequences are not touched). The sizes, partition_size, context_lens and workspace
+ *    must be those of the partitions call it follows on the same stream; it launches
+ *    nothing when every context is one partition. Errors: PKV_ERR_INVALID_ARG,
+ *    PKV_ERR_WORKSPACE, PKV_ERR_CUDA.
+ * The partitions call followed by the merge gives the bits of pkv_paged_attention_decode.
+ * The partitions call may be repeated on the same workspace without a merge between. */
+int pkv_paged_attention_decode_partitions(void *out, const void *q, const void *k_cache,
+                                          const void *v_cache, const int32_t *block_tables,
+                                          const int32_t *context_lens, int num_seqs,
+                                          int num_heads, int num_kv_heads, int head_dim,
+                                          int block_size, int max_blocks_per_seq, int num_blocks,
+                                          int max_context_len, float scale, int dtype,
+                                          int partition_size, void *workspace,
+                                          size_t workspace_bytes, pkv_stream_t stream);
+
+int pkv_paged_attention_merge(void *out, const int32_t *context_lens, int num_seqs, int num_heads,
+                              int num_kv_heads, int head_dim, int block_size, int max_context_len,
+                              int partition_size, int dtype, void *workspace,
+                              size_t workspace_bytes, pkv_stream_t stream);
+
 /* ------------------------------------------------------------------------------
  * pkv_paged_attention_decode for callers that cannot allocate device memory.
  * The paper has no counterpart: this is a library convenience.
@@ -339,6 +367,20 @@ int pkv_paged_decode_step(void *out, const void *q, const void *k_new, const voi
                           int num_blocks, int max_context_len, float scale, int dtype,
                           int partition_size, void *workspace, size_t workspace_bytes,
                           pkv_stream_t stream);
+
+/* The write-and-decode launch of pkv_paged_decode_step alone (never the in-launch merge):
+ * every newest token written, one-partition sequences' outputs, the others' partials left
+ * in `workspace` for pkv_paged_attention_merge (same sizes and workspace). Arguments,
+ * workspace rules and errors as pkv_paged_decode_step; followed by the merge it gives the
+ * bits of pkv_paged_decode_step. */
+int pkv_paged_decode_step_partitions(void *out, const void *q, const void *k_new,
+                                     const void *v_new, void *k_cache, void *v_cache,
+                                     const int32_t *block_tables, const int32_t *context_lens,
+                                     int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                     int block_size, int max_blocks_per_seq, int num_blocks,
+                                     int max_context_len, float scale, int dtype,
+                                     int partition_size, void *workspace, size_t workspace_bytes,
+                                     pkv_stream_t stream);
 
 int pkv_decode_step_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
                                    int block_size, int max_context_len, int partition_size,

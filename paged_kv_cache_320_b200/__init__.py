@@ -16,10 +16,13 @@ from ._binding import (  # noqa: F401
     pkv_decode_step_workspace_size,
     pkv_device_append,
     pkv_paged_decode_step,
+    pkv_paged_decode_step_partitions,
     pkv_decode_workspace_size,
     pkv_get_device_status,
     pkv_paged_attention_decode,
     pkv_paged_attention_decode_noalloc,
+    pkv_paged_attention_decode_partitions,
+    pkv_paged_attention_merge,
     pkv_paged_attention_decode_shared_prefix,
     pkv_paged_attention_decode_shared_prefix_planned,
     pkv_shared_prefix_plan,

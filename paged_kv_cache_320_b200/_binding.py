@@ -66,6 +66,8 @@ def lib() -> ctypes.CDLL:
                                                  ctypes.c_float, I, I, P, SZ, P]
         L.pkv_paged_attention_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I,
                                                          I, I, ctypes.c_float, I, I, P]
+        L.pkv_paged_attention_decode_partitions.argtypes = L.pkv_paged_attention_decode.argtypes
+        L.pkv_paged_attention_merge.argtypes = [P, P, I, I, I, I, I, I, I, I, P, SZ, P]
         L.pkv_decode_workspace_size.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(SZ)]
         L.pkv_paged_attention_decode_shared_prefix.argtypes = [
             P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, ctypes.c_float, I, I, P, SZ, P]
@@ -90,6 +92,7 @@ def lib() -> ctypes.CDLL:
                                 ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_double)]
         L.pkv_paged_decode_step.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I,
                                             ctypes.c_float, I, I, P, SZ, P]
+        L.pkv_paged_decode_step_partitions.argtypes = L.pkv_paged_decode_step.argtypes
         L.pkv_decode_step_workspace_size.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(SZ)]
         L.pkv_device_append.argtypes = [P, P, P, I, P, P, P, I, I, I, I, I, P]
         L.pkv_alloc_refcounts.argtypes = [P, P, I]
@@ -107,6 +110,8 @@ def lib() -> ctypes.CDLL:
                                              ctypes.POINTER(ctypes.c_int64),
                                              ctypes.POINTER(ctypes.c_int64)]
         for name in ("pkv_paged_attention_decode", "pkv_paged_attention_decode_noalloc",
+                     "pkv_paged_attention_decode_partitions", "pkv_paged_attention_merge",
+                     "pkv_paged_decode_step_partitions",
                      "pkv_paged_attention_decode_shared_prefix",
                      "pkv_decode_shared_prefix_workspace_size", "pkv_decode_workspace_size",
                      "pkv_decode_partition_size", "pkv_decode_shared_prefix_partition_size",
@@ -258,6 +263,37 @@ def pkv_paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_l
     """out/q [B, Hq, D]; k_cache/v_cache [NB, Hkv, BS, D]; block_tables int32 [B, MB];
     context_lens int32 [B]; workspace: uint8 tensor of pkv_decode_workspace_size bytes
     (allocated here when None and needed)."""
+    return _decode("pkv_paged_attention_decode", out, q, k_cache, v_cache, block_tables,
+                   context_lens, max_context_len, scale, partition_size, workspace, stream)
+
+
+def pkv_paged_attention_decode_partitions(out, q, k_cache, v_cache, block_tables, context_lens,
+                                          max_context_len, workspace, scale=None,
+                                          partition_size=0, stream=None):
+    """The decode kernel of pkv_paged_attention_decode alone: one-partition sequences'
+    outputs, the others' partials left in workspace for pkv_paged_attention_merge."""
+    return _decode("pkv_paged_attention_decode_partitions", out, q, k_cache, v_cache,
+                   block_tables, context_lens, max_context_len, scale, partition_size, workspace,
+                   stream)
+
+
+def pkv_paged_attention_merge(out, context_lens, num_kv_heads, block_size, max_context_len,
+                              workspace, partition_size=0, stream=None):
+    """Merge of the partials a partitions call left in workspace into out [B, Hq, D]."""
+    import torch
+    _need(out, "out")
+    _need(context_lens, "context_lens", out.device, torch.int32, out.shape[0])
+    _need(workspace, "workspace", out.device)
+    B, Hq, D = out.shape
+    _check(lib().pkv_paged_attention_merge(
+        _ptr(out), _ptr(context_lens), B, Hq, int(num_kv_heads), D, int(block_size),
+        int(max_context_len), int(partition_size), _dtype_code(out), _ptr(workspace),
+        _nbytes(workspace), _stream(stream)), "pkv_paged_attention_merge")
+    return out
+
+
+def _decode(name, out, q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale,
+            partition_size, workspace, stream):
     B, Hq, D, NB, Hkv, BS = _decode_shapes(out, q, k_cache, v_cache, block_tables,
                                            context_lens)
     if scale is None:
@@ -271,11 +307,10 @@ def pkv_paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_l
         _need(workspace, "workspace", q.device)
     ws_ptr = _ptr(workspace) if workspace is not None else None
     ws_bytes = _nbytes(workspace) if workspace is not None else 0
-    _check(lib().pkv_paged_attention_decode(
+    _check(getattr(lib(), name)(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
         B, Hq, Hkv, D, BS, block_tables.shape[1], NB, int(max_context_len), float(scale),
-        _dtype_code(q), int(partition_size), ws_ptr, ws_bytes, _stream(stream)),
-        "pkv_paged_attention_decode")
+        _dtype_code(q), int(partition_size), ws_ptr, ws_bytes, _stream(stream)), name)
     return out
 
 
@@ -356,6 +391,22 @@ def pkv_paged_decode_step(out, q, k_new, v_new, k_cache, v_cache, block_tables, 
     """Cache write of each sequence's newest token + decode attention in one launch.
     k_new/v_new [B, Hkv, D]; workspace: uint8 device tensor of
     pkv_decode_step_workspace_size bytes, zero-filled before its first use (torch.zeros)."""
+    return _step("pkv_paged_decode_step", out, q, k_new, v_new, k_cache, v_cache, block_tables,
+                 context_lens, max_context_len, workspace, scale, partition_size, stream)
+
+
+def pkv_paged_decode_step_partitions(out, q, k_new, v_new, k_cache, v_cache, block_tables,
+                                     context_lens, max_context_len, workspace, scale=None,
+                                     partition_size=0, stream=None):
+    """The write-and-decode launch of pkv_paged_decode_step alone (merge with
+    pkv_paged_attention_merge on the same workspace)."""
+    return _step("pkv_paged_decode_step_partitions", out, q, k_new, v_new, k_cache, v_cache,
+                 block_tables, context_lens, max_context_len, workspace, scale, partition_size,
+                 stream)
+
+
+def _step(name, out, q, k_new, v_new, k_cache, v_cache, block_tables, context_lens,
+          max_context_len, workspace, scale, partition_size, stream):
     B, Hq, D, NB, Hkv, BS = _decode_shapes(out, q, k_cache, v_cache, block_tables,
                                            context_lens, k_new, v_new)
     if tuple(k_new.shape) != (B, Hkv, D) or v_new.shape != k_new.shape:
@@ -363,11 +414,11 @@ def pkv_paged_decode_step(out, q, k_new, v_new, k_cache, v_cache, block_tables, 
     _need(workspace, "workspace", q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
-    _check(lib().pkv_paged_decode_step(
+    _check(getattr(lib(), name)(
         _ptr(out), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
         _ptr(block_tables), _ptr(context_lens), B, Hq, Hkv, D, BS, block_tables.shape[1], NB,
         int(max_context_len), float(scale), _dtype_code(q), int(partition_size), _ptr(workspace),
-        _nbytes(workspace), _stream(stream)), "pkv_paged_decode_step")
+        _nbytes(workspace), _stream(stream)), name)
     return out
 
 

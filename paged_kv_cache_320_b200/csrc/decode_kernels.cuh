@@ -63,12 +63,13 @@ struct StageInfo {
 };
 constexpr int kFirst = 1, kLast = 2, kEnd = 4;
 
-// Dynamic work distribution: producers take item indices from `next`. The reduce
-// kernel, which follows every decode that has a workspace, re-arms it (next = 0, the
-// step kernel's barrier counters 0, armed = kSchedArmed) for the next call; a header
-// that is not armed (a workspace never used before) makes that call fall back to the
-// static schedule. The same header serves paged_decode_step_kernel, whose grid
-// barrier and exit count live in `arrive`, `gen` and `exit` (unused by the others).
+// Dynamic work distribution: producers take item indices from `next`. A launch that
+// found the header armed leaves it armed: its last CTA out (counted in `exit`) resets
+// the counters. The reduce kernel, which follows every decode that has a workspace,
+// re-arms it too (next = 0, arrive = exit = 0, armed = kSchedArmed); a header that is
+// not armed (a workspace never used before) makes that call fall back to the static
+// schedule. The same header serves paged_decode_step_kernel, whose grid barrier lives
+// in `arrive` and `gen`.
 constexpr unsigned kSchedArmed = 0x9A6EDC0Du;
 struct SchedHeader {
     unsigned armed;
@@ -584,8 +585,8 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 
 // The work-item loop shared by the decode kernels: warp 4 produces, warps 0-3
 // consume, until the item list is exhausted (barriers already initialised).
-// sched_mode 0: take items from prm.sched only if its header is armed (kSchedArmed);
-// sched_mode 1: the caller validated prm.sched (dynamic whenever it is non-null).
+// dynamic: take items from prm.sched->next (the caller checked the header), else the
+// static schedule.
 // kStep: before loading the page that holds a sequence's last token (position
 // len_s - 1), the producer writes that token's K and V rows (prm.k_new / prm.v_new,
 // [B][Hkv][D]) for its KV head into the cache, so the cache write of the decode step
@@ -593,7 +594,7 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 template <typename T, int D, int BS, bool kStep>
 __device__ __forceinline__ void decode_items(const CUtensorMap *tmap_k, const CUtensorMap *tmap_v,
                                              const CUtensorMap *tmap_q, const DecodeParams &prm,
-                                             DecodeSmem<D> &sm, int sched_mode) {
+                                             DecodeSmem<D> &sm, bool dynamic) {
     using L = DecodeLayout<D>;
     constexpr int kBPS = kStageTokens / BS;   // blocks per stage
     constexpr int H = L::kHalves;
@@ -647,13 +648,6 @@ __device__ __forceinline__ void decode_items(const CUtensorMap *tmap_k, const CU
         }                                                                               \
     }
 
-        // dynamic schedule when the workspace header is armed (read before any CTA
-        // can change it: no CTA takes from `next` unless it saw the header armed)
-        const bool dynamic =
-            prm.sched != nullptr &&
-            (sched_mode == 1 ||
-             __shfl_sync(0xffffffffu, lane == 0 ? *(volatile unsigned *)&prm.sched->armed : 0u,
-                         0) == kSchedArmed);
         // Every CTA's first item is its index (the grid never exceeds the item count);
         // later tickets come from the counter, offset by the grid. A ticket is requested
         // one item before it is resolved, so the atomic's latency overlaps a whole item;
@@ -857,16 +851,46 @@ __device__ __forceinline__ void decode_items(const CUtensorMap *tmap_k, const CU
     }
 }
 
+// Whether this launch takes its items from the workspace counter: the header is armed.
+// Read by every CTA before it changes anything; `armed` is written again only by the
+// last CTA out (sched_exit), so every CTA of a launch decides alike.
+__device__ __forceinline__ bool sched_is_armed(const DecodeParams &prm, int *flag) {
+    if (threadIdx.x == 0)
+        *flag = prm.sched != nullptr && *(volatile unsigned *)&prm.sched->armed == kSchedArmed;
+    __syncthreads();
+    return *flag != 0;
+}
+
+// End of a dynamically scheduled launch: the last CTA out re-arms the header (counter
+// and step counters 0), so the next launch on the workspace may run without a merge
+// kernel in between. Every CTA of the launch calls it (all threads).
+__device__ __forceinline__ void sched_exit(SchedHeader *h) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const unsigned t = atomicAdd(&h->exit, 1u);
+        if (t == gridDim.x - 1) {
+            h->next = 0;
+            h->arrive = 0;
+            h->exit = 0;
+            __threadfence();
+            h->armed = kSchedArmed;
+        }
+    }
+}
+
 template <typename T, int D, int BS>
 __global__ void __launch_bounds__(kDecodeThreads, 2)
 paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
                               const __grid_constant__ CUtensorMap tmap_v,
                               const __grid_constant__ CUtensorMap tmap_q, DecodeParams prm) {
+    __shared__ int s_dyn;
     DecodeSmem<D> sm(aligned_dynamic_smem(), prm.group);
     sm.init_barriers();
     pdl_wait_and_release();
-    __syncthreads();
-    decode_items<T, D, BS, false>(&tmap_k, &tmap_v, &tmap_q, prm, sm, 0);
+    const bool dyn = sched_is_armed(prm, &s_dyn);
+    decode_items<T, D, BS, false>(&tmap_k, &tmap_v, &tmap_q, prm, sm, dyn);
+    if (*(volatile int *)&s_dyn) sched_exit(prm.sched);   // reread: nothing held across the loop
 }
 
 // The same with the decode step's cache write (each sequence's newest token written by
@@ -877,11 +901,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
 paged_decode_partition_write_kernel(const __grid_constant__ CUtensorMap tmap_k,
                                     const __grid_constant__ CUtensorMap tmap_v,
                                     const __grid_constant__ CUtensorMap tmap_q, DecodeParams prm) {
+    __shared__ int s_dyn;
     DecodeSmem<D> sm(aligned_dynamic_smem(), prm.group);
     sm.init_barriers();
     pdl_wait_and_release();
-    __syncthreads();
-    decode_items<T, D, BS, true>(&tmap_k, &tmap_v, &tmap_q, prm, sm, 0);
+    const bool dyn = sched_is_armed(prm, &s_dyn);
+    decode_items<T, D, BS, true>(&tmap_k, &tmap_v, &tmap_q, prm, sm, dyn);
+    if (*(volatile int *)&s_dyn) sched_exit(prm.sched);   // reread: nothing held across the loop
 }
 
 // Log-sum-exp merge of n partials (m_j in log2 units, l_j, normalised o_j) of one

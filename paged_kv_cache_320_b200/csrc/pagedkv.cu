@@ -491,7 +491,7 @@ int step_merges_in_kernel(int B, int Hq, long long items, int pmax, int nsm) {
 template <typename T, int D>
 int dispatch_step(int BS, const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mq,
                   const pkv::DecodeParams &prm, long long items, int merge, int in_kernel,
-                  cudaStream_t st) {
+                  bool launch_merge, cudaStream_t st) {
     if (in_kernel) {
         switch (BS) {
             case 8: return launch_step<T, D, 8>(mk, mv, mq, prm, items, merge, st);
@@ -500,7 +500,8 @@ int dispatch_step(int BS, const CUtensorMap &mk, const CUtensorMap &mv, const CU
         }
         return PKV_ERR_INVALID_ARG;
     }
-    // the work counter is only used when the reduce kernel follows to re-arm it
+    // the work counter is used only when some context spans several partitions (the
+    // merge kernel then arms the header; with one partition per context nothing would)
     pkv::DecodeParams p = prm;
     if (!merge) p.sched = nullptr;
     int rc = PKV_ERR_INVALID_ARG;
@@ -509,7 +510,7 @@ int dispatch_step(int BS, const CUtensorMap &mk, const CUtensorMap &mv, const CU
         case 16: rc = launch_decode<T, D, 16, true>(mk, mv, mq, p, items, st); break;
         case 32: rc = launch_decode<T, D, 32, true>(mk, mv, mq, p, items, st); break;
     }
-    if (rc == PKV_OK && merge) rc = launch_reduce<T, D>(p, st);
+    if (rc == PKV_OK && merge && launch_merge) rc = launch_reduce<T, D>(p, st);
     return rc;
 }
 
@@ -562,13 +563,17 @@ int pkv_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int
     return PKV_OK;
 }
 
-int pkv_paged_attention_decode(void *out, const void *q, const void *k_cache,
-                               const void *v_cache, const int32_t *block_tables,
-                               const int32_t *context_lens, int num_seqs, int num_heads,
-                               int num_kv_heads, int head_dim, int block_size,
-                               int max_blocks_per_seq, int num_blocks, int max_context_len,
-                               float scale, int dtype, int partition_size, void *workspace,
-                               size_t workspace_bytes, pkv_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// pkv_paged_attention_decode (with_merge) or its partition launch alone.
+int decode_impl(void *out, const void *q, const void *k_cache, const void *v_cache,
+                const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
+                int num_heads, int num_kv_heads, int head_dim, int block_size,
+                int max_blocks_per_seq, int num_blocks, int max_context_len, float scale,
+                int dtype, int partition_size, void *workspace, size_t workspace_bytes,
+                pkv_stream_t stream, bool with_merge) {
     int P;
     int rc = check_decode_sizes(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
                                 max_context_len, partition_size, &P);
@@ -628,17 +633,88 @@ int pkv_paged_attention_decode(void *out, const void *q, const void *k_cache,
     if (dtype == PKV_BF16) {
         rc = head_dim == 128 ? dispatch_bs<__nv_bfloat16, 128>(block_size, mk, mv, mq, prm, items, st)
                              : dispatch_bs<__nv_bfloat16, 64>(block_size, mk, mv, mq, prm, items, st);
-        if (rc == PKV_OK && pmax > 1)
+        if (rc == PKV_OK && pmax > 1 && with_merge)
             rc = head_dim == 128 ? launch_reduce<__nv_bfloat16, 128>(prm, st)
                                  : launch_reduce<__nv_bfloat16, 64>(prm, st);
     } else {
         rc = head_dim == 128 ? dispatch_bs<__half, 128>(block_size, mk, mv, mq, prm, items, st)
                              : dispatch_bs<__half, 64>(block_size, mk, mv, mq, prm, items, st);
-        if (rc == PKV_OK && pmax > 1)
+        if (rc == PKV_OK && pmax > 1 && with_merge)
             rc = head_dim == 128 ? launch_reduce<__half, 128>(prm, st)
                                  : launch_reduce<__half, 64>(prm, st);
     }
     return rc;
+}
+
+}  // namespace
+
+extern "C" {
+
+int pkv_paged_attention_decode(void *out, const void *q, const void *k_cache,
+                               const void *v_cache, const int32_t *block_tables,
+                               const int32_t *context_lens, int num_seqs, int num_heads,
+                               int num_kv_heads, int head_dim, int block_size,
+                               int max_blocks_per_seq, int num_blocks, int max_context_len,
+                               float scale, int dtype, int partition_size, void *workspace,
+                               size_t workspace_bytes, pkv_stream_t stream) {
+    return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs, num_heads,
+                       num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,
+                       max_context_len, scale, dtype, partition_size, workspace, workspace_bytes,
+                       stream, true);
+}
+
+int pkv_paged_attention_decode_partitions(void *out, const void *q, const void *k_cache,
+                                          const void *v_cache, const int32_t *block_tables,
+                                          const int32_t *context_lens, int num_seqs,
+                                          int num_heads, int num_kv_heads, int head_dim,
+                                          int block_size, int max_blocks_per_seq, int num_blocks,
+                                          int max_context_len, float scale, int dtype,
+                                          int partition_size, void *workspace,
+                                          size_t workspace_bytes, pkv_stream_t stream) {
+    return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs, num_heads,
+                       num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,
+                       max_context_len, scale, dtype, partition_size, workspace, workspace_bytes,
+                       stream, false);
+}
+
+int pkv_paged_attention_merge(void *out, const int32_t *context_lens, int num_seqs, int num_heads,
+                              int num_kv_heads, int head_dim, int block_size, int max_context_len,
+                              int partition_size, int dtype, void *workspace,
+                              size_t workspace_bytes, pkv_stream_t stream) {
+    int P;
+    int rc = check_decode_sizes(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                max_context_len, partition_size, &P);
+    if (rc != PKV_OK) return rc;
+    if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_ERR_INVALID_ARG;
+    const WsLayout ws = ws_layout(num_seqs, num_heads, head_dim, max_context_len, P);
+    if (num_seqs == 0 || ws.total == 0) return PKV_OK;   // every context is one partition
+    if (!out || !context_lens || !aligned(out, 2) || !aligned(context_lens, 4))
+        return PKV_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < ws.total || !aligned(workspace, 16))
+        return PKV_ERR_WORKSPACE;
+    unsigned int *status;
+    if ((rc = device_status_ptr(&status)) != PKV_OK) return rc;
+    uint8_t *wsb = static_cast<uint8_t *>(workspace);
+    pkv::DecodeParams prm{};
+    prm.out = out;
+    prm.context_lens = context_lens;
+    prm.sched = reinterpret_cast<pkv::SchedHeader *>(wsb);
+    prm.ws_seq_base = reinterpret_cast<int32_t *>(wsb + ws.seq_base);
+    prm.ws_ml = reinterpret_cast<float *>(wsb + ws.ml);
+    prm.ws_o = reinterpret_cast<float *>(wsb + ws.o);
+    prm.status = status;
+    prm.num_seqs = num_seqs;
+    prm.num_heads = num_heads;
+    prm.num_kv_heads = num_kv_heads;
+    prm.group = num_heads / num_kv_heads;
+    prm.max_context_len = max_context_len;
+    prm.partition = P;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (dtype == PKV_BF16)
+        return head_dim == 128 ? launch_reduce<__nv_bfloat16, 128>(prm, st)
+                               : launch_reduce<__nv_bfloat16, 64>(prm, st);
+    return head_dim == 128 ? launch_reduce<__half, 128>(prm, st)
+                           : launch_reduce<__half, 64>(prm, st);
 }
 
 int pkv_paged_attention_decode_noalloc(void *out, const void *q, const void *k_cache,
@@ -678,13 +754,17 @@ int pkv_decode_step_workspace_size(int num_seqs, int num_heads, int num_kv_heads
     return PKV_OK;
 }
 
-int pkv_paged_decode_step(void *out, const void *q, const void *k_new, const void *v_new,
-                          void *k_cache, void *v_cache, const int32_t *block_tables,
-                          const int32_t *context_lens, int num_seqs, int num_heads,
-                          int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
-                          int num_blocks, int max_context_len, float scale, int dtype,
-                          int partition_size, void *workspace, size_t workspace_bytes,
-                          pkv_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// pkv_paged_decode_step (split = false) or the write-and-decode launch alone (split).
+int step_impl(void *out, const void *q, const void *k_new, const void *v_new, void *k_cache,
+              void *v_cache, const int32_t *block_tables, const int32_t *context_lens,
+              int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+              int max_blocks_per_seq, int num_blocks, int max_context_len, float scale, int dtype,
+              int partition_size, void *workspace, size_t workspace_bytes, pkv_stream_t stream,
+              bool split) {
     int P;
     int rc = check_decode_sizes(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
                                 max_context_len, partition_size, &P);
@@ -748,16 +828,49 @@ int pkv_paged_decode_step(void *out, const void *q, const void *k_new, const voi
     const int merge = pmax > 1;
     int nsm;
     if ((rc = sm_count(&nsm)) != PKV_OK) return rc;
-    const int ink = step_merges_in_kernel(num_seqs, num_heads, items, pmax, nsm);
+    const int ink = split ? 0 : step_merges_in_kernel(num_seqs, num_heads, items, pmax, nsm);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (dtype == PKV_BF16)
         return head_dim == 128 ? dispatch_step<__nv_bfloat16, 128>(block_size, mk, mv, mq, prm,
-                                                                   items, merge, ink, st)
+                                                                   items, merge, ink, !split, st)
                                : dispatch_step<__nv_bfloat16, 64>(block_size, mk, mv, mq, prm,
-                                                                  items, merge, ink, st);
+                                                                  items, merge, ink, !split, st);
     return head_dim == 128
-               ? dispatch_step<__half, 128>(block_size, mk, mv, mq, prm, items, merge, ink, st)
-               : dispatch_step<__half, 64>(block_size, mk, mv, mq, prm, items, merge, ink, st);
+               ? dispatch_step<__half, 128>(block_size, mk, mv, mq, prm, items, merge, ink,
+                                            !split, st)
+               : dispatch_step<__half, 64>(block_size, mk, mv, mq, prm, items, merge, ink,
+                                           !split, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int pkv_paged_decode_step(void *out, const void *q, const void *k_new, const void *v_new,
+                          void *k_cache, void *v_cache, const int32_t *block_tables,
+                          const int32_t *context_lens, int num_seqs, int num_heads,
+                          int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                          int num_blocks, int max_context_len, float scale, int dtype,
+                          int partition_size, void *workspace, size_t workspace_bytes,
+                          pkv_stream_t stream) {
+    return step_impl(out, q, k_new, v_new, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                     num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                     num_blocks, max_context_len, scale, dtype, partition_size, workspace,
+                     workspace_bytes, stream, false);
+}
+
+int pkv_paged_decode_step_partitions(void *out, const void *q, const void *k_new,
+                                     const void *v_new, void *k_cache, void *v_cache,
+                                     const int32_t *block_tables, const int32_t *context_lens,
+                                     int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                     int block_size, int max_blocks_per_seq, int num_blocks,
+                                     int max_context_len, float scale, int dtype,
+                                     int partition_size, void *workspace, size_t workspace_bytes,
+                                     pkv_stream_t stream) {
+    return step_impl(out, q, k_new, v_new, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                     num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                     num_blocks, max_context_len, scale, dtype, partition_size, workspace,
+                     workspace_bytes, stream, true);
 }
 
 int pkv_decode_step_launches(int num_seqs, int num_heads, int num_kv_heads, int head_dim,

@@ -112,7 +112,7 @@ paged_decode_step_kernel(const __grid_constant__ CUtensorMap tmap_k,
     __syncthreads();
     if (!s_flag) return;   // same decision in every CTA: nothing has written the header
 
-    decode_items<T, D, BS, true>(&tmap_k, &tmap_v, &tmap_q, prm, sm, 1);
+    decode_items<T, D, BS, true>(&tmap_k, &tmap_v, &tmap_q, prm, sm, hdr != nullptr);
     if (!hdr) return;
 
     if (merge) {

@@ -152,6 +152,16 @@ def test_step_and_shared_prefix_checks_without_a_device():
     assert L.pkv_decode_step_workspace_size(4, 8, 2, 64, 16, 64, 64, ctypes.byref(one)) == 0
     assert L.pkv_decode_step_workspace_size(4, 8, 2, 64, 16, 1024, 64, ctypes.byref(many)) == 0
     assert one.value == 256 and many.value > one.value
+    # merge alone: nothing to merge without partitions or sequences; bad dtype; no workspace
+    assert L.pkv_paged_attention_merge(None, None, 0, 8, 2, 64, 16, 1000, 64, 0, None, 0,
+                                       None) == B.PKV_OK
+    assert L.pkv_paged_attention_merge(None, None, 4, 8, 2, 64, 16, 64, 64, 0, None, 0,
+                                       None) == B.PKV_OK
+    assert L.pkv_paged_attention_merge(None, None, 4, 8, 2, 64, 16, 1000, 64, 3, None, 0,
+                                       None) == B.PKV_ERR_INVALID_ARG
+    buf = ctypes.create_string_buffer(64)
+    assert L.pkv_paged_attention_merge(ctypes.addressof(buf), ctypes.addressof(buf), 4, 8, 2, 64,
+                                       16, 1000, 64, 0, None, 0, None) == B.PKV_ERR_WORKSPACE
     # device append: negative sizes, missing cursor
     assert L.pkv_device_append(None, None, None, 0, None, None, None, 4, 8, 16, 64, 128,
                                None) == B.PKV_ERR_INVALID_ARG

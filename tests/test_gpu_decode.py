@@ -286,3 +286,34 @@ def test_items_of_256_blocks(cuda_device, BS, P):
     q, kc, vc, bt, lens, max_len = random_case(rng, [9000, P, P + 1, 300, 2 * P - 5], 16, 2, 128,
                                                BS, dtype)
     check_case(q, kc, vc, bt, lens, max_len, dtype, 0.09, P, f"BS={BS} P={P}")
+
+
+@pytest.mark.parametrize("nseq,Hq,Hkv,D,BS,P,dtype", [
+    (40, 32, 8, 128, 16, 64, synth.BF16),      # sequence-major order, many partitions
+    (20, 16, 16, 128, 32, 128, synth.F16),     # longest-first order (<= 32 sequences)
+    (300, 8, 2, 64, 8, 256, synth.F16),
+    (7, 64, 8, 128, 16, 0, synth.BF16)])
+def test_partitions_then_merge_equal_the_decode(cuda_device, nseq, Hq, Hkv, D, BS, P, dtype):
+    """The two launches of the decode as separate calls give its bits; the partitions
+    call repeated on one workspace without a merge in between (each launch re-arms the
+    work counter it used) gives the same partials, and the oracle agrees."""
+    rng = np.random.default_rng(nseq + Hq + D + BS + P)
+    lens = list(rng.integers(1, 1500, nseq))
+    q, kc, vc, bt, lens, max_len = random_case(rng, lens, Hq, Hkv, D, BS, dtype)
+    qd, kcd, vcd = to_dev(q, dtype), to_dev(kc, dtype), to_dev(vc, dtype)
+    btd, lensd = torch.from_numpy(bt).cuda(), torch.from_numpy(lens).cuda()
+    ref_out = decode_dev(qd, kcd, vcd, btd, lensd, max_len, 0.07, P)
+    need = pkv.pkv_decode_workspace_size(nseq, Hq, Hkv, D, BS, max_len, P)
+    ws = torch.full((max(need, 16),), 0x5A, dtype=torch.uint8, device="cuda")
+    pkv.pkv_get_device_status(clear=True)
+    for rep in range(3):
+        out = torch.full_like(qd, float("nan"))
+        for _ in range(rep + 1):
+            pkv.pkv_paged_attention_decode_partitions(out, qd, kcd, vcd, btd, lensd, max_len, ws,
+                                                      scale=0.07, partition_size=P)
+        pkv.pkv_paged_attention_merge(out, lensd, Hkv, BS, max_len, ws, partition_size=P)
+        torch.cuda.synchronize()
+        assert pkv.pkv_get_device_status() == 0
+        assert np.array_equal(to_bits(out), to_bits(ref_out)), rep
+    ref = A.paged_decode_attention(q, kc, vc, bt, lens, 0.07, dtype)
+    assert_close(to_bits(out), ref, dtype, "partitions + merge")

@@ -578,3 +578,34 @@ def test_grid_barrier_gives_up_and_the_workspace_recovers(cuda_device):
     ek, ev, ref = oracle_step(dtype, case)
     assert np.array_equal(to_bits(kcd), ek) and np.array_equal(to_bits(vcd), ev)
     assert_close(to_bits(out2), ref, dtype, "step after a barrier timeout")
+
+
+@pytest.mark.parametrize("Hq,Hkv,D,BS,P", [(32, 8, 128, 16, 64), (16, 16, 128, 16, 512),
+                                           (8, 2, 64, 32, 128)])
+def test_step_partitions_then_merge_equal_the_step(cuda_device, Hq, Hkv, D, BS, P):
+    """The write-and-decode launch alone, then the merge, on one workspace, step after
+    step: the bits of the fused step call (which for these shapes may merge in its own
+    launch) and the same cache writes."""
+    rng = np.random.default_rng(Hq * 7 + BS + P)
+    dtype = synth.F16
+    lens = list(rng.integers(1, 1300, 37))
+    q, kc, vc, bt, lens, max_len, slots, kn, vn = step_case(rng, lens, Hq, Hkv, D, BS, dtype)
+    qd, knd, vnd = to_dev(q, dtype), to_dev(kn, dtype), to_dev(vn, dtype)
+    btd, lensd = torch.from_numpy(bt).cuda(), torch.from_numpy(lens).cuda()
+    kc1, vc1 = to_dev(kc, dtype), to_dev(vc, dtype)
+    out1 = torch.empty_like(qd)
+    pkv.pkv_get_device_status(clear=True)
+    pkv.pkv_paged_decode_step(out1, qd, knd, vnd, kc1, vc1, btd, lensd, max_len,
+                              step_ws(q, kc, max_len, P), partition_size=P)
+    ws = step_ws(q, kc, max_len, P)
+    for rep in range(3):
+        kc2, vc2 = to_dev(kc, dtype), to_dev(vc, dtype)
+        out2 = torch.full_like(qd, float("nan"))
+        pkv.pkv_paged_decode_step_partitions(out2, qd, knd, vnd, kc2, vc2, btd, lensd, max_len,
+                                             ws, partition_size=P)
+        pkv.pkv_paged_attention_merge(out2, lensd, Hkv, BS, max_len, ws, partition_size=P)
+        torch.cuda.synchronize()
+        assert pkv.pkv_get_device_status() == 0
+        assert np.array_equal(to_bits(out1), to_bits(out2)), rep
+        assert torch.equal(kc1.view(torch.int16), kc2.view(torch.int16))
+        assert torch.equal(vc1.view(torch.int16), vc2.view(torch.int16))
