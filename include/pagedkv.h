@@ -178,8 +178,9 @@ int pkv_paged_attention_decode_noalloc(void *out, const void *q, const void *k_c
  * batches where groups of sequences share their first pages (parallel sampling, common
  * prompts: "vLLM" entity page, 是什么; "分页 KV Cache 分析" §3.2). Each shared prefix page
  * of a KV head is read once for up to 16 query rows (the G heads of up to 16/G member
- * sequences) instead of once per sequence; private suffixes are read per sequence; the
- * pieces are merged exactly (log-sum-exp).
+ * sequences) instead of once per sequence; private suffixes are read per sequence, in the
+ * same work item as the prefix where both fit in one partition (then written directly),
+ * else as pieces merged exactly (log-sum-exp).
  *
  * group_start  device int32 [num_groups + 1]: sequences group_start[g] ..
  *              group_start[g+1]-1 form group g (0 = group_start[0] < ... <
@@ -192,8 +193,8 @@ int pkv_paged_attention_decode_noalloc(void *out, const void *q, const void *k_c
  * PKV_STATUS_BAD_LEN. Workspace: pkv_decode_shared_prefix_workspace_size bytes of device
  * memory, 16-byte aligned, owned by the caller, no initial contents required (else
  * PKV_ERR_WORKSPACE). partition_size 0 selects this path's own automatic size
- * (pkv_decode_shared_prefix_partition_size: 1024 tokens for groups up to 4, 2048 above,
- * at most 256 blocks, smaller for small batches). Other arguments, limits and errors as
+ * (pkv_decode_shared_prefix_partition_size: 2048 tokens, at most 256 blocks, smaller for
+ * small batches). Other arguments, limits and errors as
  * pkv_paged_attention_decode (num_groups >= 1, <= num_seqs). Three kernel launches.
  * ---------------------------------------------------------------------------- */
 int pkv_paged_attention_decode_shared_prefix(

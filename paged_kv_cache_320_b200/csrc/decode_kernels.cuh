@@ -372,9 +372,12 @@ __device__ __forceinline__ void reset_state(WarpState<D> &st) {
 // One warp's share of a stage: tokens tok0 .. tok0+15 of the stage's K and V tiles
 // (tok0 a multiple of 16), of which the first `valid` belong to the sequence.
 //   S = Q K^T (two n-tiles of 8 tokens), scale, mask, online softmax, O += P V.
-template <typename T, int D, int BS>
+// kRows: only query rows r0 <= row < r1 attend to these tokens (the others' scores are
+// -inf); a row that has attended to nothing yet keeps m = -inf, l = 0, o = 0.
+template <typename T, int D, int BS, bool kRows = false>
 __device__ __forceinline__ void consume_stage(WarpState<D> &st, uint32_t kbase, uint32_t vbase,
-                                              int tok0, int lane, int valid, float scale_log2) {
+                                              int tok0, int lane, int valid, float scale_log2,
+                                              int r0 = 0, int r1 = kMaxGroup) {
     constexpr int H = D / 64;
     constexpr int NT = D / 8;
     const int tig = lane & 3;
@@ -397,14 +400,17 @@ __device__ __forceinline__ void consume_stage(WarpState<D> &st, uint32_t kbase, 
         }
     }
     // scale, mask, online softmax (rows gid and gid+8)
+    const int gid = lane >> 2;
+    const bool row0_in = !kRows || (gid >= r0 && gid < r1);
+    const bool row1_in = !kRows || (gid + 8 >= r0 && gid + 8 < r1);
     float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
             const bool in_seq = 8 * nt + 2 * tig + e < valid;
-            sc[nt][e] = in_seq ? sc[nt][e] * scale_log2 : -INFINITY;
-            sc[nt][2 + e] = in_seq ? sc[nt][2 + e] * scale_log2 : -INFINITY;
+            sc[nt][e] = in_seq && row0_in ? sc[nt][e] * scale_log2 : -INFINITY;
+            sc[nt][2 + e] = in_seq && row1_in ? sc[nt][2 + e] * scale_log2 : -INFINITY;
             mx0 = fmaxf(mx0, sc[nt][e]);
             mx1 = fmaxf(mx1, sc[nt][2 + e]);
         }
@@ -414,7 +420,11 @@ __device__ __forceinline__ void consume_stage(WarpState<D> &st, uint32_t kbase, 
     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
     const float mn0 = fmaxf(st.m0, mx0), mn1 = fmaxf(st.m1, mx1);
-    const float a0 = ex2(st.m0 - mn0), a1 = ex2(st.m1 - mn1);
+    // with row masks a row may still have seen nothing (max -inf): subtract 0 instead,
+    // so that its weights are 0 rather than NaN
+    const float ms0 = kRows && mn0 == -INFINITY ? 0.f : mn0;
+    const float ms1 = kRows && mn1 == -INFINITY ? 0.f : mn1;
+    const float a0 = ex2(st.m0 - ms0), a1 = ex2(st.m1 - ms1);
     st.m0 = mn0;
     st.m1 = mn1;
     float ps0 = 0.f, ps1 = 0.f;
@@ -422,8 +432,8 @@ __device__ __forceinline__ void consume_stage(WarpState<D> &st, uint32_t kbase, 
     for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-            sc[nt][e] = ex2(sc[nt][e] - mn0);
-            sc[nt][2 + e] = ex2(sc[nt][2 + e] - mn1);
+            sc[nt][e] = ex2(sc[nt][e] - ms0);
+            sc[nt][2 + e] = ex2(sc[nt][2 + e] - ms1);
             ps0 += sc[nt][e];
             ps1 += sc[nt][2 + e];
         }

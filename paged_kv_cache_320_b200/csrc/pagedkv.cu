@@ -178,14 +178,13 @@ int auto_partition(int B, int Hq, int Hkv, int BS, int max_len) {
     return p;
 }
 
-// Automatic partition size of the shared-prefix decode: 1024 tokens for groups up to 4
-// and 2048 above (same block and batch limits). Its prefix items carry 16 query rows, so
-// the per-item costs (query rows in, a four-warp merge and 16 partial rows out) are larger
-// than a plain item's; on 16 prompts x 8 samples with a 1024-token prefix, 1024 measured
-// 9 % faster than 512, 256 slower, 2048 equal.
+// Automatic partition size of the shared-prefix decode: 2048 tokens (same block and
+// batch limits as the plain decode's). An item carries up to 16 query rows and, where
+// they fit in one partition's stages, a chunk's last prefix partition and its members'
+// first suffix partition together, which then need no merge.
 int auto_shared_partition(int B, int Hq, int Hkv, int BS, int max_len) {
-    const int G = Hq / Hkv;
-    int p = G <= 4 ? 1024 : 2048;
+    (void)Hq;
+    int p = 2048;
     if (p > pkv::kMaxItemBlocks * BS) p = pkv::kMaxItemBlocks * BS;
     while (p > 64 && (long long)B * Hkv * cdiv(max_len, p) < 1024) p /= 2;
     return p;

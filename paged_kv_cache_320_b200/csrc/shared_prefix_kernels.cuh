@@ -15,7 +15,18 @@
 // at the first logical block where a member's table differs from the group's first
 // member, so a wrong declaration costs sharing, never correctness); the decode kernel
 // runs the items with the same TMA / mbarrier / tensor-core pipeline as plain decode;
-// the reduce merges each (sequence, head)'s partials.
+// the reduce merges the partials of the (sequence, head) pairs whose work was split.
+//
+// Work items. The members of a group are taken R = 16 / G at a time ("chunks", 16 query
+// rows). A chunk's tokens are its prefix, cut into partitions of P tokens, and its
+// members' suffixes, cut into partitions of P tokens per member (suffix partition k of a
+// chunk holds every member's tokens [pre + kP, pre + (k+1)P)). An item is one of them
+// for one KV head, or the last prefix partition and the first suffix partition
+// together when their 64-token stages fit in one partition's budget. The item's stages
+// come in segments (the prefix pages, then each member's own pages); during a member's
+// segment only that member's G rows attend. A chunk that is one item writes its output
+// directly; otherwise each item leaves one partial per row (empty for rows it did not
+// touch) for the reduce.
 #pragma once
 
 #include "decode_kernels.cuh"
@@ -23,15 +34,21 @@
 namespace pkv {
 
 struct SharedItem {
-    int table_seq;   // sequence whose block-table row holds the item's pages
-    int tok0;        // first token (a multiple of the block size)
-    int ntok;        // tokens
-    int hk;          // KV head
+    int table_seq;   // the group's first member: its block-table row holds the prefix pages
+    int pre;         // the group's shared tokens (a multiple of the block size)
     int first_seq;   // query rows: sequences first_seq .. first_seq + nseq - 1, G heads each
     int nseq;
-    int part;        // index of this piece in each row's list of partials
-    int pad;
+    int hk;          // KV head
+    int part;        // index of this item among its chunk's items (its partials' index)
+    int npp;         // prefix partitions of the chunk
+    int nps2;        // 2 x suffix partitions of the chunk, + 1 if the last prefix partition
+                     // and the first suffix partition are one item
 };
+
+// Items of a chunk: prefix partitions, then suffix partitions, one fewer if fused.
+__host__ __device__ __forceinline__ int chunk_parts(int npp, int nps2) {
+    return npp + (nps2 >> 1) - (nps2 & 1);
+}
 
 struct SharedCounters {
     unsigned next;    // next work item (0 after the plan and after every reduce)
@@ -59,9 +76,10 @@ struct SharedParams {
     int *row_base;     // [B] scratch row of (s, h, j) = row_base[s] + h * np[s] + j
     int *seq_group;    // [B] group of each sequence (plan scratch)
     int *gpre;         // [B] shared tokens per group (plan scratch)
-    int *gmin;         // [B] shortest member per group (plan scratch)
-    int *gmis;         // [B] first logical block where a member's table differs (plan scratch)
-    int *ioff;         // [B] first suffix item of each sequence (plan scratch)
+    int *gmin;         // [B] shortest member, then first chunk, per group (plan scratch)
+    int *gmis;         // [B] first block where a member's table differs per group, then
+                       //     first item per chunk (plan scratch)
+    int *ioff;         // [B] 2 x suffix partitions + fused, per chunk (plan scratch)
     float *ws_o;       // [rows][D]
     float *ws_ml;      // [rows][2]
     void *out;
@@ -147,7 +165,7 @@ shared_prefix_plan_kernel(SharedParams p) {
     int *gmis = in_smem ? plan_smem + 3 * B : p.gmis;
     int *slen = in_smem ? plan_smem + 4 * B : p.np;          // clamped lengths
     int *gfirst = in_smem ? plan_smem + 5 * B : p.row_base;  // first member of each group
-    int *ioff = in_smem ? plan_smem + 6 * B : p.ioff;        // suffix-item offsets
+    int *ioff = in_smem ? plan_smem + 6 * B : p.ioff;        // per-chunk partition counts
     if (tid == 0) {
         bad = 0;
         max_pre_blocks = 0;
@@ -206,113 +224,132 @@ shared_prefix_plan_kernel(SharedParams p) {
         if (mis != 0x7fffffff) atomicMin(&gmis[g], mis);
     }
     __syncthreads();
-    // pass 3 (per group): shared length and prefix-item offsets
-    int base_items = 0;
+    // pass 3 (per group): shared length; chunks of R members; first chunk of each group
+    const int S = P / kStageTokens;   // 64-token stages per partition
+    int n_chunks = 0;
     for (int g0 = 0; g0 < ng; g0 += kPlanThreads) {
         const int g = g0 + tid;
-        int pre = 0, cnt = 0;
+        int cnt = 0;
         if (g < ng) {
             const int first = gfirst[g];
             const int last = bad ? g + 1 : p.group_start[g + 1];
             const int shortest = gmin[g];
-            pre = min(gpre[g], shortest - shortest % BS);
+            int pre = min(gpre[g], shortest - shortest % BS);
             pre = min(pre, min(gmis[g], pre / BS) * BS);
-            if (pre > 0) cnt = Hkv * ((last - first + R - 1) / R) * ((pre + P - 1) / P);
+            gpre[g] = pre;
+            cnt = (last - first + R - 1) / R;
         }
         int total;
-        const int at = base_items + block_exclusive_scan(cnt, sm, &total);
-        if (g < ng) {
-            gpre[g] = pre;   // only thread g reads gpre[g] in this pass
-            gmin[g] = at;    // first prefix item of group g
-        }
-        base_items += total;
+        const int at = n_chunks + block_exclusive_scan(cnt, sm, &total);
+        if (g < ng) gmin[g] = at;   // first chunk of group g (only thread g reads gmin[g] here)
+        n_chunks += total;
     }
-    const int n_prefix = base_items;
+    int *chunk_base = gmin;
+    int *item_base = gmis;    // per chunk (n_chunks <= B)
+    int *chunk_nps2 = ioff;   // per chunk
     __syncthreads();
-    // pass 3b (per prefix item): item i belongs to the group g with gmin[g] <= i
-    for (int i = tid; i < n_prefix && i < p.max_items; i += kPlanThreads) {
-        const int g = owner_of(gmin, ng, i);
-        const int first = gfirst[g];
+    // pass 4 (per chunk): prefix and suffix partitions, fusion, first item
+    int n_items = 0;
+    for (int c0 = 0; c0 < n_chunks; c0 += kPlanThreads) {
+        const int ch = c0 + tid;
+        int cnt = 0;
+        if (ch < n_chunks) {
+            const int g = owner_of(chunk_base, ng, ch);
+            const int first = gfirst[g] + (ch - chunk_base[g]) * R;
+            const int last = bad ? g + 1 : p.group_start[g + 1];
+            const int nseq = min(R, last - first);
+            const int pre = gpre[g];
+            const int npp = (pre + P - 1) / P;
+            int nps = 0, st0 = 0;
+            for (int m = 0; m < nseq; ++m) {
+                const int suf = slen[first + m] - pre;   // >= 0: pre <= the shortest member
+                nps = max(nps, (suf + P - 1) / P);
+                st0 += (min(P, suf) + kStageTokens - 1) / kStageTokens;
+            }
+            if (npp == 0 && nps == 0) nps = 1;   // empty contexts: one item writes zeros
+            const int pre_last = npp ? (pre - (npp - 1) * P + kStageTokens - 1) / kStageTokens : 0;
+            const int fuse = npp > 0 && nps > 0 && pre_last + st0 <= S;
+            chunk_nps2[ch] = 2 * nps + fuse;
+            cnt = Hkv * chunk_parts(npp, 2 * nps + fuse);
+        }
+        int total;
+        const int at = n_items + block_exclusive_scan(cnt, sm, &total);
+        if (ch < n_chunks) item_base[ch] = at;
+        n_items += total;
+    }
+    __syncthreads();
+    // pass 5 (per item): chunk, KV head and part
+    for (int i = tid; i < n_items && i < p.max_items; i += kPlanThreads) {
+        const int ch = owner_of(item_base, n_chunks, i);
+        const int g = owner_of(chunk_base, ng, ch);
+        const int first = gfirst[g] + (ch - chunk_base[g]) * R;
         const int last = bad ? g + 1 : p.group_start[g + 1];
         const int pre = gpre[g];
         const int npp = (pre + P - 1) / P;
-        const int chunks = (last - first + R - 1) / R;
-        int local = i - gmin[g];
-        const int j = local % npp;
-        local /= npp;
-        const int c = local % chunks;
-        const int hk = local / chunks;
+        const int nps2 = chunk_nps2[ch];
+        const int np = chunk_parts(npp, nps2);
+        const int local = i - item_base[ch];
         SharedItem it;
-        it.table_seq = first;
-        it.tok0 = j * P;
-        it.ntok = min(P, pre - j * P);
-        it.hk = hk;
-        it.first_seq = first + c * R;
-        it.nseq = min(R, last - (first + c * R));
-        it.part = j;
-        it.pad = 0;
+        it.table_seq = gfirst[g];
+        it.pre = pre;
+        it.first_seq = first;
+        it.nseq = min(R, last - first);
+        it.hk = local / np;
+        it.part = local - it.hk * np;
+        it.npp = npp;
+        it.nps2 = nps2;
         p.items[i] = it;
     }
     __syncthreads();
-    // pass 4 (per sequence): partial counts, scratch rows, suffix-item offsets
+    // pass 6 (per sequence): partials per (sequence, head) = its chunk's items, then the
+    // scratch rows. slen becomes the partial count (in the workspace it is p.np itself),
+    // and row_base may overwrite gfirst only once every count is known.
+    for (int s = tid; s < B; s += kPlanThreads) {
+        const int g = seq_group[s];
+        const int ch = chunk_base[g] + (s - gfirst[g]) / R;
+        slen[s] = chunk_parts((gpre[g] + P - 1) / P, chunk_nps2[ch]);
+    }
+    __syncthreads();
     int base_rows = 0;
     for (int s0 = 0; s0 < B; s0 += kPlanThreads) {
         const int s = s0 + tid;
-        int pre = 0, npp = 0, nps = 0;
+        const int np = s < B ? slen[s] : 0;
+        int total_rows;
+        const int row = base_rows + block_exclusive_scan(np, sm, &total_rows);
         if (s < B) {
-            pre = gpre[seq_group[s]];
-            npp = (pre + P - 1) / P;
-            nps = max(1, (slen[s] - pre + P - 1) / P);
-        }
-        int total_items, total_rows;
-        const int at = base_items + block_exclusive_scan(s < B ? Hkv * nps : 0, sm, &total_items);
-        const int row =
-            base_rows + block_exclusive_scan(s < B ? (npp + nps) : 0, sm, &total_rows);
-        if (s < B) {
-            ioff[s] = at - n_prefix;   // first suffix item of s (relative)
             p.row_base[s] = row * p.num_heads;
+            p.np[s] = np;
         }
-        base_items += total_items;
         base_rows += total_rows;
     }
-    __syncthreads();
-    // pass 4b (per suffix item)
-    for (int i = tid; i < base_items - n_prefix && n_prefix + i < p.max_items;
-         i += kPlanThreads) {
-        const int s = owner_of(ioff, B, i);
-        const int pre = gpre[seq_group[s]];
-        const int npp = (pre + P - 1) / P;
-        const int len = slen[s];
-        const int nps = max(1, (len - pre + P - 1) / P);
-        const int local = i - ioff[s];
-        const int hk = local / nps, j = local - hk * nps;
-        SharedItem it;
-        it.table_seq = s;
-        it.tok0 = pre + j * P;
-        it.ntok = max(0, min(P, len - pre - j * P));
-        it.hk = hk;
-        it.first_seq = s;
-        it.nseq = 1;
-        it.part = npp + j;
-        it.pad = 0;
-        p.items[n_prefix + i] = it;
-    }
-    // partial counts last: np aliases the length scratch when it lives in the workspace
-    __syncthreads();
-    for (int s = tid; s < B; s += kPlanThreads) {
-        const int pre = gpre[seq_group[s]];
-        const int npp = (pre + P - 1) / P;
-        p.np[s] = npp + max(1, (slen[s] - pre + P - 1) / P);
-    }
     if (tid == 0) {
-        if (base_items > p.max_items) atomicOr(p.status, kStatusBadLen);
-        p.counters->count = min(base_items, p.max_items);
+        if (n_items > p.max_items) atomicOr(p.status, kStatusBadLen);
+        p.counters->count = min(n_items, p.max_items);
         p.counters->sig[0] = kPlanMagic;
         p.counters->sig[1] = B;
         p.counters->sig[2] = p.num_heads | (Hkv << 16);
         p.counters->sig[3] = P;
     }
 }
+
+// The producer's view of an item: its descriptor (lane k < 8 holds field k), each
+// member's token count in this item's suffix partition (lane m), and which segments
+// have tokens (bit 0: the prefix partition, bit 1 + m: member m's suffix part).
+struct SharedItemCtx {
+    int idx;
+    int f;
+    int mtok;
+    unsigned mask;
+    bool valid;
+};
+
+// One segment: tokens [tok0, tok0 + ntok) of sequence `seq`'s pages, attended by query
+// rows [r0, r1) of the item.
+struct SharedSeg {
+    int seq, tok0, ntok, r0, r1;
+    int sidx;        // 0: prefix partition, 1 + m: member m's suffix partition
+    bool first, last, valid;
+};
 
 template <typename T, int D, int BS>
 __global__ void __launch_bounds__(kDecodeThreads, 2)
@@ -336,6 +373,7 @@ paged_decode_shared_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int lane = threadIdx.x & 31;
     const int G = prm.group;
     const int Hkv = prm.num_kv_heads;
+    const int P = prm.partition;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < L::kStages; ++i) {
@@ -362,44 +400,91 @@ paged_decode_shared_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const int count = prm.counters->count;
         int it = 0;
         bool ok = true;
-        // item descriptor: lane k < 8 holds field k
-        auto fetch = [&](int idx) {
-            int v = 0;
-            if (idx < count && lane < 8) v = reinterpret_cast<const int *>(prm.items + idx)[lane];
-            return v;
-        };
         auto take = [&]() {
             unsigned v = 0;
             if (lane == 0) v = atomicAdd(&prm.counters->next, 1u);
-            v = __shfl_sync(0xffffffffu, v, 0);
-            return v > 0x7fffffffu ? 0x7fffffff : (int)v;
+            return v > 0x7fffffffu ? 0x7fffffff : (int)v;   // lives in lane 0
         };
-        // an item's slice of its block-table row: entry e in lane e % 32, register e / 32
-        auto load_entries = [&](int f, int (&ent)[kMaxItemBlocks / 32]) {
-            const int table_seq = __shfl_sync(0xffffffffu, f, 0);
-            const int tok0 = __shfl_sync(0xffffffffu, f, 1);
-            const int ntok = __shfl_sync(0xffffffffu, f, 2);
-            const int nblk = (ntok + BS - 1) / BS;
+        auto field = [&](const SharedItemCtx &c, int k) { return __shfl_sync(0xffffffffu, c.f, k); };
+        // descriptor, members' suffix-part token counts, non-empty segments
+        auto load_item = [&](int idx) {
+            SharedItemCtx c;
+            c.idx = idx;
+            c.valid = idx < count;
+            c.f = c.valid && lane < 8 ? reinterpret_cast<const int *>(prm.items + idx)[lane] : 0;
+            c.mtok = 0;
+            c.mask = 0u;
+            if (!c.valid) return c;
+            const int pre = field(c, 1), first = field(c, 2), nseq = field(c, 3);
+            const int j = field(c, 5), npp = field(c, 6), nps2 = field(c, 7);
+            const int k = j - npp + (nps2 & 1);   // suffix partition of this item, if any
+            if (k >= 0 && k < (nps2 >> 1) && lane < nseq) {
+                const int len = clamp_len(prm.context_lens[first + lane], prm.max_context_len);
+                c.mtok = max(0, min(P, len - pre - k * P));
+            }
+            c.mask = (__ballot_sync(0xffffffffu, c.mtok > 0) << 1) | (j < npp ? 1u : 0u);
+            return c;
+        };
+        // segment sidx of item c (sidx < 0: the empty item's single stage of no tokens)
+        auto make_seg = [&](const SharedItemCtx &c, int sidx) {
+            SharedSeg g;
+            g.valid = c.valid;
+            g.sidx = sidx;
+            const int nseq = field(c, 3);
+            const int m = sidx - 1;
+            const int mt = __shfl_sync(0xffffffffu, c.mtok, max(m, 0));
+            if (sidx <= 0) {
+                const int j = field(c, 5), pre = field(c, 1);
+                g.seq = sidx == 0 ? field(c, 0) : field(c, 2);
+                g.tok0 = sidx == 0 ? j * P : 0;
+                g.ntok = sidx == 0 ? min(P, pre - j * P) : 0;
+                g.r0 = 0;
+                g.r1 = nseq * G;
+            } else {
+                const int j = field(c, 5), npp = field(c, 6), nps2 = field(c, 7);
+                g.seq = field(c, 2) + m;
+                g.tok0 = field(c, 1) + (j - npp + (nps2 & 1)) * P;
+                g.ntok = mt;
+                g.r0 = m * G;
+                g.r1 = (m + 1) * G;
+            }
+            const unsigned below = sidx <= 0 ? 0u : (c.mask & ((1u << sidx) - 1u));
+            const unsigned above = sidx < 0 ? 0u : (c.mask & ~((2u << sidx) - 1u));
+            g.first = below == 0u;
+            g.last = above == 0u;
+            return g;
+        };
+        auto first_seg = [&](const SharedItemCtx &c) {
+            return make_seg(c, c.mask ? __ffs(c.mask) - 1 : -1);
+        };
+        // a segment's slice of its block-table row: entry e in lane e % 32, register e / 32
+        auto load_entries = [&](const SharedSeg &g, int (&ent)[kMaxItemBlocks / 32]) {
+            const int nblk = g.valid ? (g.ntok + BS - 1) / BS : 0;
             const int32_t *bt =
-                prm.block_tables + (size_t)table_seq * prm.max_blocks_per_seq + tok0 / BS;
+                prm.block_tables + (size_t)(g.valid ? g.seq : 0) * prm.max_blocks_per_seq +
+                (g.valid ? g.tok0 / BS : 0);
 #pragma unroll
             for (int k = 0; k < kMaxItemBlocks / 32; ++k) {
                 const int e = k * 32 + lane;
                 ent[k] = e < nblk ? bt[e] : 0;
             }
         };
-        int cur_idx = take();
-        int cur_f = fetch(cur_idx);
+        int pending = take();
+        SharedItemCtx cur_item = load_item(__shfl_sync(0xffffffffu, pending, 0));
+        pending = take();
+        SharedSeg cur = first_seg(cur_item);
         int ent[kMaxItemBlocks / 32];
-        if (cur_idx < count) load_entries(cur_f, ent);
-        while (cur_idx < count && ok) {
-            const int ntok = __shfl_sync(0xffffffffu, cur_f, 2);
-            const int hk = __shfl_sync(0xffffffffu, cur_f, 3);
-            const int first_seq = __shfl_sync(0xffffffffu, cur_f, 4);
-            const int nseq = __shfl_sync(0xffffffffu, cur_f, 5);
-            const int part = __shfl_sync(0xffffffffu, cur_f, 6);
-            const int nst = max(1, (ntok + kStageTokens - 1) / kStageTokens);
-            int nxt_idx = 0, nxt_f = 0;
+        load_entries(cur, ent);
+        while (cur.valid && ok) {
+            const int hk = field(cur_item, 4);
+            const int first_seq = field(cur_item, 2);
+            const int nseq = field(cur_item, 3);
+            const int part = field(cur_item, 5);
+            const int nparts = chunk_parts(field(cur_item, 6), field(cur_item, 7));
+            const int nst = max(1, (cur.ntok + kStageTokens - 1) / kStageTokens);
+            SharedItemCtx nxt_item = cur_item;
+            SharedSeg nxt;
+            nxt.valid = false;
             int nxt_ent[kMaxItemBlocks / 32];
             for (int st = 0; st < nst; ++st, ++it) {
                 const int slot = it % L::kStages;
@@ -409,7 +494,7 @@ paged_decode_shared_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     ok = false;
                     break;
                 }
-                const int sntok = max(0, min(kStageTokens, ntok - st * kStageTokens));
+                const int sntok = max(0, min(kStageTokens, cur.ntok - st * kStageTokens));
                 const int nb_st = (sntok + BS - 1) / BS;
                 const int e0 = st * kBPS;
                 const int reg = e0 >> 5;
@@ -421,11 +506,12 @@ paged_decode_shared_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 const uint32_t bar = smem_u32(&full[slot]);
                 if (lane == 0) {
                     StageInfo in;
-                    in.s = first_seq; in.hk = hk; in.p = part; in.npart = nseq;
-                    in.item = cur_idx;
+                    in.s = first_seq; in.hk = hk; in.p = part; in.npart = nparts;
+                    in.item = nseq;
                     in.ntok = sntok;
-                    in.flags = (st == 0 ? kFirst : 0) | (st == nst - 1 ? kLast : 0);
-                    in.pad = 0;
+                    in.flags = (cur.first && st == 0 ? kFirst : 0) |
+                               (cur.last && st == nst - 1 ? kLast : 0);
+                    in.pad = cur.r0 | (cur.r1 << 16);
                     info[slot] = in;
                     mbar_arrive_expect_tx(bar, (uint32_t)(nb_st * BS * L::kRowBytes * 2));
                 }
@@ -451,14 +537,20 @@ paged_decode_shared_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     }
                 }
                 if (st == 0) {
-                    // the next item and its table slice, while this item's stages stream
-                    nxt_idx = take();
-                    nxt_f = fetch(nxt_idx);
-                    if (nxt_idx < count) load_entries(nxt_f, nxt_ent);
+                    // the next segment and its table slice, while this one streams
+                    if (!cur.last) {
+                        const unsigned above = cur_item.mask & ~((2u << cur.sidx) - 1u);
+                        nxt = make_seg(cur_item, __ffs(above) - 1);
+                    } else {
+                        nxt_item = load_item(__shfl_sync(0xffffffffu, pending, 0));
+                        if (nxt_item.valid) pending = take();
+                        nxt = first_seg(nxt_item);
+                    }
+                    load_entries(nxt, nxt_ent);
                 }
             }
-            cur_idx = nxt_idx;
-            cur_f = nxt_f;
+            cur = nxt;
+            cur_item = nxt_item;
 #pragma unroll
             for (int k = 0; k < kMaxItemBlocks / 32; ++k) ent[k] = nxt_ent[k];
         }
@@ -502,7 +594,7 @@ paged_decode_shared_kernel(const __grid_constant__ CUtensorMap tmap_k,
         }
         const StageInfo in = info[slot];
         if (in.flags & kEnd) break;
-        const int nrows = in.npart * G;
+        const int nrows = in.item * G;
 
         if (in.flags & kFirst) {
             // A fragments of the item's rows r = member * G + head (rows >= nrows are zero)
@@ -527,8 +619,9 @@ paged_decode_shared_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const int valid = in.ntok - 16 * w;
         if (valid > 0) {
             const uint8_t *stage = ring + slot * L::kStageBytes;
-            consume_stage<T, D, BS>(st, smem_u32(stage), smem_u32(stage + L::kKBytes), 16 * w,
-                                    lane, valid, prm.scale_log2);
+            consume_stage<T, D, BS, true>(st, smem_u32(stage), smem_u32(stage + L::kKBytes),
+                                          16 * w, lane, valid, prm.scale_log2, in.pad & 0xffff,
+                                          in.pad >> 16);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&empty[slot]));
@@ -536,23 +629,33 @@ paged_decode_shared_kernel(const __grid_constant__ CUtensorMap tmap_k,
         if (in.flags & kLast) {
             merge_warps<D>(st, nrows, obuf, L::kObufStride, ml, w, lane);
             const int tid = threadIdx.x;
-            for (int idx = tid; idx < nrows * D; idx += kConsumerWarps * 32) {
-                const int r = idx / D, dim = idx - r * D;
-                const int s = in.s + r / G, h = in.hk * G + r % G;
-                const size_t row = (size_t)prm.row_base[s] + (size_t)h * prm.np[s] + in.p;
-                prm.ws_o[row * D + dim] = obuf[r * L::kObufStride + dim];
-            }
-            if (tid < nrows) {
-                const int s = in.s + tid / G, h = in.hk * G + tid % G;
-                const size_t row = (size_t)prm.row_base[s] + (size_t)h * prm.np[s] + in.p;
-                reinterpret_cast<float2 *>(prm.ws_ml)[row] = row_stats(ml, tid);
+            if (in.npart == 1) {
+                // the chunk is this one item: final output
+                for (int idx = tid; idx < nrows * D; idx += kConsumerWarps * 32) {
+                    const int r = idx / D, dim = idx - r * D;
+                    const int s = in.s + r / G, h = in.hk * G + r % G;
+                    reinterpret_cast<T *>(prm.out)[((size_t)s * prm.num_heads + h) * D + dim] =
+                        from_float<T>(obuf[r * L::kObufStride + dim]);
+                }
+            } else {
+                for (int idx = tid; idx < nrows * D; idx += kConsumerWarps * 32) {
+                    const int r = idx / D, dim = idx - r * D;
+                    const int s = in.s + r / G, h = in.hk * G + r % G;
+                    const size_t row = (size_t)prm.row_base[s] + (size_t)h * prm.np[s] + in.p;
+                    prm.ws_o[row * D + dim] = obuf[r * L::kObufStride + dim];
+                }
+                if (tid < nrows) {
+                    const int s = in.s + tid / G, h = in.hk * G + tid % G;
+                    const size_t row = (size_t)prm.row_base[s] + (size_t)h * prm.np[s] + in.p;
+                    reinterpret_cast<float2 *>(prm.ws_ml)[row] = row_stats(ml, tid);
+                }
             }
         }
     }
 }
 
-// Merge of every (sequence, head)'s partials: rows row_base[s] + h*np[s] + j, j < np[s];
-// one warp per pair.
+// Merge of the partials of every (sequence, head) whose chunk was split into several
+// items: rows row_base[s] + h*np[s] + j, j < np[s]; one warp per pair.
 template <typename T, int D>
 __global__ void __launch_bounds__(kReduceWarps * 32)
 paged_decode_shared_reduce_kernel(SharedParams prm) {
@@ -568,6 +671,7 @@ paged_decode_shared_reduce_kernel(SharedParams prm) {
     const int s = pair / prm.num_heads;
     const int h = pair - s * prm.num_heads;
     const int np = prm.np[s];
+    if (np == 1) return;   // written by the decode kernel
     const size_t row0 = (size_t)prm.row_base[s] + (size_t)h * np;
     warp_merge<T, D>(reinterpret_cast<const float2 *>(prm.ws_ml) + row0, 1,
                      prm.ws_o + row0 * D, D, np,

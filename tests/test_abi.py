@@ -81,15 +81,15 @@ def test_pair_count_must_fit_an_int():
 
 def test_shared_prefix_auto_partition_choices():
     f = pkv.pkv_decode_shared_prefix_partition_size
-    assert f(128, 32, 8, 128, 16, 1300) == 1024        # G = 4: twice the plain path's 512
+    assert f(128, 32, 8, 128, 16, 1300) == 2048        # G = 4: prefix and suffixes in one item
     assert f(8, 64, 8, 128, 16, 131072) == 2048        # G = 8
-    assert f(128, 32, 8, 128, 8, 1300) == 1024         # 128 blocks of 8
+    assert f(128, 32, 8, 128, 8, 1300) == 2048         # 256 blocks of 8
     assert f(4, 8, 8, 64, 16, 128) == 64               # tiny batch: halved like the plain path
     assert f(128, 32, 8, 128, 16, 1300, 256) == 256    # an explicit size is kept
     with pytest.raises(pkv.PagedKVError):
         f(8, 64, 8, 128, 8, 131072, 4096)               # 512 blocks of 8
     assert pkv.pkv_decode_shared_prefix_workspace_size(128, 32, 8, 128, 16, 1300) == \
-        pkv.pkv_decode_shared_prefix_workspace_size(128, 32, 8, 128, 16, 1300, 1024)
+        pkv.pkv_decode_shared_prefix_workspace_size(128, 32, 8, 128, 16, 1300, 2048)
 
 
 def test_decode_rejects_bad_args_without_a_device():

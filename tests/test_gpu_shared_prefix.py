@@ -236,3 +236,63 @@ def test_planned_call_with_other_sizes_writes_nothing(cuda_device):
                                                          ws, partition_size=64)
     assert pkv.pkv_get_device_status() & pkv._binding.STATUS_WORKSPACE
     assert (out == 3.0).all()
+
+
+def explicit_case(rng, groups, Hq, Hkv, D, BS, dtype):
+    """groups: (prefix tokens, [suffix tokens of each member]); members share the
+    prefix's pages. Unwritten rows hold the NaN canary."""
+    tables, lens, starts, pre = [], [], [0], []
+    page = 0
+    for ptok, sufs in groups:
+        assert ptok % BS == 0
+        shared = list(range(page, page + ptok // BS))
+        page += ptok // BS
+        for suf in sufs:
+            own = -(-suf // BS)
+            tables.append(shared + list(range(page, page + own)))
+            page += own
+            lens.append(ptok + suf)
+        starts.append(starts[-1] + len(sufs))
+        pre.append(ptok)
+    nb = page + 2
+    relabel = rng.permutation(nb)
+    mb = max(1, max(len(t) for t in tables)) + 1
+    bt = np.full((len(tables), mb), -1, np.int32)
+    for s, t in enumerate(tables):
+        bt[s, :len(t)] = relabel[t]
+    lens = np.array(lens, np.int32)
+    kc = synth.round_to_bits(rng.standard_normal((nb, Hkv, BS, D), dtype=np.float32), dtype)
+    vc = synth.round_to_bits(rng.standard_normal((nb, Hkv, BS, D), dtype=np.float32), dtype)
+    used = np.zeros((nb, BS), bool)
+    for s, n in enumerate(lens):
+        for t in range(int(n)):
+            used[bt[s, t // BS], t % BS] = True
+    kc.transpose(0, 2, 1, 3)[~used] = synth.CANARY[dtype]
+    vc.transpose(0, 2, 1, 3)[~used] = synth.CANARY[dtype]
+    q = synth.round_to_bits(rng.standard_normal((len(lens), Hq, D), dtype=np.float32), dtype)
+    return (q, kc, vc, bt, lens, np.array(starts, np.int32), np.array(pre, np.int32),
+            mb * BS)
+
+
+@pytest.mark.parametrize("Hq,Hkv,BS", [(32, 8, 16), (16, 2, 32), (8, 8, 8)])
+def test_chunks_fused_split_and_empty(cuda_device, Hq, Hkv, BS):
+    """Chunks whose prefix and suffixes form one item (written directly) next to chunks
+    split into several items (merged): members with no suffix, suffixes longer than a
+    partition, a group whose members hold nothing at all, and groups of one; each at the
+    automatic partition and at small ones."""
+    rng = np.random.default_rng(Hq + Hkv + BS)
+    dtype = synth.F16
+    groups = [(64 * BS, [0, 3, 0, 700, 1, 0, 65, 64, 2]),   # mixed suffixes, some none
+              (0, [0, 0, 0]),                                  # empty contexts
+              (2 * BS, [1]),                                   # a group of one
+              (0, [900]),
+              (10 * BS, [0, 0]),                               # the prefix is everything
+              (5 * BS, [130, 2, 2500, 17])]
+    q, kc, vc, bt, lens, starts, pre, max_len = explicit_case(rng, groups, Hq, Hkv, 128, BS,
+                                                              dtype)
+    ref = A.paged_decode_attention(q, kc, vc, bt, lens, 0.09, dtype)
+    pkv.pkv_get_device_status(clear=True)
+    for partition in (0, 256, 64):
+        got = run_shared(q, kc, vc, bt, lens, starts, pre, max_len, dtype, 0.09, partition)
+        assert_close(got, ref, dtype, f"P={partition}")
+    assert pkv.pkv_get_device_status() == 0
