@@ -541,7 +541,7 @@ def gpu_arm(args, rank, world, local_rank, light=False):
         launches_per_layer = pkv.pkv_decode_step_launches(
             B, sp.num_heads, sp.num_kv_heads, sp.head_dim, sp.block_size, max_len, P)
         launches_per_step = L * launches_per_layer
-        kernel_key = ("paged_decode_partition_write" if launches_per_layer > 1
+        kernel_key = ("paged_decode_partition_write" if launches_per_layer > 1 or pmax == 1
                       else "paged_decode_step")
     else:
         launches_per_layer = 3 if shared else 2 + (1 if pmax > 1 else 0)
@@ -629,6 +629,7 @@ def gpu_arm(args, rank, world, local_rank, light=False):
     traffic = None if shared else read_traffic(args.workload, sp.block_size, kernel_key)
     if fused:
         call_desc = ("write-and-decode kernel + merge kernel" if launches_per_layer > 1 else
+                     "write-and-decode kernel (one partition per context)" if pmax == 1 else
                      "step kernel (cache write, decode and merge in one launch)")
     else:
         call_desc = ("plan (one per step) + shared-prefix decode + merge" if shared else

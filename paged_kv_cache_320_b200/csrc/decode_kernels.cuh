@@ -232,7 +232,10 @@ struct ItemWalker {
 // canonical item number (sequence-major, as ItemWalker numbers them), which indexes
 // the partials.
 constexpr int kMaxStageCount = kMaxItemBlocks * 32 / kStageTokens;   // P <= 256 blocks of 32
-constexpr int kOrderMaxSeqs = 32;   // longest-first order up to this batch size
+#ifndef PKV_ORDER_MAX_SEQS
+#define PKV_ORDER_MAX_SEQS 64
+#endif
+constexpr int kOrderMaxSeqs = PKV_ORDER_MAX_SEQS;   // longest-first order up to this batch size
 
 __device__ __forceinline__ int clamp_ctx(int len, const DecodeParams &prm, bool flag) {
     if (len < 0 || len > prm.max_context_len) {
@@ -861,19 +864,29 @@ __device__ __forceinline__ void decode_items(const CUtensorMap *tmap_k, const CU
     }
 }
 
-// Whether this launch takes its items from the workspace counter: the header is armed.
-// Read by every CTA before it changes anything; `armed` is written again only by the
-// last CTA out (sched_exit), so every CTA of a launch decides alike.
-__device__ __forceinline__ bool sched_is_armed(const DecodeParams &prm, int *flag) {
-    if (threadIdx.x == 0)
-        *flag = prm.sched != nullptr && *(volatile unsigned *)&prm.sched->armed == kSchedArmed;
+// How a launch uses the workspace header: kSchedDynamic when it is armed (items from the
+// counter, the last CTA out re-arms it); kSchedArmZero when it is zero and the caller
+// guarantees a zero-filled workspace (static schedule, and the last CTA out arms it);
+// kSchedStatic otherwise. Read by every CTA before it changes anything; `armed` is
+// written again only by the last CTA out (sched_exit), so every CTA decides alike.
+constexpr int kSchedStatic = 0, kSchedDynamic = 1, kSchedArmZero = 2;
+__device__ __forceinline__ int sched_mode(const DecodeParams &prm, bool zero_filled, int *flag) {
+    if (threadIdx.x == 0) {
+        int m = kSchedStatic;
+        if (prm.sched != nullptr) {
+            const unsigned a = *(volatile unsigned *)&prm.sched->armed;
+            m = a == kSchedArmed ? kSchedDynamic : (zero_filled && a == 0u ? kSchedArmZero
+                                                                           : kSchedStatic);
+        }
+        *flag = m;
+    }
     __syncthreads();
-    return *flag != 0;
+    return *flag;
 }
 
-// End of a dynamically scheduled launch: the last CTA out re-arms the header (counter
-// and step counters 0), so the next launch on the workspace may run without a merge
-// kernel in between. Every CTA of the launch calls it (all threads).
+// End of a launch that found the header armed or zero: the last CTA out (re-)arms it
+// (counter and step counters 0), so the next launch on the workspace may run without a
+// merge kernel in between. Every CTA of the launch calls it (all threads).
 __device__ __forceinline__ void sched_exit(SchedHeader *h) {
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -894,13 +907,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
 paged_decode_partition_kernel(const __grid_constant__ CUtensorMap tmap_k,
                               const __grid_constant__ CUtensorMap tmap_v,
                               const __grid_constant__ CUtensorMap tmap_q, DecodeParams prm) {
-    __shared__ int s_dyn;
+    __shared__ int s_mode;
     DecodeSmem<D> sm(aligned_dynamic_smem(), prm.group);
     sm.init_barriers();
     pdl_wait_and_release();
-    const bool dyn = sched_is_armed(prm, &s_dyn);
-    decode_items<T, D, BS, false>(&tmap_k, &tmap_v, &tmap_q, prm, sm, dyn);
-    if (*(volatile int *)&s_dyn) sched_exit(prm.sched);   // reread: nothing held across the loop
+    const int mode = sched_mode(prm, false, &s_mode);   // a decode workspace may hold anything
+    decode_items<T, D, BS, false>(&tmap_k, &tmap_v, &tmap_q, prm, sm, mode == kSchedDynamic);
+    // reread: nothing held across the loop
+    if (*(volatile int *)&s_mode != kSchedStatic) sched_exit(prm.sched);
 }
 
 // The same with the decode step's cache write (each sequence's newest token written by
@@ -911,13 +925,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
 paged_decode_partition_write_kernel(const __grid_constant__ CUtensorMap tmap_k,
                                     const __grid_constant__ CUtensorMap tmap_v,
                                     const __grid_constant__ CUtensorMap tmap_q, DecodeParams prm) {
-    __shared__ int s_dyn;
+    __shared__ int s_mode;
     DecodeSmem<D> sm(aligned_dynamic_smem(), prm.group);
     sm.init_barriers();
     pdl_wait_and_release();
-    const bool dyn = sched_is_armed(prm, &s_dyn);
-    decode_items<T, D, BS, true>(&tmap_k, &tmap_v, &tmap_q, prm, sm, dyn);
-    if (*(volatile int *)&s_dyn) sched_exit(prm.sched);   // reread: nothing held across the loop
+    const int mode = sched_mode(prm, true, &s_mode);    // a step workspace starts zero-filled
+    decode_items<T, D, BS, true>(&tmap_k, &tmap_v, &tmap_q, prm, sm, mode == kSchedDynamic);
+    // reread: nothing held across the loop
+    if (*(volatile int *)&s_mode != kSchedStatic) sched_exit(prm.sched);
 }
 
 // Log-sum-exp merge of n partials (m_j in log2 units, l_j, normalised o_j) of one

@@ -166,12 +166,18 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 int cdiv(int a, int b) { return (a + b - 1) / b; }
 
-// Automatic partition size: 512 tokens for GQA groups up to 4 and 2048 above (the
-// fp32 partials grow with the group; measured best at the GQA-4 and GQA-8 workloads),
-// at most 256 blocks, halved while the batch offers fewer than 1024 work items (about
-// 7 per CTA on 148 SMs).
+// Automatic partition size. One partition per context (no partials, no merge) when
+// every context fits one work item (256 blocks), the batch is small enough for the
+// longest-first item order (so the long items start first and the launch drains on
+// short ones) and offers at least 1024 items. Otherwise 512 tokens for GQA groups up to 4
+// and 2048 above (the fp32 partials grow with the group; measured best at the GQA-4 and
+// GQA-8 workloads), at most 256 blocks, halved while the batch offers fewer than 1024
+// work items (about 7 per CTA on 148 SMs).
 int auto_partition(int B, int Hq, int Hkv, int BS, int max_len) {
     const int G = Hq / Hkv;
+    if (max_len <= pkv::kMaxItemBlocks * BS && B <= pkv::kOrderMaxSeqs &&
+        (long long)B * Hkv >= 1024)
+        return std::max(pkv::kStageTokens, cdiv(max_len, pkv::kStageTokens) * pkv::kStageTokens);
     int p = G <= 4 ? 512 : 2048;
     if (p > pkv::kMaxItemBlocks * BS) p = pkv::kMaxItemBlocks * BS;
     while (p > 64 && (long long)B * Hkv * cdiv(max_len, p) < 1024) p /= 2;
@@ -499,10 +505,9 @@ int dispatch_step(int BS, const CUtensorMap &mk, const CUtensorMap &mv, const CU
         }
         return PKV_ERR_INVALID_ARG;
     }
-    // the work counter is used only when some context spans several partitions (the
-    // merge kernel then arms the header; with one partition per context nothing would)
-    pkv::DecodeParams p = prm;
-    if (!merge) p.sched = nullptr;
+    // the header (zero-filled at first, then armed by the last CTA out of each launch)
+    // holds the work counter whether or not the contexts span several partitions
+    const pkv::DecodeParams &p = prm;
     int rc = PKV_ERR_INVALID_ARG;
     switch (BS) {
         case 8: rc = launch_decode<T, D, 8, true>(mk, mv, mq, p, items, st); break;

@@ -70,6 +70,11 @@ def test_auto_partition_choices():
     with pytest.raises(pkv.PagedKVError):
         pkv.pkv_decode_partition_size(8, 64, 8, 128, 8, 131072, 4096)            # 512 of 8
     assert pkv.pkv_decode_partition_size(4, 8, 8, 64, 16, 128) == 64          # tiny batch
+    # every context one item: at most 64 sequences (longest-first order), >= 1024 items
+    assert pkv.pkv_decode_partition_size(64, 32, 32, 128, 16, 2100) == 2112
+    assert pkv.pkv_decode_partition_size(64, 32, 32, 128, 16, 4097) == 512    # > 256 blocks
+    assert pkv.pkv_decode_partition_size(65, 32, 32, 128, 16, 2100) == 512    # > 64 sequences
+    assert pkv.pkv_decode_partition_size(31, 32, 32, 128, 16, 2100) == 512    # < 1024 items
 
 
 def test_pair_count_must_fit_an_int():
