@@ -476,6 +476,7 @@ def gpu_arm(args, rank, world, local_rank, light=False):
     outs = [torch.empty_like(wl.q[l]) for l in range(L)]
     stream = torch.cuda.current_stream(dev)
     kv_layer, roof_layer = algorithmic_bytes(wl)
+    roof_layer_all = roof_layer
     kv_step = kv_layer * L
     shared = args.decode == "shared"
     if shared:
@@ -657,7 +658,8 @@ def gpu_arm(args, rank, world, local_rank, light=False):
         roofline["merge_kernel_us"] = round(merge_us, 2)
     if light:
         return {
-            "workload": args.workload, "block_size": sp.block_size, "layers": L,
+            "workload": args.workload, "decode": args.decode, "block_size": sp.block_size,
+            "layers": L,
             "num_seqs": B, "num_heads": sp.num_heads, "num_kv_heads": sp.num_kv_heads,
             "dtype": synth.DTYPE_NAMES[sp.dtype], "partition_size": P,
             "sum_context_tokens": int(wl.context_lens.sum()), "kv_bytes_per_step": kv_step,
@@ -665,6 +667,12 @@ def gpu_arm(args, rank, world, local_rank, light=False):
             "pct_of_hbm_peak": round(100 * value / world / peak, 2),
             "tokens_per_s": round(tokens_per_s, 1),
             "launches_per_layer": launches_per_layer,
+            **({"unique_kv_bytes_per_step": (roof_layer - (roof_layer_all - kv_layer)) * L,
+                "value_unique": round((roof_layer - (roof_layer_all - kv_layer)) * L * world
+                                      / (ms_step * 1e-3) / 1e9, 1),
+                "note": "value counts logical K/V bytes (every sequence's whole context); the "
+                        "roofline counts the bytes the path must read (each shared prefix once "
+                        "per KV head, every private suffix)"} if shared else {}),
             "eager": {"value": round(eager_value, 1), "ms_per_step": round(ms["eager"], 4)},
             "roofline": roofline, "clocks": clocks.summary()}
 
@@ -709,6 +717,8 @@ def gpu_arm(args, rank, world, local_rank, light=False):
         "tokens_per_s": round(tokens_per_s, 1),
         "pct_of_hbm_peak": round(100 * value / world / peak, 2),
         "pct_of_nominal_8tbs": round(100 * value / world / 8000.0, 2),
+        **({"value_unique": round((roof_layer - (roof_layer_all - kv_layer)) * L * world
+                                  / (ms_step * 1e-3) / 1e9, 1)} if shared else {}),
         "memory_utilisation": memory,
         "eager": {"value": round(eager_value, 1), "unit": "GB/s",
                   "ms_per_step": round(ms["eager"], 4),
@@ -1184,22 +1194,27 @@ def reference_arm(args, rank):
     }
 
 
-CONFIG_WORKLOADS = [("llama3_8b_gqa", 16), ("long_context", 8), ("long_context", 16),
-                    ("long_context", 32)]
+# (workload, block size, decode, layers): the Llama-3-8B-shaped GQA and long-context
+# workloads with the plain decode, and the shared-prefix workload with the shared-prefix-aware
+# decode over 8 layers (one plan per step serves them all)
+CONFIG_WORKLOADS = [("llama3_8b_gqa", 16, "plain", 0), ("long_context", 8, "plain", 0),
+                    ("long_context", 16, "plain", 0), ("long_context", 32, "plain", 0),
+                    ("shared_prefix", 16, "shared", 8)]
 
 
 def run_configs(args, local_rank):
-    """The other decode workloads at their own sizes (Llama-3-8B-shaped GQA; long context at
-    block sizes 8, 16 and 32), each timed like the headline workload: the fused step as CUDA
-    graph replays, `steps` timed after `warmup`, its dominant kernel alone, clocks sampled
-    during its timed region."""
+    """The other decode workloads at their own sizes, each timed like the headline
+    workload: the step as CUDA graph replays, `steps` timed after `warmup`, its dominant
+    kernel alone, clocks sampled during its timed region."""
     import torch
     out = {}
-    for workload, bs in CONFIG_WORKLOADS:
+    for workload, bs, decode, layers in CONFIG_WORKLOADS:
         sub = argparse.Namespace(**vars(args))
-        sub.workload, sub.block_size, sub.layers, sub.batch = workload, bs, 0, 0
-        sub.decode, sub.swap, sub.prefix_cache, sub.partition = "plain", False, False, 0
-        out[f"{workload}_bs{bs}"] = gpu_arm(sub, 0, 1, local_rank, light=True)
+        sub.workload, sub.block_size, sub.layers, sub.batch = workload, bs, layers, 0
+        sub.decode, sub.swap, sub.prefix_cache, sub.partition = decode, False, False, 0
+        key = f"{workload}_bs{bs}" + (f"_{decode}_decode_{layers}_layers" if decode != "plain"
+                                      else "")
+        out[key] = gpu_arm(sub, 0, 1, local_rank, light=True)
         torch.cuda.empty_cache()
     return out
 
