@@ -293,7 +293,7 @@ int dispatch_bs(int BS, const CUtensorMap &mk, const CUtensorMap &mv, const CUte
 }
 
 // ---- shared-prefix decode ------------------------------------------------
-// Workspace: [counters 256 B][np, row_base, seq_group, gpre, gmin, gmis, ioff, pbase: B ints each]
+// Workspace: [counters 256 B][np, row_base, seq_group, gpre, gmin, gmis, ioff: B ints each]
 // [chunk completion counters: B x Hkv ints][items][partials (max, sum)][partial outputs].
 struct SharedWs {
     size_t ints, done, items, ml, o, total;
@@ -307,7 +307,7 @@ SharedWs shared_ws_layout(int B, int Hq, int Hkv, int D, int max_len, int P) {
     w.max_items = (int)std::min<long long>(2LL * Hkv * B * pmax, INT_MAX / 2);
     w.rows = (long long)B * Hq * (pmax + 1);
     w.ints = sizeof(pkv::SharedCounters);
-    w.done = w.ints + 8 * align_up((size_t)B * sizeof(int), 256);
+    w.done = w.ints + 7 * align_up((size_t)B * sizeof(int), 256);
     w.items = w.done + align_up((size_t)B * Hkv * sizeof(int), 256);
     w.ml = w.items + align_up((size_t)w.max_items * sizeof(pkv::SharedItem), 256);
     w.o = w.ml + align_up((size_t)w.rows * 2 * sizeof(float), 256);
@@ -348,7 +348,7 @@ int launch_shared_decode(const CUtensorMap &mk, const CUtensorMap &mv,
 
 int launch_shared_plan(const pkv::SharedParams &prm, cudaStream_t st) {
     const size_t plan_smem =
-        prm.num_seqs <= pkv::kPlanSmemSeqs ? (size_t)8 * prm.num_seqs * sizeof(int) : 0;
+        prm.num_seqs <= pkv::kPlanSmemSeqs ? (size_t)7 * prm.num_seqs * sizeof(int) : 0;
     {
         int dev;
         if (current_device(&dev) != PKV_OK) return PKV_ERR_CUDA;
@@ -357,7 +357,7 @@ int launch_shared_plan(const pkv::SharedParams &prm, cudaStream_t st) {
         if (!attr[dev]) {
             if (cudaFuncSetAttribute(pkv::shared_prefix_plan_kernel,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     8 * pkv::kPlanSmemSeqs * (int)sizeof(int)) != cudaSuccess)
+                                     7 * pkv::kPlanSmemSeqs * (int)sizeof(int)) != cudaSuccess)
                 return PKV_ERR_CUDA;
             attr[dev] = true;
         }
@@ -394,7 +394,6 @@ pkv::SharedParams shared_params(const SharedWs &ws, void *workspace, int num_seq
     prm.gmin = reinterpret_cast<int *>(wsb + ws.ints + 4 * ib);
     prm.gmis = reinterpret_cast<int *>(wsb + ws.ints + 5 * ib);
     prm.ioff = reinterpret_cast<int *>(wsb + ws.ints + 6 * ib);
-    prm.pbase = reinterpret_cast<int *>(wsb + ws.ints + 7 * ib);
     prm.chunk_done = reinterpret_cast<int *>(wsb + ws.done);
     prm.items = reinterpret_cast<pkv::SharedItem *>(wsb + ws.items);
     prm.ws_ml = reinterpret_cast<float *>(wsb + ws.ml);

@@ -17,15 +17,16 @@
 // runs the items with the same TMA / mbarrier / tensor-core pipeline as plain decode;
 // the reduce merges the partials of the (sequence, head) pairs whose work was split.
 //
-// Work items. A prefix item streams one partition (P tokens) of a group's shared prefix,
-// once for up to 32 query rows (the G heads of 32 / G members: two MMA row tiles, one per
-// warp pair, each warp taking half of every 64-token stage); the group's members are
-// taken 32 / G at a time. A suffix item streams suffix partition k of up to 16 / G
-// members (a "chunk", 16 rows): every member's own tokens [pre + kP, pre + (k+1)P), in
-// one segment per member during which only that member's G rows attend. Every (sequence,
-// head) thus has np = (prefix partitions) + (its chunk's suffix partitions) partials; when
-// np is 1 the item writes the output directly, otherwise each item leaves its partial and
-// the last item of the chunk to finish (per KV head) merges them (log-sum-exp).
+// Work items. The members of a group are taken R = 16 / G at a time ("chunks", 16 query
+// rows). A chunk's tokens are its prefix, cut into partitions of P tokens, and its
+// members' suffixes, cut into partitions of P tokens per member (suffix partition k of a
+// chunk holds every member's tokens [pre + kP, pre + (k+1)P)). An item is one of them
+// for one KV head, or the last prefix partition and the first suffix partition
+// together when their 64-token stages fit in one partition's budget. The item's stages
+// come in segments (the prefix pages, then each member's own pages); during a member's
+// segment only that member's G rows attend. A chunk that is one item writes its output
+// directly; otherwise each item leaves one partial per row (empty for rows it did not
+// touch) for the reduce.
 #pragma once
 
 #include "decode_kernels.cuh"
@@ -38,10 +39,16 @@ struct SharedItem {
     int first_seq;   // query rows: sequences first_seq .. first_seq + nseq - 1, G heads each
     int nseq;
     int hk;          // KV head
-    int part;        // the partials' index: j for prefix partition j, npp + k for suffix k
-    int k;           // prefix partition j, or suffix partition k
-    int prefix;      // 1: a prefix item (up to 32 rows), 0: a suffix item (up to 16 rows)
+    int part;        // index of this item among its chunk's items (its partials' index)
+    int npp;         // prefix partitions of the chunk
+    int nps2;        // 2 x suffix partitions of the chunk, + 1 if the last prefix partition
+                     // and the first suffix partition are one item
 };
+
+// Items of a chunk: prefix partitions, then suffix partitions, one fewer if fused.
+__host__ __device__ __forceinline__ int chunk_parts(int npp, int nps2) {
+    return npp + (nps2 >> 1) - (nps2 & 1);
+}
 
 struct SharedCounters {
     unsigned next;    // next work item (0 after the plan and after every decode launch)
@@ -74,8 +81,7 @@ struct SharedParams {
     int *gmin;         // [B] shortest member, then first chunk, per group (plan scratch)
     int *gmis;         // [B] first block where a member's table differs per group, then
                        //     first item per chunk (plan scratch)
-    int *ioff;         // [B] suffix partitions per chunk (plan scratch)
-    int *pbase;        // [B] first prefix item per group (plan scratch)
+    int *ioff;         // [B] 2 x suffix partitions + fused, per chunk (plan scratch)
     int *chunk_done;   // [B][Hkv] items of a split chunk finished, by first member (0 between
                        //          launches: the plan zeroes them, the chunk's merger resets)
     float *ws_o;       // [rows][D]
@@ -127,7 +133,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *sm, int *total) 
 }
 
 // Per-sequence scratch arrays of the plan kept in shared memory up to this batch size
-// (8 ints per sequence); larger batches use the workspace copies.
+// (7 ints per sequence); larger batches use the workspace copies.
 constexpr int kPlanSmemSeqs = 6144;
 
 // Largest i in [0, n) with off[i] <= x (off ascending, off[0] = 0).
@@ -153,8 +159,7 @@ shared_prefix_plan_kernel(SharedParams p) {
     __shared__ int bad, max_pre_blocks;
     const int B = p.num_seqs, Hkv = p.num_kv_heads, G = p.group, P = p.partition;
     const int BS = p.block_size;
-    const int R = kMaxGroup / G;       // members per suffix chunk (16 rows)
-    const int R2 = 2 * R;              // members per prefix item (two chunks, <= 32 rows)
+    const int R = kMaxGroup / G;   // member sequences per 16-row prefix item
     const int tid = threadIdx.x;
     // scratch: in shared memory when it fits (generic pointers address either space)
     const bool in_smem = B <= kPlanSmemSeqs;
@@ -165,7 +170,6 @@ shared_prefix_plan_kernel(SharedParams p) {
     int *slen = in_smem ? plan_smem + 4 * B : p.np;          // clamped lengths
     int *gfirst = in_smem ? plan_smem + 5 * B : p.row_base;  // first member of each group
     int *ioff = in_smem ? plan_smem + 6 * B : p.ioff;        // per-chunk partition counts
-    int *pbase = in_smem ? plan_smem + 7 * B : p.pbase;      // per-group prefix items
     for (int i = tid; i < B * Hkv; i += kPlanThreads) p.chunk_done[i] = 0;
     if (tid == 0) {
         bad = 0;
@@ -226,12 +230,12 @@ shared_prefix_plan_kernel(SharedParams p) {
         if (mis != 0x7fffffff) atomicMin(&gmis[g], mis);
     }
     __syncthreads();
-    // pass 3 (per group): shared length; suffix chunks of R members (first chunk of each
-    // group); prefix items (first of each group)
-    int n_chunks = 0, n_prefix = 0;
+    // pass 3 (per group): shared length; chunks of R members; first chunk of each group
+    const int S = P / kStageTokens;   // 64-token stages per partition
+    int n_chunks = 0;
     for (int g0 = 0; g0 < ng; g0 += kPlanThreads) {
         const int g = g0 + tid;
-        int cnt = 0, pcnt = 0;
+        int cnt = 0;
         if (g < ng) {
             const int first = gfirst[g];
             const int last = bad ? g + 1 : p.group_start[g + 1];
@@ -240,24 +244,18 @@ shared_prefix_plan_kernel(SharedParams p) {
             pre = min(pre, min(gmis[g], pre / BS) * BS);
             gpre[g] = pre;
             cnt = (last - first + R - 1) / R;
-            pcnt = pre > 0 ? Hkv * ((pre + P - 1) / P) * ((last - first + R2 - 1) / R2) : 0;
         }
-        int total, ptotal;
+        int total;
         const int at = n_chunks + block_exclusive_scan(cnt, sm, &total);
-        const int pat = n_prefix + block_exclusive_scan(pcnt, sm, &ptotal);
-        if (g < ng) {
-            gmin[g] = at;    // first chunk of group g (only thread g reads gmin[g] here)
-            pbase[g] = pat;
-        }
+        if (g < ng) gmin[g] = at;   // first chunk of group g (only thread g reads gmin[g] here)
         n_chunks += total;
-        n_prefix += ptotal;
     }
     int *chunk_base = gmin;
     int *item_base = gmis;    // per chunk (n_chunks <= B)
-    int *chunk_nps = ioff;    // per chunk
+    int *chunk_nps2 = ioff;   // per chunk
     __syncthreads();
-    // pass 4 (per chunk): suffix partitions (the most any member needs), first suffix item
-    int n_items = n_prefix;
+    // pass 4 (per chunk): prefix and suffix partitions, fusion, first item
+    int n_items = 0;
     for (int c0 = 0; c0 < n_chunks; c0 += kPlanThreads) {
         const int ch = c0 + tid;
         int cnt = 0;
@@ -267,12 +265,18 @@ shared_prefix_plan_kernel(SharedParams p) {
             const int last = bad ? g + 1 : p.group_start[g + 1];
             const int nseq = min(R, last - first);
             const int pre = gpre[g];
-            int nps = 0;
-            for (int m = 0; m < nseq; ++m)   // >= 0: pre <= the shortest member
-                nps = max(nps, (slen[first + m] - pre + P - 1) / P);
-            if (pre == 0 && nps == 0) nps = 1;   // empty contexts: one item writes zeros
-            chunk_nps[ch] = nps;
-            cnt = Hkv * nps;
+            const int npp = (pre + P - 1) / P;
+            int nps = 0, st0 = 0;
+            for (int m = 0; m < nseq; ++m) {
+                const int suf = slen[first + m] - pre;   // >= 0: pre <= the shortest member
+                nps = max(nps, (suf + P - 1) / P);
+                st0 += (min(P, suf) + kStageTokens - 1) / kStageTokens;
+            }
+            if (npp == 0 && nps == 0) nps = 1;   // empty contexts: one item writes zeros
+            const int pre_last = npp ? (pre - (npp - 1) * P + kStageTokens - 1) / kStageTokens : 0;
+            const int fuse = npp > 0 && nps > 0 && pre_last + st0 <= S;
+            chunk_nps2[ch] = 2 * nps + fuse;
+            cnt = Hkv * chunk_parts(npp, 2 * nps + fuse);
         }
         int total;
         const int at = n_items + block_exclusive_scan(cnt, sm, &total);
@@ -280,58 +284,36 @@ shared_prefix_plan_kernel(SharedParams p) {
         n_items += total;
     }
     __syncthreads();
-    // pass 5a (per prefix item): group, KV head, member chunk of R2, prefix partition
-    for (int i = tid; i < n_prefix && i < p.max_items; i += kPlanThreads) {
-        const int g = owner_of(pbase, ng, i);
-        const int first = gfirst[g];
-        const int last = bad ? g + 1 : p.group_start[g + 1];
-        const int pre = gpre[g];
-        const int npp = (pre + P - 1) / P;
-        const int npc = (last - first + R2 - 1) / R2;
-        int local = i - pbase[g];
-        const int j = local % npp;
-        local /= npp;
-        const int pc = local % npc;
-        SharedItem it;
-        it.table_seq = first;
-        it.pre = pre;
-        it.first_seq = first + pc * R2;
-        it.nseq = min(R2, last - it.first_seq);
-        it.hk = local / npc;
-        it.part = j;
-        it.k = j;
-        it.prefix = 1;
-        p.items[i] = it;
-    }
-    // pass 5b (per suffix item): chunk, KV head, suffix partition
-    for (int i = n_prefix + tid; i < n_items && i < p.max_items; i += kPlanThreads) {
+    // pass 5 (per item): chunk, KV head and part
+    for (int i = tid; i < n_items && i < p.max_items; i += kPlanThreads) {
         const int ch = owner_of(item_base, n_chunks, i);
         const int g = owner_of(chunk_base, ng, ch);
         const int first = gfirst[g] + (ch - chunk_base[g]) * R;
         const int last = bad ? g + 1 : p.group_start[g + 1];
         const int pre = gpre[g];
-        const int nps = chunk_nps[ch];
+        const int npp = (pre + P - 1) / P;
+        const int nps2 = chunk_nps2[ch];
+        const int np = chunk_parts(npp, nps2);
         const int local = i - item_base[ch];
         SharedItem it;
         it.table_seq = gfirst[g];
         it.pre = pre;
         it.first_seq = first;
         it.nseq = min(R, last - first);
-        it.hk = local / nps;
-        it.k = local - it.hk * nps;
-        it.part = (pre + P - 1) / P + it.k;
-        it.prefix = 0;
+        it.hk = local / np;
+        it.part = local - it.hk * np;
+        it.npp = npp;
+        it.nps2 = nps2;
         p.items[i] = it;
     }
     __syncthreads();
-    // pass 6 (per sequence): partials per (sequence, head) = prefix partitions + its chunk's
-    // suffix partitions, then the scratch rows. slen becomes the partial count (in the
-    // workspace it is p.np itself), and row_base may overwrite gfirst only once every count
-    // is known.
+    // pass 6 (per sequence): partials per (sequence, head) = its chunk's items, then the
+    // scratch rows. slen becomes the partial count (in the workspace it is p.np itself),
+    // and row_base may overwrite gfirst only once every count is known.
     for (int s = tid; s < B; s += kPlanThreads) {
         const int g = seq_group[s];
         const int ch = chunk_base[g] + (s - gfirst[g]) / R;
-        slen[s] = (gpre[g] + P - 1) / P + chunk_nps[ch];
+        slen[s] = chunk_parts((gpre[g] + P - 1) / P, chunk_nps2[ch]);
     }
     __syncthreads();
     int base_rows = 0;
@@ -356,215 +338,6 @@ shared_prefix_plan_kernel(SharedParams p) {
     }
 }
 
-constexpr int kWide = 8;   // StageInfo flag: a 32-row item (two row tiles, one per warp pair)
-
-// End of a 32-row item: warps 2t and 2t+1 hold row tile t (rows 16t .. 16t + 15), each
-// for its half of every stage. Combines each pair's states and hands tile t's normalised
-// rows to emit(t, obuf) one tile at a time (the 16-row obuf is reused); the pair's (m, l)
-// per row stay in ml[warp * 16 + row]. All 128 consumer threads call it.
-template <int D, class Emit>
-__device__ __forceinline__ void merge_warp_pairs(WarpState<D> &st, float *obuf, int obuf_stride,
-                                                 float2 *ml, int w, int lane, Emit &&emit) {
-    constexpr int NT = D / 8;
-    const int gid = lane >> 2;
-    const int tig = lane & 3;
-    float lt0 = st.l0 + __shfl_xor_sync(0xffffffffu, st.l0, 1);
-    lt0 += __shfl_xor_sync(0xffffffffu, lt0, 2);
-    float lt1 = st.l1 + __shfl_xor_sync(0xffffffffu, st.l1, 1);
-    lt1 += __shfl_xor_sync(0xffffffffu, lt1, 2);
-    named_bar_sync(1, kConsumerWarps * 32);
-    if (tig == 0) {
-        ml[w * kMaxGroup + gid] = make_float2(st.m0, lt0);
-        ml[w * kMaxGroup + gid + 8] = make_float2(st.m1, lt1);
-    }
-    named_bar_sync(1, kConsumerWarps * 32);
-    const int partner = w ^ 1;
-    float fr[2];
-#pragma unroll
-    for (int rr = 0; rr < 2; ++rr) {
-        const int row = gid + 8 * rr;
-        const float2 a = ml[w * kMaxGroup + row], b = ml[partner * kMaxGroup + row];
-        const float M = fmaxf(a.x, b.x);
-        const float Lsum = M == -INFINITY ? 0.f : a.y * ex2(a.x - M) + b.y * ex2(b.x - M);
-        fr[rr] = Lsum > 0.f ? ex2(a.x - M) / Lsum : 0.f;
-    }
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            if (w == 2 * t + half) {
-#pragma unroll
-                for (int rr = 0; rr < 2; ++rr) {
-                    float2 *dst = reinterpret_cast<float2 *>(obuf + (gid + 8 * rr) * obuf_stride +
-                                                             2 * tig);
-#pragma unroll
-                    for (int n = 0; n < NT; ++n) {
-                        float2 v = make_float2(st.o[n][2 * rr] * fr[rr],
-                                               st.o[n][2 * rr + 1] * fr[rr]);
-                        if (half) {
-                            const float2 prev = dst[n * 4];
-                            v.x += prev.x;
-                            v.y += prev.y;
-                        }
-                        dst[n * 4] = v;
-                    }
-                }
-            }
-            named_bar_sync(1, kConsumerWarps * 32);
-        }
-        emit(t);
-        named_bar_sync(1, kConsumerWarps * 32);
-    }
-}
-
-// (M, L) of one row of tile t over its warp pair's (m, l).
-__device__ __forceinline__ float2 pair_row_stats(const float2 *ml, int t, int row) {
-    const float2 a = ml[2 * t * kMaxGroup + row], b = ml[(2 * t + 1) * kMaxGroup + row];
-    const float M = fmaxf(a.x, b.x);
-    const float Lsum = M == -INFINITY ? 0.f : a.y * ex2(a.x - M) + b.y * ex2(b.x - M);
-    return make_float2(M, Lsum);
-}
-
-// The consumer warps of paged_decode_shared_kernel: stages in ring order. A 16-row item
-// (suffix) gives each warp 16 tokens of every stage; a 32-row item (prefix) gives warp w
-// row tile w / 2 and tokens 32 (w % 2) .. + 31. At the end of an item, rows whose
-// (sequence, head) has one partial go straight to `out`; otherwise the item's partials go
-// to the workspace, and the last item of each chunk (16 rows) to finish merges its rows.
-template <typename T, int D, int BS>
-__device__ __forceinline__ void shared_consume(const SharedParams &prm, const uint8_t *ring,
-                                               float *obuf, StageInfo *info, uint64_t *full,
-                                               uint64_t *empty, float2 *ml, int warp,
-                                               int lane) {
-    using L = DecodeLayout<D>;
-    const int G = prm.group;
-    const int R = kMaxGroup / G;
-    const int w = warp;
-    const int gid = lane >> 2;
-    const int tig = lane & 3;
-    const int tid = threadIdx.x;   // 0..127
-    constexpr int KS = D / 16;
-    WarpState<D> st;
-    reset_state(st);
-    const T *qg = reinterpret_cast<const T *>(prm.q);
-    __shared__ int s_last[2];
-
-    // one finished row r of the item: output, or partial j of its (sequence, head)
-    auto put_row = [&](const StageInfo &in, int r, const float *src, float2 stats) {
-        const int s = in.s + r / G, h = in.hk * G + r % G;
-        const int np = prm.np[s];
-        if (np == 1) {
-            T *out = reinterpret_cast<T *>(prm.out) + ((size_t)s * prm.num_heads + h) * D;
-            for (int d = lane; d < D; d += 32) out[d] = from_float<T>(src[d]);
-        } else {
-            const size_t row = (size_t)prm.row_base[s] + (size_t)h * np + in.p;
-            for (int d = lane; d < D; d += 32) prm.ws_o[row * D + d] = src[d];
-            if (lane == 0) reinterpret_cast<float2 *>(prm.ws_ml)[row] = stats;
-        }
-    };
-
-    for (int it = 0;; ++it) {
-        const int slot = it % L::kStages;
-        if (!warp_wait(smem_u32(&full[slot]), (it / L::kStages) & 1)) {
-            if (lane == 0) atomicOr(prm.status, kStatusTimeout);
-            break;
-        }
-        const StageInfo in = info[slot];
-        if (in.flags & kEnd) break;
-        const int nrows = in.item * G;
-        const bool wide = (in.flags & kWide) != 0;
-        const int tile = wide ? (w >> 1) : 0;
-
-        if (in.flags & kFirst) {
-            // A fragments of this warp's row tile (rows >= nrows are zero)
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                const int r = tile * 16 + gid + 8 * half;
-                const uint32_t *qr = nullptr;
-                if (r < nrows) {
-                    const int s = in.s + r / G, h = in.hk * G + r % G;
-                    qr = reinterpret_cast<const uint32_t *>(
-                        qg + ((size_t)s * prm.num_heads + h) * D);
-                }
-#pragma unroll
-                for (int ks = 0; ks < KS; ++ks) {
-                    st.qa[ks][half] = qr ? __ldg(qr + ks * 8 + tig) : 0u;
-                    st.qa[ks][2 + half] = qr ? __ldg(qr + ks * 8 + tig + 4) : 0u;
-                }
-            }
-            reset_state(st);
-        }
-
-        const uint8_t *stage = ring + slot * L::kStageBytes;
-        if (wide) {
-            // this warp's 32 tokens as two 16-token slices; every row attends
-#pragma unroll
-            for (int sub = 0; sub < 2; ++sub) {
-                const int tok0 = 32 * (w & 1) + 16 * sub;
-                const int valid = in.ntok - tok0;
-                if (valid > 0)
-                    consume_stage<T, D, BS>(st, smem_u32(stage), smem_u32(stage + L::kKBytes),
-                                            tok0, lane, valid, prm.scale_log2);
-            }
-        } else {
-            const int valid = in.ntok - 16 * w;
-            if (valid > 0)
-                consume_stage<T, D, BS, true>(st, smem_u32(stage), smem_u32(stage + L::kKBytes),
-                                              16 * w, lane, valid, prm.scale_log2,
-                                              in.pad & 0xffff, in.pad >> 16);
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&empty[slot]));
-
-        if (in.flags & kLast) {
-            if (wide) {
-                merge_warp_pairs<D>(st, obuf, L::kObufStride, ml, w, lane, [&](int t) {
-                    for (int r = 16 * t + w; r < min(nrows, 16 * t + 16); r += kConsumerWarps)
-                        put_row(in, r, obuf + (r - 16 * t) * L::kObufStride,
-                                pair_row_stats(ml, t, r - 16 * t));
-                });
-            } else {
-                merge_warps<D>(st, nrows, obuf, L::kObufStride, ml, w, lane);
-                for (int r = w; r < nrows; r += kConsumerWarps)
-                    put_row(in, r, obuf + r * L::kObufStride, row_stats(ml, r));
-            }
-            // chunks (16 rows) of this item whose (sequence, head)s have several partials:
-            // publish, count, and the chunk's last item merges them
-            const int nchunks = (in.item + R - 1) / R;
-            __threadfence();
-            named_bar_sync(1, kConsumerWarps * 32);
-            if (tid < nchunks) {
-                const int s0 = in.s + tid * R;
-                int last = 0;
-                if (prm.np[s0] > 1) {
-                    int *done = prm.chunk_done + (size_t)s0 * prm.num_kv_heads + in.hk;
-                    last = atomicAdd(done, 1) == prm.np[s0] - 1;
-                }
-                s_last[tid] = last;
-            }
-            named_bar_sync(1, kConsumerWarps * 32);
-            for (int c = 0; c < nchunks; ++c) {
-                if (!s_last[c]) continue;
-                __threadfence();
-                const int s0 = in.s + c * R;
-                const int rows = min(R, in.item - c * R) * G;
-                for (int r = w; r < rows; r += kConsumerWarps) {
-                    const int s = s0 + r / G, h = in.hk * G + r % G;
-                    const int np = prm.np[s];
-                    const size_t row0 = (size_t)prm.row_base[s] + (size_t)h * np;
-                    warp_merge<T, D>(reinterpret_cast<const float2 *>(prm.ws_ml) + row0, 1,
-                                     prm.ws_o + row0 * D, D, np,
-                                     reinterpret_cast<T *>(prm.out) +
-                                         ((size_t)s * prm.num_heads + h) * D,
-                                     lane);
-                }
-                if (tid == 0)   // ready for the next launch over this plan
-                    prm.chunk_done[(size_t)s0 * prm.num_kv_heads + in.hk] = 0;
-            }
-            named_bar_sync(1, kConsumerWarps * 32);   // s_last is reused by the next item
-        }
-    }
-}
-
 // The producer's view of an item: its descriptor (lane k < 8 holds field k), each
 // member's token count in this item's suffix partition (lane m), and which segments
 // have tokens (bit 0: the prefix partition, bit 1 + m: member m's suffix part).
@@ -583,6 +356,114 @@ struct SharedSeg {
     int sidx;        // 0: prefix partition, 1 + m: member m's suffix partition
     bool first, last, valid;
 };
+
+// The consumer warps of paged_decode_shared_kernel: stages in ring order; at the end of an
+// item, the result of a chunk that is one item goes straight to `out`; otherwise the item's
+// partials go to the workspace, and the last of the chunk's items to finish (per KV head,
+// counted in chunk_done) merges them into `out`.
+template <typename T, int D, int BS>
+__device__ __forceinline__ void shared_consume(const SharedParams &prm, const uint8_t *ring,
+                                               float *obuf, StageInfo *info, uint64_t *full,
+                                               uint64_t *empty, float2 *ml, int warp,
+                                               int lane) {
+    using L = DecodeLayout<D>;
+    const int G = prm.group;
+    const int w = warp;
+    const int gid = lane >> 2;
+    const int tig = lane & 3;
+    constexpr int KS = D / 16;
+    WarpState<D> st;
+    reset_state(st);
+    const T *qg = reinterpret_cast<const T *>(prm.q);
+    __shared__ int s_last;
+
+    for (int it = 0;; ++it) {
+        const int slot = it % L::kStages;
+        if (!warp_wait(smem_u32(&full[slot]), (it / L::kStages) & 1)) {
+            if (lane == 0) atomicOr(prm.status, kStatusTimeout);
+            break;
+        }
+        const StageInfo in = info[slot];
+        if (in.flags & kEnd) break;
+        const int nrows = in.item * G;
+
+        if (in.flags & kFirst) {
+            // A fragments of the item's rows r = member * G + head (rows >= nrows are zero)
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int r = gid + 8 * half;
+                const uint32_t *qr = nullptr;
+                if (r < nrows) {
+                    const int s = in.s + r / G, h = in.hk * G + r % G;
+                    qr = reinterpret_cast<const uint32_t *>(
+                        qg + ((size_t)s * prm.num_heads + h) * D);
+                }
+#pragma unroll
+                for (int ks = 0; ks < KS; ++ks) {
+                    st.qa[ks][half] = qr ? __ldg(qr + ks * 8 + tig) : 0u;
+                    st.qa[ks][2 + half] = qr ? __ldg(qr + ks * 8 + tig + 4) : 0u;
+                }
+            }
+            reset_state(st);
+        }
+
+        const int valid = in.ntok - 16 * w;
+        if (valid > 0) {
+            const uint8_t *stage = ring + slot * L::kStageBytes;
+            consume_stage<T, D, BS, true>(st, smem_u32(stage), smem_u32(stage + L::kKBytes),
+                                          16 * w, lane, valid, prm.scale_log2, in.pad & 0xffff,
+                                          in.pad >> 16);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&empty[slot]));
+
+        if (in.flags & kLast) {
+            merge_warps<D>(st, nrows, obuf, L::kObufStride, ml, w, lane);
+            const int tid = threadIdx.x;
+            if (in.npart == 1) {
+                // the chunk is this one item: final output
+                for (int idx = tid; idx < nrows * D; idx += kConsumerWarps * 32) {
+                    const int r = idx / D, dim = idx - r * D;
+                    const int s = in.s + r / G, h = in.hk * G + r % G;
+                    reinterpret_cast<T *>(prm.out)[((size_t)s * prm.num_heads + h) * D + dim] =
+                        from_float<T>(obuf[r * L::kObufStride + dim]);
+                }
+            } else {
+                for (int idx = tid; idx < nrows * D; idx += kConsumerWarps * 32) {
+                    const int r = idx / D, dim = idx - r * D;
+                    const int s = in.s + r / G, h = in.hk * G + r % G;
+                    const size_t row = (size_t)prm.row_base[s] + (size_t)h * prm.np[s] + in.p;
+                    prm.ws_o[row * D + dim] = obuf[r * L::kObufStride + dim];
+                }
+                if (tid < nrows) {
+                    const int s = in.s + tid / G, h = in.hk * G + tid % G;
+                    const size_t row = (size_t)prm.row_base[s] + (size_t)h * prm.np[s] + in.p;
+                    reinterpret_cast<float2 *>(prm.ws_ml)[row] = row_stats(ml, tid);
+                }
+                // publish the partials; the chunk's last item to arrive merges every row
+                __threadfence();
+                named_bar_sync(1, kConsumerWarps * 32);
+                int *done = prm.chunk_done + (size_t)in.s * prm.num_kv_heads + in.hk;
+                if (tid == 0) s_last = atomicAdd(done, 1) == in.npart - 1;
+                named_bar_sync(1, kConsumerWarps * 32);
+                if (s_last) {
+                    __threadfence();
+                    for (int r = w; r < nrows; r += kConsumerWarps) {
+                        const int s = in.s + r / G, h = in.hk * G + r % G;
+                        const int np = prm.np[s];
+                        const size_t row0 = (size_t)prm.row_base[s] + (size_t)h * np;
+                        warp_merge<T, D>(reinterpret_cast<const float2 *>(prm.ws_ml) + row0, 1,
+                                         prm.ws_o + row0 * D, D, np,
+                                         reinterpret_cast<T *>(prm.out) +
+                                             ((size_t)s * prm.num_heads + h) * D,
+                                         lane);
+                    }
+                    if (tid == 0) *done = 0;   // ready for the next launch over this plan
+                }
+            }
+        }
+    }
+}
 
 template <typename T, int D, int BS>
 __global__ void __launch_bounds__(kDecodeThreads, 2)
@@ -639,7 +520,7 @@ paged_decode_shared_kernel(const __grid_constant__ CUtensorMap tmap_k,
             return v > 0x7fffffffu ? 0x7fffffff : (int)v;   // lives in lane 0
         };
         auto field = [&](const SharedItemCtx &c, int k) { return __shfl_sync(0xffffffffu, c.f, k); };
-        // descriptor; for a suffix item, the members' token counts and non-empty segments
+        // descriptor, members' suffix-part token counts, non-empty segments
         auto load_item = [&](int idx) {
             SharedItemCtx c;
             c.idx = idx;
@@ -648,16 +529,14 @@ paged_decode_shared_kernel(const __grid_constant__ CUtensorMap tmap_k,
             c.mtok = 0;
             c.mask = 0u;
             if (!c.valid) return c;
-            if (field(c, 7)) {   // prefix partition j: one segment
-                c.mask = 1u;
-                return c;
-            }
-            const int pre = field(c, 1), first = field(c, 2), nseq = field(c, 3), k = field(c, 6);
-            if (lane < nseq) {
+            const int pre = field(c, 1), first = field(c, 2), nseq = field(c, 3);
+            const int j = field(c, 5), npp = field(c, 6), nps2 = field(c, 7);
+            const int k = j - npp + (nps2 & 1);   // suffix partition of this item, if any
+            if (k >= 0 && k < (nps2 >> 1) && lane < nseq) {
                 const int len = clamp_len(prm.context_lens[first + lane], prm.max_context_len);
                 c.mtok = max(0, min(P, len - pre - k * P));
             }
-            c.mask = __ballot_sync(0xffffffffu, c.mtok > 0) << 1;
+            c.mask = (__ballot_sync(0xffffffffu, c.mtok > 0) << 1) | (j < npp ? 1u : 0u);
             return c;
         };
         // segment sidx of item c (sidx < 0: the empty item's single stage of no tokens)
@@ -669,15 +548,16 @@ paged_decode_shared_kernel(const __grid_constant__ CUtensorMap tmap_k,
             const int m = sidx - 1;
             const int mt = __shfl_sync(0xffffffffu, c.mtok, max(m, 0));
             if (sidx <= 0) {
-                const int j = field(c, 6), pre = field(c, 1);
+                const int j = field(c, 5), pre = field(c, 1);
                 g.seq = sidx == 0 ? field(c, 0) : field(c, 2);
                 g.tok0 = sidx == 0 ? j * P : 0;
                 g.ntok = sidx == 0 ? min(P, pre - j * P) : 0;
                 g.r0 = 0;
                 g.r1 = nseq * G;
             } else {
+                const int j = field(c, 5), npp = field(c, 6), nps2 = field(c, 7);
                 g.seq = field(c, 2) + m;
-                g.tok0 = field(c, 1) + field(c, 6) * P;
+                g.tok0 = field(c, 1) + (j - npp + (nps2 & 1)) * P;
                 g.ntok = mt;
                 g.r0 = m * G;
                 g.r1 = (m + 1) * G;
@@ -714,7 +594,7 @@ paged_decode_shared_kernel(const __grid_constant__ CUtensorMap tmap_k,
             const int first_seq = field(cur_item, 2);
             const int nseq = field(cur_item, 3);
             const int part = field(cur_item, 5);
-            const int wide = field(cur_item, 7) && nseq * G > kMaxGroup ? kWide : 0;
+            const int nparts = chunk_parts(field(cur_item, 6), field(cur_item, 7));
             const int nst = max(1, (cur.ntok + kStageTokens - 1) / kStageTokens);
             SharedItemCtx nxt_item = cur_item;
             SharedSeg nxt;
@@ -740,11 +620,11 @@ paged_decode_shared_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 const uint32_t bar = smem_u32(&full[slot]);
                 if (lane == 0) {
                     StageInfo in;
-                    in.s = first_seq; in.hk = hk; in.p = part; in.npart = 0;
+                    in.s = first_seq; in.hk = hk; in.p = part; in.npart = nparts;
                     in.item = nseq;
                     in.ntok = sntok;
                     in.flags = (cur.first && st == 0 ? kFirst : 0) |
-                               (cur.last && st == nst - 1 ? kLast : 0) | wide;
+                               (cur.last && st == nst - 1 ? kLast : 0);
                     in.pad = cur.r0 | (cur.r1 << 16);
                     info[slot] = in;
                     mbar_arrive_expect_tx(bar, (uint32_t)(nb_st * BS * L::kRowBytes * 2));

