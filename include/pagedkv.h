@@ -177,10 +177,10 @@ int pkv_paged_attention_decode_noalloc(void *out, const void *q, const void *k_c
  * Shared-prefix-aware decode: the same result as pkv_paged_attention_decode, for
  * batches where groups of sequences share their first pages (parallel sampling, common
  * prompts: "vLLM" entity page, 是什么; "分页 KV Cache 分析" §3.2). Each shared prefix page
- * of a KV head is read once for up to 32 query rows (the G heads of up to 32/G member
- * sequences) instead of once per sequence; private suffixes are read per sequence (16/G
- * sequences per work item); the pieces are merged exactly (log-sum-exp) inside the decode
- * launch by the last piece of each group of 16/G sequences to finish.
+ * of a KV head is read once for up to 16 query rows (the G heads of up to 16/G member
+ * sequences) instead of once per sequence; private suffixes are read per sequence, in the
+ * same work item as the prefix where both fit in one partition (then written directly),
+ * else as pieces merged exactly (log-sum-exp).
  *
  * group_start  device int32 [num_groups + 1]: sequences group_start[g] ..
  *              group_start[g+1]-1 form group g (0 = group_start[0] < ... <
