@@ -274,12 +274,14 @@ def explicit_case(rng, groups, Hq, Hkv, D, BS, dtype):
             mb * BS)
 
 
-@pytest.mark.parametrize("Hq,Hkv,BS", [(32, 8, 16), (16, 2, 32), (8, 8, 8)])
+@pytest.mark.parametrize("Hq,Hkv,BS", [(32, 8, 16), (16, 2, 32), (8, 8, 8), (12, 2, 16),
+                                        (10, 2, 8)])
 def test_chunks_fused_split_and_empty(cuda_device, Hq, Hkv, BS):
     """Chunks whose prefix and suffixes form one item (written directly) next to chunks
-    split into several items (merged): members with no suffix, suffixes longer than a
-    partition, a group whose members hold nothing at all, and groups of one; each at the
-    automatic partition and at small ones."""
+    split into several items (merged in the launch by the chunk's last item): members with
+    no suffix, suffixes longer than a partition, a group whose members hold nothing at all,
+    groups of one and a group of 19 members; G = 6 and 5 leave chunks of fewer than 16
+    rows; each at the automatic partition and at small ones."""
     rng = np.random.default_rng(Hq + Hkv + BS)
     dtype = synth.F16
     groups = [(64 * BS, [0, 3, 0, 700, 1, 0, 65, 64, 2]),   # mixed suffixes, some none
@@ -287,7 +289,8 @@ def test_chunks_fused_split_and_empty(cuda_device, Hq, Hkv, BS):
               (2 * BS, [1]),                                   # a group of one
               (0, [900]),
               (10 * BS, [0, 0]),                               # the prefix is everything
-              (5 * BS, [130, 2, 2500, 17])]
+              (5 * BS, [130, 2, 2500, 17]),
+              (3 * BS, [int(x) for x in rng.integers(0, 90, 19)])]        # 19 members
     q, kc, vc, bt, lens, starts, pre, max_len = explicit_case(rng, groups, Hq, Hkv, 128, BS,
                                                               dtype)
     ref = A.paged_decode_attention(q, kc, vc, bt, lens, 0.09, dtype)
