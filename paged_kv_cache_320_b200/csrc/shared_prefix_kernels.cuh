@@ -589,6 +589,11 @@ paged_decode_shared_kernel(const __grid_constant__ CUtensorMap tmap_k,
         SharedSeg cur = first_seg(cur_item);
         int ent[kMaxItemBlocks / 32];
         load_entries(cur, ent);
+        // The next item is looked up while the current item's first segment streams (its
+        // descriptor and lengths are a chain of dependent loads), and each segment's table
+        // slice while the segment before it streams.
+        SharedItemCtx nxt_item = cur_item;
+        nxt_item.valid = false;
         while (cur.valid && ok) {
             const int hk = field(cur_item, 4);
             const int first_seq = field(cur_item, 2);
@@ -596,7 +601,6 @@ paged_decode_shared_kernel(const __grid_constant__ CUtensorMap tmap_k,
             const int part = field(cur_item, 5);
             const int nparts = chunk_parts(field(cur_item, 6), field(cur_item, 7));
             const int nst = max(1, (cur.ntok + kStageTokens - 1) / kStageTokens);
-            SharedItemCtx nxt_item = cur_item;
             SharedSeg nxt;
             nxt.valid = false;
             int nxt_ent[kMaxItemBlocks / 32];
@@ -651,20 +655,21 @@ paged_decode_shared_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     }
                 }
                 if (st == 0) {
-                    // the next segment and its table slice, while this one streams
+                    if (cur.first) {
+                        nxt_item = load_item(__shfl_sync(0xffffffffu, pending, 0));
+                        if (nxt_item.valid) pending = take();
+                    }
                     if (!cur.last) {
                         const unsigned above = cur_item.mask & ~((2u << cur.sidx) - 1u);
                         nxt = make_seg(cur_item, __ffs(above) - 1);
                     } else {
-                        nxt_item = load_item(__shfl_sync(0xffffffffu, pending, 0));
-                        if (nxt_item.valid) pending = take();
                         nxt = first_seg(nxt_item);
                     }
                     load_entries(nxt, nxt_ent);
                 }
             }
+            if (cur.last) cur_item = nxt_item;
             cur = nxt;
-            cur_item = nxt_item;
 #pragma unroll
             for (int k = 0; k < kMaxItemBlocks / 32; ++k) ent[k] = nxt_ent[k];
         }
