@@ -545,8 +545,8 @@ def gpu_arm(args, rank, world, local_rank, light=False):
         kernel_key = ("paged_decode_partition_write" if launches_per_layer > 1 or pmax == 1
                       else "paged_decode_step")
     else:
-        launches_per_layer = 2 if shared else 2 + (1 if pmax > 1 else 0)
-        launches_per_step = (2 * L + 1) if shared else L * launches_per_layer
+        launches_per_layer = 3 if shared else 2 + (1 if pmax > 1 else 0)
+        launches_per_step = (3 * L + 1) if shared else L * launches_per_layer
         kernel_key = "paged_decode_shared" if shared else "paged_decode_partition"
     split = not shared and (not fused or launches_per_layer > 1)
 
@@ -633,7 +633,7 @@ def gpu_arm(args, rank, world, local_rank, light=False):
                      "write-and-decode kernel (one partition per context)" if pmax == 1 else
                      "step kernel (cache write, decode and merge in one launch)")
     else:
-        call_desc = ("cache write + plan (one per step) + shared-prefix decode" if shared else
+        call_desc = ("plan (one per step) + shared-prefix decode + merge" if shared else
                      "cache write + partition kernel" + (" + merge kernel" if pmax > 1 else ""))
     roofline = {
         "kernel": f"{kernel_key}_kernel",

@@ -195,8 +195,7 @@ int pkv_paged_attention_decode_noalloc(void *out, const void *q, const void *k_c
  * PKV_ERR_WORKSPACE). partition_size 0 selects this path's own automatic size
  * (pkv_decode_shared_prefix_partition_size: 2048 tokens, at most 256 blocks, smaller for
  * small batches). Other arguments, limits and errors as
- * pkv_paged_attention_decode (num_groups >= 1, <= num_seqs). Two kernel launches (the plan, then
- * the decode, whose last work item of a split chunk merges that chunk's partials).
+ * pkv_paged_attention_decode (num_groups >= 1, <= num_seqs). Three kernel launches.
  * ---------------------------------------------------------------------------- */
 int pkv_paged_attention_decode_shared_prefix(
     void *out, const void *q, const void *k_cache, const void *v_cache,
@@ -209,9 +208,9 @@ int pkv_paged_attention_decode_shared_prefix(
 /* The same call in two parts, so that one plan serves every layer of a step (the plan
  * depends only on the tables, lengths and groups, which the layers share):
  * pkv_shared_prefix_plan builds the item list in the workspace (one launch);
- * pkv_paged_attention_decode_shared_prefix_planned runs the decode over it (one launch, which
- * leaves the workspace ready for the next) and may be called any number of times on the same
- * workspace, ordered on one stream, while the tables and lengths stay as planned. A planned call whose sizes
+ * pkv_paged_attention_decode_shared_prefix_planned runs the decode and the merge over it
+ * (two launches) and may be called any number of times on the same workspace, ordered on
+ * one stream, while the tables and lengths stay as planned. A planned call whose sizes
  * (num_seqs, num_heads, num_kv_heads, partition size) differ from the plan's writes nothing
  * and sets PKV_STATUS_WORKSPACE. Arguments as pkv_paged_attention_decode_shared_prefix;
  * pkv_paged_attention_decode_shared_prefix is the plan followed by one planned call. */

@@ -294,9 +294,9 @@ int dispatch_bs(int BS, const CUtensorMap &mk, const CUtensorMap &mv, const CUte
 
 // ---- shared-prefix decode ------------------------------------------------
 // Workspace: [counters 256 B][np, row_base, seq_group, gpre, gmin, gmis, ioff: B ints each]
-// [chunk completion counters: B x Hkv ints][items][partials (max, sum)][partial outputs].
+// [items][partials (max, sum)][partial outputs].
 struct SharedWs {
-    size_t ints, done, items, ml, o, total;
+    size_t ints, items, ml, o, total;
     int max_items;
     long long rows;
 };
@@ -307,8 +307,7 @@ SharedWs shared_ws_layout(int B, int Hq, int Hkv, int D, int max_len, int P) {
     w.max_items = (int)std::min<long long>(2LL * Hkv * B * pmax, INT_MAX / 2);
     w.rows = (long long)B * Hq * (pmax + 1);
     w.ints = sizeof(pkv::SharedCounters);
-    w.done = w.ints + 7 * align_up((size_t)B * sizeof(int), 256);
-    w.items = w.done + align_up((size_t)B * Hkv * sizeof(int), 256);
+    w.items = w.ints + 7 * align_up((size_t)B * sizeof(int), 256);
     w.ml = w.items + align_up((size_t)w.max_items * sizeof(pkv::SharedItem), 256);
     w.o = w.ml + align_up((size_t)w.rows * 2 * sizeof(float), 256);
     w.total = w.o + (size_t)w.rows * D * sizeof(float);
@@ -367,14 +366,20 @@ int launch_shared_plan(const pkv::SharedParams &prm, cudaStream_t st) {
 }
 
 template <typename T, int D>
-int dispatch_shared_decode(int BS, const CUtensorMap &mk, const CUtensorMap &mv,
-                           const pkv::SharedParams &prm, cudaStream_t st) {
+int launch_shared_decode_reduce(int BS, const CUtensorMap &mk, const CUtensorMap &mv,
+                                const pkv::SharedParams &prm, cudaStream_t st) {
+    int rc;
     switch (BS) {
-        case 8: return launch_shared_decode<T, D, 8>(mk, mv, prm, st);
-        case 16: return launch_shared_decode<T, D, 16>(mk, mv, prm, st);
-        case 32: return launch_shared_decode<T, D, 32>(mk, mv, prm, st);
+        case 8: rc = launch_shared_decode<T, D, 8>(mk, mv, prm, st); break;
+        case 16: rc = launch_shared_decode<T, D, 16>(mk, mv, prm, st); break;
+        case 32: rc = launch_shared_decode<T, D, 32>(mk, mv, prm, st); break;
+        default: return PKV_ERR_INVALID_ARG;
     }
-    return PKV_ERR_INVALID_ARG;
+    if (rc != PKV_OK) return rc;
+    const long long pairs = (long long)prm.num_seqs * prm.num_heads;
+    const long long grid = (pairs + pkv::kReduceWarps - 1) / pkv::kReduceWarps;
+    return launch(pkv::paged_decode_shared_reduce_kernel<T, D>, dim3((unsigned)grid),
+                  dim3(pkv::kReduceWarps * 32), 0, st, prm);
 }
 
 // Workspace pointers and sizes of the shared-prefix path (no output, query or scale).
@@ -394,7 +399,6 @@ pkv::SharedParams shared_params(const SharedWs &ws, void *workspace, int num_seq
     prm.gmin = reinterpret_cast<int *>(wsb + ws.ints + 4 * ib);
     prm.gmis = reinterpret_cast<int *>(wsb + ws.ints + 5 * ib);
     prm.ioff = reinterpret_cast<int *>(wsb + ws.ints + 6 * ib);
-    prm.chunk_done = reinterpret_cast<int *>(wsb + ws.done);
     prm.items = reinterpret_cast<pkv::SharedItem *>(wsb + ws.items);
     prm.ws_ml = reinterpret_cast<float *>(wsb + ws.ml);
     prm.ws_o = reinterpret_cast<float *>(wsb + ws.o);
@@ -1016,10 +1020,10 @@ int pkv_paged_attention_decode_shared_prefix_planned(
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (dtype == PKV_BF16)
         return head_dim == 128
-                   ? dispatch_shared_decode<__nv_bfloat16, 128>(block_size, mk, mv, prm, st)
-                   : dispatch_shared_decode<__nv_bfloat16, 64>(block_size, mk, mv, prm, st);
-    return head_dim == 128 ? dispatch_shared_decode<__half, 128>(block_size, mk, mv, prm, st)
-                           : dispatch_shared_decode<__half, 64>(block_size, mk, mv, prm, st);
+                   ? launch_shared_decode_reduce<__nv_bfloat16, 128>(block_size, mk, mv, prm, st)
+                   : launch_shared_decode_reduce<__nv_bfloat16, 64>(block_size, mk, mv, prm, st);
+    return head_dim == 128 ? launch_shared_decode_reduce<__half, 128>(block_size, mk, mv, prm, st)
+                           : launch_shared_decode_reduce<__half, 64>(block_size, mk, mv, prm, st);
 }
 
 int pkv_paged_attention_decode_shared_prefix(

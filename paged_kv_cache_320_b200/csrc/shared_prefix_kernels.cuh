@@ -51,13 +51,11 @@ __host__ __device__ __forceinline__ int chunk_parts(int npp, int nps2) {
 }
 
 struct SharedCounters {
-    unsigned next;    // next work item (0 after the plan and after every decode launch)
+    unsigned next;    // next work item (0 after the plan and after every reduce)
     int count;        // items in the list
     int sig[4];       // sizes the plan was built for (kPlanMagic, B, Hq | Hkv << 16, P)
-    unsigned exit;    // CTAs of the current decode launch that have finished
-    int pad[57];
+    int pad[58];
 };
-static_assert(sizeof(SharedCounters) == 256, "shared-prefix workspace header size");
 
 // The plan stays valid for every layer of a step (it depends on the tables, lengths and
 // groups only): decode and reduce launches check that the workspace holds a plan for
@@ -82,8 +80,6 @@ struct SharedParams {
     int *gmis;         // [B] first block where a member's table differs per group, then
                        //     first item per chunk (plan scratch)
     int *ioff;         // [B] 2 x suffix partitions + fused, per chunk (plan scratch)
-    int *chunk_done;   // [B][Hkv] items of a split chunk finished, by first member (0 between
-                       //          launches: the plan zeroes them, the chunk's merger resets)
     float *ws_o;       // [rows][D]
     float *ws_ml;      // [rows][2]
     void *out;
@@ -170,12 +166,10 @@ shared_prefix_plan_kernel(SharedParams p) {
     int *slen = in_smem ? plan_smem + 4 * B : p.np;          // clamped lengths
     int *gfirst = in_smem ? plan_smem + 5 * B : p.row_base;  // first member of each group
     int *ioff = in_smem ? plan_smem + 6 * B : p.ioff;        // per-chunk partition counts
-    for (int i = tid; i < B * Hkv; i += kPlanThreads) p.chunk_done[i] = 0;
     if (tid == 0) {
         bad = 0;
         max_pre_blocks = 0;
         p.counters->next = 0u;
-        p.counters->exit = 0u;
         const int ng = p.num_groups;
         if (ng < 1 || ng > B || p.group_start[0] != 0 || p.group_start[ng] != B) bad = 1;
     }
@@ -356,114 +350,6 @@ struct SharedSeg {
     int sidx;        // 0: prefix partition, 1 + m: member m's suffix partition
     bool first, last, valid;
 };
-
-// The consumer warps of paged_decode_shared_kernel: stages in ring order; at the end of an
-// item, the result of a chunk that is one item goes straight to `out`; otherwise the item's
-// partials go to the workspace, and the last of the chunk's items to finish (per KV head,
-// counted in chunk_done) merges them into `out`.
-template <typename T, int D, int BS>
-__device__ __forceinline__ void shared_consume(const SharedParams &prm, const uint8_t *ring,
-                                               float *obuf, StageInfo *info, uint64_t *full,
-                                               uint64_t *empty, float2 *ml, int warp,
-                                               int lane) {
-    using L = DecodeLayout<D>;
-    const int G = prm.group;
-    const int w = warp;
-    const int gid = lane >> 2;
-    const int tig = lane & 3;
-    constexpr int KS = D / 16;
-    WarpState<D> st;
-    reset_state(st);
-    const T *qg = reinterpret_cast<const T *>(prm.q);
-    __shared__ int s_last;
-
-    for (int it = 0;; ++it) {
-        const int slot = it % L::kStages;
-        if (!warp_wait(smem_u32(&full[slot]), (it / L::kStages) & 1)) {
-            if (lane == 0) atomicOr(prm.status, kStatusTimeout);
-            break;
-        }
-        const StageInfo in = info[slot];
-        if (in.flags & kEnd) break;
-        const int nrows = in.item * G;
-
-        if (in.flags & kFirst) {
-            // A fragments of the item's rows r = member * G + head (rows >= nrows are zero)
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                const int r = gid + 8 * half;
-                const uint32_t *qr = nullptr;
-                if (r < nrows) {
-                    const int s = in.s + r / G, h = in.hk * G + r % G;
-                    qr = reinterpret_cast<const uint32_t *>(
-                        qg + ((size_t)s * prm.num_heads + h) * D);
-                }
-#pragma unroll
-                for (int ks = 0; ks < KS; ++ks) {
-                    st.qa[ks][half] = qr ? __ldg(qr + ks * 8 + tig) : 0u;
-                    st.qa[ks][2 + half] = qr ? __ldg(qr + ks * 8 + tig + 4) : 0u;
-                }
-            }
-            reset_state(st);
-        }
-
-        const int valid = in.ntok - 16 * w;
-        if (valid > 0) {
-            const uint8_t *stage = ring + slot * L::kStageBytes;
-            consume_stage<T, D, BS, true>(st, smem_u32(stage), smem_u32(stage + L::kKBytes),
-                                          16 * w, lane, valid, prm.scale_log2, in.pad & 0xffff,
-                                          in.pad >> 16);
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&empty[slot]));
-
-        if (in.flags & kLast) {
-            merge_warps<D>(st, nrows, obuf, L::kObufStride, ml, w, lane);
-            const int tid = threadIdx.x;
-            if (in.npart == 1) {
-                // the chunk is this one item: final output
-                for (int idx = tid; idx < nrows * D; idx += kConsumerWarps * 32) {
-                    const int r = idx / D, dim = idx - r * D;
-                    const int s = in.s + r / G, h = in.hk * G + r % G;
-                    reinterpret_cast<T *>(prm.out)[((size_t)s * prm.num_heads + h) * D + dim] =
-                        from_float<T>(obuf[r * L::kObufStride + dim]);
-                }
-            } else {
-                for (int idx = tid; idx < nrows * D; idx += kConsumerWarps * 32) {
-                    const int r = idx / D, dim = idx - r * D;
-                    const int s = in.s + r / G, h = in.hk * G + r % G;
-                    const size_t row = (size_t)prm.row_base[s] + (size_t)h * prm.np[s] + in.p;
-                    prm.ws_o[row * D + dim] = obuf[r * L::kObufStride + dim];
-                }
-                if (tid < nrows) {
-                    const int s = in.s + tid / G, h = in.hk * G + tid % G;
-                    const size_t row = (size_t)prm.row_base[s] + (size_t)h * prm.np[s] + in.p;
-                    reinterpret_cast<float2 *>(prm.ws_ml)[row] = row_stats(ml, tid);
-                }
-                // publish the partials; the chunk's last item to arrive merges every row
-                __threadfence();
-                named_bar_sync(1, kConsumerWarps * 32);
-                int *done = prm.chunk_done + (size_t)in.s * prm.num_kv_heads + in.hk;
-                if (tid == 0) s_last = atomicAdd(done, 1) == in.npart - 1;
-                named_bar_sync(1, kConsumerWarps * 32);
-                if (s_last) {
-                    __threadfence();
-                    for (int r = w; r < nrows; r += kConsumerWarps) {
-                        const int s = in.s + r / G, h = in.hk * G + r % G;
-                        const int np = prm.np[s];
-                        const size_t row0 = (size_t)prm.row_base[s] + (size_t)h * np;
-                        warp_merge<T, D>(reinterpret_cast<const float2 *>(prm.ws_ml) + row0, 1,
-                                         prm.ws_o + row0 * D, D, np,
-                                         reinterpret_cast<T *>(prm.out) +
-                                             ((size_t)s * prm.num_heads + h) * D,
-                                         lane);
-                    }
-                    if (tid == 0) *done = 0;   // ready for the next launch over this plan
-                }
-            }
-        }
-    }
-}
 
 template <typename T, int D, int BS>
 __global__ void __launch_bounds__(kDecodeThreads, 2)
@@ -693,20 +579,108 @@ paged_decode_shared_kernel(const __grid_constant__ CUtensorMap tmap_k,
             for (int j = max(0, it - L::kStages); j < it; ++j)
                 warp_wait(smem_u32(&full[j % L::kStages]), (j / L::kStages) & 1);
         }
-    } else {
-        shared_consume<T, D, BS>(prm, ring, obuf, info, full, empty, ml, warp, lane);
+        return;
     }
-    // the last CTA out leaves the work counter at 0 for the next launch over this plan
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        const unsigned t = atomicAdd(&prm.counters->exit, 1u);
-        if (t == gridDim.x - 1) {
-            prm.counters->next = 0u;
-            prm.counters->exit = 0u;
-            __threadfence();
+
+    // ---------------------------------------------------------------- consumers
+    const int w = warp;
+    const int gid = lane >> 2;
+    const int tig = lane & 3;
+    constexpr int KS = D / 16;
+    WarpState<D> st;
+    reset_state(st);
+    const T *qg = reinterpret_cast<const T *>(prm.q);
+
+    for (int it = 0;; ++it) {
+        const int slot = it % L::kStages;
+        if (!warp_wait(smem_u32(&full[slot]), (it / L::kStages) & 1)) {
+            if (lane == 0) atomicOr(prm.status, kStatusTimeout);
+            break;
+        }
+        const StageInfo in = info[slot];
+        if (in.flags & kEnd) break;
+        const int nrows = in.item * G;
+
+        if (in.flags & kFirst) {
+            // A fragments of the item's rows r = member * G + head (rows >= nrows are zero)
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int r = gid + 8 * half;
+                const uint32_t *qr = nullptr;
+                if (r < nrows) {
+                    const int s = in.s + r / G, h = in.hk * G + r % G;
+                    qr = reinterpret_cast<const uint32_t *>(
+                        qg + ((size_t)s * prm.num_heads + h) * D);
+                }
+#pragma unroll
+                for (int ks = 0; ks < KS; ++ks) {
+                    st.qa[ks][half] = qr ? __ldg(qr + ks * 8 + tig) : 0u;
+                    st.qa[ks][2 + half] = qr ? __ldg(qr + ks * 8 + tig + 4) : 0u;
+                }
+            }
+            reset_state(st);
+        }
+
+        const int valid = in.ntok - 16 * w;
+        if (valid > 0) {
+            const uint8_t *stage = ring + slot * L::kStageBytes;
+            consume_stage<T, D, BS, true>(st, smem_u32(stage), smem_u32(stage + L::kKBytes),
+                                          16 * w, lane, valid, prm.scale_log2, in.pad & 0xffff,
+                                          in.pad >> 16);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&empty[slot]));
+
+        if (in.flags & kLast) {
+            merge_warps<D>(st, nrows, obuf, L::kObufStride, ml, w, lane);
+            const int tid = threadIdx.x;
+            if (in.npart == 1) {
+                // the chunk is this one item: final output
+                for (int idx = tid; idx < nrows * D; idx += kConsumerWarps * 32) {
+                    const int r = idx / D, dim = idx - r * D;
+                    const int s = in.s + r / G, h = in.hk * G + r % G;
+                    reinterpret_cast<T *>(prm.out)[((size_t)s * prm.num_heads + h) * D + dim] =
+                        from_float<T>(obuf[r * L::kObufStride + dim]);
+                }
+            } else {
+                for (int idx = tid; idx < nrows * D; idx += kConsumerWarps * 32) {
+                    const int r = idx / D, dim = idx - r * D;
+                    const int s = in.s + r / G, h = in.hk * G + r % G;
+                    const size_t row = (size_t)prm.row_base[s] + (size_t)h * prm.np[s] + in.p;
+                    prm.ws_o[row * D + dim] = obuf[r * L::kObufStride + dim];
+                }
+                if (tid < nrows) {
+                    const int s = in.s + tid / G, h = in.hk * G + tid % G;
+                    const size_t row = (size_t)prm.row_base[s] + (size_t)h * prm.np[s] + in.p;
+                    reinterpret_cast<float2 *>(prm.ws_ml)[row] = row_stats(ml, tid);
+                }
+            }
         }
     }
+}
+
+// Merge of the partials of every (sequence, head) whose chunk was split into several
+// items: rows row_base[s] + h*np[s] + j, j < np[s]; one warp per pair.
+template <typename T, int D>
+__global__ void __launch_bounds__(kReduceWarps * 32)
+paged_decode_shared_reduce_kernel(SharedParams prm) {
+    pdl_wait_and_release();
+    if (!plan_matches(prm.counters, prm.num_seqs, prm.num_heads, prm.num_kv_heads, prm.partition))
+        return;
+    // the decode launch has finished (stream order): re-arm the work counter for the next
+    // decode over the same plan
+    if (blockIdx.x == 0 && threadIdx.x == 0) prm.counters->next = 0u;
+    const int lane = threadIdx.x & 31;
+    const int pair = blockIdx.x * kReduceWarps + (threadIdx.x >> 5);
+    if (pair >= prm.num_seqs * prm.num_heads) return;
+    const int s = pair / prm.num_heads;
+    const int h = pair - s * prm.num_heads;
+    const int np = prm.np[s];
+    if (np == 1) return;   // written by the decode kernel
+    const size_t row0 = (size_t)prm.row_base[s] + (size_t)h * np;
+    warp_merge<T, D>(reinterpret_cast<const float2 *>(prm.ws_ml) + row0, 1,
+                     prm.ws_o + row0 * D, D, np,
+                     reinterpret_cast<T *>(prm.out) + ((size_t)s * prm.num_heads + h) * D, lane);
 }
 
 }  // namespace pkv
