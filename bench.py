@@ -291,22 +291,35 @@ def cow_arm(args, rank, world, local_rank):
     # calls); two steps in flight with double-buffered inputs and outputs, as in e2e_arm
     NBUF = 2
     pin = dict(pin_memory=True)
-    q_h = torch.empty(tuple(q.shape), dtype=dt, **pin); q_h.copy_(q.cpu())
-    kn_h = torch.empty(tuple(kn.shape), dtype=dt, **pin); kn_h.copy_(kn.cpu())
-    vn_h = torch.empty(tuple(vn.shape), dtype=dt, **pin); vn_h.copy_(vn.cpu())
+
+    def packed(parts, device=None):
+        """One byte buffer holding each (shape, dtype) part at a 256-byte aligned offset,
+        and a view of each part: one copy moves all of them."""
+        offs, total = [], 0
+        for shape, dtp in parts:
+            offs.append(total)
+            n = int(np.prod(shape)) * torch.empty((), dtype=dtp).element_size()
+            total += -(-n // 256) * 256
+        buf = (torch.empty(total, dtype=torch.uint8, device=device) if device is not None
+               else torch.empty(total, dtype=torch.uint8, **pin))
+        views = []
+        for (shape, dtp), o in zip(parts, offs):
+            n = int(np.prod(shape)) * torch.empty((), dtype=dtp).element_size()
+            views.append(buf[o:o + n].view(dtp).view(shape))
+        return buf, views
+
+    # this step's query and new K/V rows (one H2D copy), and the host block manager's
+    # results (slots, copy-on-write pairs, tables, lengths: one H2D copy)
+    act_parts = [(tuple(q.shape), dt), (tuple(kn.shape), dt), (tuple(vn.shape), dt)]
+    tab_parts = [((B,), torch.int64), ((n_pairs, 2), torch.int32), (tuple(tables.shape), torch.int32),
+                 ((B,), torch.int32)]
+    act_h, (q_h, kn_h, vn_h) = packed(act_parts)
+    q_h.copy_(q.cpu()); kn_h.copy_(kn.cpu()); vn_h.copy_(vn.cpu())
+    tab_h = [packed(tab_parts) for _ in range(NBUF)]
+    act_e = [packed(act_parts, dev) for _ in range(NBUF)]
+    tab_e = [packed(tab_parts, dev) for _ in range(NBUF)]
     out_h = [torch.empty(tuple(q.shape), dtype=dt, **pin) for _ in range(NBUF)]
-    sl_h = [torch.empty(B, dtype=torch.int64, **pin) for _ in range(NBUF)]
-    pr_h = [torch.empty((n_pairs, 2), dtype=torch.int32, **pin) for _ in range(NBUF)]
-    bt_h = [torch.empty(tuple(tables.shape), dtype=torch.int32, **pin) for _ in range(NBUF)]
-    ln_h = [torch.empty(B, dtype=torch.int32, **pin) for _ in range(NBUF)]
-    q_e = [torch.empty_like(q) for _ in range(NBUF)]
-    kn_e = [torch.empty_like(kn) for _ in range(NBUF)]
-    vn_e = [torch.empty_like(vn) for _ in range(NBUF)]
     out_e = [torch.empty_like(out) for _ in range(NBUF)]
-    sl_e = [torch.empty_like(slots_d) for _ in range(NBUF)]
-    pr_e = [torch.empty_like(pairs_d) for _ in range(NBUF)]
-    bt_e = [torch.empty_like(bt_d) for _ in range(NBUF)]
-    ln_e = [torch.empty_like(lens_d) for _ in range(NBUF)]
     copy_in = torch.cuda.Stream(dev)
     copy_out = torch.cuda.Stream(dev)
 
@@ -323,22 +336,24 @@ def cow_arm(args, rank, world, local_rank):
         if cw.shape[0] != n_pairs:
             raise RuntimeError("copy-on-write pair count changed")
         ev_h2d[b].synchronize()            # the H2D that last read these host buffers is done
-        sl_h[b].numpy()[:] = sl
-        pr_h[b].numpy()[:] = cw
-        bt_h[b].numpy()[:] = tb
-        ln_h[b].numpy()[:] = ln
+        sl_h, pr_h, bt_h, ln_h = tab_h[b][1]
+        sl_h.numpy()[:] = sl
+        pr_h.numpy()[:] = cw
+        bt_h.numpy()[:] = tb
+        ln_h.numpy()[:] = ln
         copy_in.wait_event(ev_done[b])     # buffer set b's kernels (two steps ago) are done
         with torch.cuda.stream(copy_in):
-            for d_, h_ in ((q_e[b], q_h), (kn_e[b], kn_h), (vn_e[b], vn_h), (sl_e[b], sl_h[b]),
-                           (pr_e[b], pr_h[b]), (bt_e[b], bt_h[b]), (ln_e[b], ln_h[b])):
-                d_.copy_(h_, non_blocking=True)
+            act_e[b][0].copy_(act_h, non_blocking=True)
+            tab_e[b][0].copy_(tab_h[b][0], non_blocking=True)
         ev_h2d[b].record(copy_in)
         stream.wait_event(ev_h2d[b])
         stream.wait_event(ev_d2h[b])       # out_e[b] has been read back
-        pkv.pkv_copy_blocks(kp, vp, pr_e[b], sp.num_kv_heads, sp.head_dim, sp.block_size,
+        q_d, kn_d, vn_d = act_e[b][1]
+        sl_d, pr_d, bt_dd, ln_d = tab_e[b][1]
+        pkv.pkv_copy_blocks(kp, vp, pr_d, sp.num_kv_heads, sp.head_dim, sp.block_size,
                             cs.num_blocks, dtype_code, stream=stream)
-        pkv.pkv_reshape_and_cache(kn_e[b], vn_e[b], kc, vc, sl_e[b], stream=stream)
-        pkv.pkv_paged_attention_decode(out_e[b], q_e[b], kc, vc, bt_e[b], ln_e[b], max_len,
+        pkv.pkv_reshape_and_cache(kn_d, vn_d, kc, vc, sl_d, stream=stream)
+        pkv.pkv_paged_attention_decode(out_e[b], q_d, kc, vc, bt_dd, ln_d, max_len,
                                        scale=1 / math.sqrt(sp.head_dim), partition_size=P,
                                        workspace=ws, stream=stream)
         ev_done[b].record(stream)
@@ -363,8 +378,7 @@ def cow_arm(args, rank, world, local_rank):
     e2e_ms = reduce_max(a.elapsed_time(b) / args.steps, dist, dev)
     mgr.close()
     peak, peak_kind = read_peaks()
-    h2d = ((q_h.numel() + kn_h.numel() + vn_h.numel()) * 2 + B * 8 + n_pairs * 8 +
-           bt_h[0].numel() * 4 + B * 4)
+    h2d = act_h.numel() + tab_h[0][0].numel()   # bytes of the two packed copies
     pmax = max(1, -(-max_len // P))
     return {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
@@ -385,8 +399,10 @@ def cow_arm(args, rank, world, local_rank):
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(out_h[0].numel() * 2),
                 "includes": "host batched frees, forks and appends (copy-on-write pairs), table "
-                            "export, pinned H2D, copy_blocks + cache write + decode, D2H; two "
-                            "steps in flight (double-buffered inputs and outputs)"},
+                            "export, pinned H2D (two packed copies: q / k_new / v_new, and "
+                            "slots / pairs / tables / lengths), copy_blocks + cache write + "
+                            "decode, D2H; two steps in flight (double-buffered inputs and "
+                            "outputs)"},
         "gpu_launches": args.steps * (3 + (1 if pmax > 1 else 0)),
     }
 
