@@ -609,3 +609,38 @@ def test_step_partitions_then_merge_equal_the_step(cuda_device, Hq, Hkv, D, BS, 
         assert np.array_equal(to_bits(out1), to_bits(out2)), rep
         assert torch.equal(kc1.view(torch.int16), kc2.view(torch.int16))
         assert torch.equal(vc1.view(torch.int16), vc2.view(torch.int16))
+
+
+def test_one_partition_steps_arm_and_reuse_the_header(cuda_device):
+    """Contexts that are one partition each (the automatic choice for up to 64 sequences of
+    short contexts with at least 1024 items): the first launch on a zero-filled workspace
+    runs the static schedule and arms the header, the next ones take their items from the
+    work counter; every launch equals the cache write + decode and the oracle."""
+    rng = np.random.default_rng(77)
+    dtype, Hq, Hkv, D, BS = synth.F16, 32, 32, 128, 16
+    lens = list(rng.integers(1, 1500, 40))
+    q, kc, vc, bt, lens, max_len, slots, kn, vn = step_case(rng, lens, Hq, Hkv, D, BS, dtype)
+    P = pkv.pkv_decode_partition_size(len(lens), Hq, Hkv, D, BS, max_len)
+    assert P >= max_len                                   # one partition per context
+    assert pkv.pkv_decode_step_launches(len(lens), Hq, Hkv, D, BS, max_len) == 1
+    ws = step_ws(q, kc, max_len, 0)
+    assert ws.numel() == 256                              # the header alone
+    ek, ev = C.reshape_and_cache(kn, vn, kc, vc, slots)
+    ref = A.paged_decode_attention(q, ek, ev, bt, lens, 1 / np.sqrt(D), dtype)
+    qd, knd, vnd = to_dev(q, dtype), to_dev(kn, dtype), to_dev(vn, dtype)
+    btd, lensd = torch.from_numpy(bt).cuda(), torch.from_numpy(lens).cuda()
+    pkv.pkv_get_device_status(clear=True)
+    first = None
+    for launch in range(4):
+        kcd, vcd = to_dev(kc, dtype), to_dev(vc, dtype)
+        out = torch.full_like(qd, float("nan"))
+        pkv.pkv_paged_decode_step(out, qd, knd, vnd, kcd, vcd, btd, lensd, max_len, ws)
+        torch.cuda.synchronize()
+        assert pkv.pkv_get_device_status() == 0
+        assert header(ws)[0].item() == K_SCHED_ARMED and header(ws)[1].item() == 0
+        assert np.array_equal(to_bits(kcd), ek) and np.array_equal(to_bits(vcd), ev)
+        if first is None:
+            first = to_bits(out)
+            assert_close(first, ref, dtype, "one-partition step")
+        else:
+            assert np.array_equal(to_bits(out), first), launch
