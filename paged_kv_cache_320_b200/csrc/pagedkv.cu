@@ -345,6 +345,26 @@ int launch_shared_decode(const CUtensorMap &mk, const CUtensorMap &mv,
     return launch(kern, dim3((unsigned)grid), dim3(pkv::kDecodeThreads), smem, st, mk, mv, prm);
 }
 
+// CTAs per SM of the shared-prefix decode launch (its shared memory against the SM's;
+// launch bounds allow two), for the plan's item placement.
+int shared_decode_slots(int D, int *slots) {
+    int dev;
+    if (current_device(&dev) != PKV_OK) return PKV_ERR_CUDA;
+    int cap = 0;
+    if (cudaDeviceGetAttribute(&cap, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) !=
+        cudaSuccess)
+        return PKV_ERR_CUDA;
+    const size_t smem =
+        D == 128 ? 1024 + pkv::DecodeLayout<128>::kRingBytes +
+                       pkv::DecodeLayout<128>::obuf_bytes(pkv::kMaxGroup) +
+                       pkv::DecodeLayout<128>::kMetaBytes
+                 : 1024 + pkv::DecodeLayout<64>::kRingBytes +
+                       pkv::DecodeLayout<64>::obuf_bytes(pkv::kMaxGroup) +
+                       pkv::DecodeLayout<64>::kMetaBytes;
+    *slots = (int)std::min<size_t>(2, (size_t)cap / (smem + 1024));
+    return PKV_OK;
+}
+
 int launch_shared_plan(const pkv::SharedParams &prm, cudaStream_t st) {
     const size_t plan_smem =
         prm.num_seqs <= pkv::kPlanSmemSeqs ? (size_t)7 * prm.num_seqs * sizeof(int) : 0;
@@ -978,6 +998,8 @@ int pkv_shared_prefix_plan(const int32_t *block_tables, const int32_t *context_l
     prm.group_start = group_start;
     prm.prefix_lens = prefix_lens;
     prm.num_groups = num_groups;
+    if ((rc = sm_count(&prm.sms)) != PKV_OK) return rc;
+    if ((rc = shared_decode_slots(head_dim, &prm.slots)) != PKV_OK) return rc;
     return launch_shared_plan(prm, reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -91,10 +91,12 @@ struct SharedParams {
     unsigned *status;
     int num_groups, num_seqs, num_heads, num_kv_heads, group;
     int max_blocks_per_seq, num_blocks, max_context_len, partition, block_size, max_items;
+    int sms, slots;      // the decode launch's SMs and CTAs per SM (item placement)
     float scale_log2;
 };
 
 constexpr int kPlanThreads = 1024;
+constexpr int kPlanBins = 1024;   // stage-count bins of the item placement (longer ones share the top)
 
 __device__ __forceinline__ int clamp_len(int len, int max_len) {
     return len < 0 ? 0 : (len > max_len ? max_len : len);
@@ -152,6 +154,7 @@ shared_prefix_plan_kernel(SharedParams p) {
     pdl_wait_and_release();
     extern __shared__ int plan_smem[];
     __shared__ int sm[kPlanThreads / 32];
+    __shared__ int plan_bins[kPlanBins];
     __shared__ int bad, max_pre_blocks;
     const int B = p.num_seqs, Hkv = p.num_kv_heads, G = p.group, P = p.partition;
     const int BS = p.block_size;
@@ -278,8 +281,8 @@ shared_prefix_plan_kernel(SharedParams p) {
         n_items += total;
     }
     __syncthreads();
-    // pass 5 (per item): chunk, KV head and part
-    for (int i = tid; i < n_items && i < p.max_items; i += kPlanThreads) {
+    // pass 5 (per item): chunk, KV head and part; the item's 64-token stages
+    auto make_item = [&](int i, int *stages) {
         const int ch = owner_of(item_base, n_chunks, i);
         const int g = owner_of(chunk_base, ng, ch);
         const int first = gfirst[g] + (ch - chunk_base[g]) * R;
@@ -298,7 +301,45 @@ shared_prefix_plan_kernel(SharedParams p) {
         it.part = local - it.hk * np;
         it.npp = npp;
         it.nps2 = nps2;
-        p.items[i] = it;
+        const int j = it.part, k = j - npp + (nps2 & 1);
+        int st = j < npp ? (min(P, pre - j * P) + kStageTokens - 1) / kStageTokens : 0;
+        if (k >= 0 && k < (nps2 >> 1))
+            for (int m = 0; m < it.nseq; ++m)
+                st += (max(0, min(P, slen[first + m] - pre - k * P)) + kStageTokens - 1) /
+                      kStageTokens;
+        *stages = max(st, 1);
+        return it;
+    };
+    // Placement: every CTA starts on the item at its own index and the launch's CTAs sit
+    // `slots` to an SM in index order (CTA c on SM c mod sms), so with no more items than
+    // CTAs the items of one SM run side by side. Items are ranked longest first (counting
+    // sort on stage counts); the sms longest go to the first slot of each SM and the
+    // others pair up longest with shortest in the second slots, which evens out the SMs'
+    // loads. With more items than CTAs, or another number of slots, the order is longest
+    // first. The placement moves items only: results do not depend on it.
+    for (int c = tid; c < kPlanBins; c += kPlanThreads) plan_bins[c] = 0;
+    __syncthreads();
+    const int n_put = min(n_items, p.max_items);
+    for (int i = tid; i < n_put; i += kPlanThreads) {
+        int st;
+        make_item(i, &st);
+        atomicAdd(&plan_bins[kPlanBins - 1 - min(st, kPlanBins - 1)], 1);   // longest first
+    }
+    __syncthreads();
+    {
+        int total;
+        const int v = tid < kPlanBins ? plan_bins[tid] : 0;
+        const int at = block_exclusive_scan(v, sm, &total);
+        if (tid < kPlanBins) plan_bins[tid] = at;
+    }
+    __syncthreads();
+    const bool paired = p.slots == 2 && n_put <= p.sms * 2 && n_put > p.sms;
+    for (int i = tid; i < n_put; i += kPlanThreads) {
+        int st;
+        const SharedItem it = make_item(i, &st);
+        const int r = atomicAdd(&plan_bins[kPlanBins - 1 - min(st, kPlanBins - 1)], 1);
+        const int pos = paired && r >= p.sms ? p.sms + (n_put - 1 - r) : r;
+        p.items[pos] = it;
     }
     __syncthreads();
     // pass 6 (per sequence): partials per (sequence, head) = its chunk's items, then the
