@@ -242,19 +242,19 @@ def cow_arm(args, rank, world, local_rank):
     kv_step = int(lens.astype(np.int64).sum()) * sp.num_kv_heads * sp.head_dim * 4
     ev = {"copy": [], "decode": []}
 
-    def step(record=False):
+    def step(record=False, s=stream):
         e = [torch.cuda.Event(enable_timing=True) for _ in range(3)] if record else None
         if record:
-            e[0].record(stream)
+            e[0].record(s)
         pkv.pkv_copy_blocks(kp, vp, pairs_d, sp.num_kv_heads, sp.head_dim, sp.block_size,
-                            cs.num_blocks, dtype_code, stream=stream)
-        pkv.pkv_reshape_and_cache(kn, vn, kc, vc, slots_d, stream=stream)
+                            cs.num_blocks, dtype_code, stream=s)
+        pkv.pkv_reshape_and_cache(kn, vn, kc, vc, slots_d, stream=s)
         if record:
-            e[1].record(stream)
+            e[1].record(s)
         pkv.pkv_paged_attention_decode(out, q, kc, vc, bt_d, lens_d, max_len, scale=1 / math.sqrt(
-            sp.head_dim), partition_size=P, workspace=ws, stream=stream)
+            sp.head_dim), partition_size=P, workspace=ws, stream=s)
         if record:
-            e[2].record(stream)
+            e[2].record(s)
             ev["copy"].append((e[0], e[1]))
             ev["decode"].append((e[1], e[2]))
 
@@ -270,13 +270,27 @@ def cow_arm(args, rank, world, local_rank):
     for _ in range(args.warmup):
         step()
     barrier()
+    # per-kernel split from eager steps with events between the launches
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step(record=True)
+    t1.record(stream)
+    barrier()
+    eager_ms = reduce_max(t0.elapsed_time(t1) / args.steps, dist, dev)
+    # the step as a CUDA graph replay (as the other workloads are timed)
+    g_step = record_graph(lambda s: step(s=s), dev, stream)
+    for _ in range(args.warmup):
+        g_step.replay()
+    barrier()
     with ClockSampler(local_rank) as clocks:
         barrier()
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
         for _ in range(args.steps):
-            step(record=True)
+            g_step.replay()
         t1.record(stream)
         barrier()
     ms_step = reduce_max(t0.elapsed_time(t1) / args.steps, dist, dev)
@@ -320,13 +334,31 @@ def cow_arm(args, rank, world, local_rank):
     tab_e = [packed(tab_parts, dev) for _ in range(NBUF)]
     out_h = [torch.empty(tuple(q.shape), dtype=dt, **pin) for _ in range(NBUF)]
     out_e = [torch.empty_like(out) for _ in range(NBUF)]
+
     copy_in = torch.cuda.Stream(dev)
     copy_out = torch.cuda.Stream(dev)
+
+    # The step's three kernels (copy_blocks, cache write, decode), recorded once per buffer
+    # set as a CUDA graph; the copies stay on their own streams so that they overlap the
+    # other buffer set's kernels.
+    def kernels(b):
+        def rec(s):
+            q_d, kn_d, vn_d = act_e[b][1]
+            sl_d, pr_d, bt_dd, ln_d = tab_e[b][1]
+            pkv.pkv_copy_blocks(kp, vp, pr_d, sp.num_kv_heads, sp.head_dim, sp.block_size,
+                                cs.num_blocks, dtype_code, stream=s)
+            pkv.pkv_reshape_and_cache(kn_d, vn_d, kc, vc, sl_d, stream=s)
+            pkv.pkv_paged_attention_decode(out_e[b], q_d, kc, vc, bt_dd, ln_d, max_len,
+                                           scale=1 / math.sqrt(sp.head_dim), partition_size=P,
+                                           workspace=ws, stream=s)
+        return rec
+
+    graphs = [record_graph(kernels(b), dev, stream) for b in range(NBUF)]
 
     def evs():
         return [torch.cuda.Event() for _ in range(NBUF)]
 
-    ev_h2d, ev_in, ev_done, ev_d2h = evs(), evs(), evs(), evs()
+    ev_h2d, ev_done, ev_d2h = evs(), evs(), evs()
     kstep = [0]
 
     def e2e_step():
@@ -348,14 +380,8 @@ def cow_arm(args, rank, world, local_rank):
         ev_h2d[b].record(copy_in)
         stream.wait_event(ev_h2d[b])
         stream.wait_event(ev_d2h[b])       # out_e[b] has been read back
-        q_d, kn_d, vn_d = act_e[b][1]
-        sl_d, pr_d, bt_dd, ln_d = tab_e[b][1]
-        pkv.pkv_copy_blocks(kp, vp, pr_d, sp.num_kv_heads, sp.head_dim, sp.block_size,
-                            cs.num_blocks, dtype_code, stream=stream)
-        pkv.pkv_reshape_and_cache(kn_d, vn_d, kc, vc, sl_d, stream=stream)
-        pkv.pkv_paged_attention_decode(out_e[b], q_d, kc, vc, bt_dd, ln_d, max_len,
-                                       scale=1 / math.sqrt(sp.head_dim), partition_size=P,
-                                       workspace=ws, stream=stream)
+        with torch.cuda.stream(stream):
+            graphs[b].replay()
         ev_done[b].record(stream)
         copy_out.wait_event(ev_done[b])
         with torch.cuda.stream(copy_out):
@@ -391,6 +417,11 @@ def cow_arm(args, rank, world, local_rank):
                    "parallelism": f"replicas x{world}"},
         "tokens_per_s": round(tokens_per_s, 1),
         "pct_of_hbm_peak": round(100 * value / world / peak, 2),
+        "timed": "CUDA graph replays of the step (copy_blocks, cache write, decode)",
+        "eager": {"value": round(weak_scaling_rates(kv_step, B, world, eager_ms)[0], 1),
+                  "unit": "GB/s", "ms_per_step": round(eager_ms, 4),
+                  "note": "the same steps launched one kernel at a time, with events between "
+                          "the launches (the copy / decode split below)"},
         "copy_and_write_us": round(copy_us, 2),
         "copy_blocks_bytes": copy_bytes,
         "decode_us": round(dec_us, 2),
@@ -401,8 +432,8 @@ def cow_arm(args, rank, world, local_rank):
                 "includes": "host batched frees, forks and appends (copy-on-write pairs), table "
                             "export, pinned H2D (two packed copies: q / k_new / v_new, and "
                             "slots / pairs / tables / lengths), copy_blocks + cache write + "
-                            "decode, D2H; two steps in flight (double-buffered inputs and "
-                            "outputs)"},
+                            "decode (one CUDA graph per buffer set), D2H; two steps in flight "
+                            "(double-buffered inputs and outputs, copies on their own streams)"},
         "gpu_launches": args.steps * (3 + (1 if pmax > 1 else 0)),
     }
 
