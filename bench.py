@@ -18,6 +18,8 @@ the step time is the maximum over ranks.
 from __future__ import annotations
 
 import argparse
+import contextlib
+import gc
 import hashlib
 import json
 import math
@@ -388,19 +390,20 @@ def cow_arm(args, rank, world, local_rank):
             out_h[b].copy_(out_e[b], non_blocking=True)
         ev_d2h[b].record(copy_out)
 
-    for _ in range(args.warmup):
-        e2e_step()
-    barrier()
-    a = torch.cuda.Event(enable_timing=True)
-    b = torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    copy_in.wait_event(a)
-    for _ in range(args.steps):
-        e2e_step()
-    stream.wait_stream(copy_out)
-    stream.wait_stream(copy_in)
-    b.record(stream)
-    barrier()
+    with host_loop():
+        for _ in range(args.warmup):
+            e2e_step()
+        barrier()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        copy_in.wait_event(a)
+        for _ in range(args.steps):
+            e2e_step()
+        stream.wait_stream(copy_out)
+        stream.wait_stream(copy_in)
+        b.record(stream)
+        barrier()
     e2e_ms = reduce_max(a.elapsed_time(b) / args.steps, dist, dev)
     mgr.close()
     peak, peak_kind = read_peaks()
@@ -433,7 +436,8 @@ def cow_arm(args, rank, world, local_rank):
                             "export, pinned H2D (two packed copies: q / k_new / v_new, and "
                             "slots / pairs / tables / lengths), copy_blocks + cache write + "
                             "decode (one CUDA graph per buffer set), D2H; two steps in flight "
-                            "(double-buffered inputs and outputs, copies on their own streams)"},
+                            "(double-buffered inputs and outputs, copies on their own streams); "
+                            "Python's garbage collector paused during the loop"},
         "gpu_launches": args.steps * (3 + (1 if pmax > 1 else 0)),
     }
 
@@ -453,6 +457,18 @@ def weak_scaling_rates(kv_bytes_per_rank_step, seqs_per_rank, world, ms_step):
     (the slowest rank's): K/V GB/s and decode tokens/s summed over ranks."""
     sec = ms_step * 1e-3
     return kv_bytes_per_rank_step * world / sec / 1e9, seqs_per_rank * world / sec
+
+
+@contextlib.contextmanager
+def host_loop():
+    """A latency-bound host loop: Python's cyclic garbage collector runs before it and is
+    paused during it (a collection in the middle of a step stalls the launches)."""
+    gc.collect()
+    gc.disable()
+    try:
+        yield
+    finally:
+        gc.enable()
 
 
 def record_graph(fn, dev, stream):
@@ -1085,23 +1101,24 @@ def e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, worl
         ev_step_done[b].record(stream)
         ev_d2h_done[b].record(copy_out)
 
-    for _ in range(args.warmup):
-        one_step()
-    torch.cuda.synchronize(dev)
-    barrier()
-    kv_total[0] = 0
-    host_s[0] = 0.0
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    copy_in.wait_event(t0)
-    for _ in range(args.steps):
-        one_step()
-    stream.wait_stream(copy_out)
-    stream.wait_stream(copy_in)
-    t1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
+    with host_loop():
+        for _ in range(args.warmup):
+            one_step()
+        torch.cuda.synchronize(dev)
+        barrier()
+        kv_total[0] = 0
+        host_s[0] = 0.0
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        copy_in.wait_event(t0)
+        for _ in range(args.steps):
+            one_step()
+        stream.wait_stream(copy_out)
+        stream.wait_stream(copy_in)
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
     ms = max_over_ranks(t0.elapsed_time(t1)) / args.steps
     if fused:
         # the device's tables and lengths must equal the host allocator's after all steps
@@ -1119,12 +1136,13 @@ def e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, worl
                          "list resident on the GPU; the host allocator mirrors it with one "
                          "batched call), pinned H2D of every layer's q/k_new/v_new, the fused "
                          "step's launches per layer, D2H of every layer's output; two steps in "
-                         "flight"
+                         "flight; Python's garbage collector paused during the loop"
                          if fused else
                          "host block-manager append (one batched call) and table export, pinned "
                          "H2D of slots/tables/lengths and every layer's q/k_new/v_new, all "
                          "layers' kernels, D2H of every layer's output; two steps in flight "
-                         "(double-buffered inputs and outputs)")}
+                         "(double-buffered inputs and outputs); Python's garbage collector "
+                         "paused during the loop")}
 
 
 # ----------------------------------------------------------------------------
@@ -1252,7 +1270,8 @@ CONFIG_WORKLOADS = [("llama3_8b_gqa", 16, "plain", 0), ("long_context", 8, "plai
 def run_configs(args, local_rank):
     """The other decode workloads at their own sizes, each timed like the headline
     workload: the step as CUDA graph replays, `steps` timed after `warmup`, its dominant
-    kernel alone, clocks sampled during its timed region."""
+    kernel alone, clocks sampled during its timed region; then the copy-on-write step
+    (copy_blocks, cache write, decode) with its end-to-end loop."""
     import torch
     out = {}
     for workload, bs, decode, layers in CONFIG_WORKLOADS:
@@ -1263,6 +1282,11 @@ def run_configs(args, local_rank):
                                       else "")
         out[key] = gpu_arm(sub, 0, 1, local_rank, light=True)
         torch.cuda.empty_cache()
+    sub = argparse.Namespace(**vars(args))
+    sub.workload, sub.block_size, sub.layers, sub.batch, sub.partition = \
+        "shared_prefix_cow", 0, 0, 0, 0
+    out["shared_prefix_cow_bs16"] = cow_arm(sub, 0, 1, local_rank)
+    torch.cuda.empty_cache()
     return out
 
 
@@ -1367,13 +1391,18 @@ def main(argv=None):
         # one process per GPU: start them under torch.distributed.run with these arguments
         return subprocess.call(launch_command(argv, args.gpus, free_port()))
 
+    # the default line (one GPU, the headline workload at its own sizes) also carries the
+    # other workloads, the copy-on-write step, the swap and the prefix-cache legs
+    full = (world == 1 and not args.no_configs and args.workload == "llama7b_mha"
+            and args.decode == "plain" and not args.block_size and not args.layers
+            and not args.batch and not args.partition)
+    if full:
+        args.swap = args.prefix_cache = True
     arm = cow_arm if args.workload == "shared_prefix_cow" else gpu_arm
     res = run_ranks(args, arm)
     if res is None:
         return 0
-    if (world == 1 and not args.no_configs and args.workload == "llama7b_mha"
-            and args.decode == "plain" and not args.block_size and not args.layers
-            and not args.batch and not args.partition):
+    if full:
         res["configs"] = run_configs(args, local_rank)
     if world == 1 and not args.no_cpu_baseline and args.workload != "shared_prefix_cow":
         res["cpu_baseline"] = cpu_baseline(args)
