@@ -296,6 +296,8 @@ def cow_arm(args, rank, world, local_rank):
         t1.record(stream)
         barrier()
     ms_step = reduce_max(t0.elapsed_time(t1) / args.steps, dist, dev)
+    percentiles = step_percentiles(g_step.replay, args.steps, stream, dev)
+    barrier()
     if pkv.pkv_get_device_status(stream=stream) != 0:
         raise RuntimeError("device status word set during the benchmark")
     copy_us = 1e3 * statistics.mean(a.elapsed_time(b) for a, b in ev["copy"])
@@ -421,6 +423,7 @@ def cow_arm(args, rank, world, local_rank):
         "tokens_per_s": round(tokens_per_s, 1),
         "pct_of_hbm_peak": round(100 * value / world / peak, 2),
         "timed": "CUDA graph replays of the step (copy_blocks, cache write, decode)",
+        "step_ms_percentiles": percentiles,
         "eager": {"value": round(weak_scaling_rates(kv_step, B, world, eager_ms)[0], 1),
                   "unit": "GB/s", "ms_per_step": round(eager_ms, 4),
                   "note": "the same steps launched one kernel at a time, with events between "
@@ -482,6 +485,27 @@ def record_graph(fn, dev, stream):
         fn(side)
     stream.wait_stream(side)
     return g
+
+
+def step_percentiles(run, steps, stream, dev):
+    """p10 / p50 / p90 of one step's time (ms): `steps` more steps, each between its own
+    CUDA events on `stream` (run after the timed region, on this rank)."""
+    import torch
+    pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(max(1, steps))]
+    with torch.cuda.stream(stream):
+        for a, b in pairs:
+            a.record(stream)
+            run()
+            b.record(stream)
+    torch.cuda.synchronize(dev)
+    per = sorted(a.elapsed_time(b) for a, b in pairs)
+
+    def q(f):
+        return round(per[min(len(per) - 1, int(round(f * (len(per) - 1))))], 4)
+
+    return {"p10": q(0.1), "p50": q(0.5), "p90": q(0.9), "n": len(per),
+            "timed": "each step between its own CUDA events, after the timed region"}
 
 
 def time_replays(g, replays, stream):
@@ -673,6 +697,10 @@ def gpu_arm(args, rank, world, local_rank, light=False):
         for name, g in graphs.items():
             ms[name] = time_replays(g, args.steps, stream)
             barrier()
+    g_step = graphs.get("step")
+    percentiles = step_percentiles(g_step.replay if g_step is not None else lambda: step(stream),
+                                   args.steps, stream, dev)
+    barrier()
     graphs.clear()
     if pkv.pkv_get_device_status(stream=stream) != 0:
         raise RuntimeError("device status word set during the benchmark")
@@ -737,6 +765,7 @@ def gpu_arm(args, rank, world, local_rank, light=False):
                         "roofline counts the bytes the path must read (each shared prefix once "
                         "per KV head, every private suffix)"} if shared else {}),
             "eager": {"value": round(eager_value, 1), "ms_per_step": round(ms["eager"], 4)},
+            "step_ms_percentiles": percentiles,
             "roofline": roofline, "clocks": clocks.summary()}
 
     roofline["hbm_read_probe_gbs"] = round(hbm_read_probe(dev, stream), 1)
@@ -786,6 +815,7 @@ def gpu_arm(args, rank, world, local_rank, light=False):
         "eager": {"value": round(eager_value, 1), "unit": "GB/s",
                   "ms_per_step": round(ms["eager"], 4),
                   "note": "the same steps launched one kernel at a time (no graph)"},
+        "step_ms_percentiles": percentiles,
         **({"swap_blocks": swap} if swap else {}),
         **({"prefix_cache": prefix_cache} if prefix_cache else {}),
         "clocks": clocks.summary(),
