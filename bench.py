@@ -203,7 +203,10 @@ def cow_arm(args, rank, world, local_rank):
     kid_parents = np.repeat(np.array(parents, np.int64), samples)
     live = [False]
 
-    def host_step():
+    def host_step(**outs):
+        """Frees the samples (after the first step), forks them again from their parents and
+        appends one token to each, exporting their tables in the same call (into the given
+        arrays, e.g. views of a pinned buffer, when there are any)."""
         if live[0]:
             st, done = mgr.pkv_seq_free_batch(kids)
             if st != 0:
@@ -212,11 +215,10 @@ def cow_arm(args, rank, world, local_rank):
         if st != 0:
             raise RuntimeError(f"fork failed ({st})")
         live[0] = True
-        st, done, slots, cows = mgr.pkv_seq_append_batch(kids, 1)
+        st, done, slots, cows, tables, lens = mgr.pkv_seq_append_tables(kids, 1, **outs)
         if st != 0:
             raise RuntimeError(f"append failed ({st})")
-        st, tables, lens = mgr.pkv_block_tables(kids)
-        return slots[:, 0].copy(), cows.copy(), tables, lens
+        return slots[:, 0], cows, tables, lens
 
     dt = synth.torch_dtype(sp.dtype)
 
@@ -228,7 +230,7 @@ def cow_arm(args, rank, world, local_rank):
     out = torch.empty_like(q)
     kp = torch.tensor([kc.data_ptr()], dtype=torch.int64, device=dev)
     vp = torch.tensor([vc.data_ptr()], dtype=torch.int64, device=dev)
-    slots, cows, tables, lens = host_step()
+    slots, cows, tables, lens = (x.copy() for x in host_step())
     n_pairs = cows.shape[0]
     max_len = cs.max_blocks_per_seq * sp.block_size
     P = pkv.pkv_decode_partition_size(B, sp.num_heads, sp.num_kv_heads, sp.head_dim,
@@ -329,7 +331,7 @@ def cow_arm(args, rank, world, local_rank):
     # this step's query and new K/V rows (one H2D copy), and the host block manager's
     # results (slots, copy-on-write pairs, tables, lengths: one H2D copy)
     act_parts = [(tuple(q.shape), dt), (tuple(kn.shape), dt), (tuple(vn.shape), dt)]
-    tab_parts = [((B,), torch.int64), ((n_pairs, 2), torch.int32), (tuple(tables.shape), torch.int32),
+    tab_parts = [((B,), torch.int64), ((B, 2), torch.int32), (tuple(tables.shape), torch.int32),
                  ((B,), torch.int32)]
     act_h, (q_h, kn_h, vn_h) = packed(act_parts)
     q_h.copy_(q.cpu()); kn_h.copy_(kn.cpu()); vn_h.copy_(vn.cpu())
@@ -349,8 +351,8 @@ def cow_arm(args, rank, world, local_rank):
         def rec(s):
             q_d, kn_d, vn_d = act_e[b][1]
             sl_d, pr_d, bt_dd, ln_d = tab_e[b][1]
-            pkv.pkv_copy_blocks(kp, vp, pr_d, sp.num_kv_heads, sp.head_dim, sp.block_size,
-                                cs.num_blocks, dtype_code, stream=s)
+            pkv.pkv_copy_blocks(kp, vp, pr_d[:n_pairs], sp.num_kv_heads, sp.head_dim,
+                                sp.block_size, cs.num_blocks, dtype_code, stream=s)
             pkv.pkv_reshape_and_cache(kn_d, vn_d, kc, vc, sl_d, stream=s)
             pkv.pkv_paged_attention_decode(out_e[b], q_d, kc, vc, bt_dd, ln_d, max_len,
                                            scale=1 / math.sqrt(sp.head_dim), partition_size=P,
@@ -365,18 +367,21 @@ def cow_arm(args, rank, world, local_rank):
     ev_h2d, ev_done, ev_d2h = evs(), evs(), evs()
     kstep = [0]
 
+    # the block manager writes slots, pairs, tables and lengths straight into the pinned
+    # buffer set of the step
+    tab_np = []
+    for b in range(NBUF):
+        sl_h, pr_h, bt_h, ln_h = tab_h[b][1]
+        tab_np.append(dict(slots_out=sl_h.numpy().reshape(B, 1), cows_out=pr_h.numpy(),
+                           tables_out=bt_h.numpy(), lens_out=ln_h.numpy()))
+
     def e2e_step():
         b = kstep[0] % NBUF
         kstep[0] += 1
-        sl, cw, tb, ln = host_step()
+        ev_h2d[b].synchronize()            # the H2D that last read these host buffers is done
+        sl, cw, tb, ln = host_step(**tab_np[b])
         if cw.shape[0] != n_pairs:
             raise RuntimeError("copy-on-write pair count changed")
-        ev_h2d[b].synchronize()            # the H2D that last read these host buffers is done
-        sl_h, pr_h, bt_h, ln_h = tab_h[b][1]
-        sl_h.numpy()[:] = sl
-        pr_h.numpy()[:] = cw
-        bt_h.numpy()[:] = tb
-        ln_h.numpy()[:] = ln
         copy_in.wait_event(ev_done[b])     # buffer set b's kernels (two steps ago) are done
         with torch.cuda.stream(copy_in):
             act_e[b][0].copy_(act_h, non_blocking=True)
@@ -435,8 +440,9 @@ def cow_arm(args, rank, world, local_rank):
         "e2e": {"value": round(kv_step * world / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(out_h[0].numel() * 2),
-                "includes": "host batched frees, forks and appends (copy-on-write pairs), table "
-                            "export, pinned H2D (two packed copies: q / k_new / v_new, and "
+                "includes": "host batched frees, forks and appends (copy-on-write pairs) with "
+                            "the table export in the same call, written into the pinned buffer; "
+                            "pinned H2D (two packed copies: q / k_new / v_new, and "
                             "slots / pairs / tables / lengths), copy_blocks + cache write + "
                             "decode (one CUDA graph per buffer set), D2H; two steps in flight "
                             "(double-buffered inputs and outputs, copies on their own streams); "
@@ -1082,16 +1088,16 @@ def e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, worl
             if st != 0 or len(cows):
                 raise RuntimeError(f"host mirror append failed ({st})")
         else:
-            st, done, sl, cows = mgr.pkv_seq_append_batch(ids, 1)
+            ev_tables[b].synchronize()      # the H2D that last read these host buffers is done
+            th = time.perf_counter()
+            # appends and table export in one call, written into the pinned buffers
+            st, done, sl, cows, tables, lens = mgr.pkv_seq_append_tables(
+                ids, 1, slots_out=slots_h[b].numpy().reshape(B, 1), tables_out=bt_h[b].numpy(),
+                lens_out=lens_h[b].numpy())
             if st != 0 or len(cows):
                 raise RuntimeError(f"append failed ({st}) or needed a copy in an unshared workload")
-            st, tables, lens = mgr.pkv_block_tables(ids)
             host_s[0] += time.perf_counter() - th
             th = None
-            ev_tables[b].synchronize()      # the H2D that last read these host buffers is done
-            slots_h[b].numpy()[:] = sl[:, 0]
-            bt_h[b].numpy()[:] = tables
-            lens_h[b].numpy()[:] = lens
         if th is not None:
             host_s[0] += time.perf_counter() - th
         mirror_lens[:] += 1
@@ -1168,8 +1174,8 @@ def e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, worl
                          "step's launches per layer, D2H of every layer's output; two steps in "
                          "flight; Python's garbage collector paused during the loop"
                          if fused else
-                         "host block-manager append (one batched call) and table export, pinned "
-                         "H2D of slots/tables/lengths and every layer's q/k_new/v_new, all "
+                         "host block-manager append and table export (one call, into the pinned "
+                         "buffers), pinned H2D of slots/tables/lengths and every layer's q/k_new/v_new, all "
                          "layers' kernels, D2H of every layer's output; two steps in flight "
                          "(double-buffered inputs and outputs); Python's garbage collector "
                          "paused during the loop")}

@@ -437,6 +437,17 @@ int pkv_seq_append_batch(pkv_alloc *a, const int64_t *seq_ids, int n, int n_toke
                          int64_t *slots_out, int32_t *cow_pairs_out, int *n_cow_out,
                          int *n_done_out);
 
+/* A decode step's host work in one call: pkv_seq_append_batch (same arguments, same results)
+ * and then, if every append succeeded, pkv_block_tables of the same sequences into host
+ * tables_out [n][max_blocks_per_seq] (unused entries -1) and lens_out [n] (may be NULL).
+ * "分页 KV Cache 分析" §2.3: each step the block manager extends every running sequence,
+ * handing out a page when its last one is full, and the kernel reads the updated tables.
+ * On a failed append the tables are not written. Errors: those of pkv_seq_append_batch;
+ * PKV_ERR_INVALID_ARG (tables_out NULL with n > 0: nothing changes). */
+int pkv_seq_append_tables(pkv_alloc *a, const int64_t *seq_ids, int n, int n_tokens,
+                          int64_t *slots_out, int32_t *cow_pairs_out, int *n_cow_out,
+                          int *n_done_out, int32_t *tables_out, int32_t *lens_out);
+
 /* Errors: PKV_ERR_UNKNOWN_SEQ (no parent), PKV_ERR_SEQ_EXISTS (child id in use). */
 int pkv_seq_fork(pkv_alloc *a, int64_t parent, int64_t child);
 

@@ -85,6 +85,8 @@ def lib() -> ctypes.CDLL:
         L.pkv_seq_append.argtypes = [P, I64, I, P, P, ctypes.POINTER(I)]
         L.pkv_seq_append_batch.argtypes = [P, P, I, I, P, P, ctypes.POINTER(I),
                                            ctypes.POINTER(I)]
+        L.pkv_seq_append_tables.argtypes = [P, P, I, I, P, P, ctypes.POINTER(I),
+                                            ctypes.POINTER(I), P, P]
         L.pkv_seq_fork.argtypes = [P, I64, I64]
         L.pkv_seq_free.argtypes = [P, I64]
         L.pkv_block_tables.argtypes = [P, P, I, P, P]
@@ -125,7 +127,8 @@ def lib() -> ctypes.CDLL:
                      "pkv_seq_fork_batch",
                      "pkv_seq_free_batch", "pkv_shared_prefix_plan",
                      "pkv_paged_attention_decode_shared_prefix_planned",
-                     "pkv_seq_append_tokens", "pkv_seq_share_prefix", "pkv_prefix_cache_stats"):
+                     "pkv_seq_append_tokens", "pkv_seq_share_prefix", "pkv_prefix_cache_stats",
+                     "pkv_seq_append_tables"):
             getattr(L, name).restype = I
         _lib = L
     return _lib
@@ -593,6 +596,38 @@ class BlockManager:
                                         slots.ctypes.data, cows.ctypes.data,
                                         ctypes.byref(n_cow), ctypes.byref(n_done))
         return rc, n_done.value, slots[:n, :n_tokens], cows[:n_cow.value]
+
+    def pkv_seq_append_tables(self, seq_ids, n_tokens, slots_out=None, cows_out=None,
+                              tables_out=None, lens_out=None):
+        """pkv_seq_append_batch then, if it succeeded, pkv_block_tables of the same sequences,
+        in one call. Returns (status, n_done, slots [n, n_tokens], cow pairs [k, 2], tables
+        [n, max_blocks_per_seq], lens [n]). Each output may be given as a writable C-contiguous
+        array of the right dtype and shape (e.g. a view of a pinned host buffer; cows_out with
+        room for n * n_tokens pairs): the library then writes into it."""
+        import numpy as np
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        n = ids.shape[0]
+        mb = self.max_blocks_per_seq
+
+        def out(arr, shape, dtype, what):
+            if arr is None:
+                return np.zeros(shape, dtype=dtype)
+            if (not isinstance(arr, np.ndarray) or arr.dtype != dtype or tuple(arr.shape) != shape
+                    or not arr.flags.c_contiguous or not arr.flags.writeable):
+                raise ValueError(f"{what} must be a writable C-contiguous {np.dtype(dtype)} "
+                                 f"array of shape {shape}")
+            return arr
+
+        slots = out(slots_out, (n, int(n_tokens)), np.int64, "slots_out")
+        cows = out(cows_out, (n * int(n_tokens), 2), np.int32, "cows_out")
+        tables = out(tables_out, (n, mb), np.int32, "tables_out")
+        lens = out(lens_out, (n,), np.int32, "lens_out")
+        n_cow, n_done = ctypes.c_int(0), ctypes.c_int(0)
+        rc = lib().pkv_seq_append_tables(self._h, ids.ctypes.data, n, int(n_tokens),
+                                         slots.ctypes.data, cows.ctypes.data,
+                                         ctypes.byref(n_cow), ctypes.byref(n_done),
+                                         tables.ctypes.data, lens.ctypes.data)
+        return rc, n_done.value, slots, cows[:n_cow.value], tables, lens
 
     def pkv_alloc_free_list(self, max_out=None):
         """Blocks the next allocations would take, in order (int32 array)."""

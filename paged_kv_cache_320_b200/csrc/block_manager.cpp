@@ -377,6 +377,18 @@ int pkv_seq_append_batch(pkv_alloc *a, const int64_t *seq_ids, int n, int n_toke
     return PKV_OK;
 }
 
+int pkv_seq_append_tables(pkv_alloc *a, const int64_t *seq_ids, int n, int n_tokens,
+                          int64_t *slots_out, int32_t *cow_pairs_out, int *n_cow_out,
+                          int *n_done_out, int32_t *tables_out, int32_t *lens_out) {
+    if (n_done_out) *n_done_out = 0;
+    if (n_cow_out) *n_cow_out = 0;
+    if (n > 0 && !tables_out) return PKV_ERR_INVALID_ARG;
+    const int rc = pkv_seq_append_batch(a, seq_ids, n, n_tokens, slots_out, cow_pairs_out,
+                                        n_cow_out, n_done_out);
+    if (rc != PKV_OK) return rc;
+    return pkv_block_tables(a, seq_ids, n, tables_out, lens_out);
+}
+
 int pkv_seq_fork(pkv_alloc *a, int64_t parent, int64_t child) {
     return guarded([&]() -> int {
         if (!a) return PKV_ERR_INVALID_ARG;

@@ -133,6 +133,81 @@ def test_batched_append_equals_appends_in_order(seed):
 
 
 @pytest.mark.parametrize("seed", range(30))
+def test_append_with_tables_equals_the_model(seed):
+    """pkv_seq_append_tables == the model's appends in order, then its block tables and
+    lengths of the same sequences; on a failed append the caller's tables are untouched
+    and the sequences before the failing one keep their appends. Outputs written into
+    caller arrays (as into a pinned buffer) equal the returned ones."""
+    rng = np.random.default_rng(900 + seed)
+    nb, bs, mb = int(rng.integers(6, 30)), int(rng.choice([2, 4, 8])), int(rng.integers(2, 6))
+    order = rng.permutation(nb)
+    c = BlockManager(nb, bs, mb, order)
+    m = BM.BlockManagerModel(nb, bs, mb, order)
+    for s in range(4):
+        n0 = int(rng.integers(1, bs * 2))
+        assert c.pkv_seq_append(s, n0)[0] == m.append(s, n0)[0]
+    if rng.random() < 0.5:
+        assert c.pkv_seq_fork(0, 7) == m.fork(0, 7)
+    for _ in range(6):
+        ids = [int(x) for x in rng.choice([0, 1, 2, 3, 7, 9], size=int(rng.integers(1, 6)))]
+        k = int(rng.integers(0, 3))
+        given = rng.random() < 0.5
+        outs = {}
+        if given:
+            outs = dict(slots_out=np.full((len(ids), k), -7, np.int64),
+                        cows_out=np.full((len(ids) * k, 2), -7, np.int32),
+                        tables_out=np.full((len(ids), mb), -7, np.int32),
+                        lens_out=np.full(len(ids), -7, np.int32))
+        st, done, slots, cows, tables, lens = c.pkv_seq_append_tables(ids, k, **outs)
+        exp_slots, exp_cows, exp_done, exp_st = [], [], 0, 0
+        for sid in ids:
+            s2, sl, cw = m.append(sid, k)
+            if s2 != 0:
+                exp_st = s2
+                break
+            exp_slots.append(sl)
+            exp_cows += [list(x) for x in cw]
+            exp_done += 1
+        assert st == exp_st and done == exp_done
+        for i in range(done):
+            assert slots[i].tolist() == exp_slots[i]
+        assert cows.tolist() == exp_cows
+        if st == 0:
+            for i, sid in enumerate(ids):
+                row, n = m.block_table(sid)
+                assert tables[i].tolist() == row and lens[i] == n
+        elif given:
+            assert (outs["tables_out"] == -7).all() and (outs["lens_out"] == -7).all()
+        if given:
+            assert outs["tables_out"] is tables and outs["slots_out"] is slots
+        compare_states(c, m, sorted(m.tables))
+    c.close()
+
+
+def test_append_with_tables_rejects_missing_or_wrong_outputs():
+    c = BlockManager(16, 4, 4)
+    assert c.pkv_seq_append(1, 3)[0] == 0
+    with pytest.raises(ValueError):
+        c.pkv_seq_append_tables([1], 1, tables_out=np.zeros((1, 3), np.int32))   # shape
+    with pytest.raises(ValueError):
+        c.pkv_seq_append_tables([1], 1, slots_out=np.zeros((1, 1), np.int32))    # dtype
+    from paged_kv_cache_320_b200 import _binding as B
+    import ctypes
+    # the C call refuses a missing tables_out before changing anything
+    ids = np.array([1], np.int64)
+    slots = np.zeros(1, np.int64)
+    cows = np.zeros((1, 2), np.int32)
+    n_cow, done = ctypes.c_int(0), ctypes.c_int(0)
+    rc = B.lib().pkv_seq_append_tables(c._h, ids.ctypes.data, 1, 1, slots.ctypes.data,
+                                       cows.ctypes.data, ctypes.byref(n_cow), ctypes.byref(done),
+                                       None, None)
+    assert rc == B.PKV_ERR_INVALID_ARG
+    st, tables, lens = c.pkv_block_tables([1])
+    assert lens.tolist() == [3]
+    c.close()
+
+
+@pytest.mark.parametrize("seed", range(30))
 def test_batched_fork_and_free_equal_calls_in_order(seed):
     """pkv_seq_fork_batch / pkv_seq_free_batch == the single calls in order, against the
     model; on the first failure the calls before it keep their effects."""
