@@ -988,12 +988,22 @@ def swap_measurement(wl, dev, stream, budget=512 << 20, reps=5):
                                                stream=stream)
     out_gbs = timed(lambda: swap(1))
     in_gbs = timed(lambda: swap(0))
+    # the same swap through a 64 MiB device staging buffer and one large copy per chunk
+    staging = torch.empty(64 << 20, dtype=torch.uint8, device=dev)
+    staged = lambda to_host: pkv.pkv_swap_blocks_staged(
+        kp, vp, ids_d, host, to_host, sp.num_kv_heads, sp.head_dim, sp.block_size,
+        wl.num_blocks, code, staging, stream=stream)
+    staged_out_gbs = timed(lambda: staged(1))
+    staged_in_gbs = timed(lambda: staged(0))
+    del staging
     dbuf = torch.empty(nbytes // 2, dtype=torch.int16, device=dev)
     with torch.cuda.stream(stream):
         d2h = timed(lambda: host.copy_(dbuf, non_blocking=True))
         h2d = timed(lambda: dbuf.copy_(host, non_blocking=True))
     return {"sequences": len(seqs), "blocks": len(ids), "bytes": nbytes,
             "out_gbs": round(out_gbs, 1), "in_gbs": round(in_gbs, 1),
+            "staged_out_gbs": round(staged_out_gbs, 1), "staged_in_gbs": round(staged_in_gbs, 1),
+            "staging_bytes": 64 << 20,
             "contiguous_d2h_gbs": round(d2h, 1), "contiguous_h2d_gbs": round(h2d, 1)}
 
 

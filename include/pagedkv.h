@@ -298,6 +298,23 @@ int pkv_swap_blocks(void *const *k_caches, void *const *v_caches, int num_layers
                     size_t host_buffer_bytes, int to_host, int num_kv_heads, int head_dim,
                     int block_size, int num_blocks, int dtype, pkv_stream_t stream);
 
+/* The same swap (same arguments, same host buffer layout and contents) moved in large
+ * copies: the listed tiles are gathered into (or scattered from) `staging`, a DEVICE buffer
+ * of staging_bytes (16-byte aligned, at least one tile = Hkv*BS*D*2 bytes), and each full
+ * staging buffer crosses the host link as one cudaMemcpyAsync, so the link runs at the rate
+ * of its copy engine rather than of the SMs' stores to mapped memory. Chunks follow one
+ * another on `stream` (a gather or scatter launch and one copy per floor(staging_bytes /
+ * tile) tiles). host_buffer must be pinned host memory (the copies are asynchronous only
+ * from it). Tiles of ids outside [0, num_blocks) set PKV_STATUS_BAD_PAIR and are zero in
+ * the host buffer (to_host = 1) or not written (to_host = 0). Errors: as pkv_swap_blocks;
+ * PKV_ERR_WORKSPACE (staging missing, misaligned or smaller than a tile); PKV_ERR_INVALID_ARG
+ * (staging not device memory). */
+int pkv_swap_blocks_staged(void *const *k_caches, void *const *v_caches, int num_layers,
+                           const int32_t *block_ids, int num_ids, void *host_buffer,
+                           size_t host_buffer_bytes, int to_host, int num_kv_heads,
+                           int head_dim, int block_size, int num_blocks, int dtype,
+                           void *staging, size_t staging_bytes, pkv_stream_t stream);
+
 /* ------------------------------------------------------------------------------
  * Decode step on the device ("分页 KV Cache 分析" §3.1: each decode step writes the new
  * token's K/V into its page, then attention reads the pages; §2.3: the block manager

@@ -29,5 +29,6 @@ from ._binding import (  # noqa: F401
     pkv_decode_shared_prefix_workspace_size,
     pkv_reshape_and_cache,
     pkv_swap_blocks,
+    pkv_swap_blocks_staged,
 )
 from ._binding import PKV_BF16, PKV_F16  # noqa: F401

@@ -80,6 +80,7 @@ def lib() -> ctypes.CDLL:
         L.pkv_copy_blocks.argtypes = [P, P, I, P, I, I, I, I, I, I, P]
         L.pkv_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), I, P]
         L.pkv_swap_blocks.argtypes = [P, P, I, P, I, P, SZ, I, I, I, I, I, I, P]
+        L.pkv_swap_blocks_staged.argtypes = [P, P, I, P, I, P, SZ, I, I, I, I, I, I, P, SZ, P]
         L.pkv_alloc_create.argtypes = [ctypes.POINTER(P), I, I, I, P]
         L.pkv_alloc_destroy.argtypes = [P]
         L.pkv_seq_append.argtypes = [P, I64, I, P, P, ctypes.POINTER(I)]
@@ -128,7 +129,7 @@ def lib() -> ctypes.CDLL:
                      "pkv_seq_free_batch", "pkv_shared_prefix_plan",
                      "pkv_paged_attention_decode_shared_prefix_planned",
                      "pkv_seq_append_tokens", "pkv_seq_share_prefix", "pkv_prefix_cache_stats",
-                     "pkv_seq_append_tables"):
+                     "pkv_seq_append_tables", "pkv_swap_blocks_staged"):
             getattr(L, name).restype = I
         _lib = L
     return _lib
@@ -537,6 +538,24 @@ def pkv_swap_blocks(k_cache_ptrs, v_cache_ptrs, block_ids, host_buffer, to_host,
                                  _nbytes(host_buffer), int(to_host),
                                  num_kv_heads, head_dim, block_size, num_blocks, dtype,
                                  _stream(stream)), "pkv_swap_blocks")
+
+
+def pkv_swap_blocks_staged(k_cache_ptrs, v_cache_ptrs, block_ids, host_buffer, to_host,
+                           num_kv_heads, head_dim, block_size, num_blocks, dtype, staging,
+                           stream=None):
+    """pkv_swap_blocks through a device staging tensor (uint8, CUDA) and large copies (see
+    pagedkv.h)."""
+    import torch
+    n = block_ids.numel()
+    _cache_ptrs(k_cache_ptrs, v_cache_ptrs)
+    _need(block_ids, "block_ids", k_cache_ptrs.device, torch.int32)
+    _need(staging, "staging", k_cache_ptrs.device, torch.uint8)
+    _check(lib().pkv_swap_blocks_staged(_ptr(k_cache_ptrs), _ptr(v_cache_ptrs),
+                                        k_cache_ptrs.numel(), _ptr(block_ids), n,
+                                        _ptr(host_buffer), _nbytes(host_buffer), int(to_host),
+                                        num_kv_heads, head_dim, block_size, num_blocks, dtype,
+                                        _ptr(staging), _nbytes(staging), _stream(stream)),
+           "pkv_swap_blocks_staged")
 
 
 def pkv_get_device_status(clear=True, stream=None) -> int:

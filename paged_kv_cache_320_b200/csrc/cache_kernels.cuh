@@ -104,4 +104,41 @@ swap_blocks_kernel(void *const *__restrict__ k_caches, void *const *__restrict__
     for (; t < block_vecs; t += 256) dst[t] = src[t];
 }
 
+// Staged swap: tiles t0 .. t0 + count - 1 of the swap's flat order (tile t = the block
+// block_ids[t % n_blocks] of layer (t / n_blocks) / 2, K for even t / n_blocks, V for odd,
+// the host buffer's order) between the caches and a device staging buffer, one CTA per
+// tile, so that each chunk crosses the host link as one large copy.
+//   to_staging = 1: staging[j] = tile t0 + j   (a tile with a bad id is zero-filled)
+//   to_staging = 0: tile t0 + j = staging[j]    (a tile with a bad id is not written)
+__global__ void __launch_bounds__(256)
+swap_stage_kernel(void *const *__restrict__ k_caches, void *const *__restrict__ v_caches,
+                  const int32_t *__restrict__ block_ids, int n_blocks, uint4 *staging,
+                  long long t0, int num_blocks, int block_vecs, int to_staging,
+                  unsigned *status) {
+    pdl_wait_and_release();
+    const long long t = t0 + blockIdx.x;
+    const long long lk = t / n_blocks;
+    const int i = (int)(t - lk * n_blocks);
+    const int layer = (int)(lk >> 1);
+    const int kv = (int)(lk & 1);
+    const int b = block_ids[i];
+    uint4 *st = staging + (long long)blockIdx.x * block_vecs;
+    if (b < 0 || b >= num_blocks) {
+        if (threadIdx.x == 0 && kv == 0 && layer == 0) atomicOr(status, 2u /* bad pair */);
+        if (to_staging)
+            for (int v = threadIdx.x; v < block_vecs; v += 256) st[v] = make_uint4(0, 0, 0, 0);
+        return;
+    }
+    uint4 *cache = reinterpret_cast<uint4 *>(kv ? v_caches[layer] : k_caches[layer]) +
+                   (long long)b * block_vecs;
+    const uint4 *src = to_staging ? cache : st;
+    uint4 *dst = to_staging ? st : cache;
+    int v = threadIdx.x;
+    for (; v + 3 * 256 < block_vecs; v += 4 * 256) {
+        const uint4 a = src[v], c = src[v + 256], d = src[v + 512], e = src[v + 768];
+        dst[v] = a; dst[v + 256] = c; dst[v + 512] = d; dst[v + 768] = e;
+    }
+    for (; v < block_vecs; v += 256) dst[v] = src[v];
+}
+
 }  // namespace pkv

@@ -1168,6 +1168,69 @@ int pkv_swap_blocks(void *const *k_caches, void *const *v_caches, int num_layers
                   status);
 }
 
+int pkv_swap_blocks_staged(void *const *k_caches, void *const *v_caches, int num_layers,
+                           const int32_t *block_ids, int num_ids, void *host_buffer,
+                           size_t host_buffer_bytes, int to_host, int num_kv_heads,
+                           int head_dim, int block_size, int num_blocks, int dtype,
+                           void *staging, size_t staging_bytes, pkv_stream_t stream) {
+    if (num_ids < 0 || num_layers < 1 || num_layers > 65535 || num_kv_heads < 1 ||
+        num_blocks < 1 || (to_host != 0 && to_host != 1))
+        return PKV_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return PKV_ERR_INVALID_ARG;
+    if (block_size != 8 && block_size != 16 && block_size != 32) return PKV_ERR_INVALID_ARG;
+    if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_ERR_INVALID_ARG;
+    if (num_ids == 0) return PKV_OK;
+    if (!k_caches || !v_caches || !block_ids || !host_buffer || !aligned(host_buffer, 16))
+        return PKV_ERR_INVALID_ARG;
+    const long long vecs = (long long)num_kv_heads * block_size * head_dim * 2 / 16;
+    if (vecs >= INT_MAX) return PKV_ERR_INVALID_ARG;
+    const unsigned long long tile = (unsigned long long)vecs * 16;
+    const long long total = (long long)num_layers * 2 * num_ids;
+    if (host_buffer_bytes < (unsigned long long)total * tile) return PKV_ERR_INVALID_ARG;
+    if (!staging || !aligned(staging, 16) || staging_bytes < tile) return PKV_ERR_WORKSPACE;
+    // the copies are asynchronous only from pinned memory: anything else is refused
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, host_buffer) != cudaSuccess) {
+        cudaGetLastError();
+        return PKV_ERR_INVALID_ARG;
+    }
+    if (attr.type != cudaMemoryTypeHost) return PKV_ERR_INVALID_ARG;
+    if (cudaPointerGetAttributes(&attr, staging) != cudaSuccess) {
+        cudaGetLastError();
+        return PKV_ERR_INVALID_ARG;
+    }
+    if (attr.type != cudaMemoryTypeDevice) return PKV_ERR_INVALID_ARG;
+    unsigned int *status;
+    int rc;
+    if ((rc = device_status_ptr(&status)) != PKV_OK) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const long long per = (long long)std::min<unsigned long long>(staging_bytes / tile, INT_MAX);
+    char *host = static_cast<char *>(host_buffer);
+    for (long long t0 = 0; t0 < total; t0 += per) {
+        const long long cnt = std::min(per, total - t0);
+        char *h = host + (unsigned long long)t0 * tile;
+        const size_t bytes = (size_t)((unsigned long long)cnt * tile);
+        if (to_host) {
+            if ((rc = launch(pkv::swap_stage_kernel, dim3((unsigned)cnt), dim3(256), 0, st,
+                             k_caches, v_caches, block_ids, num_ids,
+                             static_cast<uint4 *>(staging), t0, num_blocks, (int)vecs, 1,
+                             status)) != PKV_OK)
+                return rc;
+            if (cudaMemcpyAsync(h, staging, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+                return PKV_ERR_CUDA;
+        } else {
+            if (cudaMemcpyAsync(staging, h, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
+                return PKV_ERR_CUDA;
+            if ((rc = launch(pkv::swap_stage_kernel, dim3((unsigned)cnt), dim3(256), 0, st,
+                             k_caches, v_caches, block_ids, num_ids,
+                             static_cast<uint4 *>(staging), t0, num_blocks, (int)vecs, 0,
+                             status)) != PKV_OK)
+                return rc;
+        }
+    }
+    return PKV_OK;
+}
+
 int pkv_get_device_status(uint32_t *status_out, int clear, pkv_stream_t stream) {
     if (!status_out) return PKV_ERR_INVALID_ARG;
     if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)

@@ -134,6 +134,18 @@ def test_cache_op_checks_without_a_device():
     assert L.pkv_copy_blocks(None, None, 0, None, 3, 8, 64, 16, 64, 0, None) == B.PKV_ERR_INVALID_ARG
 
 
+def test_staged_swap_checks_without_a_device():
+    L = B.lib()
+    args = (None, None, 1, None)
+    # nothing to move; bad head_dim; missing pointers (all before any CUDA call)
+    assert L.pkv_swap_blocks_staged(*args, 0, None, 0, 1, 8, 128, 16, 64, 0, None, 0,
+                                    None) == B.PKV_OK
+    assert L.pkv_swap_blocks_staged(*args, 4, None, 0, 1, 8, 96, 16, 64, 0, None, 0,
+                                    None) == B.PKV_ERR_INVALID_ARG
+    assert L.pkv_swap_blocks_staged(*args, 4, None, 0, 1, 8, 128, 16, 64, 0, None, 0,
+                                    None) == B.PKV_ERR_INVALID_ARG
+
+
 def test_status_strings():
     L = B.lib()
     for code in range(-10, 1):

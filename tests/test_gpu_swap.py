@@ -73,3 +73,73 @@ def test_swap_bad_id_skipped_and_reported(cuda_device):
     np.testing.assert_array_equal(b[0, 0, 0], kcs[0][2])
     np.testing.assert_array_equal(b[0, 0, 2], kcs[0][4])
     assert (b[0, :, 1] == 0).all()
+
+
+@pytest.mark.parametrize("L,D,BS,tiles", [(1, 128, 16, 1), (3, 128, 8, 5), (2, 64, 32, 64),
+                                          (2, 128, 16, 7)])
+def test_staged_swap_out_and_in_bit_exact(cuda_device, L, D, BS, tiles):
+    """The staged swap (gather into a device buffer of `tiles` tiles, one large copy per
+    chunk; 1 tile: a copy per tile, 5 or 7: ragged last chunk, 64: a single chunk) gives the
+    oracle's host buffer and cache contents, and the same buffer as the one-kernel swap."""
+    rng = np.random.default_rng(90 + L + D + BS + tiles)
+    NB, Hkv, dtype = 40, 8, synth.BF16
+    kcs, vcs, kd, vd, kp, vp = setup(rng, L, NB, Hkv, BS, D, dtype)
+    out_ids = np.array(rng.choice(NB, size=13, replace=False), np.int32)
+    tile = Hkv * BS * D * 2
+    staging = torch.empty(tiles * tile + 16, dtype=torch.uint8, device="cuda")
+    buf = torch.full((L, 2, 13, Hkv, BS, D), -1, dtype=torch.int16).pin_memory()
+    ids_d = torch.from_numpy(out_ids).cuda()
+    pkv.pkv_swap_blocks_staged(kp, vp, ids_d, buf, 1, Hkv, D, BS, NB, pkv.PKV_BF16, staging)
+    torch.cuda.synchronize()
+    expect = C.swap_out(kcs, vcs, out_ids)
+    np.testing.assert_array_equal(buf.numpy().view(np.uint16), expect)
+    direct = torch.zeros_like(buf).pin_memory()
+    pkv.pkv_swap_blocks(kp, vp, ids_d, direct, 1, Hkv, D, BS, NB, pkv.PKV_BF16)
+    torch.cuda.synchronize()
+    assert torch.equal(direct, buf)
+    in_ids = np.array([b for b in range(NB) if b not in out_ids][:13], np.int32)
+    pkv.pkv_swap_blocks_staged(kp, vp, torch.from_numpy(in_ids).cuda(), buf, 0, Hkv, D, BS, NB,
+                               pkv.PKV_BF16, staging)
+    torch.cuda.synchronize()
+    ek, ev = C.swap_in(kcs, vcs, in_ids, expect)
+    for layer in range(L):
+        np.testing.assert_array_equal(to_bits(kd[layer]), ek[layer])
+        np.testing.assert_array_equal(to_bits(vd[layer]), ev[layer])
+    assert pkv.pkv_get_device_status() == 0
+
+
+def test_staged_swap_rejects_bad_buffers_and_zeroes_bad_ids(cuda_device):
+    rng = np.random.default_rng(91)
+    NB, Hkv, BS, D = 8, 2, 16, 64
+    kcs, vcs, kd, vd, kp, vp = setup(rng, 1, NB, Hkv, BS, D, synth.F16)
+    tile = Hkv * BS * D * 2
+    ids = torch.tensor([1, 2], dtype=torch.int32, device="cuda")
+    buf = torch.empty((1, 2, 2, Hkv, BS, D), dtype=torch.int16).pin_memory()
+    # staging smaller than one tile
+    with pytest.raises(pkv.PagedKVError) as e:
+        pkv.pkv_swap_blocks_staged(kp, vp, ids, buf, 1, Hkv, D, BS, NB, pkv.PKV_F16,
+                                   torch.empty(tile - 16, dtype=torch.uint8, device="cuda"))
+    assert e.value.code == pkv._binding.PKV_ERR_WORKSPACE
+    # staging in host memory: refused by the binding
+    with pytest.raises(ValueError):
+        pkv.pkv_swap_blocks_staged(kp, vp, ids, buf, 1, Hkv, D, BS, NB, pkv.PKV_F16,
+                                   torch.empty(4 * tile, dtype=torch.uint8))
+    staging = torch.empty(4 * tile, dtype=torch.uint8, device="cuda")
+    # host buffer pageable, or too small
+    for bad in (torch.empty((1, 2, 2, Hkv, BS, D), dtype=torch.int16),
+                torch.empty((1, 2, 1, Hkv, BS, D), dtype=torch.int16).pin_memory()):
+        with pytest.raises(pkv.PagedKVError) as e:
+            pkv.pkv_swap_blocks_staged(kp, vp, ids, bad, 1, Hkv, D, BS, NB, pkv.PKV_F16,
+                                       staging)
+        assert e.value.code == pkv._binding.PKV_ERR_INVALID_ARG
+    # an out-of-pool id: its tiles are zero in the host buffer, the others exact
+    buf3 = torch.full((1, 2, 3, Hkv, BS, D), 7, dtype=torch.int16).pin_memory()
+    pkv.pkv_get_device_status(clear=True)
+    pkv.pkv_swap_blocks_staged(kp, vp, torch.tensor([2, NB + 5, 4], dtype=torch.int32,
+                                                    device="cuda"),
+                               buf3, 1, Hkv, D, BS, NB, pkv.PKV_F16, staging)
+    assert pkv.pkv_get_device_status(clear=True) & pkv._binding.STATUS_BAD_PAIR
+    b = buf3.numpy().view(np.uint16)
+    np.testing.assert_array_equal(b[0, 0, 0], kcs[0][2])
+    np.testing.assert_array_equal(b[0, 1, 2], vcs[0][4])
+    assert (b[0, :, 1] == 0).all()
