@@ -300,15 +300,18 @@ int pkv_swap_blocks(void *const *k_caches, void *const *v_caches, int num_layers
 
 /* The same swap (same arguments, same host buffer layout and contents) moved in large
  * copies: the listed tiles are gathered into (or scattered from) `staging`, a DEVICE buffer
- * of staging_bytes (16-byte aligned, at least one tile = Hkv*BS*D*2 bytes), and each full
- * staging buffer crosses the host link as one cudaMemcpyAsync, so the link runs at the rate
- * of its copy engine rather than of the SMs' stores to mapped memory. Chunks follow one
- * another on `stream` (a gather or scatter launch and one copy per floor(staging_bytes /
- * tile) tiles). host_buffer must be pinned host memory (the copies are asynchronous only
- * from it). Tiles of ids outside [0, num_blocks) set PKV_STATUS_BAD_PAIR and are zero in
- * the host buffer (to_host = 1) or not written (to_host = 0). Errors: as pkv_swap_blocks;
- * PKV_ERR_WORKSPACE (staging missing, misaligned or smaller than a tile); PKV_ERR_INVALID_ARG
- * (staging not device memory). */
+ * of staging_bytes (16-byte aligned, at least two tiles of Hkv*BS*D*2 bytes), used as two
+ * halves: each half, once full, crosses the host link as one cudaMemcpyAsync while the
+ * other half is gathered (or scattered), so the link runs at the rate of its copy engine
+ * rather than of the SMs' stores to mapped memory. The copies run on a stream of the
+ * library's, ordered after the work `stream` holds at the call by an event, and `stream`
+ * waits for the last of them: as for pkv_swap_blocks, the host buffer is complete (or may
+ * be refilled) once `stream` reaches this point. Calls that use this path are serialised
+ * on the host while they enqueue. host_buffer must be pinned host memory (the copies are
+ * asynchronous only from it). Tiles of ids outside [0, num_blocks) set PKV_STATUS_BAD_PAIR
+ * and are zero in the host buffer (to_host = 1) or not written (to_host = 0). Errors: as
+ * pkv_swap_blocks; PKV_ERR_WORKSPACE (staging missing, misaligned or smaller than two
+ * tiles); PKV_ERR_INVALID_ARG (staging not device memory); PKV_ERR_CUDA. */
 int pkv_swap_blocks_staged(void *const *k_caches, void *const *v_caches, int num_layers,
                            const int32_t *block_ids, int num_ids, void *host_buffer,
                            size_t host_buffer_bytes, int to_host, int num_kv_heads,

@@ -54,6 +54,16 @@ int device_status_ptr(unsigned int **out) {
 // once per device with cudaGetSymbolAddress.
 constexpr size_t kNoAllocScratchBytes = PKV_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+// Per device: the library's copy stream and events of the staged swap (created on first
+// use, kept until exit), and the lock that keeps one call's sequence of them whole.
+struct SwapSide {
+    bool ready = false;
+    cudaStream_t cs = nullptr;
+    cudaEvent_t start = nullptr, fill[2] = {nullptr, nullptr}, drain[2] = {nullptr, nullptr};
+};
+SwapSide g_swap_side[kMaxDevices];
+std::mutex g_swap_mu;
+
 void *g_noalloc_ptr[kMaxDevices];
 
 int noalloc_scratch_ptr(void **out) {
@@ -1187,7 +1197,7 @@ int pkv_swap_blocks_staged(void *const *k_caches, void *const *v_caches, int num
     const unsigned long long tile = (unsigned long long)vecs * 16;
     const long long total = (long long)num_layers * 2 * num_ids;
     if (host_buffer_bytes < (unsigned long long)total * tile) return PKV_ERR_INVALID_ARG;
-    if (!staging || !aligned(staging, 16) || staging_bytes < tile) return PKV_ERR_WORKSPACE;
+    if (!staging || !aligned(staging, 16) || staging_bytes < 2 * tile) return PKV_ERR_WORKSPACE;
     // the copies are asynchronous only from pinned memory: anything else is refused
     cudaPointerAttributes attr;
     if (cudaPointerGetAttributes(&attr, host_buffer) != cudaSuccess) {
@@ -1203,30 +1213,72 @@ int pkv_swap_blocks_staged(void *const *k_caches, void *const *v_caches, int num
     unsigned int *status;
     int rc;
     if ((rc = device_status_ptr(&status)) != PKV_OK) return rc;
+    int dev;
+    if ((rc = current_device(&dev)) != PKV_OK) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const long long per = (long long)std::min<unsigned long long>(staging_bytes / tile, INT_MAX);
+    // Two halves of the staging buffer: while the copy engine moves one half over the link
+    // (on a stream of the library's, `cs`), the next gather fills the other half on `st`
+    // (or, into the device, the next copy fills one half while the previous scatter drains
+    // the other). Events order each half's fill after its last drain.
+    const long long per = (long long)std::min<unsigned long long>(staging_bytes / 2 / tile,
+                                                                  INT_MAX);
+    if (per < 1) return PKV_ERR_WORKSPACE;
+    std::lock_guard<std::mutex> lk(g_swap_mu);   // the side stream and events are shared
+    SwapSide &side = g_swap_side[dev];
+    if (!side.ready) {
+        if (cudaStreamCreateWithFlags(&side.cs, cudaStreamNonBlocking) != cudaSuccess)
+            return PKV_ERR_CUDA;
+        for (cudaEvent_t *e : {&side.start, &side.fill[0], &side.fill[1], &side.drain[0],
+                               &side.drain[1]})
+            if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess)
+                return PKV_ERR_CUDA;
+        side.ready = true;
+    }
+    cudaStream_t cs = side.cs;
     char *host = static_cast<char *>(host_buffer);
-    for (long long t0 = 0; t0 < total; t0 += per) {
+    char *halves[2] = {static_cast<char *>(staging),
+                       static_cast<char *>(staging) + (size_t)per * tile};
+    if (cudaEventRecord(side.start, st) != cudaSuccess) return PKV_ERR_CUDA;
+    if (cudaStreamWaitEvent(cs, side.start, 0) != cudaSuccess) return PKV_ERR_CUDA;
+    long long k = 0;
+    for (long long t0 = 0; t0 < total; t0 += per, ++k) {
+        const int h = (int)(k & 1);
         const long long cnt = std::min(per, total - t0);
-        char *h = host + (unsigned long long)t0 * tile;
+        char *hp = host + (unsigned long long)t0 * tile;
         const size_t bytes = (size_t)((unsigned long long)cnt * tile);
+        uint4 *stg = reinterpret_cast<uint4 *>(halves[h]);
         if (to_host) {
+            // gather k into half h once copy k-2 has read it, then copy it out
+            if (k >= 2 && cudaStreamWaitEvent(st, side.drain[h], 0) != cudaSuccess)
+                return PKV_ERR_CUDA;
             if ((rc = launch(pkv::swap_stage_kernel, dim3((unsigned)cnt), dim3(256), 0, st,
-                             k_caches, v_caches, block_ids, num_ids,
-                             static_cast<uint4 *>(staging), t0, num_blocks, (int)vecs, 1,
-                             status)) != PKV_OK)
+                             k_caches, v_caches, block_ids, num_ids, stg, t0, num_blocks,
+                             (int)vecs, 1, status)) != PKV_OK)
                 return rc;
-            if (cudaMemcpyAsync(h, staging, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+            if (cudaEventRecord(side.fill[h], st) != cudaSuccess ||
+                cudaStreamWaitEvent(cs, side.fill[h], 0) != cudaSuccess ||
+                cudaMemcpyAsync(hp, stg, bytes, cudaMemcpyDeviceToHost, cs) != cudaSuccess ||
+                cudaEventRecord(side.drain[h], cs) != cudaSuccess)
                 return PKV_ERR_CUDA;
         } else {
-            if (cudaMemcpyAsync(staging, h, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
+            // copy k into half h once scatter k-2 has read it, then scatter it
+            if (k >= 2 && cudaStreamWaitEvent(cs, side.drain[h], 0) != cudaSuccess)
+                return PKV_ERR_CUDA;
+            if (cudaMemcpyAsync(stg, hp, bytes, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
+                cudaEventRecord(side.fill[h], cs) != cudaSuccess ||
+                cudaStreamWaitEvent(st, side.fill[h], 0) != cudaSuccess)
                 return PKV_ERR_CUDA;
             if ((rc = launch(pkv::swap_stage_kernel, dim3((unsigned)cnt), dim3(256), 0, st,
-                             k_caches, v_caches, block_ids, num_ids,
-                             static_cast<uint4 *>(staging), t0, num_blocks, (int)vecs, 0,
-                             status)) != PKV_OK)
+                             k_caches, v_caches, block_ids, num_ids, stg, t0, num_blocks,
+                             (int)vecs, 0, status)) != PKV_OK)
                 return rc;
+            if (cudaEventRecord(side.drain[h], st) != cudaSuccess) return PKV_ERR_CUDA;
         }
+    }
+    if (to_host) {
+        // `st` reaches the end of the call once every copy has landed in host memory
+        for (int h = 0; h < 2 && h < k; ++h)
+            if (cudaStreamWaitEvent(st, side.drain[h], 0) != cudaSuccess) return PKV_ERR_CUDA;
     }
     return PKV_OK;
 }

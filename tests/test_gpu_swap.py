@@ -75,12 +75,13 @@ def test_swap_bad_id_skipped_and_reported(cuda_device):
     assert (b[0, :, 1] == 0).all()
 
 
-@pytest.mark.parametrize("L,D,BS,tiles", [(1, 128, 16, 1), (3, 128, 8, 5), (2, 64, 32, 64),
+@pytest.mark.parametrize("L,D,BS,tiles", [(1, 128, 16, 2), (3, 128, 8, 5), (2, 64, 32, 64),
                                           (2, 128, 16, 7)])
 def test_staged_swap_out_and_in_bit_exact(cuda_device, L, D, BS, tiles):
-    """The staged swap (gather into a device buffer of `tiles` tiles, one large copy per
-    chunk; 1 tile: a copy per tile, 5 or 7: ragged last chunk, 64: a single chunk) gives the
-    oracle's host buffer and cache contents, and the same buffer as the one-kernel swap."""
+    """The staged swap (a device buffer of `tiles` tiles in two halves, one large copy per
+    half-buffer chunk; 2 tiles: a copy per tile, 5 or 7: ragged last chunk, 64: one or two
+    chunks) gives the oracle's host buffer and cache contents, and the same buffer as the
+    one-kernel swap."""
     rng = np.random.default_rng(90 + L + D + BS + tiles)
     NB, Hkv, dtype = 40, 8, synth.BF16
     kcs, vcs, kd, vd, kp, vp = setup(rng, L, NB, Hkv, BS, D, dtype)
@@ -115,10 +116,10 @@ def test_staged_swap_rejects_bad_buffers_and_zeroes_bad_ids(cuda_device):
     tile = Hkv * BS * D * 2
     ids = torch.tensor([1, 2], dtype=torch.int32, device="cuda")
     buf = torch.empty((1, 2, 2, Hkv, BS, D), dtype=torch.int16).pin_memory()
-    # staging smaller than one tile
+    # staging smaller than two tiles (one per half)
     with pytest.raises(pkv.PagedKVError) as e:
         pkv.pkv_swap_blocks_staged(kp, vp, ids, buf, 1, Hkv, D, BS, NB, pkv.PKV_F16,
-                                   torch.empty(tile - 16, dtype=torch.uint8, device="cuda"))
+                                   torch.empty(2 * tile - 16, dtype=torch.uint8, device="cuda"))
     assert e.value.code == pkv._binding.PKV_ERR_WORKSPACE
     # staging in host memory: refused by the binding
     with pytest.raises(ValueError):
