@@ -144,3 +144,35 @@ def test_staged_swap_rejects_bad_buffers_and_zeroes_bad_ids(cuda_device):
     np.testing.assert_array_equal(b[0, 0, 0], kcs[0][2])
     np.testing.assert_array_equal(b[0, 1, 2], vcs[0][4])
     assert (b[0, :, 1] == 0).all()
+
+
+def test_staged_swap_replays_in_a_cuda_graph(cuda_device):
+    """The staged swap's copies run on a stream of the library's, joined to the caller's by
+    events: recorded into a CUDA graph on the caller's stream, a replay gives the oracle's
+    host buffer (the copy stream is part of the graph)."""
+    rng = np.random.default_rng(92)
+    L, NB, Hkv, BS, D = 2, 24, 4, 16, 128
+    kcs, vcs, kd, vd, kp, vp = setup(rng, L, NB, Hkv, BS, D, synth.BF16)
+    ids = np.array(rng.choice(NB, size=9, replace=False), np.int32)
+    ids_d = torch.from_numpy(ids).cuda()
+    tile = Hkv * BS * D * 2
+    staging = torch.empty(4 * tile, dtype=torch.uint8, device="cuda")   # 2 tiles per half
+    buf = torch.zeros((L, 2, 9, Hkv, BS, D), dtype=torch.int16).pin_memory()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):   # eager first call: creates the library's copy stream
+        pkv.pkv_swap_blocks_staged(kp, vp, ids_d, buf, 1, Hkv, D, BS, NB, pkv.PKV_BF16, staging,
+                                   stream=side)
+    side.synchronize()
+    buf.zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        pkv.pkv_swap_blocks_staged(kp, vp, ids_d, buf, 1, Hkv, D, BS, NB, pkv.PKV_BF16, staging,
+                                   stream=side)
+    torch.cuda.synchronize()
+    assert (buf.numpy() == 0).all()          # recording moved nothing
+    g.replay()
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(buf.numpy().view(np.uint16), C.swap_out(kcs, vcs, ids))
+    del g
+    assert pkv.pkv_get_device_status() == 0
