@@ -441,9 +441,10 @@ paged_decode_shared_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const int count = prm.counters->count;
         int it = 0;
         bool ok = true;
+        // CTA c starts on item c (the plan's placement); the counter hands out the rest
         auto take = [&]() {
             unsigned v = 0;
-            if (lane == 0) v = atomicAdd(&prm.counters->next, 1u);
+            if (lane == 0) v = atomicAdd(&prm.counters->next, 1u) + gridDim.x;
             return v > 0x7fffffffu ? 0x7fffffff : (int)v;   // lives in lane 0
         };
         auto field = [&](const SharedItemCtx &c, int k) { return __shfl_sync(0xffffffffu, c.f, k); };
@@ -510,9 +511,8 @@ paged_decode_shared_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 ent[k] = e < nblk ? bt[e] : 0;
             }
         };
+        SharedItemCtx cur_item = load_item(blockIdx.x);
         int pending = take();
-        SharedItemCtx cur_item = load_item(__shfl_sync(0xffffffffu, pending, 0));
-        pending = take();
         SharedSeg cur = first_seg(cur_item);
         int ent[kMaxItemBlocks / 32];
         load_entries(cur, ent);
