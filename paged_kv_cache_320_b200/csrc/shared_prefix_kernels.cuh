@@ -310,13 +310,14 @@ shared_prefix_plan_kernel(SharedParams p) {
         *stages = max(st, 1);
         return it;
     };
-    // Placement: every CTA starts on the item at its own index and the launch's CTAs sit
-    // `slots` to an SM in index order (CTA c on SM c mod sms), so with no more items than
-    // CTAs the items of one SM run side by side. Items are ranked longest first (counting
-    // sort on stage counts); the sms longest go to the first slot of each SM and the
-    // others pair up longest with shortest in the second slots, which evens out the SMs'
-    // loads. With more items than CTAs, or another number of slots, the order is longest
-    // first. The placement moves items only: results do not depend on it.
+    // Placement: every CTA starts on the item at its own index. Items are ranked longest
+    // first (counting sort on stage counts); the sms longest are items 0 .. sms-1 and, with
+    // two CTAs per SM, the others follow shortest first, so that item sms + c goes to CTA
+    // sms + c, which shares CTA c's SM when the launch fills the SMs in index order (on
+    // B200 it does so for part of the SMs only: the first wave is spread GPC by GPC). That
+    // pairs long items with short ones on an SM and evens out the SMs' loads. With more
+    // items than CTAs, or another number of slots, the order is longest first. The
+    // placement moves items only: results do not depend on it.
     for (int c = tid; c < kPlanBins; c += kPlanThreads) plan_bins[c] = 0;
     __syncthreads();
     const int n_put = min(n_items, p.max_items);
