@@ -523,6 +523,21 @@ int pkv_seq_append_tokens(pkv_alloc *a, int64_t seq_id, const int32_t *tokens, i
 int pkv_seq_share_prefix(pkv_alloc *a, int64_t seq_id, const int32_t *tokens, int n_tokens,
                          int *n_cached_out);
 
+/* Groups for the shared-prefix-aware decode, read from the tables ("分页 KV Cache 分析" §3.2:
+ * requests with a common prompt share its pages; "vLLM" entity page, 是什么: parallel samples
+ * share their prompt's blocks). Sequences whose first full block is the same physical block
+ * form a group (in the order of their first member in seq_ids, members in seq_ids order); a
+ * sequence with no full block is a group of one. order_out [n]: the sequence ids, grouped;
+ * group_start_out [n + 1]: the first num_groups + 1 entries are the group boundaries in that
+ * order (0 = group_start[0] < ... = n); prefix_lens_out [n]: the first num_groups entries
+ * are block_size x the leading blocks every member's table holds in common, counting only
+ * each member's full blocks (0 for a group of one). Build the block tables, lengths and
+ * queries in order_out's order and pass these as group_start / prefix_lens to
+ * pkv_paged_attention_decode_shared_prefix. Errors: PKV_ERR_UNKNOWN_SEQ; PKV_ERR_INVALID_ARG
+ * (an id listed twice, a NULL output with n > 0); nothing is written past the check. */
+int pkv_prefix_groups(const pkv_alloc *a, const int64_t *seq_ids, int n, int64_t *order_out,
+                      int32_t *group_start_out, int32_t *prefix_lens_out, int *num_groups_out);
+
 /* Blocks in the cache, of which evictable; tokens queried by pkv_seq_share_prefix and
  * tokens it found cached. Any output pointer may be NULL. */
 int pkv_prefix_cache_stats(const pkv_alloc *a, int *cached_blocks, int *evictable_blocks,

@@ -259,6 +259,43 @@ class BlockManagerModel:
         row = list(self.tables[seq]) + [-1] * (self.mb - len(self.tables[seq]))
         return row, self.lens[seq]
 
+    def prefix_groups(self, seqs):
+        """Groups of sequences that share their prompt's pages ("分页 KV Cache 分析" §3.2;
+        "vLLM" entity page, 是什么), as the shared-prefix decode takes them. Reading (the
+        pages fix no rule): sequences whose first full block is the same physical block are
+        one group, groups in order of their first member, members in the given order; a
+        sequence without a full block is alone. A group's prefix is the number of leading
+        blocks all members hold in common, each member counting only its full blocks, times
+        the block size (0 alone). Returns (order, group_start, prefix_lens)."""
+        seqs = [int(x) for x in seqs]
+        if len(set(seqs)) != len(seqs):
+            raise ValueError("a sequence listed twice")
+        groups, by_first = [], {}
+        for s_ in seqs:
+            table, n = self.tables[s_], self.lens[s_]
+            if n >= self.bs and table:
+                key = table[0]
+                if key in by_first:
+                    groups[by_first[key]].append(s_)
+                    continue
+                by_first[key] = len(groups)
+            groups.append([s_])
+        order, starts, prefixes = [], [], []
+        for members in groups:
+            starts.append(len(order))
+            order += members
+            if len(members) == 1:
+                prefixes.append(0)
+                continue
+            full = min(self.lens[m] // self.bs for m in members)
+            common = 0
+            while common < full and all(self.tables[m][common] == self.tables[members[0]][common]
+                                        for m in members):
+                common += 1
+            prefixes.append(common * self.bs)
+        starts.append(len(order))
+        return order, starts, prefixes
+
     def stats(self):
         free = self.available()
         held = self.nb - free

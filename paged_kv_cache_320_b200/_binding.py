@@ -88,6 +88,7 @@ def lib() -> ctypes.CDLL:
                                            ctypes.POINTER(I)]
         L.pkv_seq_append_tables.argtypes = [P, P, I, I, P, P, ctypes.POINTER(I),
                                             ctypes.POINTER(I), P, P]
+        L.pkv_prefix_groups.argtypes = [P, P, I, P, P, P, ctypes.POINTER(I)]
         L.pkv_seq_fork.argtypes = [P, I64, I64]
         L.pkv_seq_free.argtypes = [P, I64]
         L.pkv_block_tables.argtypes = [P, P, I, P, P]
@@ -129,7 +130,7 @@ def lib() -> ctypes.CDLL:
                      "pkv_seq_free_batch", "pkv_shared_prefix_plan",
                      "pkv_paged_attention_decode_shared_prefix_planned",
                      "pkv_seq_append_tokens", "pkv_seq_share_prefix", "pkv_prefix_cache_stats",
-                     "pkv_seq_append_tables", "pkv_swap_blocks_staged"):
+                     "pkv_seq_append_tables", "pkv_swap_blocks_staged", "pkv_prefix_groups"):
             getattr(L, name).restype = I
         _lib = L
     return _lib
@@ -647,6 +648,22 @@ class BlockManager:
                                          ctypes.byref(n_cow), ctypes.byref(n_done),
                                          tables.ctypes.data, lens.ctypes.data)
         return rc, n_done.value, slots, cows[:n_cow.value], tables, lens
+
+    def pkv_prefix_groups(self, seq_ids):
+        """Groups of sequences sharing their first pages, for the shared-prefix decode.
+        Returns (status, order int64 [n], group_start int32 [groups + 1], prefix_lens int32
+        [groups])."""
+        import numpy as np
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        n = ids.shape[0]
+        order = np.zeros(max(n, 1), dtype=np.int64)
+        starts = np.zeros(n + 1, dtype=np.int32)
+        prefixes = np.zeros(max(n, 1), dtype=np.int32)
+        ng = ctypes.c_int(0)
+        rc = lib().pkv_prefix_groups(self._h, ids.ctypes.data, n, order.ctypes.data,
+                                     starts.ctypes.data, prefixes.ctypes.data, ctypes.byref(ng))
+        g = ng.value
+        return rc, order[:n], starts[:g + 1], prefixes[:g]
 
     def pkv_alloc_free_list(self, max_out=None):
         """Blocks the next allocations would take, in order (int32 array)."""

@@ -11,6 +11,8 @@
 // seeded by initial_order, free walks a table from its last block, all-or-nothing
 // appends). Pure host code: no CUDA call.
 #include <algorithm>
+#include <climits>
+#include <cstdint>
 #include <cstring>
 #include <list>
 #include <memory>
@@ -467,6 +469,67 @@ int pkv_block_tables(const pkv_alloc *a, const int64_t *seq_ids, int n, int32_t 
         if (lens_out) lens_out[i] = (int32_t)s.len;
     }
     return PKV_OK;
+}
+
+int pkv_prefix_groups(const pkv_alloc *a, const int64_t *seq_ids, int n, int64_t *order_out,
+                      int32_t *group_start_out, int32_t *prefix_lens_out, int *num_groups_out) {
+    return guarded([&]() -> int {
+        if (!a || n < 0 || !num_groups_out ||
+            (n > 0 && (!seq_ids || !order_out || !group_start_out || !prefix_lens_out)))
+            return PKV_ERR_INVALID_ARG;
+        *num_groups_out = 0;
+        if (n == 0) {
+            if (group_start_out) group_start_out[0] = 0;
+            return PKV_OK;
+        }
+        const int bs = a->block_size;
+        std::vector<const Seq *> seqs(n);
+        std::unordered_map<int64_t, int> seen;
+        seen.reserve((size_t)n * 2);
+        for (int i = 0; i < n; ++i) {
+            seqs[i] = a->find(seq_ids[i]);
+            if (!seqs[i]) return PKV_ERR_UNKNOWN_SEQ;
+            if (!seen.emplace(seq_ids[i], i).second) return PKV_ERR_INVALID_ARG;   // repeated
+        }
+        // key: the physical block holding a sequence's first full block; none (own group)
+        // for a sequence without a full block
+        std::unordered_map<int32_t, int> group_of_block;
+        std::vector<std::vector<int>> groups;
+        for (int i = 0; i < n; ++i) {
+            const Seq &s = *seqs[i];
+            if (s.len >= bs && !s.table.empty()) {
+                auto it = group_of_block.find(s.table[0]);
+                if (it != group_of_block.end()) {
+                    groups[it->second].push_back(i);
+                    continue;
+                }
+                group_of_block.emplace(s.table[0], (int)groups.size());
+            }
+            groups.push_back({i});
+        }
+        int at = 0;
+        for (size_t g = 0; g < groups.size(); ++g) {
+            const std::vector<int> &m = groups[g];
+            group_start_out[g] = at;
+            int64_t common = 0;   // leading blocks every member holds, full in each
+            if (m.size() > 1) {
+                common = INT64_MAX;
+                for (int i : m) common = std::min<int64_t>(common, seqs[i]->len / bs);
+                const std::vector<int32_t> &t0 = seqs[m[0]]->table;
+                for (size_t k = 1; k < m.size(); ++k) {
+                    const std::vector<int32_t> &t = seqs[m[k]]->table;
+                    int64_t b = 0;
+                    while (b < common && t[(size_t)b] == t0[(size_t)b]) ++b;
+                    common = b;
+                }
+            }
+            prefix_lens_out[g] = (int32_t)std::min<int64_t>(common * bs, INT32_MAX);
+            for (int i : m) order_out[at++] = seq_ids[i];
+        }
+        group_start_out[groups.size()] = at;
+        *num_groups_out = (int)groups.size();
+        return PKV_OK;
+    });
 }
 
 int pkv_alloc_free_list(const pkv_alloc *a, int32_t *blocks_out, int max_out, int *n_out) {

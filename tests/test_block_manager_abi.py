@@ -322,3 +322,82 @@ def test_host_allocation_failure_is_a_status_not_an_exception():
     lines = r.stdout.split("\n")
     assert lines[0] == f"{B.PKV_ERR_HOST_MEMORY} True"
     assert lines[1] == f"{B.PKV_OK} True"
+
+
+def test_prefix_groups_hand_worked():
+    """bs 4. Sequence 1: 9 tokens (blocks a, b, c; c holds one token). 2 and 3 are forked
+    from 1; 2 then appends 3 tokens, so its shared partial block c is copied (c') and it
+    has 12 tokens = 3 full blocks a, b, c'. 4: 2 tokens (no full block). 5: 6 tokens of its
+    own. Listed as [4, 2, 5, 1, 3]: group {4} (no full block), group {2, 1, 3} (first block
+    a; full blocks 3, 2, 2 -> at most 2 in common, and a, b are common: prefix 8), group {5}."""
+    c = BlockManager(64, 4, 8)
+    m = BM.BlockManagerModel(64, 4, 8)
+    for mgr in (c, m):
+        ap = mgr.pkv_seq_append if mgr is c else mgr.append
+        fk = mgr.pkv_seq_fork if mgr is c else mgr.fork
+        ap(1, 9)
+        fk(1, 2)
+        fk(1, 3)
+        ap(2, 3)
+        ap(4, 2)
+        ap(5, 6)
+    st, order, starts, pre = c.pkv_prefix_groups([4, 2, 5, 1, 3])
+    assert st == 0
+    assert order.tolist() == [4, 2, 1, 3, 5]
+    assert starts.tolist() == [0, 1, 4, 5]
+    assert pre.tolist() == [0, 8, 0]
+    assert m.prefix_groups([4, 2, 5, 1, 3]) == ([4, 2, 1, 3, 5], [0, 1, 4, 5], [0, 8, 0])
+    # unknown and repeated ids are refused
+    from paged_kv_cache_320_b200 import _binding as B
+    assert c.pkv_prefix_groups([1, 77])[0] == B.PKV_ERR_UNKNOWN_SEQ
+    assert c.pkv_prefix_groups([1, 2, 1])[0] == B.PKV_ERR_INVALID_ARG
+    st, order, starts, pre = c.pkv_prefix_groups([])
+    assert st == 0 and len(order) == 0 and starts.tolist() == [0] and len(pre) == 0
+    c.close()
+
+
+@pytest.mark.parametrize("seed", range(20))
+def test_prefix_groups_match_the_model(seed):
+    """Seeded streams of appends, forks, frees and prefix-cached admissions: the library's
+    groups equal the oracle model's for a random subset of the live sequences."""
+    rng = np.random.default_rng(1300 + seed)
+    nb, bs, mb = 64, int(rng.choice([2, 4, 8])), 12
+    c = BlockManager(nb, bs, mb)
+    m = BM.BlockManagerModel(nb, bs, mb)
+    assert c.pkv_alloc_set_prefix_cache(1) == 0
+    m.set_prefix_cache(True)
+    prompts = [rng.integers(0, 50, int(rng.integers(1, 4 * bs)), dtype=np.int32).tolist()
+               for _ in range(3)]
+    live, nxt = [], 0
+    for _ in range(40):
+        op = rng.random()
+        if op < 0.35 or not live:
+            toks = prompts[int(rng.integers(0, 3))] + \
+                rng.integers(0, 50, int(rng.integers(1, bs + 2)), dtype=np.int32).tolist()
+            st, got = c.pkv_seq_share_prefix(nxt, toks[:-1])
+            assert (st, got) == m.share_prefix(nxt, toks[:-1])
+            st2 = c.pkv_seq_append_tokens(nxt, toks[got:])[0]
+            assert st2 == m.append_tokens(nxt, toks[got:])[0]
+            if st == 0 and st2 == 0:
+                live.append(nxt)
+            elif st == 0:
+                assert c.pkv_seq_free(nxt) == m.free(nxt) == 0
+            nxt += 1
+        elif op < 0.55:
+            parent = int(rng.choice(live))
+            if c.pkv_seq_fork(parent, nxt) == m.fork(parent, nxt) == 0:
+                live.append(nxt)
+            nxt += 1
+        elif op < 0.8:
+            s_ = int(rng.choice(live))
+            k = int(rng.integers(1, bs + 1))
+            assert c.pkv_seq_append(s_, k)[0] == m.append(s_, k)[0]
+        else:
+            s_ = live.pop(int(rng.integers(0, len(live))))
+            assert c.pkv_seq_free(s_) == m.free(s_) == 0
+        if live:
+            pick = [int(x) for x in rng.permutation(live)[:int(rng.integers(1, len(live) + 1))]]
+            st, order, starts, pre = c.pkv_prefix_groups(pick)
+            assert st == 0
+            assert (order.tolist(), starts.tolist(), pre.tolist()) == m.prefix_groups(pick)
+    c.close()

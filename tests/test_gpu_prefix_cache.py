@@ -15,7 +15,8 @@ returns the same statuses, cached-token counts, slots and tables (bit-exact); th
 pool equals the oracle's cache writes; every live sequence's pages hold exactly the K/V of
 its own prefixes; the decode over the shared pages equals the oracle's attention on the
 model's tables (4e-3 + 1e-2|ref|). And the sharing is physical: requests on the same
-prompt hold the same prompt blocks."""
+prompt hold the same prompt blocks; pkv_prefix_groups finds them (as the oracle's model
+groups them) and the shared-prefix-aware decode over those groups equals the oracle too."""
 import numpy as np
 import pytest
 import torch
@@ -131,4 +132,29 @@ def test_decode_over_prefix_cached_blocks(cuda_device):
         assert pkv.pkv_get_device_status() == 0
         ref = A.paged_decode_attention(q, kc_o, vc_o, mt, ml, 1 / np.sqrt(D), DT)
         assert_close(to_bits(out), ref, DT, f"prefix-cached decode, partition {P}")
+
+    # the groups the block manager finds for the shared-prefix-aware decode: the oracle
+    # model's grouping of the same tables, one group per prompt holding at least the
+    # prompt's full blocks, and the grouped decode equal to the oracle's attention
+    st, order, gstart, gpre = lib_mgr.pkv_prefix_groups(ids)
+    morder, mstart, mpre = model.prefix_groups(ids)
+    assert st == 0
+    assert order.tolist() == morder and gstart.tolist() == mstart and gpre.tolist() == mpre
+    pos = {int(s): i for i, s in enumerate(ids)}
+    perm = np.array([pos[int(s)] for s in order])
+    for p, rows in by_prompt.items():
+        members = {int(ids[i]) for i in rows}
+        g = [k for k in range(len(gstart) - 1)
+             if members <= set(order[gstart[k]:gstart[k + 1]].tolist())]
+        assert len(g) == 1 and gpre[g[0]] >= len(prompts[p]) // BS * BS
+    qg, tg, lg = q[perm], tables[perm], lens[perm]
+    for P in (64, 0):
+        pkv.pkv_paged_attention_decode_shared_prefix(
+            out, to_dev(qg, DT), kc_d, vc_d, torch.from_numpy(np.ascontiguousarray(tg)).cuda(),
+            torch.from_numpy(np.ascontiguousarray(lg)).cuda(), torch.from_numpy(gstart).cuda(),
+            torch.from_numpy(gpre).cuda(), MB * BS, partition_size=P)
+        torch.cuda.synchronize()
+        assert pkv.pkv_get_device_status() == 0
+        ref = A.paged_decode_attention(qg, kc_o, vc_o, mt[perm], ml[perm], 1 / np.sqrt(D), DT)
+        assert_close(to_bits(out), ref, DT, f"prefix-cached shared-prefix decode, partition {P}")
     lib_mgr.close()
