@@ -780,6 +780,9 @@ def gpu_arm(args, rank, world, local_rank, light=False):
     memory = memory_utilisation(wl, mem_mgr, sp0.max_len)   # the workload's own length cap
     mem_mgr.close()
     prefix_cache = prefix_cache_measurement(sp) if args.prefix_cache else None
+    if prefix_cache is not None:
+        prefix_cache["decode"] = prefix_cache_decode_measurement(dev, stream, args.steps,
+                                                                 args.warmup)
 
     # ---- end to end: host block manager + pinned host buffers through the public API
     e2e = e2e_arm(args, wl, P, max_len, ws, dev, stream, barrier, max_over_ranks, world, decode,
@@ -922,6 +925,92 @@ def prefix_cache_measurement(sp, requests=1024, concurrency=128, decode_len=64, 
                     "admit_us_per_request": round(1e6 * admit_s / len(reqs), 2)}
         mgr.close()
     return out
+
+
+def prefix_cache_decode_measurement(dev, stream, steps, warmup, requests=128, prompts=4,
+                                    prefix=1024, seed=12):
+    """Prefix caching feeding the shared-prefix-aware decode: `requests` requests over
+    `prompts` system prompts of `prefix` tokens plus private questions of 32..511 tokens
+    are admitted through the block manager with the cache on (the later requests of a
+    prompt find its blocks), one decode token is appended to each, pkv_prefix_groups
+    groups them, and the decode over their tables is timed as CUDA graph replays, plain
+    and shared-prefix-aware (Llama-3-8B-shaped heads: 32 query / 8 KV, head_dim 128, bf16,
+    block size 16; cache contents random)."""
+    import torch
+    import paged_kv_cache_320_b200 as pkv
+    rng = np.random.default_rng(seed)
+    bs, hq, hkv, d = 16, 32, 8, 128
+    system = [rng.integers(0, 32000, prefix, dtype=np.int32) for _ in range(prompts)]
+    mb = -(-(prefix + 512 + 1) // bs)
+    nb = requests * mb
+    mgr = pkv.BlockManager(nb, bs, mb)
+    mgr.pkv_alloc_set_prefix_cache(1)
+    cached = 0
+    for r in range(requests):
+        toks = np.concatenate([system[r % prompts],
+                               rng.integers(0, 32000, int(rng.integers(32, 512)),
+                                            dtype=np.int32)])
+        st, got = mgr.pkv_seq_share_prefix(r, toks[:-1])
+        st2 = mgr.pkv_seq_append_tokens(r, toks[got:])[0]
+        st3 = mgr.pkv_seq_append_tokens(r, rng.integers(0, 32000, 1, dtype=np.int32))[0]
+        if st or st2 or st3:
+            raise RuntimeError("prefix-cache admission failed")
+        cached += got
+    st, order, gstart, gpre = mgr.pkv_prefix_groups(np.arange(requests))
+    st2, tables, lens = mgr.pkv_block_tables(order)
+    mgr.close()
+    if st or st2:
+        raise RuntimeError("prefix groups failed")
+    row = hkv * d * 2 * 2
+    logical = int(lens.astype(np.int64).sum()) * row
+    held = {}
+    for t, n in zip(tables, lens):
+        for j in range(-(-int(n) // bs)):
+            held[int(t[j])] = max(held.get(int(t[j]), 0), min(bs, int(n) - j * bs))
+    unique = sum(held.values()) * row
+    kc = torch.randn((nb, hkv, bs, d), device=dev).to(torch.bfloat16)
+    vc = torch.randn((nb, hkv, bs, d), device=dev).to(torch.bfloat16)
+    q = torch.randn((requests, hq, d), device=dev).to(torch.bfloat16)
+    out = torch.empty_like(q)
+    bt = torch.from_numpy(tables).to(dev)
+    ln = torch.from_numpy(lens).to(dev)
+    gs = torch.from_numpy(gstart).to(dev)
+    gp = torch.from_numpy(gpre).to(dev)
+    max_len = mb * bs
+    ws_p = torch.zeros(max(16, pkv.pkv_decode_workspace_size(
+        requests, hq, hkv, d, bs, max_len,
+        pkv.pkv_decode_partition_size(requests, hq, hkv, d, bs, max_len))),
+        dtype=torch.uint8, device=dev)
+    ws_s = torch.zeros(max(16, pkv.pkv_decode_shared_prefix_workspace_size(
+        requests, hq, hkv, d, bs, max_len)), dtype=torch.uint8, device=dev)
+    calls = {
+        "plain": lambda s: pkv.pkv_paged_attention_decode(out, q, kc, vc, bt, ln, max_len,
+                                                          workspace=ws_p, stream=s),
+        "shared": lambda s: pkv.pkv_paged_attention_decode_shared_prefix(
+            out, q, kc, vc, bt, ln, gs, gp, max_len, workspace=ws_s, stream=s)}
+    res = {"requests": requests, "prompts": prompts, "prefix_tokens": prefix,
+           "prefill_tokens_cached": cached, "groups": int(len(gstart) - 1),
+           "shared_prefix_tokens_per_group": sorted(set(int(x) for x in gpre)),
+           "logical_kv_bytes": logical, "unique_kv_bytes": unique}
+    for name, fn in calls.items():
+        with torch.cuda.stream(stream):
+            for _ in range(warmup):
+                fn(stream)
+        torch.cuda.synchronize(dev)
+        g = record_graph(fn, dev, stream)
+        for _ in range(warmup):
+            g.replay()
+        torch.cuda.synchronize(dev)
+        ms = time_replays(g, steps, stream)
+        del g
+        res[name] = {"us": round(ms * 1e3, 2), "logical_gbs": round(logical / (ms * 1e-3) / 1e9, 1),
+                     "unique_gbs": round(unique / (ms * 1e-3) / 1e9, 1)}
+    if pkv.pkv_get_device_status(stream=stream) != 0:
+        raise RuntimeError("device status word set during the prefix-cache decode")
+    res["speedup"] = round(res["plain"]["us"] / res["shared"]["us"], 3)
+    del kc, vc
+    torch.cuda.empty_cache()
+    return res
 
 
 def memory_utilisation(wl, mgr, max_len=None):
