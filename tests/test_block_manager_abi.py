@@ -347,6 +347,11 @@ def test_prefix_groups_hand_worked():
     assert starts.tolist() == [0, 1, 4, 5]
     assert pre.tolist() == [0, 8, 0]
     assert m.prefix_groups([4, 2, 5, 1, 3]) == ([4, 2, 1, 3, 5], [0, 1, 4, 5], [0, 8, 0])
+    # 1 and 3 alone still share the partly filled block c: only full blocks count, so the
+    # prefix is 8 tokens (a, b), not 12
+    st, order, starts, pre = c.pkv_prefix_groups([3, 1])
+    assert (st, order.tolist(), starts.tolist(), pre.tolist()) == (0, [3, 1], [0, 2], [8])
+    assert m.prefix_groups([3, 1]) == ([3, 1], [0, 2], [8])
     # unknown and repeated ids are refused
     from paged_kv_cache_320_b200 import _binding as B
     assert c.pkv_prefix_groups([1, 77])[0] == B.PKV_ERR_UNKNOWN_SEQ
