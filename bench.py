@@ -283,20 +283,24 @@ def cow_arm(args, rank, world, local_rank):
     t1.record(stream)
     barrier()
     eager_ms = reduce_max(t0.elapsed_time(t1) / args.steps, dist, dev)
-    # the step as a CUDA graph replay (as the other workloads are timed)
+    # the step as a CUDA graph (as the other workloads are timed): `steps` consecutive
+    # steps in one graph launched once, so the host cannot leave gaps between them; the
+    # one-step graph gives the per-step percentiles
     g_step = record_graph(lambda s: step(s=s), dev, stream)
     for _ in range(args.warmup):
         g_step.replay()
+    g_k = record_graph(lambda s: [step(s=s) for _ in range(args.steps)], dev, stream)
+    g_k.replay()
     barrier()
     with ClockSampler(local_rank) as clocks:
         barrier()
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
-        for _ in range(args.steps):
-            g_step.replay()
+        g_k.replay()
         t1.record(stream)
         barrier()
+    del g_k
     ms_step = reduce_max(t0.elapsed_time(t1) / args.steps, dist, dev)
     percentiles = step_percentiles(g_step.replay, args.steps, stream, dev)
     barrier()
@@ -427,7 +431,8 @@ def cow_arm(args, rank, world, local_rank):
                    "parallelism": f"replicas x{world}"},
         "tokens_per_s": round(tokens_per_s, 1),
         "pct_of_hbm_peak": round(100 * value / world / peak, 2),
-        "timed": "CUDA graph replays of the step (copy_blocks, cache write, decode)",
+        "timed": "CUDA graph of `steps` consecutive steps (copy_blocks, cache write, decode), "
+                 "launched once",
         "step_ms_percentiles": percentiles,
         "eager": {"value": round(weak_scaling_rates(kv_step, B, world, eager_ms)[0], 1),
                   "unit": "GB/s", "ms_per_step": round(eager_ms, 4),
@@ -675,18 +680,25 @@ def gpu_arm(args, rank, world, local_rank, light=False):
         step(stream)
     barrier()
     graphs = {}
+    g_step = None
     if not args.no_graph:
-        # the step recorded once as a CUDA graph (every layer's launches) and replayed: the
-        # headline timing, as a serving loop runs a decode step; the dominant kernel's and
-        # the merge kernel's launches alone in graphs of their own
-        graphs["step"] = record_graph(step, dev, stream)
+        # the step's launches (every layer's) recorded as a CUDA graph: the headline timing,
+        # as a serving loop runs a decode step; the dominant kernel's and the merge kernel's
+        # launches alone in graphs of their own. Each is timed as one graph of `steps`
+        # consecutive copies, launched once, so the host cannot leave gaps between steps;
+        # the one-step graph gives the per-step percentiles.
+        fns = {"step": step}
         if split:
-            graphs["kernel"] = record_graph(kernel_only, dev, stream)
+            fns["kernel"] = kernel_only
             if pmax > 1:
-                graphs["merge"] = record_graph(merge_only, dev, stream)
-        for g in graphs.values():
-            for _ in range(args.warmup):
-                g.replay()
+                fns["merge"] = merge_only
+        g_step = record_graph(step, dev, stream)
+        for _ in range(args.warmup):
+            g_step.replay()
+        for name, fn in fns.items():
+            graphs[name] = record_graph(lambda s, fn=fn: [fn(s) for _ in range(args.steps)],
+                                        dev, stream)
+            graphs[name].replay()   # upload, and one more warm-up pass
         barrier()
     ms = {}
     with ClockSampler(local_rank) as clocks:
@@ -701,13 +713,13 @@ def gpu_arm(args, rank, world, local_rank, light=False):
         barrier()
         ms["eager"] = t0.elapsed_time(t1) / args.steps
         for name, g in graphs.items():
-            ms[name] = time_replays(g, args.steps, stream)
+            ms[name] = time_replays(g, 1, stream) / args.steps
             barrier()
-    g_step = graphs.get("step")
     percentiles = step_percentiles(g_step.replay if g_step is not None else lambda: step(stream),
                                    args.steps, stream, dev)
     barrier()
     graphs.clear()
+    g_step = None
     if pkv.pkv_get_device_status(stream=stream) != 0:
         raise RuntimeError("device status word set during the benchmark")
 
@@ -744,9 +756,9 @@ def gpu_arm(args, rank, world, local_rank, light=False):
         "traffic": traffic,
         "algorithmic_bytes_per_launch": roof_layer,
         "avg_launch_us": round(kernel_us, 2),
-        "timed": ("CUDA graph of the kernel's launches alone (all layers), replayed `steps` "
-                  "times between CUDA events" if "kernel" in ms else
-                  "the step's CUDA graph replays (one launch per layer)"),
+        "timed": ("CUDA graph of the kernel's launches alone (all layers), `steps` copies in "
+                  "one graph launched once between CUDA events" if "kernel" in ms else
+                  "the step's CUDA graph (one launch per layer), `steps` copies launched once"),
         "call_level": {"includes": call_desc, "us_per_layer": round(call_us, 2),
                        "achieved": round(call_achieved, 1),
                        "frac": round(call_achieved / peak, 4)},
@@ -810,7 +822,8 @@ def gpu_arm(args, rank, world, local_rank, light=False):
             "partition_size": P,
             "decode": args.decode,
             "step": "fused" if fused else "separate",
-            "timed": "eager launches" if args.no_graph else "CUDA graph replays of the step",
+            "timed": "eager launches" if args.no_graph else
+                     "CUDA graph of `steps` consecutive steps, launched once",
             "kv_bytes_per_step": kv_step,
             "l2": f"inputs larger than L2: {kv_layer / 1e6:.0f} MB of K/V per layer vs 126 MB L2",
             "parallelism": f"replicas x{world}",
